@@ -1,0 +1,56 @@
+"""Plant plausible mistakes in a copy of the oracle and check that the pins
+catch every one (CPU only).  The real oracle file is never modified: each
+mutant is an edited copy compiled into a temporary library."""
+import pytest
+
+import oracle as O
+from tests import oracle_pins as P
+
+MUTANTS = [
+    ("scale dropped", "s[r] = dot * scale;", "s[r] = dot;"),
+    ("tie break reversed", "return (a->i < b->i) ? -1 : (a->i > b->i) ? 1 : 0;",
+     "return (a->i > b->i) ? -1 : (a->i < b->i) ? 1 : 0;"),
+    ("selection left in value order", "qsort(S, (size_t)keff, sizeof(int32_t), by_int_asc);", ""),
+    ("wrong GQA group", "const int g = h / G;\n      const int64_t kv_base",
+     "const int g = h % Hkv;\n      const int64_t kv_base"),
+    ("sparse head reads every row", "attend_rows(sh, q, K, V, kv_base, S, count, o, NULL);",
+     "attend_rows(sh, q, K, V, kv_base, NULL, n, o, NULL);"),
+    ("never refreshed after layer 0", "if (!fresh[s]) {", "if (!fresh[s] || l > 0) {"),
+    ("group mean over the wrong heads", "(((int64_t)l * B + b) * Hq + (g * G + t)) * d;",
+     "(((int64_t)l * B + b) * Hq + (t)) * d;"),
+    ("logits against V", "for (int j = 0; j < d; ++j) dot += q[j] * widen(K, sh->dtype, off + j);",
+     "for (int j = 0; j < d; ++j) dot += q[j] * widen(V, sh->dtype, off + j);"),
+    ("layer-0 rule dropped", "is_ret[h] = all_retrieval || role_row[h] != 0;",
+     "is_ret[h] = role_row[h] != 0;"),
+    ("padding not -1", "for (int64_t j = keff; j < k; ++j) S[j] = -1;",
+     "for (int64_t j = keff; j < k; ++j) S[j] = 0;"),
+    ("last inherited row dropped", "while (count < k && S[count] >= 0) ++count;",
+     "while (count < k - 1 && S[count] >= 0) ++count;"),
+    ("bf16 widened with the wrong shift", "uint32_t bits = ((uint32_t)h) << 16;",
+     "uint32_t bits = ((uint32_t)h) << 15;"),
+    ("softmax not normalised", "for (int j = 0; j < d; ++j) o[j] /= z;", ""),
+    ("token stride ignored", "int64_t off = kv_base + i * sh->s_token;\n    double dot",
+     "int64_t off = kv_base + i * sh->d;\n    double dot"),
+    ("value row from the wrong token",
+     "for (int j = 0; j < d; ++j) o[j] += p * widen(V, sh->dtype, off + j);",
+     "for (int j = 0; j < d; ++j) o[j] += p * widen(V, sh->dtype, kv_base + r * sh->s_token + j);"),
+    ("smallest instead of largest", "if (a->x > b->x) return -1;\n  if (a->x < b->x) return 1;",
+     "if (a->x < b->x) return -1;\n  if (a->x > b->x) return 1;"),
+]
+
+
+def caught(ora) -> str | None:
+    for pin in P.ALL_PINS:
+        try:
+            pin(ora)
+        except (AssertionError, ValueError) as e:   # a failed pin or a rejected call
+            return f"{pin.__name__}: {str(e)[:80]}"
+    return None
+
+
+@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_mutant_is_caught(tmp_path, name, old, new):
+    src = O.source_text()
+    assert src.count(old) == 1, f"mutation anchor for '{name}' not unique in oracle.c"
+    mutant = O.compile_variant(src.replace(old, new), str(tmp_path / "libmutant.so"))
+    assert caught(mutant) is not None, f"no pin catches the planted mistake '{name}'"

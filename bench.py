@@ -1,0 +1,436 @@
+"""Throughput of the hybrid-head sparse decode step (attention stack) on B200.
+
+Default workload: the Llama3-8B-shaped attention stack (32 layers, 32 query /
+8 KV heads, d=128, bf16) at n = 131072 tokens with token budget k = 4096,
+batch 1, layer 0 all retrieval and 2 retrieval query heads per later layer at
+seeded positions; synthetic seeded data.  One step = one pass of the whole
+L-layer stack (dense retrieval heads + top-k selection + sparse gathered
+heads, every layer), launched as one CUDA graph.
+
+Prints one JSON line on rank 0.  `--impl reference` times the fp64 CPU
+oracle instead (a bounded sample of the same workload, host cores).
+Multi-GPU (torchrun): every rank runs its own replica of the step (the path
+has no exchange step); value = all ranks' steps / the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "attn-stack decode steps/s at 128K ctx, k=4096; HBM GB/s vs peak"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+ATTN_SOURCES = ["attn_kernel.cu", "lyc_plan.h", "lyc_device.cuh"]
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["lyc", "reference"], default="lyc")
+    ap.add_argument("--n", type=int, default=131072)
+    ap.add_argument("--k", type=int, default=4096)
+    ap.add_argument("--retrieval-heads", type=int, default=2,
+                    help="retrieval query heads per layer after layer 0; -1 = all (dense baseline)")
+    ap.add_argument("--select-mode", choices=["per_qhead", "kvgroup_mean"], default="per_qhead")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-layers", type=int, default=2,
+                    help="oracle sample: layers 0..cpu_layers-1 of the step")
+    return ap.parse_args(argv)
+
+
+def workload_spec(args):
+    from hybrid_head_sparse_b200 import workloads as W
+    spec = W.LLAMA3_8B_128K.with_(n=args.n, k=args.k)
+    if args.retrieval_heads < 0:
+        spec = spec.with_(roles="all", name=spec.name + "-dense")
+    else:
+        spec = spec.with_(retrieval_per_layer=args.retrieval_heads,
+                          name=spec.name + f"-r{args.retrieval_heads}")
+    return spec
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def attn_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in ATTN_SOURCES:
+        with open(os.path.join(ROOT, "hybrid_head_sparse_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per attention launch from the committed ncu summary, if it
+    was taken on the current kernel source."""
+    path = os.path.join(ROOT, "profiles", "attn_layer_kernel_traffic.md")
+    if not os.path.exists(path):
+        return None
+    want = attn_source_hash()
+    for line in open(path):
+        if line.startswith("traffic-record:"):
+            try:
+                rec = json.loads(line.split(":", 1)[1])
+            except ValueError:
+                continue
+            if rec.get("source_sha") == want and rec.get("workload") == workload:
+                return rec.get("bytes_per_launch")
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.idx = device_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        try:
+            for line in open(self.path):
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9 and parts[1].isdigit():
+                    rows.append(parts)
+        except OSError:
+            pass
+        finally:
+            if self.path and os.path.exists(self.path):
+                os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        sm = [int(r[1]) for r in rows]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": int(rows[0][2]),
+                "reasons": reasons, "samples": len(rows),
+                "power_w_max": max(float(r[3]) for r in rows if r[3].replace(".", "").isdigit())
+                if any(r[3].replace(".", "").isdigit() for r in rows) else None}
+
+
+# ---------------------------------------------------------------- oracle timing
+
+
+def oracle_sample_seconds(spec, host_stack, cpu_layers: int):
+    """Time the oracle on layers 0..cpu_layers-1 (full n, every head) and
+    scale to one whole step: layer 0 + (L-1) x the mean of the later layers."""
+    import oracle as O
+    times = []
+    S = None
+    for l in range(cpu_layers):
+        t0 = time.perf_counter()
+        _, S, _, _ = O.layer(host_stack, l, spec.k, S, all_retrieval=(l == 0), n=spec.n)
+        times.append(time.perf_counter() - t0)
+    later = times[1:] if len(times) > 1 else times
+    est = times[0] + (spec.L - 1) * (sum(later) / len(later))
+    return est, times
+
+
+def cpu_cores() -> int:
+    n = os.environ.get("OMP_NUM_THREADS")
+    if n and n.isdigit():
+        return int(n)
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def host_sample_stack(spec, data, cpu_layers: int):
+    import oracle as O
+    from hybrid_head_sparse_b200 import workloads as W
+    layers = list(range(cpu_layers))
+    return O.Stack(W.host_view(data["q"][layers]), W.host_view(data["k"][layers]),
+                   W.host_view(data["v"][layers]), data["role"][layers].copy(), O.SELECT_PER_QHEAD)
+
+
+def sample_text(spec, cpu_layers):
+    return (f"oracle (fp64 C, OpenMP) on layers 0..{cpu_layers - 1} of one step at full size "
+            f"(n={spec.n}, k={spec.k}, all {spec.Hq} heads); step time = layer 0 + "
+            f"{spec.L - 1} x mean(later sampled layers)")
+
+
+# ---------------------------------------------------------------- reference arm
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle as O
+    from hybrid_head_sparse_b200 import workloads as W
+    O.build()
+    spec = workload_spec(args)
+    cl = max(1, min(args.cpu_layers, spec.L))
+    sample = W.make_stack(spec.with_(L=cl), "cpu")
+    st = host_sample_stack(spec, sample, cl)
+    for _ in range(args.warmup):
+        oracle_sample_seconds(spec, st, cl)
+    ests = []
+    for _ in range(args.steps):
+        est, _ = oracle_sample_seconds(spec, st, cl)
+        ests.append(est)
+    sec = sum(ests) / len(ests)
+    value = 1.0 / sec
+    cores = cpu_cores()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "steps/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": sec * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": spec.name, "L": spec.L, "B": spec.B, "Hq": spec.Hq,
+                   "Hkv": spec.Hkv, "d": spec.d, "n": spec.n, "k": spec.k,
+                   "retrieval_heads_per_layer": args.retrieval_heads,
+                   "select_mode": "per_qhead"},
+        "cpu_baseline": {"value": value, "unit": "steps/s", "cores": cores, "kind": "oracle",
+                         "sample": sample_text(spec, cl) + "; inputs drawn on the host with the "
+                         "same recipe"},
+        "e2e": {"value": value, "unit": "steps/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- library arm
+
+
+def run_lyc(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from hybrid_head_sparse_b200 import build as Bld
+    from hybrid_head_sparse_b200 import lyc, workloads as W
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        from datetime import timedelta
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    Bld.build()
+    lyc.load()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    spec = workload_spec(args)
+    data = W.make_stack(spec, dev)
+    torch.cuda.synchronize()
+    ctx = lyc.Lyc(spec.L, spec.B, spec.Hq, spec.Hkv, spec.d, spec.n, spec.k, dtype=spec.dtype,
+                  select_mode=args.select_mode, device=local)
+    out = torch.empty((spec.L, spec.B, spec.Hq, spec.d), device=dev)
+    S = torch.empty((spec.B, ctx.Hs, spec.k), dtype=torch.int32, device=dev)
+    role = data["role"]
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        ctx.decode_step(data["q"], data["k"], data["v"], spec.n, role, spec.k, out, S, stream=stream)
+
+    for _ in range(max(args.warmup, 1)):
+        step()
+    torch.cuda.synchronize()
+    rc = ctx.sync_status()
+    if rc != 0:
+        raise RuntimeError(f"device status after warm-up: {lyc.lyc_status_string(rc)}")
+
+    # ---- timed region: K graph replays, device-timed, max over ranks
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    clocks = clk.summary()
+    ms_total = ev0.elapsed_time(ev1)
+    if world > 1:
+        t = torch.tensor([ms_total], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total = float(t.item())
+    ms_step = ms_total / args.steps
+    value = world * args.steps / (ms_total / 1e3)
+    rc = ctx.sync_status()
+    if rc != 0:
+        raise RuntimeError(f"device status after timing: {lyc.lyc_status_string(rc)}")
+
+    # ---- per-kernel device times: the same K steps again with event nodes in the graph
+    ctx.set_timing(True)
+    step()
+    torch.cuda.synchronize()
+    ctx.kernel_times()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    ms_step_timed = ev0.elapsed_time(ev1) / args.steps
+    ktimes = ctx.kernel_times()
+    ctx.set_timing(False)
+    nsteps_t = args.steps
+    attn_ms = sum(t[2] for t in ktimes if t[0] == 0) / nsteps_t
+    topk_ms = sum(t[2] for t in ktimes if t[0] == 1) / nsteps_t
+    attn_launches = sum(1 for t in ktimes if t[0] == 0) // nsteps_t
+    topk_launches = sum(1 for t in ktimes if t[0] == 1) // nsteps_t
+
+    analytic, distinct = ctx.step_bytes(role, spec.n, spec.k)
+    peak, peak_kind = measured_peaks()
+    achieved = distinct / (attn_ms / 1e3) / 1e9
+    traffic = profiled_traffic(spec.name)
+    roofline = {
+        "bound": "hbm", "kernel": "attn_layer_kernel (pooled dense + sparse attention, one launch per layer)",
+        "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+        "frac": round(achieved / peak, 4), "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
+        "traffic": traffic,
+        "algorithmic_bytes_per_launch": distinct / attn_launches,
+        "avg_launch_ms": attn_ms / attn_launches,
+        "note": ("achieved = K+V bytes the kernel must read (dense groups: n rows; each sparse pass: "
+                 "k rows) / CUDA-event time of the attention launches, averaged over the layers of "
+                 "K timed steps"),
+    }
+    step_gbs = analytic / (ms_step / 1e3) / 1e9
+
+    # ---- end to end through the host-buffer entry point
+    e2e = None
+    if not args.no_e2e:
+        q_h = data["q"].cpu().pin_memory()
+        out_h = torch.empty(out.shape, dtype=torch.float32).pin_memory()
+        S_h = torch.empty(S.shape, dtype=torch.int32).pin_memory()
+
+        def hstep():
+            ctx.decode_step_host(q_h, data["k"], data["v"], spec.n, role, spec.k, out_h, S_h,
+                                 stream=stream)
+
+        for _ in range(2):
+            hstep()
+        torch.cuda.synchronize()
+        barrier()
+        ev0.record(stream)
+        for _ in range(args.steps):
+            hstep()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        ms_e2e = ev0.elapsed_time(ev1)
+        if world > 1:
+            t = torch.tensor([ms_e2e], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms_e2e = float(t.item())
+        e2e = {"value": world * args.steps / (ms_e2e / 1e3), "unit": "steps/s",
+               "h2d_bytes_per_step": q_h.numel() * q_h.element_size(),
+               "d2h_bytes_per_step": out_h.numel() * 4 + S_h.numel() * 4,
+               "note": "lyc_decode_step_host: q from pinned host memory in, outputs and sets back "
+                       "to pinned host memory, every step; KV cache resident on the device"}
+        rc = ctx.sync_status()
+        if rc != 0:
+            raise RuntimeError(f"device status after e2e: {lyc.lyc_status_string(rc)}")
+
+    # ---- the oracle on the host cores (rank 0, one GPU only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle as O
+        O.build()
+        cl = max(1, min(args.cpu_layers, spec.L))
+        st = host_sample_stack(spec, data, cl)
+        est, times = oracle_sample_seconds(spec, st, cl)
+        cpu = {"value": 1.0 / est, "unit": "steps/s", "cores": cpu_cores(), "kind": "oracle",
+               "sample": sample_text(spec, cl) + f"; sampled layer seconds {[round(t, 3) for t in times]}"}
+
+    launches_per_step = attn_launches + topk_launches + 1
+    line = {
+        "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic (seeded N(0,1) q/K/V, sinks + 256 planted heavy hitters per KV head)",
+        "config": {"workload": spec.name, "L": spec.L, "B": spec.B, "Hq": spec.Hq,
+                   "Hkv": spec.Hkv, "d": spec.d, "n": spec.n, "k": spec.k,
+                   "retrieval_heads_per_layer": args.retrieval_heads,
+                   "select_mode": args.select_mode, "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (KV cache %.1f GB per GPU)" % (
+                       2 * data["k"].numel() * data["k"].element_size() / 1e9)},
+        "hbm": {"analytic_bytes_per_step": analytic, "kernel_bytes_per_step": distinct,
+                "analytic_gbs": round(step_gbs, 1),
+                "frac_of_measured_peak": round(step_gbs / peak, 4),
+                "frac_of_8tbs": round(step_gbs / NOMINAL_HBM_GBS, 4)},
+        "roofline": roofline,
+        "kernels": {"attn_ms_per_step": attn_ms, "topk_ms_per_step": topk_ms,
+                    "ms_per_step_with_event_nodes": ms_step_timed},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+    }
+    ctx.close()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_lyc(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,866 @@
+// lyc_api.cu -- host side of liblyc.so: argument checks, the per-layer work
+// planner (workload pooling), set-buffer bookkeeping, CUDA-graph capture and
+// the C entry points declared in include/lyc.h.
+//
+// The step follows the decode loop of page "LycheeDecode ..." (paper-graph-ui
+// summary), Appendix B / Algorithm 1, attention part: per layer, retrieval
+// heads attend densely and re-select their set, sparse heads attend over the
+// set they inherit and pass it on; layer 0 is all retrieval.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <list>
+#include <memory>
+#include <string>
+#include <unordered_map>
+#include <vector>
+
+#include "../../include/lyc.h"
+#include "lyc_plan.h"
+
+namespace lyc {
+int attn_nq_bucket(int nq);
+cudaError_t attn_dispatch(int dtype, int D, int nqb, const AttnParams* p, int grid,
+                          cudaStream_t stream, int* smem_out, bool configure_only);
+size_t topk_smem_for(int cl, int n);
+int topk_pick_cluster(size_t smem);
+cudaError_t topk_configure(int cl, size_t smem);
+cudaError_t topk_launch(int cl, const TopkParams* p, int ntasks, cudaStream_t stream);
+cudaError_t copy_sets_launch(const CopySetsParams* p, cudaStream_t stream);
+cudaError_t validate_sets_launch(const ValidateSetsParams* p, cudaStream_t stream);
+}  // namespace lyc
+
+using namespace lyc;
+
+namespace {
+
+constexpr int kMaxCtxLimit = 786432;  // 16-CTA top-k keeps every key in shared memory
+constexpr int kPlanCacheSize = 16;
+
+int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
+
+// One layer of a plan: offsets of its records in the plan's device buffer.
+struct LayerPlan {
+  int nseg = 0, npieces = 0, grid = 0, nqb = 1;
+  size_t off_segs = 0, off_pieces = 0, off_cta = 0;
+  int ntasks = 0;
+  size_t off_tasks = 0;
+  size_t off_trace_src = 0;  // copy table for the set trace after this layer
+};
+
+struct Plan {
+  std::vector<LayerPlan> layers;
+  unsigned char* dev = nullptr;  // all records of all layers
+  size_t dev_bytes = 0;
+  size_t off_final_src = 0;      // copy table: current buffer of each set -> caller S
+  int nsets = 0;
+  int k = 0, keff = 0, n = 0;
+  uint32_t flags = 0;
+  const void* q = nullptr;
+  float* out = nullptr;
+  int32_t* S = nullptr;
+  int32_t* trace = nullptr;
+  bool timing = false;
+  cudaGraphExec_t exec = nullptr;
+  // timing: event-record nodes of the graph, in launch order (2 per kernel)
+  std::vector<cudaGraphNode_t> ev_nodes;
+  cudaGraph_t graph = nullptr;
+  std::vector<int> kernel_kind, kernel_layer;  // per timed kernel
+};
+
+}  // namespace
+
+struct lyc_ctx {
+  lyc_config cfg{};
+  int G = 1, Hs = 1, sms = 1, topk_cl = 8;
+  int64_t nstride = 0;  // row stride of the key buffer
+  int KS = 0;           // row stride of the set buffers
+  std::string err;
+  uint32_t* status = nullptr;
+  float* keys = nullptr;
+  int32_t* sbuf = nullptr;  // [2][B][Hs][KS]
+  float* part_o = nullptr;
+  float2* part_ml = nullptr;
+  int32_t* counters = nullptr;
+  size_t max_parts = 0, max_counters = 0;
+  // host-buffer entry point staging
+  void* q_dev = nullptr;
+  float* out_dev = nullptr;
+  int32_t* S_dev = nullptr;
+  int32_t* trace = nullptr;
+  cudaStream_t last_stream = nullptr;
+  bool timing = false;
+  // plans, most recent first
+  std::list<std::pair<std::string, std::unique_ptr<Plan>>> plans;
+  // timing pool
+  std::vector<cudaEvent_t> events;        // kTimingSets * events_per_set
+  int events_per_set = 0;
+  struct Recorded { int set; Plan* plan; };
+  std::vector<Recorded> recorded;
+  int next_set = 0;
+};
+
+namespace {
+
+lyc_status fail(lyc_ctx* c, lyc_status s, const std::string& msg) {
+  if (c) c->err = msg;
+  return s;
+}
+
+lyc_status cuda_fail(lyc_ctx* c, cudaError_t e, const char* what) {
+  if (c) c->err = std::string(what) + ": " + cudaGetErrorString(e);
+  return LYC_ERR_CUDA;
+}
+
+#define LYC_CUDA(call, what)                        \
+  do {                                              \
+    cudaError_t e_ = (call);                        \
+    if (e_ != cudaSuccess) return cuda_fail(ctx, e_, what); \
+  } while (0)
+
+void free_plan(Plan* p) {
+  if (!p) return;
+  if (p->exec) cudaGraphExecDestroy(p->exec);
+  if (p->graph) cudaGraphDestroy(p->graph);
+  if (p->dev) cudaFree(p->dev);
+  p->exec = nullptr;
+  p->graph = nullptr;
+  p->dev = nullptr;
+}
+
+}  // namespace
+
+namespace {
+
+// ---------------------------------------------------------------- planner
+//
+// Builds every layer's work pool for one (role mask, n, k, flags, pointers)
+// combination and uploads it in one buffer.  Set buffers: each set slot has
+// two buffers; a refreshed slot is written into the buffer it is not
+// currently read from, so a layer's readers and its own selection never touch
+// the same memory (double buffering), and unrefreshed slots cost no copy.
+lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const lyc_kv_cache* kv,
+                      int k, uint32_t flags) {
+  const lyc_config& cfg = ctx->cfg;
+  const int L = cfg.num_layers, B = cfg.batch, Hq = cfg.num_q_heads, Hkv = cfg.num_kv_heads;
+  const int G = ctx->G, Hs = ctx->Hs;
+  const bool kvmode = cfg.select_mode == LYC_SELECT_KVGROUP_MEAN;
+  const bool s_in = (flags & LYC_STEP_S_IN) != 0;
+  const int n = static_cast<int>(kv->n);
+  const int keff = std::min(k, n);
+  const size_t es = cfg.dtype == LYC_BF16 ? 2 : 4;
+  plan->k = k;
+  plan->keff = keff;
+  plan->n = n;
+  plan->nsets = B * Hs;
+
+  struct HostLayer {
+    std::vector<Segment> segs;
+    std::vector<Piece> pieces;
+    std::vector<int32_t> cta;
+    std::vector<TopkTask> tasks;
+    std::vector<const int32_t*> trace_src;
+    int nqb = 1;
+    int grid = 0;
+  };
+  std::vector<HostLayer> hl(L);
+  std::vector<int> cur(Hs, 0);
+  auto set_ptr = [&](int buf, int b, int s) {
+    return ctx->sbuf + ((static_cast<int64_t>(buf) * B + b) * Hs + s) * ctx->KS;
+  };
+  const char* kbase = static_cast<const char*>(kv->k);
+  const char* vbase = static_cast<const char*>(kv->v);
+
+  for (int l = 0; l < L; ++l) {
+    HostLayer& H = hl[l];
+    std::vector<char> is_ret(Hq), fresh(Hs, 0);
+    for (int h = 0; h < Hq; ++h) {
+      is_ret[h] = (l == 0 && !s_in) || role[static_cast<int64_t>(l) * Hq + h] != 0;
+      if (is_ret[h]) fresh[kvmode ? h / G : h] = 1;
+    }
+    int maxnq = 1;
+    for (int b = 0; b < B; ++b) {
+      for (int g = 0; g < Hkv; ++g) {
+        const int64_t off = l * kv->s_layer + b * kv->s_batch + g * kv->s_head;
+        Segment base{};
+        base.k = kbase + off * es;
+        base.v = vbase + off * es;
+        base.s_token = kv->s_token;
+        base.b = b;
+        base.g = g;
+        for (int j = 0; j < kMaxQ; ++j) {
+          base.key_off[j] = -1;
+          base.head[j] = -1;
+        }
+        // dense segment: the group's retrieval heads (+ mean query in group mode)
+        Segment ds = base;
+        ds.kind = kDense;
+        ds.rows = n;
+        int j = 0;
+        for (int h = g * G; h < (g + 1) * G; ++h) {
+          if (!is_ret[h]) continue;
+          ds.head[j] = h;
+          ds.key_off[j] = kvmode ? -1 : (static_cast<int64_t>(b) * Hs + h) * ctx->nstride;
+          ++j;
+        }
+        if (j > 0) {
+          ds.nout = j;
+          if (kvmode) {
+            ds.head[j] = -1;
+            ds.key_off[j] = (static_cast<int64_t>(b) * Hs + g) * ctx->nstride;
+            ++j;
+          }
+          ds.nq = j;
+          maxnq = std::max(maxnq, j);
+          H.segs.push_back(ds);
+        }
+        // sparse segments: one per inherited set that sparse heads read
+        if (kvmode) {
+          Segment ss = base;
+          ss.kind = kSparse;
+          ss.rows = keff;
+          ss.idx = set_ptr(cur[g], b, g);
+          int js = 0;
+          for (int h = g * G; h < (g + 1) * G; ++h)
+            if (!is_ret[h]) ss.head[js++] = h;
+          if (js > 0) {
+            ss.nq = ss.nout = js;
+            maxnq = std::max(maxnq, js);
+            H.segs.push_back(ss);
+          }
+        } else {
+          for (int h = g * G; h < (g + 1) * G; ++h) {
+            if (is_ret[h]) continue;
+            Segment ss = base;
+            ss.kind = kSparse;
+            ss.rows = keff;
+            ss.idx = set_ptr(cur[h], b, h);
+            ss.head[0] = h;
+            ss.nq = ss.nout = 1;
+            H.segs.push_back(ss);
+          }
+        }
+      }
+    }
+    H.nqb = attn_nq_bucket(maxnq);
+
+    // workload pooling: equal runs of 64-row tiles, one run per CTA
+    std::vector<int64_t> tstart(H.segs.size() + 1, 0);
+    for (size_t s = 0; s < H.segs.size(); ++s)
+      tstart[s + 1] = tstart[s] + (H.segs[s].rows + kTileRows - 1) / kTileRows;
+    const int64_t NT = tstart.back();
+    const int grid = static_cast<int>(std::min<int64_t>(NT, ctx->sms));
+    H.grid = grid;
+    std::vector<int> npieces(H.segs.size(), 0);
+    size_t seg_i = 0;
+    for (int c = 0; c < grid; ++c) {
+      H.cta.push_back(static_cast<int32_t>(H.pieces.size()));
+      const int64_t t0 = NT * c / grid, t1 = NT * (c + 1) / grid;
+      while (seg_i < H.segs.size() && tstart[seg_i + 1] <= t0) ++seg_i;
+      for (size_t s = seg_i; s < H.segs.size() && tstart[s] < t1; ++s) {
+        const int64_t a = std::max(t0, tstart[s]) - tstart[s];
+        const int64_t e = std::min(t1, tstart[s + 1]) - tstart[s];
+        if (e <= a) continue;
+        Piece pc;
+        pc.seg = static_cast<int32_t>(s);
+        pc.r0 = static_cast<int32_t>(a * kTileRows);
+        pc.r1 = static_cast<int32_t>(std::min<int64_t>(e * kTileRows, H.segs[s].rows));
+        pc.ordinal = npieces[s]++;
+        H.pieces.push_back(pc);
+      }
+    }
+    H.cta.push_back(static_cast<int32_t>(H.pieces.size()));
+    int part = 0, cnt = 0;
+    for (size_t s = 0; s < H.segs.size(); ++s) {
+      H.segs[s].npieces = npieces[s];
+      H.segs[s].part_base = part;
+      H.segs[s].cnt_base = cnt;
+      part += npieces[s] * H.segs[s].nout;
+      cnt += H.segs[s].nout;
+    }
+    if (static_cast<size_t>(part) > ctx->max_parts || static_cast<size_t>(cnt) > ctx->max_counters)
+      return fail(ctx, LYC_ERR_UNSUPPORTED, "work pool larger than the scratch sized at create");
+
+    // selection tasks of this layer, then flip the refreshed slots
+    for (int s = 0; s < Hs; ++s) {
+      if (!fresh[s]) continue;
+      for (int b = 0; b < B; ++b) {
+        TopkTask tk;
+        tk.keys = ctx->keys + (static_cast<int64_t>(b) * Hs + s) * ctx->nstride;
+        tk.S = set_ptr(1 - cur[s], b, s);
+        H.tasks.push_back(tk);
+      }
+    }
+    for (int s = 0; s < Hs; ++s)
+      if (fresh[s]) cur[s] ^= 1;
+    for (int b = 0; b < B; ++b)
+      for (int s = 0; s < Hs; ++s) H.trace_src.push_back(set_ptr(cur[s], b, s));
+  }
+
+  // ---- one device buffer for every record
+  size_t bytes = 0;
+  auto take = [&](size_t sz) {
+    bytes = round_up(bytes, 64);
+    const size_t o = bytes;
+    bytes += sz;
+    return o;
+  };
+  plan->layers.resize(L);
+  for (int l = 0; l < L; ++l) {
+    LayerPlan& lp = plan->layers[l];
+    HostLayer& H = hl[l];
+    lp.nseg = static_cast<int>(H.segs.size());
+    lp.npieces = static_cast<int>(H.pieces.size());
+    lp.grid = H.grid;
+    lp.nqb = H.nqb;
+    lp.ntasks = static_cast<int>(H.tasks.size());
+    lp.off_segs = take(H.segs.size() * sizeof(Segment));
+    lp.off_pieces = take(H.pieces.size() * sizeof(Piece));
+    lp.off_cta = take(H.cta.size() * sizeof(int32_t));
+    lp.off_tasks = take(std::max<size_t>(1, H.tasks.size()) * sizeof(TopkTask));
+    lp.off_trace_src = take(H.trace_src.size() * sizeof(void*));
+  }
+  plan->off_final_src = take(hl[L - 1].trace_src.size() * sizeof(void*));
+  std::vector<unsigned char> host(bytes, 0);
+  for (int l = 0; l < L; ++l) {
+    const LayerPlan& lp = plan->layers[l];
+    HostLayer& H = hl[l];
+    memcpy(host.data() + lp.off_segs, H.segs.data(), H.segs.size() * sizeof(Segment));
+    memcpy(host.data() + lp.off_pieces, H.pieces.data(), H.pieces.size() * sizeof(Piece));
+    memcpy(host.data() + lp.off_cta, H.cta.data(), H.cta.size() * sizeof(int32_t));
+    if (!H.tasks.empty())
+      memcpy(host.data() + lp.off_tasks, H.tasks.data(), H.tasks.size() * sizeof(TopkTask));
+    memcpy(host.data() + lp.off_trace_src, H.trace_src.data(), H.trace_src.size() * sizeof(void*));
+  }
+  memcpy(host.data() + plan->off_final_src, hl[L - 1].trace_src.data(),
+         hl[L - 1].trace_src.size() * sizeof(void*));
+  LYC_CUDA(cudaMalloc(&plan->dev, bytes), "cudaMalloc(plan)");
+  plan->dev_bytes = bytes;
+  LYC_CUDA(cudaMemcpy(plan->dev, host.data(), bytes, cudaMemcpyHostToDevice), "upload plan");
+  return LYC_OK;
+}
+
+}  // namespace
+
+namespace {
+
+// ---------------------------------------------------------------- enqueue
+// Records an event of timing set `set` (or, while capturing, of set 0, whose
+// nodes are re-pointed at other sets before each replay).
+lyc_status record_event(lyc_ctx* ctx, Plan* plan, int set, int idx, cudaStream_t stream,
+                        bool capturing) {
+  if (!plan->timing) return LYC_OK;
+  cudaEvent_t ev = ctx->events[static_cast<size_t>(set) * ctx->events_per_set + idx];
+  if (capturing) {
+    LYC_CUDA(cudaEventRecordWithFlags(ev, stream, cudaEventRecordExternal), "event record node");
+  } else {
+    LYC_CUDA(cudaEventRecord(ev, stream), "cudaEventRecord");
+  }
+  return LYC_OK;
+}
+
+// Enqueue the whole step of `plan` on `stream` (or record it, while capturing).
+lyc_status enqueue_step(lyc_ctx* ctx, Plan* plan, cudaStream_t stream, int set, bool capturing) {
+  const lyc_config& cfg = ctx->cfg;
+  const int L = cfg.num_layers, B = cfg.batch, Hq = cfg.num_q_heads, D = cfg.head_dim;
+  const size_t es = cfg.dtype == LYC_BF16 ? 2 : 4;
+  const int dtype = cfg.dtype == LYC_BF16 ? 0 : 1;
+  if (plan->flags & LYC_STEP_S_IN) {
+    LYC_CUDA(cudaMemcpy2DAsync(ctx->sbuf, ctx->KS * sizeof(int32_t), plan->S, plan->k * sizeof(int32_t),
+                               plan->k * sizeof(int32_t), static_cast<size_t>(B) * ctx->Hs,
+                               cudaMemcpyDeviceToDevice, stream),
+             "copy S^(0) in");
+    if (plan->flags & LYC_STEP_VALIDATE_S) {
+      ValidateSetsParams vp{ctx->sbuf, ctx->status, B * ctx->Hs, ctx->KS, plan->k, plan->keff, plan->n};
+      LYC_CUDA(validate_sets_launch(&vp, stream), "validate S^(0)");
+    }
+  }
+  plan->kernel_kind.clear();
+  plan->kernel_layer.clear();
+  int ev = 0;
+  for (int l = 0; l < L; ++l) {
+    const LayerPlan& lp = plan->layers[l];
+    AttnParams ap{};
+    ap.segs = reinterpret_cast<const Segment*>(plan->dev + lp.off_segs);
+    ap.pieces = reinterpret_cast<const Piece*>(plan->dev + lp.off_pieces);
+    ap.cta_begin = reinterpret_cast<const int32_t*>(plan->dev + lp.off_cta);
+    ap.q = static_cast<const char*>(plan->q) + static_cast<size_t>(l) * B * Hq * D * es;
+    ap.out = plan->out + static_cast<size_t>(l) * B * Hq * D;
+    ap.keys = ctx->keys;
+    ap.part_o = ctx->part_o;
+    ap.part_ml = ctx->part_ml;
+    ap.counters = ctx->counters;
+    ap.status = ctx->status;
+    ap.Hq = Hq;
+    ap.G = ctx->G;
+    ap.n = plan->n;
+    ap.scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
+    ap.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
+    lyc_status st = record_event(ctx, plan, set, ev++, stream, capturing);
+    if (st != LYC_OK) return st;
+    LYC_CUDA(attn_dispatch(dtype, D, lp.nqb, &ap, lp.grid, stream, nullptr, false), "attention launch");
+    if ((st = record_event(ctx, plan, set, ev++, stream, capturing)) != LYC_OK) return st;
+    plan->kernel_kind.push_back(0);
+    plan->kernel_layer.push_back(l);
+    if (lp.ntasks > 0) {
+      TopkParams tp{};
+      tp.tasks = reinterpret_cast<const TopkTask*>(plan->dev + lp.off_tasks);
+      tp.n = plan->n;
+      tp.k = plan->k;
+      if ((st = record_event(ctx, plan, set, ev++, stream, capturing)) != LYC_OK) return st;
+      LYC_CUDA(topk_launch(ctx->topk_cl, &tp, lp.ntasks, stream), "top-k launch");
+      if ((st = record_event(ctx, plan, set, ev++, stream, capturing)) != LYC_OK) return st;
+      plan->kernel_kind.push_back(1);
+      plan->kernel_layer.push_back(l);
+    }
+    if (plan->trace) {
+      CopySetsParams cp{reinterpret_cast<const int32_t* const*>(plan->dev + lp.off_trace_src),
+                        plan->trace + static_cast<size_t>(l) * B * ctx->Hs * plan->k, B * ctx->Hs,
+                        plan->k};
+      LYC_CUDA(copy_sets_launch(&cp, stream), "trace copy");
+    }
+  }
+  CopySetsParams cp{reinterpret_cast<const int32_t* const*>(plan->dev + plan->off_final_src), plan->S,
+                    B * ctx->Hs, plan->k};
+  LYC_CUDA(copy_sets_launch(&cp, stream), "final set copy");
+  return LYC_OK;
+}
+
+lyc_status capture_plan(lyc_ctx* ctx, Plan* plan) {
+  cudaStream_t cs;
+  LYC_CUDA(cudaStreamCreateWithFlags(&cs, cudaStreamNonBlocking), "capture stream");
+  cudaError_t e = cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal);
+  if (e != cudaSuccess) {
+    cudaStreamDestroy(cs);
+    return cuda_fail(ctx, e, "begin capture");
+  }
+  lyc_status st = enqueue_step(ctx, plan, cs, 0, true);
+  cudaGraph_t graph = nullptr;
+  e = cudaStreamEndCapture(cs, &graph);
+  cudaStreamDestroy(cs);
+  if (st != LYC_OK) {
+    if (graph) cudaGraphDestroy(graph);
+    return st;
+  }
+  if (e != cudaSuccess) return cuda_fail(ctx, e, "end capture");
+  e = cudaGraphInstantiate(&plan->exec, graph, 0);
+  if (e != cudaSuccess) {
+    cudaGraphDestroy(graph);
+    return cuda_fail(ctx, e, "graph instantiate");
+  }
+  plan->graph = graph;
+  if (plan->timing) {
+    // map each event-record node to its position via the set-0 event it records
+    size_t nn = 0;
+    LYC_CUDA(cudaGraphGetNodes(graph, nullptr, &nn), "graph nodes");
+    std::vector<cudaGraphNode_t> nodes(nn);
+    LYC_CUDA(cudaGraphGetNodes(graph, nodes.data(), &nn), "graph nodes");
+    plan->ev_nodes.assign(ctx->events_per_set, nullptr);
+    for (cudaGraphNode_t nd : nodes) {
+      cudaGraphNodeType ty;
+      LYC_CUDA(cudaGraphNodeGetType(nd, &ty), "node type");
+      if (ty != cudaGraphNodeTypeEventRecord) continue;
+      cudaEvent_t ev;
+      LYC_CUDA(cudaGraphEventRecordNodeGetEvent(nd, &ev), "node event");
+      for (int i = 0; i < ctx->events_per_set; ++i)
+        if (ctx->events[i] == ev) plan->ev_nodes[i] = nd;
+    }
+  }
+  return LYC_OK;
+}
+
+std::string plan_key(const uint8_t* role, int L, int Hq, const lyc_kv_cache* kv, int k,
+                     uint32_t flags, const void* q, const float* out, const int32_t* S,
+                     const int32_t* trace, bool timing) {
+  std::string key(reinterpret_cast<const char*>(role), static_cast<size_t>(L) * Hq);
+  auto add = [&](const void* p, size_t n) { key.append(static_cast<const char*>(p), n); };
+  add(kv, sizeof(*kv));
+  add(&k, sizeof k);
+  const uint32_t f = flags & (LYC_STEP_S_IN | LYC_STEP_VALIDATE_S);
+  add(&f, sizeof f);
+  add(&q, sizeof q);
+  add(&out, sizeof out);
+  add(&S, sizeof S);
+  add(&trace, sizeof trace);
+  const char t = timing ? 1 : 0;
+  add(&t, 1);
+  return key;
+}
+
+}  // namespace
+
+namespace {
+
+struct DeviceGuard {
+  int prev = -1;
+  bool ok = true;
+  explicit DeviceGuard(int dev) {
+    if (cudaGetDevice(&prev) != cudaSuccess) prev = -1;
+    if (prev != dev) ok = cudaSetDevice(dev) == cudaSuccess;
+  }
+  ~DeviceGuard() {
+    int now = -1;
+    if (prev >= 0 && cudaGetDevice(&now) == cudaSuccess && now != prev) cudaSetDevice(prev);
+  }
+};
+
+struct TimedStep {
+  int set;
+  std::vector<int> kind, layer;
+};
+std::unordered_map<const lyc_ctx*, std::vector<TimedStep>>& timed_steps() {
+  static std::unordered_map<const lyc_ctx*, std::vector<TimedStep>> m;
+  return m;
+}
+
+int timing_sets() { return 64; }
+
+lyc_status check_kv(lyc_ctx* ctx, const lyc_kv_cache* kv) {
+  const lyc_config& c = ctx->cfg;
+  const int64_t es = c.dtype == LYC_BF16 ? 2 : 4;
+  if (!kv || !kv->k || !kv->v) return fail(ctx, LYC_ERR_INVALID_ARG, "kv cache pointer is NULL");
+  if (kv->n < 1 || kv->n > c.max_ctx) return fail(ctx, LYC_ERR_INVALID_ARG, "kv->n outside [1, max_ctx]");
+  if (kv->s_token < c.head_dim) return fail(ctx, LYC_ERR_INVALID_ARG, "s_token < head_dim");
+  if (kv->s_layer < 0 || kv->s_batch < 0 || kv->s_head < 0)
+    return fail(ctx, LYC_ERR_INVALID_ARG, "negative kv stride");
+  const int64_t strides[4] = {kv->s_layer, kv->s_batch, kv->s_head, kv->s_token};
+  for (int64_t s : strides)
+    if ((s * es) % 16 != 0) return fail(ctx, LYC_ERR_INVALID_ARG, "kv strides must be multiples of 16 bytes");
+  if ((reinterpret_cast<uintptr_t>(kv->k) | reinterpret_cast<uintptr_t>(kv->v)) & 15u)
+    return fail(ctx, LYC_ERR_INVALID_ARG, "kv base pointers must be 16-byte aligned");
+  return LYC_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* lyc_status_string(lyc_status s) {
+  switch (s) {
+    case LYC_OK: return "ok";
+    case LYC_ERR_INVALID_ARG: return "invalid argument";
+    case LYC_ERR_UNSUPPORTED: return "unsupported configuration";
+    case LYC_ERR_OOM: return "out of device memory";
+    case LYC_ERR_CUDA: return "CUDA error";
+    case LYC_ERR_BAD_INDEX: return "inherited set holds an index outside [0, n)";
+    case LYC_ERR_TIMEOUT: return "device-side wait timed out";
+  }
+  return "unknown status";
+}
+
+const char* lyc_last_error(const lyc_ctx* ctx) { return ctx ? ctx->err.c_str() : "NULL context"; }
+
+lyc_status lyc_create(const lyc_config* cfg, lyc_ctx** out) {
+  if (!cfg || !out) return LYC_ERR_INVALID_ARG;
+  *out = nullptr;
+  const lyc_config& c = *cfg;
+  if (c.num_layers < 1 || c.batch < 1 || c.num_q_heads < 1 || c.num_kv_heads < 1 ||
+      c.num_q_heads % c.num_kv_heads != 0 || c.max_ctx < 1 || c.max_k < 1 || c.flags != 0)
+    return LYC_ERR_INVALID_ARG;
+  if (c.dtype != LYC_BF16 && c.dtype != LYC_FP32) return LYC_ERR_INVALID_ARG;
+  if (c.select_mode != LYC_SELECT_PER_QHEAD && c.select_mode != LYC_SELECT_KVGROUP_MEAN)
+    return LYC_ERR_INVALID_ARG;
+  if (c.head_dim != 64 && c.head_dim != 128) return LYC_ERR_UNSUPPORTED;
+  if (c.num_q_heads / c.num_kv_heads > kMaxGroup) return LYC_ERR_UNSUPPORTED;
+  if (c.max_ctx > kMaxCtxLimit) return LYC_ERR_UNSUPPORTED;
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess || c.device < 0 || c.device >= ndev)
+    return LYC_ERR_INVALID_ARG;
+  DeviceGuard guard(c.device);
+  if (!guard.ok) return LYC_ERR_CUDA;
+
+  std::unique_ptr<lyc_ctx> holder(new lyc_ctx());
+  lyc_ctx* ctx = holder.get();
+  ctx->cfg = c;
+  ctx->G = c.num_q_heads / c.num_kv_heads;
+  ctx->Hs = c.select_mode == LYC_SELECT_KVGROUP_MEAN ? c.num_kv_heads : c.num_q_heads;
+  LYC_CUDA(cudaDeviceGetAttribute(&ctx->sms, cudaDevAttrMultiProcessorCount, c.device), "SM count");
+  ctx->nstride = round_up(c.max_ctx, 4);
+  ctx->KS = static_cast<int>(round_up(c.max_k, 4));
+  const int B = c.batch, Hq = c.num_q_heads, Hkv = c.num_kv_heads, D = c.head_dim, L = c.num_layers;
+  const size_t es = c.dtype == LYC_BF16 ? 2 : 4;
+  const size_t nseg_max = static_cast<size_t>(B) * (Hkv + Hq);
+  ctx->max_parts = (static_cast<size_t>(ctx->sms) + nseg_max) * kMaxQ;
+  ctx->max_counters = nseg_max * kMaxQ;
+  auto alloc = [&](void** p, size_t bytes) -> lyc_status {
+    if (cudaMalloc(p, bytes) != cudaSuccess) {
+      cudaGetLastError();
+      return fail(ctx, LYC_ERR_OOM, "cudaMalloc failed");
+    }
+    return LYC_OK;
+  };
+  lyc_status st;
+  if ((st = alloc(reinterpret_cast<void**>(&ctx->status), 16)) != LYC_OK ||
+      (st = alloc(reinterpret_cast<void**>(&ctx->keys),
+                  static_cast<size_t>(B) * ctx->Hs * ctx->nstride * sizeof(float))) != LYC_OK ||
+      (st = alloc(reinterpret_cast<void**>(&ctx->sbuf),
+                  2ull * B * ctx->Hs * ctx->KS * sizeof(int32_t) + 64)) != LYC_OK ||
+      (st = alloc(reinterpret_cast<void**>(&ctx->part_o), ctx->max_parts * D * sizeof(float))) != LYC_OK ||
+      (st = alloc(reinterpret_cast<void**>(&ctx->part_ml), ctx->max_parts * sizeof(float2))) != LYC_OK ||
+      (st = alloc(reinterpret_cast<void**>(&ctx->counters), ctx->max_counters * sizeof(int32_t))) != LYC_OK ||
+      (st = alloc(&ctx->q_dev, static_cast<size_t>(L) * B * Hq * D * es)) != LYC_OK ||
+      (st = alloc(reinterpret_cast<void**>(&ctx->out_dev), static_cast<size_t>(L) * B * Hq * D * sizeof(float))) != LYC_OK ||
+      (st = alloc(reinterpret_cast<void**>(&ctx->S_dev), static_cast<size_t>(B) * ctx->Hs * c.max_k * sizeof(int32_t))) != LYC_OK) {
+    lyc_destroy(holder.release());
+    return st;
+  }
+  if (cudaMemset(ctx->status, 0, 16) != cudaSuccess ||
+      cudaMemset(ctx->counters, 0, ctx->max_counters * sizeof(int32_t)) != cudaSuccess ||
+      cudaMemset(ctx->sbuf, 0xff, 2ull * B * ctx->Hs * ctx->KS * sizeof(int32_t) + 64) != cudaSuccess) {
+    lyc_destroy(holder.release());
+    return LYC_ERR_CUDA;
+  }
+  cudaError_t e;
+  // kernel attributes: shared-memory sizes and the top-k cluster size
+  const int dtype = c.dtype == LYC_BF16 ? 0 : 1;
+  for (int nqb : {1, 2, 4, 5, 9}) {
+    int smem = 0;
+    if ((e = attn_dispatch(dtype, D, nqb, nullptr, 0, nullptr, &smem, true)) != cudaSuccess) {
+      lyc_destroy(holder.release());
+      return LYC_ERR_CUDA;
+    }
+  }
+  const size_t smem16 = topk_smem_for(16, static_cast<int>(c.max_ctx));
+  const size_t smem8 = topk_smem_for(8, static_cast<int>(c.max_ctx));
+  int optin = 0;
+  cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, c.device);
+  ctx->topk_cl = (smem16 <= static_cast<size_t>(optin)) ? topk_pick_cluster(smem16) : 8;
+  if (ctx->topk_cl == 8) {
+    if (smem8 > static_cast<size_t>(optin) || topk_configure(8, smem8) != cudaSuccess) {
+      lyc_destroy(holder.release());
+      return LYC_ERR_UNSUPPORTED;
+    }
+  }
+  cudaGetLastError();
+  *out = holder.release();
+  return LYC_OK;
+}
+
+void lyc_destroy(lyc_ctx* ctx) {
+  if (!ctx) return;
+  DeviceGuard guard(ctx->cfg.device);
+  for (auto& kv : ctx->plans) free_plan(kv.second.get());
+  ctx->plans.clear();
+  for (cudaEvent_t ev : ctx->events) cudaEventDestroy(ev);
+  void* bufs[] = {ctx->status, ctx->keys, ctx->sbuf, ctx->part_o, ctx->part_ml,
+                  ctx->counters, ctx->q_dev, ctx->out_dev, ctx->S_dev};
+  for (void* b : bufs)
+    if (b) cudaFree(b);
+  timed_steps().erase(ctx);
+  delete ctx;
+}
+
+}  // extern "C"
+
+extern "C" {
+
+lyc_status lyc_decode_step(lyc_ctx* ctx, const void* q, const lyc_kv_cache* kv,
+                           const uint8_t* role_mask, int k, float* out, int32_t* S,
+                           void* stream_, uint32_t step_flags) {
+  if (!ctx) return LYC_ERR_INVALID_ARG;
+  if (!q || !role_mask || !out || !S) return fail(ctx, LYC_ERR_INVALID_ARG, "NULL tensor pointer");
+  if (k < 1 || k > ctx->cfg.max_k) return fail(ctx, LYC_ERR_INVALID_ARG, "k outside [1, max_k]");
+  if (step_flags & ~(LYC_STEP_S_IN | LYC_STEP_NO_GRAPH | LYC_STEP_VALIDATE_S))
+    return fail(ctx, LYC_ERR_INVALID_ARG, "unknown step flag");
+  lyc_status st = check_kv(ctx, kv);
+  if (st != LYC_OK) return st;
+  DeviceGuard guard(ctx->cfg.device);
+  if (!guard.ok) return fail(ctx, LYC_ERR_CUDA, "cudaSetDevice failed");
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  const lyc_config& c = ctx->cfg;
+
+  const std::string key = plan_key(role_mask, c.num_layers, c.num_q_heads, kv, k, step_flags, q, out,
+                                   S, ctx->trace, ctx->timing);
+  Plan* plan = nullptr;
+  for (auto it = ctx->plans.begin(); it != ctx->plans.end(); ++it) {
+    if (it->first == key) {
+      ctx->plans.splice(ctx->plans.begin(), ctx->plans, it);
+      plan = ctx->plans.front().second.get();
+      break;
+    }
+  }
+  if (!plan) {
+    std::unique_ptr<Plan> np(new Plan());
+    np->flags = step_flags & (LYC_STEP_S_IN | LYC_STEP_VALIDATE_S);
+    np->q = q;
+    np->out = out;
+    np->S = S;
+    np->trace = ctx->trace;
+    np->timing = ctx->timing;
+    st = build_plan(ctx, np.get(), role_mask, kv, k, step_flags);
+    if (st != LYC_OK) {
+      free_plan(np.get());
+      return st;
+    }
+    ctx->plans.emplace_front(key, std::move(np));
+    plan = ctx->plans.front().second.get();
+    while (static_cast<int>(ctx->plans.size()) > kPlanCacheSize) {
+      free_plan(ctx->plans.back().second.get());
+      ctx->plans.pop_back();
+    }
+  }
+
+  int set = 0;
+  if (plan->timing) set = ctx->next_set++ % timing_sets();
+  if (step_flags & LYC_STEP_NO_GRAPH) {
+    st = enqueue_step(ctx, plan, stream, set, false);
+    if (st != LYC_OK) return st;
+  } else {
+    if (!plan->exec) {
+      st = capture_plan(ctx, plan);
+      if (st != LYC_OK) return st;
+    }
+    if (plan->timing) {
+      for (int i = 0; i < ctx->events_per_set; ++i) {
+        if (!plan->ev_nodes[i]) continue;
+        LYC_CUDA(cudaGraphExecEventRecordNodeSetEvent(
+                     plan->exec, plan->ev_nodes[i],
+                     ctx->events[static_cast<size_t>(set) * ctx->events_per_set + i]),
+                 "retarget timing event");
+      }
+    }
+    LYC_CUDA(cudaGraphLaunch(plan->exec, stream), "graph launch");
+  }
+  if (plan->timing) {
+    auto& v = timed_steps()[ctx];
+    v.push_back(TimedStep{set, plan->kernel_kind, plan->kernel_layer});
+    if (static_cast<int>(v.size()) > timing_sets()) v.erase(v.begin());
+  }
+  ctx->last_stream = stream;
+  return LYC_OK;
+}
+
+lyc_status lyc_decode_step_host(lyc_ctx* ctx, const void* q_host, const lyc_kv_cache* kv,
+                                const uint8_t* role_mask, int k, float* out_host, int32_t* S_host,
+                                void* stream_, uint32_t step_flags) {
+  if (!ctx) return LYC_ERR_INVALID_ARG;
+  if (!q_host || !out_host || !S_host) return fail(ctx, LYC_ERR_INVALID_ARG, "NULL host pointer");
+  if (k < 1 || k > ctx->cfg.max_k) return fail(ctx, LYC_ERR_INVALID_ARG, "k outside [1, max_k]");
+  DeviceGuard guard(ctx->cfg.device);
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  const lyc_config& c = ctx->cfg;
+  const size_t es = c.dtype == LYC_BF16 ? 2 : 4;
+  const size_t qbytes = static_cast<size_t>(c.num_layers) * c.batch * c.num_q_heads * c.head_dim * es;
+  const size_t obytes = static_cast<size_t>(c.num_layers) * c.batch * c.num_q_heads * c.head_dim * 4;
+  const size_t sbytes = static_cast<size_t>(c.batch) * ctx->Hs * k * 4;
+  lyc_status st = check_kv(ctx, kv);
+  if (st != LYC_OK) return st;
+  LYC_CUDA(cudaMemcpyAsync(ctx->q_dev, q_host, qbytes, cudaMemcpyHostToDevice, stream), "q to device");
+  if (step_flags & LYC_STEP_S_IN)
+    LYC_CUDA(cudaMemcpyAsync(ctx->S_dev, S_host, sbytes, cudaMemcpyHostToDevice, stream), "S to device");
+  st = lyc_decode_step(ctx, ctx->q_dev, kv, role_mask, k, ctx->out_dev, ctx->S_dev, stream_, step_flags);
+  if (st != LYC_OK) return st;
+  LYC_CUDA(cudaMemcpyAsync(out_host, ctx->out_dev, obytes, cudaMemcpyDeviceToHost, stream), "out to host");
+  LYC_CUDA(cudaMemcpyAsync(S_host, ctx->S_dev, sbytes, cudaMemcpyDeviceToHost, stream), "S to host");
+  return LYC_OK;
+}
+
+lyc_status lyc_sync_status(lyc_ctx* ctx) {
+  if (!ctx) return LYC_ERR_INVALID_ARG;
+  DeviceGuard guard(ctx->cfg.device);
+  LYC_CUDA(ctx->last_stream ? cudaStreamSynchronize(ctx->last_stream) : cudaDeviceSynchronize(),
+           "synchronize");
+  uint32_t word = 0;
+  LYC_CUDA(cudaMemcpy(&word, ctx->status, sizeof word, cudaMemcpyDeviceToHost), "read status");
+  LYC_CUDA(cudaMemset(ctx->status, 0, sizeof word), "clear status");
+  if (word & kStatusTimeout) return fail(ctx, LYC_ERR_TIMEOUT, "a device-side wait gave up");
+  if (word & (kStatusBadIndex | kStatusEmptySoftmax))
+    return fail(ctx, LYC_ERR_BAD_INDEX, "an inherited set held an index outside [0, n)");
+  return LYC_OK;
+}
+
+lyc_status lyc_set_s_trace(lyc_ctx* ctx, int32_t* trace) {
+  if (!ctx) return LYC_ERR_INVALID_ARG;
+  ctx->trace = trace;
+  return LYC_OK;
+}
+
+lyc_status lyc_set_timing(lyc_ctx* ctx, int mode) {
+  if (!ctx || (mode != LYC_TIMING_OFF && mode != LYC_TIMING_ON)) return LYC_ERR_INVALID_ARG;
+  DeviceGuard guard(ctx->cfg.device);
+  if (mode == LYC_TIMING_ON && ctx->events.empty()) {
+    ctx->events_per_set = 4 * ctx->cfg.num_layers;
+    const size_t total = static_cast<size_t>(timing_sets()) * ctx->events_per_set;
+    ctx->events.resize(total, nullptr);
+    for (size_t i = 0; i < total; ++i)
+      LYC_CUDA(cudaEventCreate(&ctx->events[i]), "cudaEventCreate");
+  }
+  ctx->timing = mode == LYC_TIMING_ON;
+  return LYC_OK;
+}
+
+lyc_status lyc_kernel_times(lyc_ctx* ctx, lyc_kernel_time* times, int cap, int* count) {
+  if (!ctx || !count || (cap > 0 && !times)) return LYC_ERR_INVALID_ARG;
+  DeviceGuard guard(ctx->cfg.device);
+  LYC_CUDA(ctx->last_stream ? cudaStreamSynchronize(ctx->last_stream) : cudaDeviceSynchronize(),
+           "synchronize");
+  int nout = 0;
+  auto& v = timed_steps()[ctx];
+  for (const TimedStep& ts : v) {
+    for (size_t i = 0; i < ts.kind.size(); ++i) {
+      if (nout >= cap) break;
+      float ms = 0.f;
+      const size_t base = static_cast<size_t>(ts.set) * ctx->events_per_set;
+      LYC_CUDA(cudaEventElapsedTime(&ms, ctx->events[base + 2 * i], ctx->events[base + 2 * i + 1]),
+               "event elapsed time");
+      times[nout].kind = ts.kind[i];
+      times[nout].layer = ts.layer[i];
+      times[nout].ms = ms;
+      ++nout;
+    }
+  }
+  v.clear();
+  *count = nout;
+  return LYC_OK;
+}
+
+lyc_status lyc_topk_f32(lyc_ctx* ctx, const float* keys, int64_t n, int k, int32_t* S, void* stream) {
+  if (!ctx) return LYC_ERR_INVALID_ARG;
+  if (!keys || !S) return fail(ctx, LYC_ERR_INVALID_ARG, "NULL pointer");
+  if (n < 1 || n > ctx->cfg.max_ctx) return fail(ctx, LYC_ERR_INVALID_ARG, "n outside [1, max_ctx]");
+  if (k < 1 || k > ctx->cfg.max_k) return fail(ctx, LYC_ERR_INVALID_ARG, "k outside [1, max_k]");
+  DeviceGuard guard(ctx->cfg.device);
+  TopkParams tp{};
+  tp.tasks = nullptr;
+  tp.single.keys = keys;
+  tp.single.S = S;
+  tp.n = static_cast<int>(n);
+  tp.k = k;
+  LYC_CUDA(topk_launch(ctx->topk_cl, &tp, 1, static_cast<cudaStream_t>(stream)), "top-k launch");
+  ctx->last_stream = static_cast<cudaStream_t>(stream);
+  return LYC_OK;
+}
+
+lyc_status lyc_step_bytes(const lyc_config* cfg, const uint8_t* role_mask, int64_t n, int k, int s_in,
+                          uint64_t* analytic, uint64_t* distinct) {
+  if (!cfg || !role_mask || !analytic || !distinct || n < 1 || k < 1) return LYC_ERR_INVALID_ARG;
+  const lyc_config& c = *cfg;
+  if (c.num_kv_heads < 1 || c.num_q_heads % c.num_kv_heads != 0) return LYC_ERR_INVALID_ARG;
+  const int G = c.num_q_heads / c.num_kv_heads;
+  const uint64_t row = static_cast<uint64_t>(c.head_dim) * (c.dtype == LYC_BF16 ? 2 : 4) * 2;  // K + V
+  const uint64_t keff = static_cast<uint64_t>(std::min<int64_t>(k, n));
+  const bool kvmode = c.select_mode == LYC_SELECT_KVGROUP_MEAN;
+  uint64_t a = 0, d = 0;
+  for (int l = 0; l < c.num_layers; ++l) {
+    for (int g = 0; g < c.num_kv_heads; ++g) {
+      int nret = 0, nsp = 0;
+      for (int h = g * G; h < (g + 1) * G; ++h) {
+        const bool r = (l == 0 && !s_in) || role_mask[static_cast<int64_t>(l) * c.num_q_heads + h];
+        nret += r;
+        nsp += !r;
+      }
+      const uint64_t full = static_cast<uint64_t>(n) * row, part = keff * row;
+      a += nret ? full : part;
+      d += nret ? full : 0;
+      d += kvmode ? (nsp ? part : 0) : static_cast<uint64_t>(nsp) * part;
+    }
+  }
+  *analytic = a * c.batch;
+  *distinct = d * c.batch;
+  return LYC_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,100 @@
+// lyc_plan.h -- work-list records shared by the host planner and the kernels.
+//
+// One layer of the step is a pool of segments (page "LycheeDecode ...",
+// paper-graph-ui summary, Appendix C / Algorithm 2, "workload pooling"):
+//   dense segment  : one (batch b, KV group g); rows 0..n-1 of the group's
+//                    K/V; query vectors = the group's retrieval heads (plus,
+//                    in KV-group selection mode, the group's mean query,
+//                    which only produces selection keys);
+//   sparse segment : one inherited set; rows = the set's list positions
+//                    0..k_eff-1; query vectors = the sparse heads that read
+//                    that set (one head per set in per-head mode, all sparse
+//                    heads of the group in KV-group mode).
+// The pooled rows are cut into equal runs of 64-row tiles, one run per CTA.
+// A run that crosses segment boundaries becomes several pieces.  Each piece
+// writes one partial softmax state (m, l, o[d]) per output query vector; the
+// last piece of a segment to finish merges them (log-sum-exp) into `out`.
+#pragma once
+#include <stdint.h>
+
+namespace lyc {
+
+constexpr int kTileRows = 64;      // rows per pipeline stage (the pages' block size)
+constexpr int kMaxGroup = 8;       // largest Hq / Hkv supported
+constexpr int kMaxQ = kMaxGroup + 1;  // query vectors per segment (+ the mean query)
+
+enum SegKind : int32_t { kDense = 0, kSparse = 1 };
+
+struct Segment {
+  const void* k;        // K rows of (l, b, g): row i at k + i * s_token elements
+  const void* v;        // V rows, same layout
+  const int32_t* idx;   // sparse: the inherited set (list positions -> token index)
+  int64_t s_token;      // element stride between rows
+  int64_t key_off[kMaxQ];  // element offset of this query vector's selection-key row
+                           // in the key buffer, or -1
+  int32_t kind;         // SegKind
+  int32_t b, g;
+  int32_t rows;         // dense: n; sparse: k_eff (valid list entries)
+  int32_t nq;           // query vectors in use
+  int32_t nout;         // the first nout query vectors produce outputs
+  int32_t head[kMaxQ];  // query head of each vector; -1 = mean of the group's queries
+  int32_t part_base;    // first partial record of this segment
+  int32_t npieces;      // pieces the segment was cut into
+  int32_t cnt_base;     // first arrival counter of this segment (nout counters)
+  int32_t pad_;
+};
+
+struct Piece {
+  int32_t seg;      // segment index within the layer
+  int32_t r0, r1;   // row range within the segment (token or list positions)
+  int32_t ordinal;  // which piece of its segment (partials at part_base + ordinal*nout + j)
+};
+
+struct AttnParams {
+  const Segment* segs;
+  const Piece* pieces;
+  const int32_t* cta_begin;  // pieces of CTA c: [cta_begin[c], cta_begin[c+1])
+  const void* q;             // this layer's queries, [B][Hq][d]
+  float* out;                // this layer's outputs, [B][Hq][d]
+  float* keys;               // selection-key buffer
+  float* part_o;             // [parts][d]
+  float2* part_ml;           // [parts] (running max in log2 units, sum)
+  int32_t* counters;         // arrival counters, left at zero after use
+  uint32_t* status;          // device status word
+  int32_t Hq, G, n;
+  float scale_log2;          // log2(e) / sqrt(d)
+  float scale;               // 1 / sqrt(d)
+};
+
+struct TopkTask {
+  const float* keys;  // n selection keys
+  int32_t* S;         // k outputs
+};
+
+struct TopkParams {
+  const TopkTask* tasks;  // one per blockIdx.y; NULL: use `single`
+  TopkTask single;
+  int32_t n, k;
+};
+
+// copy_sets_kernel: dst[(b*Hs + s)*k + j] = src[b*Hs + s][j] for j < k
+struct CopySetsParams {
+  const int32_t* const* src;
+  int32_t* dst;
+  int32_t nsets, k;
+};
+
+// validate_sets_kernel: each of nsets sets (stride `stride`) must hold k_eff
+// ascending indices in [0, n) followed by -1 up to k
+struct ValidateSetsParams {
+  const int32_t* sets;
+  uint32_t* status;
+  int32_t nsets, stride, k, k_eff, n;
+};
+
+// status word bits
+constexpr uint32_t kStatusBadIndex = 1u;
+constexpr uint32_t kStatusTimeout = 2u;
+constexpr uint32_t kStatusEmptySoftmax = 4u;
+
+}  // namespace lyc

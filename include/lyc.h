@@ -1,0 +1,178 @@
+/*
+ * lyc.h -- C ABI of liblyc.so, the B200 (sm_100a) hybrid-head sparse
+ * decode-attention step of LycheeDecode.
+ *
+ * The operation (page "LycheeDecode: Accelerating Long-Context LLM Inference
+ * via Hybrid-Head Sparse Decoding", paper-graph-ui summary):
+ *   for each layer l = 0..L-1, batch element b and query head h
+ *   - retrieval head (section 3.4 Eq. 1; Appendix B, Algorithm 1):
+ *       o = softmax(q K^T / sqrt(d)) V over all n cached rows of h's KV group,
+ *       then S^(l+1) = argsTopK of its scores, k rows (section 3.4 Eq. 2);
+ *   - sparse head (section 3.4 Eq. 3): o = softmax(q K[S]^T / sqrt(d)) V[S]
+ *       over the k rows of the set it inherits, which it passes on unchanged;
+ *   - every head of layer 0 is a retrieval head (section 3.4, initialisation
+ *     of the propagation chain);
+ *   - GQA: query head h uses KV head h / (Hq/Hkv).  In LYC_SELECT_KVGROUP_MEAN
+ *     the group's queries are averaged before selection, one set per KV group
+ *     (section 3.4, hyperparameter summary: "Q heads average-pooled").
+ * Readings where the pages are silent: top-k is taken over the logits (same
+ * set as over softmax scores), ties go to the lower token index, -0 == +0,
+ * S is stored in ascending order and padded with -1 when k > n.
+ *
+ * Conventions for every entry point:
+ *   - All tensors are owned by the caller and must stay valid until the work
+ *     enqueued on `stream` has finished.  Device pointers live on the
+ *     context's device.  The library never frees caller memory.
+ *   - The library owns its scratch (partial softmax states, selection keys,
+ *     set buffers, work lists) and its CUDA graphs; lyc_destroy frees them.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t, NULL = legacy
+ *     default stream).  A context is not thread-safe.
+ *   - Errors found on the host are returned at once and nothing is enqueued.
+ *     Errors found on the device (bad inherited index, wait timeout) are
+ *     latched in a device status word and returned by lyc_sync_status.
+ */
+#ifndef LYC_H_
+#define LYC_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  LYC_OK = 0,
+  LYC_ERR_INVALID_ARG = -1, /* bad pointer, shape, stride, alignment or k */
+  LYC_ERR_UNSUPPORTED = -2, /* shape outside what the kernels are built for */
+  LYC_ERR_OOM = -3,         /* a library allocation failed */
+  LYC_ERR_CUDA = -4,        /* a CUDA call failed; see lyc_last_error */
+  LYC_ERR_BAD_INDEX = -5,   /* an inherited set held an index outside [0, n) */
+  LYC_ERR_TIMEOUT = -6      /* a device-side wait gave up (kernel returned early) */
+} lyc_status;
+
+typedef enum { LYC_BF16 = 0, LYC_FP32 = 1 } lyc_dtype;
+
+typedef enum {
+  LYC_SELECT_PER_QHEAD = 0,   /* one set per query head: Hs = Hq */
+  LYC_SELECT_KVGROUP_MEAN = 1 /* one set per KV head, key from the mean query: Hs = Hkv */
+} lyc_select_mode;
+
+typedef struct {
+  int num_layers;   /* L >= 1 */
+  int batch;        /* B >= 1 */
+  int num_q_heads;  /* Hq >= 1 */
+  int num_kv_heads; /* Hkv >= 1, Hq % Hkv == 0, Hq / Hkv <= 8 */
+  int head_dim;     /* d in {64, 128} */
+  int64_t max_ctx;  /* largest n any step will use, 1 <= max_ctx <= 786432 */
+  int max_k;        /* largest k any step will use, >= 1 */
+  lyc_dtype dtype;  /* element type of q, K and V */
+  lyc_select_mode select_mode;
+  int device;       /* CUDA device ordinal */
+  uint32_t flags;   /* reserved, pass 0 */
+} lyc_config;
+
+/* The KV cache of all layers.  Element (l, b, g, i, j) of K (and of V) is at
+ * element offset l*s_layer + b*s_batch + g*s_head + i*s_token + j, j < d
+ * contiguous.  All strides are in elements and must make every row start on a
+ * 16-byte boundary (s_token*elem, s_head*elem, ... multiples of 16 bytes; base
+ * pointers 16-byte aligned).  n rows are valid, the current token included
+ * (it is appended before attention, Algorithm 1). */
+typedef struct {
+  const void* k;
+  const void* v;
+  int64_t n;
+  int64_t s_layer, s_batch, s_head, s_token;
+} lyc_kv_cache;
+
+/* step_flags */
+#define LYC_STEP_S_IN 0x1u       /* S holds S^(0) on entry; role row 0 is obeyed */
+#define LYC_STEP_NO_GRAPH 0x2u   /* launch the kernels directly, no CUDA graph */
+#define LYC_STEP_VALIDATE_S 0x4u /* with S_IN: check S^(0) on the device first */
+
+typedef struct lyc_ctx lyc_ctx;
+
+/* Create a context on cfg->device.  Allocates the library's scratch for the
+ * largest step the config allows.  *out receives the context.
+ * Errors: INVALID_ARG (NULL, bad sizes), UNSUPPORTED (d, dtype, group size),
+ * OOM, CUDA. */
+lyc_status lyc_create(const lyc_config* cfg, lyc_ctx** out);
+
+/* One decode step of the L-layer attention stack.
+ *   q         device, [L][B][Hq][d] of cfg->dtype, contiguous
+ *   kv        host struct describing the device KV cache (n <= max_ctx)
+ *   role_mask host, [L][Hq] uint8, 1 = retrieval head.  Row 0 is ignored
+ *             (all retrieval) unless LYC_STEP_S_IN is set.
+ *   k         token budget, 1 <= k <= max_k; k > n selects all n rows and
+ *             pads the rest of each set with -1
+ *   out       device, [L][B][Hq][d] float32, contiguous; fully written
+ *   S         device, [B][Hs][k] int32, contiguous.  In: S^(0) when
+ *             LYC_STEP_S_IN.  Out: S^(L), each set ascending, -1 padded.
+ *   stream    cudaStream_t
+ * The first step with a given (role mask, n, k, flags, pointers) builds the
+ * work lists and captures a CUDA graph; later identical steps replay it.
+ * Errors: INVALID_ARG, CUDA (host side); BAD_INDEX, TIMEOUT (device side,
+ * via lyc_sync_status). */
+lyc_status lyc_decode_step(lyc_ctx* ctx, const void* q, const lyc_kv_cache* kv,
+                           const uint8_t* role_mask, int k, float* out, int32_t* S,
+                           void* stream, uint32_t step_flags);
+
+/* The same step with q, out and S in HOST memory (pinned memory gives
+ * asynchronous copies).  The host-to-device copy of q (and of S with
+ * LYC_STEP_S_IN) and the device-to-host copies of out and S are enqueued on
+ * `stream` around the step, into library-owned device buffers.  The KV cache
+ * stays on the device.  The host buffers must stay valid until the stream
+ * has finished the step. */
+lyc_status lyc_decode_step_host(lyc_ctx* ctx, const void* q_host, const lyc_kv_cache* kv,
+                                const uint8_t* role_mask, int k, float* out_host,
+                                int32_t* S_host, void* stream, uint32_t step_flags);
+
+/* Synchronize the stream of the last step, read and clear the device status
+ * word.  Returns LYC_OK, LYC_ERR_BAD_INDEX, LYC_ERR_TIMEOUT or LYC_ERR_CUDA. */
+lyc_status lyc_sync_status(lyc_ctx* ctx);
+
+/* Record every layer's outgoing sets: trace is device [L][B][Hs][k] int32
+ * (k of the steps that follow); trace[l] = the sets after layer l.  NULL turns
+ * recording off.  Debug and test use; it adds one small copy per layer. */
+lyc_status lyc_set_s_trace(lyc_ctx* ctx, int32_t* trace);
+
+/* Bytes one step must read from the KV cache (host-only arithmetic).
+ *   analytic: full K+V of every KV group with a retrieval head at a layer,
+ *             plus min(k, n) K+V rows for every group with sparse heads only.
+ *   distinct: K+V bytes the kernels actually read: full groups as above, and
+ *             for every sparse-head pass (per query head in PER_QHEAD mode, per
+ *             group in KVGROUP_MEAN mode) min(k, n) rows, including the passes
+ *             of sparse heads that sit in a retrieval group.
+ * s_in != 0: role row 0 is obeyed (as with LYC_STEP_S_IN). */
+lyc_status lyc_step_bytes(const lyc_config* cfg, const uint8_t* role_mask, int64_t n, int k,
+                          int s_in, uint64_t* analytic, uint64_t* distinct);
+
+/* Test hook for the selection kernel alone: S[0..k) = argsTopK(keys[0..n), k)
+ * with ties to the lower index, ascending, -1 padded.  keys and S are device
+ * pointers (keys float32 [n], S int32 [k]); n <= max_ctx, k <= max_k. */
+lyc_status lyc_topk_f32(lyc_ctx* ctx, const float* keys, int64_t n, int k, int32_t* S,
+                        void* stream);
+
+/* Per-kernel device time of the steps since the last call, from CUDA events
+ * recorded around every launch when timing is on (LYC_TIMING_ON).  Writes up
+ * to `cap` entries of {kernel kind, layer, milliseconds}; returns the count in
+ * *count.  Kinds: 0 = attention (pooled dense + sparse), 1 = top-k selection. */
+typedef struct {
+  int kind;
+  int layer;
+  float ms;
+} lyc_kernel_time;
+#define LYC_TIMING_OFF 0
+#define LYC_TIMING_ON 1
+lyc_status lyc_set_timing(lyc_ctx* ctx, int mode);
+lyc_status lyc_kernel_times(lyc_ctx* ctx, lyc_kernel_time* times, int cap, int* count);
+
+const char* lyc_status_string(lyc_status s);
+const char* lyc_last_error(const lyc_ctx* ctx);
+void lyc_destroy(lyc_ctx* ctx);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LYC_H_ */

@@ -1,0 +1,87 @@
+"""Helpers that compare the CUDA library's step with the fp64 oracle.
+
+Tolerances (stated for the decode step's outputs): fp32 inputs
+|gpu - oracle| <= 1e-5 + 1e-5 |oracle|; bf16 inputs <= 2e-3 + 2e-2 |oracle|.
+Selected sets: with tau the oracle's k_eff-th largest selection key, the GPU
+set must hold k_eff distinct ascending indices, contain every index whose key
+exceeds tau + 1e-3, hold none whose key is below tau - 1e-3, and pad with -1.
+Layers are checked with teacher forcing: layer l of the oracle inherits the
+GPU's own sets after layer l-1, so one near-tie cannot cascade.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+import oracle as O
+from hybrid_head_sparse_b200 import workloads as W
+
+TOL = {"fp32": (1e-5, 1e-5), "bf16": (2e-3, 2e-2)}
+TIE_BAND = 1e-3
+
+
+def check_set(gpu_set: np.ndarray, keys: np.ndarray, k: int, what: str):
+    n = keys.size
+    keff = min(k, n)
+    assert gpu_set.shape == (k,)
+    assert np.all(gpu_set[keff:] == -1), f"{what}: padding is not -1"
+    sel = gpu_set[:keff]
+    assert np.all(sel >= 0) and np.all(sel < n), f"{what}: index out of range"
+    assert np.all(np.diff(sel) > 0), f"{what}: not strictly ascending"
+    if keff == n:
+        return
+    tau = np.sort(keys)[::-1][keff - 1]
+    must = np.nonzero(keys > tau + TIE_BAND)[0]
+    mustnt = set(np.nonzero(keys < tau - TIE_BAND)[0].tolist())
+    s = set(sel.tolist())
+    missing = [i for i in must.tolist() if i not in s]
+    wrong = [i for i in sel.tolist() if i in mustnt]
+    assert not missing, f"{what}: {len(missing)} clearly-selected indices missing, e.g. {missing[:5]}"
+    assert not wrong, f"{what}: {len(wrong)} clearly-unselected indices chosen, e.g. {wrong[:5]}"
+
+
+def check_out(gpu: np.ndarray, ora: np.ndarray, dtype: str, what: str):
+    atol, rtol = TOL[dtype]
+    err = np.abs(gpu.astype(np.float64) - ora)
+    bound = atol + rtol * np.abs(ora)
+    bad = err > bound
+    assert not bad.any(), (f"{what}: {int(bad.sum())} of {bad.size} outputs off; "
+                           f"max err {err.max():.3e} (bound there {bound.flat[err.argmax()]:.3e})")
+    return float(err.max())
+
+
+def host_stack(data: dict, layers=None, select_mode=O.SELECT_PER_QHEAD) -> O.Stack:
+    """Host copy of the step's inputs (optionally only some layers)."""
+    q, K, V = data["q"], data["k"], data["v"]
+    role = data["role"]
+    if layers is not None:
+        idx = list(layers)
+        q, K, V, role = q[idx], K[idx], V[idx], role[idx]
+    return O.Stack(W.host_view(q), W.host_view(K), W.host_view(V),
+                   np.ascontiguousarray(role, dtype=np.uint8), select_mode)
+
+
+def check_layers(data: dict, out: np.ndarray, trace: np.ndarray, k: int, n: int, dtype: str,
+                 layers, select_mode=O.SELECT_PER_QHEAD, S0: np.ndarray | None = None):
+    """Check the chosen layers of a GPU step (out [L][B][Hq][d], trace
+    [L][B][Hs][k]) against the oracle with teacher forcing.  S0: the sets
+    handed to layer 0 (set-input mode) or None (layer 0 all retrieval)."""
+    worst = 0.0
+    for l in layers:
+        st = host_stack(data, layers=[l], select_mode=select_mode)
+        if l == 0:
+            S_in = S0
+            all_ret = S0 is None
+        else:
+            S_in = trace[l - 1]
+            all_ret = False
+        o, S_out, keys, fresh = O.layer(st, 0, k, S_in, all_retrieval=all_ret, n=n)
+        worst = max(worst, check_out(out[l], o, dtype, f"layer {l} outputs"))
+        B, Hs = S_out.shape[:2]
+        for b in range(B):
+            for s in range(Hs):
+                if fresh[s]:
+                    check_set(trace[l, b, s], keys[b, s], k, f"layer {l} b {b} set {s}")
+                else:
+                    assert np.array_equal(trace[l, b, s], S_in[b, s]), \
+                        f"layer {l} b {b} set {s}: an unrefreshed set changed"
+    return worst

@@ -1,0 +1,237 @@
+"""The CUDA library (through its C ABI) against the fp64 oracle, on a B200."""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from hybrid_head_sparse_b200 import workloads as W
+from tests import parity as P
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def lyc():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from hybrid_head_sparse_b200 import lyc as lycmod
+    lycmod.load()
+    return lycmod
+
+
+def run_step(lyc, spec: W.StackSpec, select_mode="per_qhead", data=None, s_in=None,
+             no_graph=False, k=None, n=None):
+    """One library step on the spec's inputs; returns (data, out, S, trace) on the host."""
+    data = data or W.make_stack(spec, "cuda")
+    k = k or spec.k
+    n = n or spec.n
+    ctx = lyc.Lyc(spec.L, spec.B, spec.Hq, spec.Hkv, spec.d, max(spec.rows, n), k,
+                  dtype=spec.dtype, select_mode=select_mode)
+    Hs = ctx.Hs
+    out = torch.full((spec.L, spec.B, spec.Hq, spec.d), float("nan"), device="cuda")
+    S = torch.full((spec.B, Hs, k), -7, dtype=torch.int32, device="cuda")
+    if s_in is not None:
+        S.copy_(s_in)
+    trace = torch.full((spec.L, spec.B, Hs, k), -7, dtype=torch.int32, device="cuda")
+    ctx.set_trace(trace)
+    ctx.decode_step(data["q"], data["k"], data["v"], n, data["role"], k, out, S,
+                    s_in=s_in is not None, no_graph=no_graph)
+    assert ctx.sync_status() == 0, lyc.lyc_last_error(ctx.ctx)
+    torch.cuda.synchronize()
+    res = (out.cpu().numpy(), S.cpu().numpy(), trace.cpu().numpy())
+    ctx.close()
+    return (data,) + res
+
+
+# ---------------------------------------------------------------- selection kernel
+
+
+@pytest.mark.parametrize("n,k", [(1, 1), (5, 3), (64, 64), (100, 7), (513, 64), (4096, 1000),
+                                 (131072, 4096), (131071, 4097), (1000, 999), (777, 800)])
+def test_topk_bitexact_integer_keys(lyc, n, k):
+    """Integer-valued keys with many ties: the GPU selection is bit-exact."""
+    rng = np.random.default_rng(n * 7 + k)
+    x = rng.integers(-6, 7, size=n).astype(np.float32)
+    x[rng.random(n) < 0.1] = -0.0
+    ctx = lyc.Lyc(1, 1, 1, 1, 64, max(n, 1), k, dtype="fp32")
+    keys = torch.from_numpy(x).cuda()
+    S = torch.full((k,), -7, dtype=torch.int32, device="cuda")
+    ctx.topk_f32(keys, n, k, S)
+    assert ctx.sync_status() == 0
+    exp = O.topk(x.astype(np.float64), k)
+    assert np.array_equal(S.cpu().numpy(), exp)
+    ctx.close()
+
+
+def test_topk_distinct_and_all_equal(lyc):
+    ctx = lyc.Lyc(1, 1, 1, 1, 64, 200000, 5000, dtype="fp32")
+    rng = np.random.default_rng(3)
+    for x in (rng.standard_normal(200000).astype(np.float32),
+              np.full(200000, 0.5, dtype=np.float32),
+              np.concatenate([np.full(100000, -np.inf), rng.standard_normal(100000)]).astype(np.float32)):
+        for k in (1, 4096, 5000):
+            keys = torch.from_numpy(x).cuda()
+            S = torch.full((k,), -7, dtype=torch.int32, device="cuda")
+            ctx.topk_f32(keys, x.size, k, S)
+            assert ctx.sync_status() == 0
+            assert np.array_equal(S.cpu().numpy(), O.topk(x.astype(np.float64), k))
+    ctx.close()
+
+
+# ---------------------------------------------------------------- whole steps
+
+
+def test_tiny_stack_fp32(lyc):
+    spec = W.TINY
+    data, out, S, tr = run_step(lyc, spec)
+    P.check_layers(data, out, tr, spec.k, spec.n, "fp32", range(spec.L))
+    assert np.array_equal(S, tr[-1])
+    # without teacher forcing: the oracle's own whole step agrees as well
+    o_out, o_S, _ = O.decode_step(P.host_stack(data), spec.k, trace=True)
+    P.check_out(out, o_out, "fp32", "whole step")
+
+
+def test_tiny_stack_fp32_no_graph_matches_graph(lyc):
+    spec = W.TINY
+    data, out_g, S_g, tr_g = run_step(lyc, spec)
+    _, out_n, S_n, tr_n = run_step(lyc, spec, data=data, no_graph=True)
+    assert np.array_equal(out_g, out_n) and np.array_equal(S_g, S_n) and np.array_equal(tr_g, tr_n)
+
+
+SMALL_BF16 = W.StackSpec("small-llama-like", L=4, B=2, Hq=32, Hkv=8, d=128, n=3001, k=256,
+                         retrieval_per_layer=3, n_planted=64, seed=5)
+
+
+@pytest.mark.parametrize("mode", ["per_qhead", "kvgroup_mean"])
+def test_small_bf16_stack(lyc, mode):
+    spec = SMALL_BF16
+    om = O.SELECT_PER_QHEAD if mode == "per_qhead" else O.SELECT_KVGROUP_MEAN
+    data, out, S, tr = run_step(lyc, spec, select_mode=mode)
+    P.check_layers(data, out, tr, spec.k, spec.n, "bf16", range(spec.L), select_mode=om)
+    assert np.array_equal(S, tr[-1])
+
+
+@pytest.mark.parametrize("mode", ["per_qhead", "kvgroup_mean"])
+def test_edge_shapes(lyc, mode):
+    om = O.SELECT_PER_QHEAD if mode == "per_qhead" else O.SELECT_KVGROUP_MEAN
+    cases = [
+        W.StackSpec("n1", L=2, B=1, Hq=2, Hkv=1, d=64, n=1, k=1, dtype="fp32", roles="first-head",
+                    planted="none"),
+        W.StackSpec("k>n", L=3, B=2, Hq=4, Hkv=4, d=64, n=70, k=100, dtype="fp32",
+                    retrieval_per_layer=1, planted="none"),
+        W.StackSpec("k=n", L=2, B=1, Hq=8, Hkv=2, d=128, n=130, k=130, retrieval_per_layer=2,
+                    planted="none"),
+        W.StackSpec("mha-d64-bf16", L=3, B=1, Hq=6, Hkv=6, d=64, n=1000, k=65,
+                    retrieval_per_layer=2, planted="none", seed=2),
+        W.StackSpec("group8", L=2, B=1, Hq=16, Hkv=2, d=128, n=700, k=63, retrieval_per_layer=3,
+                    planted="none", seed=4),
+        W.StackSpec("fp32-d128", L=2, B=1, Hq=4, Hkv=2, d=128, n=333, k=40, dtype="fp32",
+                    retrieval_per_layer=1, planted="none", seed=6),
+        W.StackSpec("padded-rows", L=2, B=1, Hq=4, Hkv=2, d=64, n=200, k=32, dtype="fp32",
+                    retrieval_per_layer=1, planted="none", seed=7, n_max=260),
+    ]
+    for spec in cases:
+        data, out, S, tr = run_step(lyc, spec, select_mode=mode)
+        P.check_layers(data, out, tr, spec.k, spec.n, spec.dtype, range(spec.L), select_mode=om)
+
+
+def test_k_ge_n_sparse_equals_dense(lyc):
+    spec = W.StackSpec("kgen", L=2, B=1, Hq=4, Hkv=2, d=64, n=90, k=90, dtype="fp32",
+                       roles="first-head", planted="none", seed=3)
+    data, out, S, tr = run_step(lyc, spec)
+    dense = dict(data)
+    dense["role"] = np.ones_like(data["role"])
+    _, out_d, _, _ = run_step(lyc, spec, data=dense)
+    # same rows, same order of tiles: sparse heads reproduce the dense result
+    np.testing.assert_allclose(out, out_d, rtol=1e-6, atol=1e-6)
+    assert np.array_equal(S[0, 1], np.arange(90))
+
+
+@pytest.mark.parametrize("pattern", ["blocks", "scattered"])
+def test_set_input_single_layer(lyc, pattern):
+    """One layer with inherited sets given (the single-layer kernel sweep form)."""
+    spec = W.StackSpec("one-layer", L=1, B=2, Hq=32, Hkv=8, d=128, n=16384, k=1024,
+                       planted="heavy", n_planted=64, seed=8)
+    data = W.make_stack(spec, "cuda")
+    role = np.zeros((1, 32), dtype=np.uint8)
+    role[0, [3, 17]] = 1
+    data["role"] = role
+    S0 = W.inherited_sets(spec.B, spec.Hq, spec.n, spec.k, pattern, seed=1, device="cuda")
+    _, out, S, tr = run_step(lyc, spec, data=data, s_in=S0)
+    P.check_layers(data, out, tr, spec.k, spec.n, "bf16", [0], S0=S0.cpu().numpy())
+
+
+def test_bad_inherited_index_reported(lyc):
+    """An out-of-range index handed in is skipped by the kernel's bounds check
+    and reported through the status word."""
+    spec = W.StackSpec("bad", L=1, B=1, Hq=2, Hkv=1, d=64, n=100, k=8, dtype="fp32",
+                       planted="none")
+    data = W.make_stack(spec, "cuda")
+    data["role"] = np.array([[1, 0]], dtype=np.uint8)
+    S0 = torch.arange(8, dtype=torch.int32, device="cuda").repeat(1, 2, 1).contiguous()
+    S0[0, 1, 5] = 1000
+    ctx = lyc.Lyc(1, 1, 2, 1, 64, 100, 8, dtype="fp32")
+    out = torch.zeros((1, 1, 2, 64), device="cuda")
+    S = S0.clone()
+    ctx.decode_step(data["q"], data["k"], data["v"], 100, data["role"], 8, out, S, s_in=True)
+    assert ctx.sync_status() == lyc.LYC_ERR_BAD_INDEX
+    # the context stays usable
+    S = S0.clone()
+    S[0, 1, 5] = 5
+    ctx.decode_step(data["q"], data["k"], data["v"], 100, data["role"], 8, out, S, s_in=True)
+    assert ctx.sync_status() == 0
+    ctx.close()
+
+
+def test_host_buffer_entry_matches_device_entry(lyc):
+    spec = W.TINY
+    data, out, S, _ = run_step(lyc, spec)
+    ctx = lyc.Lyc(spec.L, spec.B, spec.Hq, spec.Hkv, spec.d, spec.n, spec.k, dtype="fp32")
+    q_host = data["q"].cpu().pin_memory()
+    out_h = torch.empty((spec.L, spec.B, spec.Hq, spec.d)).pin_memory()
+    S_h = torch.empty((spec.B, ctx.Hs, spec.k), dtype=torch.int32).pin_memory()
+    ctx.decode_step_host(q_host, data["k"], data["v"], spec.n, data["role"], spec.k, out_h, S_h)
+    assert ctx.sync_status() == 0
+    assert np.array_equal(out_h.numpy(), out) and np.array_equal(S_h.numpy(), S)
+    ctx.close()
+
+
+def test_repeat_is_deterministic(lyc):
+    spec = SMALL_BF16.with_(L=3, B=1)
+    data, out1, S1, tr1 = run_step(lyc, spec)
+    _, out2, S2, tr2 = run_step(lyc, spec, data=data)
+    assert np.array_equal(out1, out2) and np.array_equal(tr1, tr2)
+
+
+def test_invalid_arguments_rejected(lyc):
+    ctx = lyc.Lyc(1, 1, 2, 1, 64, 128, 8, dtype="fp32")
+    K = torch.zeros((1, 1, 1, 128, 64), device="cuda")
+    q = torch.zeros((1, 1, 2, 64), device="cuda")
+    out = torch.zeros((1, 1, 2, 64), device="cuda")
+    S = torch.zeros((1, 2, 8), dtype=torch.int32, device="cuda")
+    role = np.ones((1, 2), dtype=np.uint8)
+    with pytest.raises(lyc.LycError):
+        ctx.decode_step(q, K, K, 129, role, 8, out, S)      # n > max_ctx
+    with pytest.raises(lyc.LycError):
+        ctx.decode_step(q, K, K, 128, role, 9, out, S)      # k > max_k
+    with pytest.raises(lyc.LycError):
+        ctx.decode_step(q, K, K, 0, role, 8, out, S)        # empty cache
+    ctx.close()
+
+
+def test_strided_rows(lyc):
+    """Rows padded past d (token stride > d): the row-gather path serves the
+    dense heads too."""
+    spec = W.StackSpec("strided", L=2, B=1, Hq=4, Hkv=2, d=64, n=300, k=40, dtype="fp32",
+                       retrieval_per_layer=1, planted="none", seed=9)
+    data = W.make_stack(spec, "cuda")
+    Kp = torch.full((2, 1, 2, 300, 68), 1e30, device="cuda")
+    Vp = torch.full((2, 1, 2, 300, 68), -1e30, device="cuda")
+    Kp[..., :64] = data["k"]
+    Vp[..., :64] = data["v"]
+    strided = dict(data)
+    strided["k"] = Kp[..., :64]
+    strided["v"] = Vp[..., :64]
+    _, out, S, tr = run_step(lyc, spec, data=strided)
+    P.check_layers(data, out, tr, spec.k, spec.n, "fp32", range(spec.L))

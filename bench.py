@@ -31,7 +31,7 @@ if ROOT not in sys.path:
 METRIC = "attn-stack decode steps/s at 128K ctx, k=4096; HBM GB/s vs peak"
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
-ATTN_SOURCES = ["attn_kernel.cu", "lyc_plan.h", "lyc_device.cuh"]
+ATTN_SOURCES = ["attn_mma_kernel.cu", "lyc_plan.h", "lyc_device.cuh"]
 
 
 def parse_args(argv=None):
@@ -42,6 +42,7 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=["lyc", "reference"], default="lyc")
     ap.add_argument("--n", type=int, default=131072)
     ap.add_argument("--k", type=int, default=4096)
+    ap.add_argument("--layers", type=int, default=32, help="layers of the stack (32 = the workload)")
     ap.add_argument("--retrieval-heads", type=int, default=2,
                     help="retrieval query heads per layer after layer 0; -1 = all (dense baseline)")
     ap.add_argument("--select-mode", choices=["per_qhead", "kvgroup_mean"], default="per_qhead")
@@ -54,7 +55,7 @@ def parse_args(argv=None):
 
 def workload_spec(args):
     from hybrid_head_sparse_b200 import workloads as W
-    spec = W.LLAMA3_8B_128K.with_(n=args.n, k=args.k)
+    spec = W.LLAMA3_8B_128K.with_(n=args.n, k=args.k, L=args.layers)
     if args.retrieval_heads < 0:
         spec = spec.with_(roles="all", name=spec.name + "-dense")
     else:
@@ -84,7 +85,7 @@ def attn_source_hash() -> str:
 def profiled_traffic(workload: str):
     """DRAM bytes per attention launch from the committed ncu summary, if it
     was taken on the current kernel source."""
-    path = os.path.join(ROOT, "profiles", "attn_layer_kernel_traffic.md")
+    path = os.path.join(ROOT, "profiles", "attn_mma_layer_kernel_traffic.md")
     if not os.path.exists(path):
         return None
     want = attn_source_hash()
@@ -336,7 +337,7 @@ def run_lyc(args):
     achieved = distinct / (attn_ms / 1e3) / 1e9
     traffic = profiled_traffic(spec.name)
     roofline = {
-        "bound": "hbm", "kernel": "attn_layer_kernel (pooled dense + sparse attention, one launch per layer)",
+        "bound": "hbm", "kernel": "attn_mma_layer_kernel (pooled dense + sparse attention, one launch per layer)",
         "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
         "frac": round(achieved / peak, 4), "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
         "traffic": traffic,

@@ -1,4 +1,5 @@
-// attn_kernel.cu -- pooled hybrid-head decode attention for one layer.
+// attn_kernel.cu -- pooled hybrid-head decode attention for one layer, fp32
+// inputs (CUDA-core path; bf16 inputs use attn_mma_kernel.cu).
 //
 // Computes, for every segment of the layer's work pool (see lyc_plan.h):
 //   retrieval heads, page "LycheeDecode ..." (paper-graph-ui summary),
@@ -257,21 +258,15 @@ __device__ __forceinline__ void attn_consumers(const AttnParams& p, unsigned cha
     const int nout = sg.nout;
     const int b = sg.b;
     const bool dense = sg.kind == kDense;
+    uint32_t outmask = 0;
+    for (int o = 0; o < nout; ++o) outmask |= 1u << sg.out_row[o];
+    const int64_t key_mean_off = sg.key_mean_off;
 
     // ---- query vectors of this segment -> shared memory (fp32, padded quarters)
     named_bar_sync(1, 256);  // previous piece is done with qs / merge area
     for (int x = tid; x < nq * D; x += 256) {
       const int j = x / D, e = x % D;
-      const int h = sg.head[j];
-      float val;
-      if (h >= 0) {
-        val = load_elem<T>(q, (static_cast<int64_t>(b) * p.Hq + h) * D + e);
-      } else {  // mean of the group's queries (KV-group selection key)
-        float s = 0.f;
-        for (int u = 0; u < p.G; ++u)
-          s += load_elem<T>(q, (static_cast<int64_t>(b) * p.Hq + sg.g * p.G + u) * D + e);
-        val = s / static_cast<float>(p.G);
-      }
+      const float val = load_elem<T>(q, (static_cast<int64_t>(b) * p.Hq + sg.head[j]) * D + e);
       qs[(j * 4 + e / C::QE) * C::QPAD + (e % C::QE)] = val;
     }
     named_bar_sync(1, 256);
@@ -328,12 +323,19 @@ __device__ __forceinline__ void attn_consumers(const AttnParams& p, unsigned cha
       }
 
       // ---- selection keys, online softmax (log2 units), probabilities -> smem
+      if (dense && c == 0 && valid && key_mean_off >= 0) {
+        float sum = 0.f;
+#pragma unroll
+        for (int j = 0; j < NQ; ++j)
+          if (j < nq) sum += acc[j];
+        p.keys[key_mean_off + r0 + row] = sum / static_cast<float>(nq) * p.scale;
+      }
 #pragma unroll
       for (int j = 0; j < NQ; ++j) {
         if (j < nq) {
           if (dense && c == 0 && valid && sg.key_off[j] >= 0)
             p.keys[sg.key_off[j] + r0 + row] = acc[j] * p.scale;
-          if (j < nout) {
+          if ((outmask >> j) & 1u) {
             const float tj = valid ? acc[j] * p.scale_log2 : -INFINITY;
             float mx = fmaxf(tj, __shfl_xor_sync(FULL, tj, 1));
             mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 2));
@@ -362,7 +364,7 @@ __device__ __forceinline__ void attn_consumers(const AttnParams& p, unsigned cha
           load_vslice<T, C::VE>(Vt + (w * 8 + r) * C::ROWB + lane * C::VE * (int)sizeof(T), v);
 #pragma unroll
           for (int j = 0; j < NQ; ++j) {
-            if (j < nout) {
+            if ((outmask >> j) & 1u) {
               const float pj = pb[j * 8 + r];
 #pragma unroll
               for (int e = 0; e < C::VE; ++e) o[j][e] = fmaf(pj, v[e], o[j][e]);
@@ -377,7 +379,7 @@ __device__ __forceinline__ void attn_consumers(const AttnParams& p, unsigned cha
     // ---- merge the 8 warps' states of this piece into one partial record
 #pragma unroll
     for (int j = 0; j < NQ; ++j) {
-      if (j < nout) {
+      if ((outmask >> j) & 1u) {
         float l = l_lane[j];
 #pragma unroll
         for (int s = 16; s >= 1; s >>= 1) l += __shfl_xor_sync(FULL, l, s);
@@ -388,7 +390,8 @@ __device__ __forceinline__ void attn_consumers(const AttnParams& p, unsigned cha
     }
     named_bar_sync(1, 256);
     for (int x = tid; x < nout * D; x += 256) {
-      const int j = x / D, e = x % D;
+      const int o = x / D, e = x % D;
+      const int j = sg.out_row[o];
       float M = -INFINITY;
 #pragma unroll
       for (int ww = 0; ww < 8; ++ww) M = fmaxf(M, mml[ww * NQ + j].x);
@@ -402,7 +405,7 @@ __device__ __forceinline__ void attn_consumers(const AttnParams& p, unsigned cha
           O = fmaf(f, mo[(ww * NQ + j) * D + e], O);
         }
       }
-      const int part = sg.part_base + pc.ordinal * nout + j;
+      const int part = sg.part_base + pc.ordinal * nout + o;
       p.part_o[static_cast<int64_t>(part) * D + e] = O;
       if (e == 0) p.part_ml[part] = make_float2(M, L);
     }
@@ -418,9 +421,9 @@ __device__ __forceinline__ void attn_consumers(const AttnParams& p, unsigned cha
     named_bar_sync(1, 256);
 
     // ---- the last piece of the segment combines every piece (log-sum-exp)
-    for (int j = 0; j < nout; ++j) {
-      if (!lastflag[j]) continue;
-      const int base = sg.part_base + j;
+    for (int o = 0; o < nout; ++o) {
+      if (!lastflag[o]) continue;
+      const int base = sg.part_base + o;
       const int np = sg.npieces;
       for (int e = tid; e < D; e += 256) {
         float M = -INFINITY;
@@ -440,9 +443,9 @@ __device__ __forceinline__ void attn_consumers(const AttnParams& p, unsigned cha
         } else if (e == 0) {
           atomicOr(p.status, kStatusEmptySoftmax);
         }
-        p.out[(static_cast<int64_t>(b) * p.Hq + sg.head[j]) * D + e] = res;
+        p.out[(static_cast<int64_t>(b) * p.Hq + sg.head[sg.out_row[o]]) * D + e] = res;
       }
-      if (tid == 0) p.counters[sg.cnt_base + j] = 0;
+      if (tid == 0) p.counters[sg.cnt_base + o] = 0;
     }
   }
 }
@@ -507,29 +510,25 @@ static cudaError_t attn_by_nq(int nqb, const AttnParams* p, int grid, cudaStream
     case 1: return attn_run<T, D, 1>(p, grid, stream, smem_out, configure_only);
     case 2: return attn_run<T, D, 2>(p, grid, stream, smem_out, configure_only);
     case 4: return attn_run<T, D, 4>(p, grid, stream, smem_out, configure_only);
-    case 5: return attn_run<T, D, 5>(p, grid, stream, smem_out, configure_only);
-    case 9: return attn_run<T, D, 9>(p, grid, stream, smem_out, configure_only);
+    case 8: return attn_run<T, D, 8>(p, grid, stream, smem_out, configure_only);
     default: return cudaErrorInvalidValue;
   }
 }
 
-// Smallest compiled query-vector count >= nq.
+// Smallest compiled query-row count >= nq (both attention kernels).
 int attn_nq_bucket(int nq) {
   if (nq <= 1) return 1;
   if (nq <= 2) return 2;
   if (nq <= 4) return 4;
-  if (nq <= 5) return 5;
-  return 9;
+  return 8;
 }
 
-// dtype: 0 = bf16, 1 = fp32.  configure_only: set the kernel's shared-memory
-// attribute and report its size, launch nothing.
-cudaError_t attn_dispatch(int dtype, int D, int nqb, const AttnParams* p, int grid,
-                          cudaStream_t stream, int* smem_out, bool configure_only) {
-  if (dtype == 0 && D == 128) return attn_by_nq<bf16_t, 128>(nqb, p, grid, stream, smem_out, configure_only);
-  if (dtype == 0 && D == 64) return attn_by_nq<bf16_t, 64>(nqb, p, grid, stream, smem_out, configure_only);
-  if (dtype == 1 && D == 64) return attn_by_nq<float, 64>(nqb, p, grid, stream, smem_out, configure_only);
-  if (dtype == 1 && D == 128) return attn_by_nq<float, 128>(nqb, p, grid, stream, smem_out, configure_only);
+// fp32 inputs (CUDA-core kernel).  configure_only: set the kernel's
+// shared-memory attribute and report its size, launch nothing.
+cudaError_t attn_simt_dispatch(int D, int nqb, const AttnParams* p, int grid, cudaStream_t stream,
+                               int* smem_out, bool configure_only) {
+  if (D == 64) return attn_by_nq<float, 64>(nqb, p, grid, stream, smem_out, configure_only);
+  if (D == 128) return attn_by_nq<float, 128>(nqb, p, grid, stream, smem_out, configure_only);
   return cudaErrorInvalidValue;
 }
 

@@ -1,0 +1,540 @@
+// attn_mma_kernel.cu -- pooled hybrid-head decode attention for one layer,
+// bf16 inputs, tensor cores.
+//
+// Computes, for every segment of the layer's work pool (lyc_plan.h):
+//   retrieval rows, page "LycheeDecode ..." (paper-graph-ui summary),
+//   section 3.4 Eq. (1): o = softmax(q K^T / sqrt(d)) V over all n cached rows,
+//   sparse rows, section 3.4 Eq. (3): the same over the rows of the set they
+//   inherit,
+// plus the selection key of every cached row for the sets refreshed at this
+// layer (Eq. 2 then runs in topk_kernel.cu), and merges the pieces of each
+// segment with log-sum-exp in the last piece to finish (Appendix C,
+// Algorithm 2 steps 5-6, without a second launch).
+//
+// Design (B200 / sm_100a):
+//   * decode attention reads every K/V byte once and does 2-8 flop per byte:
+//     HBM bound.  The CUDA-core version of this loop was issue bound (IPC
+//     0.2, DRAM 12% busy in ncu), so the two contractions run as bf16 mma
+//     with fp32 accumulation: the up-to-8 query rows of a KV group fill the
+//     M=16 side, 8 keys (q.K) or 8 output columns (P.V) the N side;
+//   * one producer warp fills a STAGES-deep ring of 64-row K/V tiles laid out
+//     as 128-byte rows with the 128B XOR swizzle, so ldmatrix reads are
+//     conflict-free: dense (contiguous) tiles by TMA tensor copies from a
+//     5-D tensor map of the whole cache (rows past n come back as zeros),
+//     gathered (sparse) rows by 16-byte cp.async, whose zero-fill form covers
+//     the ragged tail; the gather's indices arrive ahead in a small ring by
+//     bulk copy;
+//   * NW consumer warps take whole tiles in turn, keep an online softmax per
+//     query row in log2 units (p rounded to bf16 before both P.V and the row
+//     sum, so the weights stay normalised), and merge their states at the
+//     end of each piece.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "lyc_device.cuh"
+#include "lyc_plan.h"
+
+namespace lyc {
+
+typedef uint16_t bf16_t;  // bf16 bit pattern
+
+struct AttnMmaParams {
+  CUtensorMap tmk;  // 5-D map of K: (d, row, g, b, l), box 64 x 64, 128B swizzle
+  CUtensorMap tmv;  // same for V
+  AttnParams p;
+};
+
+template <int D, int NW, int STAGES>
+struct MmaCfg {
+  static constexpr int kThreads = (NW + 1) * 32;
+  static constexpr int HALVES = D / 64;                    // 128-byte column blocks per row
+  static constexpr int BLOCKB = kTileRows * 128;           // one swizzled 64 x 128 B block
+  static constexpr int TILEB = HALVES * BLOCKB;            // K (or V) tile bytes
+  static constexpr int NT_D = D / 8;                       // output n-tiles
+  static constexpr int IR = 16;                            // index ring slots
+  static constexpr int LA = 7;                             // index lookahead (tiles)
+  static_assert(IR > LA + STAGES, "index ring too small for the lookahead");
+  // shared memory (bytes from a 1024-aligned base)
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = OFF_K + STAGES * TILEB;
+  static constexpr int OFF_IDX = OFF_V + STAGES * TILEB;
+  static constexpr int OFF_MO = OFF_IDX + IR * kTileRows * 4;
+  static constexpr int OFF_MML = OFF_MO + NW * 8 * D * 4;
+  static constexpr int OFF_BAR = OFF_MML + NW * 8 * 8;
+  static constexpr int OFF_FLAGS = OFF_BAR + (2 * STAGES + IR) * 8;
+  static constexpr int SMEM = OFF_FLAGS + (kMaxQ + 2) * 4 + 1024;  // + alignment slack
+};
+
+// ---------------------------------------------------------------- PTX helpers
+__device__ __forceinline__ void ldsm_x4(uint32_t* r, uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t* r, uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+// D = A(16x16 bf16, row) * B(16x8 bf16, col) + D, fp32 accumulate
+__device__ __forceinline__ void mma_bf16(float* d, uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+      "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+// two floats -> bf16x2 (lo in the low half), round to nearest even
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+__device__ __forceinline__ void tma_load_5d(void* dst, const CUtensorMap* map, int c0, int c1, int c2,
+                                            int c3, int c4, uint64_t* bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7], %8;" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4),
+      "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+// 16-byte global -> shared copy; src_bytes = 0 writes zeros and reads nothing
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+// arrive on `bar` once this thread's earlier cp.async copies have landed
+__device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+// byte offset of 16-byte chunk `ch` (0 .. D/8-1) of tile row `r`
+__device__ __forceinline__ uint32_t swz(int r, int ch) {
+  return static_cast<uint32_t>((ch >> 3) * (kTileRows * 128) + r * 128 + (((ch & 7) ^ (r & 7)) << 4));
+}
+
+}  // namespace lyc
+
+namespace lyc {
+
+// ---------------------------------------------------------------- producer
+template <int D, int NW, int STAGES>
+__device__ __forceinline__ void mma_producer(const AttnMmaParams& P, unsigned char* smem, int pbeg,
+                                             int pend) {
+  using C = MmaCfg<D, NW, STAGES>;
+  const AttnParams& p = P.p;
+  const int lane = threadIdx.x & 31;
+  unsigned char* Ks = smem + C::OFF_K;
+  unsigned char* Vs = smem + C::OFF_V;
+  int32_t* idxring = reinterpret_cast<int32_t*>(smem + C::OFF_IDX);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + STAGES;
+  uint64_t* idxbar = bars + 2 * STAGES;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_FLAGS);
+  const uint64_t pol = l2_policy_evict_first();
+
+  // lookahead cursor: index-list copies of gathered tiles, LA tiles early
+  int la_pc = pbeg, la_r0 = (pbeg < pend) ? p.pieces[pbeg].r0 : 0, la_t = 0;
+  auto la_step = [&]() {
+    if (la_pc >= pend) return;
+    const Piece pc = p.pieces[la_pc];
+    if (p.segs[pc.seg].kind == kSparse && lane == 0) {
+      const int slot = la_t % C::IR;
+      const int nrows = min(kTileRows, pc.r1 - la_r0);
+      const uint32_t bytes = static_cast<uint32_t>(((nrows * 4) + 15) & ~15);
+      fence_proxy_async_smem();
+      mbar_arrive_expect_tx(&idxbar[slot], bytes);
+      bulk_g2s(idxring + slot * kTileRows, p.segs[pc.seg].idx + la_r0, bytes, &idxbar[slot]);
+    }
+    ++la_t;
+    la_r0 += kTileRows;
+    if (la_r0 >= pc.r1) {
+      ++la_pc;
+      if (la_pc < pend) la_r0 = p.pieces[la_pc].r0;
+    }
+  };
+  for (int a = 0; a < C::LA; ++a) la_step();
+
+  uint32_t idx_phase = 0;
+  int t = 0;
+  for (int pcI = pbeg; pcI < pend; ++pcI) {
+    const Piece pc = p.pieces[pcI];
+    const Segment& sg = p.segs[pc.seg];
+    const bool dense = sg.kind == kDense;
+    const int64_t s_token = sg.s_token;
+    const bf16_t* kb = static_cast<const bf16_t*>(sg.k);
+    const bf16_t* vb = static_cast<const bf16_t*>(sg.v);
+    const int sl = sg.l, sb = sg.b, sgg = sg.g;
+    for (int r0 = pc.r0; r0 < pc.r1; r0 += kTileRows, ++t) {
+      la_step();
+      const int nrows = min(kTileRows, pc.r1 - r0);
+      const int stage = t % STAGES;
+      if (t >= STAGES) {
+        if (!mbar_wait(&empty[stage], ((t / STAGES) - 1) & 1, abort_flag, p.status)) return;
+      }
+      unsigned char* kdst = Ks + stage * C::TILEB;
+      unsigned char* vdst = Vs + stage * C::TILEB;
+      if (dense) {
+        // TMA tensor copies; rows past n are filled with zeros by the copy
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&full[stage], 2u * C::TILEB);
+#pragma unroll
+          for (int h = 0; h < C::HALVES; ++h) {
+            tma_load_5d(kdst + h * C::BLOCKB, &P.tmk, h * 64, r0, sgg, sb, sl, &full[stage], pol);
+            tma_load_5d(vdst + h * C::BLOCKB, &P.tmv, h * 64, r0, sgg, sb, sl, &full[stage], pol);
+          }
+        } else {
+          mbar_arrive(&full[stage]);
+        }
+      } else {
+        const int slot = t % C::IR;
+        if (!mbar_wait(&idxbar[slot], (idx_phase >> slot) & 1u, abort_flag, p.status)) return;
+        idx_phase ^= 1u << slot;
+        const int32_t* ring = idxring + slot * kTileRows;
+        {  // bounds of the inherited indices (reported, never followed)
+          const int32_t ia = (lane < nrows) ? ring[lane] : 0;
+          const int32_t ib = (lane + 32 < nrows) ? ring[lane + 32] : 0;
+          if (ia < 0 || ia >= p.n || ib < 0 || ib >= p.n) atomicOr(p.status, kStatusBadIndex);
+        }
+        // lane: 16-byte chunk (lane & 15) of rows 2i + (lane >> 4)
+        constexpr int CH = D / 8;
+        const int ch = lane & 15;
+        const uint32_t kbase = smem_u32(kdst), vbase = smem_u32(vdst);
+#pragma unroll 4
+        for (int i = 0; i < kTileRows / 2; ++i) {
+          const int r = 2 * i + (lane >> 4);
+          const int32_t ix = (r < nrows) ? ring[r] : -1;
+          const bool ok = ix >= 0 && ix < p.n;
+          const int64_t off = ok ? static_cast<int64_t>(ix) * s_token : 0;
+#pragma unroll
+          for (int c = ch; c < CH; c += 16) {
+            cp_async_16(kbase + swz(r, c), kb + off + c * 8, ok ? 16u : 0u);
+            cp_async_16(vbase + swz(r, c), vb + off + c * 8, ok ? 16u : 0u);
+          }
+        }
+        cp_async_arrive(&full[stage]);
+      }
+    }
+  }
+}
+
+}  // namespace lyc
+
+namespace lyc {
+
+// ---------------------------------------------------------------- consumers
+template <int D, int NW, int STAGES>
+__device__ __forceinline__ void mma_consumers(const AttnMmaParams& P, unsigned char* smem, int pbeg,
+                                              int pend) {
+  using C = MmaCfg<D, NW, STAGES>;
+  constexpr unsigned FULL = 0xffffffffu;
+  constexpr int KSTEPS = D / 16;   // q.K k-steps
+  constexpr int NTD = C::NT_D;     // P.V n-tiles (8 columns each)
+  const AttnParams& p = P.p;
+  const int tid = threadIdx.x;     // 0 .. NW*32-1
+  const int w = tid >> 5;
+  const int lane = tid & 31;
+  const int qr = lane >> 2;        // query row held by this lane (rows 8..15 are padding)
+  const int qc = lane & 3;         // column pair within an 8-column n-tile
+  const uint32_t ksm = smem_u32(smem + C::OFF_K);
+  const uint32_t vsm = smem_u32(smem + C::OFF_V);
+  const int32_t* idxring = reinterpret_cast<const int32_t*>(smem + C::OFF_IDX);
+  float* mo = reinterpret_cast<float*>(smem + C::OFF_MO);
+  float2* mml = reinterpret_cast<float2*>(smem + C::OFF_MML);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + STAGES;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_FLAGS);
+  int* lastflag = reinterpret_cast<int*>(smem + C::OFF_FLAGS) + 1;
+  const bf16_t* q = static_cast<const bf16_t*>(p.q);
+  const float sl2 = p.scale_log2;
+
+  int t = 0;  // CTA-wide tile sequence number
+  for (int pcI = pbeg; pcI < pend; ++pcI) {
+    const Piece pc = p.pieces[pcI];
+    const Segment& sg = p.segs[pc.seg];
+    const int nq = sg.nq, nout = sg.nout, b = sg.b;
+    const bool dense = sg.kind == kDense;
+    bool is_out = false;
+    for (int o = 0; o < nout; ++o) is_out |= (sg.out_row[o] == qr);
+    const int64_t key_off = (qr < nq) ? sg.key_off[qr] : -1;
+    const int64_t key_mean_off = sg.key_mean_off;
+    const float inv_nq = 1.f / static_cast<float>(nq);
+
+    // ---- Q rows of this segment as mma A fragments (rows >= nq are zero)
+    uint32_t qa[KSTEPS][2];
+    {
+      const bf16_t* qrow = q + (static_cast<int64_t>(b) * p.Hq + sg.head[qr < nq ? qr : 0]) * D;
+#pragma unroll
+      for (int kk = 0; kk < KSTEPS; ++kk) {
+        const uint32_t lo = (qr < nq) ? *reinterpret_cast<const uint32_t*>(qrow + kk * 16 + 2 * qc) : 0u;
+        const uint32_t hi = (qr < nq) ? *reinterpret_cast<const uint32_t*>(qrow + kk * 16 + 8 + 2 * qc) : 0u;
+        qa[kk][0] = lo;
+        qa[kk][1] = hi;
+      }
+    }
+
+    float m_run = -INFINITY, l_run = 0.f;
+    float o_acc[NTD][4];
+#pragma unroll
+    for (int nt = 0; nt < NTD; ++nt) o_acc[nt][0] = o_acc[nt][1] = o_acc[nt][2] = o_acc[nt][3] = 0.f;
+
+    const int ntile = (pc.r1 - pc.r0 + kTileRows - 1) / kTileRows;
+    for (int u = 0; u < ntile; ++u, ++t) {
+      if ((t % NW) != w) continue;
+      const int r0 = pc.r0 + u * kTileRows;
+      const int nrows = min(kTileRows, pc.r1 - r0);
+      const int stage = t % STAGES;
+      mbar_wait(&full[stage], (t / STAGES) & 1, abort_flag, p.status);
+      // validity of the 64 rows (ragged tail; inherited indices out of range)
+      bool va = lane < nrows, vb = lane + 32 < nrows;
+      if (!dense) {
+        const int32_t* ring = idxring + (t % C::IR) * kTileRows;
+        if (va) { const int32_t x = ring[lane]; va = x >= 0 && x < p.n; }
+        if (vb) { const int32_t x = ring[lane + 32]; vb = x >= 0 && x < p.n; }
+      }
+      const uint64_t vmask = static_cast<uint64_t>(__ballot_sync(FULL, va)) |
+                             (static_cast<uint64_t>(__ballot_sync(FULL, vb)) << 32);
+      const uint32_t kt_base = ksm + stage * C::TILEB;
+      const uint32_t vt_base = vsm + stage * C::TILEB;
+
+      // ---- S = Q K^T: 8 n-tiles of 8 keys
+      float s[8][4];
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+      {
+        const int mi = lane >> 3, r8 = lane & 7;
+#pragma unroll
+        for (int np = 0; np < 4; ++np) {
+          const int key = 16 * np + (mi >> 1) * 8 + r8;
+#pragma unroll
+          for (int kk = 0; kk < KSTEPS; ++kk) {
+            uint32_t bfr[4];
+            ldsm_x4(bfr, kt_base + swz(key, 2 * kk + (mi & 1)));
+            mma_bf16(s[2 * np], qa[kk][0], 0u, qa[kk][1], 0u, bfr[0], bfr[1]);
+            mma_bf16(s[2 * np + 1], qa[kk][0], 0u, qa[kk][1], 0u, bfr[2], bfr[3]);
+          }
+        }
+      }
+
+      // ---- selection keys (dense segments only)
+      if (dense && key_off >= 0) {
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt) {
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int kcol = 8 * nt + 2 * qc + e;
+            if ((vmask >> kcol) & 1ull) p.keys[key_off + r0 + kcol] = s[nt][e] * p.scale;
+          }
+        }
+      }
+      if (dense && key_mean_off >= 0) {
+        // rows >= nq hold zero logits, so the sum over all 8 rows is the sum over nq
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt) {
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            float x = s[nt][e];
+            x += __shfl_xor_sync(FULL, x, 4);
+            x += __shfl_xor_sync(FULL, x, 8);
+            x += __shfl_xor_sync(FULL, x, 16);
+            const int kcol = 8 * nt + 2 * qc + e;
+            if (qr == 0 && ((vmask >> kcol) & 1ull))
+              p.keys[key_mean_off + r0 + kcol] = x * inv_nq * p.scale;
+          }
+        }
+      }
+
+      // ---- online softmax of this lane's query row (log2 units)
+      float mt = -INFINITY;
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int kcol = 8 * nt + 2 * qc + e;
+          const float tv = ((vmask >> kcol) & 1ull) ? s[nt][e] * sl2 : -INFINITY;
+          s[nt][e] = tv;
+          mt = fmaxf(mt, tv);
+        }
+      }
+      mt = fmaxf(mt, __shfl_xor_sync(FULL, mt, 1));
+      mt = fmaxf(mt, __shfl_xor_sync(FULL, mt, 2));
+      const float m_new = fmaxf(m_run, mt);
+      const bool live = is_out && m_new != -INFINITY;
+      const float sc = live ? exp2f(m_run - m_new) : 1.f;
+      m_run = is_out ? m_new : m_run;
+      uint32_t pa[8];
+      float lsum = 0.f;
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) {
+        const float p0 = live ? exp2f(s[nt][0] - m_new) : 0.f;
+        const float p1 = live ? exp2f(s[nt][1] - m_new) : 0.f;
+        pa[nt] = pack_bf16(p0, p1);
+        lsum += __uint_as_float(pa[nt] << 16) + __uint_as_float(pa[nt] & 0xffff0000u);
+      }
+      l_run = l_run * sc + lsum;
+#pragma unroll
+      for (int nt = 0; nt < NTD; ++nt) {
+        o_acc[nt][0] *= sc;
+        o_acc[nt][1] *= sc;
+      }
+
+      // ---- O += P V: 4 k-steps of 16 keys, NTD n-tiles of 8 output columns
+      {
+        const int mi = lane >> 3, r8 = lane & 7;
+#pragma unroll
+        for (int kt = 0; kt < 4; ++kt) {
+          const int key = 16 * kt + (mi & 1) * 8 + r8;
+#pragma unroll
+          for (int dp = 0; dp < NTD / 2; ++dp) {
+            uint32_t bfr[4];
+            ldsm_x4_t(bfr, vt_base + swz(key, 2 * dp + (mi >> 1)));
+            mma_bf16(o_acc[2 * dp], pa[2 * kt], 0u, pa[2 * kt + 1], 0u, bfr[0], bfr[1]);
+            mma_bf16(o_acc[2 * dp + 1], pa[2 * kt], 0u, pa[2 * kt + 1], 0u, bfr[2], bfr[3]);
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[stage]);
+    }
+
+    // ---- merge the NW warps' states of this piece into one partial record per output
+    {
+      float l = l_run;
+      l += __shfl_xor_sync(FULL, l, 1);
+      l += __shfl_xor_sync(FULL, l, 2);
+      if (qc == 0) mml[w * 8 + qr] = make_float2(m_run, l);
+#pragma unroll
+      for (int nt = 0; nt < NTD; ++nt)
+        *reinterpret_cast<float2*>(&mo[(w * 8 + qr) * D + 8 * nt + 2 * qc]) =
+            make_float2(o_acc[nt][0], o_acc[nt][1]);
+    }
+    named_bar_sync(1, NW * 32);
+    for (int x = tid; x < nout * D; x += NW * 32) {
+      const int o = x / D, e = x % D;
+      const int r = sg.out_row[o];
+      float M = -INFINITY;
+#pragma unroll
+      for (int ww = 0; ww < NW; ++ww) M = fmaxf(M, mml[ww * 8 + r].x);
+      float L = 0.f, O = 0.f;
+      if (M != -INFINITY) {
+#pragma unroll
+        for (int ww = 0; ww < NW; ++ww) {
+          const float2 ml = mml[ww * 8 + r];
+          const float f = (ml.x == -INFINITY) ? 0.f : exp2f(ml.x - M);
+          L = fmaf(f, ml.y, L);
+          O = fmaf(f, mo[(ww * 8 + r) * D + e], O);
+        }
+      }
+      const int part = sg.part_base + pc.ordinal * nout + o;
+      p.part_o[static_cast<int64_t>(part) * D + e] = O;
+      if (e == 0) p.part_ml[part] = make_float2(M, L);
+    }
+    __threadfence();
+    named_bar_sync(1, NW * 32);
+    if (tid == 0) {
+      for (int o = 0; o < nout; ++o) {
+        const int old = atomicAdd(&p.counters[sg.cnt_base + o], 1);
+        lastflag[o] = (old == sg.npieces - 1);
+      }
+      __threadfence();
+    }
+    named_bar_sync(1, NW * 32);
+
+    // ---- the last piece of the segment combines every piece (log-sum-exp)
+    for (int o = 0; o < nout; ++o) {
+      if (!lastflag[o]) continue;
+      const int base = sg.part_base + o;
+      const int np = sg.npieces;
+      for (int e = tid; e < D; e += NW * 32) {
+        float M = -INFINITY;
+        for (int u2 = 0; u2 < np; ++u2) M = fmaxf(M, __ldcg(&p.part_ml[base + u2 * nout]).x);
+        float L = 0.f, O = 0.f;
+        if (M != -INFINITY) {
+          for (int u2 = 0; u2 < np; ++u2) {
+            const float2 ml = __ldcg(&p.part_ml[base + u2 * nout]);
+            const float f = (ml.x == -INFINITY) ? 0.f : exp2f(ml.x - M);
+            L = fmaf(f, ml.y, L);
+            O = fmaf(f, __ldcg(&p.part_o[static_cast<int64_t>(base + u2 * nout) * D + e]), O);
+          }
+        }
+        float res = 0.f;
+        if (L > 0.f) {
+          res = O / L;
+        } else if (e == 0) {
+          atomicOr(p.status, kStatusEmptySoftmax);
+        }
+        p.out[(static_cast<int64_t>(b) * p.Hq + sg.head[sg.out_row[o]]) * D + e] = res;
+      }
+      if (tid == 0) p.counters[sg.cnt_base + o] = 0;
+    }
+    named_bar_sync(1, NW * 32);  // merge area and flags free for the next piece
+  }
+}
+
+}  // namespace lyc
+
+namespace lyc {
+
+// ---------------------------------------------------------------- kernel
+template <int D, int NW, int STAGES>
+__global__ void __launch_bounds__(MmaCfg<D, NW, STAGES>::kThreads, 1)
+    attn_mma_layer_kernel(const __grid_constant__ AttnMmaParams P) {
+  using C = MmaCfg<D, NW, STAGES>;
+  extern __shared__ unsigned char smem_raw[];
+  // the 128B-swizzled TMA destination needs 1024-byte alignment
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&bars[s], 32);          // full: the 32 producer lanes (+ TMA bytes)
+      mbar_init(&bars[STAGES + s], 1);  // empty: the one warp that consumed the tile
+    }
+    for (int r = 0; r < C::IR; ++r) mbar_init(&bars[2 * STAGES + r], 1);
+    *reinterpret_cast<int*>(smem + C::OFF_FLAGS) = 0;
+    fence_mbar_init();
+  }
+  if (threadIdx.x == NW * 32) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&P.tmk)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&P.tmv)) : "memory");
+  }
+  __syncthreads();
+  const int pbeg = P.p.cta_begin[blockIdx.x];
+  const int pend = P.p.cta_begin[blockIdx.x + 1];
+  if (threadIdx.x >= NW * 32) {
+    mma_producer<D, NW, STAGES>(P, smem, pbeg, pend);
+  } else {
+    mma_consumers<D, NW, STAGES>(P, smem, pbeg, pend);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+template <int D, int NW, int STAGES>
+static cudaError_t mma_run(const AttnMmaParams* P, int grid, cudaStream_t stream, int* smem_out,
+                           bool configure_only) {
+  using C = MmaCfg<D, NW, STAGES>;
+  auto kern = attn_mma_layer_kernel<D, NW, STAGES>;
+  if (configure_only) {
+    if (smem_out) *smem_out = C::SMEM;
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  }
+  kern<<<grid, C::kThreads, C::SMEM, stream>>>(*P);
+  return cudaGetLastError();
+}
+
+// bf16 inputs.  configure_only: set the shared-memory attribute, report the size.
+cudaError_t attn_mma_dispatch(int D, const AttnMmaParams* P, int grid, cudaStream_t stream,
+                              int* smem_out, bool configure_only) {
+  if (D == 128) return mma_run<128, 4, 6>(P, grid, stream, smem_out, configure_only);
+  if (D == 64) return mma_run<64, 4, 8>(P, grid, stream, smem_out, configure_only);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace lyc

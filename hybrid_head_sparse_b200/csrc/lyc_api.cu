@@ -6,6 +6,7 @@
 // summary), Appendix B / Algorithm 1, attention part: per layer, retrieval
 // heads attend densely and re-select their set, sparse heads attend over the
 // set they inherit and pass it on; layer 0 is all retrieval.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -22,9 +23,16 @@
 #include "lyc_plan.h"
 
 namespace lyc {
+struct AttnMmaParams {
+  CUtensorMap tmk;
+  CUtensorMap tmv;
+  AttnParams p;
+};
 int attn_nq_bucket(int nq);
-cudaError_t attn_dispatch(int dtype, int D, int nqb, const AttnParams* p, int grid,
-                          cudaStream_t stream, int* smem_out, bool configure_only);
+cudaError_t attn_simt_dispatch(int D, int nqb, const AttnParams* p, int grid, cudaStream_t stream,
+                               int* smem_out, bool configure_only);
+cudaError_t attn_mma_dispatch(int D, const AttnMmaParams* P, int grid, cudaStream_t stream,
+                              int* smem_out, bool configure_only);
 size_t topk_smem_for(int cl, int n);
 int topk_pick_cluster(size_t smem);
 cudaError_t topk_configure(int cl, size_t smem);
@@ -64,6 +72,7 @@ struct Plan {
   int32_t* S = nullptr;
   int32_t* trace = nullptr;
   bool timing = false;
+  CUtensorMap tmk{}, tmv{};       // bf16 path: 5-D maps of the whole K and V cache
   cudaGraphExec_t exec = nullptr;
   // timing: event-record nodes of the graph, in launch order (2 per kernel)
   std::vector<cudaGraphNode_t> ev_nodes;
@@ -135,6 +144,52 @@ void free_plan(Plan* p) {
 
 namespace {
 
+// ---------------------------------------------------------------- tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// 5-D map (d, row, KV head, batch, layer) of one cache tensor, 64 x 64 boxes
+// of 128-byte rows with the 128B swizzle; rows at or past n read as zeros.
+lyc_status encode_cache_map(lyc_ctx* ctx, CUtensorMap* map, const void* base, const lyc_kv_cache* kv) {
+  const lyc_config& c = ctx->cfg;
+  EncodeTiledFn fn = encode_tiled_fn();
+  if (!fn) return fail(ctx, LYC_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  const cuuint64_t dims[5] = {static_cast<cuuint64_t>(c.head_dim), static_cast<cuuint64_t>(kv->n),
+                              static_cast<cuuint64_t>(c.num_kv_heads), static_cast<cuuint64_t>(c.batch),
+                              static_cast<cuuint64_t>(c.num_layers)};
+  const int64_t es = 2;
+  int64_t st[4] = {kv->s_token * es, kv->s_head * es, kv->s_batch * es, kv->s_layer * es};
+  // a dimension of extent 1 is only ever read at coordinate 0: give it a
+  // harmless stride if the caller passed 0
+  for (int i = 0; i < 4; ++i)
+    if (dims[i + 1] == 1 && st[i] == 0) st[i] = (i == 0 ? c.head_dim * es : st[i - 1] * static_cast<int64_t>(dims[i]));
+  const cuuint64_t strides[4] = {static_cast<cuuint64_t>(st[0]), static_cast<cuuint64_t>(st[1]),
+                                 static_cast<cuuint64_t>(st[2]), static_cast<cuuint64_t>(st[3])};
+  const cuuint32_t box[5] = {64, static_cast<cuuint32_t>(kTileRows), 1, 1, 1};
+  const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box,
+                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(ctx, LYC_ERR_INVALID_ARG, "cuTensorMapEncodeTiled rejected the cache layout (code " +
+                                              std::to_string(static_cast<int>(r)) + ")");
+  return LYC_OK;
+}
+
 // ---------------------------------------------------------------- planner
 //
 // Builds every layer's work pool for one (role mask, n, k, flags, pointers)
@@ -156,6 +211,11 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const lyc_k
   plan->keff = keff;
   plan->n = n;
   plan->nsets = B * Hs;
+  if (cfg.dtype == LYC_BF16) {
+    lyc_status st = encode_cache_map(ctx, &plan->tmk, kv->k, kv);
+    if (st == LYC_OK) st = encode_cache_map(ctx, &plan->tmv, kv->v, kv);
+    if (st != LYC_OK) return st;
+  }
 
   struct HostLayer {
     std::vector<Segment> segs;
@@ -189,31 +249,34 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const lyc_k
         base.k = kbase + off * es;
         base.v = vbase + off * es;
         base.s_token = kv->s_token;
+        base.l = l;
         base.b = b;
         base.g = g;
+        base.key_mean_off = -1;
         for (int j = 0; j < kMaxQ; ++j) {
           base.key_off[j] = -1;
-          base.head[j] = -1;
+          base.head[j] = 0;
+          base.out_row[j] = 0;
         }
-        // dense segment: the group's retrieval heads (+ mean query in group mode)
+        // dense segment: the group's retrieval heads; in group mode every head
+        // of the group, whose mean logit is the group's selection key
         Segment ds = base;
         ds.kind = kDense;
         ds.rows = n;
-        int j = 0;
-        for (int h = g * G; h < (g + 1) * G; ++h) {
-          if (!is_ret[h]) continue;
-          ds.head[j] = h;
-          ds.key_off[j] = kvmode ? -1 : (static_cast<int64_t>(b) * Hs + h) * ctx->nstride;
-          ++j;
-        }
-        if (j > 0) {
-          ds.nout = j;
-          if (kvmode) {
-            ds.head[j] = -1;
-            ds.key_off[j] = (static_cast<int64_t>(b) * Hs + g) * ctx->nstride;
+        int nret = 0;
+        for (int h = g * G; h < (g + 1) * G; ++h) nret += is_ret[h];
+        if (nret > 0) {
+          int j = 0, o = 0;
+          for (int h = g * G; h < (g + 1) * G; ++h) {
+            if (!kvmode && !is_ret[h]) continue;
+            ds.head[j] = h;
+            if (is_ret[h]) ds.out_row[o++] = j;
+            if (!kvmode) ds.key_off[j] = (static_cast<int64_t>(b) * Hs + h) * ctx->nstride;
             ++j;
           }
           ds.nq = j;
+          ds.nout = o;
+          if (kvmode) ds.key_mean_off = (static_cast<int64_t>(b) * Hs + g) * ctx->nstride;
           maxnq = std::max(maxnq, j);
           H.segs.push_back(ds);
         }
@@ -225,7 +288,10 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const lyc_k
           ss.idx = set_ptr(cur[g], b, g);
           int js = 0;
           for (int h = g * G; h < (g + 1) * G; ++h)
-            if (!is_ret[h]) ss.head[js++] = h;
+            if (!is_ret[h]) {
+              ss.out_row[js] = js;
+              ss.head[js++] = h;
+            }
           if (js > 0) {
             ss.nq = ss.nout = js;
             maxnq = std::max(maxnq, js);
@@ -239,6 +305,7 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const lyc_k
             ss.rows = keff;
             ss.idx = set_ptr(cur[h], b, h);
             ss.head[0] = h;
+            ss.out_row[0] = 0;
             ss.nq = ss.nout = 1;
             H.segs.push_back(ss);
           }
@@ -401,7 +468,15 @@ lyc_status enqueue_step(lyc_ctx* ctx, Plan* plan, cudaStream_t stream, int set, 
     ap.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
     lyc_status st = record_event(ctx, plan, set, ev++, stream, capturing);
     if (st != LYC_OK) return st;
-    LYC_CUDA(attn_dispatch(dtype, D, lp.nqb, &ap, lp.grid, stream, nullptr, false), "attention launch");
+    if (dtype == 0) {
+      AttnMmaParams mp;
+      mp.tmk = plan->tmk;
+      mp.tmv = plan->tmv;
+      mp.p = ap;
+      LYC_CUDA(attn_mma_dispatch(D, &mp, lp.grid, stream, nullptr, false), "attention launch");
+    } else {
+      LYC_CUDA(attn_simt_dispatch(D, lp.nqb, &ap, lp.grid, stream, nullptr, false), "attention launch");
+    }
     if ((st = record_event(ctx, plan, set, ev++, stream, capturing)) != LYC_OK) return st;
     plan->kernel_kind.push_back(0);
     plan->kernel_layer.push_back(l);
@@ -616,12 +691,19 @@ lyc_status lyc_create(const lyc_config* cfg, lyc_ctx** out) {
   cudaError_t e;
   // kernel attributes: shared-memory sizes and the top-k cluster size
   const int dtype = c.dtype == LYC_BF16 ? 0 : 1;
-  for (int nqb : {1, 2, 4, 5, 9}) {
+  if (dtype == 0) {
     int smem = 0;
-    if ((e = attn_dispatch(dtype, D, nqb, nullptr, 0, nullptr, &smem, true)) != cudaSuccess) {
-      lyc_destroy(holder.release());
-      return LYC_ERR_CUDA;
+    e = attn_mma_dispatch(D, nullptr, 0, nullptr, &smem, true);
+  } else {
+    e = cudaSuccess;
+    for (int nqb : {1, 2, 4, 8}) {
+      int smem = 0;
+      if (e == cudaSuccess) e = attn_simt_dispatch(D, nqb, nullptr, 0, nullptr, &smem, true);
     }
+  }
+  if (e != cudaSuccess) {
+    lyc_destroy(holder.release());
+    return LYC_ERR_CUDA;
   }
   const size_t smem16 = topk_smem_for(16, static_cast<int>(c.max_ctx));
   const size_t smem8 = topk_smem_for(8, static_cast<int>(c.max_ctx));

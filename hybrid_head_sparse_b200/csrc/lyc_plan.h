@@ -3,17 +3,20 @@
 // One layer of the step is a pool of segments (page "LycheeDecode ...",
 // paper-graph-ui summary, Appendix C / Algorithm 2, "workload pooling"):
 //   dense segment  : one (batch b, KV group g); rows 0..n-1 of the group's
-//                    K/V; query vectors = the group's retrieval heads (plus,
-//                    in KV-group selection mode, the group's mean query,
-//                    which only produces selection keys);
+//                    K/V; query rows = the group's retrieval heads (per-head
+//                    selection: each row's logits are its selection key), or
+//                    all of the group's heads (KV-group selection: the mean of
+//                    the rows' logits is the group's key, since averaging the
+//                    queries and averaging their logits give the same number;
+//                    only the retrieval rows produce outputs);
 //   sparse segment : one inherited set; rows = the set's list positions
-//                    0..k_eff-1; query vectors = the sparse heads that read
-//                    that set (one head per set in per-head mode, all sparse
-//                    heads of the group in KV-group mode).
+//                    0..k_eff-1; query rows = the sparse heads that read that
+//                    set (one head per set in per-head mode, every sparse head
+//                    of the group in KV-group mode).
 // The pooled rows are cut into equal runs of 64-row tiles, one run per CTA.
 // A run that crosses segment boundaries becomes several pieces.  Each piece
-// writes one partial softmax state (m, l, o[d]) per output query vector; the
-// last piece of a segment to finish merges them (log-sum-exp) into `out`.
+// writes one partial softmax state (m, l, o[d]) per output row; the last piece
+// of a segment to finish merges them (log-sum-exp) into `out`.
 #pragma once
 #include <stdint.h>
 
@@ -21,7 +24,7 @@ namespace lyc {
 
 constexpr int kTileRows = 64;      // rows per pipeline stage (the pages' block size)
 constexpr int kMaxGroup = 8;       // largest Hq / Hkv supported
-constexpr int kMaxQ = kMaxGroup + 1;  // query vectors per segment (+ the mean query)
+constexpr int kMaxQ = kMaxGroup;   // query rows per segment
 
 enum SegKind : int32_t { kDense = 0, kSparse = 1 };
 
@@ -30,14 +33,17 @@ struct Segment {
   const void* v;        // V rows, same layout
   const int32_t* idx;   // sparse: the inherited set (list positions -> token index)
   int64_t s_token;      // element stride between rows
-  int64_t key_off[kMaxQ];  // element offset of this query vector's selection-key row
-                           // in the key buffer, or -1
+  int64_t key_off[kMaxQ];  // per query row: element offset of its selection-key
+                           // row in the key buffer, or -1
+  int64_t key_mean_off;    // offset of the key row that receives the mean of all
+                           // nq rows' logits (KV-group selection), or -1
   int32_t kind;         // SegKind
-  int32_t b, g;
+  int32_t l, b, g;
   int32_t rows;         // dense: n; sparse: k_eff (valid list entries)
-  int32_t nq;           // query vectors in use
-  int32_t nout;         // the first nout query vectors produce outputs
-  int32_t head[kMaxQ];  // query head of each vector; -1 = mean of the group's queries
+  int32_t nq;           // query rows in use
+  int32_t nout;         // rows that produce an output
+  int32_t head[kMaxQ];  // query head of each row
+  int32_t out_row[kMaxQ];  // output o comes from row out_row[o]
   int32_t part_base;    // first partial record of this segment
   int32_t npieces;      // pieces the segment was cut into
   int32_t cnt_base;     // first arrival counter of this segment (nout counters)
@@ -47,7 +53,7 @@ struct Segment {
 struct Piece {
   int32_t seg;      // segment index within the layer
   int32_t r0, r1;   // row range within the segment (token or list positions)
-  int32_t ordinal;  // which piece of its segment (partials at part_base + ordinal*nout + j)
+  int32_t ordinal;  // which piece of its segment (partials at part_base + ordinal*nout + o)
 };
 
 struct AttnParams {

@@ -13,19 +13,23 @@
 //
 // Design (B200 / sm_100a):
 //   * decode attention reads every K/V byte once and does 2-8 flop per byte:
-//     HBM bound.  The CUDA-core version of this loop was issue bound (IPC
-//     0.2, DRAM 12% busy in ncu), so the two contractions run as bf16 mma
-//     with fp32 accumulation: the up-to-8 query rows of a KV group fill the
-//     M=16 side, 8 keys (q.K) or 8 output columns (P.V) the N side;
-//   * one producer warp fills a STAGES-deep ring of 64-row K/V tiles laid out
-//     as 128-byte rows with the 128B XOR swizzle, so ldmatrix reads are
-//     conflict-free: dense (contiguous) tiles by TMA tensor copies from a
-//     5-D tensor map of the whole cache (rows past n come back as zeros),
-//     gathered (sparse) rows by 16-byte cp.async, whose zero-fill form covers
-//     the ragged tail; the gather's indices arrive ahead in a small ring by
-//     bulk copy;
-//   * NW consumer warps take whole tiles in turn, keep an online softmax per
-//     query row in log2 units (p rounded to bf16 before both P.V and the row
+//     HBM bound.  A CUDA-core version of this loop was issue bound (IPC 0.2,
+//     DRAM 12% busy in ncu), so both contractions run as bf16 mma with fp32
+//     accumulation, transposed so that the up-to-8 query heads of a KV group
+//     are the N=8 side and nothing is padded: S^T = K Q^T (M = 16 keys) and
+//     O^T = V^T P^T (M = 16 output columns); P^T's fragments come from S^T's
+//     by an 8x8 movmatrix transpose;
+//   * a STAGES-deep ring of 64-row K/V tiles in shared memory, 128-byte rows
+//     with the 128B XOR swizzle so that ldmatrix reads are conflict-free.
+//     Dense (contiguous) tiles arrive by TMA tensor copies from a 5-D tensor
+//     map of the whole cache (rows past n come back as zeros).  Gathered
+//     (sparse) rows arrive by 16-byte cp.async issued by NP producer warps: a
+//     gather issues from many warps or not at all (about 0.9 TB/s per issuing
+//     warp per SM measured on B200), and the zero-fill form covers the
+//     ragged tail.  The gather's indices come ahead in a small ring by bulk copy;
+//   * NC consumer warps take whole tiles in turn (each stage of the ring
+//     belongs to one of them), keep an online softmax per
+//     query head in log2 units (p rounded to bf16 before both P.V and the row
 //     sum, so the weights stay normalised), and merge their states at the
 //     end of each piece.
 #include <cuda.h>
@@ -46,23 +50,30 @@ struct AttnMmaParams {
   AttnParams p;
 };
 
-template <int D, int NW, int STAGES>
+template <int D, int NC, int NP, int STAGES>
 struct MmaCfg {
-  static constexpr int kThreads = (NW + 1) * 32;
+  static constexpr int kThreads = (NC + NP) * 32;
+  static constexpr int kProducerThreads = NP * 32;
   static constexpr int HALVES = D / 64;                    // 128-byte column blocks per row
   static constexpr int BLOCKB = kTileRows * 128;           // one swizzled 64 x 128 B block
   static constexpr int TILEB = HALVES * BLOCKB;            // K (or V) tile bytes
-  static constexpr int NT_D = D / 8;                       // output n-tiles
   static constexpr int IR = 16;                            // index ring slots
   static constexpr int LA = 7;                             // index lookahead (tiles)
   static_assert(IR > LA + STAGES, "index ring too small for the lookahead");
+  static_assert(kTileRows % (2 * NP) == 0, "rows per producer warp");
+  // Tile t sits in stage t % STAGES and is consumed by warp t % NC.  With
+  // STAGES a multiple of NC every stage belongs to one consumer warp, which
+  // takes that stage's tiles in order; so when it waits for tile t, tile
+  // t - STAGES (the stage's previous phase) is already consumed and the
+  // parity wait cannot match a phase that has not started.
+  static_assert(STAGES % NC == 0, "each stage must belong to one consumer warp");
   // shared memory (bytes from a 1024-aligned base)
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = OFF_K + STAGES * TILEB;
   static constexpr int OFF_IDX = OFF_V + STAGES * TILEB;
   static constexpr int OFF_MO = OFF_IDX + IR * kTileRows * 4;
-  static constexpr int OFF_MML = OFF_MO + NW * 8 * D * 4;
-  static constexpr int OFF_BAR = OFF_MML + NW * 8 * 8;
+  static constexpr int OFF_MML = OFF_MO + NC * 8 * D * 4;
+  static constexpr int OFF_BAR = OFF_MML + NC * 8 * 8;
   static constexpr int OFF_FLAGS = OFF_BAR + (2 * STAGES + IR) * 8;
   static constexpr int SMEM = OFF_FLAGS + (kMaxQ + 2) * 4 + 1024;  // + alignment slack
 };
@@ -93,6 +104,12 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
 }
+// 8x8 bf16 matrix transpose across the warp (fragment layout in and out)
+__device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
+  uint32_t r;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(r) : "r"(x));
+  return r;
+}
 __device__ __forceinline__ void tma_load_5d(void* dst, const CUtensorMap* map, int c0, int c1, int c2,
                                             int c3, int c4, uint64_t* bar, uint64_t policy) {
   asm volatile(
@@ -120,15 +137,22 @@ __device__ __forceinline__ uint32_t swz(int r, int ch) {
 
 }  // namespace lyc
 
+
 namespace lyc {
 
-// ---------------------------------------------------------------- producer
-template <int D, int NW, int STAGES>
-__device__ __forceinline__ void mma_producer(const AttnMmaParams& P, unsigned char* smem, int pbeg,
-                                             int pend) {
-  using C = MmaCfg<D, NW, STAGES>;
+// ---------------------------------------------------------------- producers
+// NP warps walk the CTA's tiles together.  Dense tile: one thread issues the
+// TMA copies, everyone arrives.  Gathered tile: warp pw copies rows
+// [pw*64/NP, (pw+1)*64/NP) with cp.async and every lane arrives when its own
+// copies have landed.
+template <int D, int NC, int NP, int STAGES>
+__device__ __forceinline__ void mma_producers(const AttnMmaParams& P, unsigned char* smem, int pbeg,
+                                              int pend) {
+  using C = MmaCfg<D, NC, NP, STAGES>;
   const AttnParams& p = P.p;
-  const int lane = threadIdx.x & 31;
+  const int ptid = threadIdx.x - NC * 32;  // 0 .. NP*32-1
+  const int pw = ptid >> 5;
+  const int lane = ptid & 31;
   unsigned char* Ks = smem + C::OFF_K;
   unsigned char* Vs = smem + C::OFF_V;
   int32_t* idxring = reinterpret_cast<int32_t*>(smem + C::OFF_IDX);
@@ -138,13 +162,14 @@ __device__ __forceinline__ void mma_producer(const AttnMmaParams& P, unsigned ch
   uint64_t* idxbar = bars + 2 * STAGES;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_FLAGS);
   const uint64_t pol = l2_policy_evict_first();
+  const bool leader = ptid == 0;
 
-  // lookahead cursor: index-list copies of gathered tiles, LA tiles early
+  // lookahead cursor (leader only): index-list copies of gathered tiles, LA tiles early
   int la_pc = pbeg, la_r0 = (pbeg < pend) ? p.pieces[pbeg].r0 : 0, la_t = 0;
   auto la_step = [&]() {
     if (la_pc >= pend) return;
     const Piece pc = p.pieces[la_pc];
-    if (p.segs[pc.seg].kind == kSparse && lane == 0) {
+    if (p.segs[pc.seg].kind == kSparse) {
       const int slot = la_t % C::IR;
       const int nrows = min(kTileRows, pc.r1 - la_r0);
       const uint32_t bytes = static_cast<uint32_t>(((nrows * 4) + 15) & ~15);
@@ -159,8 +184,11 @@ __device__ __forceinline__ void mma_producer(const AttnMmaParams& P, unsigned ch
       if (la_pc < pend) la_r0 = p.pieces[la_pc].r0;
     }
   };
-  for (int a = 0; a < C::LA; ++a) la_step();
+  if (leader)
+    for (int a = 0; a < C::LA; ++a) la_step();
 
+  constexpr int CH = D / 8;                  // 16-byte chunks per row
+  constexpr int ROWS_W = kTileRows / NP;     // rows per producer warp
   uint32_t idx_phase = 0;
   int t = 0;
   for (int pcI = pbeg; pcI < pend; ++pcI) {
@@ -172,7 +200,7 @@ __device__ __forceinline__ void mma_producer(const AttnMmaParams& P, unsigned ch
     const bf16_t* vb = static_cast<const bf16_t*>(sg.v);
     const int sl = sg.l, sb = sg.b, sgg = sg.g;
     for (int r0 = pc.r0; r0 < pc.r1; r0 += kTileRows, ++t) {
-      la_step();
+      if (leader) la_step();
       const int nrows = min(kTileRows, pc.r1 - r0);
       const int stage = t % STAGES;
       if (t >= STAGES) {
@@ -182,7 +210,7 @@ __device__ __forceinline__ void mma_producer(const AttnMmaParams& P, unsigned ch
       unsigned char* vdst = Vs + stage * C::TILEB;
       if (dense) {
         // TMA tensor copies; rows past n are filled with zeros by the copy
-        if (lane == 0) {
+        if (leader) {
           mbar_arrive_expect_tx(&full[stage], 2u * C::TILEB);
 #pragma unroll
           for (int h = 0; h < C::HALVES; ++h) {
@@ -197,26 +225,23 @@ __device__ __forceinline__ void mma_producer(const AttnMmaParams& P, unsigned ch
         if (!mbar_wait(&idxbar[slot], (idx_phase >> slot) & 1u, abort_flag, p.status)) return;
         idx_phase ^= 1u << slot;
         const int32_t* ring = idxring + slot * kTileRows;
-        {  // bounds of the inherited indices (reported, never followed)
+        if (pw == 0) {  // bounds of the inherited indices (reported, never followed)
           const int32_t ia = (lane < nrows) ? ring[lane] : 0;
           const int32_t ib = (lane + 32 < nrows) ? ring[lane + 32] : 0;
           if (ia < 0 || ia >= p.n || ib < 0 || ib >= p.n) atomicOr(p.status, kStatusBadIndex);
         }
-        // lane: 16-byte chunk (lane & 15) of rows 2i + (lane >> 4)
-        constexpr int CH = D / 8;
-        const int ch = lane & 15;
         const uint32_t kbase = smem_u32(kdst), vbase = smem_u32(vdst);
-#pragma unroll 4
-        for (int i = 0; i < kTileRows / 2; ++i) {
-          const int r = 2 * i + (lane >> 4);
+        // lane: chunk (lane % CH) of rows pw*ROWS_W + (lane / CH) + (32/CH)*i
+        constexpr int RPI = 32 / CH;         // rows per warp instruction
+#pragma unroll
+        for (int i = 0; i < ROWS_W / RPI; ++i) {
+          const int r = pw * ROWS_W + i * RPI + lane / CH;
+          const int c = lane % CH;
           const int32_t ix = (r < nrows) ? ring[r] : -1;
           const bool ok = ix >= 0 && ix < p.n;
           const int64_t off = ok ? static_cast<int64_t>(ix) * s_token : 0;
-#pragma unroll
-          for (int c = ch; c < CH; c += 16) {
-            cp_async_16(kbase + swz(r, c), kb + off + c * 8, ok ? 16u : 0u);
-            cp_async_16(vbase + swz(r, c), vb + off + c * 8, ok ? 16u : 0u);
-          }
+          cp_async_16(kbase + swz(r, c), kb + off + c * 8, ok ? 16u : 0u);
+          cp_async_16(vbase + swz(r, c), vb + off + c * 8, ok ? 16u : 0u);
         }
         cp_async_arrive(&full[stage]);
       }
@@ -229,19 +254,27 @@ __device__ __forceinline__ void mma_producer(const AttnMmaParams& P, unsigned ch
 namespace lyc {
 
 // ---------------------------------------------------------------- consumers
-template <int D, int NW, int STAGES>
+// Fragment bookkeeping (m16n8k16, g = lane/4, c = lane%4):
+//   S^T tile mt (16 keys):  st[mt][0..1] = keys 16mt+g,   queries 2c, 2c+1
+//                           st[mt][2..3] = keys 16mt+g+8, queries 2c, 2c+1
+//   O^T tile md (16 cols):  oa[md][0..1] = cols 16md+g,   queries 2c, 2c+1
+//                           oa[md][2..3] = cols 16md+g+8, queries 2c, 2c+1
+// so every lane owns queries q0 = 2c and q1 = 2c+1 in both, and the softmax
+// rescale needs no data movement.
+template <int D, int NC, int NP, int STAGES>
 __device__ __forceinline__ void mma_consumers(const AttnMmaParams& P, unsigned char* smem, int pbeg,
                                               int pend) {
-  using C = MmaCfg<D, NW, STAGES>;
+  using C = MmaCfg<D, NC, NP, STAGES>;
   constexpr unsigned FULL = 0xffffffffu;
-  constexpr int KSTEPS = D / 16;   // q.K k-steps
-  constexpr int NTD = C::NT_D;     // P.V n-tiles (8 columns each)
+  constexpr int KSTEPS = D / 16;   // q.K k-steps over d
+  constexpr int MD = D / 16;       // O^T m-tiles
   const AttnParams& p = P.p;
-  const int tid = threadIdx.x;     // 0 .. NW*32-1
+  const int tid = threadIdx.x;     // 0 .. NC*32-1
   const int w = tid >> 5;
   const int lane = tid & 31;
-  const int qr = lane >> 2;        // query row held by this lane (rows 8..15 are padding)
-  const int qc = lane & 3;         // column pair within an 8-column n-tile
+  const int g = lane >> 2;
+  const int c = lane & 3;
+  const int q0 = 2 * c, q1 = 2 * c + 1;
   const uint32_t ksm = smem_u32(smem + C::OFF_K);
   const uint32_t vsm = smem_u32(smem + C::OFF_V);
   const int32_t* idxring = reinterpret_cast<const int32_t*>(smem + C::OFF_IDX);
@@ -254,6 +287,7 @@ __device__ __forceinline__ void mma_consumers(const AttnMmaParams& P, unsigned c
   int* lastflag = reinterpret_cast<int*>(smem + C::OFF_FLAGS) + 1;
   const bf16_t* q = static_cast<const bf16_t*>(p.q);
   const float sl2 = p.scale_log2;
+  const int mi = lane >> 3, r8 = lane & 7;  // ldmatrix: matrix and row this lane addresses
 
   int t = 0;  // CTA-wide tile sequence number
   for (int pcI = pbeg; pcI < pend; ++pcI) {
@@ -261,33 +295,35 @@ __device__ __forceinline__ void mma_consumers(const AttnMmaParams& P, unsigned c
     const Segment& sg = p.segs[pc.seg];
     const int nq = sg.nq, nout = sg.nout, b = sg.b;
     const bool dense = sg.kind == kDense;
-    bool is_out = false;
-    for (int o = 0; o < nout; ++o) is_out |= (sg.out_row[o] == qr);
-    const int64_t key_off = (qr < nq) ? sg.key_off[qr] : -1;
+    bool out0 = false, out1 = false;
+    for (int o = 0; o < nout; ++o) {
+      out0 |= sg.out_row[o] == q0;
+      out1 |= sg.out_row[o] == q1;
+    }
+    const int64_t koff0 = (q0 < nq) ? sg.key_off[q0] : -1;
+    const int64_t koff1 = (q1 < nq) ? sg.key_off[q1] : -1;
     const int64_t key_mean_off = sg.key_mean_off;
-    const float inv_nq = 1.f / static_cast<float>(nq);
+    const float mean_scale = p.scale / static_cast<float>(nq);
 
-    // ---- Q rows of this segment as mma A fragments (rows >= nq are zero)
-    uint32_t qa[KSTEPS][2];
+    // ---- Q^T as the B operand: this lane holds query g, d = 16kk + 2c (+8)
+    uint32_t qb[KSTEPS][2];
     {
-      const bf16_t* qrow = q + (static_cast<int64_t>(b) * p.Hq + sg.head[qr < nq ? qr : 0]) * D;
+      const bf16_t* qrow = q + (static_cast<int64_t>(b) * p.Hq + sg.head[g < nq ? g : 0]) * D;
 #pragma unroll
       for (int kk = 0; kk < KSTEPS; ++kk) {
-        const uint32_t lo = (qr < nq) ? *reinterpret_cast<const uint32_t*>(qrow + kk * 16 + 2 * qc) : 0u;
-        const uint32_t hi = (qr < nq) ? *reinterpret_cast<const uint32_t*>(qrow + kk * 16 + 8 + 2 * qc) : 0u;
-        qa[kk][0] = lo;
-        qa[kk][1] = hi;
+        qb[kk][0] = (g < nq) ? *reinterpret_cast<const uint32_t*>(qrow + kk * 16 + 2 * c) : 0u;
+        qb[kk][1] = (g < nq) ? *reinterpret_cast<const uint32_t*>(qrow + kk * 16 + 8 + 2 * c) : 0u;
       }
     }
 
-    float m_run = -INFINITY, l_run = 0.f;
-    float o_acc[NTD][4];
+    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+    float oa[MD][4];
 #pragma unroll
-    for (int nt = 0; nt < NTD; ++nt) o_acc[nt][0] = o_acc[nt][1] = o_acc[nt][2] = o_acc[nt][3] = 0.f;
+    for (int md = 0; md < MD; ++md) oa[md][0] = oa[md][1] = oa[md][2] = oa[md][3] = 0.f;
 
     const int ntile = (pc.r1 - pc.r0 + kTileRows - 1) / kTileRows;
     for (int u = 0; u < ntile; ++u, ++t) {
-      if ((t % NW) != w) continue;
+      if ((t % NC) != w) continue;
       const int r0 = pc.r0 + u * kTileRows;
       const int nrows = min(kTileRows, pc.r1 - r0);
       const int stage = t % STAGES;
@@ -304,128 +340,141 @@ __device__ __forceinline__ void mma_consumers(const AttnMmaParams& P, unsigned c
       const uint32_t kt_base = ksm + stage * C::TILEB;
       const uint32_t vt_base = vsm + stage * C::TILEB;
 
-      // ---- S = Q K^T: 8 n-tiles of 8 keys
-      float s[8][4];
+      // ---- S^T = K Q^T: 4 m-tiles of 16 keys x 8 queries
+      float st[4][4];
 #pragma unroll
-      for (int nt = 0; nt < 8; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
-      {
-        const int mi = lane >> 3, r8 = lane & 7;
+      for (int mt = 0; mt < 4; ++mt) st[mt][0] = st[mt][1] = st[mt][2] = st[mt][3] = 0.f;
 #pragma unroll
-        for (int np = 0; np < 4; ++np) {
-          const int key = 16 * np + (mi >> 1) * 8 + r8;
+      for (int kk = 0; kk < KSTEPS; ++kk) {
 #pragma unroll
-          for (int kk = 0; kk < KSTEPS; ++kk) {
-            uint32_t bfr[4];
-            ldsm_x4(bfr, kt_base + swz(key, 2 * kk + (mi & 1)));
-            mma_bf16(s[2 * np], qa[kk][0], 0u, qa[kk][1], 0u, bfr[0], bfr[1]);
-            mma_bf16(s[2 * np + 1], qa[kk][0], 0u, qa[kk][1], 0u, bfr[2], bfr[3]);
-          }
+        for (int mt = 0; mt < 4; ++mt) {
+          uint32_t a[4];
+          ldsm_x4(a, kt_base + swz(16 * mt + (mi & 1) * 8 + r8, 2 * kk + (mi >> 1)));
+          mma_bf16(st[mt], a[0], a[1], a[2], a[3], qb[kk][0], qb[kk][1]);
         }
       }
 
       // ---- selection keys (dense segments only)
-      if (dense && key_off >= 0) {
+      if (dense && (koff0 >= 0 || koff1 >= 0)) {
 #pragma unroll
-        for (int nt = 0; nt < 8; ++nt) {
+        for (int mt = 0; mt < 4; ++mt) {
 #pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int kcol = 8 * nt + 2 * qc + e;
-            if ((vmask >> kcol) & 1ull) p.keys[key_off + r0 + kcol] = s[nt][e] * p.scale;
+          for (int h = 0; h < 2; ++h) {
+            const int key = 16 * mt + g + 8 * h;
+            if ((vmask >> key) & 1ull) {
+              if (koff0 >= 0) p.keys[koff0 + r0 + key] = st[mt][2 * h] * p.scale;
+              if (koff1 >= 0) p.keys[koff1 + r0 + key] = st[mt][2 * h + 1] * p.scale;
+            }
           }
         }
       }
       if (dense && key_mean_off >= 0) {
-        // rows >= nq hold zero logits, so the sum over all 8 rows is the sum over nq
+        // queries >= nq hold zero logits, so the sum over all 8 is the sum over nq
 #pragma unroll
-        for (int nt = 0; nt < 8; ++nt) {
+        for (int mt = 0; mt < 4; ++mt) {
 #pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            float x = s[nt][e];
-            x += __shfl_xor_sync(FULL, x, 4);
-            x += __shfl_xor_sync(FULL, x, 8);
-            x += __shfl_xor_sync(FULL, x, 16);
-            const int kcol = 8 * nt + 2 * qc + e;
-            if (qr == 0 && ((vmask >> kcol) & 1ull))
-              p.keys[key_mean_off + r0 + kcol] = x * inv_nq * p.scale;
+          for (int h = 0; h < 2; ++h) {
+            float x = st[mt][2 * h] + st[mt][2 * h + 1];
+            x += __shfl_xor_sync(FULL, x, 1);
+            x += __shfl_xor_sync(FULL, x, 2);
+            const int key = 16 * mt + g + 8 * h;
+            if (c == 0 && ((vmask >> key) & 1ull)) p.keys[key_mean_off + r0 + key] = x * mean_scale;
           }
         }
       }
 
-      // ---- online softmax of this lane's query row (log2 units)
-      float mt = -INFINITY;
+      // ---- online softmax for queries q0, q1 (log2 units)
+      float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
-      for (int nt = 0; nt < 8; ++nt) {
+      for (int mt = 0; mt < 4; ++mt) {
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int kcol = 8 * nt + 2 * qc + e;
-          const float tv = ((vmask >> kcol) & 1ull) ? s[nt][e] * sl2 : -INFINITY;
-          s[nt][e] = tv;
-          mt = fmaxf(mt, tv);
+        for (int h = 0; h < 2; ++h) {
+          const bool ok = (vmask >> (16 * mt + g + 8 * h)) & 1ull;
+          st[mt][2 * h] = ok ? st[mt][2 * h] * sl2 : -INFINITY;
+          st[mt][2 * h + 1] = ok ? st[mt][2 * h + 1] * sl2 : -INFINITY;
+          mx0 = fmaxf(mx0, st[mt][2 * h]);
+          mx1 = fmaxf(mx1, st[mt][2 * h + 1]);
         }
       }
-      mt = fmaxf(mt, __shfl_xor_sync(FULL, mt, 1));
-      mt = fmaxf(mt, __shfl_xor_sync(FULL, mt, 2));
-      const float m_new = fmaxf(m_run, mt);
-      const bool live = is_out && m_new != -INFINITY;
-      const float sc = live ? exp2f(m_run - m_new) : 1.f;
-      m_run = is_out ? m_new : m_run;
-      uint32_t pa[8];
-      float lsum = 0.f;
 #pragma unroll
-      for (int nt = 0; nt < 8; ++nt) {
-        const float p0 = live ? exp2f(s[nt][0] - m_new) : 0.f;
-        const float p1 = live ? exp2f(s[nt][1] - m_new) : 0.f;
-        pa[nt] = pack_bf16(p0, p1);
-        lsum += __uint_as_float(pa[nt] << 16) + __uint_as_float(pa[nt] & 0xffff0000u);
+      for (int s = 4; s <= 16; s <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(FULL, mx0, s));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(FULL, mx1, s));
       }
-      l_run = l_run * sc + lsum;
+      const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+      const bool live0 = out0 && mn0 != -INFINITY, live1 = out1 && mn1 != -INFINITY;
+      const float sc0 = live0 ? exp2f(m0 - mn0) : 1.f;
+      const float sc1 = live1 ? exp2f(m1 - mn1) : 1.f;
+      if (out0) m0 = mn0;
+      if (out1) m1 = mn1;
+      uint32_t pb[4][2];  // P^T fragments, per 16-key step: keys +0..7, +8..15
+      float ls0 = 0.f, ls1 = 0.f;
 #pragma unroll
-      for (int nt = 0; nt < NTD; ++nt) {
-        o_acc[nt][0] *= sc;
-        o_acc[nt][1] *= sc;
+      for (int mt = 0; mt < 4; ++mt) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const float pv0 = live0 ? exp2f(st[mt][2 * h] - mn0) : 0.f;
+          const float pv1 = live1 ? exp2f(st[mt][2 * h + 1] - mn1) : 0.f;
+          const uint32_t pk = pack_bf16(pv0, pv1);  // (key, q0) low, (key, q1) high
+          ls0 += __uint_as_float(pk << 16);
+          ls1 += __uint_as_float(pk & 0xffff0000u);
+          pb[mt][h] = movmatrix_t(pk);  // -> (query g, keys 2c, 2c+1)
+        }
+      }
+      l0 = l0 * sc0 + ls0;
+      l1 = l1 * sc1 + ls1;
+#pragma unroll
+      for (int md = 0; md < MD; ++md) {
+        oa[md][0] *= sc0;
+        oa[md][1] *= sc1;
+        oa[md][2] *= sc0;
+        oa[md][3] *= sc1;
       }
 
-      // ---- O += P V: 4 k-steps of 16 keys, NTD n-tiles of 8 output columns
-      {
-        const int mi = lane >> 3, r8 = lane & 7;
+      // ---- O^T += V^T P^T: 4 k-steps of 16 keys, MD m-tiles of 16 columns
 #pragma unroll
-        for (int kt = 0; kt < 4; ++kt) {
-          const int key = 16 * kt + (mi & 1) * 8 + r8;
+      for (int kt = 0; kt < 4; ++kt) {
 #pragma unroll
-          for (int dp = 0; dp < NTD / 2; ++dp) {
-            uint32_t bfr[4];
-            ldsm_x4_t(bfr, vt_base + swz(key, 2 * dp + (mi >> 1)));
-            mma_bf16(o_acc[2 * dp], pa[2 * kt], 0u, pa[2 * kt + 1], 0u, bfr[0], bfr[1]);
-            mma_bf16(o_acc[2 * dp + 1], pa[2 * kt], 0u, pa[2 * kt + 1], 0u, bfr[2], bfr[3]);
-          }
+        for (int md = 0; md < MD; ++md) {
+          uint32_t a[4];
+          ldsm_x4_t(a, vt_base + swz(16 * kt + (mi >> 1) * 8 + r8, 2 * md + (mi & 1)));
+          mma_bf16(oa[md], a[0], a[1], a[2], a[3], pb[kt][0], pb[kt][1]);
         }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[stage]);
     }
 
-    // ---- merge the NW warps' states of this piece into one partial record per output
+    // ---- merge the NC warps' states of this piece into one partial record per output
     {
-      float l = l_run;
-      l += __shfl_xor_sync(FULL, l, 1);
-      l += __shfl_xor_sync(FULL, l, 2);
-      if (qc == 0) mml[w * 8 + qr] = make_float2(m_run, l);
 #pragma unroll
-      for (int nt = 0; nt < NTD; ++nt)
-        *reinterpret_cast<float2*>(&mo[(w * 8 + qr) * D + 8 * nt + 2 * qc]) =
-            make_float2(o_acc[nt][0], o_acc[nt][1]);
+      for (int s = 4; s <= 16; s <<= 1) {
+        l0 += __shfl_xor_sync(FULL, l0, s);
+        l1 += __shfl_xor_sync(FULL, l1, s);
+      }
+      if (g == 0) {
+        mml[w * 8 + q0] = make_float2(m0, l0);
+        mml[w * 8 + q1] = make_float2(m1, l1);
+      }
+#pragma unroll
+      for (int md = 0; md < MD; ++md) {
+        mo[(w * 8 + q0) * D + 16 * md + g] = oa[md][0];
+        mo[(w * 8 + q1) * D + 16 * md + g] = oa[md][1];
+        mo[(w * 8 + q0) * D + 16 * md + g + 8] = oa[md][2];
+        mo[(w * 8 + q1) * D + 16 * md + g + 8] = oa[md][3];
+      }
     }
-    named_bar_sync(1, NW * 32);
-    for (int x = tid; x < nout * D; x += NW * 32) {
+    named_bar_sync(1, NC * 32);
+    for (int x = tid; x < nout * D; x += NC * 32) {
       const int o = x / D, e = x % D;
       const int r = sg.out_row[o];
       float M = -INFINITY;
 #pragma unroll
-      for (int ww = 0; ww < NW; ++ww) M = fmaxf(M, mml[ww * 8 + r].x);
+      for (int ww = 0; ww < NC; ++ww) M = fmaxf(M, mml[ww * 8 + r].x);
       float L = 0.f, O = 0.f;
       if (M != -INFINITY) {
 #pragma unroll
-        for (int ww = 0; ww < NW; ++ww) {
+        for (int ww = 0; ww < NC; ++ww) {
           const float2 ml = mml[ww * 8 + r];
           const float f = (ml.x == -INFINITY) ? 0.f : exp2f(ml.x - M);
           L = fmaf(f, ml.y, L);
@@ -437,7 +486,7 @@ __device__ __forceinline__ void mma_consumers(const AttnMmaParams& P, unsigned c
       if (e == 0) p.part_ml[part] = make_float2(M, L);
     }
     __threadfence();
-    named_bar_sync(1, NW * 32);
+    named_bar_sync(1, NC * 32);
     if (tid == 0) {
       for (int o = 0; o < nout; ++o) {
         const int old = atomicAdd(&p.counters[sg.cnt_base + o], 1);
@@ -445,14 +494,14 @@ __device__ __forceinline__ void mma_consumers(const AttnMmaParams& P, unsigned c
       }
       __threadfence();
     }
-    named_bar_sync(1, NW * 32);
+    named_bar_sync(1, NC * 32);
 
     // ---- the last piece of the segment combines every piece (log-sum-exp)
     for (int o = 0; o < nout; ++o) {
       if (!lastflag[o]) continue;
       const int base = sg.part_base + o;
       const int np = sg.npieces;
-      for (int e = tid; e < D; e += NW * 32) {
+      for (int e = tid; e < D; e += NC * 32) {
         float M = -INFINITY;
         for (int u2 = 0; u2 < np; ++u2) M = fmaxf(M, __ldcg(&p.part_ml[base + u2 * nout]).x);
         float L = 0.f, O = 0.f;
@@ -474,19 +523,15 @@ __device__ __forceinline__ void mma_consumers(const AttnMmaParams& P, unsigned c
       }
       if (tid == 0) p.counters[sg.cnt_base + o] = 0;
     }
-    named_bar_sync(1, NW * 32);  // merge area and flags free for the next piece
+    named_bar_sync(1, NC * 32);  // merge area and flags free for the next piece
   }
 }
 
-}  // namespace lyc
-
-namespace lyc {
-
 // ---------------------------------------------------------------- kernel
-template <int D, int NW, int STAGES>
-__global__ void __launch_bounds__(MmaCfg<D, NW, STAGES>::kThreads, 1)
+template <int D, int NC, int NP, int STAGES>
+__global__ void __launch_bounds__(MmaCfg<D, NC, NP, STAGES>::kThreads, 1)
     attn_mma_layer_kernel(const __grid_constant__ AttnMmaParams P) {
-  using C = MmaCfg<D, NW, STAGES>;
+  using C = MmaCfg<D, NC, NP, STAGES>;
   extern __shared__ unsigned char smem_raw[];
   // the 128B-swizzled TMA destination needs 1024-byte alignment
   unsigned char* smem = reinterpret_cast<unsigned char*>(
@@ -494,33 +539,33 @@ __global__ void __launch_bounds__(MmaCfg<D, NW, STAGES>::kThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&bars[s], 32);          // full: the 32 producer lanes (+ TMA bytes)
-      mbar_init(&bars[STAGES + s], 1);  // empty: the one warp that consumed the tile
+      mbar_init(&bars[s], C::kProducerThreads);  // full: every producer thread (+ TMA bytes)
+      mbar_init(&bars[STAGES + s], 1);           // empty: the one warp that consumed the tile
     }
     for (int r = 0; r < C::IR; ++r) mbar_init(&bars[2 * STAGES + r], 1);
     *reinterpret_cast<int*>(smem + C::OFF_FLAGS) = 0;
     fence_mbar_init();
   }
-  if (threadIdx.x == NW * 32) {
+  if (threadIdx.x == NC * 32) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&P.tmk)) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&P.tmv)) : "memory");
   }
   __syncthreads();
   const int pbeg = P.p.cta_begin[blockIdx.x];
   const int pend = P.p.cta_begin[blockIdx.x + 1];
-  if (threadIdx.x >= NW * 32) {
-    mma_producer<D, NW, STAGES>(P, smem, pbeg, pend);
+  if (threadIdx.x >= NC * 32) {
+    mma_producers<D, NC, NP, STAGES>(P, smem, pbeg, pend);
   } else {
-    mma_consumers<D, NW, STAGES>(P, smem, pbeg, pend);
+    mma_consumers<D, NC, NP, STAGES>(P, smem, pbeg, pend);
   }
 }
 
 // ---------------------------------------------------------------- host side
-template <int D, int NW, int STAGES>
+template <int D, int NC, int NP, int STAGES>
 static cudaError_t mma_run(const AttnMmaParams* P, int grid, cudaStream_t stream, int* smem_out,
                            bool configure_only) {
-  using C = MmaCfg<D, NW, STAGES>;
-  auto kern = attn_mma_layer_kernel<D, NW, STAGES>;
+  using C = MmaCfg<D, NC, NP, STAGES>;
+  auto kern = attn_mma_layer_kernel<D, NC, NP, STAGES>;
   if (configure_only) {
     if (smem_out) *smem_out = C::SMEM;
     return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
@@ -532,8 +577,8 @@ static cudaError_t mma_run(const AttnMmaParams* P, int grid, cudaStream_t stream
 // bf16 inputs.  configure_only: set the shared-memory attribute, report the size.
 cudaError_t attn_mma_dispatch(int D, const AttnMmaParams* P, int grid, cudaStream_t stream,
                               int* smem_out, bool configure_only) {
-  if (D == 128) return mma_run<128, 4, 6>(P, grid, stream, smem_out, configure_only);
-  if (D == 64) return mma_run<64, 4, 8>(P, grid, stream, smem_out, configure_only);
+  if (D == 128) return mma_run<128, 3, 8, 6>(P, grid, stream, smem_out, configure_only);
+  if (D == 64) return mma_run<64, 4, 8, 8>(P, grid, stream, smem_out, configure_only);
   return cudaErrorInvalidValue;
 }
 

@@ -235,3 +235,32 @@ def test_strided_rows(lyc):
     strided["v"] = Vp[..., :64]
     _, out, S, tr = run_step(lyc, spec, data=strided)
     P.check_layers(data, out, tr, spec.k, spec.n, "fp32", range(spec.L))
+
+
+# ---------------------------------------------------------------- full-size workloads
+# The whole step runs at the workload's size; the oracle checks sampled layers
+# with teacher forcing (each checked layer inherits the GPU's own sets).
+
+
+def _full_size(lyc, spec, layers, mode="per_qhead"):
+    om = O.SELECT_PER_QHEAD if mode == "per_qhead" else O.SELECT_KVGROUP_MEAN
+    data, out, S, tr = run_step(lyc, spec, select_mode=mode)
+    assert np.isfinite(out).all()
+    P.check_layers(data, out, tr, spec.k, spec.n, spec.dtype, layers, select_mode=om)
+    assert np.array_equal(S, tr[-1])
+    del data
+    torch.cuda.empty_cache()
+
+
+def test_llama3_8b_32k_full_step(lyc):
+    _full_size(lyc, W.LLAMA3_8B_32K, [0, 1, 2, 17, 31])
+
+
+@pytest.mark.parametrize("mode", ["per_qhead", "kvgroup_mean"])
+def test_llama3_8b_128k_first_layers(lyc, mode):
+    # the 128K stack's first 6 layers (same shapes per layer as the full 32)
+    _full_size(lyc, W.LLAMA3_8B_128K.with_(L=6), [0, 1, 5], mode)
+
+
+def test_qwen3_8b_64k_batch4(lyc):
+    _full_size(lyc, W.QWEN3_8B_64K_B4.with_(L=4), [0, 1, 3])

@@ -45,7 +45,7 @@ using namespace lyc;
 
 namespace {
 
-constexpr int kMaxCtxLimit = 786432;  // 16-CTA top-k keeps every key in shared memory
+constexpr int kMaxCtxLimit = 655360;  // 16-CTA top-k keeps every key in shared memory
 constexpr int kPlanCacheSize = 16;
 
 int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }

@@ -19,10 +19,13 @@
 // of a segment to finish merges them (log-sum-exp) into `out`.
 #pragma once
 #include <stdint.h>
+#include <string.h>
 
 namespace lyc {
 
 constexpr int kTileRows = 64;      // rows per pipeline stage (the pages' block size)
+constexpr int kKeyBins = 2048;     // top 11 bits of an order-preserving key encoding
+constexpr int kKeyDigitShift = 21;
 constexpr int kMaxGroup = 8;       // largest Hq / Hkv supported
 constexpr int kMaxQ = kMaxGroup;   // query rows per segment
 
@@ -97,6 +100,15 @@ struct ValidateSetsParams {
   uint32_t* status;
   int32_t nsets, stride, k, k_eff, n;
 };
+
+// Order-preserving map of an fp32 selection key to an unsigned integer
+// (larger key -> larger integer; -0 and +0 map to the same value).
+__host__ __device__ inline uint32_t order_key(float f) {
+  uint32_t b;
+  memcpy(&b, &f, sizeof b);
+  if (b == 0x80000000u) b = 0u;
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
 
 // status word bits
 constexpr uint32_t kStatusBadIndex = 1u;

@@ -5,18 +5,25 @@
 // keys, ties to the lower index (-0 == +0), written in ascending index
 // order, positions k_eff..k-1 set to -1.
 //
-// Design (B200 / sm_100a): one thread-block cluster of CL CTAs per task.
-//   1. each CTA loads its contiguous chunk of n/CL keys once into shared
-//      memory as order-preserving unsigned integers;
-//   2. radix select, most significant digit first (11 + 11 + 10 bits): each
-//      CTA histograms its candidates (warp-aggregated shared atomics), the
-//      cluster sums the histograms through distributed shared memory, and
-//      every CTA finds the same digit of the k-th largest key tau;
-//   3. stable compaction: CTAs exchange their counts of keys > tau and == tau,
-//      which fixes each CTA's output offset and how many of its ties (lowest
-//      indices first) it takes; inside a CTA warps compact in index order
-//      with ballots.
-// No pass reads global memory again after step 1.
+// Design (B200 / sm_100a): radix select of tau, the k_eff-th largest key, on
+// order-preserving 32-bit encodings (digits of 11, 11 and 10 bits), then one
+// stable compaction.  One thread-block cluster of CL CTAs per task; each CTA
+// owns a contiguous chunk of the keys, loaded once into shared memory.
+// Three cluster barriers in the common case:
+//   (1) after every CTA zeroed its totals and histogrammed its chunk's top
+//       digit with shared-memory atomics;
+//   (2) after every CTA added its non-zero bins into every CTA's totals through
+//       distributed shared memory (the adds are spread over all threads); each
+//       CTA then finds the top digit of tau by itself;
+//   (3) after every CTA copied its candidates (keys whose top digit is tau's,
+//       a few per cent of the keys), in index order, into every CTA, with its
+//       count of keys above that digit.
+// Each CTA then finds tau among the candidates, the per-CTA counts of keys
+// > tau and == tau, hence its output offset and how many of its ties (lowest
+// indices first) it takes, and writes its indices with warp ballots.  If the
+// candidates do not fit (heavily tied keys), two more radix digits run over
+// the chunks with totals pushed into every CTA, and the CTA counts are
+// exchanged instead.
 #include <cooperative_groups.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -30,24 +37,17 @@ namespace lyc {
 
 constexpr int kTopkThreads = 512;
 constexpr int kTopkWarps = kTopkThreads / 32;
-constexpr int kBins = 2048;
 
-__device__ __forceinline__ uint32_t order_key(float f) {
-  uint32_t b = __float_as_uint(f);
-  if (b == 0x80000000u) b = 0u;  // -0 == +0
-  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
-}
-
-// Exclusive prefix sum of one value per warp (lane 0 holds it) over the CTA.
-// Returns the exclusive prefix for the caller's warp and the CTA total.
-__device__ __forceinline__ void warp_exclusive_scan(uint32_t* scratch, uint32_t mine, int warp,
-                                                    int lane, uint32_t* prefix, uint32_t* total) {
+// Exclusive prefix sum of one value per warp (lane 0's) over the CTA; also the total.
+__device__ __forceinline__ void cta_warp_scan(uint32_t* scratch, uint32_t mine, int warp, int lane,
+                                              uint32_t* prefix, uint32_t* total) {
   if (lane == 0) scratch[warp] = mine;
   __syncthreads();
   uint32_t acc = 0, tot = 0;
+#pragma unroll
   for (int w = 0; w < kTopkWarps; ++w) {
     const uint32_t v = scratch[w];
-    if (w < warp) acc += v;
+    acc += (w < warp) ? v : 0u;
     tot += v;
   }
   *prefix = acc;
@@ -55,182 +55,381 @@ __device__ __forceinline__ void warp_exclusive_scan(uint32_t* scratch, uint32_t 
   __syncthreads();
 }
 
+// Find the digit d with  sum(hist[> d]) < krem <= sum(hist[>= d]).  Every
+// thread returns the same (digit, count above it).  hist has kKeyBins entries
+// (shared or global memory).
+__device__ __forceinline__ void find_digit(const uint32_t* hist, uint32_t krem, uint32_t* scratch,
+                                           uint32_t* found, int tid, int lane, int warp,
+                                           uint32_t* digit, uint32_t* above_out) {
+  constexpr int per = kKeyBins / kTopkThreads;
+  uint32_t c[per];
+  uint32_t mine = 0u;
+#pragma unroll
+  for (int q = 0; q < per; ++q) {
+    c[q] = hist[tid * per + q];
+    mine += c[q];
+  }
+  uint32_t suf = mine;  // inclusive suffix sum within the warp
+#pragma unroll
+  for (int s = 1; s < 32; s <<= 1) {
+    const uint32_t v = __shfl_down_sync(0xffffffffu, suf, s);
+    if (lane + s < 32) suf += v;
+  }
+  if (lane == 0) scratch[warp] = suf;
+  __syncthreads();
+  uint32_t above = suf - mine;
+  for (int w2 = warp + 1; w2 < kTopkWarps; ++w2) above += scratch[w2];
+#pragma unroll
+  for (int q = per - 1; q >= 0; --q) {
+    if (above < krem && above + c[q] >= krem) {
+      found[0] = static_cast<uint32_t>(tid * per + q);
+      found[1] = above;
+    }
+    above += c[q];
+  }
+  __syncthreads();
+  *digit = found[0];
+  *above_out = found[1];
+  __syncthreads();
+}
+
+}  // namespace lyc
+
+namespace lyc {
+
+// Lists the non-zero bins of hist[kKeyBins] as (bin, count) pairs in `out`
+// (bin order) and returns how many there are.
+__device__ __forceinline__ uint32_t compact_nonzero(const uint32_t* hist, uint2* out,
+                                                    uint32_t* scratch, int tid, int lane, int warp) {
+  constexpr int per = kKeyBins / kTopkThreads;
+  uint32_t c[per];
+  uint32_t mine = 0u;
+#pragma unroll
+  for (int q = 0; q < per; ++q) {
+    c[q] = hist[tid * per + q];
+    mine += c[q] != 0u;
+  }
+  uint32_t inc = mine;  // inclusive prefix within the warp
+#pragma unroll
+  for (int s = 1; s < 32; s <<= 1) {
+    const uint32_t v = __shfl_up_sync(0xffffffffu, inc, s);
+    if (lane >= s) inc += v;
+  }
+  uint32_t before, total;
+  cta_warp_scan(scratch, __shfl_sync(0xffffffffu, inc, 31), warp, lane, &before, &total);
+  uint32_t pos = before + inc - mine;
+#pragma unroll
+  for (int q = 0; q < per; ++q)
+    if (c[q]) out[pos++] = make_uint2(static_cast<uint32_t>(tid * per + q), c[q]);
+  __syncthreads();
+  return total;
+}
+
+// CTA-local radix select over the gathered candidates (source r's entries
+// at cand[r*rcap .. r*rcap + cnt[r]), all sharing the digits in `prefix`):
+// returns the krem-th largest encoded key; *krem becomes the number of
+// candidates equal to it that are to be taken.
+template <int CL>
+__device__ __forceinline__ uint32_t select_in_candidates(const uint2* cand, const uint32_t* cnt,
+                                                         int rcap, uint32_t prefix, uint32_t pmask,
+                                                         uint32_t* krem, uint32_t* hist,
+                                                         uint32_t* scratch, uint32_t* found, int tid,
+                                                         int lane, int warp) {
+#pragma unroll
+  for (int pass = 0; pass < 2; ++pass) {
+    const int sh = pass == 0 ? 10 : 0;
+    const uint32_t dmask = pass == 0 ? 0x7ffu : 0x3ffu;
+    for (int b = tid; b < kKeyBins; b += kTopkThreads) hist[b] = 0u;
+    __syncthreads();
+    for (int x = tid; x < CL * rcap; x += kTopkThreads) {
+      if (static_cast<uint32_t>(x % rcap) < cnt[x / rcap]) {
+        const uint32_t u = cand[x].x;
+        if ((u & pmask) == prefix) atomicAdd(&hist[(u >> sh) & dmask], 1u);
+      }
+    }
+    __syncthreads();
+    uint32_t dg, ab;
+    find_digit(hist, *krem, scratch, found, tid, lane, warp, &dg, &ab);
+    *krem -= ab;
+    prefix |= dg << sh;
+    pmask |= dmask << sh;
+  }
+  return prefix;
+}
+
 template <int CL>
 __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster_kernel(const TopkParams p) {
   cg::cluster_group cluster = cg::this_cluster();
+  constexpr int CAP = 4096;        // gathered candidates (all CTAs together)
+  constexpr int RCAP = CAP / CL;   // candidates one CTA may contribute
   const int rank = static_cast<int>(cluster.block_rank());
   const TopkTask task = p.tasks ? p.tasks[blockIdx.y] : p.single;
   const int n = p.n;
   const int k = p.k;
   const int keff = k < n ? k : n;
-  const int chunk = (n + CL - 1) / CL;
+  const int chunk = (((n + CL - 1) / CL) + 3) & ~3;
   const int lo = rank * chunk;
   const int cnt = max(0, min(n, lo + chunk) - lo);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const unsigned lt = (1u << lane) - 1u;
 
   extern __shared__ __align__(16) unsigned char smem[];
-  uint32_t* hist = reinterpret_cast<uint32_t*>(smem);            // [kBins]
-  uint32_t* total = hist + kBins;                                // [kBins]
-  uint32_t* xchg = total + kBins;                                // [CL][2]
-  uint32_t* scratch = xchg + 2 * CL;                             // [kTopkWarps]
-  uint32_t* found = scratch + kTopkWarps;                        // [2]: digit, count above
-  uint32_t* us = found + 4;                                      // [chunk]
+  uint2* cand = reinterpret_cast<uint2*>(smem);        // [CAP] (encoded key, index) by source CTA
+  uint32_t* loc = reinterpret_cast<uint32_t*>(cand + CAP);  // [kKeyBins] this CTA's histogram
+  uint32_t* tot = loc + kKeyBins;                      // [kKeyBins] cluster totals, top digit
+  uint32_t* src_cnt = tot + kKeyBins;                  // [CL] candidates per source CTA
+  uint32_t* src_above = src_cnt + CL;                  // [CL] keys above the pivot digit per source
+  uint32_t* src_gt = src_above + CL;                   // [CL] per source: keys > tau
+  uint32_t* src_eq = src_gt + CL;                      // [CL] per source: keys == tau
+  uint32_t* xchg = src_eq + CL;                        // [CL][2] (fallback path)
+  uint32_t* scratch = xchg + 2 * CL;                   // [kTopkWarps]
+  uint32_t* found = scratch + kTopkWarps;              // [4]
+  uint32_t* us = found + 4;                            // [chunk] encoded keys
 
-  // all indices selected: no ordering work
-  if (keff == n) {
+  if (keff == n) {  // every index is selected
     for (int x = tid; x < cnt; x += kTopkThreads) task.S[lo + x] = lo + x;
     if (rank == 0)
       for (int x = keff + tid; x < k; x += kTopkThreads) task.S[x] = -1;
     return;
   }
 
-  for (int x = tid; x < cnt; x += kTopkThreads) us[x] = order_key(task.keys[lo + x]);
+  for (int b = tid; b < kKeyBins; b += kTopkThreads) {
+    tot[b] = 0u;
+    loc[b] = 0u;
+  }
+  __syncthreads();
+  // ---- the chunk, encoded, into shared memory, and its top-digit histogram
+  const float* src = task.keys + lo;
+  const bool vec = (reinterpret_cast<uintptr_t>(src) & 15u) == 0;
+  const int nv = vec ? (cnt >> 2) : 0;
+  for (int x = tid; x < nv; x += kTopkThreads) {
+    const float4 v = reinterpret_cast<const float4*>(src)[x];
+    const uint32_t a = order_key(v.x), b = order_key(v.y), c = order_key(v.z), d = order_key(v.w);
+    us[4 * x + 0] = a;
+    us[4 * x + 1] = b;
+    us[4 * x + 2] = c;
+    us[4 * x + 3] = d;
+    atomicAdd(&loc[a >> kKeyDigitShift], 1u);
+    atomicAdd(&loc[b >> kKeyDigitShift], 1u);
+    atomicAdd(&loc[c >> kKeyDigitShift], 1u);
+    atomicAdd(&loc[d >> kKeyDigitShift], 1u);
+  }
+  for (int x = (nv << 2) + tid; x < cnt; x += kTopkThreads) {
+    const uint32_t a = order_key(src[x]);
+    us[x] = a;
+    atomicAdd(&loc[a >> kKeyDigitShift], 1u);
+  }
+  cluster.sync();  // (1) every CTA's totals are zero
 
-  // ---- radix select of tau, the k-th largest key
-  uint32_t prefix = 0u, pmask = 0u;
-  uint32_t krem = static_cast<uint32_t>(keff);
-#pragma unroll
-  for (int pass = 0; pass < 3; ++pass) {
-    const int sh = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
-    const uint32_t dmask = pass == 2 ? 0x3ffu : 0x7ffu;
-    for (int b = tid; b < kBins; b += kTopkThreads) hist[b] = 0u;
-    __syncthreads();
-    for (int base = 0; base < cnt; base += kTopkThreads) {
-      const int x = base + tid;
-      const uint32_t u = (x < cnt) ? us[x] : 0u;
-      const bool cand = (x < cnt) && ((u & pmask) == prefix);
-      const unsigned act = __ballot_sync(0xffffffffu, cand);
-      if (cand) {
-        const uint32_t dg = (u >> sh) & dmask;
-        const unsigned peers = __match_any_sync(act, dg);
-        if (lane == __ffs(peers) - 1) atomicAdd(&hist[dg], static_cast<uint32_t>(__popc(peers)));
+  // ---- top digit: add the non-zero local bins into every CTA's totals
+  {
+    uint2* nz = cand;  // (bin, count) of the non-zero local bins; free until the gather
+    const uint32_t nnz = compact_nonzero(loc, nz, scratch, tid, lane, warp);
+    for (uint32_t x = tid; x < nnz * CL; x += kTopkThreads) {
+      const uint2 e = nz[x / CL];
+      atomicAdd(cluster.map_shared_rank(tot, static_cast<int>(x % CL)) + e.x, e.y);
+    }
+  }
+  cluster.sync();  // (2)
+  uint32_t d0, above;
+  find_digit(tot, static_cast<uint32_t>(keff), scratch, found, tid, lane, warp, &d0, &above);
+  uint32_t krem = static_cast<uint32_t>(keff) - above;
+  const uint32_t ncand = tot[d0];
+
+  // ---- this CTA's candidates (top digit == d0), in index order, gathered
+  // into every CTA together with the count of its keys above the digit
+  uint32_t my_cand = 0u, my_above = 0u;
+  {
+    const int span = ((cnt + kTopkWarps - 1) / kTopkWarps + 31) & ~31;
+    const int wlo = warp * span;
+    const int whi = min(cnt, wlo + span);
+    uint32_t wc = 0u, wa = 0u;
+    for (int base = wlo; base < whi; base += 32) {
+      const int x = base + lane;
+      const uint32_t dg = (x < whi) ? (us[x] >> kKeyDigitShift) : 0u;
+      wc += __popc(__ballot_sync(0xffffffffu, x < whi && dg == d0));
+      wa += __popc(__ballot_sync(0xffffffffu, x < whi && dg > d0));
+    }
+    uint32_t c_before, a_before;
+    cta_warp_scan(scratch, wc, warp, lane, &c_before, &my_cand);
+    cta_warp_scan(scratch, wa, warp, lane, &a_before, &my_above);
+    if (my_cand <= static_cast<uint32_t>(RCAP)) {
+      // own candidates, in index order, into this CTA's region first
+      uint2* mine = cand + rank * RCAP;
+      uint32_t pos = c_before;
+      for (int base = wlo; base < whi; base += 32) {
+        const int x = base + lane;
+        const uint32_t u = (x < whi) ? us[x] : 0u;
+        const bool is_c = x < whi && (u >> kKeyDigitShift) == d0;
+        const unsigned cb = __ballot_sync(0xffffffffu, is_c);
+        if (is_c) mine[pos + __popc(cb & lt)] = make_uint2(u, static_cast<uint32_t>(lo + x));
+        pos += __popc(cb);
+      }
+      __syncthreads();
+      // then copies into the other CTAs, (entry, CTA) pairs spread over the threads
+      for (uint32_t x = tid; x < my_cand * (CL - 1); x += kTopkThreads) {
+        const uint32_t j = x / (CL - 1);
+        const int r = static_cast<int>(x % (CL - 1));
+        const int dst = r < rank ? r : r + 1;
+        cluster.map_shared_rank(cand, dst)[rank * RCAP + j] = mine[j];
       }
     }
-    cluster.sync();
-    // this CTA sums its slice of bins over the cluster and hands the sums to all
-    constexpr int slice = kBins / CL;
-    for (int b = rank * slice + tid; b < (rank + 1) * slice; b += kTopkThreads) {
-      uint32_t s = 0u;
-#pragma unroll
-      for (int r = 0; r < CL; ++r) s += cluster.map_shared_rank(hist, r)[b];
-#pragma unroll
-      for (int r = 0; r < CL; ++r) cluster.map_shared_rank(total, r)[b] = s;
+    if (tid < CL) {
+      cluster.map_shared_rank(src_cnt, tid)[rank] = my_cand;
+      cluster.map_shared_rank(src_above, tid)[rank] = my_above;
     }
-    cluster.sync();
-    // digit of tau: the one where the count of larger candidates crosses krem
-    constexpr int per = kBins / kTopkThreads;  // bins per thread
-    uint32_t mine = 0u;
-#pragma unroll
-    for (int q = 0; q < per; ++q) mine += total[tid * per + q];
-    // inclusive sum of `mine` over threads with a larger id (suffix), per warp then CTA
-    uint32_t suf = mine;
-#pragma unroll
-    for (int s = 1; s < 32; s <<= 1) {
-      const uint32_t v = __shfl_down_sync(0xffffffffu, suf, s);
-      if (lane + s < 32) suf += v;
-    }
-    if (lane == 0) scratch[warp] = suf;  // warp total
-    __syncthreads();
-    uint32_t above = suf - mine;  // strictly larger threads within the warp
-    for (int w2 = warp + 1; w2 < kTopkWarps; ++w2) above += scratch[w2];
-#pragma unroll
-    for (int q = per - 1; q >= 0; --q) {
-      const uint32_t c = total[tid * per + q];
-      if (above < krem && above + c >= krem) {
-        found[0] = static_cast<uint32_t>(tid * per + q);
-        found[1] = above;
+  }
+  cluster.sync();  // (3) candidates and counts of every CTA are here
+
+  bool fits = ncand <= static_cast<uint32_t>(CAP);
+  for (int r = 0; r < CL; ++r) fits = fits && src_cnt[r] <= static_cast<uint32_t>(RCAP);
+
+  uint32_t tau, out_base, take;
+  if (fits) {
+    // ---- tau among the gathered candidates, the same in every CTA
+    tau = select_in_candidates<CL>(cand, src_cnt, RCAP, d0 << kKeyDigitShift, 0xffe00000u, &krem,
+                                   loc, scratch, found, tid, lane, warp);
+    // per source: keys > tau and == tau (warp w counts the sources w, w+16, ...)
+    for (int r = warp; r < CL; r += kTopkWarps) {
+      const uint32_t c = src_cnt[r];
+      uint32_t g = 0u, e = 0u;
+      for (uint32_t base = 0; base < c; base += 32) {
+        const uint32_t x = base + lane;
+        const uint32_t u = (x < c) ? cand[r * RCAP + x].x : 0u;
+        g += __popc(__ballot_sync(0xffffffffu, x < c && u > tau));
+        e += __popc(__ballot_sync(0xffffffffu, x < c && u == tau));
       }
-      above += c;
+      if (lane == 0) {
+        src_gt[r] = src_above[r] + g;
+        src_eq[r] = e;
+      }
     }
     __syncthreads();
-    const uint32_t dg = found[0];
-    krem -= found[1];
-    prefix |= dg << sh;
-    pmask |= dmask << sh;
-    __syncthreads();
+    out_base = 0u;
+    uint32_t eq_prev = 0u;
+    for (int r = 0; r < rank; ++r) {
+      const uint32_t e = src_eq[r];
+      const uint32_t tk = (krem > eq_prev) ? min(krem - eq_prev, e) : 0u;
+      out_base += src_gt[r] + tk;
+      eq_prev += e;
+    }
+    take = (krem > eq_prev) ? min(krem - eq_prev, src_eq[rank]) : 0u;
+  } else {
+    // ---- too many candidates (heavily tied keys): two more radix digits over
+    // the chunks, totals pushed into every CTA, then a count exchange
+    uint32_t* tot12 = reinterpret_cast<uint32_t*>(cand);  // the candidates are not needed here
+    for (int b = tid; b < 2 * kKeyBins; b += kTopkThreads) tot12[b] = 0u;
+    cluster.sync();  // every CTA's digit-1/2 totals are zero
+    uint32_t prefix = d0 << kKeyDigitShift, pmask = 0xffe00000u;
+#pragma unroll
+    for (int pass = 1; pass <= 2; ++pass) {
+      const int sh = pass == 1 ? 10 : 0;
+      const uint32_t dmask = pass == 1 ? 0x7ffu : 0x3ffu;
+      uint32_t* tp = tot12 + (pass - 1) * kKeyBins;
+      for (int b = tid; b < kKeyBins; b += kTopkThreads) loc[b] = 0u;
+      __syncthreads();
+      for (int x = tid; x < cnt; x += kTopkThreads) {
+        const uint32_t u = us[x];
+        if ((u & pmask) == prefix) atomicAdd(&loc[(u >> sh) & dmask], 1u);
+      }
+      __syncthreads();
+      for (int x = tid; x < CL * kKeyBins; x += kTopkThreads) {
+        const int b = x % kKeyBins, r = x / kKeyBins;
+        const uint32_t c = loc[b];
+        if (c) atomicAdd(cluster.map_shared_rank(tp, r) + b, c);
+      }
+      cluster.sync();
+      uint32_t dg, ab;
+      find_digit(tp, krem, scratch, found, tid, lane, warp, &dg, &ab);
+      krem -= ab;
+      prefix |= dg << sh;
+      pmask |= dmask << sh;
+    }
+    tau = prefix;
+    uint32_t g = 0u, e = 0u;
+    for (int x = tid; x < cnt; x += kTopkThreads) {
+      const uint32_t u = us[x];
+      g += u > tau;
+      e += u == tau;
+    }
+    uint32_t dummy, gt_cta, eq_cta;
+    const unsigned FULL = 0xffffffffu;
+#pragma unroll
+    for (int s2 = 16; s2 >= 1; s2 >>= 1) {
+      g += __shfl_xor_sync(FULL, g, s2);
+      e += __shfl_xor_sync(FULL, e, s2);
+    }
+    cta_warp_scan(scratch, g, warp, lane, &dummy, &gt_cta);
+    cta_warp_scan(scratch, e, warp, lane, &dummy, &eq_cta);
+    if (tid < CL) {
+      uint32_t* xd = cluster.map_shared_rank(xchg, tid);
+      xd[2 * rank] = gt_cta;
+      xd[2 * rank + 1] = eq_cta;
+    }
+    cluster.sync();
+    out_base = 0u;
+    uint32_t eq_prev = 0u;
+    for (int r = 0; r < rank; ++r) {
+      const uint32_t gg = xchg[2 * r], ee = xchg[2 * r + 1];
+      const uint32_t tk = (krem > eq_prev) ? min(krem - eq_prev, ee) : 0u;
+      out_base += gg + tk;
+      eq_prev += ee;
+    }
+    take = (krem > eq_prev) ? min(krem - eq_prev, eq_cta) : 0u;
   }
-  const uint32_t tau = prefix;  // krem = how many keys equal to tau are taken
 
-  // ---- counts of this CTA, exchanged across the cluster
-  uint32_t gt = 0u, eq = 0u;
-  for (int base = 0; base < cnt; base += kTopkThreads) {
-    const int x = base + tid;
-    const uint32_t u = (x < cnt) ? us[x] : 0u;
-    gt += __popc(__ballot_sync(0xffffffffu, x < cnt && u > tau));
-    eq += __popc(__ballot_sync(0xffffffffu, x < cnt && u == tau));
-  }
-  uint32_t gt_cta, eq_cta, dummy;
-  warp_exclusive_scan(scratch, gt, warp, lane, &dummy, &gt_cta);
-  warp_exclusive_scan(scratch, eq, warp, lane, &dummy, &eq_cta);
-  if (tid < CL) {
-    uint32_t* dst = cluster.map_shared_rank(xchg, tid);
-    dst[2 * rank] = gt_cta;
-    dst[2 * rank + 1] = eq_cta;
-  }
-  cluster.sync();
-  uint32_t out_base = 0u, eq_before = 0u;
-  for (int r = 0; r < rank; ++r) {
-    const uint32_t g = xchg[2 * r], e = xchg[2 * r + 1];
-    const uint32_t tk = (krem > eq_before) ? min(krem - eq_before, e) : 0u;
-    out_base += g + tk;
-    eq_before += e;
-  }
-  const uint32_t take = (krem > eq_before) ? min(krem - eq_before, eq_cta) : 0u;
-
-  // ---- stable compaction: warp w owns elements [w*span, (w+1)*span)
-  const int span = ((cnt + kTopkWarps - 1) / kTopkWarps + 31) & ~31;
+  // ---- write this CTA's selected indices in index order: warp w owns
+  // [w*span, (w+1)*span), span a multiple of 128, four ballot rows per step
+  const int span = ((cnt + kTopkWarps - 1) / kTopkWarps + 127) & ~127;
   const int wlo = warp * span;
   const int whi = min(cnt, wlo + span);
-  const unsigned lt = (1u << lane) - 1u;
-  uint32_t weq = 0u;
-  for (int base = wlo; base < whi; base += 32) {
-    const int x = base + lane;
-    weq += __popc(__ballot_sync(0xffffffffu, x < whi && us[x] == tau));
-  }
-  uint32_t eq_base, eq_tot;
-  warp_exclusive_scan(scratch, weq, warp, lane, &eq_base, &eq_tot);
-  uint32_t wsel = 0u;
-  {
-    uint32_t run_eq = eq_base;
-    for (int base = wlo; base < whi; base += 32) {
-      const int x = base + lane;
+  uint32_t wgt = 0u, weq = 0u;
+  for (int base = wlo; base < whi; base += 128) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int x = base + 32 * j + lane;
       const uint32_t u = (x < whi) ? us[x] : 0u;
-      const bool is_eq = x < whi && u == tau;
-      const unsigned eb = __ballot_sync(0xffffffffu, is_eq);
-      const bool sel = (x < whi) && (u > tau || (is_eq && run_eq + __popc(eb & lt) < take));
-      wsel += __popc(__ballot_sync(0xffffffffu, sel));
-      run_eq += __popc(eb);
+      wgt += __popc(__ballot_sync(0xffffffffu, x < whi && u > tau));
+      weq += __popc(__ballot_sync(0xffffffffu, x < whi && u == tau));
     }
   }
-  uint32_t sel_base, sel_tot;
-  warp_exclusive_scan(scratch, wsel, warp, lane, &sel_base, &sel_tot);
-  {
-    uint32_t run_eq = eq_base, run_sel = out_base + sel_base;
-    for (int base = wlo; base < whi; base += 32) {
-      const int x = base + lane;
-      const uint32_t u = (x < whi) ? us[x] : 0u;
-      const bool is_eq = x < whi && u == tau;
-      const unsigned eb = __ballot_sync(0xffffffffu, is_eq);
-      const bool sel = (x < whi) && (u > tau || (is_eq && run_eq + __popc(eb & lt) < take));
+  uint32_t gt_before, eq_before, dummy2;
+  cta_warp_scan(scratch, wgt, warp, lane, &gt_before, &dummy2);
+  cta_warp_scan(scratch, weq, warp, lane, &eq_before, &dummy2);
+  uint32_t run_eq = eq_before;
+  uint32_t run_sel = out_base + gt_before + min(eq_before, take);
+  for (int base = wlo; base < whi; base += 128) {
+    uint32_t u[4];
+    unsigned gb[4], eb[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int x = base + 32 * j + lane;
+      u[j] = (x < whi) ? us[x] : 0u;
+      gb[j] = __ballot_sync(0xffffffffu, x < whi && u[j] > tau);
+      eb[j] = __ballot_sync(0xffffffffu, x < whi && u[j] == tau);
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int x = base + 32 * j + lane;
+      const bool is_eq = (eb[j] >> lane) & 1u;
+      const bool sel = ((gb[j] >> lane) & 1u) || (is_eq && run_eq + __popc(eb[j] & lt) < take);
       const unsigned sb = __ballot_sync(0xffffffffu, sel);
       const uint32_t pos = run_sel + __popc(sb & lt);
       if (sel && pos < static_cast<uint32_t>(keff)) task.S[pos] = lo + x;
       run_sel += __popc(sb);
-      run_eq += __popc(eb);
+      run_eq += __popc(eb[j]);
     }
   }
   if (rank == 0)
     for (int x = keff + tid; x < k; x += kTopkThreads) task.S[x] = -1;
-  (void)eq_tot;
-  (void)sel_tot;
-  // no CTA leaves while another may still read its shared memory: the last
-  // remote access (the count exchange) precedes the cluster.sync above.
+  // no CTA leaves while another may still access its shared memory: every
+  // remote access precedes the last cluster barrier on its path.
 }
 
 // ---------------------------------------------------------------- host side
 static size_t topk_smem_bytes(int cl, int n) {
-  const int chunk = (n + cl - 1) / cl;
-  return static_cast<size_t>(2 * kBins + 2 * cl + kTopkWarps + 4 + chunk) * 4u;
+  const int chunk = (((n + cl - 1) / cl) + 3) & ~3;
+  return static_cast<size_t>(2 * 4096 + 2 * kKeyBins + 6 * cl + kTopkWarps + 4 + chunk) * 4u;
 }
 
 template <int CL>
@@ -292,5 +491,6 @@ cudaError_t topk_configure(int cl, size_t smem) {
 cudaError_t topk_launch(int cl, const TopkParams* p, int ntasks, cudaStream_t stream) {
   return cl == 16 ? topk_run<16>(p, ntasks, stream, false, 0) : topk_run<8>(p, ntasks, stream, false, 0);
 }
+
 
 }  // namespace lyc

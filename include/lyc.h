@@ -64,7 +64,7 @@ typedef struct {
   int num_q_heads;  /* Hq >= 1 */
   int num_kv_heads; /* Hkv >= 1, Hq % Hkv == 0, Hq / Hkv <= 8 */
   int head_dim;     /* d in {64, 128} */
-  int64_t max_ctx;  /* largest n any step will use, 1 <= max_ctx <= 786432 */
+  int64_t max_ctx;  /* largest n any step will use, 1 <= max_ctx <= 655360 */
   int max_k;        /* largest k any step will use, >= 1 */
   lyc_dtype dtype;  /* element type of q, K and V */
   lyc_select_mode select_mode;

@@ -135,11 +135,16 @@ __device__ __forceinline__ void attn_producer(const AttnParams& p, unsigned char
   // Lookahead cursor: issues the index-list copy of sparse tiles LA tiles
   // before the main cursor needs them.
   int la_pc = pbeg, la_r0 = (pbeg < pend) ? p.pieces[pbeg].r0 : 0, la_t = 0;
+  bool waited = false;  // the previous layer's selection has completed
   auto la_step = [&]() {
     if (la_pc >= pend) return;
     const Piece pc = p.pieces[la_pc];
     const Segment& sg = p.segs[pc.seg];
     if (sg.kind == kSparse && lane == 0) {
+      if (!waited) {  // the inherited sets are that kernel's output
+        pdl_wait();
+        waited = true;
+      }
       const int slot = la_t % C::IR;
       const int nrows = min(kTileRows, pc.r1 - la_r0);
       const uint32_t bytes = static_cast<uint32_t>(((nrows * 4) + 15) & ~15);
@@ -467,6 +472,7 @@ __global__ void __launch_bounds__(AttnCfg<T, D, NQ, STAGES>::kThreads, 1)
     fence_mbar_init();
   }
   __syncthreads();
+  pdl_launch_dependents();
   const int pbeg = p.cta_begin[blockIdx.x];
   const int pend = p.cta_begin[blockIdx.x + 1];
   if (threadIdx.x >= C::kConsumerWarps * 32) {
@@ -474,6 +480,7 @@ __global__ void __launch_bounds__(AttnCfg<T, D, NQ, STAGES>::kThreads, 1)
   } else {
     attn_consumers<T, D, NQ, STAGES>(p, smem, pbeg, pend);
   }
+  if (threadIdx.x == 0) pdl_wait();  // complete only after the grid this one depends on
 }
 
 }  // namespace lyc
@@ -497,10 +504,23 @@ static cudaError_t attn_run(const AttnParams* p, int grid, cudaStream_t stream, 
   auto kern = attn_layer_kernel<T, D, NQ, S>;
   if (configure_only) {
     if (smem_out) *smem_out = C::SMEM;
-    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                               cudaSharedmemCarveoutMaxShared);
+    return e;
   }
-  kern<<<grid, C::kThreads, C::SMEM, stream>>>(*p);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(C::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = C::SMEM;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, *p);
 }
 
 template <typename T, int D>

@@ -166,10 +166,15 @@ __device__ __forceinline__ void mma_producers(const AttnMmaParams& P, unsigned c
 
   // lookahead cursor (leader only): index-list copies of gathered tiles, LA tiles early
   int la_pc = pbeg, la_r0 = (pbeg < pend) ? p.pieces[pbeg].r0 : 0, la_t = 0;
+  bool waited = false;  // the previous layer's selection has completed
   auto la_step = [&]() {
     if (la_pc >= pend) return;
     const Piece pc = p.pieces[la_pc];
     if (p.segs[pc.seg].kind == kSparse) {
+      if (!waited) {  // the inherited sets are that kernel's output
+        pdl_wait();
+        waited = true;
+      }
       const int slot = la_t % C::IR;
       const int nrows = min(kTileRows, pc.r1 - la_r0);
       const uint32_t bytes = static_cast<uint32_t>(((nrows * 4) + 15) & ~15);
@@ -496,32 +501,52 @@ __device__ __forceinline__ void mma_consumers(const AttnMmaParams& P, unsigned c
     }
     named_bar_sync(1, NC * 32);
 
-    // ---- the last piece of the segment combines every piece (log-sum-exp)
-    for (int o = 0; o < nout; ++o) {
-      if (!lastflag[o]) continue;
-      const int base = sg.part_base + o;
-      const int np = sg.npieces;
-      for (int e = tid; e < D; e += NC * 32) {
-        float M = -INFINITY;
-        for (int u2 = 0; u2 < np; ++u2) M = fmaxf(M, __ldcg(&p.part_ml[base + u2 * nout]).x);
-        float L = 0.f, O = 0.f;
-        if (M != -INFINITY) {
-          for (int u2 = 0; u2 < np; ++u2) {
-            const float2 ml = __ldcg(&p.part_ml[base + u2 * nout]);
-            const float f = (ml.x == -INFINITY) ? 0.f : exp2f(ml.x - M);
-            L = fmaf(f, ml.y, L);
-            O = fmaf(f, __ldcg(&p.part_o[static_cast<int64_t>(base + u2 * nout) * D + e]), O);
+    // ---- the last piece of a segment combines every piece (log-sum-exp).
+    // All finished outputs at once: thread (o, c4) owns output o's columns
+    // 4*c4 .. 4*c4+3 and folds the partials in with a running maximum, eight
+    // partials' loads in flight at a time.
+    {
+      constexpr int C4 = D / 4;
+      for (int x = tid; x < nout * C4; x += NC * 32) {
+        const int o = x / C4, c4 = x % C4;
+        if (!lastflag[o]) continue;
+        const int base = sg.part_base + o;
+        const int np = sg.npieces;
+        float M = -INFINITY, L = 0.f;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int u0 = 0; u0 < np; u0 += 8) {
+          float2 ml[8];
+          float4 ov[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int part = base + min(u0 + j, np - 1) * nout;
+            ml[j] = __ldcg(&p.part_ml[part]);
+            ov[j] = __ldcg(reinterpret_cast<const float4*>(&p.part_o[static_cast<int64_t>(part) * D + 4 * c4]));
+          }
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            if (u0 + j >= np || ml[j].x == -INFINITY) continue;
+            const float mn = fmaxf(M, ml[j].x);
+            const float a = (M == -INFINITY) ? 0.f : exp2f(M - mn);
+            const float f = exp2f(ml[j].x - mn);
+            L = L * a + f * ml[j].y;
+            acc.x = acc.x * a + f * ov[j].x;
+            acc.y = acc.y * a + f * ov[j].y;
+            acc.z = acc.z * a + f * ov[j].z;
+            acc.w = acc.w * a + f * ov[j].w;
+            M = mn;
           }
         }
-        float res = 0.f;
+        float4 res = make_float4(0.f, 0.f, 0.f, 0.f);
         if (L > 0.f) {
-          res = O / L;
-        } else if (e == 0) {
+          const float inv = 1.f / L;
+          res = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+        } else if (c4 == 0) {
           atomicOr(p.status, kStatusEmptySoftmax);
         }
-        p.out[(static_cast<int64_t>(b) * p.Hq + sg.head[sg.out_row[o]]) * D + e] = res;
+        *reinterpret_cast<float4*>(&p.out[(static_cast<int64_t>(b) * p.Hq + sg.head[sg.out_row[o]]) * D + 4 * c4]) = res;
+        if (c4 == 0) p.counters[sg.cnt_base + o] = 0;
       }
-      if (tid == 0) p.counters[sg.cnt_base + o] = 0;
     }
     named_bar_sync(1, NC * 32);  // merge area and flags free for the next piece
   }
@@ -551,6 +576,7 @@ __global__ void __launch_bounds__(MmaCfg<D, NC, NP, STAGES>::kThreads, 1)
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&P.tmv)) : "memory");
   }
   __syncthreads();
+  pdl_launch_dependents();
   const int pbeg = P.p.cta_begin[blockIdx.x];
   const int pend = P.p.cta_begin[blockIdx.x + 1];
   if (threadIdx.x >= NC * 32) {
@@ -558,6 +584,9 @@ __global__ void __launch_bounds__(MmaCfg<D, NC, NP, STAGES>::kThreads, 1)
   } else {
     mma_consumers<D, NC, NP, STAGES>(P, smem, pbeg, pend);
   }
+  // this grid completes only after the one it depends on (dense-only CTAs
+  // never waited above), so completion order follows launch order
+  if (threadIdx.x == 0) pdl_wait();
 }
 
 // ---------------------------------------------------------------- host side
@@ -568,10 +597,25 @@ static cudaError_t mma_run(const AttnMmaParams* P, int grid, cudaStream_t stream
   auto kern = attn_mma_layer_kernel<D, NC, NP, STAGES>;
   if (configure_only) {
     if (smem_out) *smem_out = C::SMEM;
-    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    // every kernel of the step asks for the same shared-memory carveout, so an
+    // SM never has to reconfigure between consecutive kernels
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                               cudaSharedmemCarveoutMaxShared);
+    return e;
   }
-  kern<<<grid, C::kThreads, C::SMEM, stream>>>(*P);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(C::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = C::SMEM;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, *P);
 }
 
 // bf16 inputs.  configure_only: set the shared-memory attribute, report the size.

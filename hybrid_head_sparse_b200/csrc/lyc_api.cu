@@ -236,6 +236,9 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const lyc_k
 
   for (int l = 0; l < L; ++l) {
     HostLayer& H = hl[l];
+    // selection keys alternate between two buffers by layer, so a layer's
+    // attention never writes the keys the previous layer's selection reads
+    const int64_t keys_base = (l & 1) * static_cast<int64_t>(B) * Hs * ctx->nstride;
     std::vector<char> is_ret(Hq), fresh(Hs, 0);
     for (int h = 0; h < Hq; ++h) {
       is_ret[h] = (l == 0 && !s_in) || role[static_cast<int64_t>(l) * Hq + h] != 0;
@@ -271,12 +274,12 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const lyc_k
             if (!kvmode && !is_ret[h]) continue;
             ds.head[j] = h;
             if (is_ret[h]) ds.out_row[o++] = j;
-            if (!kvmode) ds.key_off[j] = (static_cast<int64_t>(b) * Hs + h) * ctx->nstride;
+            if (!kvmode) ds.key_off[j] = keys_base + (static_cast<int64_t>(b) * Hs + h) * ctx->nstride;
             ++j;
           }
           ds.nq = j;
           ds.nout = o;
-          if (kvmode) ds.key_mean_off = (static_cast<int64_t>(b) * Hs + g) * ctx->nstride;
+          if (kvmode) ds.key_mean_off = keys_base + (static_cast<int64_t>(b) * Hs + g) * ctx->nstride;
           maxnq = std::max(maxnq, j);
           H.segs.push_back(ds);
         }
@@ -314,30 +317,56 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const lyc_k
     }
     H.nqb = attn_nq_bucket(maxnq);
 
-    // workload pooling: equal runs of 64-row tiles, one run per CTA
-    std::vector<int64_t> tstart(H.segs.size() + 1, 0);
-    for (size_t s = 0; s < H.segs.size(); ++s)
-      tstart[s + 1] = tstart[s] + (H.segs[s].rows + kTileRows - 1) / kTileRows;
-    const int64_t NT = tstart.back();
-    const int grid = static_cast<int>(std::min<int64_t>(NT, ctx->sms));
+    // workload pooling (two phases): the dense rows are cut into equal runs of
+    // 64-row tiles, one per CTA, and so are the gathered rows; CTA c takes its
+    // dense run, then its gathered run, so every CTA carries the same mix
+    // whatever the relative cost of streaming and gathering a tile
+    int64_t NT = 0;
+    for (const Segment& sg : H.segs) NT += (sg.rows + kTileRows - 1) / kTileRows;
+    // The previous layer's selection runs beside this layer's attention (the
+    // attention streams its dense rows meanwhile and waits for the sets only
+    // before its gathered rows).  When that selection is small, leave its SMs
+    // to it: fewer SMs still stream at full HBM bandwidth, and no CTA of this
+    // kernel then starts late behind it.
+    int avail = ctx->sms;
+    if (l > 0) {
+      const int prev = static_cast<int>(hl[l - 1].tasks.size()) * ctx->topk_cl;
+      if (prev > 0 && prev <= ctx->sms / 4) avail = ctx->sms - prev;
+    }
+    const int grid = static_cast<int>(std::min<int64_t>(NT, avail));
     H.grid = grid;
     std::vector<int> npieces(H.segs.size(), 0);
-    size_t seg_i = 0;
+    std::vector<std::vector<Piece>> per_cta(grid);
+    for (int phase = 0; phase < 2; ++phase) {
+      const int want = phase == 0 ? kDense : kSparse;
+      std::vector<size_t> ids;
+      std::vector<int64_t> tstart(1, 0);
+      for (size_t s2 = 0; s2 < H.segs.size(); ++s2) {
+        if (H.segs[s2].kind != want) continue;
+        ids.push_back(s2);
+        tstart.push_back(tstart.back() + (H.segs[s2].rows + kTileRows - 1) / kTileRows);
+      }
+      const int64_t nt = tstart.back();
+      size_t si = 0;
+      for (int c = 0; c < grid; ++c) {
+        const int64_t t0 = nt * c / grid, t1 = nt * (c + 1) / grid;
+        while (si < ids.size() && tstart[si + 1] <= t0) ++si;
+        for (size_t q = si; q < ids.size() && tstart[q] < t1; ++q) {
+          const int64_t a = std::max(t0, tstart[q]) - tstart[q];
+          const int64_t e = std::min(t1, tstart[q + 1]) - tstart[q];
+          if (e <= a) continue;
+          Piece pc;
+          pc.seg = static_cast<int32_t>(ids[q]);
+          pc.r0 = static_cast<int32_t>(a * kTileRows);
+          pc.r1 = static_cast<int32_t>(std::min<int64_t>(e * kTileRows, H.segs[ids[q]].rows));
+          pc.ordinal = npieces[ids[q]]++;
+          per_cta[c].push_back(pc);
+        }
+      }
+    }
     for (int c = 0; c < grid; ++c) {
       H.cta.push_back(static_cast<int32_t>(H.pieces.size()));
-      const int64_t t0 = NT * c / grid, t1 = NT * (c + 1) / grid;
-      while (seg_i < H.segs.size() && tstart[seg_i + 1] <= t0) ++seg_i;
-      for (size_t s = seg_i; s < H.segs.size() && tstart[s] < t1; ++s) {
-        const int64_t a = std::max(t0, tstart[s]) - tstart[s];
-        const int64_t e = std::min(t1, tstart[s + 1]) - tstart[s];
-        if (e <= a) continue;
-        Piece pc;
-        pc.seg = static_cast<int32_t>(s);
-        pc.r0 = static_cast<int32_t>(a * kTileRows);
-        pc.r1 = static_cast<int32_t>(std::min<int64_t>(e * kTileRows, H.segs[s].rows));
-        pc.ordinal = npieces[s]++;
-        H.pieces.push_back(pc);
-      }
+      for (const Piece& pc : per_cta[c]) H.pieces.push_back(pc);
     }
     H.cta.push_back(static_cast<int32_t>(H.pieces.size()));
     int part = 0, cnt = 0;
@@ -356,7 +385,7 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const lyc_k
       if (!fresh[s]) continue;
       for (int b = 0; b < B; ++b) {
         TopkTask tk;
-        tk.keys = ctx->keys + (static_cast<int64_t>(b) * Hs + s) * ctx->nstride;
+        tk.keys = ctx->keys + keys_base + (static_cast<int64_t>(b) * Hs + s) * ctx->nstride;
         tk.S = set_ptr(1 - cur[s], b, s);
         H.tasks.push_back(tk);
       }
@@ -658,7 +687,7 @@ lyc_status lyc_create(const lyc_config* cfg, lyc_ctx** out) {
   const int B = c.batch, Hq = c.num_q_heads, Hkv = c.num_kv_heads, D = c.head_dim, L = c.num_layers;
   const size_t es = c.dtype == LYC_BF16 ? 2 : 4;
   const size_t nseg_max = static_cast<size_t>(B) * (Hkv + Hq);
-  ctx->max_parts = (static_cast<size_t>(ctx->sms) + nseg_max) * kMaxQ;
+  ctx->max_parts = (2 * static_cast<size_t>(ctx->sms) + nseg_max) * kMaxQ;  // two pooling phases
   ctx->max_counters = nseg_max * kMaxQ;
   auto alloc = [&](void** p, size_t bytes) -> lyc_status {
     if (cudaMalloc(p, bytes) != cudaSuccess) {
@@ -670,7 +699,7 @@ lyc_status lyc_create(const lyc_config* cfg, lyc_ctx** out) {
   lyc_status st;
   if ((st = alloc(reinterpret_cast<void**>(&ctx->status), 16)) != LYC_OK ||
       (st = alloc(reinterpret_cast<void**>(&ctx->keys),
-                  static_cast<size_t>(B) * ctx->Hs * ctx->nstride * sizeof(float))) != LYC_OK ||
+                  2 * static_cast<size_t>(B) * ctx->Hs * ctx->nstride * sizeof(float))) != LYC_OK ||
       (st = alloc(reinterpret_cast<void**>(&ctx->sbuf),
                   2ull * B * ctx->Hs * ctx->KS * sizeof(int32_t) + 64)) != LYC_OK ||
       (st = alloc(reinterpret_cast<void**>(&ctx->part_o), ctx->max_parts * D * sizeof(float))) != LYC_OK ||

@@ -62,18 +62,24 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // Wait until the phase with `parity` of `bar` has completed.  Returns false
 // (and leaves the barrier alone) if the CTA's abort flag is set or the wait
 // exceeded kWaitLimitNs; in the latter case it sets the abort flag and the
-// timeout bit of the status word.
+// timeout bit of the status word.  The timer and the flag are looked at only
+// every 1024 polls: reading the global timer on every poll slows the wake-up.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                           uint32_t* status) {
   if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = global_timer_ns();
-  while (true) {
+  uint64_t t0 = 0;
+  for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (*abort_flag) return false;
-    if (global_timer_ns() - t0 > kWaitLimitNs) {
-      *abort_flag = 1;
-      atomicOr(status, kStatusTimeout);
-      return false;
+    if ((i & 1023u) == 0) {
+      if (*abort_flag) return false;
+      const uint64_t now = global_timer_ns();
+      if (t0 == 0) {
+        t0 = now;
+      } else if (now - t0 > kWaitLimitNs) {
+        *abort_flag = 1;
+        atomicOr(status, kStatusTimeout);
+        return false;
+      }
     }
   }
 }
@@ -114,6 +120,14 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
+
+// Programmatic dependent launch: let the next kernel in the stream start its
+// launch now / wait until the kernel this one depends on has completed and
+// its memory operations are visible (no-ops when launched without PDL).
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 // bf16 pair (packed in 32 bits, low element first) -> two floats, exactly.
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }

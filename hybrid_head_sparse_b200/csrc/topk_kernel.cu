@@ -172,6 +172,10 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster_kernel(const Top
   const int cnt = max(0, min(n, lo + chunk) - lo);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const unsigned lt = (1u << lane) - 1u;
+  // the keys are the attention kernel's output; only once it has completed
+  // may the next kernel (the next layer's attention) start its launch
+  pdl_wait();
+  pdl_launch_dependents();
 
   extern __shared__ __align__(16) unsigned char smem[];
   uint2* cand = reinterpret_cast<uint2*>(smem);        // [CAP] (encoded key, index) by source CTA
@@ -440,6 +444,9 @@ static cudaError_t topk_run(const TopkParams* p, int ntasks, cudaStream_t stream
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(max_smem));
     if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
     if (CL > 8) e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     return e;
   }
@@ -448,13 +455,15 @@ static cudaError_t topk_run(const TopkParams* p, int ntasks, cudaStream_t stream
   cfg.blockDim = dim3(kTopkThreads, 1, 1);
   cfg.dynamicSmemBytes = topk_smem_bytes(CL, p->n);
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = CL;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, kern, *p);
 }
 

@@ -502,51 +502,67 @@ __device__ __forceinline__ void mma_consumers(const AttnMmaParams& P, unsigned c
     named_bar_sync(1, NC * 32);
 
     // ---- the last piece of a segment combines every piece (log-sum-exp).
-    // All finished outputs at once: thread (o, c4) owns output o's columns
-    // 4*c4 .. 4*c4+3 and folds the partials in with a running maximum, eight
-    // partials' loads in flight at a time.
-    {
-      constexpr int C4 = D / 4;
-      for (int x = tid; x < nout * C4; x += NC * 32) {
-        const int o = x / C4, c4 = x % C4;
-        if (!lastflag[o]) continue;
-        const int base = sg.part_base + o;
-        const int np = sg.npieces;
-        float M = -INFINITY, L = 0.f;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int u0 = 0; u0 < np; u0 += 8) {
-          float2 ml[8];
-          float4 ov[8];
+    // Per finished output: warp w folds partials w, w+NC, ... with a running
+    // maximum, each lane owning four columns and eight partials' loads in
+    // flight at a time; the NC running states then merge in shared memory.
+    for (int o = 0; o < nout; ++o) {
+      if (!lastflag[o]) continue;  // the same in every thread
+      const int base = sg.part_base + o;
+      const int np = sg.npieces;
+      float M = -INFINITY, L = 0.f;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      const bool col = lane * 4 < D;
+      for (int u0 = w; u0 < np; u0 += 8 * NC) {
+        float2 ml[8];
+        float4 ov[8];
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const int part = base + min(u0 + j, np - 1) * nout;
-            ml[j] = __ldcg(&p.part_ml[part]);
-            ov[j] = __ldcg(reinterpret_cast<const float4*>(&p.part_o[static_cast<int64_t>(part) * D + 4 * c4]));
-          }
+        for (int j = 0; j < 8; ++j) {
+          const int part = base + min(u0 + j * NC, np - 1) * nout;
+          ml[j] = __ldcg(&p.part_ml[part]);
+          ov[j] = col ? __ldcg(reinterpret_cast<const float4*>(&p.part_o[static_cast<int64_t>(part) * D + lane * 4]))
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            if (u0 + j >= np || ml[j].x == -INFINITY) continue;
-            const float mn = fmaxf(M, ml[j].x);
-            const float a = (M == -INFINITY) ? 0.f : exp2f(M - mn);
-            const float f = exp2f(ml[j].x - mn);
-            L = L * a + f * ml[j].y;
-            acc.x = acc.x * a + f * ov[j].x;
-            acc.y = acc.y * a + f * ov[j].y;
-            acc.z = acc.z * a + f * ov[j].z;
-            acc.w = acc.w * a + f * ov[j].w;
-            M = mn;
+        for (int j = 0; j < 8; ++j) {
+          if (u0 + j * NC >= np || ml[j].x == -INFINITY) continue;
+          const float mn = fmaxf(M, ml[j].x);
+          const float a = (M == -INFINITY) ? 0.f : exp2f(M - mn);
+          const float f = exp2f(ml[j].x - mn);
+          L = L * a + f * ml[j].y;
+          acc.x = acc.x * a + f * ov[j].x;
+          acc.y = acc.y * a + f * ov[j].y;
+          acc.z = acc.z * a + f * ov[j].z;
+          acc.w = acc.w * a + f * ov[j].w;
+          M = mn;
+        }
+      }
+      if (lane == 0) mml[w] = make_float2(M, L);
+      if (col) *reinterpret_cast<float4*>(&mo[w * D + lane * 4]) = acc;
+      named_bar_sync(1, NC * 32);
+      for (int e = tid; e < D; e += NC * 32) {
+        float Mt = -INFINITY;
+#pragma unroll
+        for (int ww = 0; ww < NC; ++ww) Mt = fmaxf(Mt, mml[ww].x);
+        float Lt = 0.f, Ot = 0.f;
+        if (Mt != -INFINITY) {
+#pragma unroll
+          for (int ww = 0; ww < NC; ++ww) {
+            const float2 ml = mml[ww];
+            const float f = (ml.x == -INFINITY) ? 0.f : exp2f(ml.x - Mt);
+            Lt = fmaf(f, ml.y, Lt);
+            Ot = fmaf(f, mo[ww * D + e], Ot);
           }
         }
-        float4 res = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (L > 0.f) {
-          const float inv = 1.f / L;
-          res = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-        } else if (c4 == 0) {
+        float res = 0.f;
+        if (Lt > 0.f) {
+          res = Ot / Lt;
+        } else if (e == 0) {
           atomicOr(p.status, kStatusEmptySoftmax);
         }
-        *reinterpret_cast<float4*>(&p.out[(static_cast<int64_t>(b) * p.Hq + sg.head[sg.out_row[o]]) * D + 4 * c4]) = res;
-        if (c4 == 0) p.counters[sg.cnt_base + o] = 0;
+        p.out[(static_cast<int64_t>(b) * p.Hq + sg.head[sg.out_row[o]]) * D + e] = res;
       }
+      if (tid == 0) p.counters[sg.cnt_base + o] = 0;
+      named_bar_sync(1, NC * 32);  // mo / mml free again
     }
     named_bar_sync(1, NC * 32);  // merge area and flags free for the next piece
   }
@@ -557,6 +573,7 @@ template <int D, int NC, int NP, int STAGES>
 __global__ void __launch_bounds__(MmaCfg<D, NC, NP, STAGES>::kThreads, 1)
     attn_mma_layer_kernel(const __grid_constant__ AttnMmaParams P) {
   using C = MmaCfg<D, NC, NP, STAGES>;
+  const uint64_t t_start = P.p.timeline ? global_timer_ns() : 0;
   extern __shared__ unsigned char smem_raw[];
   // the 128B-swizzled TMA destination needs 1024-byte alignment
   unsigned char* smem = reinterpret_cast<unsigned char*>(
@@ -586,7 +603,11 @@ __global__ void __launch_bounds__(MmaCfg<D, NC, NP, STAGES>::kThreads, 1)
   }
   // this grid completes only after the one it depends on (dense-only CTAs
   // never waited above), so completion order follows launch order
-  if (threadIdx.x == 0) pdl_wait();
+  if (threadIdx.x == 0) {
+    pdl_wait();
+    timeline_record(P.p.timeline, P.p.timeline_cap, t_start,
+                    (kTagAttention << 32) | (static_cast<unsigned long long>(P.p.layer) << 16) | blockIdx.x);
+  }
 }
 
 // ---------------------------------------------------------------- host side

@@ -72,6 +72,8 @@ struct Plan {
   int32_t* S = nullptr;
   int32_t* trace = nullptr;
   bool timing = false;
+  unsigned long long* timeline = nullptr;
+  int timeline_cap = 0;
   CUtensorMap tmk{}, tmv{};       // bf16 path: 5-D maps of the whole K and V cache
   cudaGraphExec_t exec = nullptr;
   // timing: event-record nodes of the graph, in launch order (2 per kernel)
@@ -102,6 +104,8 @@ struct lyc_ctx {
   int32_t* trace = nullptr;
   cudaStream_t last_stream = nullptr;
   bool timing = false;
+  unsigned long long* timeline = nullptr;  // caller's buffer, or NULL
+  int timeline_cap = 0;
   // plans, most recent first
   std::list<std::pair<std::string, std::unique_ptr<Plan>>> plans;
   // timing pool
@@ -490,6 +494,9 @@ lyc_status enqueue_step(lyc_ctx* ctx, Plan* plan, cudaStream_t stream, int set, 
     ap.part_ml = ctx->part_ml;
     ap.counters = ctx->counters;
     ap.status = ctx->status;
+    ap.timeline = plan->timeline;
+    ap.timeline_cap = plan->timeline_cap;
+    ap.layer = l;
     ap.Hq = Hq;
     ap.G = ctx->G;
     ap.n = plan->n;
@@ -514,6 +521,9 @@ lyc_status enqueue_step(lyc_ctx* ctx, Plan* plan, cudaStream_t stream, int set, 
       tp.tasks = reinterpret_cast<const TopkTask*>(plan->dev + lp.off_tasks);
       tp.n = plan->n;
       tp.k = plan->k;
+      tp.timeline = plan->timeline;
+      tp.timeline_cap = plan->timeline_cap;
+      tp.layer = l;
       if ((st = record_event(ctx, plan, set, ev++, stream, capturing)) != LYC_OK) return st;
       LYC_CUDA(topk_launch(ctx->topk_cl, &tp, lp.ntasks, stream), "top-k launch");
       if ((st = record_event(ctx, plan, set, ev++, stream, capturing)) != LYC_OK) return st;
@@ -783,8 +793,9 @@ lyc_status lyc_decode_step(lyc_ctx* ctx, const void* q, const lyc_kv_cache* kv,
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
   const lyc_config& c = ctx->cfg;
 
-  const std::string key = plan_key(role_mask, c.num_layers, c.num_q_heads, kv, k, step_flags, q, out,
-                                   S, ctx->trace, ctx->timing);
+  std::string key = plan_key(role_mask, c.num_layers, c.num_q_heads, kv, k, step_flags, q, out, S,
+                             ctx->trace, ctx->timing);
+  key.append(reinterpret_cast<const char*>(&ctx->timeline), sizeof ctx->timeline);
   Plan* plan = nullptr;
   for (auto it = ctx->plans.begin(); it != ctx->plans.end(); ++it) {
     if (it->first == key) {
@@ -801,6 +812,8 @@ lyc_status lyc_decode_step(lyc_ctx* ctx, const void* q, const lyc_kv_cache* kv,
     np->S = S;
     np->trace = ctx->trace;
     np->timing = ctx->timing;
+    np->timeline = ctx->timeline;
+    np->timeline_cap = ctx->timeline_cap;
     st = build_plan(ctx, np.get(), role_mask, kv, k, step_flags);
     if (st != LYC_OK) {
       free_plan(np.get());
@@ -886,6 +899,13 @@ lyc_status lyc_sync_status(lyc_ctx* ctx) {
 lyc_status lyc_set_s_trace(lyc_ctx* ctx, int32_t* trace) {
   if (!ctx) return LYC_ERR_INVALID_ARG;
   ctx->trace = trace;
+  return LYC_OK;
+}
+
+lyc_status lyc_set_timeline(lyc_ctx* ctx, unsigned long long* buf, int cap) {
+  if (!ctx || (buf && cap < 1)) return LYC_ERR_INVALID_ARG;
+  ctx->timeline = buf;
+  ctx->timeline_cap = buf ? cap : 0;
   return LYC_OK;
 }
 

@@ -129,6 +129,18 @@ __device__ __forceinline__ void pdl_launch_dependents() {
 }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
+// One timeline record (CTA start, CTA end, tag) when a timeline buffer is set.
+__device__ __forceinline__ void timeline_record(unsigned long long* tl, int cap, uint64_t t_start,
+                                                unsigned long long tag) {
+  if (!tl) return;
+  const unsigned long long slot = atomicAdd(tl, 1ull);
+  if (slot < static_cast<unsigned long long>(cap)) {
+    tl[1 + 3 * slot] = t_start;
+    tl[2 + 3 * slot] = global_timer_ns();
+    tl[3 + 3 * slot] = tag;
+  }
+}
+
 // bf16 pair (packed in 32 bits, low element first) -> two floats, exactly.
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }

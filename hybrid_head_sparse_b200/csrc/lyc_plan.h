@@ -70,6 +70,9 @@ struct AttnParams {
   float2* part_ml;           // [parts] (running max in log2 units, sum)
   int32_t* counters;         // arrival counters, left at zero after use
   uint32_t* status;          // device status word
+  unsigned long long* timeline;  // NULL, or [1 + 3*cap]: count, then (start ns, end ns, tag)
+  int32_t timeline_cap;
+  int32_t layer;
   int32_t Hq, G, n;
   float scale_log2;          // log2(e) / sqrt(d)
   float scale;               // 1 / sqrt(d)
@@ -83,8 +86,15 @@ struct TopkTask {
 struct TopkParams {
   const TopkTask* tasks;  // one per blockIdx.y; NULL: use `single`
   TopkTask single;
+  unsigned long long* timeline;  // as in AttnParams
+  int32_t timeline_cap;
+  int32_t layer;
   int32_t n, k;
 };
+
+// Timeline tags: kind << 32 | layer << 16 | CTA
+constexpr unsigned long long kTagAttention = 0ull;
+constexpr unsigned long long kTagTopk = 1ull;
 
 // copy_sets_kernel: dst[(b*Hs + s)*k + j] = src[b*Hs + s][j] for j < k
 struct CopySetsParams {

@@ -172,6 +172,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster_kernel(const Top
   const int cnt = max(0, min(n, lo + chunk) - lo);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const unsigned lt = (1u << lane) - 1u;
+  const uint64_t t_start = p.timeline ? global_timer_ns() : 0;
   // the keys are the attention kernel's output; only once it has completed
   // may the next kernel (the next layer's attention) start its launch
   pdl_wait();
@@ -194,6 +195,10 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster_kernel(const Top
     for (int x = tid; x < cnt; x += kTopkThreads) task.S[lo + x] = lo + x;
     if (rank == 0)
       for (int x = keff + tid; x < k; x += kTopkThreads) task.S[x] = -1;
+    if (tid == 0)
+      timeline_record(p.timeline, p.timeline_cap, t_start,
+                      (kTagTopk << 32) | (static_cast<unsigned long long>(p.layer) << 16) |
+                          (blockIdx.y * CL + rank));
     return;
   }
 
@@ -426,6 +431,10 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster_kernel(const Top
   }
   if (rank == 0)
     for (int x = keff + tid; x < k; x += kTopkThreads) task.S[x] = -1;
+  if (tid == 0)
+    timeline_record(p.timeline, p.timeline_cap, t_start,
+                    (kTagTopk << 32) | (static_cast<unsigned long long>(p.layer) << 16) |
+                        (blockIdx.y * CL + rank));
   // no CTA leaves while another may still access its shared memory: every
   // remote access precedes the last cluster barrier on its path.
 }

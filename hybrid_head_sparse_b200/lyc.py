@@ -38,7 +38,8 @@ LYC_TIMING_ON = 1
 
 EXPORTED = ["lyc_create", "lyc_decode_step", "lyc_decode_step_host", "lyc_sync_status",
             "lyc_set_s_trace", "lyc_step_bytes", "lyc_topk_f32", "lyc_set_timing",
-            "lyc_kernel_times", "lyc_status_string", "lyc_last_error", "lyc_destroy"]
+            "lyc_kernel_times", "lyc_set_timeline", "lyc_status_string", "lyc_last_error",
+            "lyc_destroy"]
 
 
 class lyc_config(ctypes.Structure):
@@ -90,6 +91,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
                                  ctypes.POINTER(ctypes.c_uint64), ctypes.POINTER(ctypes.c_uint64)]
     L.lyc_topk_f32.argtypes = [P, P, ctypes.c_int64, I, P, P]
     L.lyc_set_timing.argtypes = [P, I]
+    L.lyc_set_timeline.argtypes = [P, P, I]
     L.lyc_kernel_times.argtypes = [P, ctypes.POINTER(lyc_kernel_time), I, ctypes.POINTER(I)]
     L.lyc_status_string.argtypes = [I]
     L.lyc_status_string.restype = ctypes.c_char_p
@@ -158,6 +160,10 @@ def lyc_kernel_times(ctx, cap: int = 1 << 16):
     if rc != LYC_OK:
         raise LycError(rc, "lyc_kernel_times")
     return [(arr[i].kind, arr[i].layer, arr[i].ms) for i in range(cnt.value)]
+
+
+def lyc_set_timeline(ctx, buf, cap: int) -> int:
+    return load().lyc_set_timeline(ctx, buf, cap)
 
 
 def lyc_status_string(code: int) -> str:
@@ -274,6 +280,12 @@ class Lyc:
 
     def kernel_times(self):
         return lyc_kernel_times(self.ctx)
+
+    def set_timeline(self, buf, cap: int):
+        """buf: device int64 tensor of 1 + 3*cap words (word 0 zeroed), or None."""
+        self._timeline = buf
+        self._check(lyc_set_timeline(self.ctx, None if buf is None else buf.data_ptr(), cap),
+                    "lyc_set_timeline")
 
     def topk_f32(self, keys, n, k, S, stream=None):
         self._check(lyc_topk_f32(self.ctx, keys.data_ptr(), n, k, S.data_ptr(),

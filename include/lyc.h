@@ -167,6 +167,14 @@ typedef struct {
 lyc_status lyc_set_timing(lyc_ctx* ctx, int mode);
 lyc_status lyc_kernel_times(lyc_ctx* ctx, lyc_kernel_time* times, int cap, int* count);
 
+/* Device timeline of the steps that follow: buf is device memory of
+ * 1 + 3*cap unsigned 64-bit words; the caller zeroes word 0.  Every CTA of the
+ * attention and selection kernels appends (start ns, end ns, tag) read from
+ * the GPU's global timer, tag = kind << 32 | layer << 16 | CTA (kind 0 =
+ * attention, 1 = selection); word 0 counts the records (records past cap are
+ * dropped).  NULL turns it off.  Profiling use. */
+lyc_status lyc_set_timeline(lyc_ctx* ctx, unsigned long long* buf, int cap);
+
 const char* lyc_status_string(lyc_status s);
 const char* lyc_last_error(const lyc_ctx* ctx);
 void lyc_destroy(lyc_ctx* ctx);

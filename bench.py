@@ -37,8 +37,8 @@ ATTN_SOURCES = ["attn_mma_kernel.cu", "lyc_plan.h", "lyc_device.cuh"]
 def parse_args(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["lyc", "reference"], default="lyc")
     ap.add_argument("--n", type=int, default=131072)
     ap.add_argument("--k", type=int, default=4096)
@@ -98,6 +98,33 @@ def profiled_traffic(workload: str):
             if rec.get("source_sha") == want and rec.get("workload") == workload:
                 return rec.get("bytes_per_launch")
     return None
+
+
+def max_over_ranks(x: float, device=None) -> float:
+    """The largest x over the ranks of the default process group (x itself
+    without one).  Every rank must call it at the same point."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_steps_per_s(world: int, steps: int, ms_slowest: float) -> float:
+    """Whole-job throughput of replicas: every rank ran `steps` steps and the
+    job took as long as its slowest rank."""
+    return world * steps / (ms_slowest / 1e3)
+
+
+def percentiles(xs):
+    xs = sorted(xs)
+
+    def q(f):
+        i = min(len(xs) - 1, max(0, int(round(f * (len(xs) - 1)))))
+        return xs[i]
+    return {"p10": q(0.10), "p50": q(0.50), "p90": q(0.90)}
 
 
 class ClockSampler:
@@ -184,12 +211,13 @@ def cpu_cores() -> int:
         return os.cpu_count() or 1
 
 
-def host_sample_stack(spec, data, cpu_layers: int):
+def host_sample_stack(spec, data, cpu_layers: int, select_mode: str = "per_qhead"):
     import oracle as O
     from hybrid_head_sparse_b200 import workloads as W
     layers = list(range(cpu_layers))
+    mode = O.SELECT_KVGROUP_MEAN if select_mode == "kvgroup_mean" else O.SELECT_PER_QHEAD
     return O.Stack(W.host_view(data["q"][layers]), W.host_view(data["k"][layers]),
-                   W.host_view(data["v"][layers]), data["role"][layers].copy(), O.SELECT_PER_QHEAD)
+                   W.host_view(data["v"][layers]), data["role"][layers].copy(), mode)
 
 
 def sample_text(spec, cpu_layers):
@@ -211,7 +239,7 @@ def run_reference(args):
     spec = workload_spec(args)
     cl = max(1, min(args.cpu_layers, spec.L))
     sample = W.make_stack(spec.with_(L=cl), "cpu")
-    st = host_sample_stack(spec, sample, cl)
+    st = host_sample_stack(spec, sample, cl, args.select_mode)
     for _ in range(args.warmup):
         oracle_sample_seconds(spec, st, cl)
     ests = []
@@ -229,7 +257,7 @@ def run_reference(args):
         "config": {"workload": spec.name, "L": spec.L, "B": spec.B, "Hq": spec.Hq,
                    "Hkv": spec.Hkv, "d": spec.d, "n": spec.n, "k": spec.k,
                    "retrieval_heads_per_layer": args.retrieval_heads,
-                   "select_mode": "per_qhead"},
+                   "select_mode": args.select_mode},
         "cpu_baseline": {"value": value, "unit": "steps/s", "cores": cores, "kind": "oracle",
                          "sample": sample_text(spec, cl) + "; inputs drawn on the host with the "
                          "same recipe"},
@@ -294,21 +322,19 @@ def run_lyc(args):
     ev1 = torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
     with ClockSampler(local) as clk:
-        ev0.record(stream)
-        for _ in range(args.steps):
+        evs[0].record(stream)
+        for i in range(args.steps):
             step()
-        ev1.record(stream)
+            evs[i + 1].record(stream)
         torch.cuda.synchronize()
     barrier()
     clocks = clk.summary()
-    ms_total = ev0.elapsed_time(ev1)
-    if world > 1:
-        t = torch.tensor([ms_total], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total = max_over_ranks(evs[0].elapsed_time(evs[-1]), dev)
+    step_ms = percentiles([evs[i].elapsed_time(evs[i + 1]) for i in range(args.steps)])
     ms_step = ms_total / args.steps
-    value = world * args.steps / (ms_total / 1e3)
+    value = job_steps_per_s(world, args.steps, ms_total)
     rc = ctx.sync_status()
     if rc != 0:
         raise RuntimeError(f"device status after timing: {lyc.lyc_status_string(rc)}")
@@ -369,12 +395,8 @@ def run_lyc(args):
             hstep()
         ev1.record(stream)
         torch.cuda.synchronize()
-        ms_e2e = ev0.elapsed_time(ev1)
-        if world > 1:
-            t = torch.tensor([ms_e2e], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms_e2e = float(t.item())
-        e2e = {"value": world * args.steps / (ms_e2e / 1e3), "unit": "steps/s",
+        ms_e2e = max_over_ranks(ev0.elapsed_time(ev1), dev)
+        e2e = {"value": job_steps_per_s(world, args.steps, ms_e2e), "unit": "steps/s",
                "h2d_bytes_per_step": q_h.numel() * q_h.element_size(),
                "d2h_bytes_per_step": out_h.numel() * 4 + S_h.numel() * 4,
                "note": "lyc_decode_step_host: q from pinned host memory in, outputs and sets back "
@@ -389,7 +411,7 @@ def run_lyc(args):
         import oracle as O
         O.build()
         cl = max(1, min(args.cpu_layers, spec.L))
-        st = host_sample_stack(spec, data, cl)
+        st = host_sample_stack(spec, data, cl, args.select_mode)
         est, times = oracle_sample_seconds(spec, st, cl)
         cpu = {"value": 1.0 / est, "unit": "steps/s", "cores": cpu_cores(), "kind": "oracle",
                "sample": sample_text(spec, cl) + f"; sampled layer seconds {[round(t, 3) for t in times]}"}
@@ -398,6 +420,7 @@ def run_lyc(args):
     line = {
         "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "step_ms_distribution": {k: round(v, 4) for k, v in step_ms.items()},
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic (seeded N(0,1) q/K/V, sinks + 256 planted heavy hitters per KV head)",
         "config": {"workload": spec.name, "L": spec.L, "B": spec.B, "Hq": spec.Hq,

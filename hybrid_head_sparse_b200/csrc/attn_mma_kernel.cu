@@ -47,13 +47,18 @@ typedef uint16_t bf16_t;  // bf16 bit pattern
 struct AttnMmaParams {
   CUtensorMap tmk;  // 5-D map of K: (d, row, g, b, l), box 64 x 64, 128B swizzle
   CUtensorMap tmv;  // same for V
+  CUtensorMap tgk;  // 2-D map of K: (d, flattened row), box 64 x 1, 128B swizzle (row gathers)
+  CUtensorMap tgv;  // same for V
   AttnParams p;
 };
 
-template <int D, int NC, int NP, int STAGES>
+template <int D, int NC, int NP, int STAGES, bool GT>
 struct MmaCfg {
   static constexpr int kThreads = (NC + NP) * 32;
   static constexpr int kProducerThreads = NP * 32;
+  // arrivals that complete a full barrier: with row gathers by TMA the one
+  // leader thread arms every tile; otherwise every producer thread arrives
+  static constexpr int kFullCount = GT ? 1 : NP * 32;
   static constexpr int HALVES = D / 64;                    // 128-byte column blocks per row
   static constexpr int BLOCKB = kTileRows * 128;           // one swizzled 64 x 128 B block
   static constexpr int TILEB = HALVES * BLOCKB;            // K (or V) tile bytes
@@ -119,6 +124,17 @@ __device__ __forceinline__ void tma_load_5d(void* dst, const CUtensorMap* map, i
       "r"(smem_u32(bar)), "l"(policy)
       : "memory");
 }
+// four rows (coordinates y0..y3 of a 2-D tensor map with a one-row box) at
+// column x, into 4 consecutive box rows at dst; rows outside the map read as zeros
+__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, int x, int4 y,
+                                            uint64_t* bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cta.global.tile::gather4.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%2, %3, %4, %5, %6}], [%7], %8;" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y.x), "r"(y.y), "r"(y.z), "r"(y.w),
+      "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
 // 16-byte global -> shared copy; src_bytes = 0 writes zeros and reads nothing
 __device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, uint32_t src_bytes) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
@@ -145,10 +161,10 @@ namespace lyc {
 // TMA copies, everyone arrives.  Gathered tile: warp pw copies rows
 // [pw*64/NP, (pw+1)*64/NP) with cp.async and every lane arrives when its own
 // copies have landed.
-template <int D, int NC, int NP, int STAGES>
+template <int D, int NC, int NP, int STAGES, bool GT>
 __device__ __forceinline__ void mma_producers(const AttnMmaParams& P, unsigned char* smem, int pbeg,
                                               int pend) {
-  using C = MmaCfg<D, NC, NP, STAGES>;
+  using C = MmaCfg<D, NC, NP, STAGES, GT>;
   const AttnParams& p = P.p;
   const int ptid = threadIdx.x - NC * 32;  // 0 .. NP*32-1
   const int pw = ptid >> 5;
@@ -162,6 +178,7 @@ __device__ __forceinline__ void mma_producers(const AttnMmaParams& P, unsigned c
   uint64_t* idxbar = bars + 2 * STAGES;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_FLAGS);
   const uint64_t pol = l2_policy_evict_first();
+  const uint64_t pol_keep = l2_policy_evict_normal();  // gathered rows may be read again
   const bool leader = ptid == 0;
 
   // lookahead cursor (leader only): index-list copies of gathered tiles, LA tiles early
@@ -222,9 +239,38 @@ __device__ __forceinline__ void mma_producers(const AttnMmaParams& P, unsigned c
             tma_load_5d(kdst + h * C::BLOCKB, &P.tmk, h * 64, r0, sgg, sb, sl, &full[stage], pol);
             tma_load_5d(vdst + h * C::BLOCKB, &P.tmv, h * 64, r0, sgg, sb, sl, &full[stage], pol);
           }
-        } else {
+        } else if (!GT) {
           mbar_arrive(&full[stage]);
         }
+      } else if (GT) {
+        // TMA row gathers: lane j < 16 brings K rows 4j .. 4j+3, lane 16 + j the
+        // same V rows, one 128-byte column block per copy.  Rows past the
+        // tile's end and out-of-range indices get a coordinate past the map,
+        // which reads as zeros (and is reported below, never followed).
+        const int slot = t % C::IR;
+        if (!mbar_wait(&idxbar[slot], (idx_phase >> slot) & 1u, abort_flag, p.status)) return;
+        idx_phase ^= 1u << slot;
+        if (leader) mbar_arrive_expect_tx(&full[stage], 2u * C::TILEB);
+        const int j = lane & 15;
+        const int4 ix = reinterpret_cast<const int4*>(idxring + slot * kTileRows)[j];
+        const int xs[4] = {ix.x, ix.y, ix.z, ix.w};
+        int ys[4];
+        bool bad = false;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const bool in_tile = 4 * j + e < nrows;
+          const bool ok = xs[e] >= 0 && xs[e] < p.n;
+          bad |= in_tile && !ok;
+          ys[e] = (in_tile && ok) ? sg.row_base + xs[e] : p.gather_rows;
+        }
+        if (bad) atomicOr(p.status, kStatusBadIndex);
+        const bool isv = lane >= 16;
+        unsigned char* dst = (isv ? vdst : kdst) + 4 * j * 128;
+        const CUtensorMap* map = isv ? &P.tgv : &P.tgk;
+#pragma unroll
+        for (int h = 0; h < C::HALVES; ++h)
+          tma_gather4(dst + h * C::BLOCKB, map, h * 64, make_int4(ys[0], ys[1], ys[2], ys[3]),
+                      &full[stage], pol_keep);
       } else {
         const int slot = t % C::IR;
         if (!mbar_wait(&idxbar[slot], (idx_phase >> slot) & 1u, abort_flag, p.status)) return;
@@ -266,10 +312,10 @@ namespace lyc {
 //                           oa[md][2..3] = cols 16md+g+8, queries 2c, 2c+1
 // so every lane owns queries q0 = 2c and q1 = 2c+1 in both, and the softmax
 // rescale needs no data movement.
-template <int D, int NC, int NP, int STAGES>
+template <int D, int NC, int NP, int STAGES, bool GT>
 __device__ __forceinline__ void mma_consumers(const AttnMmaParams& P, unsigned char* smem, int pbeg,
                                               int pend) {
-  using C = MmaCfg<D, NC, NP, STAGES>;
+  using C = MmaCfg<D, NC, NP, STAGES, GT>;
   constexpr unsigned FULL = 0xffffffffu;
   constexpr int KSTEPS = D / 16;   // q.K k-steps over d
   constexpr int MD = D / 16;       // O^T m-tiles
@@ -569,10 +615,10 @@ __device__ __forceinline__ void mma_consumers(const AttnMmaParams& P, unsigned c
 }
 
 // ---------------------------------------------------------------- kernel
-template <int D, int NC, int NP, int STAGES>
-__global__ void __launch_bounds__(MmaCfg<D, NC, NP, STAGES>::kThreads, 1)
+template <int D, int NC, int NP, int STAGES, bool GT>
+__global__ void __launch_bounds__(MmaCfg<D, NC, NP, STAGES, GT>::kThreads, 1)
     attn_mma_layer_kernel(const __grid_constant__ AttnMmaParams P) {
-  using C = MmaCfg<D, NC, NP, STAGES>;
+  using C = MmaCfg<D, NC, NP, STAGES, GT>;
   const uint64_t t_start = P.p.timeline ? global_timer_ns() : 0;
   extern __shared__ unsigned char smem_raw[];
   // the 128B-swizzled TMA destination needs 1024-byte alignment
@@ -581,7 +627,7 @@ __global__ void __launch_bounds__(MmaCfg<D, NC, NP, STAGES>::kThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&bars[s], C::kProducerThreads);  // full: every producer thread (+ TMA bytes)
+      mbar_init(&bars[s], C::kFullCount);  // full: arrivals + TMA bytes
       mbar_init(&bars[STAGES + s], 1);           // empty: the one warp that consumed the tile
     }
     for (int r = 0; r < C::IR; ++r) mbar_init(&bars[2 * STAGES + r], 1);
@@ -591,15 +637,19 @@ __global__ void __launch_bounds__(MmaCfg<D, NC, NP, STAGES>::kThreads, 1)
   if (threadIdx.x == NC * 32) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&P.tmk)) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&P.tmv)) : "memory");
+    if (GT) {
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&P.tgk)) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&P.tgv)) : "memory");
+    }
   }
   __syncthreads();
   pdl_launch_dependents();
   const int pbeg = P.p.cta_begin[blockIdx.x];
   const int pend = P.p.cta_begin[blockIdx.x + 1];
   if (threadIdx.x >= NC * 32) {
-    mma_producers<D, NC, NP, STAGES>(P, smem, pbeg, pend);
+    mma_producers<D, NC, NP, STAGES, GT>(P, smem, pbeg, pend);
   } else {
-    mma_consumers<D, NC, NP, STAGES>(P, smem, pbeg, pend);
+    mma_consumers<D, NC, NP, STAGES, GT>(P, smem, pbeg, pend);
   }
   // this grid completes only after the one it depends on (dense-only CTAs
   // never waited above), so completion order follows launch order
@@ -611,11 +661,11 @@ __global__ void __launch_bounds__(MmaCfg<D, NC, NP, STAGES>::kThreads, 1)
 }
 
 // ---------------------------------------------------------------- host side
-template <int D, int NC, int NP, int STAGES>
+template <int D, int NC, int NP, int STAGES, bool GT>
 static cudaError_t mma_run(const AttnMmaParams* P, int grid, cudaStream_t stream, int* smem_out,
                            bool configure_only) {
-  using C = MmaCfg<D, NC, NP, STAGES>;
-  auto kern = attn_mma_layer_kernel<D, NC, NP, STAGES>;
+  using C = MmaCfg<D, NC, NP, STAGES, GT>;
+  auto kern = attn_mma_layer_kernel<D, NC, NP, STAGES, GT>;
   if (configure_only) {
     if (smem_out) *smem_out = C::SMEM;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
@@ -642,8 +692,28 @@ static cudaError_t mma_run(const AttnMmaParams* P, int grid, cudaStream_t stream
 // bf16 inputs.  configure_only: set the shared-memory attribute, report the size.
 cudaError_t attn_mma_dispatch(int D, const AttnMmaParams* P, int grid, cudaStream_t stream,
                               int* smem_out, bool configure_only) {
-  if (D == 128) return mma_run<128, 3, 8, 6>(P, grid, stream, smem_out, configure_only);
-  if (D == 64) return mma_run<64, 4, 8, 8>(P, grid, stream, smem_out, configure_only);
+  // gathered rows by TMA (one producer warp) when the planner built the
+  // row-gather maps, else by cp.async from eight producer warps
+  if (configure_only) {
+    int s1 = 0, s2 = 0;
+    cudaError_t e = cudaErrorInvalidValue;
+    if (D == 128) {
+      e = mma_run<128, 6, 8, 6, false>(P, grid, stream, &s1, true);
+      if (e == cudaSuccess) e = mma_run<128, 6, 1, 6, true>(P, grid, stream, &s2, true);
+    } else if (D == 64) {
+      e = mma_run<64, 4, 8, 8, false>(P, grid, stream, &s1, true);
+      if (e == cudaSuccess) e = mma_run<64, 4, 1, 8, true>(P, grid, stream, &s2, true);
+    }
+    if (smem_out) *smem_out = s1 > s2 ? s1 : s2;
+    return e;
+  }
+  const bool gt = P->p.gather_rows > 0;
+  if (D == 128)
+    return gt ? mma_run<128, 6, 1, 6, true>(P, grid, stream, smem_out, false)
+              : mma_run<128, 6, 8, 6, false>(P, grid, stream, smem_out, false);
+  if (D == 64)
+    return gt ? mma_run<64, 4, 1, 8, true>(P, grid, stream, smem_out, false)
+              : mma_run<64, 4, 8, 8, false>(P, grid, stream, smem_out, false);
   return cudaErrorInvalidValue;
 }
 

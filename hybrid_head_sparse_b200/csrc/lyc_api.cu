@@ -26,6 +26,8 @@ namespace lyc {
 struct AttnMmaParams {
   CUtensorMap tmk;
   CUtensorMap tmv;
+  CUtensorMap tgk;
+  CUtensorMap tgv;
   AttnParams p;
 };
 int attn_nq_bucket(int nq);
@@ -75,6 +77,8 @@ struct Plan {
   unsigned long long* timeline = nullptr;
   int timeline_cap = 0;
   CUtensorMap tmk{}, tmv{};       // bf16 path: 5-D maps of the whole K and V cache
+  CUtensorMap tgk{}, tgv{};       // bf16 path: 2-D row-gather maps (when gather_rows > 0)
+  int32_t gather_rows = 0;        // rows of the row-gather maps; 0 = none
   cudaGraphExec_t exec = nullptr;
   // timing: event-record nodes of the graph, in launch order (2 per kernel)
   std::vector<cudaGraphNode_t> ev_nodes;
@@ -194,6 +198,43 @@ lyc_status encode_cache_map(lyc_ctx* ctx, CUtensorMap* map, const void* base, co
   return LYC_OK;
 }
 
+// Rows of a flattened 2-D view (d, row) of the cache in which row
+// (l*s_layer + b*s_batch + g*s_head)/s_token + i is token i of (l, b, g), or 0
+// when the strides do not allow one (a head, batch or layer stride that is
+// not a whole number of rows) or the rows do not fit a 32-bit coordinate.
+int64_t gather_map_rows(const lyc_config& c, const lyc_kv_cache* kv) {
+  const int64_t st = kv->s_token;
+  if (st <= 0) return 0;
+  if ((c.num_kv_heads > 1 && kv->s_head % st) || (c.batch > 1 && kv->s_batch % st) ||
+      (c.num_layers > 1 && kv->s_layer % st))
+    return 0;
+  if (kv->s_head < 0 || kv->s_batch < 0 || kv->s_layer < 0) return 0;
+  const int64_t last = (c.num_layers - 1) * kv->s_layer + (c.batch - 1) * kv->s_batch +
+                       (c.num_kv_heads - 1) * kv->s_head;
+  const int64_t rows = last / st + kv->n;
+  return rows < 0x7fffffffll ? rows : 0;
+}
+
+// The 2-D row-gather map of one cache tensor: boxes of one 128-byte row
+// (64 bf16), 128B swizzle, so that a four-row gather lands in the same
+// swizzled tile layout as the 5-D map's tiles.
+lyc_status encode_gather_map(lyc_ctx* ctx, CUtensorMap* map, const void* base, const lyc_kv_cache* kv,
+                             int64_t rows) {
+  EncodeTiledFn fn = encode_tiled_fn();
+  if (!fn) return fail(ctx, LYC_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(ctx->cfg.head_dim), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kv->s_token * 2)};
+  const cuuint32_t box[2] = {64, 1};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(ctx, LYC_ERR_INVALID_ARG, "cuTensorMapEncodeTiled rejected the row-gather view (code " +
+                                              std::to_string(static_cast<int>(r)) + ")");
+  return LYC_OK;
+}
+
 // ---------------------------------------------------------------- planner
 //
 // Builds every layer's work pool for one (role mask, n, k, flags, pointers)
@@ -215,10 +256,18 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const lyc_k
   plan->keff = keff;
   plan->n = n;
   plan->nsets = B * Hs;
+  plan->gather_rows = 0;
   if (cfg.dtype == LYC_BF16) {
     lyc_status st = encode_cache_map(ctx, &plan->tmk, kv->k, kv);
     if (st == LYC_OK) st = encode_cache_map(ctx, &plan->tmv, kv->v, kv);
     if (st != LYC_OK) return st;
+    const int64_t rows = (cfg.flags & LYC_CFG_TMA_GATHER) ? gather_map_rows(cfg, kv) : 0;
+    if (rows > 0) {
+      st = encode_gather_map(ctx, &plan->tgk, kv->k, kv, rows);
+      if (st == LYC_OK) st = encode_gather_map(ctx, &plan->tgv, kv->v, kv, rows);
+      if (st != LYC_OK) return st;
+      plan->gather_rows = static_cast<int32_t>(rows);
+    }
   }
 
   struct HostLayer {
@@ -256,6 +305,7 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const lyc_k
         base.k = kbase + off * es;
         base.v = vbase + off * es;
         base.s_token = kv->s_token;
+        base.row_base = plan->gather_rows > 0 ? static_cast<int32_t>(off / kv->s_token) : 0;
         base.l = l;
         base.b = b;
         base.g = g;
@@ -508,7 +558,10 @@ lyc_status enqueue_step(lyc_ctx* ctx, Plan* plan, cudaStream_t stream, int set, 
       AttnMmaParams mp;
       mp.tmk = plan->tmk;
       mp.tmv = plan->tmv;
+      mp.tgk = plan->tgk;
+      mp.tgv = plan->tgv;
       mp.p = ap;
+      mp.p.gather_rows = plan->gather_rows;
       LYC_CUDA(attn_mma_dispatch(D, &mp, lp.grid, stream, nullptr, false), "attention launch");
     } else {
       LYC_CUDA(attn_simt_dispatch(D, lp.nqb, &ap, lp.grid, stream, nullptr, false), "attention launch");
@@ -672,7 +725,8 @@ lyc_status lyc_create(const lyc_config* cfg, lyc_ctx** out) {
   *out = nullptr;
   const lyc_config& c = *cfg;
   if (c.num_layers < 1 || c.batch < 1 || c.num_q_heads < 1 || c.num_kv_heads < 1 ||
-      c.num_q_heads % c.num_kv_heads != 0 || c.max_ctx < 1 || c.max_k < 1 || c.flags != 0)
+      c.num_q_heads % c.num_kv_heads != 0 || c.max_ctx < 1 || c.max_k < 1 ||
+      (c.flags & ~LYC_CFG_TMA_GATHER) != 0)
     return LYC_ERR_INVALID_ARG;
   if (c.dtype != LYC_BF16 && c.dtype != LYC_FP32) return LYC_ERR_INVALID_ARG;
   if (c.select_mode != LYC_SELECT_PER_QHEAD && c.select_mode != LYC_SELECT_KVGROUP_MEAN)

@@ -50,7 +50,7 @@ struct Segment {
   int32_t part_base;    // first partial record of this segment
   int32_t npieces;      // pieces the segment was cut into
   int32_t cnt_base;     // first arrival counter of this segment (nout counters)
-  int32_t pad_;
+  int32_t row_base;     // row of (l, b, g, token 0) in the flattened row-gather map
 };
 
 struct Piece {
@@ -74,6 +74,9 @@ struct AttnParams {
   int32_t timeline_cap;
   int32_t layer;
   int32_t Hq, G, n;
+  int32_t gather_rows;       // rows of the flattened row-gather maps (an index past
+                             // the last row, used for rows that must read as zeros);
+                             // 0: no such maps, gathered rows come by cp.async
   float scale_log2;          // log2(e) / sqrt(d)
   float scale;               // 1 / sqrt(d)
 };

@@ -29,6 +29,8 @@ LYC_FP32 = 1
 LYC_SELECT_PER_QHEAD = 0
 LYC_SELECT_KVGROUP_MEAN = 1
 
+LYC_CFG_TMA_GATHER = 0x1
+
 LYC_STEP_S_IN = 0x1
 LYC_STEP_NO_GRAPH = 0x2
 LYC_STEP_VALIDATE_S = 0x4
@@ -216,9 +218,9 @@ class Lyc:
     """One library context.  Tensors are passed by device pointer."""
 
     def __init__(self, L, B, Hq, Hkv, d, max_ctx, max_k, dtype="bf16", select_mode="per_qhead",
-                 device=0):
+                 device=0, flags=0):
         self.cfg = lyc_config(L, B, Hq, Hkv, d, max_ctx, max_k, _dtype_code(dtype),
-                              _mode_code(select_mode), device, 0)
+                              _mode_code(select_mode), device, flags)
         self.ctx = lyc_create(self.cfg)
         self.Hs = Hkv if self.cfg.select_mode == LYC_SELECT_KVGROUP_MEAN else Hq
         self._trace = None

@@ -69,8 +69,18 @@ typedef struct {
   lyc_dtype dtype;  /* element type of q, K and V */
   lyc_select_mode select_mode;
   int device;       /* CUDA device ordinal */
-  uint32_t flags;   /* reserved, pass 0 */
+  uint32_t flags;   /* 0, or LYC_CFG_* bits below */
 } lyc_config;
+
+/* cfg.flags: gather the inherited K/V rows with TMA four-row gathers
+ * (cp.async.bulk.tensor ... tile::gather4, one producer warp) instead of
+ * 16-byte cp.async copies from eight producer warps.  Measured on B200 the
+ * TMA form lands a gathered tile several times later than cp.async, so it is
+ * off by default; it is kept for comparison.  It needs a flattened row view of
+ * the cache (head, batch and layer strides that are whole multiples of
+ * s_token, under 2^31 rows); without one the library uses cp.async anyway.
+ * Results are the same either way. */
+#define LYC_CFG_TMA_GATHER 0x1u
 
 /* The KV cache of all layers.  Element (l, b, g, i, j) of K (and of V) is at
  * element offset l*s_layer + b*s_batch + g*s_head + i*s_token + j, j < d

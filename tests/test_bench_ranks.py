@@ -1,0 +1,72 @@
+"""Multi-rank logic of bench.py on CPU: two gloo ranks stand in for two GPUs.
+
+The step has no exchange between replicas, so the only cross-rank work is the
+timing reduction: every rank times its own K steps, the job time is the
+slowest rank's, and the whole-job value counts every rank's steps.
+"""
+import multiprocessing as mp
+import os
+import socket
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, ms, steps, q):
+    import torch.distributed as dist
+    import bench
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    from datetime import timedelta
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
+    try:
+        slow = bench.max_over_ranks(ms[rank])
+        q.put((rank, slow, bench.job_steps_per_s(world, steps, slow)))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_gloo_two_ranks():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    ms = [12.5, 20.0]
+    steps = 10
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, ms, steps, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    got = [q.get(timeout=120) for _ in procs]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, slow, value in got:
+        assert slow == 20.0                       # the slowest rank's time, on every rank
+        assert value == pytest.approx(2 * steps / 0.020)  # all ranks' steps / that time
+
+
+def test_single_process_needs_no_group():
+    import bench
+    assert bench.max_over_ranks(3.25) == 3.25
+    assert bench.job_steps_per_s(1, 50, 100.0) == pytest.approx(500.0)
+
+
+def test_reference_arm_only_rank0_works(monkeypatch, capsys):
+    import bench
+    monkeypatch.setenv("RANK", "1")
+    args = bench.parse_args(["--impl", "reference", "--gpus", "2"])
+    assert bench.run_reference(args) == 0
+    assert capsys.readouterr().out == ""          # ranks other than 0 print nothing
+
+
+def test_percentiles():
+    import bench
+    p = bench.percentiles([5.0, 1.0, 3.0, 2.0, 4.0])
+    assert (p["p10"], p["p50"], p["p90"]) == (1.0, 3.0, 5.0)

@@ -20,14 +20,19 @@ def lyc():
     return lycmod
 
 
+GATHERS = ["cp_async", "tma"]
+
+
 def run_step(lyc, spec: W.StackSpec, select_mode="per_qhead", data=None, s_in=None,
-             no_graph=False, k=None, n=None):
-    """One library step on the spec's inputs; returns (data, out, S, trace) on the host."""
+             no_graph=False, k=None, n=None, gather="cp_async"):
+    """One library step on the spec's inputs; returns (data, out, S, trace) on the host.
+    gather: "cp_async" (the default) or "tma" (four-row TMA gathers where the layout allows)."""
     data = data or W.make_stack(spec, "cuda")
     k = k or spec.k
     n = n or spec.n
+    flags = lyc.LYC_CFG_TMA_GATHER if gather == "tma" else 0
     ctx = lyc.Lyc(spec.L, spec.B, spec.Hq, spec.Hkv, spec.d, max(spec.rows, n), k,
-                  dtype=spec.dtype, select_mode=select_mode)
+                  dtype=spec.dtype, select_mode=select_mode, flags=flags)
     Hs = ctx.Hs
     out = torch.full((spec.L, spec.B, spec.Hq, spec.d), float("nan"), device="cuda")
     S = torch.full((spec.B, Hs, k), -7, dtype=torch.int32, device="cuda")
@@ -103,11 +108,12 @@ SMALL_BF16 = W.StackSpec("small-llama-like", L=4, B=2, Hq=32, Hkv=8, d=128, n=30
                          retrieval_per_layer=3, n_planted=64, seed=5)
 
 
+@pytest.mark.parametrize("gather", GATHERS)
 @pytest.mark.parametrize("mode", ["per_qhead", "kvgroup_mean"])
-def test_small_bf16_stack(lyc, mode):
+def test_small_bf16_stack(lyc, mode, gather):
     spec = SMALL_BF16
     om = O.SELECT_PER_QHEAD if mode == "per_qhead" else O.SELECT_KVGROUP_MEAN
-    data, out, S, tr = run_step(lyc, spec, select_mode=mode)
+    data, out, S, tr = run_step(lyc, spec, select_mode=mode, gather=gather)
     P.check_layers(data, out, tr, spec.k, spec.n, "bf16", range(spec.L), select_mode=om)
     assert np.array_equal(S, tr[-1])
 
@@ -148,8 +154,9 @@ def test_k_ge_n_sparse_equals_dense(lyc):
     assert np.array_equal(S[0, 1], np.arange(90))
 
 
+@pytest.mark.parametrize("gather", GATHERS)
 @pytest.mark.parametrize("pattern", ["blocks", "scattered"])
-def test_set_input_single_layer(lyc, pattern):
+def test_set_input_single_layer(lyc, pattern, gather):
     """One layer with inherited sets given (the single-layer kernel sweep form)."""
     spec = W.StackSpec("one-layer", L=1, B=2, Hq=32, Hkv=8, d=128, n=16384, k=1024,
                        planted="heavy", n_planted=64, seed=8)
@@ -158,8 +165,61 @@ def test_set_input_single_layer(lyc, pattern):
     role[0, [3, 17]] = 1
     data["role"] = role
     S0 = W.inherited_sets(spec.B, spec.Hq, spec.n, spec.k, pattern, seed=1, device="cuda")
-    _, out, S, tr = run_step(lyc, spec, data=data, s_in=S0)
+    _, out, S, tr = run_step(lyc, spec, data=data, s_in=S0, gather=gather)
     P.check_layers(data, out, tr, spec.k, spec.n, "bf16", [0], S0=S0.cpu().numpy())
+
+
+@pytest.mark.parametrize("gather", GATHERS)
+def test_ragged_sets_bf16(lyc, gather):
+    """k not a multiple of the 64-row tile nor of the four-row gather: the
+    last tile of every gathered segment is partial."""
+    spec = W.StackSpec("ragged", L=3, B=1, Hq=8, Hkv=2, d=128, n=2000, k=199,
+                       retrieval_per_layer=2, planted="heavy", n_planted=16, seed=11)
+    data, out, S, tr = run_step(lyc, spec, gather=gather)
+    P.check_layers(data, out, tr, spec.k, spec.n, "bf16", range(spec.L))
+
+
+def test_head_stride_not_whole_rows_falls_back(lyc):
+    """A KV-head stride that is not a whole number of rows has no flattened
+    row view: asked for TMA gathers, the library gathers with cp.async and the
+    result is the same."""
+    spec = W.StackSpec("odd-head-stride", L=2, B=1, Hq=8, Hkv=2, d=128, n=600, k=100,
+                       retrieval_per_layer=2, planted="none", seed=12)
+    data = W.make_stack(spec, "cuda")
+    L, B, Hkv, n, d = 2, 1, 2, 600, 128
+    s_token, s_head = d, n * d + 64          # 128 bytes between heads: not a whole row
+    s_batch = Hkv * s_head
+    s_layer = B * s_batch
+
+    def restride(t):
+        flat = torch.zeros(L * s_layer + 64, dtype=t.dtype, device="cuda")
+        v = flat.as_strided((L, B, Hkv, n, d), (s_layer, s_batch, s_head, s_token, 1))
+        v.copy_(t)
+        return v
+    odd = dict(data)
+    odd["k"], odd["v"] = restride(data["k"]), restride(data["v"])
+    _, out, S, tr = run_step(lyc, spec, data=odd, gather="tma")
+    P.check_layers(data, out, tr, spec.k, spec.n, "bf16", range(spec.L))
+
+
+@pytest.mark.parametrize("gather", GATHERS)
+def test_bad_inherited_index_reported_bf16(lyc, gather):
+    spec = W.StackSpec("bad16", L=1, B=1, Hq=2, Hkv=1, d=128, n=300, k=70, planted="none")
+    data = W.make_stack(spec, "cuda")
+    data["role"] = np.array([[1, 0]], dtype=np.uint8)
+    S0 = torch.arange(70, dtype=torch.int32, device="cuda").repeat(1, 2, 1).contiguous()
+    flags = lyc.LYC_CFG_TMA_GATHER if gather == "tma" else 0
+    ctx = lyc.Lyc(1, 1, 2, 1, 128, 300, 70, flags=flags)
+    out = torch.zeros((1, 1, 2, 128), device="cuda")
+    for bad in (300, -3):
+        S = S0.clone()
+        S[0, 1, 66] = bad
+        ctx.decode_step(data["q"], data["k"], data["v"], 300, data["role"], 70, out, S, s_in=True)
+        assert ctx.sync_status() == lyc.LYC_ERR_BAD_INDEX
+    S = S0.clone()
+    ctx.decode_step(data["q"], data["k"], data["v"], 300, data["role"], 70, out, S, s_in=True)
+    assert ctx.sync_status() == 0
+    ctx.close()
 
 
 def test_bad_inherited_index_reported(lyc):
@@ -235,6 +295,22 @@ def test_strided_rows(lyc):
     strided["v"] = Vp[..., :64]
     _, out, S, tr = run_step(lyc, spec, data=strided)
     P.check_layers(data, out, tr, spec.k, spec.n, "fp32", range(spec.L))
+
+
+@pytest.mark.parametrize("gather", GATHERS)
+def test_strided_rows_bf16(lyc, gather):
+    """bf16 rows padded to 136 elements (272-byte token stride): the tensor
+    maps and the row gathers follow the stride."""
+    spec = W.StackSpec("strided16", L=3, B=2, Hq=8, Hkv=2, d=128, n=777, k=130,
+                       retrieval_per_layer=2, planted="heavy", n_planted=8, seed=13)
+    data = W.make_stack(spec, "cuda")
+    pad = dict(data)
+    for name, fill in (("k", 3.0), ("v", -3.0)):
+        t = torch.full((3, 2, 2, 777, 136), fill, dtype=torch.bfloat16, device="cuda")
+        t[..., :128] = data[name]
+        pad[name] = t[..., :128]
+    _, out, S, tr = run_step(lyc, spec, data=pad, gather=gather)
+    P.check_layers(data, out, tr, spec.k, spec.n, "bf16", range(spec.L))
 
 
 # ---------------------------------------------------------------- full-size workloads

@@ -54,8 +54,10 @@ struct AttnMmaParams {
 
 template <int D, int NC, int NP, int STAGES, bool GT>
 struct MmaCfg {
-  static constexpr int kThreads = (NC + NP) * 32;
+  // warps: NC consumers, one epilogue warp, NP producers
+  static constexpr int kThreads = (NC + 1 + NP) * 32;
   static constexpr int kProducerThreads = NP * 32;
+  static constexpr int kFirstProducer = (NC + 1) * 32;  // thread index
   // arrivals that complete a full barrier: with row gathers by TMA the one
   // leader thread arms every tile; otherwise every producer thread arrives
   static constexpr int kFullCount = GT ? 1 : NP * 32;
@@ -72,15 +74,15 @@ struct MmaCfg {
   // t - STAGES (the stage's previous phase) is already consumed and the
   // parity wait cannot match a phase that has not started.
   static_assert(STAGES % NC == 0, "each stage must belong to one consumer warp");
+  static_assert(NC <= kMaxConsumerWarps, "piece-state ring sized for kMaxConsumerWarps");
   // shared memory (bytes from a 1024-aligned base)
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = OFF_K + STAGES * TILEB;
   static constexpr int OFF_IDX = OFF_V + STAGES * TILEB;
-  static constexpr int OFF_MO = OFF_IDX + IR * kTileRows * 4;
-  static constexpr int OFF_MML = OFF_MO + NC * 8 * D * 4;
-  static constexpr int OFF_BAR = OFF_MML + NC * 8 * 8;
-  static constexpr int OFF_FLAGS = OFF_BAR + (2 * STAGES + IR) * 8;
-  static constexpr int SMEM = OFF_FLAGS + (kMaxQ + 2) * 4 + 1024;  // + alignment slack
+  static constexpr int OFF_BAR = OFF_IDX + IR * kTileRows * 4;
+  // barriers: full[STAGES], empty[STAGES], idx[IR], slot_full[PS], slot_free[PS]
+  static constexpr int OFF_FLAGS = OFF_BAR + (2 * STAGES + IR + 2 * kPartSlots) * 8;
+  static constexpr int SMEM = OFF_FLAGS + 16 + 1024;  // + alignment slack
 };
 
 // ---------------------------------------------------------------- PTX helpers
@@ -166,7 +168,7 @@ __device__ __forceinline__ void mma_producers(const AttnMmaParams& P, unsigned c
                                               int pend) {
   using C = MmaCfg<D, NC, NP, STAGES, GT>;
   const AttnParams& p = P.p;
-  const int ptid = threadIdx.x - NC * 32;  // 0 .. NP*32-1
+  const int ptid = threadIdx.x - C::kFirstProducer;  // 0 .. NP*32-1
   const int pw = ptid >> 5;
   const int lane = ptid & 31;
   unsigned char* Ks = smem + C::OFF_K;
@@ -329,13 +331,12 @@ __device__ __forceinline__ void mma_consumers(const AttnMmaParams& P, unsigned c
   const uint32_t ksm = smem_u32(smem + C::OFF_K);
   const uint32_t vsm = smem_u32(smem + C::OFF_V);
   const int32_t* idxring = reinterpret_cast<const int32_t*>(smem + C::OFF_IDX);
-  float* mo = reinterpret_cast<float*>(smem + C::OFF_MO);
-  float2* mml = reinterpret_cast<float2*>(smem + C::OFF_MML);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* full = bars;
   uint64_t* empty = bars + STAGES;
+  uint64_t* slot_full = bars + 2 * STAGES + C::IR;
+  uint64_t* slot_free = slot_full + kPartSlots;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_FLAGS);
-  int* lastflag = reinterpret_cast<int*>(smem + C::OFF_FLAGS) + 1;
   const bf16_t* q = static_cast<const bf16_t*>(p.q);
   const float sl2 = p.scale_log2;
   const int mi = lane >> 3, r8 = lane & 7;  // ldmatrix: matrix and row this lane addresses
@@ -496,85 +497,133 @@ __device__ __forceinline__ void mma_consumers(const AttnMmaParams& P, unsigned c
       if (lane == 0) mbar_arrive(&empty[stage]);
     }
 
-    // ---- merge the NC warps' states of this piece into one partial record per output
+    // ---- hand this warp's state of the piece to the epilogue warp: slot
+    // (piece % kPartSlots) of this CTA's ring, rows that produce an output
     {
 #pragma unroll
-      for (int s = 4; s <= 16; s <<= 1) {
-        l0 += __shfl_xor_sync(FULL, l0, s);
-        l1 += __shfl_xor_sync(FULL, l1, s);
+      for (int s2 = 4; s2 <= 16; s2 <<= 1) {
+        l0 += __shfl_xor_sync(FULL, l0, s2);
+        l1 += __shfl_xor_sync(FULL, l1, s2);
       }
+      const int pi = pcI - pbeg;
+      const int slot = pi % kPartSlots;
+      if (pi >= kPartSlots)
+        mbar_wait(&slot_free[slot], ((pi / kPartSlots) - 1) & 1, abort_flag, p.status);
+      const int64_t rec = ((static_cast<int64_t>(blockIdx.x) * kPartSlots + slot) * NC + w) * kMaxQ;
       if (g == 0) {
-        mml[w * 8 + q0] = make_float2(m0, l0);
-        mml[w * 8 + q1] = make_float2(m1, l1);
+        if (out0) p.wpart_ml[rec + q0] = make_float2(m0, l0);
+        if (out1) p.wpart_ml[rec + q1] = make_float2(m1, l1);
       }
+      float* o0 = p.wpart_o + (rec + q0) * D;
+      float* o1 = p.wpart_o + (rec + q1) * D;
 #pragma unroll
       for (int md = 0; md < MD; ++md) {
-        mo[(w * 8 + q0) * D + 16 * md + g] = oa[md][0];
-        mo[(w * 8 + q1) * D + 16 * md + g] = oa[md][1];
-        mo[(w * 8 + q0) * D + 16 * md + g + 8] = oa[md][2];
-        mo[(w * 8 + q1) * D + 16 * md + g + 8] = oa[md][3];
+        if (out0) {
+          o0[16 * md + g] = oa[md][0];
+          o0[16 * md + g + 8] = oa[md][2];
+        }
+        if (out1) {
+          o1[16 * md + g] = oa[md][1];
+          o1[16 * md + g + 8] = oa[md][3];
+        }
       }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&slot_full[slot]);  // release: the writes above
     }
-    named_bar_sync(1, NC * 32);
-    for (int x = tid; x < nout * D; x += NC * 32) {
-      const int o = x / D, e = x % D;
+  }
+}
+
+// ---------------------------------------------------------------- epilogue warp
+// Takes the pieces in the CTA's order.  For each: waits for the NC consumer
+// warps' states, merges them (log-sum-exp) into the piece's partial record,
+// frees the slot, counts the arrival; the last piece of a segment to arrive
+// combines every piece's partial into the output (Appendix C, Algorithm 2,
+// steps 5-6).  The consumers never wait for this work unless they run
+// kPartSlots pieces ahead.  Lane j owns columns 4j .. 4j+3.
+template <int D, int NC, int NP, int STAGES, bool GT>
+__device__ __forceinline__ void mma_epilogue(const AttnMmaParams& P, unsigned char* smem, int pbeg,
+                                             int pend) {
+  using C = MmaCfg<D, NC, NP, STAGES, GT>;
+  constexpr unsigned FULL = 0xffffffffu;
+  const AttnParams& p = P.p;
+  const int lane = threadIdx.x & 31;
+  const bool col = lane * 4 < D;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* slot_full = bars + 2 * STAGES + C::IR;
+  uint64_t* slot_free = slot_full + kPartSlots;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_FLAGS);
+  for (int pcI = pbeg; pcI < pend; ++pcI) {
+    const Piece pc = p.pieces[pcI];
+    const Segment& sg = p.segs[pc.seg];
+    const int nout = sg.nout, b = sg.b;
+    const int pi = pcI - pbeg;
+    const int slot = pi % kPartSlots;
+    if (!mbar_wait(&slot_full[slot], (pi / kPartSlots) & 1, abort_flag, p.status)) return;
+    const int64_t rec0 = (static_cast<int64_t>(blockIdx.x) * kPartSlots + slot) * NC * kMaxQ;
+    for (int o = 0; o < nout; ++o) {
       const int r = sg.out_row[o];
+      float2 ml[NC];
+      float4 ov[NC];
+#pragma unroll
+      for (int ww = 0; ww < NC; ++ww) {
+        ml[ww] = p.wpart_ml[rec0 + ww * kMaxQ + r];
+        ov[ww] = col ? *reinterpret_cast<const float4*>(p.wpart_o + (rec0 + ww * kMaxQ + r) * D + lane * 4)
+                     : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
       float M = -INFINITY;
 #pragma unroll
-      for (int ww = 0; ww < NC; ++ww) M = fmaxf(M, mml[ww * 8 + r].x);
-      float L = 0.f, O = 0.f;
+      for (int ww = 0; ww < NC; ++ww) M = fmaxf(M, ml[ww].x);
+      float Lr = 0.f;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
       if (M != -INFINITY) {
 #pragma unroll
         for (int ww = 0; ww < NC; ++ww) {
-          const float2 ml = mml[ww * 8 + r];
-          const float f = (ml.x == -INFINITY) ? 0.f : exp2f(ml.x - M);
-          L = fmaf(f, ml.y, L);
-          O = fmaf(f, mo[(ww * 8 + r) * D + e], O);
+          const float f = (ml[ww].x == -INFINITY) ? 0.f : exp2f(ml[ww].x - M);
+          Lr = fmaf(f, ml[ww].y, Lr);
+          acc.x = fmaf(f, ov[ww].x, acc.x);
+          acc.y = fmaf(f, ov[ww].y, acc.y);
+          acc.z = fmaf(f, ov[ww].z, acc.z);
+          acc.w = fmaf(f, ov[ww].w, acc.w);
         }
       }
       const int part = sg.part_base + pc.ordinal * nout + o;
-      p.part_o[static_cast<int64_t>(part) * D + e] = O;
-      if (e == 0) p.part_ml[part] = make_float2(M, L);
+      if (col) *reinterpret_cast<float4*>(&p.part_o[static_cast<int64_t>(part) * D + lane * 4]) = acc;
+      if (lane == 0) p.part_ml[part] = make_float2(M, Lr);
     }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&slot_free[slot]);  // the consumers may reuse the slot
+    // publish the partials, then count this piece's arrival per output
     __threadfence();
-    named_bar_sync(1, NC * 32);
-    if (tid == 0) {
-      for (int o = 0; o < nout; ++o) {
-        const int old = atomicAdd(&p.counters[sg.cnt_base + o], 1);
-        lastflag[o] = (old == sg.npieces - 1);
-      }
-      __threadfence();
-    }
-    named_bar_sync(1, NC * 32);
-
-    // ---- the last piece of a segment combines every piece (log-sum-exp).
-    // Per finished output: warp w folds partials w, w+NC, ... with a running
-    // maximum, each lane owning four columns and eight partials' loads in
-    // flight at a time; the NC running states then merge in shared memory.
-    for (int o = 0; o < nout; ++o) {
-      if (!lastflag[o]) continue;  // the same in every thread
+    __syncwarp();
+    int last = 0;
+    if (lane < nout) last = atomicAdd(&p.counters[sg.cnt_base + lane], 1) == sg.npieces - 1;
+    unsigned lastmask = __ballot_sync(FULL, last);
+    if (lastmask) __threadfence();  // acquire the other pieces' partials
+    while (lastmask) {
+      const int o = __ffs(lastmask) - 1;
+      lastmask &= lastmask - 1;
+      constexpr int kFold = 8;  // partials in flight per lane
       const int base = sg.part_base + o;
       const int np = sg.npieces;
-      float M = -INFINITY, L = 0.f;
+      float M = -INFINITY, Lr = 0.f;
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      const bool col = lane * 4 < D;
-      for (int u0 = w; u0 < np; u0 += 8 * NC) {
-        float2 ml[8];
-        float4 ov[8];
+      for (int u0 = 0; u0 < np; u0 += kFold) {
+        float2 ml[kFold];
+        float4 ov[kFold];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int part = base + min(u0 + j * NC, np - 1) * nout;
+        for (int j = 0; j < kFold; ++j) {
+          const int part = base + min(u0 + j, np - 1) * nout;
           ml[j] = __ldcg(&p.part_ml[part]);
           ov[j] = col ? __ldcg(reinterpret_cast<const float4*>(&p.part_o[static_cast<int64_t>(part) * D + lane * 4]))
                       : make_float4(0.f, 0.f, 0.f, 0.f);
         }
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          if (u0 + j * NC >= np || ml[j].x == -INFINITY) continue;
+        for (int j = 0; j < kFold; ++j) {
+          if (u0 + j >= np || ml[j].x == -INFINITY) continue;
           const float mn = fmaxf(M, ml[j].x);
           const float a = (M == -INFINITY) ? 0.f : exp2f(M - mn);
           const float f = exp2f(ml[j].x - mn);
-          L = L * a + f * ml[j].y;
+          Lr = Lr * a + f * ml[j].y;
           acc.x = acc.x * a + f * ov[j].x;
           acc.y = acc.y * a + f * ov[j].y;
           acc.z = acc.z * a + f * ov[j].z;
@@ -582,35 +631,17 @@ __device__ __forceinline__ void mma_consumers(const AttnMmaParams& P, unsigned c
           M = mn;
         }
       }
-      if (lane == 0) mml[w] = make_float2(M, L);
-      if (col) *reinterpret_cast<float4*>(&mo[w * D + lane * 4]) = acc;
-      named_bar_sync(1, NC * 32);
-      for (int e = tid; e < D; e += NC * 32) {
-        float Mt = -INFINITY;
-#pragma unroll
-        for (int ww = 0; ww < NC; ++ww) Mt = fmaxf(Mt, mml[ww].x);
-        float Lt = 0.f, Ot = 0.f;
-        if (Mt != -INFINITY) {
-#pragma unroll
-          for (int ww = 0; ww < NC; ++ww) {
-            const float2 ml = mml[ww];
-            const float f = (ml.x == -INFINITY) ? 0.f : exp2f(ml.x - Mt);
-            Lt = fmaf(f, ml.y, Lt);
-            Ot = fmaf(f, mo[ww * D + e], Ot);
-          }
-        }
-        float res = 0.f;
-        if (Lt > 0.f) {
-          res = Ot / Lt;
-        } else if (e == 0) {
-          atomicOr(p.status, kStatusEmptySoftmax);
-        }
-        p.out[(static_cast<int64_t>(b) * p.Hq + sg.head[sg.out_row[o]]) * D + e] = res;
+      float4 res = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (Lr > 0.f) {
+        const float inv = 1.f / Lr;
+        res = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+      } else if (lane == 0) {
+        atomicOr(p.status, kStatusEmptySoftmax);
       }
-      if (tid == 0) p.counters[sg.cnt_base + o] = 0;
-      named_bar_sync(1, NC * 32);  // mo / mml free again
+      if (col)
+        *reinterpret_cast<float4*>(&p.out[(static_cast<int64_t>(b) * p.Hq + sg.head[sg.out_row[o]]) * D + lane * 4]) = res;
+      if (lane == 0) p.counters[sg.cnt_base + o] = 0;
     }
-    named_bar_sync(1, NC * 32);  // merge area and flags free for the next piece
   }
 }
 
@@ -631,10 +662,14 @@ __global__ void __launch_bounds__(MmaCfg<D, NC, NP, STAGES, GT>::kThreads, 1)
       mbar_init(&bars[STAGES + s], 1);           // empty: the one warp that consumed the tile
     }
     for (int r = 0; r < C::IR; ++r) mbar_init(&bars[2 * STAGES + r], 1);
+    for (int r = 0; r < kPartSlots; ++r) {
+      mbar_init(&bars[2 * STAGES + C::IR + r], NC);  // slot full: every consumer warp
+      mbar_init(&bars[2 * STAGES + C::IR + kPartSlots + r], 1);  // slot free: the epilogue warp
+    }
     *reinterpret_cast<int*>(smem + C::OFF_FLAGS) = 0;
     fence_mbar_init();
   }
-  if (threadIdx.x == NC * 32) {
+  if (threadIdx.x == C::kFirstProducer) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&P.tmk)) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&P.tmv)) : "memory");
     if (GT) {
@@ -646,13 +681,17 @@ __global__ void __launch_bounds__(MmaCfg<D, NC, NP, STAGES, GT>::kThreads, 1)
   pdl_launch_dependents();
   const int pbeg = P.p.cta_begin[blockIdx.x];
   const int pend = P.p.cta_begin[blockIdx.x + 1];
-  if (threadIdx.x >= NC * 32) {
+  if (threadIdx.x >= C::kFirstProducer) {
     mma_producers<D, NC, NP, STAGES, GT>(P, smem, pbeg, pend);
+  } else if (threadIdx.x >= NC * 32) {
+    mma_epilogue<D, NC, NP, STAGES, GT>(P, smem, pbeg, pend);
   } else {
     mma_consumers<D, NC, NP, STAGES, GT>(P, smem, pbeg, pend);
   }
   // this grid completes only after the one it depends on (dense-only CTAs
-  // never waited above), so completion order follows launch order
+  // never waited above), so completion order follows launch order; the
+  // timeline's end is the end of the CTA's last warp
+  if (P.p.timeline) __syncthreads();
   if (threadIdx.x == 0) {
     pdl_wait();
     timeline_record(P.p.timeline, P.p.timeline_cap, t_start,

@@ -99,6 +99,9 @@ struct lyc_ctx {
   int32_t* sbuf = nullptr;  // [2][B][Hs][KS]
   float* part_o = nullptr;
   float2* part_ml = nullptr;
+  // bf16 path: per CTA ring of the consumer warps' piece states
+  float* wpart_o = nullptr;
+  float2* wpart_ml = nullptr;
   int32_t* counters = nullptr;
   size_t max_parts = 0, max_counters = 0;
   // host-buffer entry point staging
@@ -542,6 +545,8 @@ lyc_status enqueue_step(lyc_ctx* ctx, Plan* plan, cudaStream_t stream, int set, 
     ap.keys = ctx->keys;
     ap.part_o = ctx->part_o;
     ap.part_ml = ctx->part_ml;
+    ap.wpart_o = ctx->wpart_o;
+    ap.wpart_ml = ctx->wpart_ml;
     ap.counters = ctx->counters;
     ap.status = ctx->status;
     ap.timeline = plan->timeline;
@@ -775,6 +780,14 @@ lyc_status lyc_create(const lyc_config* cfg, lyc_ctx** out) {
     lyc_destroy(holder.release());
     return st;
   }
+  if (c.dtype == LYC_BF16) {
+    const size_t recs = static_cast<size_t>(ctx->sms) * kPartSlots * kMaxConsumerWarps * kMaxQ;
+    if ((st = alloc(reinterpret_cast<void**>(&ctx->wpart_o), recs * D * sizeof(float))) != LYC_OK ||
+        (st = alloc(reinterpret_cast<void**>(&ctx->wpart_ml), recs * sizeof(float2))) != LYC_OK) {
+      lyc_destroy(holder.release());
+      return st;
+    }
+  }
   if (cudaMemset(ctx->status, 0, 16) != cudaSuccess ||
       cudaMemset(ctx->counters, 0, ctx->max_counters * sizeof(int32_t)) != cudaSuccess ||
       cudaMemset(ctx->sbuf, 0xff, 2ull * B * ctx->Hs * ctx->KS * sizeof(int32_t) + 64) != cudaSuccess) {
@@ -821,7 +834,8 @@ void lyc_destroy(lyc_ctx* ctx) {
   ctx->plans.clear();
   for (cudaEvent_t ev : ctx->events) cudaEventDestroy(ev);
   void* bufs[] = {ctx->status, ctx->keys, ctx->sbuf, ctx->part_o, ctx->part_ml,
-                  ctx->counters, ctx->q_dev, ctx->out_dev, ctx->S_dev};
+                  ctx->wpart_o, ctx->wpart_ml, ctx->counters, ctx->q_dev, ctx->out_dev,
+                  ctx->S_dev};
   for (void* b : bufs)
     if (b) cudaFree(b);
   timed_steps().erase(ctx);

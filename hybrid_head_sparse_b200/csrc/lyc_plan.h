@@ -28,6 +28,10 @@ constexpr int kKeyBins = 2048;     // top 11 bits of an order-preserving key enc
 constexpr int kKeyDigitShift = 21;
 constexpr int kMaxGroup = 8;       // largest Hq / Hkv supported
 constexpr int kMaxQ = kMaxGroup;   // query rows per segment
+constexpr int kMaxConsumerWarps = 8;
+// pieces a CTA's consumer warps may run ahead of its epilogue warp: the ring
+// of per-warp partial states between them has this many slots
+constexpr int kPartSlots = 4;
 
 enum SegKind : int32_t { kDense = 0, kSparse = 1 };
 
@@ -69,6 +73,8 @@ struct AttnParams {
   float* part_o;             // [parts][d]
   float2* part_ml;           // [parts] (running max in log2 units, sum)
   int32_t* counters;         // arrival counters, left at zero after use
+  float* wpart_o;            // per CTA: [kPartSlots][consumer warp][kMaxQ][d] piece states
+  float2* wpart_ml;          // per CTA: [kPartSlots][consumer warp][kMaxQ] (max, sum)
   uint32_t* status;          // device status word
   unsigned long long* timeline;  // NULL, or [1 + 3*cap]: count, then (start ns, end ns, tag)
   int32_t timeline_cap;

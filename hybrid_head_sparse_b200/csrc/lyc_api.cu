@@ -719,6 +719,9 @@ const char* lyc_status_string(lyc_status s) {
     case LYC_ERR_CUDA: return "CUDA error";
     case LYC_ERR_BAD_INDEX: return "inherited set holds an index outside [0, n)";
     case LYC_ERR_TIMEOUT: return "device-side wait timed out";
+    case LYC_ERR_SCRATCH_LIMIT:
+      return "request exceeds the fixed scratch of the allocation-free entry point "
+             "(LYC_NOALLOC_MAX_SETS / LYC_NOALLOC_MAX_CTAS)";
   }
   return "unknown status";
 }

@@ -23,6 +23,10 @@ LYC_ERR_OOM = -3
 LYC_ERR_CUDA = -4
 LYC_ERR_BAD_INDEX = -5
 LYC_ERR_TIMEOUT = -6
+LYC_ERR_SCRATCH_LIMIT = -7
+
+LYC_NOALLOC_MAX_SETS = 256
+LYC_NOALLOC_MAX_CTAS = 32
 
 LYC_BF16 = 0
 LYC_FP32 = 1
@@ -41,7 +45,7 @@ LYC_TIMING_ON = 1
 EXPORTED = ["lyc_create", "lyc_decode_step", "lyc_decode_step_host", "lyc_sync_status",
             "lyc_set_s_trace", "lyc_step_bytes", "lyc_topk_f32", "lyc_set_timing",
             "lyc_kernel_times", "lyc_set_timeline", "lyc_status_string", "lyc_last_error",
-            "lyc_destroy"]
+            "lyc_destroy", "lyc_sparse_attention_noalloc"]
 
 
 class lyc_config(ctypes.Structure):
@@ -101,6 +105,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     L.lyc_last_error.restype = ctypes.c_char_p
     L.lyc_destroy.argtypes = [P]
     L.lyc_destroy.restype = None
+    L.lyc_sparse_attention_noalloc.argtypes = [P, ctypes.POINTER(lyc_kv_cache), I, I, I, I, P, I,
+                                               P, P, P]
     for name in EXPORTED:
         if name not in ("lyc_status_string", "lyc_last_error", "lyc_destroy"):
             getattr(L, name).restype = I
@@ -126,6 +132,15 @@ def lyc_decode_step(ctx, q, kv: lyc_kv_cache, role_mask, k, out, S, stream, flag
 def lyc_decode_step_host(ctx, q, kv: lyc_kv_cache, role_mask, k, out, S, stream, flags) -> int:
     return load().lyc_decode_step_host(ctx, q, ctypes.byref(kv), role_mask, k, out, S, stream,
                                        flags)
+
+
+def lyc_sparse_attention_noalloc(q, kv: lyc_kv_cache, batch, num_q_heads, num_kv_heads,
+                                 head_dim, S, k, out, status, stream) -> int:
+    """The allocation-free sparse attention of one layer (include/lyc.h).
+    Pointers are ints (device addresses); status may be None."""
+    return load().lyc_sparse_attention_noalloc(q, ctypes.byref(kv), batch, num_q_heads,
+                                               num_kv_heads, head_dim, S, k, out, status,
+                                               stream)
 
 
 def lyc_sync_status(ctx) -> int:

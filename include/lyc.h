@@ -48,7 +48,8 @@ typedef enum {
   LYC_ERR_OOM = -3,         /* a library allocation failed */
   LYC_ERR_CUDA = -4,        /* a CUDA call failed; see lyc_last_error */
   LYC_ERR_BAD_INDEX = -5,   /* an inherited set held an index outside [0, n) */
-  LYC_ERR_TIMEOUT = -6      /* a device-side wait gave up (kernel returned early) */
+  LYC_ERR_TIMEOUT = -6,     /* a device-side wait gave up (kernel returned early) */
+  LYC_ERR_SCRATCH_LIMIT = -7 /* lyc_sparse_attention_noalloc: the request exceeds its fixed scratch */
 } lyc_status;
 
 typedef enum { LYC_BF16 = 0, LYC_FP32 = 1 } lyc_dtype;
@@ -184,6 +185,53 @@ lyc_status lyc_kernel_times(lyc_ctx* ctx, lyc_kernel_time* times, int cap, int* 
  * attention, 1 = selection); word 0 counts the records (records past cap are
  * dropped).  NULL turns it off.  Profiling use. */
 lyc_status lyc_set_timeline(lyc_ctx* ctx, unsigned long long* buf, int cap);
+
+/* ---- Allocation-free sparse attention (no counterpart in the paper).
+ *
+ * For callers that cannot allocate device memory: code running under a
+ * framework whose caching allocator owns the device memory (a raw cudaMalloc
+ * fragments that pool and can fail while the pool holds the free memory), or
+ * a latency-critical serving path on which cudaMalloc / cudaFree may
+ * synchronize the device.  lyc_create allocates its scratch, so these callers
+ * cannot hold a context; this entry point needs none and calls no cudaMalloc,
+ * cudaFree or allocating library routine.
+ *
+ * It computes the sparse-head attention of one layer, the same arithmetic as
+ * a sparse head of lyc_decode_step (paper-graph-ui summary, section 3.4
+ * Eq. 3), bf16 inputs: for every batch element b and query head h,
+ *   out[b][h] = softmax(q[b][h] K[S[b][h]]^T / sqrt(d)) V[S[b][h]]
+ * over the first min(k, n) entries of the set S[b][h] (entries past n are the
+ * -1 padding of k > n), with query head h reading KV head h / (Hq / Hkv).
+ *   q       device, [B][Hq][d] bf16, contiguous, 4-byte aligned
+ *   kv      host struct; K, V bf16 [B][Hkv][n][d] with the usual strides
+ *           (s_layer ignored; strides and base pointers as for lyc_decode_step)
+ *   S       device, [B][Hq][k] int32, contiguous, 16-byte aligned, k % 4 == 0;
+ *           indices in [0, n) (others are skipped and reported)
+ *   out     device, [B][Hq][d] float32, contiguous, 16-byte aligned; fully written
+ *   status  NULL, or a device or host uint32 that receives the device status
+ *           word when the work completes (0 = ok, bit 0 = an index outside [0, n))
+ *   stream  cudaStream_t; the work is asynchronous on it
+ * Limits: B * Hq <= LYC_NOALLOC_MAX_SETS, head_dim in {64, 128}, Hq / Hkv <= 8;
+ * the launch uses at most LYC_NOALLOC_MAX_CTAS CTAs.  Larger requests return
+ * LYC_ERR_SCRATCH_LIMIT and enqueue nothing.
+ * Scratch: one file-scope device array of LYC_NOALLOC_SCRATCH_BYTES bytes per
+ * device, shared by every call; it keeps the last call's contents, and each
+ * call clears the parts that must start at zero (arrival counters, status
+ * word).  Calls that overlap on the GPU (different streams with no ordering
+ * between them, or host threads racing) race on it.
+ * Set-up: the first call on a device (with that device current) looks up the
+ * array's address with cudaGetSymbolAddress and sets the kernel's attributes;
+ * make that first call before any stream capture.  A host mutex serializes
+ * the calls' host side.
+ * Errors: INVALID_ARG (pointers, alignment, shapes, k), UNSUPPORTED (d, group
+ * size), SCRATCH_LIMIT, CUDA. */
+#define LYC_NOALLOC_MAX_SETS 256
+#define LYC_NOALLOC_MAX_CTAS 32
+#define LYC_NOALLOC_SCRATCH_BYTES (5u << 20)
+lyc_status lyc_sparse_attention_noalloc(const void* q, const lyc_kv_cache* kv, int batch,
+                                        int num_q_heads, int num_kv_heads, int head_dim,
+                                        const int32_t* S, int k, float* out, uint32_t* status,
+                                        void* stream);
 
 const char* lyc_status_string(lyc_status s);
 const char* lyc_last_error(const lyc_ctx* ctx);

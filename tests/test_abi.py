@@ -34,7 +34,7 @@ def test_every_declared_symbol_is_exported(lyc):
 
 
 def test_status_strings(lyc):
-    for code in (0, -1, -2, -3, -4, -5, -6):
+    for code in (0, -1, -2, -3, -4, -5, -6, -7):
         assert lyc.lyc_status_string(code)
 
 

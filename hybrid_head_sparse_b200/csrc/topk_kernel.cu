@@ -172,11 +172,11 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster_kernel(const Top
   const int cnt = max(0, min(n, lo + chunk) - lo);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const unsigned lt = (1u << lane) - 1u;
-  const uint64_t t_start = p.timeline ? global_timer_ns() : 0;
   // the keys are the attention kernel's output; only once it has completed
   // may the next kernel (the next layer's attention) start its launch
   pdl_wait();
   pdl_launch_dependents();
+  const uint64_t t_start = p.timeline ? global_timer_ns() : 0;  // work starts here
 
   extern __shared__ __align__(16) unsigned char smem[];
   uint2* cand = reinterpret_cast<uint2*>(smem);        // [CAP] (encoded key, index) by source CTA

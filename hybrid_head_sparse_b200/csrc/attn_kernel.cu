@@ -473,6 +473,7 @@ __global__ void __launch_bounds__(AttnCfg<T, D, NQ, STAGES>::kThreads, 1)
   }
   __syncthreads();
   pdl_launch_dependents();
+  if (p.wait_prev) pdl_wait();  // the previous launch writes what this one reads or writes
   const int pbeg = p.cta_begin[blockIdx.x];
   const int pend = p.cta_begin[blockIdx.x + 1];
   if (threadIdx.x >= C::kConsumerWarps * 32) {

@@ -534,17 +534,62 @@ __device__ __forceinline__ void mma_consumers(const AttnMmaParams& P, unsigned c
 }
 
 // ---------------------------------------------------------------- epilogue warp
-// Takes the pieces in the CTA's order.  For each: waits for the NC consumer
-// warps' states, merges them (log-sum-exp) into the piece's partial record,
-// frees the slot, counts the arrival; the last piece of a segment to arrive
-// combines every piece's partial into the output (Appendix C, Algorithm 2,
-// steps 5-6).  The consumers never wait for this work unless they run
-// kPartSlots pieces ahead.  Lane j owns columns 4j .. 4j+3.
+// Two jobs (Appendix C, Algorithm 2, steps 5-6):
+//  1. first, the cross-piece combine of the previous layer: this CTA takes
+//     the (segment, output) tasks t = blockIdx.x, blockIdx.x + gridDim.x, ...
+//     and folds each output's piece partials (log-sum-exp) into that layer's
+//     output.  The previous layer's attention completed before this launch
+//     began (the selection between the two waited for it), so its partials
+//     are in place; running the combine here keeps it off the critical path;
+//  2. then, per piece of this CTA in order: wait for the NC consumer warps'
+//     states, merge them per output, and write the piece's partial (or, for a
+//     segment of one piece, the output itself).
+// The consumers never wait for this work unless they run kPartSlots pieces
+// ahead.  Lane j owns columns 4j .. 4j+3.
+
+// Running log-sum-exp state of one lane (4 columns).
+struct LseAcc {
+  float M, L;
+  float4 o;
+};
+__device__ __forceinline__ void lse_init(LseAcc& a) {
+  a.M = -INFINITY;
+  a.L = 0.f;
+  a.o = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+__device__ __forceinline__ void lse_add(LseAcc& a, float2 ml, float4 ov) {
+  if (ml.x == -INFINITY) return;
+  const float mn = fmaxf(a.M, ml.x);
+  const float s = (a.M == -INFINITY) ? 0.f : exp2f(a.M - mn);
+  const float f = exp2f(ml.x - mn);
+  a.L = a.L * s + f * ml.y;
+  a.o.x = a.o.x * s + f * ov.x;
+  a.o.y = a.o.y * s + f * ov.y;
+  a.o.z = a.o.z * s + f * ov.z;
+  a.o.w = a.o.w * s + f * ov.w;
+  a.M = mn;
+}
+
+// out[b][head of output o] = the normalised state (0 and a status bit if the
+// softmax had no valid row)
+__device__ __forceinline__ void lse_finish(const LseAcc& a, float* out, const AttnParams& p,
+                                           const Segment& sg, int o, int lane, bool col, int D) {
+  float4 res = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (a.L > 0.f) {
+    const float inv = 1.f / a.L;
+    res = make_float4(a.o.x * inv, a.o.y * inv, a.o.z * inv, a.o.w * inv);
+  } else if (lane == 0) {
+    atomicOr(p.status, kStatusEmptySoftmax);
+  }
+  if (col)
+    *reinterpret_cast<float4*>(
+        &out[(static_cast<int64_t>(sg.b) * p.Hq + sg.head[sg.out_row[o]]) * D + lane * 4]) = res;
+}
+
 template <int D, int NC, int NP, int STAGES, bool GT>
 __device__ __forceinline__ void mma_epilogue(const AttnMmaParams& P, unsigned char* smem, int pbeg,
                                              int pend) {
   using C = MmaCfg<D, NC, NP, STAGES, GT>;
-  constexpr unsigned FULL = 0xffffffffu;
   const AttnParams& p = P.p;
   const int lane = threadIdx.x & 31;
   const bool col = lane * 4 < D;
@@ -552,96 +597,76 @@ __device__ __forceinline__ void mma_epilogue(const AttnMmaParams& P, unsigned ch
   uint64_t* slot_full = bars + 2 * STAGES + C::IR;
   uint64_t* slot_free = slot_full + kPartSlots;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_FLAGS);
+
+  // ---- 1. the previous layer's cross-piece combine (after that launch has
+  // completed: the launch just before this one may be it)
+  if (p.prev_ntasks > 0) pdl_wait();
+  for (int t = blockIdx.x; t < p.prev_ntasks; t += gridDim.x) {
+    const int2 task = p.prev_tasks[t];
+    const Segment& sg = p.prev_segs[task.x];
+    const int o = task.y, nout = sg.nout, np = sg.npieces;
+    const int64_t idx0 = sg.part_base + o;
+    LseAcc acc;
+    lse_init(acc);
+    for (int u0 = 0; u0 < np; u0 += 8) {  // eight partials in flight per lane
+      float2 ml[8];
+      float4 ov[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int64_t idx = idx0 + static_cast<int64_t>(min(u0 + j, np - 1)) * nout;
+        ml[j] = __ldcg(&p.prev_part_ml[idx]);
+        ov[j] = col ? __ldcg(reinterpret_cast<const float4*>(&p.prev_part_o[idx * D + lane * 4]))
+                    : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (u0 + j < np) lse_add(acc, ml[j], ov[j]);
+    }
+    lse_finish(acc, p.prev_out, p, sg, o, lane, col, D);
+  }
+
+  // ---- 2. this layer's pieces
   for (int pcI = pbeg; pcI < pend; ++pcI) {
     const Piece pc = p.pieces[pcI];
     const Segment& sg = p.segs[pc.seg];
-    const int nout = sg.nout, b = sg.b;
+    const int nout = sg.nout;
     const int pi = pcI - pbeg;
     const int slot = pi % kPartSlots;
     if (!mbar_wait(&slot_full[slot], (pi / kPartSlots) & 1, abort_flag, p.status)) return;
     const int64_t rec0 = (static_cast<int64_t>(blockIdx.x) * kPartSlots + slot) * NC * kMaxQ;
-    for (int o = 0; o < nout; ++o) {
-      const int r = sg.out_row[o];
-      float2 ml[NC];
-      float4 ov[NC];
+    // load every output's NC warp states first (all in flight), then merge
+    for (int o0 = 0; o0 < nout; o0 += 2) {
+      float2 ml[2][NC];
+      float4 ov[2][NC];
 #pragma unroll
-      for (int ww = 0; ww < NC; ++ww) {
-        ml[ww] = p.wpart_ml[rec0 + ww * kMaxQ + r];
-        ov[ww] = col ? *reinterpret_cast<const float4*>(p.wpart_o + (rec0 + ww * kMaxQ + r) * D + lane * 4)
-                     : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-      float M = -INFINITY;
-#pragma unroll
-      for (int ww = 0; ww < NC; ++ww) M = fmaxf(M, ml[ww].x);
-      float Lr = 0.f;
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (M != -INFINITY) {
+      for (int h = 0; h < 2; ++h) {
+        const int r = sg.out_row[min(o0 + h, nout - 1)];
 #pragma unroll
         for (int ww = 0; ww < NC; ++ww) {
-          const float f = (ml[ww].x == -INFINITY) ? 0.f : exp2f(ml[ww].x - M);
-          Lr = fmaf(f, ml[ww].y, Lr);
-          acc.x = fmaf(f, ov[ww].x, acc.x);
-          acc.y = fmaf(f, ov[ww].y, acc.y);
-          acc.z = fmaf(f, ov[ww].z, acc.z);
-          acc.w = fmaf(f, ov[ww].w, acc.w);
+          ml[h][ww] = p.wpart_ml[rec0 + ww * kMaxQ + r];
+          ov[h][ww] = col ? *reinterpret_cast<const float4*>(p.wpart_o + (rec0 + ww * kMaxQ + r) * D + lane * 4)
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
         }
       }
-      const int part = sg.part_base + pc.ordinal * nout + o;
-      if (col) *reinterpret_cast<float4*>(&p.part_o[static_cast<int64_t>(part) * D + lane * 4]) = acc;
-      if (lane == 0) p.part_ml[part] = make_float2(M, Lr);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int o = o0 + h;
+        if (o >= nout) break;
+        LseAcc acc;
+        lse_init(acc);
+#pragma unroll
+        for (int ww = 0; ww < NC; ++ww) lse_add(acc, ml[h][ww], ov[h][ww]);
+        if (sg.npieces == 1) {
+          lse_finish(acc, p.out, p, sg, o, lane, col, D);  // the whole segment is this piece
+        } else {
+          const int64_t idx = sg.part_base + static_cast<int64_t>(pc.ordinal) * nout + o;
+          if (col) *reinterpret_cast<float4*>(&p.part_o[idx * D + lane * 4]) = acc.o;
+          if (lane == 0) p.part_ml[idx] = make_float2(acc.M, acc.L);
+        }
+      }
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&slot_free[slot]);  // the consumers may reuse the slot
-    // publish the partials, then count this piece's arrival per output
-    __threadfence();
-    __syncwarp();
-    int last = 0;
-    if (lane < nout) last = atomicAdd(&p.counters[sg.cnt_base + lane], 1) == sg.npieces - 1;
-    unsigned lastmask = __ballot_sync(FULL, last);
-    if (lastmask) __threadfence();  // acquire the other pieces' partials
-    while (lastmask) {
-      const int o = __ffs(lastmask) - 1;
-      lastmask &= lastmask - 1;
-      constexpr int kFold = 8;  // partials in flight per lane
-      const int base = sg.part_base + o;
-      const int np = sg.npieces;
-      float M = -INFINITY, Lr = 0.f;
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int u0 = 0; u0 < np; u0 += kFold) {
-        float2 ml[kFold];
-        float4 ov[kFold];
-#pragma unroll
-        for (int j = 0; j < kFold; ++j) {
-          const int part = base + min(u0 + j, np - 1) * nout;
-          ml[j] = __ldcg(&p.part_ml[part]);
-          ov[j] = col ? __ldcg(reinterpret_cast<const float4*>(&p.part_o[static_cast<int64_t>(part) * D + lane * 4]))
-                      : make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-#pragma unroll
-        for (int j = 0; j < kFold; ++j) {
-          if (u0 + j >= np || ml[j].x == -INFINITY) continue;
-          const float mn = fmaxf(M, ml[j].x);
-          const float a = (M == -INFINITY) ? 0.f : exp2f(M - mn);
-          const float f = exp2f(ml[j].x - mn);
-          Lr = Lr * a + f * ml[j].y;
-          acc.x = acc.x * a + f * ov[j].x;
-          acc.y = acc.y * a + f * ov[j].y;
-          acc.z = acc.z * a + f * ov[j].z;
-          acc.w = acc.w * a + f * ov[j].w;
-          M = mn;
-        }
-      }
-      float4 res = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (Lr > 0.f) {
-        const float inv = 1.f / Lr;
-        res = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-      } else if (lane == 0) {
-        atomicOr(p.status, kStatusEmptySoftmax);
-      }
-      if (col)
-        *reinterpret_cast<float4*>(&p.out[(static_cast<int64_t>(b) * p.Hq + sg.head[sg.out_row[o]]) * D + lane * 4]) = res;
-      if (lane == 0) p.counters[sg.cnt_base + o] = 0;
-    }
   }
 }
 
@@ -679,6 +704,7 @@ __global__ void __launch_bounds__(MmaCfg<D, NC, NP, STAGES, GT>::kThreads, 1)
   }
   __syncthreads();
   pdl_launch_dependents();
+  if (P.p.wait_prev) pdl_wait();  // the previous launch writes what this one reads or writes
   const int pbeg = P.p.cta_begin[blockIdx.x];
   const int pend = P.p.cta_begin[blockIdx.x + 1];
   if (threadIdx.x >= C::kFirstProducer) {

@@ -59,6 +59,8 @@ struct LayerPlan {
   int ntasks = 0;
   size_t off_tasks = 0;
   size_t off_trace_src = 0;  // copy table for the set trace after this layer
+  size_t off_combine = 0;    // bf16: (segment, output) pairs combined by the next launch
+  int ncombine = 0;
 };
 
 struct Plan {
@@ -67,6 +69,8 @@ struct Plan {
   size_t dev_bytes = 0;
   size_t off_final_src = 0;      // copy table: current buffer of each set -> caller S
   int nsets = 0;
+  int combine_grid = 1;       // bf16: CTAs of the launch that combines the last layer
+  size_t off_empty_cta = 0;   // its CTA offsets (all zero: no pieces)
   int k = 0, keff = 0, n = 0;
   uint32_t flags = 0;
   const void* q = nullptr;
@@ -279,6 +283,7 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const lyc_k
     std::vector<int32_t> cta;
     std::vector<TopkTask> tasks;
     std::vector<const int32_t*> trace_src;
+    std::vector<int2> combine;  // bf16: (segment, output) left to the next launch
     int nqb = 1;
     int grid = 0;
   };
@@ -426,6 +431,10 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const lyc_k
       for (const Piece& pc : per_cta[c]) H.pieces.push_back(pc);
     }
     H.cta.push_back(static_cast<int32_t>(H.pieces.size()));
+    // partial records (one per piece and output) and arrival counters (one
+    // per output; the fp32 kernel's last-arrival combine); the bf16 kernel
+    // leaves the cross-piece combine of segments cut into several pieces to
+    // the next launch, as (segment, output) tasks
     int part = 0, cnt = 0;
     for (size_t s = 0; s < H.segs.size(); ++s) {
       H.segs[s].npieces = npieces[s];
@@ -433,6 +442,8 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const lyc_k
       H.segs[s].cnt_base = cnt;
       part += npieces[s] * H.segs[s].nout;
       cnt += H.segs[s].nout;
+      if (npieces[s] > 1)
+        for (int o = 0; o < H.segs[s].nout; ++o) H.combine.push_back(make_int2(static_cast<int>(s), o));
     }
     if (static_cast<size_t>(part) > ctx->max_parts || static_cast<size_t>(cnt) > ctx->max_counters)
       return fail(ctx, LYC_ERR_UNSUPPORTED, "work pool larger than the scratch sized at create");
@@ -475,8 +486,13 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const lyc_k
     lp.off_cta = take(H.cta.size() * sizeof(int32_t));
     lp.off_tasks = take(std::max<size_t>(1, H.tasks.size()) * sizeof(TopkTask));
     lp.off_trace_src = take(H.trace_src.size() * sizeof(void*));
+    lp.ncombine = static_cast<int>(H.combine.size());
+    lp.off_combine = take(std::max<size_t>(1, H.combine.size()) * sizeof(int2));
   }
   plan->off_final_src = take(hl[L - 1].trace_src.size() * sizeof(void*));
+  // the last layer's combine runs in a launch of its own, whose CTAs have no pieces
+  plan->combine_grid = std::max(1, std::min(ctx->sms, plan->layers[L - 1].ncombine));
+  plan->off_empty_cta = take((plan->combine_grid + 1) * sizeof(int32_t));
   std::vector<unsigned char> host(bytes, 0);
   for (int l = 0; l < L; ++l) {
     const LayerPlan& lp = plan->layers[l];
@@ -487,6 +503,8 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const lyc_k
     if (!H.tasks.empty())
       memcpy(host.data() + lp.off_tasks, H.tasks.data(), H.tasks.size() * sizeof(TopkTask));
     memcpy(host.data() + lp.off_trace_src, H.trace_src.data(), H.trace_src.size() * sizeof(void*));
+    if (!H.combine.empty())
+      memcpy(host.data() + lp.off_combine, H.combine.data(), H.combine.size() * sizeof(int2));
   }
   memcpy(host.data() + plan->off_final_src, hl[L - 1].trace_src.data(),
          hl[L - 1].trace_src.size() * sizeof(void*));
@@ -516,6 +534,19 @@ lyc_status record_event(lyc_ctx* ctx, Plan* plan, int set, int idx, cudaStream_t
 }
 
 // Enqueue the whole step of `plan` on `stream` (or record it, while capturing).
+// Layer `pl`'s cross-piece combine tasks, for the launch that follows it.
+void set_prev_combine(lyc_ctx* ctx, Plan* plan, int pl, AttnParams* ap) {
+  const lyc_config& cfg = ctx->cfg;
+  const LayerPlan& pp = plan->layers[pl];
+  const int D = cfg.head_dim;
+  ap->prev_segs = reinterpret_cast<const Segment*>(plan->dev + pp.off_segs);
+  ap->prev_tasks = reinterpret_cast<const int2*>(plan->dev + pp.off_combine);
+  ap->prev_ntasks = pp.ncombine;
+  ap->prev_part_o = ctx->part_o + (pl & 1) * ctx->max_parts * D;
+  ap->prev_part_ml = ctx->part_ml + (pl & 1) * ctx->max_parts;
+  ap->prev_out = plan->out + static_cast<size_t>(pl) * cfg.batch * cfg.num_q_heads * D;
+}
+
 lyc_status enqueue_step(lyc_ctx* ctx, Plan* plan, cudaStream_t stream, int set, bool capturing) {
   const lyc_config& cfg = ctx->cfg;
   const int L = cfg.num_layers, B = cfg.batch, Hq = cfg.num_q_heads, D = cfg.head_dim;
@@ -543,8 +574,8 @@ lyc_status enqueue_step(lyc_ctx* ctx, Plan* plan, cudaStream_t stream, int set, 
     ap.q = static_cast<const char*>(plan->q) + static_cast<size_t>(l) * B * Hq * D * es;
     ap.out = plan->out + static_cast<size_t>(l) * B * Hq * D;
     ap.keys = ctx->keys;
-    ap.part_o = ctx->part_o;
-    ap.part_ml = ctx->part_ml;
+    ap.part_o = ctx->part_o + (l & 1) * ctx->max_parts * D;
+    ap.part_ml = ctx->part_ml + (l & 1) * ctx->max_parts;
     ap.wpart_o = ctx->wpart_o;
     ap.wpart_ml = ctx->wpart_ml;
     ap.counters = ctx->counters;
@@ -557,6 +588,10 @@ lyc_status enqueue_step(lyc_ctx* ctx, Plan* plan, cudaStream_t stream, int set, 
     ap.n = plan->n;
     ap.scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
     ap.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
+    // without a selection launch in between, the previous layer's attention
+    // may still be running: its selection keys share the key buffer of the
+    // layer after this one, and its partials are combined by this launch
+    ap.wait_prev = (l > 0 && plan->layers[l - 1].ntasks == 0) ? 1 : 0;
     lyc_status st = record_event(ctx, plan, set, ev++, stream, capturing);
     if (st != LYC_OK) return st;
     if (dtype == 0) {
@@ -567,6 +602,7 @@ lyc_status enqueue_step(lyc_ctx* ctx, Plan* plan, cudaStream_t stream, int set, 
       mp.tgv = plan->tgv;
       mp.p = ap;
       mp.p.gather_rows = plan->gather_rows;
+      if (l > 0) set_prev_combine(ctx, plan, l - 1, &mp.p);
       LYC_CUDA(attn_mma_dispatch(D, &mp, lp.grid, stream, nullptr, false), "attention launch");
     } else {
       LYC_CUDA(attn_simt_dispatch(D, lp.nqb, &ap, lp.grid, stream, nullptr, false), "attention launch");
@@ -594,6 +630,36 @@ lyc_status enqueue_step(lyc_ctx* ctx, Plan* plan, cudaStream_t stream, int set, 
                         plan->k};
       LYC_CUDA(copy_sets_launch(&cp, stream), "trace copy");
     }
+  }
+  if (dtype == 0) {
+    // the last layer's cross-piece combine: the same kernel with no pieces
+    AttnMmaParams mp;
+    mp.tmk = plan->tmk;
+    mp.tmv = plan->tmv;
+    mp.tgk = plan->tgk;
+    mp.tgv = plan->tgv;
+    AttnParams& ap = mp.p;
+    ap = AttnParams{};
+    const LayerPlan& lp = plan->layers[L - 1];
+    ap.segs = reinterpret_cast<const Segment*>(plan->dev + lp.off_segs);
+    ap.pieces = reinterpret_cast<const Piece*>(plan->dev + lp.off_pieces);
+    ap.cta_begin = reinterpret_cast<const int32_t*>(plan->dev + plan->off_empty_cta);
+    ap.q = plan->q;
+    ap.out = plan->out;
+    ap.status = ctx->status;
+    ap.wpart_o = ctx->wpart_o;
+    ap.wpart_ml = ctx->wpart_ml;
+    ap.layer = L;
+    ap.Hq = Hq;
+    ap.G = ctx->G;
+    ap.n = plan->n;
+    set_prev_combine(ctx, plan, L - 1, &ap);
+    lyc_status st = record_event(ctx, plan, set, ev++, stream, capturing);
+    if (st != LYC_OK) return st;
+    LYC_CUDA(attn_mma_dispatch(D, &mp, plan->combine_grid, stream, nullptr, false), "combine launch");
+    if ((st = record_event(ctx, plan, set, ev++, stream, capturing)) != LYC_OK) return st;
+    plan->kernel_kind.push_back(0);
+    plan->kernel_layer.push_back(L - 1);
   }
   CopySetsParams cp{reinterpret_cast<const int32_t* const*>(plan->dev + plan->off_final_src), plan->S,
                     B * ctx->Hs, plan->k};
@@ -759,7 +825,8 @@ lyc_status lyc_create(const lyc_config* cfg, lyc_ctx** out) {
   const int B = c.batch, Hq = c.num_q_heads, Hkv = c.num_kv_heads, D = c.head_dim, L = c.num_layers;
   const size_t es = c.dtype == LYC_BF16 ? 2 : 4;
   const size_t nseg_max = static_cast<size_t>(B) * (Hkv + Hq);
-  ctx->max_parts = (2 * static_cast<size_t>(ctx->sms) + nseg_max) * kMaxQ;  // two pooling phases
+  // pieces per layer <= 2 * sms + segments (two pooling phases)
+  ctx->max_parts = (2 * static_cast<size_t>(ctx->sms) + nseg_max) * kMaxQ;
   ctx->max_counters = nseg_max * kMaxQ;
   auto alloc = [&](void** p, size_t bytes) -> lyc_status {
     if (cudaMalloc(p, bytes) != cudaSuccess) {
@@ -774,8 +841,8 @@ lyc_status lyc_create(const lyc_config* cfg, lyc_ctx** out) {
                   2 * static_cast<size_t>(B) * ctx->Hs * ctx->nstride * sizeof(float))) != LYC_OK ||
       (st = alloc(reinterpret_cast<void**>(&ctx->sbuf),
                   2ull * B * ctx->Hs * ctx->KS * sizeof(int32_t) + 64)) != LYC_OK ||
-      (st = alloc(reinterpret_cast<void**>(&ctx->part_o), ctx->max_parts * D * sizeof(float))) != LYC_OK ||
-      (st = alloc(reinterpret_cast<void**>(&ctx->part_ml), ctx->max_parts * sizeof(float2))) != LYC_OK ||
+      (st = alloc(reinterpret_cast<void**>(&ctx->part_o), 2 * ctx->max_parts * D * sizeof(float))) != LYC_OK ||
+      (st = alloc(reinterpret_cast<void**>(&ctx->part_ml), 2 * ctx->max_parts * sizeof(float2))) != LYC_OK ||
       (st = alloc(reinterpret_cast<void**>(&ctx->counters), ctx->max_counters * sizeof(int32_t))) != LYC_OK ||
       (st = alloc(&ctx->q_dev, static_cast<size_t>(L) * B * Hq * D * es)) != LYC_OK ||
       (st = alloc(reinterpret_cast<void**>(&ctx->out_dev), static_cast<size_t>(L) * B * Hq * D * sizeof(float))) != LYC_OK ||
@@ -984,7 +1051,7 @@ lyc_status lyc_set_timing(lyc_ctx* ctx, int mode) {
   if (!ctx || (mode != LYC_TIMING_OFF && mode != LYC_TIMING_ON)) return LYC_ERR_INVALID_ARG;
   DeviceGuard guard(ctx->cfg.device);
   if (mode == LYC_TIMING_ON && ctx->events.empty()) {
-    ctx->events_per_set = 4 * ctx->cfg.num_layers;
+    ctx->events_per_set = 4 * ctx->cfg.num_layers + 2;  // + the last layer's combine launch
     const size_t total = static_cast<size_t>(timing_sets()) * ctx->events_per_set;
     ctx->events.resize(total, nullptr);
     for (size_t i = 0; i < total; ++i)

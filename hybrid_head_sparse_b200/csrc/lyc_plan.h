@@ -53,7 +53,7 @@ struct Segment {
   int32_t out_row[kMaxQ];  // output o comes from row out_row[o]
   int32_t part_base;    // first partial record of this segment
   int32_t npieces;      // pieces the segment was cut into
-  int32_t cnt_base;     // first arrival counter of this segment (nout counters)
+  int32_t cnt_base;     // first arrival counter of this segment
   int32_t row_base;     // row of (l, b, g, token 0) in the flattened row-gather map
 };
 
@@ -75,6 +75,16 @@ struct AttnParams {
   int32_t* counters;         // arrival counters, left at zero after use
   float* wpart_o;            // per CTA: [kPartSlots][consumer warp][kMaxQ][d] piece states
   float2* wpart_ml;          // per CTA: [kPartSlots][consumer warp][kMaxQ] (max, sum)
+  // bf16 path: the cross-piece combine of a layer runs in the next launch
+  // (the previous layer's outputs, taken by this launch's epilogue warps)
+  const Segment* prev_segs;  // previous layer's segments
+  const int2* prev_tasks;    // (segment, output) pairs of segments cut into > 1 piece
+  int32_t prev_ntasks;
+  const float* prev_part_o;  // previous layer's piece partials
+  const float2* prev_part_ml;
+  float* prev_out;           // previous layer's outputs, [B][Hq][d]
+  int32_t wait_prev;         // 1: wait for the previous launch to complete before any
+                             // work (it is not a selection launch, which would have)
   uint32_t* status;          // device status word
   unsigned long long* timeline;  // NULL, or [1 + 3*cap]: count, then (start ns, end ns, tag)
   int32_t timeline_cap;

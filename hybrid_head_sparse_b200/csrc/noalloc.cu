@@ -52,16 +52,21 @@ namespace {
 constexpr int kNaMaxSets = LYC_NOALLOC_MAX_SETS;   // batch * query heads
 constexpr int kNaMaxCtas = LYC_NOALLOC_MAX_CTAS;   // CTAs of the attention launch
 constexpr int kNaMaxD = 128;
-constexpr int kNaMaxParts = kNaMaxCtas + kNaMaxSets;  // pieces: one per CTA run and segment cut
+constexpr int kNaMaxPieces = kNaMaxCtas + kNaMaxSets;  // one per CTA run and segment cut
+constexpr int kNaMaxParts = kNaMaxPieces;              // one partial per piece (one output each)
+constexpr int kNaMaxCounters = kNaMaxSets;
 
 constexpr size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 // scratch layout (byte offsets)
 constexpr size_t kOffSegs = 0;
 constexpr size_t kOffPieces = align256(kOffSegs + sizeof(Segment) * kNaMaxSets);
-constexpr size_t kOffCta = align256(kOffPieces + sizeof(Piece) * kNaMaxParts);
-constexpr size_t kPlanBytes = align256(kOffCta + sizeof(int32_t) * (kNaMaxCtas + 1));
-constexpr size_t kOffCounters = kPlanBytes;  // [kNaMaxSets] int32, then the status word
-constexpr size_t kOffStatus = kOffCounters + sizeof(int32_t) * kNaMaxSets;
+constexpr size_t kOffCta = align256(kOffPieces + sizeof(Piece) * kNaMaxPieces);
+// the combine launch: (segment, output) tasks and CTA offsets with no pieces
+constexpr size_t kOffTasks = align256(kOffCta + sizeof(int32_t) * (kNaMaxCtas + 1));
+constexpr size_t kOffEmptyCta = align256(kOffTasks + sizeof(int2) * kNaMaxSets);
+constexpr size_t kPlanBytes = align256(kOffEmptyCta + sizeof(int32_t) * (kNaMaxCtas + 1));
+constexpr size_t kOffCounters = kPlanBytes;  // [kNaMaxCounters] int32, then the status word
+constexpr size_t kOffStatus = kOffCounters + sizeof(int32_t) * kNaMaxCounters;
 constexpr size_t kZeroBytes = align256(kOffStatus + 16) - kOffCounters;
 constexpr size_t kOffPartO = kOffCounters + kZeroBytes;
 constexpr size_t kOffPartMl = align256(kOffPartO + sizeof(float) * kNaMaxParts * kNaMaxD);
@@ -208,7 +213,6 @@ extern "C" lyc_status lyc_sparse_attention_noalloc(const void* q, const lyc_kv_c
       sg.nq = sg.nout = 1;
       sg.head[0] = h;
       sg.out_row[0] = 0;
-      sg.cnt_base = b * Hq + h;
     }
   }
   int npc = 0;
@@ -230,12 +234,21 @@ extern "C" lyc_status lyc_sparse_attention_noalloc(const void* q, const lyc_kv_c
     }
     cta[grid] = npc;
   }
-  if (npc > kNaMaxParts) return LYC_ERR_SCRATCH_LIMIT;
-  int part = 0;
+  if (npc > kNaMaxPieces) return LYC_ERR_SCRATCH_LIMIT;
+  // partials: one per piece; segments cut into several pieces are combined
+  // by a second launch of the same kernel, one (segment, output 0) task each
+  int2* tasks = reinterpret_cast<int2*>(g_host_plan + kOffTasks);
+  int32_t* empty_cta = reinterpret_cast<int32_t*>(g_host_plan + kOffEmptyCta);
+  int part = 0, ntasks = 0;
   for (int s = 0; s < nsets; ++s) {
     segs[s].part_base = part;
+    segs[s].cnt_base = s;
     part += segs[s].npieces;
+    if (segs[s].npieces > 1) tasks[ntasks++] = make_int2(s, 0);
   }
+  if (part > kNaMaxParts) return LYC_ERR_SCRATCH_LIMIT;
+  const int cgrid = std::max(1, std::min(ntasks, grid));
+  for (int c = 0; c <= cgrid; ++c) empty_cta[c] = 0;
 
   AttnMmaParams mp;
   memset(&mp, 0, sizeof mp);
@@ -266,10 +279,23 @@ extern "C" lyc_status lyc_sparse_attention_noalloc(const void* q, const lyc_kv_c
   ap.scale = static_cast<float>(1.0 / sqrt(static_cast<double>(D)));
   ap.scale_log2 = static_cast<float>(1.4426950408889634 / sqrt(static_cast<double>(D)));
 
-  // ---- enqueue: work list in, counters and status cleared, the kernel, the status out
+  // the combine launch: no pieces, this launch's partials as its "previous layer"
+  AttnMmaParams cmp = mp;
+  cmp.p.cta_begin = reinterpret_cast<const int32_t*>(dbase + kOffEmptyCta);
+  cmp.p.prev_segs = ap.segs;
+  cmp.p.prev_tasks = reinterpret_cast<const int2*>(dbase + kOffTasks);
+  cmp.p.prev_ntasks = ntasks;
+  cmp.p.prev_part_o = ap.part_o;
+  cmp.p.prev_part_ml = ap.part_ml;
+  cmp.p.prev_out = out;
+
+  // ---- enqueue: work list in, counters and status cleared, the kernel, the
+  // combine, the status out
   if (cudaMemcpyAsync(dbase, g_host_plan, kPlanBytes, cudaMemcpyHostToDevice, stream) != cudaSuccess ||
       cudaMemsetAsync(dbase + kOffCounters, 0, kZeroBytes, stream) != cudaSuccess ||
       attn_mma_dispatch(D, &mp, grid, stream, nullptr, false) != cudaSuccess)
+    return LYC_ERR_CUDA;
+  if (ntasks > 0 && attn_mma_dispatch(D, &cmp, cgrid, stream, nullptr, false) != cudaSuccess)
     return LYC_ERR_CUDA;
   if (status && cudaMemcpyAsync(status, dbase + kOffStatus, sizeof(uint32_t), cudaMemcpyDefault,
                                 stream) != cudaSuccess)

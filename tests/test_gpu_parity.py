@@ -169,6 +169,18 @@ def test_set_input_single_layer(lyc, pattern, gather):
     P.check_layers(data, out, tr, spec.k, spec.n, "bf16", [0], S0=S0.cpu().numpy())
 
 
+@pytest.mark.parametrize("mode", ["per_qhead", "kvgroup_mean"])
+def test_no_retrieval_after_layer0_bf16(lyc, mode):
+    """Layers with no retrieval head launch no selection: consecutive
+    attention launches follow each other directly."""
+    om = O.SELECT_PER_QHEAD if mode == "per_qhead" else O.SELECT_KVGROUP_MEAN
+    spec = W.StackSpec("r0", L=5, B=1, Hq=16, Hkv=4, d=128, n=3000, k=300,
+                       retrieval_per_layer=0, planted="heavy", n_planted=16, seed=14)
+    data, out, S, tr = run_step(lyc, spec, select_mode=mode)
+    P.check_layers(data, out, tr, spec.k, spec.n, "bf16", range(spec.L), select_mode=om)
+    assert np.array_equal(S, tr[0])  # nothing refreshed after layer 0
+
+
 @pytest.mark.parametrize("gather", GATHERS)
 def test_ragged_sets_bf16(lyc, gather):
     """k not a multiple of the 64-row tile nor of the four-row gather: the

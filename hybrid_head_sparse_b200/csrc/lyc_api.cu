@@ -39,6 +39,7 @@ size_t topk_smem_for(int cl, int n);
 int topk_pick_cluster(size_t smem);
 cudaError_t topk_configure(int cl, size_t smem);
 cudaError_t topk_launch(int cl, const TopkParams* p, int ntasks, cudaStream_t stream);
+int topk_max_clusters(int cl, size_t smem);
 cudaError_t copy_sets_launch(const CopySetsParams* p, cudaStream_t stream);
 cudaError_t validate_sets_launch(const ValidateSetsParams* p, cudaStream_t stream);
 }  // namespace lyc
@@ -61,6 +62,7 @@ struct LayerPlan {
   size_t off_trace_src = 0;  // copy table for the set trace after this layer
   size_t off_combine = 0;    // bf16: (segment, output) pairs combined by the next launch
   int ncombine = 0;
+  int topk_cl = 16;          // cluster size of the selection launch
 };
 
 struct Plan {
@@ -95,6 +97,8 @@ struct Plan {
 struct lyc_ctx {
   lyc_config cfg{};
   int G = 1, Hs = 1, sms = 1, topk_cl = 8;
+  unsigned topk_cls = 0;  // bit c: cluster size c is configured for max_ctx (c in 4, 8, 16)
+  int topk_resident[17] = {};  // clusters of size c resident at once (at max_ctx's smem)
   int64_t nstride = 0;  // row stride of the key buffer
   int KS = 0;           // row stride of the set buffers
   std::string err;
@@ -242,6 +246,21 @@ lyc_status encode_gather_map(lyc_ctx* ctx, CUtensorMap* map, const void* base, c
   return LYC_OK;
 }
 
+// Cluster size of a selection launch of `ntasks` sets: the largest configured
+// size whose clusters can all be resident at once (one wave: the next
+// layer's attention launches only once every selection CTA has started),
+// else the smallest.
+int pick_topk_cluster(const lyc_ctx* ctx, int ntasks) {
+  int best = 0, smallest = 0;
+  for (int cl : {16, 8, 4}) {
+    if (!(ctx->topk_cls & (1u << cl))) continue;
+    smallest = cl;
+    const int resident = ctx->topk_resident[cl] > 0 ? ctx->topk_resident[cl] : ctx->sms / cl;
+    if (!best && ntasks <= resident) best = cl;
+  }
+  return best ? best : smallest;
+}
+
 // ---------------------------------------------------------------- planner
 //
 // Builds every layer's work pool for one (role mask, n, k, flags, pointers)
@@ -286,6 +305,7 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const lyc_k
     std::vector<int2> combine;  // bf16: (segment, output) left to the next launch
     int nqb = 1;
     int grid = 0;
+    int topk_cl = 16;           // cluster size of this layer's selection launch
   };
   std::vector<HostLayer> hl(L);
   std::vector<int> cur(Hs, 0);
@@ -392,7 +412,7 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const lyc_k
     // kernel then starts late behind it.
     int avail = ctx->sms;
     if (l > 0) {
-      const int prev = static_cast<int>(hl[l - 1].tasks.size()) * ctx->topk_cl;
+      const int prev = static_cast<int>(hl[l - 1].tasks.size()) * hl[l - 1].topk_cl;
       if (prev > 0 && prev <= ctx->sms / 4) avail = ctx->sms - prev;
     }
     const int grid = static_cast<int>(std::min<int64_t>(NT, avail));
@@ -460,6 +480,7 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const lyc_k
     }
     for (int s = 0; s < Hs; ++s)
       if (fresh[s]) cur[s] ^= 1;
+    H.topk_cl = pick_topk_cluster(ctx, static_cast<int>(H.tasks.size()));
     for (int b = 0; b < B; ++b)
       for (int s = 0; s < Hs; ++s) H.trace_src.push_back(set_ptr(cur[s], b, s));
   }
@@ -481,6 +502,7 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const lyc_k
     lp.grid = H.grid;
     lp.nqb = H.nqb;
     lp.ntasks = static_cast<int>(H.tasks.size());
+    lp.topk_cl = H.topk_cl;
     lp.off_segs = take(H.segs.size() * sizeof(Segment));
     lp.off_pieces = take(H.pieces.size() * sizeof(Piece));
     lp.off_cta = take(H.cta.size() * sizeof(int32_t));
@@ -619,7 +641,7 @@ lyc_status enqueue_step(lyc_ctx* ctx, Plan* plan, cudaStream_t stream, int set, 
       tp.timeline_cap = plan->timeline_cap;
       tp.layer = l;
       if ((st = record_event(ctx, plan, set, ev++, stream, capturing)) != LYC_OK) return st;
-      LYC_CUDA(topk_launch(ctx->topk_cl, &tp, lp.ntasks, stream), "top-k launch");
+      LYC_CUDA(topk_launch(lp.topk_cl, &tp, lp.ntasks, stream), "top-k launch");
       if ((st = record_event(ctx, plan, set, ev++, stream, capturing)) != LYC_OK) return st;
       plan->kernel_kind.push_back(1);
       plan->kernel_layer.push_back(l);
@@ -892,6 +914,17 @@ lyc_status lyc_create(const lyc_config* cfg, lyc_ctx** out) {
       return LYC_ERR_UNSUPPORTED;
     }
   }
+  ctx->topk_cls = 1u << ctx->topk_cl;
+  // smaller clusters (bigger chunks per CTA) for layers with many sets, so
+  // that one selection launch fits the GPU in one wave
+  for (int cl : {8, 4}) {
+    if (cl >= ctx->topk_cl) continue;
+    const size_t sm = topk_smem_for(cl, static_cast<int>(c.max_ctx));
+    if (sm <= static_cast<size_t>(optin) && topk_configure(cl, sm) == cudaSuccess) ctx->topk_cls |= 1u << cl;
+  }
+  for (int cl : {16, 8, 4})
+    if (ctx->topk_cls & (1u << cl))
+      ctx->topk_resident[cl] = topk_max_clusters(cl, topk_smem_for(cl, static_cast<int>(c.max_ctx)));
   cudaGetLastError();
   *out = holder.release();
   return LYC_OK;

@@ -501,13 +501,54 @@ int topk_pick_cluster(size_t smem) {
   return 8;
 }
 
+// How many clusters of `cl` CTAs with `smem` bytes each can be resident at
+// once (0 if unknown); cl must have been configured.
+template <int CL>
+static int topk_max_clusters_t(size_t smem) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(CL, 1, 1);
+  cfg.blockDim = dim3(kTopkThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CL;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, topk_cluster_kernel<CL>, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  return n;
+}
+
+int topk_max_clusters(int cl, size_t smem) {
+  switch (cl) {
+    case 16: return topk_max_clusters_t<16>(smem);
+    case 8: return topk_max_clusters_t<8>(smem);
+    case 4: return topk_max_clusters_t<4>(smem);
+  }
+  return 0;
+}
+
 cudaError_t topk_configure(int cl, size_t smem) {
-  return cl == 16 ? topk_run<16>(nullptr, 0, nullptr, true, smem)
-                  : topk_run<8>(nullptr, 0, nullptr, true, smem);
+  switch (cl) {
+    case 16: return topk_run<16>(nullptr, 0, nullptr, true, smem);
+    case 8: return topk_run<8>(nullptr, 0, nullptr, true, smem);
+    case 4: return topk_run<4>(nullptr, 0, nullptr, true, smem);
+  }
+  return cudaErrorInvalidValue;
 }
 
 cudaError_t topk_launch(int cl, const TopkParams* p, int ntasks, cudaStream_t stream) {
-  return cl == 16 ? topk_run<16>(p, ntasks, stream, false, 0) : topk_run<8>(p, ntasks, stream, false, 0);
+  switch (cl) {
+    case 16: return topk_run<16>(p, ntasks, stream, false, 0);
+    case 8: return topk_run<8>(p, ntasks, stream, false, 0);
+    case 4: return topk_run<4>(p, ntasks, stream, false, 0);
+  }
+  return cudaErrorInvalidValue;
 }
 
 

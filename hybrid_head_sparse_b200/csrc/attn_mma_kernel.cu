@@ -185,12 +185,17 @@ __device__ __forceinline__ void mma_producers(const AttnMmaParams& P, unsigned c
 
   // lookahead cursor (leader only): index-list copies of gathered tiles, LA tiles early
   int la_pc = pbeg, la_r0 = (pbeg < pend) ? p.pieces[pbeg].r0 : 0, la_t = 0;
-  bool waited = false;  // the previous layer's selection has completed
+  bool waited = false;  // the previous launch (a selection) has completed
   auto la_step = [&]() {
     if (la_pc >= pend) return;
     const Piece pc = p.pieces[la_pc];
-    if (p.segs[pc.seg].kind == kSparse) {
-      if (!waited) {  // the inherited sets are that kernel's output
+    const Segment& ls = p.segs[pc.seg];
+    if (ls.kind == kSparse) {
+      // a set the previous launch writes is read only once it has completed;
+      // sets of earlier selections were complete before that launch began
+      // (each selection waits for the attention before it, which waits for
+      // the selection before it), and the bulk copy reads them at L2
+      if (ls.dep && !waited) {
         pdl_wait();
         waited = true;
       }

@@ -315,6 +315,7 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const lyc_k
   const char* kbase = static_cast<const char*>(kv->k);
   const char* vbase = static_cast<const char*>(kv->v);
 
+  std::vector<char> prev_fresh(Hs, 1);  // slots the previous layer's selection wrote
   for (int l = 0; l < L; ++l) {
     HostLayer& H = hl[l];
     // selection keys alternate between two buffers by layer, so a layer's
@@ -379,6 +380,7 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const lyc_k
             }
           if (js > 0) {
             ss.nq = ss.nout = js;
+            ss.dep = prev_fresh[g];
             maxnq = std::max(maxnq, js);
             H.segs.push_back(ss);
           }
@@ -392,6 +394,7 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const lyc_k
             ss.head[0] = h;
             ss.out_row[0] = 0;
             ss.nq = ss.nout = 1;
+            ss.dep = prev_fresh[h];
             H.segs.push_back(ss);
           }
         }
@@ -399,10 +402,13 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const lyc_k
     }
     H.nqb = attn_nq_bucket(maxnq);
 
-    // workload pooling (two phases): the dense rows are cut into equal runs of
-    // 64-row tiles, one per CTA, and so are the gathered rows; CTA c takes its
-    // dense run, then its gathered run, so every CTA carries the same mix
-    // whatever the relative cost of streaming and gathering a tile
+    // workload pooling (two phases): the dense rows are cut into equal runs
+    // of 64-row tiles, one per CTA, and so are the gathered rows; CTA c takes
+    // its dense run, then its gathered run, so every CTA carries the same mix
+    // whatever the relative cost of streaming and gathering a tile.  The
+    // gathered rows list the sets that an earlier layer's selection wrote
+    // first and those the previous layer's selection writes (the only rows
+    // that wait for it) last, so that few CTAs wait, and late.
     int64_t NT = 0;
     for (const Segment& sg : H.segs) NT += (sg.rows + kTileRows - 1) / kTileRows;
     // The previous layer's selection runs beside this layer's attention (the
@@ -420,13 +426,17 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const lyc_k
     std::vector<int> npieces(H.segs.size(), 0);
     std::vector<std::vector<Piece>> per_cta(grid);
     for (int phase = 0; phase < 2; ++phase) {
-      const int want = phase == 0 ? kDense : kSparse;
       std::vector<size_t> ids;
       std::vector<int64_t> tstart(1, 0);
-      for (size_t s2 = 0; s2 < H.segs.size(); ++s2) {
-        if (H.segs[s2].kind != want) continue;
-        ids.push_back(s2);
-        tstart.push_back(tstart.back() + (H.segs[s2].rows + kTileRows - 1) / kTileRows);
+      for (int dep = 0; dep < 2; ++dep) {
+        for (size_t s2 = 0; s2 < H.segs.size(); ++s2) {
+          const Segment& cs = H.segs[s2];
+          if ((cs.kind == kDense ? 0 : 1) != phase || (phase == 1 && cs.dep != dep) ||
+              (phase == 0 && dep == 1))
+            continue;
+          ids.push_back(s2);
+          tstart.push_back(tstart.back() + (cs.rows + kTileRows - 1) / kTileRows);
+        }
       }
       const int64_t nt = tstart.back();
       size_t si = 0;
@@ -480,6 +490,7 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const lyc_k
     }
     for (int s = 0; s < Hs; ++s)
       if (fresh[s]) cur[s] ^= 1;
+    prev_fresh = fresh;
     H.topk_cl = pick_topk_cluster(ctx, static_cast<int>(H.tasks.size()));
     for (int b = 0; b < B; ++b)
       for (int s = 0; s < Hs; ++s) H.trace_src.push_back(set_ptr(cur[s], b, s));

@@ -55,6 +55,8 @@ struct Segment {
   int32_t npieces;      // pieces the segment was cut into
   int32_t cnt_base;     // first arrival counter of this segment
   int32_t row_base;     // row of (l, b, g, token 0) in the flattened row-gather map
+  int32_t dep;          // sparse: the set is the previous launch's output (wait for it)
+  int32_t pad_;
 };
 
 struct Piece {

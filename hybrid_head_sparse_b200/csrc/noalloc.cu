@@ -211,6 +211,7 @@ extern "C" lyc_status lyc_sparse_attention_noalloc(const void* q, const lyc_kv_c
       sg.g = g;
       sg.rows = keff;
       sg.nq = sg.nout = 1;
+      sg.dep = 1;  // the caller's sets: read after whatever ran before on the stream
       sg.head[0] = h;
       sg.out_row[0] = 0;
     }

@@ -37,6 +37,8 @@ namespace lyc {
 
 constexpr int kTopkThreads = 512;
 constexpr int kTopkWarps = kTopkThreads / 32;
+constexpr int kTopkCandCap = 4096;  // pivot-digit candidates gathered from the whole cluster
+constexpr int kTopkSelCap = 4096;   // one CTA's keys at or above the pivot digit
 
 // Exclusive prefix sum of one value per warp (lane 0's) over the CTA; also the total.
 __device__ __forceinline__ void cta_warp_scan(uint32_t* scratch, uint32_t mine, int warp, int lane,
@@ -160,8 +162,10 @@ __device__ __forceinline__ uint32_t select_in_candidates(const uint2* cand, cons
 template <int CL>
 __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster_kernel(const TopkParams p) {
   cg::cluster_group cluster = cg::this_cluster();
-  constexpr int CAP = 4096;        // gathered candidates (all CTAs together)
-  constexpr int RCAP = CAP / CL;   // candidates one CTA may contribute
+  constexpr int CAP = kTopkCandCap;   // gathered candidates (all CTAs together)
+  constexpr int RCAP = CAP / CL;      // candidates one CTA may contribute
+  constexpr int SELCAP = kTopkSelCap; // this CTA's keys at or above the pivot digit
+  constexpr unsigned FULL = 0xffffffffu;
   const int rank = static_cast<int>(cluster.block_rank());
   const TopkTask task = p.tasks ? p.tasks[blockIdx.y] : p.single;
   const int n = p.n;
@@ -180,7 +184,8 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster_kernel(const Top
 
   extern __shared__ __align__(16) unsigned char smem[];
   uint2* cand = reinterpret_cast<uint2*>(smem);        // [CAP] (encoded key, index) by source CTA
-  uint32_t* loc = reinterpret_cast<uint32_t*>(cand + CAP);  // [kKeyBins] this CTA's histogram
+  uint2* sel = cand + CAP;                             // [SELCAP] this CTA's keys >= pivot digit
+  uint32_t* loc = reinterpret_cast<uint32_t*>(sel + SELCAP);  // [kKeyBins] this CTA's histogram
   uint32_t* tot = loc + kKeyBins;                      // [kKeyBins] cluster totals, top digit
   uint32_t* src_cnt = tot + kKeyBins;                  // [CL] candidates per source CTA
   uint32_t* src_above = src_cnt + CL;                  // [CL] keys above the pivot digit per source
@@ -189,7 +194,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster_kernel(const Top
   uint32_t* xchg = src_eq + CL;                        // [CL][2] (fallback path)
   uint32_t* scratch = xchg + 2 * CL;                   // [kTopkWarps]
   uint32_t* found = scratch + kTopkWarps;              // [4]
-  uint32_t* us = found + 4;                            // [chunk] encoded keys
+  uint32_t* us = found + 4;                            // [chunk] encoded keys (16-byte aligned)
 
   if (keff == n) {  // every index is selected
     for (int x = tid; x < cnt; x += kTopkThreads) task.S[lo + x] = lo + x;
@@ -207,28 +212,48 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster_kernel(const Top
     loc[b] = 0u;
   }
   __syncthreads();
+  // Every pass over the chunk gives warp w the contiguous range [wlo, whi)
+  // and walks it 128 keys at a time, lane l holding keys 4l .. 4l+3 of the
+  // step: 16-byte shared-memory accesses without bank conflicts, and index
+  // order = (step, lane, element).
+  const int span = ((cnt + kTopkWarps - 1) / kTopkWarps + 127) & ~127;
+  const int wlo = min(cnt, warp * span);
+  const int whi = min(cnt, wlo + span);
+  auto load4 = [&](int x0, uint32_t* u) {  // four encoded keys from shared memory
+    if (x0 + 3 < whi) {
+      const uint4 v = *reinterpret_cast<const uint4*>(us + x0);
+      u[0] = v.x; u[1] = v.y; u[2] = v.z; u[3] = v.w;
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) u[e] = (x0 + e < whi) ? us[x0 + e] : 0u;
+    }
+  };
+
   // ---- the chunk, encoded, into shared memory, and its top-digit histogram
-  const float* src = task.keys + lo;
-  const bool vec = (reinterpret_cast<uintptr_t>(src) & 15u) == 0;
-  const int nv = vec ? (cnt >> 2) : 0;
-  for (int x = tid; x < nv; x += kTopkThreads) {
-    const float4 v = reinterpret_cast<const float4*>(src)[x];
-    const uint32_t a = order_key(v.x), b = order_key(v.y), c = order_key(v.z), d = order_key(v.w);
-    us[4 * x + 0] = a;
-    us[4 * x + 1] = b;
-    us[4 * x + 2] = c;
-    us[4 * x + 3] = d;
-    atomicAdd(&loc[a >> kKeyDigitShift], 1u);
-    atomicAdd(&loc[b >> kKeyDigitShift], 1u);
-    atomicAdd(&loc[c >> kKeyDigitShift], 1u);
-    atomicAdd(&loc[d >> kKeyDigitShift], 1u);
+  {
+    const float* src = task.keys + lo;
+    const bool vec = (reinterpret_cast<uintptr_t>(src) & 15u) == 0;
+    for (int base = wlo; base < whi; base += 128) {
+      const int x0 = base + 4 * lane;
+      uint32_t u[4];
+      if (vec && x0 + 3 < whi) {
+        const float4 v = *reinterpret_cast<const float4*>(src + x0);
+        u[0] = order_key(v.x); u[1] = order_key(v.y); u[2] = order_key(v.z); u[3] = order_key(v.w);
+        *reinterpret_cast<uint4*>(us + x0) = make_uint4(u[0], u[1], u[2], u[3]);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          u[e] = (x0 + e < whi) ? order_key(src[x0 + e]) : 0u;
+          if (x0 + e < whi) us[x0 + e] = u[e];
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if (x0 + e < whi) atomicAdd(&loc[u[e] >> kKeyDigitShift], 1u);
+    }
   }
-  for (int x = (nv << 2) + tid; x < cnt; x += kTopkThreads) {
-    const uint32_t a = order_key(src[x]);
-    us[x] = a;
-    atomicAdd(&loc[a >> kKeyDigitShift], 1u);
-  }
-  cluster.sync();  // (1) every CTA's totals are zero
+  __syncthreads();
+  cluster.sync();  // (1) every CTA's totals are zero and its histogram complete
 
   // ---- top digit: add the non-zero local bins into every CTA's totals
   {
@@ -245,48 +270,86 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster_kernel(const Top
   uint32_t krem = static_cast<uint32_t>(keff) - above;
   const uint32_t ncand = tot[d0];
 
-  // ---- this CTA's candidates (top digit == d0), in index order, gathered
-  // into every CTA together with the count of its keys above the digit
-  uint32_t my_cand = 0u, my_above = 0u;
+  // ---- pass over the chunk: per warp, keys above the pivot digit and keys
+  // on it (the candidates)
+  uint32_t my_cand = 0u, my_above = 0u, c_before = 0u, a_before = 0u;
   {
-    const int span = ((cnt + kTopkWarps - 1) / kTopkWarps + 31) & ~31;
-    const int wlo = warp * span;
-    const int whi = min(cnt, wlo + span);
     uint32_t wc = 0u, wa = 0u;
-    for (int base = wlo; base < whi; base += 32) {
-      const int x = base + lane;
-      const uint32_t dg = (x < whi) ? (us[x] >> kKeyDigitShift) : 0u;
-      wc += __popc(__ballot_sync(0xffffffffu, x < whi && dg == d0));
-      wa += __popc(__ballot_sync(0xffffffffu, x < whi && dg > d0));
+    for (int base = wlo; base < whi; base += 128) {
+      const int x0 = base + 4 * lane;
+      uint32_t u[4];
+      load4(x0, u);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const bool ok = x0 + e < whi;
+        const uint32_t dg = u[e] >> kKeyDigitShift;
+        wc += (ok && dg == d0) ? 1u : 0u;
+        wa += (ok && dg > d0) ? 1u : 0u;
+      }
     }
-    uint32_t c_before, a_before;
+#pragma unroll
+    for (int s2 = 16; s2 >= 1; s2 >>= 1) {
+      wc += __shfl_xor_sync(FULL, wc, s2);
+      wa += __shfl_xor_sync(FULL, wa, s2);
+    }
     cta_warp_scan(scratch, wc, warp, lane, &c_before, &my_cand);
     cta_warp_scan(scratch, wa, warp, lane, &a_before, &my_above);
-    if (my_cand <= static_cast<uint32_t>(RCAP)) {
-      // own candidates, in index order, into this CTA's region first
-      uint2* mine = cand + rank * RCAP;
-      uint32_t pos = c_before;
-      for (int base = wlo; base < whi; base += 32) {
-        const int x = base + lane;
-        const uint32_t u = (x < whi) ? us[x] : 0u;
-        const bool is_c = x < whi && (u >> kKeyDigitShift) == d0;
-        const unsigned cb = __ballot_sync(0xffffffffu, is_c);
-        if (is_c) mine[pos + __popc(cb & lt)] = make_uint2(u, static_cast<uint32_t>(lo + x));
-        pos += __popc(cb);
+  }
+  // this CTA's keys at or above the pivot digit, in index order, into `sel`
+  // (when they fit), and its candidates into its region of `cand`
+  const bool sel_fits = my_above + my_cand <= static_cast<uint32_t>(SELCAP);
+  const bool cand_fits = my_cand <= static_cast<uint32_t>(RCAP);
+  uint2* mine = cand + rank * RCAP;
+  if (sel_fits || cand_fits) {
+    uint32_t cpos = c_before, spos = a_before + c_before;
+    for (int base = wlo; base < whi; base += 128) {
+      const int x0 = base + 4 * lane;
+      uint32_t u[4];
+      load4(x0, u);
+      // one ballot per element slot: a lane's entries come after every entry
+      // of the lanes below it (index order is lane, then element)
+      unsigned bc[4], bs[4];
+      uint32_t oc = cpos, os = spos, tc = 0u, ts = 0u;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const bool ok = x0 + e < whi;
+        const uint32_t dg = u[e] >> kKeyDigitShift;
+        bc[e] = __ballot_sync(FULL, ok && dg == d0);
+        bs[e] = __ballot_sync(FULL, ok && dg >= d0);
+        oc += __popc(bc[e] & lt);
+        os += __popc(bs[e] & lt);
+        tc += __popc(bc[e]);
+        ts += __popc(bs[e]);
       }
-      __syncthreads();
-      // then copies into the other CTAs, (entry, CTA) pairs spread over the threads
-      for (uint32_t x = tid; x < my_cand * (CL - 1); x += kTopkThreads) {
-        const uint32_t j = x / (CL - 1);
-        const int r = static_cast<int>(x % (CL - 1));
-        const int dst = r < rank ? r : r + 1;
-        cluster.map_shared_rank(cand, dst)[rank * RCAP + j] = mine[j];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint2 ent = make_uint2(u[e], static_cast<uint32_t>(lo + x0 + e));
+        if ((bs[e] >> lane) & 1u) {
+          if (sel_fits) sel[os] = ent;
+          ++os;
+        }
+        if ((bc[e] >> lane) & 1u) {
+          if (cand_fits) mine[oc] = ent;
+          ++oc;
+        }
       }
+      cpos += tc;
+      spos += ts;
     }
-    if (tid < CL) {
-      cluster.map_shared_rank(src_cnt, tid)[rank] = my_cand;
-      cluster.map_shared_rank(src_above, tid)[rank] = my_above;
+  }
+  __syncthreads();
+  // candidates into the other CTAs, (entry, CTA) pairs spread over the threads
+  if (cand_fits) {
+    for (uint32_t x = tid; x < my_cand * (CL - 1); x += kTopkThreads) {
+      const uint32_t j = x / (CL - 1);
+      const int r = static_cast<int>(x % (CL - 1));
+      const int dst = r < rank ? r : r + 1;
+      cluster.map_shared_rank(cand, dst)[rank * RCAP + j] = mine[j];
     }
+  }
+  if (tid < CL) {
+    cluster.map_shared_rank(src_cnt, tid)[rank] = my_cand;
+    cluster.map_shared_rank(src_above, tid)[rank] = my_above;
   }
   cluster.sync();  // (3) candidates and counts of every CTA are here
 
@@ -387,48 +450,55 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster_kernel(const Top
     take = (krem > eq_prev) ? min(krem - eq_prev, eq_cta) : 0u;
   }
 
-  // ---- write this CTA's selected indices in index order: warp w owns
-  // [w*span, (w+1)*span), span a multiple of 128, four ballot rows per step
-  const int span = ((cnt + kTopkWarps - 1) / kTopkWarps + 127) & ~127;
-  const int wlo = warp * span;
-  const int whi = min(cnt, wlo + span);
-  uint32_t wgt = 0u, weq = 0u;
-  for (int base = wlo; base < whi; base += 128) {
+  // ---- write this CTA's selected indices in index order, from `sel` when it
+  // holds every key at or above the pivot digit (few), else from the whole
+  // chunk.  Warp w owns entries [w*span, (w+1)*span) of the list, span a
+  // multiple of 128, four ballot rows per step.
+  auto emit = [&](auto get, int len) {
+    const int sp = ((len + kTopkWarps - 1) / kTopkWarps + 127) & ~127;
+    const int elo = min(len, warp * sp);
+    const int ehi = min(len, elo + sp);
+    uint32_t wgt = 0u, weq = 0u;
+    for (int base = elo; base < ehi; base += 128) {
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int x = base + 32 * j + lane;
-      const uint32_t u = (x < whi) ? us[x] : 0u;
-      wgt += __popc(__ballot_sync(0xffffffffu, x < whi && u > tau));
-      weq += __popc(__ballot_sync(0xffffffffu, x < whi && u == tau));
+      for (int j = 0; j < 4; ++j) {
+        const int x = base + 32 * j + lane;
+        const uint32_t u = (x < ehi) ? get(x).x : 0u;
+        wgt += __popc(__ballot_sync(FULL, x < ehi && u > tau));
+        weq += __popc(__ballot_sync(FULL, x < ehi && u == tau));
+      }
     }
-  }
-  uint32_t gt_before, eq_before, dummy2;
-  cta_warp_scan(scratch, wgt, warp, lane, &gt_before, &dummy2);
-  cta_warp_scan(scratch, weq, warp, lane, &eq_before, &dummy2);
-  uint32_t run_eq = eq_before;
-  uint32_t run_sel = out_base + gt_before + min(eq_before, take);
-  for (int base = wlo; base < whi; base += 128) {
-    uint32_t u[4];
-    unsigned gb[4], eb[4];
+    uint32_t gt_before, eq_before, dummy2;
+    cta_warp_scan(scratch, wgt, warp, lane, &gt_before, &dummy2);
+    cta_warp_scan(scratch, weq, warp, lane, &eq_before, &dummy2);
+    uint32_t run_eq = eq_before;
+    uint32_t run_sel = out_base + gt_before + min(eq_before, take);
+    for (int base = elo; base < ehi; base += 128) {
+      uint2 ent[4];
+      unsigned gb[4], eb[4];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int x = base + 32 * j + lane;
-      u[j] = (x < whi) ? us[x] : 0u;
-      gb[j] = __ballot_sync(0xffffffffu, x < whi && u[j] > tau);
-      eb[j] = __ballot_sync(0xffffffffu, x < whi && u[j] == tau);
-    }
+      for (int j = 0; j < 4; ++j) {
+        const int x = base + 32 * j + lane;
+        ent[j] = (x < ehi) ? get(x) : make_uint2(0u, 0u);
+        gb[j] = __ballot_sync(FULL, x < ehi && ent[j].x > tau);
+        eb[j] = __ballot_sync(FULL, x < ehi && ent[j].x == tau);
+      }
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int x = base + 32 * j + lane;
-      const bool is_eq = (eb[j] >> lane) & 1u;
-      const bool sel = ((gb[j] >> lane) & 1u) || (is_eq && run_eq + __popc(eb[j] & lt) < take);
-      const unsigned sb = __ballot_sync(0xffffffffu, sel);
-      const uint32_t pos = run_sel + __popc(sb & lt);
-      if (sel && pos < static_cast<uint32_t>(keff)) task.S[pos] = lo + x;
-      run_sel += __popc(sb);
-      run_eq += __popc(eb[j]);
+      for (int j = 0; j < 4; ++j) {
+        const bool is_eq = (eb[j] >> lane) & 1u;
+        const bool pick = ((gb[j] >> lane) & 1u) || (is_eq && run_eq + __popc(eb[j] & lt) < take);
+        const unsigned sb = __ballot_sync(FULL, pick);
+        const uint32_t pos = run_sel + __popc(sb & lt);
+        if (pick && pos < static_cast<uint32_t>(keff)) task.S[pos] = static_cast<int32_t>(ent[j].y);
+        run_sel += __popc(sb);
+        run_eq += __popc(eb[j]);
+      }
     }
-  }
+  };
+  if (fits && sel_fits)
+    emit([&](int x) { return sel[x]; }, static_cast<int>(my_above + my_cand));
+  else
+    emit([&](int x) { return make_uint2(us[x], static_cast<uint32_t>(lo + x)); }, cnt);
   if (rank == 0)
     for (int x = keff + tid; x < k; x += kTopkThreads) task.S[x] = -1;
   if (tid == 0)
@@ -442,7 +512,8 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster_kernel(const Top
 // ---------------------------------------------------------------- host side
 static size_t topk_smem_bytes(int cl, int n) {
   const int chunk = (((n + cl - 1) / cl) + 3) & ~3;
-  return static_cast<size_t>(2 * 4096 + 2 * kKeyBins + 6 * cl + kTopkWarps + 4 + chunk) * 4u;
+  return static_cast<size_t>(2 * kTopkCandCap + 2 * kTopkSelCap + 2 * kKeyBins + 6 * cl + kTopkWarps +
+                             4 + chunk) * 4u;
 }
 
 template <int CL>

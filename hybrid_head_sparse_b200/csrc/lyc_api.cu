@@ -246,17 +246,24 @@ lyc_status encode_gather_map(lyc_ctx* ctx, CUtensorMap* map, const void* base, c
   return LYC_OK;
 }
 
-// Cluster size of a selection launch of `ntasks` sets: the largest configured
-// size whose clusters can all be resident at once (one wave: the next
-// layer's attention launches only once every selection CTA has started),
-// else the smallest.
+// Cluster size of a selection launch of `ntasks` sets.  A small selection (a
+// few sets) runs beside the next layer's attention, on SMs the planner takes
+// from that attention: clusters of 8 (measured on B200 at 128K keys: the best
+// balance between the selection's latency, which the next layer's dense rows
+// hide, and the SMs taken from the attention; 16 takes twice the SMs, 4 takes
+// longer than the dense rows last).  A large selection (layer 0) takes the
+// largest size whose clusters are all resident at once, so that it runs in
+// one wave and the next layer starts right away; else the smallest size.
 int pick_topk_cluster(const lyc_ctx* ctx, int ntasks) {
+  auto resident = [&](int cl) {
+    return ctx->topk_resident[cl] > 0 ? ctx->topk_resident[cl] : ctx->sms / cl;
+  };
+  if (ntasks * 16 <= ctx->sms / 4 && (ctx->topk_cls & (1u << 8)) && ntasks <= resident(8)) return 8;
   int best = 0, smallest = 0;
   for (int cl : {16, 8, 4}) {
     if (!(ctx->topk_cls & (1u << cl))) continue;
     smallest = cl;
-    const int resident = ctx->topk_resident[cl] > 0 ? ctx->topk_resident[cl] : ctx->sms / cl;
-    if (!best && ntasks <= resident) best = cl;
+    if (!best && ntasks <= resident(cl)) best = cl;
   }
   return best ? best : smallest;
 }

@@ -46,6 +46,8 @@ def parse_args(argv=None):
     ap.add_argument("--retrieval-heads", type=int, default=2,
                     help="retrieval query heads per layer after layer 0; -1 = all (dense baseline)")
     ap.add_argument("--select-mode", choices=["per_qhead", "kvgroup_mean"], default="per_qhead")
+    ap.add_argument("--attn-kernel", choices=["mma", "tcgen05"], default="mma",
+                    help="bf16 attention kernel: mma.sync (default) or tcgen05/TMEM")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-layers", type=int, default=2,
@@ -301,7 +303,8 @@ def run_lyc(args):
     data = W.make_stack(spec, dev)
     torch.cuda.synchronize()
     ctx = lyc.Lyc(spec.L, spec.B, spec.Hq, spec.Hkv, spec.d, spec.n, spec.k, dtype=spec.dtype,
-                  select_mode=args.select_mode, device=local)
+                  select_mode=args.select_mode, device=local,
+                  flags=lyc.LYC_CFG_TCGEN05 if args.attn_kernel == "tcgen05" else 0)
     out = torch.empty((spec.L, spec.B, spec.Hq, spec.d), device=dev)
     S = torch.empty((spec.B, ctx.Hs, spec.k), dtype=torch.int32, device=dev)
     role = data["role"]
@@ -355,23 +358,29 @@ def run_lyc(args):
     nsteps_t = args.steps
     attn_ms = sum(t[2] for t in ktimes if t[0] == 0) / nsteps_t
     topk_ms = sum(t[2] for t in ktimes if t[0] == 1) / nsteps_t
+    # attention launches: one per layer plus the launch that combines the last
+    # layer's split rows; the roofline's per-launch figures are per layer
     attn_launches = sum(1 for t in ktimes if t[0] == 0) // nsteps_t
     topk_launches = sum(1 for t in ktimes if t[0] == 1) // nsteps_t
+    per_layer = spec.L
 
     analytic, distinct = ctx.step_bytes(role, spec.n, spec.k)
     peak, peak_kind = measured_peaks()
     achieved = distinct / (attn_ms / 1e3) / 1e9
     traffic = profiled_traffic(spec.name)
     roofline = {
-        "bound": "hbm", "kernel": "attn_mma_layer_kernel (pooled dense + sparse attention, one launch per layer)",
+        "bound": "hbm",
+        "kernel": ("attn_tc_layer_kernel" if args.attn_kernel == "tcgen05" else "attn_mma_layer_kernel")
+                  + " (pooled dense + sparse attention, one launch per layer)",
         "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
         "frac": round(achieved / peak, 4), "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
         "traffic": traffic,
-        "algorithmic_bytes_per_launch": distinct / attn_launches,
-        "avg_launch_ms": attn_ms / attn_launches,
+        "algorithmic_bytes_per_launch": distinct / per_layer,
+        "avg_launch_ms": attn_ms / per_layer,
         "note": ("achieved = K+V bytes the kernel must read (dense groups: n rows; each sparse pass: "
-                 "k rows) / CUDA-event time of the attention launches, averaged over the layers of "
-                 "K timed steps"),
+                 "k rows) / CUDA-event time of the attention launches (one per layer, plus the "
+                 "small launch that combines the last layer's split rows), per layer, over K "
+                 "timed steps"),
     }
     step_gbs = analytic / (ms_step / 1e3) / 1e9
 
@@ -426,7 +435,8 @@ def run_lyc(args):
         "config": {"workload": spec.name, "L": spec.L, "B": spec.B, "Hq": spec.Hq,
                    "Hkv": spec.Hkv, "d": spec.d, "n": spec.n, "k": spec.k,
                    "retrieval_heads_per_layer": args.retrieval_heads,
-                   "select_mode": args.select_mode, "parallelism": f"replicas x{world}",
+                   "select_mode": args.select_mode, "attn_kernel": args.attn_kernel,
+                   "parallelism": f"replicas x{world}",
                    "l2": "inputs larger than L2 (KV cache %.1f GB per GPU)" % (
                        2 * data["k"].numel() * data["k"].element_size() / 1e9)},
         "hbm": {"analytic_bytes_per_step": analytic, "kernel_bytes_per_step": distinct,

@@ -35,6 +35,9 @@ cudaError_t attn_simt_dispatch(int D, int nqb, const AttnParams* p, int grid, cu
                                int* smem_out, bool configure_only);
 cudaError_t attn_mma_dispatch(int D, const AttnMmaParams* P, int grid, cudaStream_t stream,
                               int* smem_out, bool configure_only);
+cudaError_t attn_tc_dispatch(const AttnMmaParams* P, int grid, cudaStream_t stream, int* smem_out,
+                             bool configure_only);
+int attn_tc_tile_rows();
 size_t topk_smem_for(int cl, int n);
 int topk_pick_cluster(size_t smem);
 cudaError_t topk_configure(int cl, size_t smem);
@@ -85,6 +88,7 @@ struct Plan {
   CUtensorMap tmk{}, tmv{};       // bf16 path: 5-D maps of the whole K and V cache
   CUtensorMap tgk{}, tgv{};       // bf16 path: 2-D row-gather maps (when gather_rows > 0)
   int32_t gather_rows = 0;        // rows of the row-gather maps; 0 = none
+  bool use_tc = false;            // bf16: the tcgen05 attention kernel
   cudaGraphExec_t exec = nullptr;
   // timing: event-record nodes of the graph, in launch order (2 per kernel)
   std::vector<cudaGraphNode_t> ev_nodes;
@@ -183,7 +187,8 @@ EncodeTiledFn encode_tiled_fn() {
 
 // 5-D map (d, row, KV head, batch, layer) of one cache tensor, 64 x 64 boxes
 // of 128-byte rows with the 128B swizzle; rows at or past n read as zeros.
-lyc_status encode_cache_map(lyc_ctx* ctx, CUtensorMap* map, const void* base, const lyc_kv_cache* kv) {
+lyc_status encode_cache_map(lyc_ctx* ctx, CUtensorMap* map, const void* base, const lyc_kv_cache* kv,
+                            int tile_rows) {
   const lyc_config& c = ctx->cfg;
   EncodeTiledFn fn = encode_tiled_fn();
   if (!fn) return fail(ctx, LYC_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
@@ -198,7 +203,7 @@ lyc_status encode_cache_map(lyc_ctx* ctx, CUtensorMap* map, const void* base, co
     if (dims[i + 1] == 1 && st[i] == 0) st[i] = (i == 0 ? c.head_dim * es : st[i - 1] * static_cast<int64_t>(dims[i]));
   const cuuint64_t strides[4] = {static_cast<cuuint64_t>(st[0]), static_cast<cuuint64_t>(st[1]),
                                  static_cast<cuuint64_t>(st[2]), static_cast<cuuint64_t>(st[3])};
-  const cuuint32_t box[5] = {64, static_cast<cuuint32_t>(kTileRows), 1, 1, 1};
+  const cuuint32_t box[5] = {64, static_cast<cuuint32_t>(tile_rows), 1, 1, 1};
   const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box,
                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -290,9 +295,14 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const lyc_k
   plan->n = n;
   plan->nsets = B * Hs;
   plan->gather_rows = 0;
+  // bf16 with head_dim 128 runs on the tcgen05 kernel (128-row tiles) when
+  // the config asks for it (and q is 16-byte aligned), else on the mma.sync one
+  plan->use_tc = cfg.dtype == LYC_BF16 && cfg.head_dim == 128 && (cfg.flags & LYC_CFG_TCGEN05) &&
+                 !(cfg.flags & LYC_CFG_TMA_GATHER) && (reinterpret_cast<uintptr_t>(plan->q) & 15u) == 0;
+  const int TR = plan->use_tc ? attn_tc_tile_rows() : kTileRows;
   if (cfg.dtype == LYC_BF16) {
-    lyc_status st = encode_cache_map(ctx, &plan->tmk, kv->k, kv);
-    if (st == LYC_OK) st = encode_cache_map(ctx, &plan->tmv, kv->v, kv);
+    lyc_status st = encode_cache_map(ctx, &plan->tmk, kv->k, kv, TR);
+    if (st == LYC_OK) st = encode_cache_map(ctx, &plan->tmv, kv->v, kv, TR);
     if (st != LYC_OK) return st;
     const int64_t rows = (cfg.flags & LYC_CFG_TMA_GATHER) ? gather_map_rows(cfg, kv) : 0;
     if (rows > 0) {
@@ -417,7 +427,7 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const lyc_k
     // first and those the previous layer's selection writes (the only rows
     // that wait for it) last, so that few CTAs wait, and late.
     int64_t NT = 0;
-    for (const Segment& sg : H.segs) NT += (sg.rows + kTileRows - 1) / kTileRows;
+    for (const Segment& sg : H.segs) NT += (sg.rows + TR - 1) / TR;
     // The previous layer's selection runs beside this layer's attention (the
     // attention streams its dense rows meanwhile and waits for the sets only
     // before its gathered rows).  When that selection is small, leave its SMs
@@ -442,7 +452,7 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const lyc_k
               (phase == 0 && dep == 1))
             continue;
           ids.push_back(s2);
-          tstart.push_back(tstart.back() + (cs.rows + kTileRows - 1) / kTileRows);
+          tstart.push_back(tstart.back() + (cs.rows + TR - 1) / TR);
         }
       }
       const int64_t nt = tstart.back();
@@ -456,8 +466,8 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const lyc_k
           if (e <= a) continue;
           Piece pc;
           pc.seg = static_cast<int32_t>(ids[q]);
-          pc.r0 = static_cast<int32_t>(a * kTileRows);
-          pc.r1 = static_cast<int32_t>(std::min<int64_t>(e * kTileRows, H.segs[ids[q]].rows));
+          pc.r0 = static_cast<int32_t>(a * TR);
+          pc.r1 = static_cast<int32_t>(std::min<int64_t>(e * TR, H.segs[ids[q]].rows));
           pc.ordinal = npieces[ids[q]]++;
           per_cta[c].push_back(pc);
         }
@@ -643,7 +653,9 @@ lyc_status enqueue_step(lyc_ctx* ctx, Plan* plan, cudaStream_t stream, int set, 
       mp.p = ap;
       mp.p.gather_rows = plan->gather_rows;
       if (l > 0) set_prev_combine(ctx, plan, l - 1, &mp.p);
-      LYC_CUDA(attn_mma_dispatch(D, &mp, lp.grid, stream, nullptr, false), "attention launch");
+      LYC_CUDA(plan->use_tc ? attn_tc_dispatch(&mp, lp.grid, stream, nullptr, false)
+                            : attn_mma_dispatch(D, &mp, lp.grid, stream, nullptr, false),
+               "attention launch");
     } else {
       LYC_CUDA(attn_simt_dispatch(D, lp.nqb, &ap, lp.grid, stream, nullptr, false), "attention launch");
     }
@@ -696,7 +708,9 @@ lyc_status enqueue_step(lyc_ctx* ctx, Plan* plan, cudaStream_t stream, int set, 
     set_prev_combine(ctx, plan, L - 1, &ap);
     lyc_status st = record_event(ctx, plan, set, ev++, stream, capturing);
     if (st != LYC_OK) return st;
-    LYC_CUDA(attn_mma_dispatch(D, &mp, plan->combine_grid, stream, nullptr, false), "combine launch");
+    LYC_CUDA(plan->use_tc ? attn_tc_dispatch(&mp, plan->combine_grid, stream, nullptr, false)
+                          : attn_mma_dispatch(D, &mp, plan->combine_grid, stream, nullptr, false),
+             "combine launch");
     if ((st = record_event(ctx, plan, set, ev++, stream, capturing)) != LYC_OK) return st;
     plan->kernel_kind.push_back(0);
     plan->kernel_layer.push_back(L - 1);
@@ -840,7 +854,7 @@ lyc_status lyc_create(const lyc_config* cfg, lyc_ctx** out) {
   const lyc_config& c = *cfg;
   if (c.num_layers < 1 || c.batch < 1 || c.num_q_heads < 1 || c.num_kv_heads < 1 ||
       c.num_q_heads % c.num_kv_heads != 0 || c.max_ctx < 1 || c.max_k < 1 ||
-      (c.flags & ~LYC_CFG_TMA_GATHER) != 0)
+      (c.flags & ~(LYC_CFG_TMA_GATHER | LYC_CFG_TCGEN05)) != 0)
     return LYC_ERR_INVALID_ARG;
   if (c.dtype != LYC_BF16 && c.dtype != LYC_FP32) return LYC_ERR_INVALID_ARG;
   if (c.select_mode != LYC_SELECT_PER_QHEAD && c.select_mode != LYC_SELECT_KVGROUP_MEAN)
@@ -910,6 +924,7 @@ lyc_status lyc_create(const lyc_config* cfg, lyc_ctx** out) {
   if (dtype == 0) {
     int smem = 0;
     e = attn_mma_dispatch(D, nullptr, 0, nullptr, &smem, true);
+    if (e == cudaSuccess && D == 128) e = attn_tc_dispatch(nullptr, 0, nullptr, &smem, true);
   } else {
     e = cudaSuccess;
     for (int nqb : {1, 2, 4, 8}) {

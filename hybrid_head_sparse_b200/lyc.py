@@ -34,6 +34,7 @@ LYC_SELECT_PER_QHEAD = 0
 LYC_SELECT_KVGROUP_MEAN = 1
 
 LYC_CFG_TMA_GATHER = 0x1
+LYC_CFG_TCGEN05 = 0x2
 
 LYC_STEP_S_IN = 0x1
 LYC_STEP_NO_GRAPH = 0x2

@@ -12,8 +12,9 @@ n in {4K, 16K, 64K, 256K, 512K}, budget k in {256, 1024, 4096, 8192}.
   sorted.  Bytes = the K and V rows of every pass: one pass per query head in
   per-head selection mode, one per KV group in group mode.
 
-Each case is timed with CUDA events around the attention launch (the library's
-timing mode) over R replays of the captured step, with the L2 flushed (a
+Each case is timed with CUDA events around the attention launches (the
+library's timing mode: the layer's launch and the small launch that combines
+its split rows) over R replays of the captured step, with the L2 flushed (a
 256 MiB write) before every replay.  One JSON line per case goes to stdout.
 
 Usage: python -m hybrid_head_sparse_b200.sweep [--quick] [--gather cp_async|tma]
@@ -48,8 +49,9 @@ def measured_hbm_gbs() -> float | None:
 
 
 def attn_ms(ctx, run, flush, reps: int):
-    """Mean CUDA-event time of the attention launch (and of the selection
-    launch, if any) over `reps` replays, L2 flushed before each."""
+    """CUDA-event time per replay of the attention launches (the layer's, plus
+    the launch that combines its split rows) and of the selection launch, if
+    any, over `reps` replays, L2 flushed before each."""
     ctx.set_timing(True)
     run()
     torch.cuda.synchronize()
@@ -60,9 +62,9 @@ def attn_ms(ctx, run, flush, reps: int):
     torch.cuda.synchronize()
     t = ctx.kernel_times()
     ctx.set_timing(False)
-    a = [x[2] for x in t if x[0] == 0]
+    a = sum(x[2] for x in t if x[0] == 0) / reps
     s = [x[2] for x in t if x[0] == 1]
-    return float(np.mean(a)), (float(np.mean(s)) if s else None)
+    return float(a), (float(sum(s) / reps) if s else None)
 
 
 def main(argv=None) -> int:

@@ -82,6 +82,14 @@ typedef struct {
  * s_token, under 2^31 rows); without one the library uses cp.async anyway.
  * Results are the same either way. */
 #define LYC_CFG_TMA_GATHER 0x1u
+/* cfg.flags: run bf16 attention with head_dim 128 on the tcgen05 tensor-core
+ * kernel (accumulators in tensor memory, 128-row tiles, one MMA-issuing
+ * thread) instead of the mma.sync kernel (64-row tiles, register
+ * accumulators, six consumer warps).  Measured on B200 the mma.sync kernel is
+ * faster for this path (it keeps more bytes in flight per SM: six 32 KiB
+ * stages consumed in parallel against three 64 KiB stages consumed in turn),
+ * so it is the default; results agree within rounding. */
+#define LYC_CFG_TCGEN05 0x2u
 
 /* The KV cache of all layers.  Element (l, b, g, i, j) of K (and of V) is at
  * element offset l*s_layer + b*s_batch + g*s_head + i*s_token + j, j < d

@@ -20,17 +20,20 @@ def lyc():
     return lycmod
 
 
-GATHERS = ["cp_async", "tma"]
+# bf16 attention kernels: "cp_async" (mma.sync with cp.async gathers, the
+# default), "tma" (mma.sync with TMA gathers), "tc" (tcgen05, head_dim 128)
+GATHERS = ["cp_async", "tma", "tc"]
 
 
 def run_step(lyc, spec: W.StackSpec, select_mode="per_qhead", data=None, s_in=None,
              no_graph=False, k=None, n=None, gather="cp_async"):
     """One library step on the spec's inputs; returns (data, out, S, trace) on the host.
-    gather: "cp_async" (the default) or "tma" (four-row TMA gathers where the layout allows)."""
+    gather: "cp_async" (the default mma.sync kernel), "tma" (the mma.sync kernel
+    with four-row TMA gathers where the layout allows) or "tc" (the tcgen05 kernel)."""
     data = data or W.make_stack(spec, "cuda")
     k = k or spec.k
     n = n or spec.n
-    flags = lyc.LYC_CFG_TMA_GATHER if gather == "tma" else 0
+    flags = {"cp_async": 0, "tma": lyc.LYC_CFG_TMA_GATHER, "tc": lyc.LYC_CFG_TCGEN05}[gather]
     ctx = lyc.Lyc(spec.L, spec.B, spec.Hq, spec.Hkv, spec.d, max(spec.rows, n), k,
                   dtype=spec.dtype, select_mode=select_mode, flags=flags)
     Hs = ctx.Hs
@@ -220,7 +223,7 @@ def test_bad_inherited_index_reported_bf16(lyc, gather):
     data = W.make_stack(spec, "cuda")
     data["role"] = np.array([[1, 0]], dtype=np.uint8)
     S0 = torch.arange(70, dtype=torch.int32, device="cuda").repeat(1, 2, 1).contiguous()
-    flags = lyc.LYC_CFG_TMA_GATHER if gather == "tma" else 0
+    flags = {"cp_async": 0, "tma": lyc.LYC_CFG_TMA_GATHER, "tc": lyc.LYC_CFG_TCGEN05}[gather]
     ctx = lyc.Lyc(1, 1, 2, 1, 128, 300, 70, flags=flags)
     out = torch.zeros((1, 1, 2, 128), device="cuda")
     for bad in (300, -3):
@@ -330,9 +333,9 @@ def test_strided_rows_bf16(lyc, gather):
 # with teacher forcing (each checked layer inherits the GPU's own sets).
 
 
-def _full_size(lyc, spec, layers, mode="per_qhead"):
+def _full_size(lyc, spec, layers, mode="per_qhead", gather="cp_async"):
     om = O.SELECT_PER_QHEAD if mode == "per_qhead" else O.SELECT_KVGROUP_MEAN
-    data, out, S, tr = run_step(lyc, spec, select_mode=mode)
+    data, out, S, tr = run_step(lyc, spec, select_mode=mode, gather=gather)
     assert np.isfinite(out).all()
     P.check_layers(data, out, tr, spec.k, spec.n, spec.dtype, layers, select_mode=om)
     assert np.array_equal(S, tr[-1])
@@ -344,10 +347,11 @@ def test_llama3_8b_32k_full_step(lyc):
     _full_size(lyc, W.LLAMA3_8B_32K, [0, 1, 2, 17, 31])
 
 
+@pytest.mark.parametrize("gather", ["cp_async", "tc"])
 @pytest.mark.parametrize("mode", ["per_qhead", "kvgroup_mean"])
-def test_llama3_8b_128k_first_layers(lyc, mode):
+def test_llama3_8b_128k_first_layers(lyc, mode, gather):
     # the 128K stack's first 6 layers (same shapes per layer as the full 32)
-    _full_size(lyc, W.LLAMA3_8B_128K.with_(L=6), [0, 1, 5], mode)
+    _full_size(lyc, W.LLAMA3_8B_128K.with_(L=6), [0, 1, 5], mode, gather)
 
 
 def test_qwen3_8b_64k_batch4(lyc):

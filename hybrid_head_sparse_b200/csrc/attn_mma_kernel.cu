@@ -7,9 +7,10 @@
 //   sparse rows, section 3.4 Eq. (3): the same over the rows of the set they
 //   inherit,
 // plus the selection key of every cached row for the sets refreshed at this
-// layer (Eq. 2 then runs in topk_kernel.cu), and merges the pieces of each
-// segment with log-sum-exp in the last piece to finish (Appendix C,
-// Algorithm 2 steps 5-6, without a second launch).
+// layer (Eq. 2 then runs in topk_kernel.cu).  The pieces of a segment cut
+// over several CTAs are merged with log-sum-exp (Appendix C, Algorithm 2
+// steps 5-6) by the epilogue warps of the next launch, so no CTA waits for
+// another's partials.
 //
 // Design (B200 / sm_100a):
 //   * decode attention reads every K/V byte once and does 2-8 flop per byte:
@@ -54,10 +55,11 @@ struct AttnMmaParams {
 
 template <int D, int NC, int NP, int STAGES, bool GT>
 struct MmaCfg {
-  // warps: NC consumers, one epilogue warp, NP producers
-  static constexpr int kThreads = (NC + 1 + NP) * 32;
+  // warps: NC consumers, one epilogue warp, one scheduler warp, NP producers
+  static constexpr int kThreads = (NC + 2 + NP) * 32;
   static constexpr int kProducerThreads = NP * 32;
-  static constexpr int kFirstProducer = (NC + 1) * 32;  // thread index
+  static constexpr int kScheduler = (NC + 1) * 32;      // thread index of its warp
+  static constexpr int kFirstProducer = (NC + 2) * 32;  // thread index
   // arrivals that complete a full barrier: with row gathers by TMA the one
   // leader thread arms every tile; otherwise every producer thread arrives
   static constexpr int kFullCount = GT ? 1 : NP * 32;
@@ -65,8 +67,6 @@ struct MmaCfg {
   static constexpr int BLOCKB = kTileRows * 128;           // one swizzled 64 x 128 B block
   static constexpr int TILEB = HALVES * BLOCKB;            // K (or V) tile bytes
   static constexpr int IR = 16;                            // index ring slots
-  static constexpr int LA = 7;                             // index lookahead (tiles)
-  static_assert(IR > LA + STAGES, "index ring too small for the lookahead");
   static_assert(kTileRows % (2 * NP) == 0, "rows per producer warp");
   // Tile t sits in stage t % STAGES and is consumed by warp t % NC.  With
   // STAGES a multiple of NC every stage belongs to one consumer warp, which
@@ -75,15 +75,46 @@ struct MmaCfg {
   // parity wait cannot match a phase that has not started.
   static_assert(STAGES % NC == 0, "each stage must belong to one consumer warp");
   static_assert(NC <= kMaxConsumerWarps, "piece-state ring sized for kMaxConsumerWarps");
+  // warps that read the pool ring (all but the scheduler, which writes it)
+  static constexpr int kRingReaders = NC + 1 + NP;
   // shared memory (bytes from a 1024-aligned base)
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = OFF_K + STAGES * TILEB;
   static constexpr int OFF_IDX = OFF_V + STAGES * TILEB;
   static constexpr int OFF_BAR = OFF_IDX + IR * kTileRows * 4;
-  // barriers: full[STAGES], empty[STAGES], idx[IR], slot_full[PS], slot_free[PS]
-  static constexpr int OFF_FLAGS = OFF_BAR + (2 * STAGES + IR + 2 * kPartSlots) * 8;
-  static constexpr int SMEM = OFF_FLAGS + 16 + 1024;  // + alignment slack
+  // barriers: full[STAGES], empty[STAGES], idx[IR], slot_full[PS], slot_free[PS],
+  // unit_full[R], unit_empty[R], idx_free[IR]
+  static constexpr int BAR_UNIT = 2 * STAGES + IR + 2 * kPartSlots;
+  static constexpr int BAR_IDXFREE = BAR_UNIT + 2 * kPoolRing;
+  static constexpr int OFF_FLAGS = OFF_BAR + (BAR_IDXFREE + IR) * 8;
+  static constexpr int OFF_RING = OFF_FLAGS + 16;  // kPoolRing pool pieces
+  static constexpr int SMEM = OFF_RING + kPoolRing * 16 + 1024;  // + alignment slack
 };
+
+// Piece i of the CTA, for every warp but the scheduler: its own pieces
+// first, then the pool pieces the scheduler took, from the ring (false at the
+// end of both).  Each warp calls it for i = 0, 1, ... in order.
+template <class C>
+__device__ __forceinline__ bool cta_piece(const AttnParams& p, unsigned char* smem, int pbeg, int nhome,
+                                          int i, int lane, Piece* out) {
+  if (i < nhome) {
+    *out = p.pieces[pbeg + i];
+    return true;
+  }
+  if (p.pool_n <= 0) return false;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* unit_full = bars + C::BAR_UNIT;
+  uint64_t* unit_empty = unit_full + kPoolRing;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_FLAGS);
+  const int k = i - nhome;
+  const int r = k % kPoolRing;
+  if (!mbar_wait(&unit_full[r], (k / kPoolRing) & 1, abort_flag, p.status)) return false;
+  const Piece pc = reinterpret_cast<const Piece*>(smem + C::OFF_RING)[r];
+  __syncwarp();
+  if (lane == 0) mbar_arrive(&unit_empty[r]);
+  *out = pc;
+  return pc.seg >= 0;
+}
 
 // ---------------------------------------------------------------- PTX helpers
 __device__ __forceinline__ void ldsm_x4(uint32_t* r, uint32_t addr) {
@@ -158,6 +189,102 @@ __device__ __forceinline__ uint32_t swz(int r, int ch) {
 
 namespace lyc {
 
+// ---------------------------------------------------------------- scheduler
+// One thread walks the CTA's pieces ahead of the producers: its own pieces,
+// then pool units it takes by the launch's atomic cursor, each published as a
+// ring entry, ending with an entry of segment -1.  For every gathered tile it
+// copies the tile's slice of the index list into the index ring (a bulk
+// copy) once the ring slot is free, i.e. once the tile IR places earlier has
+// been consumed; a pool unit is taken at that same point for its first tile,
+// so every CTA holds about IR tiles of work ahead, however early it started.
+// Before the first tile of a set written by a selection of this step it
+// waits for that selection's ready flag.  Its waits hold up no copy issue.
+template <int D, int NC, int NP, int STAGES, bool GT>
+__device__ __forceinline__ void mma_scheduler(const AttnMmaParams& P, unsigned char* smem, int pbeg,
+                                              int pend) {
+  using C = MmaCfg<D, NC, NP, STAGES, GT>;
+  const AttnParams& p = P.p;
+  int32_t* idxring = reinterpret_cast<int32_t*>(smem + C::OFF_IDX);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* idxbar = bars + 2 * STAGES;
+  uint64_t* unit_full = bars + C::BAR_UNIT;
+  uint64_t* unit_empty = unit_full + kPoolRing;
+  uint64_t* idx_free = bars + C::BAR_IDXFREE;
+  Piece* ring = reinterpret_cast<Piece*>(smem + C::OFF_RING);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_FLAGS);
+  const int nhome = pend - pbeg;
+  int32_t* cursor = p.pool_n > 0
+                        ? p.pool_cursors + static_cast<int64_t>(*p.epoch & 1u) * p.pool_stride + p.layer
+                        : nullptr;
+  // Slot of tile tt in the index ring is free once tile tt - IR is consumed.
+  // The scheduler waits on every tile in order, dense ones included: a
+  // parity wait tells phases apart only when the waiter is at most one phase
+  // ahead of the barrier.
+  auto slot_free = [&](int tt) {
+    return tt < C::IR || mbar_wait(&idx_free[tt % C::IR], ((tt / C::IR) - 1) & 1, abort_flag, p.status);
+  };
+  const uint32_t* acquired = nullptr;  // the last ready flag waited on
+  bool waited = false;                 // the previous launch has completed
+  int t = 0;                           // CTA-wide tile sequence number
+  for (int i = 0;; ++i) {
+    Piece pc;
+    if (i < nhome) {
+      pc = p.pieces[pbeg + i];
+    } else {
+      if (!cursor) break;
+      const int k = i - nhome;
+      const int r = k % kPoolRing;
+      if (!slot_free(t)) break;
+      if (k >= kPoolRing && !mbar_wait(&unit_empty[r], ((k / kPoolRing) - 1) & 1, abort_flag, p.status))
+        break;
+      const int u = atomicAdd(cursor, 1);
+      if (u < p.pool_n) {
+        const int q = u % p.pool_ups;
+        pc.seg = __ldg(&p.pool_segs[u / p.pool_ups]);
+        pc.r0 = q * (kPoolTiles * kTileRows);
+        pc.r1 = min(pc.r0 + kPoolTiles * kTileRows, p.pool_rows);
+        pc.ordinal = q;
+      } else {
+        pc.seg = -1;
+        pc.r0 = pc.r1 = pc.ordinal = 0;
+      }
+      ring[r] = pc;
+      mbar_arrive(&unit_full[r]);  // release: the entry above
+      if (pc.seg < 0) break;
+    }
+    const Segment& sg = p.segs[pc.seg];
+    if (sg.kind != kSparse) {
+      for (int r0 = pc.r0; r0 < pc.r1; r0 += kTileRows, ++t)
+        if (!slot_free(t)) return;
+      continue;
+    }
+    // A set that a selection of this step writes is read once that
+    // selection has raised its ready flag (the selection may still be
+    // running).  Otherwise a set the previous launch writes is read once
+    // that launch has completed.  The bulk copies read the set through the
+    // async proxy, hence the proxy fence after the acquire.
+    if (sg.ready) {
+      if (sg.ready != acquired) {
+        wait_flag(sg.ready, *p.epoch + 1u, abort_flag, p.status);
+        fence_proxy_async_global();
+        acquired = sg.ready;
+      }
+    } else if (sg.dep && !waited) {
+      pdl_wait();
+      waited = true;
+    }
+    for (int r0 = pc.r0; r0 < pc.r1; r0 += kTileRows, ++t) {
+      const int slot = t % C::IR;
+      if (!slot_free(t)) return;
+      const int nrows = min(kTileRows, pc.r1 - r0);
+      const uint32_t bytes = static_cast<uint32_t>(((nrows * 4) + 15) & ~15);
+      fence_proxy_async_smem();
+      mbar_arrive_expect_tx(&idxbar[slot], bytes);
+      bulk_g2s(idxring + slot * kTileRows, sg.idx + r0, bytes, &idxbar[slot]);
+    }
+  }
+}
+
 // ---------------------------------------------------------------- producers
 // NP warps walk the CTA's tiles together.  Dense tile: one thread issues the
 // TMA copies, everyone arrives.  Gathered tile: warp pw copies rows
@@ -183,45 +310,15 @@ __device__ __forceinline__ void mma_producers(const AttnMmaParams& P, unsigned c
   const uint64_t pol_keep = l2_policy_evict_normal();  // gathered rows may be read again
   const bool leader = ptid == 0;
 
-  // lookahead cursor (leader only): index-list copies of gathered tiles, LA tiles early
-  int la_pc = pbeg, la_r0 = (pbeg < pend) ? p.pieces[pbeg].r0 : 0, la_t = 0;
-  bool waited = false;  // the previous launch (a selection) has completed
-  auto la_step = [&]() {
-    if (la_pc >= pend) return;
-    const Piece pc = p.pieces[la_pc];
-    const Segment& ls = p.segs[pc.seg];
-    if (ls.kind == kSparse) {
-      // a set the previous launch writes is read only once it has completed;
-      // sets of earlier selections were complete before that launch began
-      // (each selection waits for the attention before it, which waits for
-      // the selection before it), and the bulk copy reads them at L2
-      if (ls.dep && !waited) {
-        pdl_wait();
-        waited = true;
-      }
-      const int slot = la_t % C::IR;
-      const int nrows = min(kTileRows, pc.r1 - la_r0);
-      const uint32_t bytes = static_cast<uint32_t>(((nrows * 4) + 15) & ~15);
-      fence_proxy_async_smem();
-      mbar_arrive_expect_tx(&idxbar[slot], bytes);
-      bulk_g2s(idxring + slot * kTileRows, p.segs[pc.seg].idx + la_r0, bytes, &idxbar[slot]);
-    }
-    ++la_t;
-    la_r0 += kTileRows;
-    if (la_r0 >= pc.r1) {
-      ++la_pc;
-      if (la_pc < pend) la_r0 = p.pieces[la_pc].r0;
-    }
-  };
-  if (leader)
-    for (int a = 0; a < C::LA; ++a) la_step();
+  const int nhome = pend - pbeg;
 
   constexpr int CH = D / 8;                  // 16-byte chunks per row
   constexpr int ROWS_W = kTileRows / NP;     // rows per producer warp
   uint32_t idx_phase = 0;
   int t = 0;
-  for (int pcI = pbeg; pcI < pend; ++pcI) {
-    const Piece pc = p.pieces[pcI];
+  for (int pi = 0;; ++pi) {
+    Piece pc;
+    if (!cta_piece<C>(p, smem, pbeg, nhome, pi, lane, &pc)) break;
     const Segment& sg = p.segs[pc.seg];
     const bool dense = sg.kind == kDense;
     const int64_t s_token = sg.s_token;
@@ -229,7 +326,6 @@ __device__ __forceinline__ void mma_producers(const AttnMmaParams& P, unsigned c
     const bf16_t* vb = static_cast<const bf16_t*>(sg.v);
     const int sl = sg.l, sb = sg.b, sgg = sg.g;
     for (int r0 = pc.r0; r0 < pc.r1; r0 += kTileRows, ++t) {
-      if (leader) la_step();
       const int nrows = min(kTileRows, pc.r1 - r0);
       const int stage = t % STAGES;
       if (t >= STAGES) {
@@ -311,6 +407,13 @@ __device__ __forceinline__ void mma_producers(const AttnMmaParams& P, unsigned c
 
 namespace lyc {
 
+// The ring of piece states this CTA uses: the SM's own when CTAs of two
+// launches may run at once (a CTA of this kernel has the SM to itself: the
+// shared memory of two does not fit), else the block's.
+__device__ __forceinline__ int cta_ring(const AttnParams& p) {
+  return p.wpart_by_sm ? static_cast<int>(sm_index()) : static_cast<int>(blockIdx.x);
+}
+
 // ---------------------------------------------------------------- consumers
 // Fragment bookkeeping (m16n8k16, g = lane/4, c = lane%4):
 //   S^T tile mt (16 keys):  st[mt][0..1] = keys 16mt+g,   queries 2c, 2c+1
@@ -341,14 +444,16 @@ __device__ __forceinline__ void mma_consumers(const AttnMmaParams& P, unsigned c
   uint64_t* empty = bars + STAGES;
   uint64_t* slot_full = bars + 2 * STAGES + C::IR;
   uint64_t* slot_free = slot_full + kPartSlots;
+  uint64_t* idx_free = bars + C::BAR_IDXFREE;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_FLAGS);
   const bf16_t* q = static_cast<const bf16_t*>(p.q);
   const float sl2 = p.scale_log2;
   const int mi = lane >> 3, r8 = lane & 7;  // ldmatrix: matrix and row this lane addresses
 
   int t = 0;  // CTA-wide tile sequence number
-  for (int pcI = pbeg; pcI < pend; ++pcI) {
-    const Piece pc = p.pieces[pcI];
+  for (int pi = 0;; ++pi) {
+    Piece pc;
+    if (!cta_piece<C>(p, smem, pbeg, pend - pbeg, pi, lane, &pc)) break;
     const Segment& sg = p.segs[pc.seg];
     const int nq = sg.nq, nout = sg.nout, b = sg.b;
     const bool dense = sg.kind == kDense;
@@ -499,7 +604,10 @@ __device__ __forceinline__ void mma_consumers(const AttnMmaParams& P, unsigned c
         }
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[stage]);
+      if (lane == 0) {
+        mbar_arrive(&empty[stage]);
+        mbar_arrive(&idx_free[t % C::IR]);  // the tile's index slice is no longer read
+      }
     }
 
     // ---- hand this warp's state of the piece to the epilogue warp: slot
@@ -510,11 +618,10 @@ __device__ __forceinline__ void mma_consumers(const AttnMmaParams& P, unsigned c
         l0 += __shfl_xor_sync(FULL, l0, s2);
         l1 += __shfl_xor_sync(FULL, l1, s2);
       }
-      const int pi = pcI - pbeg;
       const int slot = pi % kPartSlots;
       if (pi >= kPartSlots)
         mbar_wait(&slot_free[slot], ((pi / kPartSlots) - 1) & 1, abort_flag, p.status);
-      const int64_t rec = ((static_cast<int64_t>(blockIdx.x) * kPartSlots + slot) * NC + w) * kMaxQ;
+      const int64_t rec = ((static_cast<int64_t>(cta_ring(p)) * kPartSlots + slot) * NC + w) * kMaxQ;
       if (g == 0) {
         if (out0) p.wpart_ml[rec + q0] = make_float2(m0, l0);
         if (out1) p.wpart_ml[rec + q1] = make_float2(m1, l1);
@@ -603,9 +710,19 @@ __device__ __forceinline__ void mma_epilogue(const AttnMmaParams& P, unsigned ch
   uint64_t* slot_free = slot_full + kPartSlots;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_FLAGS);
 
-  // ---- 1. the previous layer's cross-piece combine (after that launch has
-  // completed: the launch just before this one may be it)
-  if (p.prev_ntasks > 0) pdl_wait();
+  // ---- 1. the previous layer's cross-piece combine, after that launch has
+  // completed.  The wait also comes before any partial of this launch is
+  // written: this launch may start while the previous attention launch still
+  // runs, and that launch reads the partials of the layer before it, which
+  // share this launch's buffer.  With a flag for it, wait on the flag (the
+  // selection in between may still run); else on griddepcontrol.wait, which
+  // returns once every earlier launch of the chain has completed.
+  if (p.prev_done) {
+    if (lane == 0) wait_flag(p.prev_done, *p.epoch + 1u, abort_flag, p.status);
+    __syncwarp();
+  } else {
+    pdl_wait();
+  }
   for (int t = blockIdx.x; t < p.prev_ntasks; t += gridDim.x) {
     const int2 task = p.prev_tasks[t];
     const Segment& sg = p.prev_segs[task.x];
@@ -631,14 +748,14 @@ __device__ __forceinline__ void mma_epilogue(const AttnMmaParams& P, unsigned ch
   }
 
   // ---- 2. this layer's pieces
-  for (int pcI = pbeg; pcI < pend; ++pcI) {
-    const Piece pc = p.pieces[pcI];
+  for (int pi = 0;; ++pi) {
+    Piece pc;
+    if (!cta_piece<C>(p, smem, pbeg, pend - pbeg, pi, lane, &pc)) break;
     const Segment& sg = p.segs[pc.seg];
     const int nout = sg.nout;
-    const int pi = pcI - pbeg;
     const int slot = pi % kPartSlots;
     if (!mbar_wait(&slot_full[slot], (pi / kPartSlots) & 1, abort_flag, p.status)) return;
-    const int64_t rec0 = (static_cast<int64_t>(blockIdx.x) * kPartSlots + slot) * NC * kMaxQ;
+    const int64_t rec0 = (static_cast<int64_t>(cta_ring(p)) * kPartSlots + slot) * NC * kMaxQ;
     // load every output's NC warp states first (all in flight), then merge
     for (int o0 = 0; o0 < nout; o0 += 2) {
       float2 ml[2][NC];
@@ -696,6 +813,11 @@ __global__ void __launch_bounds__(MmaCfg<D, NC, NP, STAGES, GT>::kThreads, 1)
       mbar_init(&bars[2 * STAGES + C::IR + r], NC);  // slot full: every consumer warp
       mbar_init(&bars[2 * STAGES + C::IR + kPartSlots + r], 1);  // slot free: the epilogue warp
     }
+    for (int r = 0; r < kPoolRing; ++r) {
+      mbar_init(&bars[C::BAR_UNIT + r], 1);                             // unit full: the scheduler
+      mbar_init(&bars[C::BAR_UNIT + kPoolRing + r], C::kRingReaders);  // unit empty: every reader
+    }
+    for (int r = 0; r < C::IR; ++r) mbar_init(&bars[C::BAR_IDXFREE + r], 1);  // the tile's consumer
     *reinterpret_cast<int*>(smem + C::OFF_FLAGS) = 0;
     fence_mbar_init();
   }
@@ -710,19 +832,37 @@ __global__ void __launch_bounds__(MmaCfg<D, NC, NP, STAGES, GT>::kThreads, 1)
   __syncthreads();
   pdl_launch_dependents();
   if (P.p.wait_prev) pdl_wait();  // the previous launch writes what this one reads or writes
-  const int pbeg = P.p.cta_begin[blockIdx.x];
-  const int pend = P.p.cta_begin[blockIdx.x + 1];
-  if (threadIdx.x >= C::kFirstProducer) {
-    mma_producers<D, NC, NP, STAGES, GT>(P, smem, pbeg, pend);
-  } else if (threadIdx.x >= NC * 32) {
-    mma_epilogue<D, NC, NP, STAGES, GT>(P, smem, pbeg, pend);
+  static_assert(2 * C::SMEM > 232448, "the per-SM ring needs one CTA per SM");
+  if (cta_ring(P.p) >= P.p.wpart_slots) {
+    if (threadIdx.x == 0) atomicOr(P.p.status, kStatusScratch);
   } else {
-    mma_consumers<D, NC, NP, STAGES, GT>(P, smem, pbeg, pend);
+    const int pbeg = P.p.cta_begin[blockIdx.x];
+    const int pend = P.p.cta_begin[blockIdx.x + 1];
+    if (threadIdx.x >= C::kFirstProducer) {
+      mma_producers<D, NC, NP, STAGES, GT>(P, smem, pbeg, pend);
+    } else if (threadIdx.x >= C::kScheduler) {
+      if (threadIdx.x == C::kScheduler) mma_scheduler<D, NC, NP, STAGES, GT>(P, smem, pbeg, pend);
+    } else if (threadIdx.x >= NC * 32) {
+      mma_epilogue<D, NC, NP, STAGES, GT>(P, smem, pbeg, pend);
+    } else {
+      mma_consumers<D, NC, NP, STAGES, GT>(P, smem, pbeg, pend);
+    }
+  }
+  // every write of the CTA is done (and fenced) before its arrival on the
+  // launch's done counter; the last CTA to arrive raises the flag
+  if (P.p.done) __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0 && P.p.done) {
+    const uint32_t prev = atomicAdd(&P.p.done[0], 1u);
+    if (prev == gridDim.x - 1) {
+      P.p.done[0] = 0u;
+      __threadfence();
+      st_release_u32(&P.p.done[1], *P.p.epoch + 1u);
+    }
   }
   // this grid completes only after the one it depends on (dense-only CTAs
   // never waited above), so completion order follows launch order; the
   // timeline's end is the end of the CTA's last warp
-  if (P.p.timeline) __syncthreads();
   if (threadIdx.x == 0) {
     pdl_wait();
     timeline_record(P.p.timeline, P.p.timeline_cap, t_start,

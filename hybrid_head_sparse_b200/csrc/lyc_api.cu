@@ -54,6 +54,7 @@ namespace {
 constexpr int kMaxCtxLimit = 655360;  // 16-CTA top-k keeps every key in shared memory
 constexpr int kPlanCacheSize = 16;
 
+
 int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
 
 // One layer of a plan: offsets of its records in the plan's device buffer.
@@ -65,6 +66,9 @@ struct LayerPlan {
   size_t off_trace_src = 0;  // copy table for the set trace after this layer
   size_t off_combine = 0;    // bf16: (segment, output) pairs combined by the next launch
   int ncombine = 0;
+  size_t off_pool = 0;       // mma kernel: the pool's segments
+  int pool_nsegs = 0, pool_ups = 0;
+  int64_t pool_tiles = 0, tiles = 0;  // tiles in the pool, in the whole layer
   int topk_cl = 16;          // cluster size of the selection launch
 };
 
@@ -114,6 +118,14 @@ struct lyc_ctx {
   // bf16 path: per CTA ring of the consumer warps' piece states
   float* wpart_o = nullptr;
   float2* wpart_ml = nullptr;
+  int wpart_slots = 0;
+  // per (layer, b, slot): {arrival counter, ready flag} of the selection task
+  // that writes the slot at that layer; then per layer the same pair for the
+  // attention launch; then the step epoch
+  uint32_t* flags = nullptr;
+  uint32_t* attn_flags = nullptr;
+  int32_t* pool_cursors = nullptr;  // [2][L + 1], by epoch parity
+  uint32_t* epoch = nullptr;
   int32_t* counters = nullptr;
   size_t max_parts = 0, max_counters = 0;
   // host-buffer entry point staging
@@ -253,9 +265,10 @@ lyc_status encode_gather_map(lyc_ctx* ctx, CUtensorMap* map, const void* base, c
 
 // Cluster size of a selection launch of `ntasks` sets.  A small selection (a
 // few sets) runs beside the next layer's attention, on SMs the planner takes
-// from that attention: clusters of 8 (measured on B200 at 128K keys: the best
-// balance between the selection's latency, which the next layer's dense rows
-// hide, and the SMs taken from the attention; 16 takes twice the SMs, 4 takes
+// from that attention: clusters of 16 where they fit, else 8.  The next
+// attention launch has CTAs that take those SMs back (pool units only) once
+// the selection is done, so a faster selection costs it little (measured on
+// B200 at 128K keys: 16 beats 8 by ~1% with the overlapped launches; 4 takes
 // longer than the dense rows last).  A large selection (layer 0) takes the
 // largest size whose clusters are all resident at once, so that it runs in
 // one wave and the next layer starts right away; else the smallest size.
@@ -263,6 +276,7 @@ int pick_topk_cluster(const lyc_ctx* ctx, int ntasks) {
   auto resident = [&](int cl) {
     return ctx->topk_resident[cl] > 0 ? ctx->topk_resident[cl] : ctx->sms / cl;
   };
+  if (ntasks * 16 <= ctx->sms / 4 && (ctx->topk_cls & (1u << 16)) && ntasks <= resident(16)) return 16;
   if (ntasks * 16 <= ctx->sms / 4 && (ctx->topk_cls & (1u << 8)) && ntasks <= resident(8)) return 8;
   int best = 0, smallest = 0;
   for (int cl : {16, 8, 4}) {
@@ -300,6 +314,9 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const lyc_k
   plan->use_tc = cfg.dtype == LYC_BF16 && cfg.head_dim == 128 && (cfg.flags & LYC_CFG_TCGEN05) &&
                  !(cfg.flags & LYC_CFG_TMA_GATHER) && (reinterpret_cast<uintptr_t>(plan->q) & 15u) == 0;
   const int TR = plan->use_tc ? attn_tc_tile_rows() : kTileRows;
+  // the mma kernel takes gathered rows from a pool at run time (its launches
+  // of consecutive layers may overlap, see enqueue)
+  const bool use_pool = cfg.dtype == LYC_BF16 && !plan->use_tc;
   if (cfg.dtype == LYC_BF16) {
     lyc_status st = encode_cache_map(ctx, &plan->tmk, kv->k, kv, TR);
     if (st == LYC_OK) st = encode_cache_map(ctx, &plan->tmv, kv->v, kv, TR);
@@ -323,6 +340,9 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const lyc_k
     int nqb = 1;
     int grid = 0;
     int topk_cl = 16;           // cluster size of this layer's selection launch
+    std::vector<int32_t> pool_segs;  // mma kernel: segments of the pool, in order
+    int pool_ups = 0;                // units per pool segment
+    int64_t tiles = 0, pool_tiles = 0;
   };
   std::vector<HostLayer> hl(L);
   std::vector<int> cur(Hs, 0);
@@ -333,11 +353,17 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const lyc_k
   const char* vbase = static_cast<const char*>(kv->v);
 
   std::vector<char> prev_fresh(Hs, 1);  // slots the previous layer's selection wrote
+  std::vector<int> writer(Hs, -1);      // layer whose selection wrote each slot's current set
+  auto ready_flag = [&](int s, int b) -> const uint32_t* {
+    if (writer[s] < 0) return nullptr;
+    return ctx->flags + ((static_cast<int64_t>(writer[s]) * B + b) * Hs + s) * 2 + 1;
+  };
   for (int l = 0; l < L; ++l) {
     HostLayer& H = hl[l];
-    // selection keys alternate between two buffers by layer, so a layer's
-    // attention never writes the keys the previous layer's selection reads
-    const int64_t keys_base = (l & 1) * static_cast<int64_t>(B) * Hs * ctx->nstride;
+    // every layer has key rows of its own, so no attention launch writes keys
+    // that an earlier selection may still read (launches of consecutive
+    // layers may overlap in time)
+    const int64_t keys_base = l * static_cast<int64_t>(B) * Hs * ctx->nstride;
     std::vector<char> is_ret(Hq), fresh(Hs, 0);
     for (int h = 0; h < Hq; ++h) {
       is_ret[h] = (l == 0 && !s_in) || role[static_cast<int64_t>(l) * Hq + h] != 0;
@@ -398,6 +424,7 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const lyc_k
           if (js > 0) {
             ss.nq = ss.nout = js;
             ss.dep = prev_fresh[g];
+            ss.ready = ready_flag(g, b);
             maxnq = std::max(maxnq, js);
             H.segs.push_back(ss);
           }
@@ -412,6 +439,7 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const lyc_k
             ss.out_row[0] = 0;
             ss.nq = ss.nout = 1;
             ss.dep = prev_fresh[h];
+            ss.ready = ready_flag(h, b);
             H.segs.push_back(ss);
           }
         }
@@ -419,13 +447,17 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const lyc_k
     }
     H.nqb = attn_nq_bucket(maxnq);
 
-    // workload pooling (two phases): the dense rows are cut into equal runs
-    // of 64-row tiles, one per CTA, and so are the gathered rows; CTA c takes
-    // its dense run, then its gathered run, so every CTA carries the same mix
-    // whatever the relative cost of streaming and gathering a tile.  The
-    // gathered rows list the sets that an earlier layer's selection wrote
-    // first and those the previous layer's selection writes (the only rows
-    // that wait for it) last, so that few CTAs wait, and late.
+    // Workload pooling.  The dense rows are cut into equal runs of tiles, one
+    // per CTA.  The gathered rows:
+    //  * mma kernel: go to a pool of kPoolTiles-tile units, which the CTAs
+    //    take at run time once their dense run is done (an atomic cursor per
+    //    launch), sets of earlier selections first, those the previous
+    //    layer's selection writes (the only rows that wait for it) last.  A
+    //    CTA that starts late (the launches of consecutive layers overlap) or
+    //    streams slowly then simply takes fewer units;
+    //  * other kernels: are cut into equal runs too, taken after the dense
+    //    run, the previous selection's sets last, so that few CTAs wait, and
+    //    late.
     int64_t NT = 0;
     for (const Segment& sg : H.segs) NT += (sg.rows + TR - 1) / TR;
     // The previous layer's selection runs beside this layer's attention (the
@@ -438,11 +470,16 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const lyc_k
       const int prev = static_cast<int>(hl[l - 1].tasks.size()) * hl[l - 1].topk_cl;
       if (prev > 0 && prev <= ctx->sms / 4) avail = ctx->sms - prev;
     }
-    const int grid = static_cast<int>(std::min<int64_t>(NT, avail));
+    // With the pool the launch also has CTAs for the selection's SMs: they
+    // start once it is done and take pool units only; the dense runs go to
+    // the `home` CTAs that start at once.
+    H.tiles = NT;
+    const int grid = static_cast<int>(std::min<int64_t>(NT, use_pool ? ctx->sms : avail));
+    const int home = std::min(grid, avail);
     H.grid = grid;
     std::vector<int> npieces(H.segs.size(), 0);
     std::vector<std::vector<Piece>> per_cta(grid);
-    for (int phase = 0; phase < 2; ++phase) {
+    for (int phase = 0; phase < (use_pool ? 1 : 2); ++phase) {
       std::vector<size_t> ids;
       std::vector<int64_t> tstart(1, 0);
       for (int dep = 0; dep < 2; ++dep) {
@@ -456,9 +493,10 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const lyc_k
         }
       }
       const int64_t nt = tstart.back();
+      const int cut = use_pool ? home : grid;
       size_t si = 0;
-      for (int c = 0; c < grid; ++c) {
-        const int64_t t0 = nt * c / grid, t1 = nt * (c + 1) / grid;
+      for (int c = 0; c < cut; ++c) {
+        const int64_t t0 = nt * c / cut, t1 = nt * (c + 1) / cut;
         while (si < ids.size() && tstart[si + 1] <= t0) ++si;
         for (size_t q = si; q < ids.size() && tstart[q] < t1; ++q) {
           const int64_t a = std::max(t0, tstart[q]) - tstart[q];
@@ -472,6 +510,17 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const lyc_k
           per_cta[c].push_back(pc);
         }
       }
+    }
+    if (use_pool) {
+      // every sparse segment has keff rows: ups units each, unit q = ordinal q
+      H.pool_ups = static_cast<int>((keff + kPoolTiles * kTileRows - 1) / (kPoolTiles * kTileRows));
+      for (int dep = 0; dep < 2; ++dep)
+        for (size_t s2 = 0; s2 < H.segs.size(); ++s2)
+          if (H.segs[s2].kind == kSparse && H.segs[s2].dep == dep) {
+            H.pool_segs.push_back(static_cast<int32_t>(s2));
+            npieces[s2] = H.pool_ups;
+            H.pool_tiles += (H.segs[s2].rows + TR - 1) / TR;
+          }
     }
     for (int c = 0; c < grid; ++c) {
       H.cta.push_back(static_cast<int32_t>(H.pieces.size()));
@@ -502,11 +551,15 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const lyc_k
         TopkTask tk;
         tk.keys = ctx->keys + keys_base + (static_cast<int64_t>(b) * Hs + s) * ctx->nstride;
         tk.S = set_ptr(1 - cur[s], b, s);
+        tk.done = ctx->flags + ((static_cast<int64_t>(l) * B + b) * Hs + s) * 2;
         H.tasks.push_back(tk);
       }
     }
     for (int s = 0; s < Hs; ++s)
-      if (fresh[s]) cur[s] ^= 1;
+      if (fresh[s]) {
+        cur[s] ^= 1;
+        writer[s] = l;
+      }
     prev_fresh = fresh;
     H.topk_cl = pick_topk_cluster(ctx, static_cast<int>(H.tasks.size()));
     for (int b = 0; b < B; ++b)
@@ -538,6 +591,11 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const lyc_k
     lp.off_trace_src = take(H.trace_src.size() * sizeof(void*));
     lp.ncombine = static_cast<int>(H.combine.size());
     lp.off_combine = take(std::max<size_t>(1, H.combine.size()) * sizeof(int2));
+    lp.pool_nsegs = static_cast<int>(H.pool_segs.size());
+    lp.pool_ups = H.pool_ups;
+    lp.tiles = H.tiles;
+    lp.pool_tiles = H.pool_tiles;
+    lp.off_pool = take(std::max<size_t>(1, H.pool_segs.size()) * sizeof(int32_t));
   }
   plan->off_final_src = take(hl[L - 1].trace_src.size() * sizeof(void*));
   // the last layer's combine runs in a launch of its own, whose CTAs have no pieces
@@ -555,6 +613,8 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const lyc_k
     memcpy(host.data() + lp.off_trace_src, H.trace_src.data(), H.trace_src.size() * sizeof(void*));
     if (!H.combine.empty())
       memcpy(host.data() + lp.off_combine, H.combine.data(), H.combine.size() * sizeof(int2));
+    if (!H.pool_segs.empty())
+      memcpy(host.data() + lp.off_pool, H.pool_segs.data(), H.pool_segs.size() * sizeof(int32_t));
   }
   memcpy(host.data() + plan->off_final_src, hl[L - 1].trace_src.data(),
          hl[L - 1].trace_src.size() * sizeof(void*));
@@ -615,6 +675,22 @@ lyc_status enqueue_step(lyc_ctx* ctx, Plan* plan, cudaStream_t stream, int set, 
   plan->kernel_kind.clear();
   plan->kernel_layer.clear();
   int ev = 0;
+  // bf16 on the mma kernel: ready and done flags, the per-SM piece-state
+  // ring and the pool make it safe for its launches to overlap the previous
+  // layer's (the previous attention, and the selection between them)
+  const bool early = dtype == 0 && !plan->use_tc;
+  // ... and each selection may then let the next attention launch before it
+  // has read its keys, so that the next attention's CTAs take the SMs of the
+  // previous attention's tail as they free up.  They then start staggered,
+  // and their dense runs are static: this pays when the next layer's pool
+  // (taken at run time) is large enough to absorb the stagger (measured on
+  // B200: a pool of ~1/3 of the tiles gains, ~1/9 loses), else the next
+  // attention launches once the selection has its keys.
+  auto early_trigger = [&](int l) {
+    if (!early || l + 1 >= L) return false;
+    const LayerPlan& nx = plan->layers[l + 1];
+    return nx.tiles > 0 && 5 * nx.pool_tiles >= nx.tiles;
+  };
   for (int l = 0; l < L; ++l) {
     const LayerPlan& lp = plan->layers[l];
     AttnParams ap{};
@@ -628,6 +704,21 @@ lyc_status enqueue_step(lyc_ctx* ctx, Plan* plan, cudaStream_t stream, int set, 
     ap.part_ml = ctx->part_ml + (l & 1) * ctx->max_parts;
     ap.wpart_o = ctx->wpart_o;
     ap.wpart_ml = ctx->wpart_ml;
+    ap.wpart_by_sm = 1;
+    ap.wpart_slots = ctx->wpart_slots;
+    ap.epoch = ctx->epoch;
+    if (early) {
+      // done flags between consecutive attention launches, and the pool of
+      // gathered rows (mma kernel only)
+      ap.done = ctx->attn_flags + 2 * l;
+      ap.prev_done = l > 0 ? ctx->attn_flags + 2 * (l - 1) + 1 : nullptr;
+      ap.pool_segs = reinterpret_cast<const int32_t*>(plan->dev + lp.off_pool);
+      ap.pool_n = lp.pool_nsegs * lp.pool_ups;
+      ap.pool_ups = lp.pool_ups;
+      ap.pool_rows = plan->keff;
+      ap.pool_stride = L + 1;
+      ap.pool_cursors = ctx->pool_cursors;
+    }
     ap.counters = ctx->counters;
     ap.status = ctx->status;
     ap.timeline = plan->timeline;
@@ -638,10 +729,12 @@ lyc_status enqueue_step(lyc_ctx* ctx, Plan* plan, cudaStream_t stream, int set, 
     ap.n = plan->n;
     ap.scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
     ap.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
-    // without a selection launch in between, the previous layer's attention
-    // may still be running: its selection keys share the key buffer of the
-    // layer after this one, and its partials are combined by this launch
-    ap.wait_prev = (l > 0 && plan->layers[l - 1].ntasks == 0) ? 1 : 0;
+    // Without a selection launch in between, the previous layer's attention
+    // may still be running.  The mma kernel needs no wait for it: its
+    // readers of sets wait on the sets' ready flags, its partials are written
+    // only after its epilogue's griddepcontrol.wait, and its piece-state ring
+    // is the SM's own.  The other kernels wait for it at their start.
+    ap.wait_prev = (l > 0 && plan->layers[l - 1].ntasks == 0 && !early) ? 1 : 0;
     lyc_status st = record_event(ctx, plan, set, ev++, stream, capturing);
     if (st != LYC_OK) return st;
     if (dtype == 0) {
@@ -665,6 +758,8 @@ lyc_status enqueue_step(lyc_ctx* ctx, Plan* plan, cudaStream_t stream, int set, 
     if (lp.ntasks > 0) {
       TopkParams tp{};
       tp.tasks = reinterpret_cast<const TopkTask*>(plan->dev + lp.off_tasks);
+      tp.epoch = ctx->epoch;
+      tp.early = early_trigger(l) ? 1 : 0;
       tp.n = plan->n;
       tp.k = plan->k;
       tp.timeline = plan->timeline;
@@ -701,6 +796,10 @@ lyc_status enqueue_step(lyc_ctx* ctx, Plan* plan, cudaStream_t stream, int set, 
     ap.status = ctx->status;
     ap.wpart_o = ctx->wpart_o;
     ap.wpart_ml = ctx->wpart_ml;
+    ap.wpart_by_sm = 1;
+    ap.wpart_slots = ctx->wpart_slots;
+    ap.epoch = ctx->epoch;
+    if (early) ap.prev_done = ctx->attn_flags + 2 * (L - 1) + 1;
     ap.layer = L;
     ap.Hq = Hq;
     ap.G = ctx->G;
@@ -716,7 +815,7 @@ lyc_status enqueue_step(lyc_ctx* ctx, Plan* plan, cudaStream_t stream, int set, 
     plan->kernel_layer.push_back(L - 1);
   }
   CopySetsParams cp{reinterpret_cast<const int32_t* const*>(plan->dev + plan->off_final_src), plan->S,
-                    B * ctx->Hs, plan->k};
+                    B * ctx->Hs, plan->k, ctx->epoch, ctx->pool_cursors, L + 1};
   LYC_CUDA(copy_sets_launch(&cp, stream), "final set copy");
   return LYC_OK;
 }
@@ -879,8 +978,10 @@ lyc_status lyc_create(const lyc_config* cfg, lyc_ctx** out) {
   const int B = c.batch, Hq = c.num_q_heads, Hkv = c.num_kv_heads, D = c.head_dim, L = c.num_layers;
   const size_t es = c.dtype == LYC_BF16 ? 2 : 4;
   const size_t nseg_max = static_cast<size_t>(B) * (Hkv + Hq);
-  // pieces per layer <= 2 * sms + segments (two pooling phases)
-  ctx->max_parts = (2 * static_cast<size_t>(ctx->sms) + nseg_max) * kMaxQ;
+  // pieces per layer <= 2 * sms + segments (two pooling phases), plus the
+  // pool units of the mma kernel (every sparse segment cut into units)
+  const size_t units = (static_cast<size_t>(c.max_k) + kPoolTiles * kTileRows - 1) / (kPoolTiles * kTileRows);
+  ctx->max_parts = (2 * static_cast<size_t>(ctx->sms) + nseg_max + nseg_max * units) * kMaxQ;
   ctx->max_counters = nseg_max * kMaxQ;
   auto alloc = [&](void** p, size_t bytes) -> lyc_status {
     if (cudaMalloc(p, bytes) != cudaSuccess) {
@@ -890,9 +991,14 @@ lyc_status lyc_create(const lyc_config* cfg, lyc_ctx** out) {
     return LYC_OK;
   };
   lyc_status st;
+  // ready flags: two words per (layer, b, slot) and per layer, then the
+  // pool cursors, then the epoch
+  const size_t flag_words = static_cast<size_t>(L) * B * ctx->Hs * 2 + static_cast<size_t>(L) * 2 +
+                            2 * (static_cast<size_t>(L) + 1) + 4;
   if ((st = alloc(reinterpret_cast<void**>(&ctx->status), 16)) != LYC_OK ||
       (st = alloc(reinterpret_cast<void**>(&ctx->keys),
-                  2 * static_cast<size_t>(B) * ctx->Hs * ctx->nstride * sizeof(float))) != LYC_OK ||
+                  static_cast<size_t>(L) * B * ctx->Hs * ctx->nstride * sizeof(float))) != LYC_OK ||
+      (st = alloc(reinterpret_cast<void**>(&ctx->flags), flag_words * sizeof(uint32_t))) != LYC_OK ||
       (st = alloc(reinterpret_cast<void**>(&ctx->sbuf),
                   2ull * B * ctx->Hs * ctx->KS * sizeof(int32_t) + 64)) != LYC_OK ||
       (st = alloc(reinterpret_cast<void**>(&ctx->part_o), 2 * ctx->max_parts * D * sizeof(float))) != LYC_OK ||
@@ -904,8 +1010,14 @@ lyc_status lyc_create(const lyc_config* cfg, lyc_ctx** out) {
     lyc_destroy(holder.release());
     return st;
   }
+  ctx->attn_flags = ctx->flags + static_cast<size_t>(L) * B * ctx->Hs * 2;
+  ctx->pool_cursors = reinterpret_cast<int32_t*>(ctx->attn_flags + static_cast<size_t>(L) * 2);
+  ctx->epoch = ctx->flags + (flag_words - 4);
   if (c.dtype == LYC_BF16) {
-    const size_t recs = static_cast<size_t>(ctx->sms) * kPartSlots * kMaxConsumerWarps * kMaxQ;
+    // one ring per SM index (the SM a CTA runs on owns it; SM indices need
+    // not be dense, so twice the count, at least 256)
+    ctx->wpart_slots = std::max(256, 2 * ctx->sms);
+    const size_t recs = static_cast<size_t>(ctx->wpart_slots) * kPartSlots * kMaxConsumerWarps * kMaxQ;
     if ((st = alloc(reinterpret_cast<void**>(&ctx->wpart_o), recs * D * sizeof(float))) != LYC_OK ||
         (st = alloc(reinterpret_cast<void**>(&ctx->wpart_ml), recs * sizeof(float2))) != LYC_OK) {
       lyc_destroy(holder.release());
@@ -913,6 +1025,7 @@ lyc_status lyc_create(const lyc_config* cfg, lyc_ctx** out) {
     }
   }
   if (cudaMemset(ctx->status, 0, 16) != cudaSuccess ||
+      cudaMemset(ctx->flags, 0, flag_words * sizeof(uint32_t)) != cudaSuccess ||
       cudaMemset(ctx->counters, 0, ctx->max_counters * sizeof(int32_t)) != cudaSuccess ||
       cudaMemset(ctx->sbuf, 0xff, 2ull * B * ctx->Hs * ctx->KS * sizeof(int32_t) + 64) != cudaSuccess) {
     lyc_destroy(holder.release());
@@ -969,7 +1082,7 @@ void lyc_destroy(lyc_ctx* ctx) {
   for (auto& kv : ctx->plans) free_plan(kv.second.get());
   ctx->plans.clear();
   for (cudaEvent_t ev : ctx->events) cudaEventDestroy(ev);
-  void* bufs[] = {ctx->status, ctx->keys, ctx->sbuf, ctx->part_o, ctx->part_ml,
+  void* bufs[] = {ctx->status, ctx->keys, ctx->flags, ctx->sbuf, ctx->part_o, ctx->part_ml,
                   ctx->wpart_o, ctx->wpart_ml, ctx->counters, ctx->q_dev, ctx->out_dev,
                   ctx->S_dev};
   for (void* b : bufs)
@@ -1095,6 +1208,8 @@ lyc_status lyc_sync_status(lyc_ctx* ctx) {
   LYC_CUDA(cudaMemcpy(&word, ctx->status, sizeof word, cudaMemcpyDeviceToHost), "read status");
   LYC_CUDA(cudaMemset(ctx->status, 0, sizeof word), "clear status");
   if (word & kStatusTimeout) return fail(ctx, LYC_ERR_TIMEOUT, "a device-side wait gave up");
+  if (word & kStatusScratch)
+    return fail(ctx, LYC_ERR_CUDA, "a CTA ran on an SM index beyond the per-SM scratch (no work done)");
   if (word & (kStatusBadIndex | kStatusEmptySoftmax))
     return fail(ctx, LYC_ERR_BAD_INDEX, "an inherited set held an index outside [0, n)");
   return LYC_OK;

@@ -32,6 +32,11 @@ constexpr int kMaxConsumerWarps = 8;
 // pieces a CTA's consumer warps may run ahead of its epilogue warp: the ring
 // of per-warp partial states between them has this many slots
 constexpr int kPartSlots = 4;
+// Pool of gathered rows that CTAs take at run time, kPoolTiles tiles at a
+// time; a CTA's leader publishes the pool pieces it took into a ring of
+// kPoolRing entries that every warp of the CTA reads in order.
+constexpr int kPoolTiles = 4;
+constexpr int kPoolRing = 16;
 
 enum SegKind : int32_t { kDense = 0, kSparse = 1 };
 
@@ -57,6 +62,9 @@ struct Segment {
   int32_t row_base;     // row of (l, b, g, token 0) in the flattened row-gather map
   int32_t dep;          // sparse: the set is the previous launch's output (wait for it)
   int32_t pad_;
+  const uint32_t* ready;  // sparse: flag word of the selection that wrote the set in
+                          // this step (it holds the step's epoch + 1 once the set is
+                          // complete), or NULL when the set comes from the caller
 };
 
 struct Piece {
@@ -89,6 +97,24 @@ struct AttnParams {
                              // work (it is not a selection launch, which would have)
   uint32_t* status;          // device status word
   unsigned long long* timeline;  // NULL, or [1 + 3*cap]: count, then (start ns, end ns, tag)
+  const uint32_t* epoch;     // this step's epoch (the `ready` flags hold epoch + 1), or NULL
+  uint32_t* done;            // NULL, or {arrival counter, flag} of this launch: the last CTA
+                             // to finish raises the flag to epoch + 1
+  const uint32_t* prev_done; // NULL, or the flag of the previous layer's attention launch:
+                             // the epilogue waits on it (else on griddepcontrol.wait)
+  // the pool (mma kernel): after its own pieces a CTA takes units u = 0, 1, ...
+  // by an atomic cursor; unit u is rows [q * kPoolTiles * 64, ...) of segment
+  // pool_segs[u / pool_ups], q = u % pool_ups, ordinal q (its partial record)
+  const int32_t* pool_segs;
+  int32_t pool_n;            // units in the pool (0: none)
+  int32_t pool_ups;          // units per pool segment
+  int32_t pool_rows;         // rows of every pool segment
+  int32_t pool_stride;       // cursors per epoch parity
+  int32_t* pool_cursors;     // [2][pool_stride]: this launch's is [(epoch & 1)][layer]
+  int32_t wpart_by_sm;       // 1: the piece-state ring of a CTA is the one of the SM it runs
+                             // on (CTAs of consecutive launches may overlap in time); 0: of
+                             // its block index
+  int32_t wpart_slots;       // rings allocated
   int32_t timeline_cap;
   int32_t layer;
   int32_t Hq, G, n;
@@ -102,11 +128,16 @@ struct AttnParams {
 struct TopkTask {
   const float* keys;  // n selection keys
   int32_t* S;         // k outputs
+  uint32_t* done;     // NULL, or {arrival counter, ready flag}: the last CTA of the task
+                      // to finish resets the counter and sets the flag to epoch + 1
 };
 
 struct TopkParams {
   const TopkTask* tasks;  // one per blockIdx.y; NULL: use `single`
   TopkTask single;
+  const uint32_t* epoch;  // this step's epoch (for the ready flags), or NULL
+  int32_t early;          // 1: let the next launch start before this one has read its keys
+                          // (its readers wait on the ready flags); 0: only after
   unsigned long long* timeline;  // as in AttnParams
   int32_t timeline_cap;
   int32_t layer;
@@ -122,6 +153,9 @@ struct CopySetsParams {
   const int32_t* const* src;
   int32_t* dst;
   int32_t nsets, k;
+  uint32_t* epoch;  // the step's last launch: advance the epoch once the copy is done (or NULL)
+  int32_t* pool_cursors;  // with epoch: zero the next step's pool cursors, [2][pool_stride]
+  int32_t pool_stride;
 };
 
 // validate_sets_kernel: each of nsets sets (stride `stride`) must hold k_eff
@@ -145,5 +179,6 @@ __host__ __device__ inline uint32_t order_key(float f) {
 constexpr uint32_t kStatusBadIndex = 1u;
 constexpr uint32_t kStatusTimeout = 2u;
 constexpr uint32_t kStatusEmptySoftmax = 4u;
+constexpr uint32_t kStatusScratch = 8u;  // an SM index beyond the per-SM scratch
 
 }  // namespace lyc

@@ -13,6 +13,17 @@ __global__ void copy_sets_kernel(const CopySetsParams p) {
   const int32_t* src = p.src[set];
   int32_t* dst = p.dst + static_cast<int64_t>(set) * p.k;
   for (int j = threadIdx.x; j < p.k; j += blockDim.x) dst[j] = src[j];
+  // the step's last launch (every launch of the step has completed before it
+  // starts, and the next step's launches start after it ends): the next
+  // step's ready flags are told apart from this step's by the epoch
+  if (p.epoch && set == 0) {
+    const uint32_t e = *p.epoch;
+    if (p.pool_cursors)
+      for (int j = threadIdx.x; j < p.pool_stride; j += blockDim.x)
+        p.pool_cursors[static_cast<int64_t>((e + 1u) & 1u) * p.pool_stride + j] = 0;
+    __syncthreads();
+    if (threadIdx.x == 0) *p.epoch = e + 1u;
+  }
 }
 
 __global__ void validate_sets_kernel(const ValidateSetsParams p) {
@@ -32,7 +43,7 @@ __global__ void validate_sets_kernel(const ValidateSetsParams p) {
 }
 
 cudaError_t copy_sets_launch(const CopySetsParams* p, cudaStream_t stream) {
-  if (p->nsets <= 0) return cudaSuccess;
+  if (p->nsets <= 0) return cudaSuccess;  // never the case: a step has B * Hs >= 1 sets
   copy_sets_kernel<<<p->nsets, 256, 0, stream>>>(*p);
   return cudaGetLastError();
 }

@@ -269,6 +269,8 @@ extern "C" lyc_status lyc_sparse_attention_noalloc(const void* q, const lyc_kv_c
   ap.counters = reinterpret_cast<int32_t*>(dbase + kOffCounters);
   ap.wpart_o = reinterpret_cast<float*>(dbase + kOffWpartO);
   ap.wpart_ml = reinterpret_cast<float2*>(dbase + kOffWpartMl);
+  ap.wpart_by_sm = 0;  // one ring per CTA: the two launches of a call never overlap on an SM ring
+  ap.wpart_slots = kNaMaxCtas;
   ap.status = reinterpret_cast<uint32_t*>(dbase + kOffStatus);
   ap.timeline = nullptr;
   ap.timeline_cap = 0;

@@ -159,6 +159,25 @@ __device__ __forceinline__ uint32_t select_in_candidates(const uint2* cand, cons
   return prefix;
 }
 
+// Every CTA of a task calls this once its writes of S are issued: the last of
+// the CL to arrive resets the arrival counter and raises the task's ready
+// flag to the step's epoch + 1 (release: each arrival fences its CTA's writes
+// first, the flag store follows the last arrival).
+template <int CL>
+__device__ __forceinline__ void topk_signal_done(const TopkParams& p, const TopkTask& task, int tid) {
+  if (!task.done) return;
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) {
+    const uint32_t prev = atomicAdd(&task.done[0], 1u);
+    if (prev == static_cast<uint32_t>(CL - 1)) {
+      task.done[0] = 0u;
+      __threadfence();
+      st_release_u32(&task.done[1], (p.epoch ? *p.epoch : 0u) + 1u);
+    }
+  }
+}
+
 template <int CL>
 __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster_kernel(const TopkParams p) {
   cg::cluster_group cluster = cg::this_cluster();
@@ -176,10 +195,13 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster_kernel(const Top
   const int cnt = max(0, min(n, lo + chunk) - lo);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const unsigned lt = (1u << lane) - 1u;
-  // the keys are the attention kernel's output; only once it has completed
-  // may the next kernel (the next layer's attention) start its launch
+  // The keys are the attention kernel's output: read only once it has
+  // completed.  The next kernel (the next layer's attention) may start its
+  // launch before that when its readers of this selection's sets wait on the
+  // ready flags (p.early), else only after.
+  if (p.early) pdl_launch_dependents();
   pdl_wait();
-  pdl_launch_dependents();
+  if (!p.early) pdl_launch_dependents();
   const uint64_t t_start = p.timeline ? global_timer_ns() : 0;  // work starts here
 
   extern __shared__ __align__(16) unsigned char smem[];
@@ -200,6 +222,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster_kernel(const Top
     for (int x = tid; x < cnt; x += kTopkThreads) task.S[lo + x] = lo + x;
     if (rank == 0)
       for (int x = keff + tid; x < k; x += kTopkThreads) task.S[x] = -1;
+    topk_signal_done<CL>(p, task, tid);
     if (tid == 0)
       timeline_record(p.timeline, p.timeline_cap, t_start,
                       (kTagTopk << 32) | (static_cast<unsigned long long>(p.layer) << 16) |
@@ -501,6 +524,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster_kernel(const Top
     emit([&](int x) { return make_uint2(us[x], static_cast<uint32_t>(lo + x)); }, cnt);
   if (rank == 0)
     for (int x = keff + tid; x < k; x += kTopkThreads) task.S[x] = -1;
+  topk_signal_done<CL>(p, task, tid);
   if (tid == 0)
     timeline_record(p.timeline, p.timeline_cap, t_start,
                     (kTagTopk << 32) | (static_cast<unsigned long long>(p.layer) << 16) |

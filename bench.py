@@ -87,18 +87,21 @@ def attn_source_hash() -> str:
 def profiled_traffic(workload: str):
     """DRAM bytes per attention launch from the committed ncu summary, if it
     was taken on the current kernel source."""
-    path = os.path.join(ROOT, "profiles", "attn_mma_layer_kernel_traffic.md")
-    if not os.path.exists(path):
+    pdir = os.path.join(ROOT, "profiles")
+    if not os.path.isdir(pdir):
         return None
     want = attn_source_hash()
-    for line in open(path):
-        if line.startswith("traffic-record:"):
-            try:
-                rec = json.loads(line.split(":", 1)[1])
-            except ValueError:
-                continue
-            if rec.get("source_sha") == want and rec.get("workload") == workload:
-                return rec.get("bytes_per_launch")
+    for name in sorted(os.listdir(pdir)):
+        if not name.startswith("attn_mma_layer_kernel") or not name.endswith(".md"):
+            continue
+        for line in open(os.path.join(pdir, name)):
+            if line.startswith("traffic-record:"):
+                try:
+                    rec = json.loads(line.split(":", 1)[1])
+                except ValueError:
+                    continue
+                if rec.get("source_sha") == want and rec.get("workload") == workload:
+                    return rec.get("bytes_per_launch")
     return None
 
 

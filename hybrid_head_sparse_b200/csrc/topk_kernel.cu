@@ -161,14 +161,16 @@ __device__ __forceinline__ uint32_t select_in_candidates(const uint2* cand, cons
 
 // Every CTA of a task calls this once its writes of S are issued: the last of
 // the CL to arrive resets the arrival counter and raises the task's ready
-// flag to the step's epoch + 1 (release: each arrival fences its CTA's writes
-// first, the flag store follows the last arrival).
+// flag to the step's epoch + 1.  Release: the CTA barrier orders every
+// thread's writes before thread 0's device-scope fence, which precedes its
+// arrival; the last arrival fences again before the flag store.  (One fence
+// per CTA: a fence in every thread stalls the whole CTA on memory barriers.)
 template <int CL>
 __device__ __forceinline__ void topk_signal_done(const TopkParams& p, const TopkTask& task, int tid) {
   if (!task.done) return;
-  __threadfence();
   __syncthreads();
   if (tid == 0) {
+    __threadfence();
     const uint32_t prev = atomicAdd(&task.done[0], 1u);
     if (prev == static_cast<uint32_t>(CL - 1)) {
       task.done[0] = 0u;

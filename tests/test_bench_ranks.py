@@ -70,3 +70,20 @@ def test_percentiles():
     import bench
     p = bench.percentiles([5.0, 1.0, 3.0, 2.0, 4.0])
     assert (p["p10"], p["p50"], p["p90"]) == (1.0, 3.0, 5.0)
+
+
+def test_traffic_record_lookup(tmp_path, monkeypatch):
+    """The bench takes DRAM traffic from a committed ncu summary only when the
+    summary was taken on the current attention-kernel source and workload."""
+    import bench
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    (prof / "attn_mma_layer_kernel_some-workload.md").write_text(
+        "summary\n"
+        'traffic-record: {"workload": "w1", "source_sha": "abc", "bytes_per_launch": 123}\n')
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "attn_source_hash", lambda: "abc")
+    assert bench.profiled_traffic("w1") == 123
+    assert bench.profiled_traffic("w2") is None
+    monkeypatch.setattr(bench, "attn_source_hash", lambda: "def")
+    assert bench.profiled_traffic("w1") is None

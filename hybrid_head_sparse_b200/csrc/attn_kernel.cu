@@ -201,8 +201,8 @@ __device__ __forceinline__ void attn_producer(const AttnParams& p, unsigned char
           ia = r0 + lane;
           ib = r0 + lane + 32;
         }
-        const bool va = lane < nrows && ia >= 0 && ia < p.n;
-        const bool vb2 = lane + 32 < nrows && ib >= 0 && ib < p.n;
+        const bool va = lane < nrows && ia >= 0 && ia < sg.nvalid;
+        const bool vb2 = lane + 32 < nrows && ib >= 0 && ib < sg.nvalid;
         if ((lane < nrows && !va) || (lane + 32 < nrows && !vb2)) atomicOr(p.status, kStatusBadIndex);
         const uint32_t ma = __ballot_sync(0xffffffffu, va);
         const uint32_t mb = __ballot_sync(0xffffffffu, vb2);

@@ -237,16 +237,19 @@ __device__ __forceinline__ void mma_scheduler(const AttnMmaParams& P, unsigned c
       if (!slot_free(t)) break;
       if (k >= kPoolRing && !mbar_wait(&unit_empty[r], ((k / kPoolRing) - 1) & 1, abort_flag, p.status))
         break;
-      const int u = atomicAdd(cursor, 1);
-      if (u < p.pool_n) {
+      // the next unit that holds rows (units past a shorter segment's end are skipped)
+      pc.seg = -1;
+      pc.r0 = pc.r1 = pc.ordinal = 0;
+      for (int u = atomicAdd(cursor, 1); u < p.pool_n; u = atomicAdd(cursor, 1)) {
         const int q = u % p.pool_ups;
-        pc.seg = __ldg(&p.pool_segs[u / p.pool_ups]);
+        const int seg = __ldg(&p.pool_segs[u / p.pool_ups]);
+        const int rows = p.segs[seg].rows;
+        if (q * (kPoolTiles * kTileRows) >= rows) continue;
+        pc.seg = seg;
         pc.r0 = q * (kPoolTiles * kTileRows);
-        pc.r1 = min(pc.r0 + kPoolTiles * kTileRows, p.pool_rows);
+        pc.r1 = min(pc.r0 + kPoolTiles * kTileRows, rows);
         pc.ordinal = q;
-      } else {
-        pc.seg = -1;
-        pc.r0 = pc.r1 = pc.ordinal = 0;
+        break;
       }
       ring[r] = pc;
       mbar_arrive(&unit_full[r]);  // release: the entry above
@@ -290,7 +293,7 @@ __device__ __forceinline__ void mma_scheduler(const AttnMmaParams& P, unsigned c
 // TMA copies, everyone arrives.  Gathered tile: warp pw copies rows
 // [pw*64/NP, (pw+1)*64/NP) with cp.async and every lane arrives when its own
 // copies have landed.
-template <int D, int NC, int NP, int STAGES, bool GT>
+template <int D, int NC, int NP, int STAGES, bool GT, bool PG>
 __device__ __forceinline__ void mma_producers(const AttnMmaParams& P, unsigned char* smem, int pbeg,
                                               int pend) {
   using C = MmaCfg<D, NC, NP, STAGES, GT>;
@@ -325,6 +328,13 @@ __device__ __forceinline__ void mma_producers(const AttnMmaParams& P, unsigned c
     const bf16_t* kb = static_cast<const bf16_t*>(sg.k);
     const bf16_t* vb = static_cast<const bf16_t*>(sg.v);
     const int sl = sg.l, sb = sg.b, sgg = sg.g;
+    // the segment's constants in registers (the copies below are asm with a
+    // memory clobber: fields read through `sg` would be reloaded after each)
+    const int nvalid = sg.nvalid;
+    const int32_t* bt = sg.bt;
+    const int page_rows = sg.page_rows;
+    const int64_t s_page = sg.s_page;
+    const int32_t row_base = sg.row_base;
     for (int r0 = pc.r0; r0 < pc.r1; r0 += kTileRows, ++t) {
       const int nrows = min(kTileRows, pc.r1 - r0);
       const int stage = t % STAGES;
@@ -337,10 +347,18 @@ __device__ __forceinline__ void mma_producers(const AttnMmaParams& P, unsigned c
         // TMA tensor copies; rows past n are filled with zeros by the copy
         if (leader) {
           mbar_arrive_expect_tx(&full[stage], 2u * C::TILEB);
+          // contiguous: map (d, row, g, b, l); paged: map (d, g, row in page, page, l),
+          // a tile never crosses a page (page_rows is a multiple of 64)
+          int c1 = r0, c2 = sgg, c3 = sb;
+          if (PG) {
+            c1 = sgg;
+            c2 = r0 % page_rows;
+            c3 = __ldg(&bt[r0 / page_rows]);
+          }
 #pragma unroll
           for (int h = 0; h < C::HALVES; ++h) {
-            tma_load_5d(kdst + h * C::BLOCKB, &P.tmk, h * 64, r0, sgg, sb, sl, &full[stage], pol);
-            tma_load_5d(vdst + h * C::BLOCKB, &P.tmv, h * 64, r0, sgg, sb, sl, &full[stage], pol);
+            tma_load_5d(kdst + h * C::BLOCKB, &P.tmk, h * 64, c1, c2, c3, sl, &full[stage], pol);
+            tma_load_5d(vdst + h * C::BLOCKB, &P.tmv, h * 64, c1, c2, c3, sl, &full[stage], pol);
           }
         } else if (!GT) {
           mbar_arrive(&full[stage]);
@@ -362,9 +380,9 @@ __device__ __forceinline__ void mma_producers(const AttnMmaParams& P, unsigned c
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const bool in_tile = 4 * j + e < nrows;
-          const bool ok = xs[e] >= 0 && xs[e] < p.n;
+          const bool ok = xs[e] >= 0 && xs[e] < nvalid;
           bad |= in_tile && !ok;
-          ys[e] = (in_tile && ok) ? sg.row_base + xs[e] : p.gather_rows;
+          ys[e] = (in_tile && ok) ? row_base + xs[e] : p.gather_rows;
         }
         if (bad) atomicOr(p.status, kStatusBadIndex);
         const bool isv = lane >= 16;
@@ -382,7 +400,7 @@ __device__ __forceinline__ void mma_producers(const AttnMmaParams& P, unsigned c
         if (pw == 0) {  // bounds of the inherited indices (reported, never followed)
           const int32_t ia = (lane < nrows) ? ring[lane] : 0;
           const int32_t ib = (lane + 32 < nrows) ? ring[lane + 32] : 0;
-          if (ia < 0 || ia >= p.n || ib < 0 || ib >= p.n) atomicOr(p.status, kStatusBadIndex);
+          if (ia < 0 || ia >= nvalid || ib < 0 || ib >= nvalid) atomicOr(p.status, kStatusBadIndex);
         }
         const uint32_t kbase = smem_u32(kdst), vbase = smem_u32(vdst);
         // lane: chunk (lane % CH) of rows pw*ROWS_W + (lane / CH) + (32/CH)*i
@@ -392,8 +410,16 @@ __device__ __forceinline__ void mma_producers(const AttnMmaParams& P, unsigned c
           const int r = pw * ROWS_W + i * RPI + lane / CH;
           const int c = lane % CH;
           const int32_t ix = (r < nrows) ? ring[r] : -1;
-          const bool ok = ix >= 0 && ix < p.n;
-          const int64_t off = ok ? static_cast<int64_t>(ix) * s_token : 0;
+          const bool ok = ix >= 0 && ix < nvalid;
+          // contiguous rows, or row ix % page_rows of page bt[ix / page_rows]
+          int64_t off = 0;
+          if (ok) {
+            if (PG)
+              off = static_cast<int64_t>(__ldg(&bt[ix / page_rows])) * s_page +
+                    static_cast<int64_t>(ix % page_rows) * s_token;
+            else
+              off = static_cast<int64_t>(ix) * s_token;
+          }
           cp_async_16(kbase + swz(r, c), kb + off + c * 8, ok ? 16u : 0u);
           cp_async_16(vbase + swz(r, c), vb + off + c * 8, ok ? 16u : 0u);
         }
@@ -466,6 +492,7 @@ __device__ __forceinline__ void mma_consumers(const AttnMmaParams& P, unsigned c
     const int64_t koff1 = (q1 < nq) ? sg.key_off[q1] : -1;
     const int64_t key_mean_off = sg.key_mean_off;
     const float mean_scale = p.scale / static_cast<float>(nq);
+    const int nvalid = sg.nvalid;
 
     // ---- Q^T as the B operand: this lane holds query g, d = 16kk + 2c (+8)
     uint32_t qb[KSTEPS][2];
@@ -494,8 +521,8 @@ __device__ __forceinline__ void mma_consumers(const AttnMmaParams& P, unsigned c
       bool va = lane < nrows, vb = lane + 32 < nrows;
       if (!dense) {
         const int32_t* ring = idxring + (t % C::IR) * kTileRows;
-        if (va) { const int32_t x = ring[lane]; va = x >= 0 && x < p.n; }
-        if (vb) { const int32_t x = ring[lane + 32]; vb = x >= 0 && x < p.n; }
+        if (va) { const int32_t x = ring[lane]; va = x >= 0 && x < nvalid; }
+        if (vb) { const int32_t x = ring[lane + 32]; vb = x >= 0 && x < nvalid; }
       }
       const uint64_t vmask = static_cast<uint64_t>(__ballot_sync(FULL, va)) |
                              (static_cast<uint64_t>(__ballot_sync(FULL, vb)) << 32);
@@ -793,7 +820,7 @@ __device__ __forceinline__ void mma_epilogue(const AttnMmaParams& P, unsigned ch
 }
 
 // ---------------------------------------------------------------- kernel
-template <int D, int NC, int NP, int STAGES, bool GT>
+template <int D, int NC, int NP, int STAGES, bool GT, bool PG>
 __global__ void __launch_bounds__(MmaCfg<D, NC, NP, STAGES, GT>::kThreads, 1)
     attn_mma_layer_kernel(const __grid_constant__ AttnMmaParams P) {
   using C = MmaCfg<D, NC, NP, STAGES, GT>;
@@ -839,7 +866,7 @@ __global__ void __launch_bounds__(MmaCfg<D, NC, NP, STAGES, GT>::kThreads, 1)
     const int pbeg = P.p.cta_begin[blockIdx.x];
     const int pend = P.p.cta_begin[blockIdx.x + 1];
     if (threadIdx.x >= C::kFirstProducer) {
-      mma_producers<D, NC, NP, STAGES, GT>(P, smem, pbeg, pend);
+      mma_producers<D, NC, NP, STAGES, GT, PG>(P, smem, pbeg, pend);
     } else if (threadIdx.x >= C::kScheduler) {
       if (threadIdx.x == C::kScheduler) mma_scheduler<D, NC, NP, STAGES, GT>(P, smem, pbeg, pend);
     } else if (threadIdx.x >= NC * 32) {
@@ -871,11 +898,11 @@ __global__ void __launch_bounds__(MmaCfg<D, NC, NP, STAGES, GT>::kThreads, 1)
 }
 
 // ---------------------------------------------------------------- host side
-template <int D, int NC, int NP, int STAGES, bool GT>
+template <int D, int NC, int NP, int STAGES, bool GT, bool PG = false>
 static cudaError_t mma_run(const AttnMmaParams* P, int grid, cudaStream_t stream, int* smem_out,
                            bool configure_only) {
   using C = MmaCfg<D, NC, NP, STAGES, GT>;
-  auto kern = attn_mma_layer_kernel<D, NC, NP, STAGES, GT>;
+  auto kern = attn_mma_layer_kernel<D, NC, NP, STAGES, GT, PG>;
   if (configure_only) {
     if (smem_out) *smem_out = C::SMEM;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
@@ -909,21 +936,28 @@ cudaError_t attn_mma_dispatch(int D, const AttnMmaParams* P, int grid, cudaStrea
     cudaError_t e = cudaErrorInvalidValue;
     if (D == 128) {
       e = mma_run<128, 6, 8, 6, false>(P, grid, stream, &s1, true);
+      if (e == cudaSuccess) e = mma_run<128, 6, 8, 6, false, true>(P, grid, stream, &s1, true);
       if (e == cudaSuccess) e = mma_run<128, 6, 1, 6, true>(P, grid, stream, &s2, true);
     } else if (D == 64) {
       e = mma_run<64, 4, 8, 8, false>(P, grid, stream, &s1, true);
+      if (e == cudaSuccess) e = mma_run<64, 4, 8, 8, false, true>(P, grid, stream, &s1, true);
       if (e == cudaSuccess) e = mma_run<64, 4, 1, 8, true>(P, grid, stream, &s2, true);
     }
     if (smem_out) *smem_out = s1 > s2 ? s1 : s2;
     return e;
   }
+  // a paged cache (the planner never pairs it with the row-gather maps) runs
+  // on its own instantiation, so the contiguous one carries no paging code
   const bool gt = P->p.gather_rows > 0;
+  const bool pg = P->p.paged != 0;
   if (D == 128)
     return gt ? mma_run<128, 6, 1, 6, true>(P, grid, stream, smem_out, false)
-              : mma_run<128, 6, 8, 6, false>(P, grid, stream, smem_out, false);
+           : pg ? mma_run<128, 6, 8, 6, false, true>(P, grid, stream, smem_out, false)
+                : mma_run<128, 6, 8, 6, false>(P, grid, stream, smem_out, false);
   if (D == 64)
     return gt ? mma_run<64, 4, 1, 8, true>(P, grid, stream, smem_out, false)
-              : mma_run<64, 4, 8, 8, false>(P, grid, stream, smem_out, false);
+           : pg ? mma_run<64, 4, 8, 8, false, true>(P, grid, stream, smem_out, false)
+                : mma_run<64, 4, 8, 8, false>(P, grid, stream, smem_out, false);
   return cudaErrorInvalidValue;
 }
 

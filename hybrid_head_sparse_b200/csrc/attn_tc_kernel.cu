@@ -221,7 +221,7 @@ __device__ __forceinline__ void tc_producers(const AttnMmaParams& P, unsigned ch
           for (int i = 0; i < kTcRows / 32; ++i) {
             const int r = lane + 32 * i;
             const int32_t ix = (r < nrows) ? ring[r] : 0;
-            bad |= ix < 0 || ix >= p.n;
+            bad |= ix < 0 || ix >= sg.nvalid;
           }
           if (bad) atomicOr(p.status, kStatusBadIndex);
         }
@@ -231,7 +231,7 @@ __device__ __forceinline__ void tc_producers(const AttnMmaParams& P, unsigned ch
           const int r = pw * ROWS_W + i * RPI + lane / CH;
           const int c = lane % CH;
           const int32_t ix = (r < nrows) ? ring[r] : -1;
-          const bool ok = ix >= 0 && ix < p.n;
+          const bool ok = ix >= 0 && ix < sg.nvalid;
           const int64_t off = ok ? static_cast<int64_t>(ix) * s_token : 0;
           cp_async_16(kbase + tswz(r, c), kb + off + c * 8, ok ? 16u : 0u);
           cp_async_16(vbase + tswz(r, c), vb + off + c * 8, ok ? 16u : 0u);
@@ -506,7 +506,7 @@ __device__ __forceinline__ void tc_softmax(const AttnMmaParams& P, unsigned char
         // waited for them) before this read
         if (!mbar_wait(&br.full[t % STAGES], (t / STAGES) & 1, abort_flag, p.status)) return;
         const int32_t x = idxring[(t % C::IR) * kTcRows + kr];
-        valid = x >= 0 && x < p.n;
+        valid = x >= 0 && x < sg.nvalid;
       }
       float x[8];  // logits in log2 units; -inf for rows or queries not in use
       bool over = false;

@@ -44,6 +44,7 @@ cudaError_t topk_configure(int cl, size_t smem);
 cudaError_t topk_launch(int cl, const TopkParams* p, int ntasks, cudaStream_t stream);
 int topk_max_clusters(int cl, size_t smem);
 cudaError_t copy_sets_launch(const CopySetsParams* p, cudaStream_t stream);
+cudaError_t append_rows_launch(const AppendParams* p, cudaStream_t stream);
 cudaError_t validate_sets_launch(const ValidateSetsParams* p, cudaStream_t stream);
 }  // namespace lyc
 
@@ -81,6 +82,11 @@ struct Plan {
   int combine_grid = 1;       // bf16: CTAs of the launch that combines the last layer
   size_t off_empty_cta = 0;   // its CTA offsets (all zero: no pieces)
   int k = 0, keff = 0, n = 0;
+  std::vector<int64_t> nb;        // rows of each batch element
+  bool append = false;            // the step writes the current token's K and V first
+  bool paged = false;             // the cache is paged
+  AppendParams ap_append{};       // (its n array lives in the plan buffer)
+  size_t off_n = 0;
   uint32_t flags = 0;
   const void* q = nullptr;
   float* out = nullptr;
@@ -179,6 +185,56 @@ void free_plan(Plan* p) {
 
 namespace {
 
+// ---------------------------------------------------------------- KV views
+// The KV cache of one step, from either entry point: every batch element's
+// row count, and contiguous or paged rows (the layout of lyc_kv_batch).
+struct KvView {
+  const void* k = nullptr;
+  const void* v = nullptr;
+  int64_t nmax = 0;
+  std::vector<int64_t> n;  // per batch element
+  int64_t s_layer = 0, s_batch = 0, s_head = 0, s_token = 0, s_page = 0;
+  const int32_t* bt = nullptr;
+  int32_t page_rows = 0, max_blocks = 0;
+  int64_t num_pages = 0;
+  const void* k_new = nullptr;
+  const void* v_new = nullptr;
+  bool paged() const { return bt != nullptr; }
+};
+
+KvView view_of(const lyc_kv_cache* kv, int B) {
+  KvView w;
+  w.k = kv->k;
+  w.v = kv->v;
+  w.nmax = kv->n;
+  w.n.assign(B, kv->n);
+  w.s_layer = kv->s_layer;
+  w.s_batch = kv->s_batch;
+  w.s_head = kv->s_head;
+  w.s_token = kv->s_token;
+  return w;
+}
+
+KvView view_of(const lyc_kv_batch* kv, int B) {
+  KvView w;
+  w.k = kv->k;
+  w.v = kv->v;
+  w.n.assign(kv->n, kv->n + B);
+  for (int64_t x : w.n) w.nmax = std::max(w.nmax, x);
+  w.s_layer = kv->s_layer;
+  w.s_batch = kv->s_batch;
+  w.s_head = kv->s_head;
+  w.s_token = kv->s_token;
+  w.s_page = kv->s_page;
+  w.bt = kv->block_table;
+  w.page_rows = kv->page_rows;
+  w.max_blocks = kv->max_blocks;
+  w.num_pages = kv->num_pages;
+  w.k_new = kv->k_new;
+  w.v_new = kv->v_new;
+  return w;
+}
+
 // ---------------------------------------------------------------- tensor maps
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -197,25 +253,37 @@ EncodeTiledFn encode_tiled_fn() {
   return fn;
 }
 
-// 5-D map (d, row, KV head, batch, layer) of one cache tensor, 64 x 64 boxes
-// of 128-byte rows with the 128B swizzle; rows at or past n read as zeros.
-lyc_status encode_cache_map(lyc_ctx* ctx, CUtensorMap* map, const void* base, const lyc_kv_cache* kv,
+// 5-D map of one cache tensor, 64 x 64 boxes of 128-byte rows with the 128B
+// swizzle: contiguous rows (d, row, KV head, batch, layer), rows at or past
+// the longest element's n read as zeros; or paged (d, KV head, row in page,
+// page, layer), a box never crossing a page.
+lyc_status encode_cache_map(lyc_ctx* ctx, CUtensorMap* map, const void* base, const KvView& kv,
                             int tile_rows) {
   const lyc_config& c = ctx->cfg;
   EncodeTiledFn fn = encode_tiled_fn();
   if (!fn) return fail(ctx, LYC_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
-  const cuuint64_t dims[5] = {static_cast<cuuint64_t>(c.head_dim), static_cast<cuuint64_t>(kv->n),
-                              static_cast<cuuint64_t>(c.num_kv_heads), static_cast<cuuint64_t>(c.batch),
-                              static_cast<cuuint64_t>(c.num_layers)};
   const int64_t es = 2;
-  int64_t st[4] = {kv->s_token * es, kv->s_head * es, kv->s_batch * es, kv->s_layer * es};
+  cuuint64_t dims[5] = {static_cast<cuuint64_t>(c.head_dim), static_cast<cuuint64_t>(kv.nmax),
+                        static_cast<cuuint64_t>(c.num_kv_heads), static_cast<cuuint64_t>(c.batch),
+                        static_cast<cuuint64_t>(c.num_layers)};
+  int64_t st[4] = {kv.s_token * es, kv.s_head * es, kv.s_batch * es, kv.s_layer * es};
+  cuuint32_t box[5] = {64, static_cast<cuuint32_t>(tile_rows), 1, 1, 1};
+  if (kv.paged()) {
+    dims[1] = static_cast<cuuint64_t>(c.num_kv_heads);
+    dims[2] = static_cast<cuuint64_t>(kv.page_rows);
+    dims[3] = static_cast<cuuint64_t>(kv.num_pages);
+    st[0] = kv.s_head * es;
+    st[1] = kv.s_token * es;
+    st[2] = kv.s_page * es;
+    box[1] = 1;
+    box[2] = static_cast<cuuint32_t>(tile_rows);
+  }
   // a dimension of extent 1 is only ever read at coordinate 0: give it a
   // harmless stride if the caller passed 0
   for (int i = 0; i < 4; ++i)
     if (dims[i + 1] == 1 && st[i] == 0) st[i] = (i == 0 ? c.head_dim * es : st[i - 1] * static_cast<int64_t>(dims[i]));
   const cuuint64_t strides[4] = {static_cast<cuuint64_t>(st[0]), static_cast<cuuint64_t>(st[1]),
                                  static_cast<cuuint64_t>(st[2]), static_cast<cuuint64_t>(st[3])};
-  const cuuint32_t box[5] = {64, static_cast<cuuint32_t>(tile_rows), 1, 1, 1};
   const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box,
                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -230,28 +298,28 @@ lyc_status encode_cache_map(lyc_ctx* ctx, CUtensorMap* map, const void* base, co
 // (l*s_layer + b*s_batch + g*s_head)/s_token + i is token i of (l, b, g), or 0
 // when the strides do not allow one (a head, batch or layer stride that is
 // not a whole number of rows) or the rows do not fit a 32-bit coordinate.
-int64_t gather_map_rows(const lyc_config& c, const lyc_kv_cache* kv) {
-  const int64_t st = kv->s_token;
-  if (st <= 0) return 0;
-  if ((c.num_kv_heads > 1 && kv->s_head % st) || (c.batch > 1 && kv->s_batch % st) ||
-      (c.num_layers > 1 && kv->s_layer % st))
+int64_t gather_map_rows(const lyc_config& c, const KvView& kv) {
+  const int64_t st = kv.s_token;
+  if (st <= 0 || kv.paged()) return 0;
+  if ((c.num_kv_heads > 1 && kv.s_head % st) || (c.batch > 1 && kv.s_batch % st) ||
+      (c.num_layers > 1 && kv.s_layer % st))
     return 0;
-  if (kv->s_head < 0 || kv->s_batch < 0 || kv->s_layer < 0) return 0;
-  const int64_t last = (c.num_layers - 1) * kv->s_layer + (c.batch - 1) * kv->s_batch +
-                       (c.num_kv_heads - 1) * kv->s_head;
-  const int64_t rows = last / st + kv->n;
+  if (kv.s_head < 0 || kv.s_batch < 0 || kv.s_layer < 0) return 0;
+  const int64_t last = (c.num_layers - 1) * kv.s_layer + (c.batch - 1) * kv.s_batch +
+                       (c.num_kv_heads - 1) * kv.s_head;
+  const int64_t rows = last / st + kv.nmax;
   return rows < 0x7fffffffll ? rows : 0;
 }
 
 // The 2-D row-gather map of one cache tensor: boxes of one 128-byte row
 // (64 bf16), 128B swizzle, so that a four-row gather lands in the same
 // swizzled tile layout as the 5-D map's tiles.
-lyc_status encode_gather_map(lyc_ctx* ctx, CUtensorMap* map, const void* base, const lyc_kv_cache* kv,
+lyc_status encode_gather_map(lyc_ctx* ctx, CUtensorMap* map, const void* base, const KvView& kv,
                              int64_t rows) {
   EncodeTiledFn fn = encode_tiled_fn();
   if (!fn) return fail(ctx, LYC_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(ctx->cfg.head_dim), static_cast<cuuint64_t>(rows)};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kv->s_token * 2)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kv.s_token * 2)};
   const cuuint32_t box[2] = {64, 1};
   const cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
@@ -294,19 +362,21 @@ int pick_topk_cluster(const lyc_ctx* ctx, int ntasks) {
 // two buffers; a refreshed slot is written into the buffer it is not
 // currently read from, so a layer's readers and its own selection never touch
 // the same memory (double buffering), and unrefreshed slots cost no copy.
-lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const lyc_kv_cache* kv,
+lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const KvView& kv,
                       int k, uint32_t flags) {
   const lyc_config& cfg = ctx->cfg;
   const int L = cfg.num_layers, B = cfg.batch, Hq = cfg.num_q_heads, Hkv = cfg.num_kv_heads;
   const int G = ctx->G, Hs = ctx->Hs;
   const bool kvmode = cfg.select_mode == LYC_SELECT_KVGROUP_MEAN;
   const bool s_in = (flags & LYC_STEP_S_IN) != 0;
-  const int n = static_cast<int>(kv->n);
+  const int n = static_cast<int>(kv.nmax);  // the longest element's rows
   const int keff = std::min(k, n);
   const size_t es = cfg.dtype == LYC_BF16 ? 2 : 4;
   plan->k = k;
   plan->keff = keff;
   plan->n = n;
+  plan->nb = kv.n;
+  plan->paged = kv.paged();
   plan->nsets = B * Hs;
   plan->gather_rows = 0;
   // bf16 with head_dim 128 runs on the tcgen05 kernel (128-row tiles) when
@@ -318,13 +388,13 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const lyc_k
   // of consecutive layers may overlap, see enqueue)
   const bool use_pool = cfg.dtype == LYC_BF16 && !plan->use_tc;
   if (cfg.dtype == LYC_BF16) {
-    lyc_status st = encode_cache_map(ctx, &plan->tmk, kv->k, kv, TR);
-    if (st == LYC_OK) st = encode_cache_map(ctx, &plan->tmv, kv->v, kv, TR);
+    lyc_status st = encode_cache_map(ctx, &plan->tmk, kv.k, kv, TR);
+    if (st == LYC_OK) st = encode_cache_map(ctx, &plan->tmv, kv.v, kv, TR);
     if (st != LYC_OK) return st;
     const int64_t rows = (cfg.flags & LYC_CFG_TMA_GATHER) ? gather_map_rows(cfg, kv) : 0;
     if (rows > 0) {
-      st = encode_gather_map(ctx, &plan->tgk, kv->k, kv, rows);
-      if (st == LYC_OK) st = encode_gather_map(ctx, &plan->tgv, kv->v, kv, rows);
+      st = encode_gather_map(ctx, &plan->tgk, kv.k, kv, rows);
+      if (st == LYC_OK) st = encode_gather_map(ctx, &plan->tgv, kv.v, kv, rows);
       if (st != LYC_OK) return st;
       plan->gather_rows = static_cast<int32_t>(rows);
     }
@@ -349,8 +419,8 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const lyc_k
   auto set_ptr = [&](int buf, int b, int s) {
     return ctx->sbuf + ((static_cast<int64_t>(buf) * B + b) * Hs + s) * ctx->KS;
   };
-  const char* kbase = static_cast<const char*>(kv->k);
-  const char* vbase = static_cast<const char*>(kv->v);
+  const char* kbase = static_cast<const char*>(kv.k);
+  const char* vbase = static_cast<const char*>(kv.v);
 
   std::vector<char> prev_fresh(Hs, 1);  // slots the previous layer's selection wrote
   std::vector<int> writer(Hs, -1);      // layer whose selection wrote each slot's current set
@@ -371,13 +441,22 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const lyc_k
     }
     int maxnq = 1;
     for (int b = 0; b < B; ++b) {
+      const int nb = static_cast<int>(kv.n[b]);  // this element's rows
+      const int keffb = std::min(k, nb);
       for (int g = 0; g < Hkv; ++g) {
-        const int64_t off = l * kv->s_layer + b * kv->s_batch + g * kv->s_head;
+        // row 0 of (l, b, g); paged: of page 0, rows found through b's block table
+        const int64_t off = l * kv.s_layer + (kv.paged() ? 0 : b * kv.s_batch) + g * kv.s_head;
         Segment base{};
         base.k = kbase + off * es;
         base.v = vbase + off * es;
-        base.s_token = kv->s_token;
-        base.row_base = plan->gather_rows > 0 ? static_cast<int32_t>(off / kv->s_token) : 0;
+        base.s_token = kv.s_token;
+        base.row_base = plan->gather_rows > 0 ? static_cast<int32_t>(off / kv.s_token) : 0;
+        base.nvalid = nb;
+        if (kv.paged()) {
+          base.bt = kv.bt + static_cast<int64_t>(b) * kv.max_blocks;
+          base.page_rows = kv.page_rows;
+          base.s_page = kv.s_page;
+        }
         base.l = l;
         base.b = b;
         base.g = g;
@@ -391,7 +470,7 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const lyc_k
         // of the group, whose mean logit is the group's selection key
         Segment ds = base;
         ds.kind = kDense;
-        ds.rows = n;
+        ds.rows = nb;
         int nret = 0;
         for (int h = g * G; h < (g + 1) * G; ++h) nret += is_ret[h];
         if (nret > 0) {
@@ -413,7 +492,7 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const lyc_k
         if (kvmode) {
           Segment ss = base;
           ss.kind = kSparse;
-          ss.rows = keff;
+          ss.rows = keffb;
           ss.idx = set_ptr(cur[g], b, g);
           int js = 0;
           for (int h = g * G; h < (g + 1) * G; ++h)
@@ -433,7 +512,7 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const lyc_k
             if (is_ret[h]) continue;
             Segment ss = base;
             ss.kind = kSparse;
-            ss.rows = keff;
+            ss.rows = keffb;
             ss.idx = set_ptr(cur[h], b, h);
             ss.head[0] = h;
             ss.out_row[0] = 0;
@@ -512,13 +591,17 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const lyc_k
       }
     }
     if (use_pool) {
-      // every sparse segment has keff rows: ups units each, unit q = ordinal q
-      H.pool_ups = static_cast<int>((keff + kPoolTiles * kTileRows - 1) / (kPoolTiles * kTileRows));
+      // a sparse segment of r rows has ceil(r / unit) units, unit q = ordinal q;
+      // the pool counts pool_ups per segment (the most any has), and the
+      // scheduler skips the units past a shorter segment's end
+      constexpr int kUnitRows = kPoolTiles * kTileRows;
       for (int dep = 0; dep < 2; ++dep)
         for (size_t s2 = 0; s2 < H.segs.size(); ++s2)
           if (H.segs[s2].kind == kSparse && H.segs[s2].dep == dep) {
+            const int units = (H.segs[s2].rows + kUnitRows - 1) / kUnitRows;
             H.pool_segs.push_back(static_cast<int32_t>(s2));
-            npieces[s2] = H.pool_ups;
+            H.pool_ups = std::max(H.pool_ups, units);
+            npieces[s2] = units;
             H.pool_tiles += (H.segs[s2].rows + TR - 1) / TR;
           }
     }
@@ -552,6 +635,7 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const lyc_k
         tk.keys = ctx->keys + keys_base + (static_cast<int64_t>(b) * Hs + s) * ctx->nstride;
         tk.S = set_ptr(1 - cur[s], b, s);
         tk.done = ctx->flags + ((static_cast<int64_t>(l) * B + b) * Hs + s) * 2;
+        tk.n = static_cast<int32_t>(kv.n[b]);
         H.tasks.push_back(tk);
       }
     }
@@ -598,6 +682,7 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const lyc_k
     lp.off_pool = take(std::max<size_t>(1, H.pool_segs.size()) * sizeof(int32_t));
   }
   plan->off_final_src = take(hl[L - 1].trace_src.size() * sizeof(void*));
+  plan->off_n = take(static_cast<size_t>(B) * sizeof(int64_t));
   // the last layer's combine runs in a launch of its own, whose CTAs have no pieces
   plan->combine_grid = std::max(1, std::min(ctx->sms, plan->layers[L - 1].ncombine));
   plan->off_empty_cta = take((plan->combine_grid + 1) * sizeof(int32_t));
@@ -618,8 +703,31 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const lyc_k
   }
   memcpy(host.data() + plan->off_final_src, hl[L - 1].trace_src.data(),
          hl[L - 1].trace_src.size() * sizeof(void*));
+  memcpy(host.data() + plan->off_n, kv.n.data(), static_cast<size_t>(B) * sizeof(int64_t));
   LYC_CUDA(cudaMalloc(&plan->dev, bytes), "cudaMalloc(plan)");
   plan->dev_bytes = bytes;
+  if (kv.k_new) {
+    AppendParams& a = plan->ap_append;
+    a.k_new = static_cast<const unsigned char*>(kv.k_new);
+    a.v_new = static_cast<const unsigned char*>(kv.v_new);
+    a.k = static_cast<unsigned char*>(const_cast<void*>(kv.k));
+    a.v = static_cast<unsigned char*>(const_cast<void*>(kv.v));
+    a.n = reinterpret_cast<const int64_t*>(plan->dev + plan->off_n);
+    a.s_layer = kv.s_layer;
+    a.s_batch = kv.s_batch;
+    a.s_head = kv.s_head;
+    a.s_token = kv.s_token;
+    a.s_page = kv.s_page;
+    a.bt = kv.bt;
+    a.page_rows = kv.page_rows;
+    a.max_blocks = kv.max_blocks;
+    a.L = L;
+    a.B = B;
+    a.Hkv = Hkv;
+    a.elem_bytes = static_cast<int32_t>(es);
+    a.row_bytes = static_cast<int32_t>(cfg.head_dim * es);
+    plan->append = true;
+  }
   LYC_CUDA(cudaMemcpy(plan->dev, host.data(), bytes, cudaMemcpyHostToDevice), "upload plan");
   return LYC_OK;
 }
@@ -662,14 +770,21 @@ lyc_status enqueue_step(lyc_ctx* ctx, Plan* plan, cudaStream_t stream, int set, 
   const int L = cfg.num_layers, B = cfg.batch, Hq = cfg.num_q_heads, D = cfg.head_dim;
   const size_t es = cfg.dtype == LYC_BF16 ? 2 : 4;
   const int dtype = cfg.dtype == LYC_BF16 ? 0 : 1;
+  // the current token's K and V into the cache, before any layer reads it
+  if (plan->append) LYC_CUDA(append_rows_launch(&plan->ap_append, stream), "append K/V rows");
   if (plan->flags & LYC_STEP_S_IN) {
     LYC_CUDA(cudaMemcpy2DAsync(ctx->sbuf, ctx->KS * sizeof(int32_t), plan->S, plan->k * sizeof(int32_t),
                                plan->k * sizeof(int32_t), static_cast<size_t>(B) * ctx->Hs,
                                cudaMemcpyDeviceToDevice, stream),
              "copy S^(0) in");
     if (plan->flags & LYC_STEP_VALIDATE_S) {
-      ValidateSetsParams vp{ctx->sbuf, ctx->status, B * ctx->Hs, ctx->KS, plan->k, plan->keff, plan->n};
-      LYC_CUDA(validate_sets_launch(&vp, stream), "validate S^(0)");
+      // per batch element: its sets hold min(k, n[b]) indices below n[b]
+      for (int b = 0; b < B; ++b) {
+        const int nb = static_cast<int>(plan->nb[b]);
+        ValidateSetsParams vp{ctx->sbuf + static_cast<int64_t>(b) * ctx->Hs * ctx->KS, ctx->status, ctx->Hs,
+                              ctx->KS, plan->k, std::min(plan->k, nb), nb};
+        LYC_CUDA(validate_sets_launch(&vp, stream), "validate S^(0)");
+      }
     }
   }
   plan->kernel_kind.clear();
@@ -715,7 +830,6 @@ lyc_status enqueue_step(lyc_ctx* ctx, Plan* plan, cudaStream_t stream, int set, 
       ap.pool_segs = reinterpret_cast<const int32_t*>(plan->dev + lp.off_pool);
       ap.pool_n = lp.pool_nsegs * lp.pool_ups;
       ap.pool_ups = lp.pool_ups;
-      ap.pool_rows = plan->keff;
       ap.pool_stride = L + 1;
       ap.pool_cursors = ctx->pool_cursors;
     }
@@ -745,6 +859,7 @@ lyc_status enqueue_step(lyc_ctx* ctx, Plan* plan, cudaStream_t stream, int set, 
       mp.tgv = plan->tgv;
       mp.p = ap;
       mp.p.gather_rows = plan->gather_rows;
+      mp.p.paged = plan->paged ? 1 : 0;
       if (l > 0) set_prev_combine(ctx, plan, l - 1, &mp.p);
       LYC_CUDA(plan->use_tc ? attn_tc_dispatch(&mp, lp.grid, stream, nullptr, false)
                             : attn_mma_dispatch(D, &mp, lp.grid, stream, nullptr, false),
@@ -863,12 +978,21 @@ lyc_status capture_plan(lyc_ctx* ctx, Plan* plan) {
   return LYC_OK;
 }
 
-std::string plan_key(const uint8_t* role, int L, int Hq, const lyc_kv_cache* kv, int k,
+std::string plan_key(const uint8_t* role, int L, int Hq, const KvView& kv, int k,
                      uint32_t flags, const void* q, const float* out, const int32_t* S,
                      const int32_t* trace, bool timing) {
   std::string key(reinterpret_cast<const char*>(role), static_cast<size_t>(L) * Hq);
   auto add = [&](const void* p, size_t n) { key.append(static_cast<const char*>(p), n); };
-  add(kv, sizeof(*kv));
+  add(&kv.k, sizeof kv.k);
+  add(&kv.v, sizeof kv.v);
+  add(kv.n.data(), kv.n.size() * sizeof(int64_t));
+  const int64_t st[5] = {kv.s_layer, kv.s_batch, kv.s_head, kv.s_token, kv.s_page};
+  add(st, sizeof st);
+  add(&kv.bt, sizeof kv.bt);
+  const int64_t pg[3] = {kv.page_rows, kv.max_blocks, kv.num_pages};
+  add(pg, sizeof pg);
+  add(&kv.k_new, sizeof kv.k_new);
+  add(&kv.v_new, sizeof kv.v_new);
   add(&k, sizeof k);
   const uint32_t f = flags & (LYC_STEP_S_IN | LYC_STEP_VALIDATE_S);
   add(&f, sizeof f);
@@ -922,6 +1046,42 @@ lyc_status check_kv(lyc_ctx* ctx, const lyc_kv_cache* kv) {
     if ((s * es) % 16 != 0) return fail(ctx, LYC_ERR_INVALID_ARG, "kv strides must be multiples of 16 bytes");
   if ((reinterpret_cast<uintptr_t>(kv->k) | reinterpret_cast<uintptr_t>(kv->v)) & 15u)
     return fail(ctx, LYC_ERR_INVALID_ARG, "kv base pointers must be 16-byte aligned");
+  return LYC_OK;
+}
+
+lyc_status check_kv_batch(lyc_ctx* ctx, const lyc_kv_batch* kv) {
+  const lyc_config& c = ctx->cfg;
+  const int64_t es = c.dtype == LYC_BF16 ? 2 : 4;
+  if (!kv || !kv->k || !kv->v || !kv->n) return fail(ctx, LYC_ERR_INVALID_ARG, "kv pointer is NULL");
+  int64_t nmax = 0;
+  for (int b = 0; b < c.batch; ++b) {
+    if (kv->n[b] < 1 || kv->n[b] > c.max_ctx)
+      return fail(ctx, LYC_ERR_INVALID_ARG, "kv->n[b] outside [1, max_ctx]");
+    nmax = std::max(nmax, kv->n[b]);
+  }
+  const bool paged = kv->block_table != nullptr;
+  if (kv->s_token < c.head_dim || kv->s_head < c.head_dim)
+    return fail(ctx, LYC_ERR_INVALID_ARG, "s_token and s_head must be at least head_dim");
+  if (kv->s_layer < 0 || kv->s_batch < 0 || kv->s_page < 0)
+    return fail(ctx, LYC_ERR_INVALID_ARG, "negative kv stride");
+  const int64_t strides[5] = {kv->s_layer, paged ? 0 : kv->s_batch, kv->s_head, kv->s_token,
+                              paged ? kv->s_page : 0};
+  for (int64_t s : strides)
+    if ((s * es) % 16 != 0) return fail(ctx, LYC_ERR_INVALID_ARG, "kv strides must be multiples of 16 bytes");
+  if ((reinterpret_cast<uintptr_t>(kv->k) | reinterpret_cast<uintptr_t>(kv->v)) & 15u)
+    return fail(ctx, LYC_ERR_INVALID_ARG, "kv base pointers must be 16-byte aligned");
+  if (paged) {
+    if (c.dtype != LYC_BF16 || (c.flags & LYC_CFG_TCGEN05))
+      return fail(ctx, LYC_ERR_UNSUPPORTED, "a paged cache needs bf16 on the default (mma.sync) kernel");
+    if (kv->page_rows < 64 || kv->page_rows % 64 != 0)
+      return fail(ctx, LYC_ERR_INVALID_ARG, "page_rows must be a positive multiple of 64");
+    if (kv->max_blocks < (nmax + kv->page_rows - 1) / kv->page_rows || kv->num_pages < 1 || kv->s_page < 1)
+      return fail(ctx, LYC_ERR_INVALID_ARG, "block table too short, or no pages");
+  }
+  if ((kv->k_new == nullptr) != (kv->v_new == nullptr))
+    return fail(ctx, LYC_ERR_INVALID_ARG, "k_new and v_new must both be given or both NULL");
+  if ((reinterpret_cast<uintptr_t>(kv->k_new) | reinterpret_cast<uintptr_t>(kv->v_new)) & 15u)
+    return fail(ctx, LYC_ERR_INVALID_ARG, "k_new and v_new must be 16-byte aligned");
   return LYC_OK;
 }
 
@@ -1093,18 +1253,12 @@ void lyc_destroy(lyc_ctx* ctx) {
 
 }  // extern "C"
 
-extern "C" {
+namespace {
 
-lyc_status lyc_decode_step(lyc_ctx* ctx, const void* q, const lyc_kv_cache* kv,
-                           const uint8_t* role_mask, int k, float* out, int32_t* S,
-                           void* stream_, uint32_t step_flags) {
-  if (!ctx) return LYC_ERR_INVALID_ARG;
-  if (!q || !role_mask || !out || !S) return fail(ctx, LYC_ERR_INVALID_ARG, "NULL tensor pointer");
-  if (k < 1 || k > ctx->cfg.max_k) return fail(ctx, LYC_ERR_INVALID_ARG, "k outside [1, max_k]");
-  if (step_flags & ~(LYC_STEP_S_IN | LYC_STEP_NO_GRAPH | LYC_STEP_VALIDATE_S))
-    return fail(ctx, LYC_ERR_INVALID_ARG, "unknown step flag");
-  lyc_status st = check_kv(ctx, kv);
-  if (st != LYC_OK) return st;
+// The step on a checked KV view (both entry points).
+lyc_status step_impl(lyc_ctx* ctx, const void* q, const KvView& kv, const uint8_t* role_mask, int k,
+                     float* out, int32_t* S, void* stream_, uint32_t step_flags) {
+  lyc_status st = LYC_OK;
   DeviceGuard guard(ctx->cfg.device);
   if (!guard.ok) return fail(ctx, LYC_ERR_CUDA, "cudaSetDevice failed");
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
@@ -1172,6 +1326,39 @@ lyc_status lyc_decode_step(lyc_ctx* ctx, const void* q, const lyc_kv_cache* kv,
   }
   ctx->last_stream = stream;
   return LYC_OK;
+}
+
+lyc_status check_step_args(lyc_ctx* ctx, const void* q, const uint8_t* role_mask, int k, const float* out,
+                           const int32_t* S, uint32_t step_flags) {
+  if (!q || !role_mask || !out || !S) return fail(ctx, LYC_ERR_INVALID_ARG, "NULL tensor pointer");
+  if (k < 1 || k > ctx->cfg.max_k) return fail(ctx, LYC_ERR_INVALID_ARG, "k outside [1, max_k]");
+  if (step_flags & ~(LYC_STEP_S_IN | LYC_STEP_NO_GRAPH | LYC_STEP_VALIDATE_S))
+    return fail(ctx, LYC_ERR_INVALID_ARG, "unknown step flag");
+  return LYC_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+lyc_status lyc_decode_step(lyc_ctx* ctx, const void* q, const lyc_kv_cache* kv,
+                           const uint8_t* role_mask, int k, float* out, int32_t* S,
+                           void* stream_, uint32_t step_flags) {
+  if (!ctx) return LYC_ERR_INVALID_ARG;
+  lyc_status st = check_step_args(ctx, q, role_mask, k, out, S, step_flags);
+  if (st == LYC_OK) st = check_kv(ctx, kv);
+  if (st != LYC_OK) return st;
+  return step_impl(ctx, q, view_of(kv, ctx->cfg.batch), role_mask, k, out, S, stream_, step_flags);
+}
+
+lyc_status lyc_decode_step_batch(lyc_ctx* ctx, const void* q, const lyc_kv_batch* kv,
+                                 const uint8_t* role_mask, int k, float* out, int32_t* S,
+                                 void* stream_, uint32_t step_flags) {
+  if (!ctx) return LYC_ERR_INVALID_ARG;
+  lyc_status st = check_step_args(ctx, q, role_mask, k, out, S, step_flags);
+  if (st == LYC_OK) st = check_kv_batch(ctx, kv);
+  if (st != LYC_OK) return st;
+  return step_impl(ctx, q, view_of(kv, ctx->cfg.batch), role_mask, k, out, S, stream_, step_flags);
 }
 
 lyc_status lyc_decode_step_host(lyc_ctx* ctx, const void* q_host, const lyc_kv_cache* kv,

@@ -65,6 +65,11 @@ struct Segment {
   const uint32_t* ready;  // sparse: flag word of the selection that wrote the set in
                           // this step (it holds the step's epoch + 1 once the set is
                           // complete), or NULL when the set comes from the caller
+  int32_t nvalid;         // rows of (l, b): inherited indices must lie in [0, nvalid)
+  int32_t page_rows;      // paged cache: rows per page; 0: contiguous rows
+  const int32_t* bt;      // paged cache: the block-table row of b (row i is in page bt[i / page_rows],
+                          // at k + page * s_page + (i % page_rows) * s_token); NULL: contiguous
+  int64_t s_page;         // paged cache: element stride between pages
 };
 
 struct Piece {
@@ -107,8 +112,8 @@ struct AttnParams {
   // pool_segs[u / pool_ups], q = u % pool_ups, ordinal q (its partial record)
   const int32_t* pool_segs;
   int32_t pool_n;            // units in the pool (0: none)
-  int32_t pool_ups;          // units per pool segment
-  int32_t pool_rows;         // rows of every pool segment
+  int32_t pool_ups;          // units per pool segment (the most any has; a unit past a
+                             // segment's rows is skipped)
   int32_t pool_stride;       // cursors per epoch parity
   int32_t* pool_cursors;     // [2][pool_stride]: this launch's is [(epoch & 1)][layer]
   int32_t wpart_by_sm;       // 1: the piece-state ring of a CTA is the one of the SM it runs
@@ -118,6 +123,7 @@ struct AttnParams {
   int32_t timeline_cap;
   int32_t layer;
   int32_t Hq, G, n;
+  int32_t paged;             // 1: the segments' rows are in pages (Segment::bt)
   int32_t gather_rows;       // rows of the flattened row-gather maps (an index past
                              // the last row, used for rows that must read as zeros);
                              // 0: no such maps, gathered rows come by cp.async
@@ -130,6 +136,8 @@ struct TopkTask {
   int32_t* S;         // k outputs
   uint32_t* done;     // NULL, or {arrival counter, ready flag}: the last CTA of the task
                       // to finish resets the counter and sets the flag to epoch + 1
+  int32_t n;          // keys of this task (a batch element's rows); 0: the launch's n
+  int32_t pad_;
 };
 
 struct TopkParams {
@@ -156,6 +164,23 @@ struct CopySetsParams {
   uint32_t* epoch;  // the step's last launch: advance the epoch once the copy is done (or NULL)
   int32_t* pool_cursors;  // with epoch: zero the next step's pool cursors, [2][pool_stride]
   int32_t pool_stride;
+};
+
+// append_rows_kernel: the current token's K and V ([L][B][Hkv][row_bytes]
+// each, contiguous) written at row n[b]-1 of every (l, b, g) of the cache:
+// element offset l*s_layer + g*s_head + b*s_batch + i*s_token (contiguous), or
+// l*s_layer + g*s_head + bt[b*max_blocks + i/page_rows]*s_page +
+// (i % page_rows)*s_token (paged), i = n[b] - 1; times elem_bytes
+struct AppendParams {
+  const unsigned char* k_new;
+  const unsigned char* v_new;
+  unsigned char* k;
+  unsigned char* v;
+  const int64_t* n;  // device, [B]
+  int64_t s_layer, s_batch, s_head, s_token, s_page;
+  const int32_t* bt;
+  int32_t page_rows, max_blocks;
+  int32_t L, B, Hkv, row_bytes, elem_bytes;
 };
 
 // validate_sets_kernel: each of nsets sets (stride `stride`) must hold k_eff

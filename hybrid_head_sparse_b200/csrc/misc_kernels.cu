@@ -42,6 +42,37 @@ __global__ void validate_sets_kernel(const ValidateSetsParams p) {
   if (bad) atomicOr(p.status, kStatusBadIndex);
 }
 
+// One block per (l, b, g): 16-byte chunks of the K row, then of the V row.
+__global__ void append_rows_kernel(const AppendParams p) {
+  const int lbg = blockIdx.x;
+  const int g = lbg % p.Hkv;
+  const int b = (lbg / p.Hkv) % p.B;
+  const int l = lbg / (p.Hkv * p.B);
+  const int64_t i = p.n[b] - 1;
+  int64_t off = static_cast<int64_t>(l) * p.s_layer + static_cast<int64_t>(g) * p.s_head;
+  if (p.bt)
+    off += static_cast<int64_t>(p.bt[static_cast<int64_t>(b) * p.max_blocks + i / p.page_rows]) * p.s_page +
+           (i % p.page_rows) * p.s_token;
+  else
+    off += static_cast<int64_t>(b) * p.s_batch + i * p.s_token;
+  const int64_t dst = off * p.elem_bytes;
+  const int64_t src = static_cast<int64_t>(lbg) * p.row_bytes;
+  const int chunks = p.row_bytes / 16;
+  for (int c = threadIdx.x; c < 2 * chunks; c += blockDim.x) {
+    const bool isv = c >= chunks;
+    const int cc = isv ? c - chunks : c;
+    const uint4 x = *reinterpret_cast<const uint4*>((isv ? p.v_new : p.k_new) + src + 16 * cc);
+    *reinterpret_cast<uint4*>((isv ? p.v : p.k) + dst + 16 * cc) = x;
+  }
+}
+
+cudaError_t append_rows_launch(const AppendParams* p, cudaStream_t stream) {
+  const int blocks = p->L * p->B * p->Hkv;
+  if (blocks <= 0) return cudaSuccess;
+  append_rows_kernel<<<blocks, 64, 0, stream>>>(*p);
+  return cudaGetLastError();
+}
+
 cudaError_t copy_sets_launch(const CopySetsParams* p, cudaStream_t stream) {
   if (p->nsets <= 0) return cudaSuccess;  // never the case: a step has B * Hs >= 1 sets
   copy_sets_kernel<<<p->nsets, 256, 0, stream>>>(*p);

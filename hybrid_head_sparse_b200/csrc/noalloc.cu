@@ -210,6 +210,7 @@ extern "C" lyc_status lyc_sparse_attention_noalloc(const void* q, const lyc_kv_c
       sg.b = b;
       sg.g = g;
       sg.rows = keff;
+      sg.nvalid = static_cast<int32_t>(n);
       sg.nq = sg.nout = 1;
       sg.dep = 1;  // the caller's sets: read after whatever ran before on the stream
       sg.head[0] = h;

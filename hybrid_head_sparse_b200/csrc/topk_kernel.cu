@@ -189,7 +189,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster_kernel(const Top
   constexpr unsigned FULL = 0xffffffffu;
   const int rank = static_cast<int>(cluster.block_rank());
   const TopkTask task = p.tasks ? p.tasks[blockIdx.y] : p.single;
-  const int n = p.n;
+  const int n = task.n > 0 ? task.n : p.n;
   const int k = p.k;
   const int keff = k < n ? k : n;
   const int chunk = (((n + CL - 1) / CL) + 3) & ~3;

@@ -43,7 +43,8 @@ LYC_STEP_VALIDATE_S = 0x4
 LYC_TIMING_OFF = 0
 LYC_TIMING_ON = 1
 
-EXPORTED = ["lyc_create", "lyc_decode_step", "lyc_decode_step_host", "lyc_sync_status",
+EXPORTED = ["lyc_create", "lyc_decode_step", "lyc_decode_step_host", "lyc_decode_step_batch",
+            "lyc_sync_status",
             "lyc_set_s_trace", "lyc_step_bytes", "lyc_topk_f32", "lyc_set_timing",
             "lyc_kernel_times", "lyc_set_timeline", "lyc_status_string", "lyc_last_error",
             "lyc_destroy", "lyc_sparse_attention_noalloc"]
@@ -62,6 +63,16 @@ class lyc_kv_cache(ctypes.Structure):
     _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("n", ctypes.c_int64),
                 ("s_layer", ctypes.c_int64), ("s_batch", ctypes.c_int64),
                 ("s_head", ctypes.c_int64), ("s_token", ctypes.c_int64)]
+
+
+class lyc_kv_batch(ctypes.Structure):
+    _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("n", ctypes.c_void_p),
+                ("s_layer", ctypes.c_int64), ("s_batch", ctypes.c_int64),
+                ("s_head", ctypes.c_int64), ("s_token", ctypes.c_int64),
+                ("s_page", ctypes.c_int64), ("block_table", ctypes.c_void_p),
+                ("page_rows", ctypes.c_int32), ("max_blocks", ctypes.c_int32),
+                ("num_pages", ctypes.c_int64), ("k_new", ctypes.c_void_p),
+                ("v_new", ctypes.c_void_p)]
 
 
 class lyc_kernel_time(ctypes.Structure):
@@ -92,6 +103,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     L.lyc_decode_step.argtypes = [P, P, ctypes.POINTER(lyc_kv_cache), P, I, P, P, P, ctypes.c_uint32]
     L.lyc_decode_step_host.argtypes = [P, P, ctypes.POINTER(lyc_kv_cache), P, I, P, P, P,
                                        ctypes.c_uint32]
+    L.lyc_decode_step_batch.argtypes = [P, P, ctypes.POINTER(lyc_kv_batch), P, I, P, P, P,
+                                        ctypes.c_uint32]
     L.lyc_sync_status.argtypes = [P]
     L.lyc_set_s_trace.argtypes = [P, P]
     L.lyc_step_bytes.argtypes = [ctypes.POINTER(lyc_config), P, ctypes.c_int64, I, I,
@@ -133,6 +146,11 @@ def lyc_decode_step(ctx, q, kv: lyc_kv_cache, role_mask, k, out, S, stream, flag
 def lyc_decode_step_host(ctx, q, kv: lyc_kv_cache, role_mask, k, out, S, stream, flags) -> int:
     return load().lyc_decode_step_host(ctx, q, ctypes.byref(kv), role_mask, k, out, S, stream,
                                        flags)
+
+
+def lyc_decode_step_batch(ctx, q, kv: lyc_kv_batch, role_mask, k, out, S, stream, flags) -> int:
+    return load().lyc_decode_step_batch(ctx, q, ctypes.byref(kv), role_mask, k, out, S, stream,
+                                        flags)
 
 
 def lyc_sparse_attention_noalloc(q, kv: lyc_kv_cache, batch, num_q_heads, num_kv_heads,
@@ -273,6 +291,38 @@ class Lyc:
         rc = lyc_decode_step(self.ctx, q.data_ptr(), kv, role.ctypes.data, k, out.data_ptr(),
                              S.data_ptr(), _stream_ptr(stream), flags)
         self._check(rc, "lyc_decode_step")
+
+    def decode_step_batch(self, q, K, V, n, role_mask, k, out, S, stream=None, s_in=False,
+                          validate_s=False, k_new=None, v_new=None, block_table=None,
+                          page_rows=0, strides=None):
+        """The serving form: n is a sequence of B row counts.  Contiguous cache:
+        K, V are [L][B][Hkv][rows][d]-strided tensors.  Paged cache: K, V are
+        [L][pages][page_rows][Hkv][d] tensors and block_table a device int32
+        [B][max_blocks] tensor.  k_new/v_new: [L][B][Hkv][d] rows appended at
+        n[b]-1 before attention, or None.  strides: optional (s_layer, s_batch,
+        s_head, s_token, s_page) override in elements."""
+        role = np.ascontiguousarray(role_mask, dtype=np.uint8)
+        nn = np.ascontiguousarray(np.asarray(n, dtype=np.int64))
+        self._role, self._n = role, nn  # keep alive while the call runs
+        flags = (LYC_STEP_S_IN if s_in else 0) | (LYC_STEP_VALIDATE_S if validate_s else 0)
+        assert K.stride() == V.stride() and K.shape == V.shape and K.stride(-1) == 1
+        st = K.stride()
+        if strides is not None:
+            s_layer, s_batch, s_head, s_token, s_page = strides
+        elif block_table is None:
+            s_layer, s_batch, s_head, s_token, s_page = st[0], st[1], st[2], st[3], 0
+        else:
+            s_layer, s_batch, s_head, s_token, s_page = st[0], 0, st[3], st[2], st[1]
+        kv = lyc_kv_batch(K.data_ptr(), V.data_ptr(), nn.ctypes.data, s_layer, s_batch, s_head,
+                          s_token, s_page,
+                          None if block_table is None else block_table.data_ptr(),
+                          int(page_rows), 0 if block_table is None else int(block_table.shape[1]),
+                          0 if block_table is None else int(K.shape[1]),
+                          None if k_new is None else k_new.data_ptr(),
+                          None if v_new is None else v_new.data_ptr())
+        rc = lyc_decode_step_batch(self.ctx, q.data_ptr(), kv, role.ctypes.data, k,
+                                   out.data_ptr(), S.data_ptr(), _stream_ptr(stream), flags)
+        self._check(rc, "lyc_decode_step_batch")
 
     def decode_step_host(self, q_host, K, V, n, role_mask, k, out_host, S_host, stream=None,
                          s_in=False):

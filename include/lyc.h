@@ -146,6 +146,52 @@ lyc_status lyc_decode_step_host(lyc_ctx* ctx, const void* q_host, const lyc_kv_c
                                 const uint8_t* role_mask, int k, float* out_host,
                                 int32_t* S_host, void* stream, uint32_t step_flags);
 
+/* The serving form of the step: a batch whose elements have cache lengths of
+ * their own, the cache either contiguous (as lyc_kv_cache) or in pages named
+ * by a block table, and the current token's K and V written into the cache
+ * as part of the step.  Page "LycheeDecode ..." (paper-graph-ui summary),
+ * Appendix B, Algorithm 1: each decode step appends the current token's K and
+ * V to the cache before the layer's attention; the attention and selection of
+ * every batch element then run over its own n[b] rows exactly as in
+ * lyc_decode_step (section 3.4 Eq. 1-3).
+ *
+ * Row i < n[b] of (layer l, batch b, KV head g), element j < d:
+ *   contiguous (block_table == NULL):
+ *     l*s_layer + b*s_batch + g*s_head + i*s_token + j
+ *   paged (block_table != NULL): page p = block_table[b*max_blocks + i/page_rows],
+ *     l*s_layer + p*s_page + (i % page_rows)*s_token + g*s_head + j
+ * (s_batch is unused when paged; s_page when contiguous).  Strides are in
+ * elements and must keep every row 16-byte aligned; page_rows is a multiple
+ * of 64; every page a batch element uses lies in the allocation and is used
+ * by that element only. */
+typedef struct {
+  const void* k;               /* device: K (the cache, or the page pool) */
+  const void* v;               /* device: V, same layout */
+  const int64_t* n;            /* host, [B]: rows of each element, its current token included */
+  int64_t s_layer, s_batch, s_head, s_token, s_page;
+  const int32_t* block_table;  /* device, [B][max_blocks] page indices, or NULL (contiguous) */
+  int32_t page_rows;           /* rows per page (paged) */
+  int32_t max_blocks;          /* block-table row length (paged) */
+  int64_t num_pages;           /* pages in the pool, every block-table entry below it (paged) */
+  const void* k_new;           /* device, [L][B][Hkv][d] of cfg->dtype: the current token's K,
+                                  written at row n[b]-1 of every (l, b, g) before attention;
+                                  or NULL (the cache already holds it) */
+  const void* v_new;           /* device, the same for V (NULL iff k_new is NULL) */
+} lyc_kv_batch;
+
+/* One decode step over a lyc_kv_batch; q, role_mask, k, out, S, stream and
+ * step_flags as in lyc_decode_step (LYC_STEP_S_IN: each S^(0) set of element
+ * b must hold indices below n[b]).  Every n[b] is >= 1 and <= cfg->max_ctx;
+ * element b's sets hold min(k, n[b]) indices, padded with -1.  The appended
+ * rows are written before any layer reads the cache and stay in it after the
+ * step (the caller's cache is modified).
+ * Errors: INVALID_ARG (NULL pointers, n out of range, page_rows not a
+ * multiple of 64, misaligned strides), UNSUPPORTED (paged layout with the
+ * tcgen05 kernel or fp32), CUDA; BAD_INDEX, TIMEOUT via lyc_sync_status. */
+lyc_status lyc_decode_step_batch(lyc_ctx* ctx, const void* q, const lyc_kv_batch* kv,
+                                 const uint8_t* role_mask, int k, float* out, int32_t* S,
+                                 void* stream, uint32_t step_flags);
+
 /* Synchronize the stream of the last step, read and clear the device status
  * word.  Returns LYC_OK, LYC_ERR_BAD_INDEX, LYC_ERR_TIMEOUT or LYC_ERR_CUDA. */
 lyc_status lyc_sync_status(lyc_ctx* ctx);

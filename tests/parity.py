@@ -85,3 +85,34 @@ def check_layers(data: dict, out: np.ndarray, trace: np.ndarray, k: int, n: int,
                     assert np.array_equal(trace[l, b, s], S_in[b, s]), \
                         f"layer {l} b {b} set {s}: an unrefreshed set changed"
     return worst
+
+
+def check_layers_varlen(q: np.ndarray, K: np.ndarray, V: np.ndarray, role: np.ndarray,
+                        n_list, out: np.ndarray, trace: np.ndarray, k: int, dtype: str, layers,
+                        select_mode=O.SELECT_PER_QHEAD, S0: np.ndarray | None = None):
+    """The serving form: element b of the batch is checked on its own, as a
+    one-element step over its n[b] rows (the logical cache after the append),
+    with teacher forcing as in check_layers.  q [L][B][Hq][d], K/V
+    [L][B][Hkv][rows][d] host arrays (bf16 as uint16 bit patterns)."""
+    worst = 0.0
+    for b, nb in enumerate(n_list):
+        for l in layers:
+            st = O.Stack(np.ascontiguousarray(q[l:l + 1, b:b + 1]),
+                         np.ascontiguousarray(K[l:l + 1, b:b + 1, :, :nb]),
+                         np.ascontiguousarray(V[l:l + 1, b:b + 1, :, :nb]),
+                         np.ascontiguousarray(role[l:l + 1], dtype=np.uint8), select_mode)
+            if l == 0:
+                S_in = None if S0 is None else S0[b:b + 1]
+                all_ret = S0 is None
+            else:
+                S_in = trace[l - 1, b:b + 1]
+                all_ret = False
+            o, S_out, keys, fresh = O.layer(st, 0, k, S_in, all_retrieval=all_ret)
+            worst = max(worst, check_out(out[l, b:b + 1], o, dtype, f"b {b} layer {l} outputs"))
+            for s in range(S_out.shape[1]):
+                if fresh[s]:
+                    check_set(trace[l, b, s], keys[0, s], k, f"b {b} layer {l} set {s}")
+                else:
+                    assert np.array_equal(trace[l, b, s], S_in[0, s]), \
+                        f"b {b} layer {l} set {s}: an unrefreshed set changed"
+    return worst

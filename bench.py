@@ -48,6 +48,9 @@ def parse_args(argv=None):
     ap.add_argument("--select-mode", choices=["per_qhead", "kvgroup_mean"], default="per_qhead")
     ap.add_argument("--attn-kernel", choices=["mma", "tcgen05"], default="mma",
                     help="bf16 attention kernel: mma.sync (default) or tcgen05/TMEM")
+    ap.add_argument("--serving", action="store_true",
+                    help="the serving form instead: lyc_decode_step_batch on a batch of four "
+                         "cache lengths, paged cache (64-row pages), current token appended")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-layers", type=int, default=2,
@@ -462,10 +465,126 @@ def run_lyc(args):
     return 0
 
 
+SERVING_N = (131072, 98304, 65536, 32768)
+
+
+def serving_analytic_bytes(role, n_list, k, L, Hq, Hkv, d, select_mode):
+    """The step's byte floor for per-element lengths: per layer and element,
+    n[b] rows of K and V for every KV group with a retrieval head (all groups
+    at layer 0), min(k, n[b]) rows for every other group."""
+    G = Hq // Hkv
+    total = 0
+    for l in range(L):
+        ret = [True] * Hkv if l == 0 else [bool(role[l, g * G:(g + 1) * G].any()) for g in range(Hkv)]
+        for nb in n_list:
+            for g in range(Hkv):
+                total += (nb if ret[g] else min(k, nb)) * d * 2 * 2
+    return total
+
+
+def run_serving(args):
+    """The serving form on one GPU: Llama3-8B-shaped stack, a batch of four
+    cache lengths, a paged cache of 64-row pages (shuffled), the current
+    token's K/V appended by the step; steps/s and the byte-floor rate."""
+    import numpy as np
+    import torch
+
+    from hybrid_head_sparse_b200 import build as Bld
+    from hybrid_head_sparse_b200 import lyc, workloads as W
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    Bld.build()
+    lyc.load()
+    base = workload_spec(args)
+    L, Hq, Hkv, d, k = base.L, base.Hq, base.Hkv, base.d, base.k
+    n_list = list(SERVING_N)
+    B = len(n_list)
+    page_rows = 64
+    blocks = [(nb + page_rows - 1) // page_rows for nb in n_list]
+    npages = sum(blocks)
+    rng = np.random.default_rng(7)
+    perm = rng.permutation(npages)
+    max_blocks = max(blocks)
+    bt = np.zeros((B, max_blocks), dtype=np.int32)
+    j = 0
+    for b in range(B):
+        for blk in range(blocks[b]):
+            bt[b, blk] = perm[j]
+            j += 1
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(base.seed)
+    Kp = torch.empty((L, npages, page_rows, Hkv, d), device=dev, dtype=torch.bfloat16)
+    Vp = torch.empty_like(Kp)
+    for l in range(L):  # layer by layer: bounded float32 staging
+        Kp[l] = torch.randn((npages, page_rows, Hkv, d), generator=gen, device=dev).to(torch.bfloat16)
+        Vp[l] = torch.randn((npages, page_rows, Hkv, d), generator=gen, device=dev).to(torch.bfloat16)
+    q = torch.randn((L, B, Hq, d), generator=gen, device=dev).to(torch.bfloat16)
+    k_new = torch.randn((L, B, Hkv, d), generator=gen, device=dev).to(torch.bfloat16)
+    v_new = torch.randn((L, B, Hkv, d), generator=gen, device=dev).to(torch.bfloat16)
+    role = W.role_mask(base.with_(B=B))
+    bt_dev = torch.from_numpy(bt).to(dev)
+    ctx = lyc.Lyc(L, B, Hq, Hkv, d, max(n_list), k, select_mode=args.select_mode)
+    out = torch.empty((L, B, Hq, d), device=dev)
+    S = torch.empty((B, ctx.Hs, k), dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        ctx.decode_step_batch(q, Kp, Vp, n_list, role, k, out, S, stream=stream, k_new=k_new,
+                              v_new=v_new, block_table=bt_dev, page_rows=page_rows)
+
+    for _ in range(max(args.warmup, 1)):
+        step()
+    torch.cuda.synchronize()
+    rc = ctx.sync_status()
+    if rc != 0:
+        raise RuntimeError(f"device status after warm-up: {lyc.lyc_status_string(rc)}")
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    torch.cuda.synchronize()
+    with ClockSampler(0) as clk:
+        evs[0].record(stream)
+        for i in range(args.steps):
+            step()
+            evs[i + 1].record(stream)
+        torch.cuda.synchronize()
+    ms_total = evs[0].elapsed_time(evs[-1])
+    step_ms = percentiles([evs[i].elapsed_time(evs[i + 1]) for i in range(args.steps)])
+    rc = ctx.sync_status()
+    if rc != 0:
+        raise RuntimeError(f"device status after timing: {lyc.lyc_status_string(rc)}")
+    ms_step = ms_total / args.steps
+    analytic = serving_analytic_bytes(role, n_list, k, L, Hq, Hkv, d, args.select_mode)
+    peak, _ = measured_peaks()
+    gbs = analytic / (ms_step / 1e3) / 1e9
+    line = {
+        "metric": "serving decode steps/s (batch of 4 lengths, paged cache, current token appended)",
+        "value": args.steps / (ms_total / 1e3), "unit": "steps/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "step_ms_distribution": {kk: round(v, 4) for kk, v in step_ms.items()},
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) pages, q and appended rows; shuffled 64-row pages)",
+        "config": {"workload": "llama3-8b-serving-b4-paged64", "L": L, "B": B, "Hq": Hq,
+                   "Hkv": Hkv, "d": d, "n": n_list, "k": k, "page_rows": page_rows,
+                   "retrieval_heads_per_layer": args.retrieval_heads,
+                   "select_mode": args.select_mode, "append": True, "parallelism": "replicas x1",
+                   "l2": "inputs larger than L2 (KV pages %.1f GB)" % (
+                       2 * Kp.numel() * Kp.element_size() / 1e9)},
+        "hbm": {"analytic_bytes_per_step": analytic, "analytic_gbs": round(gbs, 1),
+                "frac_of_measured_peak": round(gbs / peak, 4),
+                "frac_of_8tbs": round(gbs / NOMINAL_HBM_GBS, 4)},
+        "clocks": clk.summary(),
+    }
+    ctx.close()
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
+    if args.serving:
+        return run_serving(args)
     return run_lyc(args)
 
 

@@ -395,9 +395,31 @@ def pin_strided_layout(ora):
     assert np.array_equal(c[0], b[0]) and np.array_equal(c[1], b[1]), "padded rows"
 
 
+def pin_batch_elements_independent(ora):
+    """Batch elements do not interact (sets are per element; Algorithm 1 runs
+    per sequence), which is what lets the serving form check each element of a
+    variable-length batch as a one-element step over its own rows: the
+    batched oracle equals its per-element runs, and an element's results do
+    not move when another element's cache changes."""
+    rng = np.random.default_rng(16)
+    role = np.array([[1, 1, 1, 1], [0, 1, 0, 0], [1, 0, 0, 1]], dtype=np.uint8)
+    st = rand_stack(rng, L=3, B=3, Hq=4, Hkv=2, d=8, n=33, role=role)
+    out, S, _ = ora.decode_step(st, k=5)
+    for b in range(3):
+        one = stack(st.q[:, b:b + 1].copy(), st.k[:, b:b + 1].copy(), st.v[:, b:b + 1].copy(), role)
+        o1, S1, _ = ora.decode_step(one, k=5)
+        assert np.array_equal(o1[:, 0], out[:, b]) and np.array_equal(S1[0], S[b]), f"element {b}"
+    k2 = st.k.copy()
+    k2[:, 1] = rng.standard_normal(k2[:, 1].shape).astype(np.float32)
+    out2, S2, _ = ora.decode_step(stack(st.q, k2, st.v, role), k=5)
+    assert np.array_equal(out2[:, 0], out[:, 0]) and np.array_equal(out2[:, 2], out[:, 2])
+    assert np.array_equal(S2[0], S[0]) and np.array_equal(S2[2], S[2])
+    assert not np.array_equal(out2[:, 1], out[:, 1]), "element 1 must see its own change"
+
+
 ALL_PINS = [
     pin_topk_distinct, pin_topk_ties, pin_topk_bruteforce, pin_closed_form_bf16,
     pin_dense_textbook, pin_mpmath_attention, pin_sparse_eq3, pin_k_ge_n, pin_uniform_keys,
     pin_planted_key, pin_chain, pin_layer0_forced, pin_permutation, pin_linearity,
-    pin_kvgroup, pin_strided_layout,
+    pin_kvgroup, pin_strided_layout, pin_batch_elements_independent,
 ]

@@ -17,7 +17,11 @@ Inference via Hybrid-Head Sparse Decoding" (paper-graph-ui summary):
 * section 3.4 (propagation-chain initialisation) and Appendix B (Algorithm 1):
   every head of layer 0 is a retrieval head;
 * section 3.4 "Hyperparameter summary": under GQA the queries of a KV group
-  are averaged before token selection (``select_mode=1``).
+  are averaged before token selection (``select_mode=1``);
+* section 4.4.1 (Figure 6, Tables 5-6), section 4.1 / Appendix F and the
+  kernel section: the selection rules other than a fixed k (ratio, the
+  reasoning budget as the ratio 1/2, block top-k, top-p, threshold; see
+  ``Selection`` and the readings at the top of oracle.c).
 """
 from __future__ import annotations
 
@@ -36,6 +40,11 @@ BF16 = 0
 FP32 = 1
 SELECT_PER_QHEAD = 0
 SELECT_KVGROUP_MEAN = 1
+RULE_TOPK = 0
+RULE_RATIO = 1
+RULE_BLOCK_TOPK = 2
+RULE_TOPP = 3
+RULE_THRESHOLD = 4
 
 
 class OracleShape(ctypes.Structure):
@@ -53,6 +62,35 @@ class OracleShape(ctypes.Structure):
         ("s_head", ctypes.c_int64),
         ("s_token", ctypes.c_int64),
     ]
+
+
+class OracleSelection(ctypes.Structure):
+    _fields_ = [
+        ("rule", ctypes.c_int),
+        ("block", ctypes.c_int),
+        ("ratio_num", ctypes.c_int64),
+        ("ratio_den", ctypes.c_int64),
+        ("p", ctypes.c_double),
+        ("tau", ctypes.c_double),
+    ]
+
+
+@dataclass
+class Selection:
+    """A selection rule (section 4.4.1, Figure 6, Tables 5-6; Appendix F):
+    RULE_TOPK (fixed k), RULE_RATIO (ceil(num/den * n) rows), RULE_BLOCK_TOPK
+    (whole blocks of `block` rows, scored by their summed probability),
+    RULE_TOPP (smallest prefix reaching mass p), RULE_THRESHOLD (rows with
+    probability >= tau).  Every rule keeps at most k rows."""
+    rule: int = RULE_TOPK
+    block: int = 64
+    ratio: tuple = (1, 2)
+    p: float = 0.9
+    tau: float = 1e-3
+
+    def c(self) -> OracleSelection:
+        return OracleSelection(self.rule, self.block, int(self.ratio[0]), int(self.ratio[1]),
+                               float(self.p), float(self.tau))
 
 
 def build(force: bool = False) -> str:
@@ -82,11 +120,24 @@ class Oracle:
         L.ora_decode_step.argtypes = [ctypes.POINTER(OracleShape), p, p, p, p,
                                       ctypes.c_int, ctypes.c_int, p, p, p]
         L.ora_decode_step.restype = ctypes.c_int
+        L.ora_select.argtypes = [p, ctypes.c_int64, ctypes.c_int, ctypes.POINTER(OracleSelection), p]
+        L.ora_select.restype = ctypes.c_int
+        L.ora_layer_sel.argtypes = [ctypes.POINTER(OracleShape), ctypes.POINTER(OracleSelection),
+                                    ctypes.c_int, p, p, p, p, ctypes.c_int, ctypes.c_int, p, p,
+                                    p, p, p]
+        L.ora_layer_sel.restype = ctypes.c_int
+        L.ora_decode_step_sel.argtypes = [ctypes.POINTER(OracleShape),
+                                          ctypes.POINTER(OracleSelection), p, p, p, p,
+                                          ctypes.c_int, ctypes.c_int, p, p, p]
+        L.ora_decode_step_sel.restype = ctypes.c_int
         self.lib = L
         self.path = path
 
     def topk(self, x, k):
         return topk(x, k, self)
+
+    def select(self, x, k, sel=None):
+        return select(x, k, sel, self)
 
     def layer(self, *a, **kw):
         return layer(*a, ora=self, **kw)
@@ -175,8 +226,26 @@ def topk(x: np.ndarray, k: int, ora: Oracle | None = None) -> np.ndarray:
     return S
 
 
+def select(x: np.ndarray, k: int, sel: Selection | None = None,
+           ora: Oracle | None = None) -> np.ndarray:
+    """The set one selection rule picks from the keys x: ascending, -1 padded
+    to k (sel None: top-k)."""
+    ora = ora or default()
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    S = np.empty(k, dtype=np.int32)
+    cs = (sel or Selection()).c()
+    rc = ora.lib.ora_select(_ptr(x), x.size, k, ctypes.byref(cs), _ptr(S))
+    if rc != 0:
+        raise ValueError(f"ora_select failed ({rc})")
+    return S
+
+
+def _sel_ref(sel: Selection | None):
+    return None if sel is None else ctypes.byref(sel.c())
+
+
 def layer(st: Stack, l: int, k: int, S_in: np.ndarray | None, all_retrieval: bool,
-          n: int | None = None, ora: Oracle | None = None):
+          n: int | None = None, ora: Oracle | None = None, sel: Selection | None = None):
     """One layer.  Returns (out [B][Hq][d] f64, S_out [B][Hs][k] i32,
     keys [B][Hs][n] f64 (valid for refreshed slots), refreshed [Hs] u8)."""
     sh = st.shape(n)
@@ -191,16 +260,17 @@ def layer(st: Stack, l: int, k: int, S_in: np.ndarray | None, all_retrieval: boo
         assert S_in.shape == (B, Hs, k), S_in.shape
     role = np.ascontiguousarray(st.role, dtype=np.uint8)
     ora = ora or default()
-    rc = ora.lib.ora_layer(ctypes.byref(sh), l, _ptr(st.q), _ptr(st.k), _ptr(st.v),
-                         _ptr(role[l]), int(all_retrieval), k, _ptr(S_in), _ptr(S_out),
-                         _ptr(out), _ptr(keys), _ptr(fresh))
+    cs = (sel or Selection()).c()
+    rc = ora.lib.ora_layer_sel(ctypes.byref(sh), ctypes.byref(cs), l, _ptr(st.q), _ptr(st.k),
+                             _ptr(st.v), _ptr(role[l]), int(all_retrieval), k, _ptr(S_in),
+                             _ptr(S_out), _ptr(out), _ptr(keys), _ptr(fresh))
     if rc != 0:
         raise ValueError(f"ora_layer failed ({rc})")
     return out, S_out, keys, fresh
 
 
 def decode_step(st: Stack, k: int, S_in: np.ndarray | None = None, n: int | None = None,
-                trace: bool = False, ora: Oracle | None = None):
+                trace: bool = False, ora: Oracle | None = None, sel: Selection | None = None):
     """The whole L-layer step.  S_in given: S^(0) is S_in and role row 0 is
     obeyed; otherwise layer 0 is all retrieval.  Returns (out [L][B][Hq][d],
     S [B][Hs][k], trace [L][B][Hs][k] or None)."""
@@ -214,9 +284,10 @@ def decode_step(st: Stack, k: int, S_in: np.ndarray | None = None, n: int | None
     tr = np.full((L, B, Hs, k), -1, dtype=np.int32) if trace else None
     role = np.ascontiguousarray(st.role, dtype=np.uint8)
     ora = ora or default()
-    rc = ora.lib.ora_decode_step(ctypes.byref(sh), _ptr(st.q), _ptr(st.k), _ptr(st.v),
-                               _ptr(role), k, int(S_in is not None), _ptr(S), _ptr(out),
-                               _ptr(tr))
+    cs = (sel or Selection()).c()
+    rc = ora.lib.ora_decode_step_sel(ctypes.byref(sh), ctypes.byref(cs), _ptr(st.q), _ptr(st.k),
+                                   _ptr(st.v), _ptr(role), k, int(S_in is not None), _ptr(S),
+                                   _ptr(out), _ptr(tr))
     if rc != 0:
         raise ValueError(f"ora_decode_step failed ({rc})")
     return out, S, tr

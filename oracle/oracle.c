@@ -27,6 +27,27 @@
  *   - query head h belongs to KV group h / (Hq / Hkv);
  *   - the current token is already in the cache (no causal mask).
  *
+ * Selection rules other than a fixed k (section 4.4.1, Figure 6 and Tables
+ * 5-6 name them; section 4.1 / Appendix F give the reasoning budget; the
+ * kernel section gives the block size of 64), with the readings taken where
+ * the pages give no formula:
+ *   - the probabilities are A = softmax(x) of the selection key x (the
+ *     logits, or the pooled query's logits in KV-group mode);
+ *   - ratio: the set holds ceil(theta * n) rows (at least 1, at most k), the
+ *     largest keys; theta = num / den exactly, so the budget is an integer
+ *     computation.  The reasoning budget (50 % of the length, growing as the
+ *     length grows) is the ratio 1/2 evaluated at each step's n;
+ *   - top-p: the rows in key order (larger first, ties to the lower index)
+ *     up to and including the first at which the running sum of A reaches p;
+ *     all n if it never does; at most k;
+ *   - threshold: the rows with A >= tau, at least the largest one (a set is
+ *     never empty), at most k (then the k largest);
+ *   - block top-k: rows grouped in blocks of `block` consecutive rows (the
+ *     last one possibly shorter); a block's score is the sum of its rows' A;
+ *     the floor(k / block) best blocks (ties to the lower block) are taken
+ *     whole, so the set holds at most k rows;
+ *   - every set is written in ascending row order, padded with -1 to k.
+ *
  * Everything is fp64.  bf16 inputs are widened exactly (bits << 16), fp32
  * inputs are widened exactly.  Loops are plain; OpenMP only runs independent
  * heads side by side and changes no arithmetic.
@@ -40,6 +61,19 @@
 #define ORA_FP32 1
 #define ORA_SELECT_PER_QHEAD 0
 #define ORA_SELECT_KVGROUP_MEAN 1
+#define ORA_RULE_TOPK 0
+#define ORA_RULE_RATIO 1
+#define ORA_RULE_BLOCK_TOPK 2
+#define ORA_RULE_TOPP 3
+#define ORA_RULE_THRESHOLD 4
+
+typedef struct {
+  int rule;                      /* ORA_RULE_* */
+  int block;                     /* block top-k: rows per block */
+  int64_t ratio_num, ratio_den;  /* ratio: theta = num / den */
+  double p;                      /* top-p: the probability mass to reach */
+  double tau;                    /* threshold: the smallest probability kept */
+} ora_selection;
 
 typedef struct {
   int L, B, Hq, Hkv, d;
@@ -109,6 +143,113 @@ int ora_topk(const double* x, int64_t n, int k, int32_t* S) {
   return 0;
 }
 
+/* The m rows with the largest x (m <= n), ascending, padded with -1 to k. */
+static int topk_into(const double* x, int64_t n, int64_t m, int k, int32_t* S) {
+  int32_t* tmp = (int32_t*)malloc((size_t)m * sizeof(int32_t));
+  if (!tmp) return -3;
+  int rc = ora_topk(x, n, (int)m, tmp);
+  if (rc == 0) {
+    for (int64_t j = 0; j < m; ++j) S[j] = tmp[j];
+    for (int64_t j = m; j < k; ++j) S[j] = -1;
+  }
+  free(tmp);
+  return rc;
+}
+
+/* A = softmax(x): A_i = exp(x_i - max x) / sum_j exp(x_j - max x), in fp64. */
+static double* softmax_of(const double* x, int64_t n) {
+  double* a = (double*)malloc((size_t)n * sizeof(double));
+  if (!a) return NULL;
+  double m = -INFINITY, z = 0.0;
+  for (int64_t i = 0; i < n; ++i)
+    if (x[i] > m) m = x[i];
+  for (int64_t i = 0; i < n; ++i) {
+    a[i] = exp(x[i] - m);
+    z += a[i];
+  }
+  for (int64_t i = 0; i < n; ++i) a[i] /= z;
+  return a;
+}
+
+/* The set of one selection (Eq. 2 generalised by the rules above) from the
+   selection keys x[0..n-1]; S has k entries.  sel == NULL: top-k. */
+int ora_select(const double* x, int64_t n, int k, const ora_selection* sel, int32_t* S) {
+  if (n <= 0 || k <= 0) return -1;
+  const int rule = sel ? sel->rule : ORA_RULE_TOPK;
+  if (rule == ORA_RULE_TOPK) return ora_topk(x, n, k, S);
+  const int64_t cap = (int64_t)k < n ? (int64_t)k : n;
+  if (rule == ORA_RULE_RATIO) {
+    if (sel->ratio_num < 0 || sel->ratio_den <= 0) return -1;
+    int64_t m = (sel->ratio_num * n + sel->ratio_den - 1) / sel->ratio_den;  /* ceil */
+    if (m < 1) m = 1;
+    if (m > cap) m = cap;
+    return topk_into(x, n, m, k, S);
+  }
+  if (rule == ORA_RULE_TOPP || rule == ORA_RULE_THRESHOLD) {
+    double* a = softmax_of(x, n);
+    if (!a) return -3;
+    int64_t m = 0;
+    if (rule == ORA_RULE_THRESHOLD) {
+      for (int64_t i = 0; i < n; ++i) m += a[i] >= sel->tau;
+      if (m < 1) m = 1;
+    } else {
+      keyed* all = (keyed*)malloc((size_t)n * sizeof(keyed));
+      if (!all) {
+        free(a);
+        return -3;
+      }
+      for (int64_t i = 0; i < n; ++i) {
+        all[i].x = x[i];
+        all[i].i = i;
+      }
+      qsort(all, (size_t)n, sizeof(keyed), by_value_desc_index_asc);
+      double cum = 0.0;
+      m = n;
+      for (int64_t j = 0; j < n; ++j) {
+        cum += a[all[j].i];
+        if (cum >= sel->p) {
+          m = j + 1;
+          break;
+        }
+      }
+      free(all);
+    }
+    free(a);
+    if (m > cap) m = cap;
+    return topk_into(x, n, m, k, S);
+  }
+  if (rule == ORA_RULE_BLOCK_TOPK) {
+    const int bs = sel->block;
+    if (bs <= 0 || k < bs) return -1;
+    const int64_t nb = (n + bs - 1) / bs;
+    int64_t kb = k / bs;
+    if (kb > nb) kb = nb;
+    double* a = softmax_of(x, n);
+    double* score = (double*)calloc((size_t)nb, sizeof(double));
+    int32_t* blocks = (int32_t*)malloc((size_t)kb * sizeof(int32_t));
+    if (!a || !score || !blocks) {
+      free(a);
+      free(score);
+      free(blocks);
+      return -3;
+    }
+    for (int64_t i = 0; i < n; ++i) score[i / bs] += a[i];
+    int rc = ora_topk(score, nb, (int)kb, blocks);
+    if (rc == 0) {
+      int64_t pos = 0;
+      for (int64_t j = 0; j < kb; ++j)
+        for (int64_t i = (int64_t)blocks[j] * bs; i < ((int64_t)blocks[j] + 1) * bs && i < n; ++i)
+          S[pos++] = (int32_t)i;
+      for (; pos < k; ++pos) S[pos] = -1;
+    }
+    free(a);
+    free(score);
+    free(blocks);
+    return rc;
+  }
+  return -1;
+}
+
 /* ---------------------------------------------------------------- attention */
 
 /* Scaled dot-product attention of one query over a list of cache rows
@@ -160,10 +301,10 @@ static void attend_rows(const ora_shape* sh, const double* q, const void* K,
  *   refreshed: [Hs] or NULL; 1 where the slot was re-selected at this layer
  * Returns 0, or a negative code on a bad argument or a bad inherited index.
  */
-int ora_layer(const ora_shape* sh, int l, const void* q_all, const void* K,
-              const void* V, const uint8_t* role_row, int all_retrieval, int k,
-              const int32_t* S_in, int32_t* S_out, double* out_l, double* keys,
-              uint8_t* refreshed) {
+int ora_layer_sel(const ora_shape* sh, const ora_selection* sel, int l, const void* q_all,
+                  const void* K, const void* V, const uint8_t* role_row, int all_retrieval,
+                  int k, const int32_t* S_in, int32_t* S_out, double* out_l, double* keys,
+                  uint8_t* refreshed) {
   const int B = sh->B, Hq = sh->Hq, Hkv = sh->Hkv, d = sh->d;
   const int64_t n = sh->n;
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || d <= 0 || n <= 0 || k <= 0) return -1;
@@ -171,6 +312,9 @@ int ora_layer(const ora_shape* sh, int l, const void* q_all, const void* K,
   const int G = Hq / Hkv;
   const int Hs = slots_per_batch(sh);
   const int kv_mode = sh->select_mode == ORA_SELECT_KVGROUP_MEAN;
+  if (sel && sel->rule == ORA_RULE_BLOCK_TOPK && (sel->block <= 0 || k < sel->block)) return -1;
+  if (sel && sel->rule == ORA_RULE_RATIO && (sel->ratio_num < 0 || sel->ratio_den <= 0)) return -1;
+  if (sel && (sel->rule < ORA_RULE_TOPK || sel->rule > ORA_RULE_THRESHOLD)) return -1;
 
   /* which heads are retrieval, which slots are refreshed */
   int* is_ret = (int*)calloc((size_t)Hq, sizeof(int));
@@ -274,7 +418,7 @@ int ora_layer(const ora_shape* sh, int l, const void* q_all, const void* K,
         free(qbar);
       }
       /* per-head mode: x already holds the retrieval head's own logits */
-      ora_topk(x, n, k, Sout);
+      ora_select(x, n, k, sel, Sout);
       if (keys) memcpy(keys + ((int64_t)b * Hs + s) * n, x, (size_t)n * sizeof(double));
     }
   }
@@ -284,6 +428,14 @@ int ora_layer(const ora_shape* sh, int l, const void* q_all, const void* K,
   free(is_ret);
   free(fresh);
   return 0;
+}
+
+int ora_layer(const ora_shape* sh, int l, const void* q_all, const void* K,
+              const void* V, const uint8_t* role_row, int all_retrieval, int k,
+              const int32_t* S_in, int32_t* S_out, double* out_l, double* keys,
+              uint8_t* refreshed) {
+  return ora_layer_sel(sh, NULL, l, q_all, K, V, role_row, all_retrieval, k, S_in, S_out,
+                       out_l, keys, refreshed);
 }
 
 /* ---------------------------------------------------------------- one step */
@@ -296,9 +448,9 @@ int ora_layer(const ora_shape* sh, int l, const void* q_all, const void* K,
  *   out   : [L][B][Hq][d] fp64.
  *   trace : [L][B][Hs][k] or NULL; trace[l] = the sets after layer l.
  */
-int ora_decode_step(const ora_shape* sh, const void* q, const void* K,
-                    const void* V, const uint8_t* role, int k, int s_in,
-                    int32_t* S, double* out, int32_t* trace) {
+int ora_decode_step_sel(const ora_shape* sh, const ora_selection* sel, const void* q,
+                        const void* K, const void* V, const uint8_t* role, int k, int s_in,
+                        int32_t* S, double* out, int32_t* trace) {
   const int64_t per = (int64_t)sh->B * slots_per_batch(sh) * k;
   int32_t* cur = (int32_t*)malloc((size_t)per * sizeof(int32_t));
   int32_t* nxt = (int32_t*)malloc((size_t)per * sizeof(int32_t));
@@ -310,9 +462,9 @@ int ora_decode_step(const ora_shape* sh, const void* q, const void* K,
   int rc = 0;
   for (int l = 0; l < sh->L && rc == 0; ++l) {
     const int all_ret = (l == 0) && !s_in;
-    rc = ora_layer(sh, l, q, K, V, role + (int64_t)l * sh->Hq, all_ret, k,
-                   (l == 0 && !s_in) ? NULL : cur, nxt,
-                   out + (int64_t)l * sh->B * sh->Hq * sh->d, NULL, NULL);
+    rc = ora_layer_sel(sh, sel, l, q, K, V, role + (int64_t)l * sh->Hq, all_ret, k,
+                       (l == 0 && !s_in) ? NULL : cur, nxt,
+                       out + (int64_t)l * sh->B * sh->Hq * sh->d, NULL, NULL);
     if (trace) memcpy(trace + (int64_t)l * per, nxt, (size_t)per * sizeof(int32_t));
     int32_t* t = cur;
     cur = nxt;
@@ -322,4 +474,10 @@ int ora_decode_step(const ora_shape* sh, const void* q, const void* K,
   free(cur);
   free(nxt);
   return rc;
+}
+
+int ora_decode_step(const ora_shape* sh, const void* q, const void* K,
+                    const void* V, const uint8_t* role, int k, int s_in,
+                    int32_t* S, double* out, int32_t* trace) {
+  return ora_decode_step_sel(sh, NULL, q, K, V, role, k, s_in, S, out, trace);
 }

@@ -417,9 +417,167 @@ def pin_batch_elements_independent(ora):
     assert not np.array_equal(out2[:, 1], out[:, 1]), "element 1 must see its own change"
 
 
+# ----------------------------------------------------------------- selection rules
+# Section 4.4.1 (Figure 6, Tables 5-6) names the rules; the readings (set sizes,
+# order, the cap k, blocks scored by summed probability) are the oracle's.
+
+
+def softmax64(x: np.ndarray) -> np.ndarray:
+    e = np.exp(x - x.max())
+    return e / e.sum()
+
+
+def padded(rows, k):
+    rows = list(rows)
+    return np.array(rows + [-1] * (k - len(rows)), dtype=np.int32)
+
+
+def pin_select_topk_rule_is_topk(ora):
+    rng = np.random.default_rng(40)
+    x = rng.standard_normal(77)
+    for k in (1, 9, 77, 90):
+        assert np.array_equal(ora.select(x, k, O.Selection(O.RULE_TOPK)), library_topk(x, k))
+
+
+def pin_select_ratio(ora):
+    """ceil(num/den * n) rows (integer arithmetic), at least 1, at most k; the
+    reasoning budget (ratio 1/2) grows by one row every two steps."""
+    rng = np.random.default_rng(41)
+    for n in (1, 7, 10, 64, 301):
+        x = rng.standard_normal(n)
+        for num, den in ((1, 2), (7, 10), (1, 3), (0, 1), (3, 2), (1, 1000)):
+            m = max(1, -((-num * n) // den))
+            for k in (1, 5, 200, 400):
+                exp = library_topk(x, min(m, k))
+                exp = np.concatenate([exp, np.full(k - exp.size, -1, dtype=np.int32)])
+                got = ora.select(x, k, O.Selection(O.RULE_RATIO, ratio=(num, den)))
+                assert np.array_equal(got, exp), f"ratio {num}/{den} n={n} k={k}"
+    x = rng.standard_normal(40)
+    sizes = [int((ora.select(x[:n], 64, O.Selection(O.RULE_RATIO, ratio=(1, 2))) >= 0).sum())
+             for n in range(1, 41)]
+    assert sizes == [(n + 1) // 2 for n in range(1, 41)], sizes
+
+
+def pin_select_topp(ora):
+    """Known probabilities (1/2, 1/4, 1/8, 1/8), uniform keys, the cap, and
+    brute force: no smaller subset reaches the mass p, and the greedy set is
+    the top-m by key."""
+    w = np.array([0.125, 0.5, 0.125, 0.25])
+    x = np.log(w)
+    for pv, exp in ((0.3, [1]), (0.6, [1, 3]), (0.74, [1, 3]), (0.76, [0, 1, 3]),
+                    (0.87, [0, 1, 3]), (0.88, [0, 1, 2, 3]), (1.0, [0, 1, 2, 3])):
+        got = ora.select(x, 6, O.Selection(O.RULE_TOPP, p=pv))
+        assert np.array_equal(got, padded(exp, 6)), f"top-p {pv}: {got}"
+    assert np.array_equal(ora.select(x, 2, O.Selection(O.RULE_TOPP, p=0.99)), padded([1, 3], 2))
+    # uniform keys: A = 1/n, ties by index, m = ceil(p n)
+    for n in (8, 13):
+        for j in range(n):
+            pv = (j + 0.5) / n
+            got = ora.select(np.zeros(n), n, O.Selection(O.RULE_TOPP, p=pv))
+            assert np.array_equal(got, padded(range(j + 1), n)), f"uniform top-p n={n} j={j}"
+    # mass reached exactly (n = 8: A = 1/8 and every running sum are exact):
+    # the row that reaches p is the last one taken
+    for j in range(8):
+        got = ora.select(np.zeros(8), 8, O.Selection(O.RULE_TOPP, p=(j + 1) / 8))
+        assert np.array_equal(got, padded(range(j + 1), 8)), f"exact mass {j + 1}/8"
+    rng = np.random.default_rng(42)
+    for trial in range(80):
+        n = int(rng.integers(1, 9))
+        x = rng.standard_normal(n) * 2.0
+        a = softmax64(x)
+        pv = float(rng.uniform(0.05, 0.99))
+        got = ora.select(x, n, O.Selection(O.RULE_TOPP, p=pv))
+        m = int((got >= 0).sum())
+        best = min(len(T) for r in range(1, n + 1) for T in itertools.combinations(range(n), r)
+                   if a[list(T)].sum() >= pv - 1e-12)
+        assert m == best, f"top-p brute force: {m} vs {best}"
+        assert np.array_equal(got, padded(library_topk(x, m), n)), "top-p set is not the top-m"
+
+
+def pin_select_threshold(ora):
+    """Rows with A >= tau: exact probabilities (uniform over 8 rows gives
+    A = 1/8 exactly), at least one row, at most k; numpy count elsewhere."""
+    assert np.array_equal(ora.select(np.zeros(8), 8, O.Selection(O.RULE_THRESHOLD, tau=0.125)),
+                          np.arange(8, dtype=np.int32))
+    assert np.array_equal(ora.select(np.zeros(8), 8, O.Selection(O.RULE_THRESHOLD, tau=0.13)),
+                          padded([0], 8))
+    x = np.log(np.array([0.125, 0.5, 0.125, 0.25]))
+    assert np.array_equal(ora.select(x, 4, O.Selection(O.RULE_THRESHOLD, tau=0.2)), padded([1, 3], 4))
+    assert np.array_equal(ora.select(x, 4, O.Selection(O.RULE_THRESHOLD, tau=0.9)), padded([1], 4))
+    rng = np.random.default_rng(43)
+    for trial in range(40):
+        n = int(rng.integers(1, 300))
+        x = rng.standard_normal(n) * 3.0
+        a = softmax64(x)
+        tau = float(10 ** rng.uniform(-4, -0.5))
+        k = int(rng.integers(1, 400))
+        m = min(max(1, int((a >= tau).sum())), k, n)
+        got = ora.select(x, k, O.Selection(O.RULE_THRESHOLD, tau=tau))
+        assert np.array_equal(got, np.concatenate([library_topk(x, m),
+                                                   np.full(k - m, -1, dtype=np.int32)]))
+
+
+def pin_select_block(ora):
+    """Block 1 is top-k; blocks scored by summed probability (numpy), the
+    floor(k/block) best taken whole (ties to the lower block), the short last
+    block included; planted keys pick their blocks."""
+    rng = np.random.default_rng(44)
+    x = rng.standard_normal(50)
+    for k in (1, 7, 50, 60):
+        assert np.array_equal(ora.select(x, k, O.Selection(O.RULE_BLOCK_TOPK, block=1)),
+                              library_topk(x, k))
+    for trial in range(40):
+        n = int(rng.integers(1, 400))
+        bs = int(rng.choice([2, 4, 16, 64]))
+        k = int(rng.integers(bs, 6 * bs + 1))
+        x = rng.standard_normal(n) * 2.0
+        starts = np.arange(0, n, bs)
+        score = np.add.reduceat(softmax64(x), starts)
+        kb = min(k // bs, starts.size)
+        blocks = np.sort(np.argsort(-score, kind="stable")[:kb])
+        rows = [i for b in blocks for i in range(b * bs, min(n, (b + 1) * bs))]
+        got = ora.select(x, k, O.Selection(O.RULE_BLOCK_TOPK, block=bs))
+        assert np.array_equal(got, padded(rows, k)), f"block n={n} bs={bs} k={k}"
+    x = np.zeros(10)
+    x[9] = 8.0
+    assert np.array_equal(ora.select(x, 4, O.Selection(O.RULE_BLOCK_TOPK, block=4)), padded([8, 9], 4))
+    x = np.zeros(12)   # equal blocks: the lowest ones
+    assert np.array_equal(ora.select(x, 8, O.Selection(O.RULE_BLOCK_TOPK, block=4)),
+                          np.arange(8, dtype=np.int32))
+    with np.testing.assert_raises(ValueError):
+        ora.select(x, 3, O.Selection(O.RULE_BLOCK_TOPK, block=4))   # k below one block
+
+
+def pin_select_in_step(ora):
+    """Through a whole step: every refreshed set is the rule applied to the
+    layer's keys (the head's logits), and a sparse head attends over exactly
+    the rows of its variable-size set (textbook attention over them)."""
+    rng = np.random.default_rng(45)
+    role = np.array([[1, 1], [0, 1], [0, 0]], dtype=np.uint8)
+    st = rand_stack(rng, L=3, B=1, Hq=2, Hkv=1, d=8, n=40, role=role)
+    q, K, V = widen(st.q), widen(st.k), widen(st.v)
+    for sel in (O.Selection(O.RULE_TOPP, p=0.5), O.Selection(O.RULE_THRESHOLD, tau=0.03),
+                O.Selection(O.RULE_RATIO, ratio=(1, 4)), O.Selection(O.RULE_BLOCK_TOPK, block=4)):
+        out, S, tr = ora.decode_step(st, k=16, trace=True, sel=sel)
+        for l in range(3):
+            for h in range(2):
+                if l == 0 or role[l, h]:
+                    _, logits = textbook_attention(q[l, 0, h], K[l, 0, 0], V[l, 0, 0])
+                    exp = ora.select(logits, 16, sel)
+                    assert np.array_equal(tr[l, 0, h], exp), f"rule {sel.rule} l={l} h={h}"
+                else:
+                    rows = tr[l - 1, 0, h]
+                    rows = rows[rows >= 0]
+                    o, _ = textbook_attention(q[l, 0, h], K[l, 0, 0][rows], V[l, 0, 0][rows])
+                    close(out[l, 0, h], o, 1e-12, f"sparse head over a rule-{sel.rule} set")
+                    assert np.array_equal(tr[l, 0, h], tr[l - 1, 0, h])
+
+
 ALL_PINS = [
     pin_topk_distinct, pin_topk_ties, pin_topk_bruteforce, pin_closed_form_bf16,
     pin_dense_textbook, pin_mpmath_attention, pin_sparse_eq3, pin_k_ge_n, pin_uniform_keys,
     pin_planted_key, pin_chain, pin_layer0_forced, pin_permutation, pin_linearity,
     pin_kvgroup, pin_strided_layout, pin_batch_elements_independent,
+    pin_select_topk_rule_is_topk, pin_select_ratio, pin_select_topp, pin_select_threshold,
+    pin_select_block, pin_select_in_step,
 ]

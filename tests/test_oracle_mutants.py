@@ -34,6 +34,20 @@ MUTANTS = [
     ("value row from the wrong token",
      "for (int j = 0; j < d; ++j) o[j] += p * widen(V, sh->dtype, off + j);",
      "for (int j = 0; j < d; ++j) o[j] += p * widen(V, sh->dtype, kv_base + r * sh->s_token + j);"),
+    ("ratio rounded down", "int64_t m = (sel->ratio_num * n + sel->ratio_den - 1) / sel->ratio_den;",
+     "int64_t m = (sel->ratio_num * n) / sel->ratio_den;"),
+    ("top-p takes one row too many", "          m = j + 1;\n          break;",
+     "          m = j + 2 < n ? j + 2 : n;\n          break;"),
+    ("top-p compares strictly", "if (cum >= sel->p) {", "if (cum > sel->p) {"),
+    ("threshold compares strictly", "for (int64_t i = 0; i < n; ++i) m += a[i] >= sel->tau;",
+     "for (int64_t i = 0; i < n; ++i) m += a[i] > sel->tau;"),
+    ("threshold may be empty", "      if (m < 1) m = 1;\n    } else {", "    } else {"),
+    ("softmax of the rules unnormalised", "for (int64_t i = 0; i < n; ++i) a[i] /= z;", ""),
+    ("block score is the block's last row", "for (int64_t i = 0; i < n; ++i) score[i / bs] += a[i];",
+     "for (int64_t i = 0; i < n; ++i) score[i / bs] = a[i];"),
+    ("short last block padded to full", "i < ((int64_t)blocks[j] + 1) * bs && i < n; ++i)",
+     "i < ((int64_t)blocks[j] + 1) * bs; ++i)"),
+    ("rule ignored in the step", "      ora_select(x, n, k, sel, Sout);", "      ora_topk(x, n, k, Sout);"),
     ("smallest instead of largest", "if (a->x > b->x) return -1;\n  if (a->x < b->x) return 1;",
      "if (a->x < b->x) return -1;\n  if (a->x > b->x) return 1;"),
 ]

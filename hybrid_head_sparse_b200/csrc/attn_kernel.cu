@@ -203,7 +203,9 @@ __device__ __forceinline__ void attn_producer(const AttnParams& p, unsigned char
         }
         const bool va = lane < nrows && ia >= 0 && ia < sg.nvalid;
         const bool vb2 = lane + 32 < nrows && ib >= 0 && ib < sg.nvalid;
-        if ((lane < nrows && !va) || (lane + 32 < nrows && !vb2)) atomicOr(p.status, kStatusBadIndex);
+        if ((lane < nrows && index_bad(ia, sg.nvalid, sg.pad_ok)) ||
+            (lane + 32 < nrows && index_bad(ib, sg.nvalid, sg.pad_ok)))
+          atomicOr(p.status, kStatusBadIndex);
         const uint32_t ma = __ballot_sync(0xffffffffu, va);
         const uint32_t mb = __ballot_sync(0xffffffffu, vb2);
         if (lane == 0) {

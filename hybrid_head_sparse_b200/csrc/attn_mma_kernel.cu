@@ -331,6 +331,7 @@ __device__ __forceinline__ void mma_producers(const AttnMmaParams& P, unsigned c
     // the segment's constants in registers (the copies below are asm with a
     // memory clobber: fields read through `sg` would be reloaded after each)
     const int nvalid = sg.nvalid;
+    const int32_t pad_ok = sg.pad_ok;
     const int32_t* bt = sg.bt;
     const int page_rows = sg.page_rows;
     const int64_t s_page = sg.s_page;
@@ -381,7 +382,7 @@ __device__ __forceinline__ void mma_producers(const AttnMmaParams& P, unsigned c
         for (int e = 0; e < 4; ++e) {
           const bool in_tile = 4 * j + e < nrows;
           const bool ok = xs[e] >= 0 && xs[e] < nvalid;
-          bad |= in_tile && !ok;
+          bad |= in_tile && index_bad(xs[e], nvalid, pad_ok);
           ys[e] = (in_tile && ok) ? row_base + xs[e] : p.gather_rows;
         }
         if (bad) atomicOr(p.status, kStatusBadIndex);
@@ -400,7 +401,8 @@ __device__ __forceinline__ void mma_producers(const AttnMmaParams& P, unsigned c
         if (pw == 0) {  // bounds of the inherited indices (reported, never followed)
           const int32_t ia = (lane < nrows) ? ring[lane] : 0;
           const int32_t ib = (lane + 32 < nrows) ? ring[lane + 32] : 0;
-          if (ia < 0 || ia >= nvalid || ib < 0 || ib >= nvalid) atomicOr(p.status, kStatusBadIndex);
+          if (index_bad(ia, nvalid, pad_ok) || index_bad(ib, nvalid, pad_ok))
+            atomicOr(p.status, kStatusBadIndex);
         }
         const uint32_t kbase = smem_u32(kdst), vbase = smem_u32(vdst);
         // lane: chunk (lane % CH) of rows pw*ROWS_W + (lane / CH) + (32/CH)*i

@@ -221,7 +221,7 @@ __device__ __forceinline__ void tc_producers(const AttnMmaParams& P, unsigned ch
           for (int i = 0; i < kTcRows / 32; ++i) {
             const int r = lane + 32 * i;
             const int32_t ix = (r < nrows) ? ring[r] : 0;
-            bad |= ix < 0 || ix >= sg.nvalid;
+            bad |= index_bad(ix, sg.nvalid, sg.pad_ok);
           }
           if (bad) atomicOr(p.status, kStatusBadIndex);
         }

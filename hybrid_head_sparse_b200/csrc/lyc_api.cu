@@ -46,6 +46,7 @@ int topk_max_clusters(int cl, size_t smem);
 cudaError_t copy_sets_launch(const CopySetsParams* p, cudaStream_t stream);
 cudaError_t append_rows_launch(const AppendParams* p, cudaStream_t stream);
 cudaError_t validate_sets_launch(const ValidateSetsParams* p, cudaStream_t stream);
+cudaError_t block_scores_launch(const BlockScoreParams* p, int sms, cudaStream_t stream);
 }  // namespace lyc
 
 using namespace lyc;
@@ -71,6 +72,9 @@ struct LayerPlan {
   int pool_nsegs = 0, pool_ups = 0;
   int64_t pool_tiles = 0, tiles = 0;  // tiles in the pool, in the whole layer
   int topk_cl = 16;          // cluster size of the selection launch
+  int topk_n = 0;            // keys of the longest selection task
+  size_t off_btasks = 0;     // block selection: the block-score tasks (one per selection task)
+  int bmax = 0;              // block selection: blocks of the longest task
 };
 
 struct Plan {
@@ -83,6 +87,9 @@ struct Plan {
   size_t off_empty_cta = 0;   // its CTA offsets (all zero: no pieces)
   int k = 0, keff = 0, n = 0;
   std::vector<int64_t> nb;        // rows of each batch element
+  std::vector<int> set_rows;      // capacity of each batch element's sets (rows)
+  bool variable = false;          // sets may be shorter than their capacity (-1 padded)
+  lyc_selection sel{};            // the selection rule the plan was built for
   bool append = false;            // the step writes the current token's K and V first
   bool paged = false;             // the cache is paged
   AppendParams ap_append{};       // (its n array lives in the plan buffer)
@@ -143,6 +150,11 @@ struct lyc_ctx {
   bool timing = false;
   unsigned long long* timeline = nullptr;  // caller's buffer, or NULL
   int timeline_cap = 0;
+  // the selection rule of the steps (lyc_set_selection); block selection's
+  // score rows, [L][B][Hs][bstride]
+  lyc_selection sel{};
+  float* bkeys = nullptr;
+  int64_t bstride = 0;
   // plans, most recent first
   std::list<std::pair<std::string, std::unique_ptr<Plan>>> plans;
   // timing pool
@@ -376,6 +388,29 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const KvVie
   plan->keff = keff;
   plan->n = n;
   plan->nb = kv.n;
+  // the selection rule: how many keys a task selects at most (blocks, for
+  // block selection), and the capacity of the sets it writes (rows)
+  const lyc_selection sel = ctx->sel;
+  plan->sel = sel;
+  const int E = sel.rule == LYC_RULE_BLOCK_TOPK ? sel.block : 1;
+  if (sel.rule == LYC_RULE_BLOCK_TOPK && k < E)
+    return fail(ctx, LYC_ERR_INVALID_ARG, "block selection needs k >= block");
+  plan->variable = sel.rule == LYC_RULE_BLOCK_TOPK || sel.rule == LYC_RULE_TOPP ||
+                   sel.rule == LYC_RULE_THRESHOLD;
+  auto select_cap = [&](int64_t nb) -> int {  // keys (blocks) selected at most
+    if (sel.rule == LYC_RULE_RATIO) {
+      const int64_t m = (sel.ratio_num * nb + sel.ratio_den - 1) / sel.ratio_den;
+      return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>({m, k, nb})));
+    }
+    if (sel.rule == LYC_RULE_BLOCK_TOPK) return static_cast<int>(std::min<int64_t>(k / E, (nb + E - 1) / E));
+    return static_cast<int>(std::min<int64_t>(k, nb));
+  };
+  auto set_rows = [&](int64_t nb) -> int {  // rows a set holds at most
+    if (sel.rule == LYC_RULE_BLOCK_TOPK) return static_cast<int>(std::min<int64_t>((k / E) * E, nb));
+    return select_cap(nb);
+  };
+  plan->set_rows.clear();
+  for (int b = 0; b < B; ++b) plan->set_rows.push_back(set_rows(kv.n[b]));
   plan->paged = kv.paged();
   plan->nsets = B * Hs;
   plan->gather_rows = 0;
@@ -405,6 +440,8 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const KvVie
     std::vector<Piece> pieces;
     std::vector<int32_t> cta;
     std::vector<TopkTask> tasks;
+    std::vector<BlockTask> btasks;  // block selection: one per task
+    int topk_n = 0;
     std::vector<const int32_t*> trace_src;
     std::vector<int2> combine;  // bf16: (segment, output) left to the next launch
     int nqb = 1;
@@ -442,7 +479,7 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const KvVie
     int maxnq = 1;
     for (int b = 0; b < B; ++b) {
       const int nb = static_cast<int>(kv.n[b]);  // this element's rows
-      const int keffb = std::min(k, nb);
+      const int keffb = plan->set_rows[b];       // rows of its sets at most
       for (int g = 0; g < Hkv; ++g) {
         // row 0 of (l, b, g); paged: of page 0, rows found through b's block table
         const int64_t off = l * kv.s_layer + (kv.paged() ? 0 : b * kv.s_batch) + g * kv.s_head;
@@ -494,6 +531,7 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const KvVie
           ss.kind = kSparse;
           ss.rows = keffb;
           ss.idx = set_ptr(cur[g], b, g);
+          ss.pad_ok = plan->variable ? 1 : 0;
           int js = 0;
           for (int h = g * G; h < (g + 1) * G; ++h)
             if (!is_ret[h]) {
@@ -514,6 +552,7 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const KvVie
             ss.kind = kSparse;
             ss.rows = keffb;
             ss.idx = set_ptr(cur[h], b, h);
+            ss.pad_ok = plan->variable ? 1 : 0;
             ss.head[0] = h;
             ss.out_row[0] = 0;
             ss.nq = ss.nout = 1;
@@ -631,11 +670,24 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const KvVie
     for (int s = 0; s < Hs; ++s) {
       if (!fresh[s]) continue;
       for (int b = 0; b < B; ++b) {
-        TopkTask tk;
+        TopkTask tk{};
         tk.keys = ctx->keys + keys_base + (static_cast<int64_t>(b) * Hs + s) * ctx->nstride;
         tk.S = set_ptr(1 - cur[s], b, s);
         tk.done = ctx->flags + ((static_cast<int64_t>(l) * B + b) * Hs + s) * 2;
         tk.n = static_cast<int32_t>(kv.n[b]);
+        tk.k = select_cap(kv.n[b]);
+        if (sel.rule == LYC_RULE_BLOCK_TOPK) {
+          // the selection runs over the element's block scores
+          BlockTask bk{};
+          bk.keys = tk.keys;
+          bk.scores = ctx->bkeys + ((static_cast<int64_t>(l) * B + b) * Hs + s) * ctx->bstride;
+          bk.n = tk.n;
+          H.btasks.push_back(bk);
+          tk.keys = bk.scores;
+          tk.rows = tk.n;
+          tk.n = static_cast<int32_t>((kv.n[b] + E - 1) / E);
+        }
+        H.topk_n = std::max(H.topk_n, static_cast<int>(tk.n));
         H.tasks.push_back(tk);
       }
     }
@@ -672,6 +724,9 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const KvVie
     lp.off_pieces = take(H.pieces.size() * sizeof(Piece));
     lp.off_cta = take(H.cta.size() * sizeof(int32_t));
     lp.off_tasks = take(std::max<size_t>(1, H.tasks.size()) * sizeof(TopkTask));
+    lp.topk_n = H.topk_n;
+    lp.off_btasks = take(std::max<size_t>(1, H.btasks.size()) * sizeof(BlockTask));
+    lp.bmax = H.btasks.empty() ? 0 : H.topk_n;
     lp.off_trace_src = take(H.trace_src.size() * sizeof(void*));
     lp.ncombine = static_cast<int>(H.combine.size());
     lp.off_combine = take(std::max<size_t>(1, H.combine.size()) * sizeof(int2));
@@ -695,6 +750,8 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const KvVie
     memcpy(host.data() + lp.off_cta, H.cta.data(), H.cta.size() * sizeof(int32_t));
     if (!H.tasks.empty())
       memcpy(host.data() + lp.off_tasks, H.tasks.data(), H.tasks.size() * sizeof(TopkTask));
+    if (!H.btasks.empty())
+      memcpy(host.data() + lp.off_btasks, H.btasks.data(), H.btasks.size() * sizeof(BlockTask));
     memcpy(host.data() + lp.off_trace_src, H.trace_src.data(), H.trace_src.size() * sizeof(void*));
     if (!H.combine.empty())
       memcpy(host.data() + lp.off_combine, H.combine.data(), H.combine.size() * sizeof(int2));
@@ -781,8 +838,9 @@ lyc_status enqueue_step(lyc_ctx* ctx, Plan* plan, cudaStream_t stream, int set, 
       // per batch element: its sets hold min(k, n[b]) indices below n[b]
       for (int b = 0; b < B; ++b) {
         const int nb = static_cast<int>(plan->nb[b]);
+        const int cap = plan->set_rows[b];
         ValidateSetsParams vp{ctx->sbuf + static_cast<int64_t>(b) * ctx->Hs * ctx->KS, ctx->status, ctx->Hs,
-                              ctx->KS, plan->k, std::min(plan->k, nb), nb};
+                              ctx->KS, plan->k, cap, nb, plan->variable ? std::min(1, cap) : cap};
         LYC_CUDA(validate_sets_launch(&vp, stream), "validate S^(0)");
       }
     }
@@ -870,13 +928,28 @@ lyc_status enqueue_step(lyc_ctx* ctx, Plan* plan, cudaStream_t stream, int set, 
     if ((st = record_event(ctx, plan, set, ev++, stream, capturing)) != LYC_OK) return st;
     plan->kernel_kind.push_back(0);
     plan->kernel_layer.push_back(l);
+    if (lp.ntasks > 0 && lp.bmax > 0) {
+      // block selection: every task's block scores first
+      BlockScoreParams bp{reinterpret_cast<const BlockTask*>(plan->dev + lp.off_btasks), lp.ntasks,
+                          plan->sel.block, lp.bmax};
+      if ((st = record_event(ctx, plan, set, ev++, stream, capturing)) != LYC_OK) return st;
+      LYC_CUDA(block_scores_launch(&bp, ctx->sms, stream), "block-score launch");
+      if ((st = record_event(ctx, plan, set, ev++, stream, capturing)) != LYC_OK) return st;
+      plan->kernel_kind.push_back(2);
+      plan->kernel_layer.push_back(l);
+    }
     if (lp.ntasks > 0) {
       TopkParams tp{};
       tp.tasks = reinterpret_cast<const TopkTask*>(plan->dev + lp.off_tasks);
       tp.epoch = ctx->epoch;
       tp.early = early_trigger(l) ? 1 : 0;
-      tp.n = plan->n;
+      tp.n = lp.topk_n;
       tp.k = plan->k;
+      tp.size_rule = plan->sel.rule == LYC_RULE_TOPP        ? kSizeTopP
+                     : plan->sel.rule == LYC_RULE_THRESHOLD ? kSizeThreshold
+                                                            : kSizeFixed;
+      tp.size_x = plan->sel.rule == LYC_RULE_TOPP ? plan->sel.p : plan->sel.tau;
+      tp.expand = plan->sel.rule == LYC_RULE_BLOCK_TOPK ? plan->sel.block : 1;
       tp.timeline = plan->timeline;
       tp.timeline_cap = plan->timeline_cap;
       tp.layer = l;
@@ -1244,7 +1317,7 @@ void lyc_destroy(lyc_ctx* ctx) {
   for (cudaEvent_t ev : ctx->events) cudaEventDestroy(ev);
   void* bufs[] = {ctx->status, ctx->keys, ctx->flags, ctx->sbuf, ctx->part_o, ctx->part_ml,
                   ctx->wpart_o, ctx->wpart_ml, ctx->counters, ctx->q_dev, ctx->out_dev,
-                  ctx->S_dev};
+                  ctx->S_dev, ctx->bkeys};
   for (void* b : bufs)
     if (b) cudaFree(b);
   timed_steps().erase(ctx);
@@ -1267,6 +1340,7 @@ lyc_status step_impl(lyc_ctx* ctx, const void* q, const KvView& kv, const uint8_
   std::string key = plan_key(role_mask, c.num_layers, c.num_q_heads, kv, k, step_flags, q, out, S,
                              ctx->trace, ctx->timing);
   key.append(reinterpret_cast<const char*>(&ctx->timeline), sizeof ctx->timeline);
+  key.append(reinterpret_cast<const char*>(&ctx->sel), sizeof ctx->sel);
   Plan* plan = nullptr;
   for (auto it = ctx->plans.begin(); it != ctx->plans.end(); ++it) {
     if (it->first == key) {
@@ -1402,6 +1476,64 @@ lyc_status lyc_sync_status(lyc_ctx* ctx) {
   return LYC_OK;
 }
 
+lyc_status lyc_set_selection(lyc_ctx* ctx, const lyc_selection* sel) {
+  if (!ctx) return LYC_ERR_INVALID_ARG;
+  lyc_selection s{};
+  s.rule = LYC_RULE_TOPK;
+  if (sel) s = *sel;
+  switch (s.rule) {
+    case LYC_RULE_TOPK: break;
+    case LYC_RULE_RATIO:
+      if (s.ratio_den < 1 || s.ratio_num < 0 || s.ratio_num > (1ll << 32) || s.ratio_den > (1ll << 32))
+        return fail(ctx, LYC_ERR_INVALID_ARG, "ratio needs 0 <= num, 1 <= den (both below 2^32)");
+      break;
+    case LYC_RULE_BLOCK_TOPK:
+      if (s.block < 1 || s.block > ctx->cfg.max_k)
+        return fail(ctx, LYC_ERR_INVALID_ARG, "block selection needs 1 <= block <= max_k");
+      break;
+    case LYC_RULE_TOPP:
+      if (!(s.p > 0.0 && s.p <= 1.0)) return fail(ctx, LYC_ERR_INVALID_ARG, "top-p needs 0 < p <= 1");
+      break;
+    case LYC_RULE_THRESHOLD:
+      if (!(s.tau >= 0.0)) return fail(ctx, LYC_ERR_INVALID_ARG, "threshold needs tau >= 0");
+      break;
+    default: return fail(ctx, LYC_ERR_INVALID_ARG, "unknown selection rule");
+  }
+  // only the fields of the rule take part in the plan key
+  lyc_selection c{};
+  c.rule = s.rule;
+  if (s.rule == LYC_RULE_RATIO) {
+    c.ratio_num = s.ratio_num;
+    c.ratio_den = s.ratio_den;
+  }
+  if (s.rule == LYC_RULE_BLOCK_TOPK) c.block = s.block;
+  if (s.rule == LYC_RULE_TOPP) c.p = s.p;
+  if (s.rule == LYC_RULE_THRESHOLD) c.tau = s.tau;
+  DeviceGuard guard(ctx->cfg.device);
+  if (!guard.ok) return fail(ctx, LYC_ERR_CUDA, "cudaSetDevice failed");
+  // the cached plans hold the old rule's records (and score rows)
+  for (auto& kv : ctx->plans) free_plan(kv.second.get());
+  ctx->plans.clear();
+  if (ctx->bkeys) {
+    LYC_CUDA(cudaFree(ctx->bkeys), "cudaFree(block scores)");
+    ctx->bkeys = nullptr;
+    ctx->bstride = 0;
+  }
+  if (c.rule == LYC_RULE_BLOCK_TOPK) {
+    const lyc_config& cf = ctx->cfg;
+    ctx->bstride = round_up((ctx->nstride + c.block - 1) / c.block, 4);
+    const size_t bytes = static_cast<size_t>(cf.num_layers) * cf.batch * ctx->Hs * ctx->bstride * sizeof(float);
+    if (cudaMalloc(&ctx->bkeys, bytes) != cudaSuccess) {
+      cudaGetLastError();
+      ctx->bkeys = nullptr;
+      ctx->bstride = 0;
+      return fail(ctx, LYC_ERR_OOM, "block-score rows");
+    }
+  }
+  ctx->sel = c;
+  return LYC_OK;
+}
+
 lyc_status lyc_set_s_trace(lyc_ctx* ctx, int32_t* trace) {
   if (!ctx) return LYC_ERR_INVALID_ARG;
   ctx->trace = trace;
@@ -1419,7 +1551,8 @@ lyc_status lyc_set_timing(lyc_ctx* ctx, int mode) {
   if (!ctx || (mode != LYC_TIMING_OFF && mode != LYC_TIMING_ON)) return LYC_ERR_INVALID_ARG;
   DeviceGuard guard(ctx->cfg.device);
   if (mode == LYC_TIMING_ON && ctx->events.empty()) {
-    ctx->events_per_set = 4 * ctx->cfg.num_layers + 2;  // + the last layer's combine launch
+    // attention, block scores, selection per layer, and the last layer's combine launch
+    ctx->events_per_set = 6 * ctx->cfg.num_layers + 2;
     const size_t total = static_cast<size_t>(timing_sets()) * ctx->events_per_set;
     ctx->events.resize(total, nullptr);
     for (size_t i = 0; i < total; ++i)

@@ -13,6 +13,12 @@ namespace lyc {
 // timeout bit of the status word and lets the kernel run to its end.
 constexpr uint64_t kWaitLimitNs = 4000000000ull;
 
+// An inherited index that is an error: outside [0, nvalid), except the -1
+// padding of a set shorter than its capacity when the segment allows it.
+__device__ __forceinline__ bool index_bad(int32_t x, int32_t nvalid, int32_t pad_ok) {
+  return x >= nvalid || x < (pad_ok ? -1 : 0);
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

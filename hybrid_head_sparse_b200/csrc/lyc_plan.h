@@ -61,7 +61,7 @@ struct Segment {
   int32_t cnt_base;     // first arrival counter of this segment
   int32_t row_base;     // row of (l, b, g, token 0) in the flattened row-gather map
   int32_t dep;          // sparse: the set is the previous launch's output (wait for it)
-  int32_t pad_;
+  int32_t pad_ok;       // sparse: -1 entries are padding of a shorter set (masked, not errors)
   const uint32_t* ready;  // sparse: flag word of the selection that wrote the set in
                           // this step (it holds the step's epoch + 1 once the set is
                           // complete), or NULL when the set comes from the caller
@@ -133,12 +133,24 @@ struct AttnParams {
 
 struct TopkTask {
   const float* keys;  // n selection keys
-  int32_t* S;         // k outputs
+  int32_t* S;         // the launch's k outputs
   uint32_t* done;     // NULL, or {arrival counter, ready flag}: the last CTA of the task
                       // to finish resets the counter and sets the flag to epoch + 1
   int32_t n;          // keys of this task (a batch element's rows); 0: the launch's n
+  int32_t k;          // at most this many keys are selected; 0: the launch's k
+  int32_t rows;       // with expand > 1: the element's rows (expanded rows past it are -1)
   int32_t pad_;
 };
+
+// How many keys a task selects (at most its k, at most n):
+//  kSizeFixed     : k;
+//  kSizeTopP      : the fewest largest keys whose probabilities softmax(keys)
+//                   sum to at least size_x;
+//  kSizeThreshold : the keys whose probability is at least size_x (at least one).
+// The last two take their decision on 40-bit fixed-point weights
+// round(2^40 exp(key - max)): integer sums are exact and independent of the
+// order of the additions, so every CTA of a cluster reaches the same size.
+enum TopkSizeRule : int32_t { kSizeFixed = 0, kSizeTopP = 1, kSizeThreshold = 2 };
 
 struct TopkParams {
   const TopkTask* tasks;  // one per blockIdx.y; NULL: use `single`
@@ -149,7 +161,26 @@ struct TopkParams {
   unsigned long long* timeline;  // as in AttnParams
   int32_t timeline_cap;
   int32_t layer;
-  int32_t n, k;
+  int32_t n, k;           // k: entries of each output set
+  int32_t size_rule;      // TopkSizeRule
+  int32_t expand;         // > 1: key j stands for rows j*expand .. j*expand + expand - 1 (block
+                          // selection); the output lists those rows
+  double size_x;          // p (top-p) or tau (threshold)
+};
+
+// block_scores_kernel: per task, the score of every block of `block` rows of
+// a key row: log(sum over the block's rows of exp(key)), computed as
+// max + log(sum exp(key - max)) (ordering blocks by it orders them by their
+// summed probability)
+struct BlockTask {
+  const float* keys;  // the task's n key rows
+  float* scores;      // ceil(n / block) scores
+  int32_t n;
+  int32_t pad_;
+};
+struct BlockScoreParams {
+  const BlockTask* tasks;
+  int32_t ntasks, block, max_blocks;
 };
 
 // Timeline tags: kind << 32 | layer << 16 | CTA
@@ -183,12 +214,13 @@ struct AppendParams {
   int32_t L, B, Hkv, row_bytes, elem_bytes;
 };
 
-// validate_sets_kernel: each of nsets sets (stride `stride`) must hold k_eff
-// ascending indices in [0, n) followed by -1 up to k
+// validate_sets_kernel: each of nsets sets (stride `stride`) must hold
+// between min_valid and k_eff ascending indices in [0, n), followed by -1 up to k
 struct ValidateSetsParams {
   const int32_t* sets;
   uint32_t* status;
   int32_t nsets, stride, k, k_eff, n;
+  int32_t min_valid;
 };
 
 // Order-preserving map of an fp32 selection key to an unsigned integer

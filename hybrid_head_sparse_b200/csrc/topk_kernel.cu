@@ -24,6 +24,22 @@
 // candidates do not fit (heavily tied keys), two more radix digits run over
 // the chunks with totals pushed into every CTA, and the CTA counts are
 // exchanged instead.
+//
+// Selection rules other than a fixed k (page "LycheeDecode ...", section
+// 4.4.1, Figure 6, Tables 5-6): the number of keys to select is found first,
+// then the same selection runs with it.
+//  * top-p (the fewest largest keys whose probabilities reach p) and
+//    threshold (the keys of probability >= tau): the cluster's maximum key M
+//    is exchanged first; every key gets the weight W = round(2^40 exp(x - M))
+//    (an integer: sums are exact whatever their order, so every CTA takes the
+//    same decision).  Threshold counts W >= ceil(tau * sum W).  Top-p finds
+//    the key value at which the running mass, larger keys first, reaches
+//    T = ceil(p * sum W): a radix descent on the same digits as the
+//    selection, with per-digit counts and masses pushed into every CTA
+//    (one more cluster barrier per digit), then how many of the keys equal
+//    to that value it takes;
+//  * block selection: the keys are block scores (block_scores_kernel) and
+//    each selected block is written out as its rows.
 #include <cooperative_groups.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -39,6 +55,26 @@ constexpr int kTopkThreads = 512;
 constexpr int kTopkWarps = kTopkThreads / 32;
 constexpr int kTopkCandCap = 4096;  // pivot-digit candidates gathered from the whole cluster
 constexpr int kTopkSelCap = 4096;   // one CTA's keys at or above the pivot digit
+// words of the size-rule exchange area: vx[16], vcnt[16] (u32), then 40 u64
+constexpr int kTopkRuleWords = 32 + 80;
+
+// The fp32 key an order-preserving encoding stands for (-0 comes back as +0).
+__device__ __forceinline__ float key_from_order(uint32_t u) {
+  const uint32_t b = (u & 0x80000000u) ? (u & 0x7fffffffu) : ~u;
+  return __uint_as_float(b);
+}
+
+// 40-bit fixed-point weight of a key relative to the maximum M (x <= M):
+// round(2^40 exp(x - M)), at most 2^40.
+__device__ __forceinline__ unsigned long long key_weight(uint32_t u, float M) {
+  return __float2ull_rn(expf(key_from_order(u) - M) * 1099511627776.0f);
+}
+
+__device__ __forceinline__ unsigned long long warp_sum_u64(unsigned long long v) {
+#pragma unroll
+  for (int s = 16; s >= 1; s >>= 1) v += __shfl_xor_sync(0xffffffffu, v, s);
+  return v;
+}
 
 // Exclusive prefix sum of one value per warp (lane 0's) over the CTA; also the total.
 __device__ __forceinline__ void cta_warp_scan(uint32_t* scratch, uint32_t mine, int warp, int lane,
@@ -92,6 +128,66 @@ __device__ __forceinline__ void find_digit(const uint32_t* hist, uint32_t krem, 
   __syncthreads();
   *digit = found[0];
   *above_out = found[1];
+  __syncthreads();
+}
+
+// Find the digit d with  mass(> d) < target <= mass(>= d)  over NB bins of
+// (count, mass); every thread returns the same digit and the count and mass
+// of the bins above it.  Integer sums: the same in every CTA.
+template <int NB>
+__device__ __forceinline__ void find_digit_mass(const unsigned long long* mass, const uint32_t* cntb,
+                                                unsigned long long target, unsigned long long* scr64,
+                                                uint32_t* scr32, unsigned long long* res, int tid,
+                                                int lane, int warp, uint32_t* digit, uint32_t* cabove,
+                                                unsigned long long* mabove) {
+  constexpr int per = NB / kTopkThreads;
+  unsigned long long m[per];
+  uint32_t c[per];
+  unsigned long long mm = 0ull;
+  uint32_t mc = 0u;
+#pragma unroll
+  for (int q = 0; q < per; ++q) {
+    m[q] = mass[tid * per + q];
+    c[q] = cntb[tid * per + q];
+    mm += m[q];
+    mc += c[q];
+  }
+  unsigned long long sm = mm;  // inclusive suffix sums within the warp
+  uint32_t sc = mc;
+#pragma unroll
+  for (int s = 1; s < 32; s <<= 1) {
+    const unsigned long long vm = __shfl_down_sync(0xffffffffu, sm, s);
+    const uint32_t vc = __shfl_down_sync(0xffffffffu, sc, s);
+    if (lane + s < 32) {
+      sm += vm;
+      sc += vc;
+    }
+  }
+  if (lane == 0) {
+    scr64[warp] = sm;
+    scr32[warp] = sc;
+  }
+  __syncthreads();
+  unsigned long long am = sm - mm;
+  uint32_t ac = sc - mc;
+  for (int w2 = warp + 1; w2 < kTopkWarps; ++w2) {
+    am += scr64[w2];
+    ac += scr32[w2];
+  }
+#pragma unroll
+  for (int q = per - 1; q >= 0; --q) {
+    if (am < target && am + m[q] >= target) {
+      res[0] = static_cast<unsigned long long>(tid * per + q);
+      res[1] = ac;
+      res[2] = am;
+    }
+    am += m[q];
+    ac += c[q];
+  }
+  __syncthreads();
+  *digit = static_cast<uint32_t>(res[0]);
+  *cabove = static_cast<uint32_t>(res[1]);
+  *mabove = res[2];
   __syncthreads();
 }
 
@@ -190,8 +286,12 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster_kernel(const Top
   const int rank = static_cast<int>(cluster.block_rank());
   const TopkTask task = p.tasks ? p.tasks[blockIdx.y] : p.single;
   const int n = task.n > 0 ? task.n : p.n;
-  const int k = p.k;
-  const int keff = k < n ? k : n;
+  const int k = p.k;                                 // entries of the output set
+  const int kcap = task.k > 0 ? task.k : k;          // keys selected at most
+  const int E = p.expand > 1 ? p.expand : 1;         // rows per selected key
+  const int rows = task.rows > 0 ? task.rows : n * E;
+  const int rule = p.size_rule;
+  int keff = kcap < n ? kcap : n;
   const int chunk = (((n + CL - 1) / CL) + 3) & ~3;
   const int lo = rank * chunk;
   const int cnt = max(0, min(n, lo + chunk) - lo);
@@ -218,23 +318,59 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster_kernel(const Top
   uint32_t* xchg = src_eq + CL;                        // [CL][2] (fallback path)
   uint32_t* scratch = xchg + 2 * CL;                   // [kTopkWarps]
   uint32_t* found = scratch + kTopkWarps;              // [4]
-  uint32_t* us = found + 4;                            // [chunk] encoded keys (16-byte aligned)
+  uint32_t* vx = found + 4;                            // [16] size rules: per source, max key
+  uint32_t* vcnt = vx + 16;                            // [16] per source: keys counted
+  unsigned long long* vsum = reinterpret_cast<unsigned long long*>(vcnt + 16);  // [16] masses
+  unsigned long long* scr64 = vsum + 16;               // [16]
+  unsigned long long* res64 = scr64 + 16;              // [8]
+  uint32_t* us = reinterpret_cast<uint32_t*>(res64 + 8);  // [chunk] encoded keys (16-byte aligned)
+  // top-p, before the selection proper: cand = local masses, digit-1 mass
+  // totals; sel = digit-0 (later digit-2) mass totals, digit-2 and digit-1
+  // count totals
+  unsigned long long* lmass = reinterpret_cast<unsigned long long*>(cand);
+  unsigned long long* mt1 = lmass + kKeyBins;
+  unsigned long long* mt0 = reinterpret_cast<unsigned long long*>(sel);
+  uint32_t* ct2 = reinterpret_cast<uint32_t*>(mt0 + kKeyBins);
+  uint32_t* ct1 = ct2 + kKeyBins;
 
-  if (keff == n) {  // every index is selected
-    for (int x = tid; x < cnt; x += kTopkThreads) task.S[lo + x] = lo + x;
+  // the output: selected key j at position pos (its rows with block selection)
+  auto put = [&](uint32_t pos, int32_t j) {
+    if (E == 1) {
+      task.S[pos] = j;
+    } else {
+      for (int t = 0; t < E; ++t) {
+        const int64_t r = static_cast<int64_t>(j) * E + t;
+        task.S[static_cast<int64_t>(pos) * E + t] = r < rows ? static_cast<int32_t>(r) : -1;
+      }
+    }
+  };
+  auto all_selected = [&]() {  // every key is selected
+    for (int x = tid; x < cnt; x += kTopkThreads) put(static_cast<uint32_t>(lo + x), lo + x);
     if (rank == 0)
-      for (int x = keff + tid; x < k; x += kTopkThreads) task.S[x] = -1;
+      for (int x = keff * E + tid; x < k; x += kTopkThreads) task.S[x] = -1;
     topk_signal_done<CL>(p, task, tid);
     if (tid == 0)
       timeline_record(p.timeline, p.timeline_cap, t_start,
                       (kTagTopk << 32) | (static_cast<unsigned long long>(p.layer) << 16) |
                           (blockIdx.y * CL + rank));
+  };
+  if (rule == kSizeFixed && keff == n) {
+    all_selected();
     return;
   }
 
   for (int b = tid; b < kKeyBins; b += kTopkThreads) {
     tot[b] = 0u;
     loc[b] = 0u;
+  }
+  if (rule != kSizeFixed) {
+    if (tid < 8) res64[tid] = 0ull;
+    if (rule == kSizeTopP) {  // every total of the descent, and the local masses
+      uint32_t* a = reinterpret_cast<uint32_t*>(cand);
+      uint32_t* b2 = reinterpret_cast<uint32_t*>(sel);
+      for (int x = tid; x < 2 * kTopkCandCap; x += kTopkThreads) a[x] = 0u;
+      for (int x = tid; x < 2 * kTopkSelCap; x += kTopkThreads) b2[x] = 0u;
+    }
   }
   __syncthreads();
   // Every pass over the chunk gives warp w the contiguous range [wlo, whi)
@@ -255,6 +391,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster_kernel(const Top
   };
 
   // ---- the chunk, encoded, into shared memory, and its top-digit histogram
+  uint32_t umax = 0u;  // size rules: the largest encoded key of this thread
   {
     const float* src = task.keys + lo;
     const bool vec = (reinterpret_cast<uintptr_t>(src) & 15u) == 0;
@@ -274,11 +411,65 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster_kernel(const Top
       }
 #pragma unroll
       for (int e = 0; e < 4; ++e)
-        if (x0 + e < whi) atomicAdd(&loc[u[e] >> kKeyDigitShift], 1u);
+        if (x0 + e < whi) {
+          atomicAdd(&loc[u[e] >> kKeyDigitShift], 1u);
+          umax = max(umax, u[e]);
+        }
     }
+  }
+  if (rule != kSizeFixed) {
+    umax = __reduce_max_sync(FULL, umax);
+    if (lane == 0) atomicMax(&res64[5], static_cast<unsigned long long>(umax));
   }
   __syncthreads();
   cluster.sync();  // (1) every CTA's totals are zero and its histogram complete
+
+  // ---- size rules: the cluster's largest key, then threshold's count or
+  // top-p's digit-0 masses
+  float M = 0.f;
+  if (rule != kSizeFixed) {
+    if (tid < CL) cluster.map_shared_rank(vx, tid)[rank] = static_cast<uint32_t>(res64[5]);
+    cluster.sync();
+    uint32_t um = 0u;
+    for (int r = 0; r < CL; ++r) um = max(um, vx[r]);
+    M = key_from_order(um);
+    if (rule == kSizeThreshold) {
+      unsigned long long sw = 0ull;
+      for (int x = tid; x < cnt; x += kTopkThreads) sw += key_weight(us[x], M);
+      sw = warp_sum_u64(sw);
+      if (lane == 0) atomicAdd(&res64[4], sw);
+      __syncthreads();
+      if (tid < CL) cluster.map_shared_rank(vsum, tid)[rank] = res64[4];
+      cluster.sync();
+      unsigned long long total = 0ull;
+      for (int r = 0; r < CL; ++r) total += vsum[r];
+      const double tg = ceil(p.size_x * static_cast<double>(total));
+      const unsigned long long thr = tg <= 0.0 ? 0ull : static_cast<unsigned long long>(tg);
+      uint32_t c = 0u;
+      for (int x = tid; x < cnt; x += kTopkThreads) c += key_weight(us[x], M) >= thr ? 1u : 0u;
+      c = __reduce_add_sync(FULL, c);
+      if (lane == 0) atomicAdd(&res64[6], static_cast<unsigned long long>(c));
+      __syncthreads();
+      if (tid < CL) cluster.map_shared_rank(vcnt, tid)[rank] = static_cast<uint32_t>(res64[6]);
+      cluster.sync();
+      uint32_t m = 0u;
+      for (int r = 0; r < CL; ++r) m += vcnt[r];
+      m = max(m, 1u);
+      keff = min(keff, static_cast<int>(m));
+    } else {
+      for (int x = tid; x < cnt; x += kTopkThreads) {
+        const uint32_t u = us[x];
+        atomicAdd(&lmass[u >> kKeyDigitShift], key_weight(u, M));
+      }
+      __syncthreads();
+      for (int x = tid; x < CL * kKeyBins; x += kTopkThreads) {
+        const int b = x % kKeyBins, r = x / kKeyBins;
+        const unsigned long long w = lmass[b];
+        if (w) atomicAdd(cluster.map_shared_rank(mt0, r) + b, w);
+      }
+      __syncthreads();  // the local masses are read before `cand` is reused below
+    }
+  }
 
   // ---- top digit: add the non-zero local bins into every CTA's totals
   {
@@ -290,6 +481,81 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster_kernel(const Top
     }
   }
   cluster.sync();  // (2)
+  if (rule == kSizeTopP) {
+    // the mass to reach, and a radix descent to the key value that reaches it
+    unsigned long long tm = 0ull;
+    for (int b = tid; b < kKeyBins; b += kTopkThreads) tm += mt0[b];
+    tm = warp_sum_u64(tm);
+    if (lane == 0) scr64[warp] = tm;
+    __syncthreads();
+    unsigned long long total = 0ull;
+    for (int w2 = 0; w2 < kTopkWarps; ++w2) total += scr64[w2];
+    __syncthreads();
+    const double tg = ceil(p.size_x * static_cast<double>(total));
+    unsigned long long target =
+        tg >= static_cast<double>(total) ? total : (tg < 1.0 ? 1ull : static_cast<unsigned long long>(tg));
+    uint32_t dg, ca;
+    unsigned long long ma;
+    find_digit_mass<kKeyBins>(mt0, tot, target, scr64, scratch, res64, tid, lane, warp, &dg, &ca, &ma);
+    uint32_t m_above = ca;
+    target -= ma;
+    uint32_t prefix = dg << kKeyDigitShift, pmask = 0xffe00000u;
+    unsigned long long* mt2 = mt0;  // digit-0 totals are read: digit 2 reuses them
+    for (int b = tid; b < kKeyBins; b += kTopkThreads) mt2[b] = 0ull;
+#pragma unroll
+    for (int pass = 1; pass <= 2; ++pass) {
+      const int sh = pass == 1 ? 10 : 0;
+      const uint32_t dmask = pass == 1 ? 0x7ffu : 0x3ffu;
+      unsigned long long* mt = pass == 1 ? mt1 : mt2;
+      uint32_t* ct = pass == 1 ? ct1 : ct2;
+      for (int b = tid; b < kKeyBins; b += kTopkThreads) {
+        loc[b] = 0u;
+        lmass[b] = 0ull;
+      }
+      __syncthreads();
+      for (int x = tid; x < cnt; x += kTopkThreads) {
+        const uint32_t u = us[x];
+        if ((u & pmask) == prefix) {
+          const uint32_t d = (u >> sh) & dmask;
+          atomicAdd(&loc[d], 1u);
+          atomicAdd(&lmass[d], key_weight(u, M));
+        }
+      }
+      __syncthreads();
+      const int nbins = pass == 1 ? kKeyBins : kKeyBins / 2;
+      for (int x = tid; x < CL * nbins; x += kTopkThreads) {
+        const int b = x % nbins, r = x / nbins;
+        const uint32_t c = loc[b];
+        if (c) {
+          atomicAdd(cluster.map_shared_rank(ct, r) + b, c);
+          const unsigned long long w = lmass[b];
+          if (w) atomicAdd(cluster.map_shared_rank(mt, r) + b, w);
+        }
+      }
+      cluster.sync();
+      if (pass == 1)
+        find_digit_mass<kKeyBins>(mt, ct, target, scr64, scratch, res64, tid, lane, warp, &dg, &ca, &ma);
+      else
+        find_digit_mass<kKeyBins / 2>(mt, ct, target, scr64, scratch, res64, tid, lane, warp, &dg, &ca,
+                                      &ma);
+      m_above += ca;
+      target -= ma;
+      prefix |= dg << sh;
+      pmask |= dmask << sh;
+    }
+    // `prefix` is now the key value that reaches the mass: its keys all have
+    // the same weight; take as many of them as the rest of the mass needs
+    const uint32_t cv = ct2[prefix & 0x3ffu];
+    const unsigned long long wv = mt2[prefix & 0x3ffu] / (cv ? cv : 1u);
+    unsigned long long r = wv ? (target + wv - 1ull) / wv : cv;
+    r = r < 1ull ? 1ull : (r > cv ? cv : r);
+    keff = min(keff, static_cast<int>(m_above + static_cast<uint32_t>(r)));
+    __syncthreads();  // every read of `sel` precedes the selection's writes to it
+  }
+  if (rule != kSizeFixed && keff == n) {
+    all_selected();
+    return;
+  }
   uint32_t d0, above;
   find_digit(tot, static_cast<uint32_t>(keff), scratch, found, tid, lane, warp, &d0, &above);
   uint32_t krem = static_cast<uint32_t>(keff) - above;
@@ -514,7 +780,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster_kernel(const Top
         const bool pick = ((gb[j] >> lane) & 1u) || (is_eq && run_eq + __popc(eb[j] & lt) < take);
         const unsigned sb = __ballot_sync(FULL, pick);
         const uint32_t pos = run_sel + __popc(sb & lt);
-        if (pick && pos < static_cast<uint32_t>(keff)) task.S[pos] = static_cast<int32_t>(ent[j].y);
+        if (pick && pos < static_cast<uint32_t>(keff)) put(pos, static_cast<int32_t>(ent[j].y));
         run_sel += __popc(sb);
         run_eq += __popc(eb[j]);
       }
@@ -525,7 +791,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster_kernel(const Top
   else
     emit([&](int x) { return make_uint2(us[x], static_cast<uint32_t>(lo + x)); }, cnt);
   if (rank == 0)
-    for (int x = keff + tid; x < k; x += kTopkThreads) task.S[x] = -1;
+    for (int x = keff * E + tid; x < k; x += kTopkThreads) task.S[x] = -1;
   topk_signal_done<CL>(p, task, tid);
   if (tid == 0)
     timeline_record(p.timeline, p.timeline_cap, t_start,
@@ -539,7 +805,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster_kernel(const Top
 static size_t topk_smem_bytes(int cl, int n) {
   const int chunk = (((n + cl - 1) / cl) + 3) & ~3;
   return static_cast<size_t>(2 * kTopkCandCap + 2 * kTopkSelCap + 2 * kKeyBins + 6 * cl + kTopkWarps +
-                             4 + chunk) * 4u;
+                             4 + kTopkRuleWords + chunk) * 4u;
 }
 
 template <int CL>

@@ -43,11 +43,17 @@ LYC_STEP_VALIDATE_S = 0x4
 LYC_TIMING_OFF = 0
 LYC_TIMING_ON = 1
 
+LYC_RULE_TOPK = 0
+LYC_RULE_RATIO = 1
+LYC_RULE_BLOCK_TOPK = 2
+LYC_RULE_TOPP = 3
+LYC_RULE_THRESHOLD = 4
+
 EXPORTED = ["lyc_create", "lyc_decode_step", "lyc_decode_step_host", "lyc_decode_step_batch",
             "lyc_sync_status",
             "lyc_set_s_trace", "lyc_step_bytes", "lyc_topk_f32", "lyc_set_timing",
             "lyc_kernel_times", "lyc_set_timeline", "lyc_status_string", "lyc_last_error",
-            "lyc_destroy", "lyc_sparse_attention_noalloc"]
+            "lyc_destroy", "lyc_sparse_attention_noalloc", "lyc_set_selection"]
 
 
 class lyc_config(ctypes.Structure):
@@ -73,6 +79,12 @@ class lyc_kv_batch(ctypes.Structure):
                 ("page_rows", ctypes.c_int32), ("max_blocks", ctypes.c_int32),
                 ("num_pages", ctypes.c_int64), ("k_new", ctypes.c_void_p),
                 ("v_new", ctypes.c_void_p)]
+
+
+class lyc_selection(ctypes.Structure):
+    _fields_ = [("rule", ctypes.c_int32), ("block", ctypes.c_int32),
+                ("ratio_num", ctypes.c_int64), ("ratio_den", ctypes.c_int64),
+                ("p", ctypes.c_double), ("tau", ctypes.c_double)]
 
 
 class lyc_kernel_time(ctypes.Structure):
@@ -106,6 +118,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     L.lyc_decode_step_batch.argtypes = [P, P, ctypes.POINTER(lyc_kv_batch), P, I, P, P, P,
                                         ctypes.c_uint32]
     L.lyc_sync_status.argtypes = [P]
+    L.lyc_set_selection.argtypes = [P, ctypes.POINTER(lyc_selection)]
     L.lyc_set_s_trace.argtypes = [P, P]
     L.lyc_step_bytes.argtypes = [ctypes.POINTER(lyc_config), P, ctypes.c_int64, I, I,
                                  ctypes.POINTER(ctypes.c_uint64), ctypes.POINTER(ctypes.c_uint64)]
@@ -164,6 +177,10 @@ def lyc_sparse_attention_noalloc(q, kv: lyc_kv_cache, batch, num_q_heads, num_kv
 
 def lyc_sync_status(ctx) -> int:
     return load().lyc_sync_status(ctx)
+
+
+def lyc_set_selection(ctx, sel: lyc_selection | None) -> int:
+    return load().lyc_set_selection(ctx, None if sel is None else ctypes.byref(sel))
 
 
 def lyc_set_s_trace(ctx, trace) -> int:
@@ -336,6 +353,12 @@ class Lyc:
 
     def sync_status(self) -> int:
         return lyc_sync_status(self.ctx)
+
+    def set_selection(self, rule=LYC_RULE_TOPK, block=64, ratio=(1, 2), p=0.9, tau=1e-3):
+        """The selection rule of the steps that follow (lyc_set_selection)."""
+        sel = lyc_selection(int(rule), int(block), int(ratio[0]), int(ratio[1]), float(p),
+                            float(tau))
+        self._check(lyc_set_selection(self.ctx, sel), "lyc_set_selection")
 
     def set_trace(self, trace):
         self._trace = trace

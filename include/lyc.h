@@ -192,6 +192,57 @@ lyc_status lyc_decode_step_batch(lyc_ctx* ctx, const void* q, const lyc_kv_batch
                                  const uint8_t* role_mask, int k, float* out, int32_t* S,
                                  void* stream, uint32_t step_flags);
 
+/* ---- Selection rules (page "LycheeDecode: Accelerating Long-Context LLM
+ * Inference via Hybrid-Head Sparse Decoding", paper-graph-ui summary: section
+ * 4.4.1 with Figure 6 and Tables 5-6 compare Top-k, Top-p, Threshold and
+ * Ratio; section 4.1 / Appendix F give the reasoning budget of 50 % of the
+ * length, growing during decoding; the kernel section uses blocks of 64 rows).
+ *
+ * Every rule chooses rows from the same selection key as argsTopK (Eq. 2:
+ * the retrieval head's logits, or the pooled query's in KVGROUP_MEAN mode);
+ * A = softmax(key) are their probabilities.  A set never holds more than the
+ * step's k rows, is written ascending and padded with -1, and holds at least
+ * one row:
+ *   TOPK        : the min(k, n) largest keys (ties to the lower index);
+ *   RATIO       : the ceil(ratio_num * n / ratio_den) largest keys (integer
+ *                 arithmetic; at least 1, at most k).  The reasoning budget is
+ *                 ratio 1/2 evaluated with each step's n;
+ *   BLOCK_TOPK  : rows in blocks of `block` (the last one may be shorter); a
+ *                 block's score is the sum of its rows' A; the floor(k / block)
+ *                 best blocks (ties to the lower block) are taken whole.  Needs
+ *                 1 <= block <= k;
+ *   TOPP        : the fewest largest keys whose A sum to at least p, 0 < p <= 1;
+ *   THRESHOLD   : the keys with A >= tau, 0 <= tau.
+ * TOPP and THRESHOLD decide on 40-bit fixed-point weights round(2^40 exp(key -
+ * max key)) and BLOCK_TOPK on fp32 block scores: a row whose fp64 mass sits
+ * within rounding of the boundary may fall on either side of it.
+ * Sets of BLOCK_TOPK, TOPP and THRESHOLD can hold fewer rows than their
+ * capacity; the sparse heads attend over their valid entries only.
+ *
+ * lyc_set_selection(ctx, NULL) restores TOPK.  The rule applies to the steps
+ * that follow (every step entry point); changing it releases the cached step
+ * plans.  Errors: INVALID_ARG (unknown rule, block < 1, ratio_den < 1,
+ * ratio_num < 0, p outside (0, 1], tau < 0), OOM, CUDA.  BLOCK_TOPK with a
+ * step k below `block` fails at the step with INVALID_ARG. */
+typedef enum {
+  LYC_RULE_TOPK = 0,
+  LYC_RULE_RATIO = 1,
+  LYC_RULE_BLOCK_TOPK = 2,
+  LYC_RULE_TOPP = 3,
+  LYC_RULE_THRESHOLD = 4
+} lyc_rule;
+
+typedef struct {
+  int32_t rule;       /* lyc_rule */
+  int32_t block;      /* BLOCK_TOPK: rows per block */
+  int64_t ratio_num;  /* RATIO: theta = ratio_num / ratio_den */
+  int64_t ratio_den;
+  double p;           /* TOPP */
+  double tau;         /* THRESHOLD */
+} lyc_selection;
+
+lyc_status lyc_set_selection(lyc_ctx* ctx, const lyc_selection* sel);
+
 /* Synchronize the stream of the last step, read and clear the device status
  * word.  Returns LYC_OK, LYC_ERR_BAD_INDEX, LYC_ERR_TIMEOUT or LYC_ERR_CUDA. */
 lyc_status lyc_sync_status(lyc_ctx* ctx);
@@ -221,7 +272,8 @@ lyc_status lyc_topk_f32(lyc_ctx* ctx, const float* keys, int64_t n, int k, int32
 /* Per-kernel device time of the steps since the last call, from CUDA events
  * recorded around every launch when timing is on (LYC_TIMING_ON).  Writes up
  * to `cap` entries of {kernel kind, layer, milliseconds}; returns the count in
- * *count.  Kinds: 0 = attention (pooled dense + sparse), 1 = top-k selection. */
+ * *count.  Kinds: 0 = attention (pooled dense + sparse), 1 = top-k selection,
+ * 2 = block scores (BLOCK_TOPK only). */
 typedef struct {
   int kind;
   int layer;

@@ -51,6 +51,14 @@ def parse_args(argv=None):
     ap.add_argument("--serving", action="store_true",
                     help="the serving form instead: lyc_decode_step_batch on a batch of four "
                          "cache lengths, paged cache (64-row pages), current token appended")
+    ap.add_argument("--selection", choices=["topk", "ratio", "block", "topp", "threshold"],
+                    default="topk",
+                    help="selection rule; anything but topk prints the rule's own line instead of "
+                         "the default one")
+    ap.add_argument("--ratio", default="1/64", help="ratio rule: theta as num/den")
+    ap.add_argument("--block", type=int, default=64, help="block rule: rows per block")
+    ap.add_argument("--p", type=float, default=0.5, help="top-p rule: probability mass")
+    ap.add_argument("--tau", type=float, default=1e-4, help="threshold rule: smallest probability")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-layers", type=int, default=2,
@@ -579,12 +587,127 @@ def run_serving(args):
     return 0
 
 
+def rule_kernel_bytes(role, trace, n, L, Hq, Hkv, d, select_mode):
+    """K+V bytes the attention kernels read in one step under a selection
+    rule: n rows for every KV group with a retrieval head (all at layer 0),
+    and for every sparse pass (a sparse head in per-head mode, a group's
+    sparse heads in group mode) the valid rows of the set it inherits."""
+    import numpy as np
+    G = Hq // Hkv
+    row = d * 2 * 2
+    sizes = (trace >= 0).sum(-1)  # [L][B][Hs]
+    total = 0
+    for l in range(L):
+        ret = np.ones(Hq, dtype=bool) if l == 0 else role[l].astype(bool)
+        for b in range(trace.shape[1]):
+            for g in range(Hkv):
+                heads = range(g * G, (g + 1) * G)
+                if any(ret[h] for h in heads):
+                    total += n * row
+                if l == 0:
+                    continue
+                if select_mode == "kvgroup_mean":
+                    if not all(ret[h] for h in heads):
+                        total += int(sizes[l - 1, b, g]) * row
+                else:
+                    total += sum(int(sizes[l - 1, b, h]) * row for h in heads if not ret[h])
+    return total
+
+
+def run_rule(args):
+    """The default workload under a selection rule other than a fixed k:
+    steps/s, the observed set sizes and the rate on the bytes the kernels
+    must read for those sets."""
+    import numpy as np
+    import torch
+
+    from hybrid_head_sparse_b200 import build as Bld
+    from hybrid_head_sparse_b200 import lyc, workloads as W
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    Bld.build()
+    lyc.load()
+    spec = workload_spec(args)
+    data = W.make_stack(spec, dev)
+    ctx = lyc.Lyc(spec.L, spec.B, spec.Hq, spec.Hkv, spec.d, spec.n, spec.k, dtype=spec.dtype,
+                  select_mode=args.select_mode)
+    num, den = (int(x) for x in args.ratio.split("/"))
+    rule = {"ratio": lyc.LYC_RULE_RATIO, "block": lyc.LYC_RULE_BLOCK_TOPK, "topp": lyc.LYC_RULE_TOPP,
+            "threshold": lyc.LYC_RULE_THRESHOLD}[args.selection]
+    ctx.set_selection(rule, block=args.block, ratio=(num, den), p=args.p, tau=args.tau)
+    out = torch.empty((spec.L, spec.B, spec.Hq, spec.d), device=dev)
+    S = torch.empty((spec.B, ctx.Hs, spec.k), dtype=torch.int32, device=dev)
+    role = data["role"]
+    stream = torch.cuda.current_stream(dev)
+    # one untimed step with the set trace: the sizes the rule chose
+    trace = torch.empty((spec.L, spec.B, ctx.Hs, spec.k), dtype=torch.int32, device=dev)
+    ctx.set_trace(trace)
+    ctx.decode_step(data["q"], data["k"], data["v"], spec.n, role, spec.k, out, S, stream=stream)
+    torch.cuda.synchronize()
+    tr = trace.cpu().numpy()
+    ctx.set_trace(None)
+    sizes = (tr >= 0).sum(-1)
+
+    def step():
+        ctx.decode_step(data["q"], data["k"], data["v"], spec.n, role, spec.k, out, S, stream=stream)
+
+    for _ in range(max(args.warmup, 1)):
+        step()
+    torch.cuda.synchronize()
+    rc = ctx.sync_status()
+    if rc != 0:
+        raise RuntimeError(f"device status after warm-up: {lyc.lyc_status_string(rc)}")
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    with ClockSampler(0) as clk:
+        evs[0].record(stream)
+        for i in range(args.steps):
+            step()
+            evs[i + 1].record(stream)
+        torch.cuda.synchronize()
+    rc = ctx.sync_status()
+    if rc != 0:
+        raise RuntimeError(f"device status after timing: {lyc.lyc_status_string(rc)}")
+    ms_total = evs[0].elapsed_time(evs[-1])
+    ms_step = ms_total / args.steps
+    kbytes = rule_kernel_bytes(role, tr, spec.n, spec.L, spec.Hq, spec.Hkv, spec.d, args.select_mode)
+    peak, _ = measured_peaks()
+    gbs = kbytes / (ms_step / 1e3) / 1e9
+    params = {"ratio": {"theta": args.ratio}, "block": {"block": args.block}, "topp": {"p": args.p},
+              "threshold": {"tau": args.tau}}[args.selection]
+    line = {
+        "metric": f"decode steps/s at 128K ctx, selection rule {args.selection}",
+        "value": args.steps / (ms_total / 1e3), "unit": "steps/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "step_ms_distribution": {kk: round(v, 4) for kk, v in percentiles(
+            [evs[i].elapsed_time(evs[i + 1]) for i in range(args.steps)]).items()},
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) q/K/V, sinks + 256 planted heavy hitters per KV head)",
+        "config": {"workload": spec.name, "L": spec.L, "B": spec.B, "Hq": spec.Hq, "Hkv": spec.Hkv,
+                   "d": spec.d, "n": spec.n, "k_capacity": spec.k, "selection": args.selection,
+                   **params, "retrieval_heads_per_layer": args.retrieval_heads,
+                   "select_mode": args.select_mode, "parallelism": "replicas x1",
+                   "l2": "inputs larger than L2 (KV cache %.1f GB)" % (
+                       2 * data["k"].numel() * data["k"].element_size() / 1e9)},
+        "sets": {"rows_min": int(sizes.min()), "rows_mean": round(float(sizes.mean()), 1),
+                 "rows_max": int(sizes.max())},
+        "hbm": {"kernel_bytes_per_step": kbytes, "kernel_gbs": round(gbs, 1),
+                "frac_of_measured_peak": round(gbs / peak, 4)},
+        "clocks": clk.summary(),
+    }
+    ctx.close()
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
     if args.serving:
         return run_serving(args)
+    if args.selection != "topk":
+        return run_rule(args)
     return run_lyc(args)
 
 

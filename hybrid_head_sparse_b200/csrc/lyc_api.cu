@@ -46,7 +46,6 @@ int topk_max_clusters(int cl, size_t smem);
 cudaError_t copy_sets_launch(const CopySetsParams* p, cudaStream_t stream);
 cudaError_t append_rows_launch(const AppendParams* p, cudaStream_t stream);
 cudaError_t validate_sets_launch(const ValidateSetsParams* p, cudaStream_t stream);
-cudaError_t block_scores_launch(const BlockScoreParams* p, int sms, cudaStream_t stream);
 }  // namespace lyc
 
 using namespace lyc;
@@ -73,8 +72,6 @@ struct LayerPlan {
   int64_t pool_tiles = 0, tiles = 0;  // tiles in the pool, in the whole layer
   int topk_cl = 16;          // cluster size of the selection launch
   int topk_n = 0;            // keys of the longest selection task
-  size_t off_btasks = 0;     // block selection: the block-score tasks (one per selection task)
-  int bmax = 0;              // block selection: blocks of the longest task
 };
 
 struct Plan {
@@ -150,11 +147,8 @@ struct lyc_ctx {
   bool timing = false;
   unsigned long long* timeline = nullptr;  // caller's buffer, or NULL
   int timeline_cap = 0;
-  // the selection rule of the steps (lyc_set_selection); block selection's
-  // score rows, [L][B][Hs][bstride]
+  // the selection rule of the steps (lyc_set_selection)
   lyc_selection sel{};
-  float* bkeys = nullptr;
-  int64_t bstride = 0;
   // plans, most recent first
   std::list<std::pair<std::string, std::unique_ptr<Plan>>> plans;
   // timing pool
@@ -440,7 +434,6 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const KvVie
     std::vector<Piece> pieces;
     std::vector<int32_t> cta;
     std::vector<TopkTask> tasks;
-    std::vector<BlockTask> btasks;  // block selection: one per task
     int topk_n = 0;
     std::vector<const int32_t*> trace_src;
     std::vector<int2> combine;  // bf16: (segment, output) left to the next launch
@@ -677,13 +670,7 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const KvVie
         tk.n = static_cast<int32_t>(kv.n[b]);
         tk.k = select_cap(kv.n[b]);
         if (sel.rule == LYC_RULE_BLOCK_TOPK) {
-          // the selection runs over the element's block scores
-          BlockTask bk{};
-          bk.keys = tk.keys;
-          bk.scores = ctx->bkeys + ((static_cast<int64_t>(l) * B + b) * Hs + s) * ctx->bstride;
-          bk.n = tk.n;
-          H.btasks.push_back(bk);
-          tk.keys = bk.scores;
+          // the selection runs over the element's blocks (scored from its keys)
           tk.rows = tk.n;
           tk.n = static_cast<int32_t>((kv.n[b] + E - 1) / E);
         }
@@ -725,8 +712,6 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const KvVie
     lp.off_cta = take(H.cta.size() * sizeof(int32_t));
     lp.off_tasks = take(std::max<size_t>(1, H.tasks.size()) * sizeof(TopkTask));
     lp.topk_n = H.topk_n;
-    lp.off_btasks = take(std::max<size_t>(1, H.btasks.size()) * sizeof(BlockTask));
-    lp.bmax = H.btasks.empty() ? 0 : H.topk_n;
     lp.off_trace_src = take(H.trace_src.size() * sizeof(void*));
     lp.ncombine = static_cast<int>(H.combine.size());
     lp.off_combine = take(std::max<size_t>(1, H.combine.size()) * sizeof(int2));
@@ -750,8 +735,6 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const KvVie
     memcpy(host.data() + lp.off_cta, H.cta.data(), H.cta.size() * sizeof(int32_t));
     if (!H.tasks.empty())
       memcpy(host.data() + lp.off_tasks, H.tasks.data(), H.tasks.size() * sizeof(TopkTask));
-    if (!H.btasks.empty())
-      memcpy(host.data() + lp.off_btasks, H.btasks.data(), H.btasks.size() * sizeof(BlockTask));
     memcpy(host.data() + lp.off_trace_src, H.trace_src.data(), H.trace_src.size() * sizeof(void*));
     if (!H.combine.empty())
       memcpy(host.data() + lp.off_combine, H.combine.data(), H.combine.size() * sizeof(int2));
@@ -928,16 +911,6 @@ lyc_status enqueue_step(lyc_ctx* ctx, Plan* plan, cudaStream_t stream, int set, 
     if ((st = record_event(ctx, plan, set, ev++, stream, capturing)) != LYC_OK) return st;
     plan->kernel_kind.push_back(0);
     plan->kernel_layer.push_back(l);
-    if (lp.ntasks > 0 && lp.bmax > 0) {
-      // block selection: every task's block scores first
-      BlockScoreParams bp{reinterpret_cast<const BlockTask*>(plan->dev + lp.off_btasks), lp.ntasks,
-                          plan->sel.block, lp.bmax};
-      if ((st = record_event(ctx, plan, set, ev++, stream, capturing)) != LYC_OK) return st;
-      LYC_CUDA(block_scores_launch(&bp, ctx->sms, stream), "block-score launch");
-      if ((st = record_event(ctx, plan, set, ev++, stream, capturing)) != LYC_OK) return st;
-      plan->kernel_kind.push_back(2);
-      plan->kernel_layer.push_back(l);
-    }
     if (lp.ntasks > 0) {
       TopkParams tp{};
       tp.tasks = reinterpret_cast<const TopkTask*>(plan->dev + lp.off_tasks);
@@ -1317,7 +1290,7 @@ void lyc_destroy(lyc_ctx* ctx) {
   for (cudaEvent_t ev : ctx->events) cudaEventDestroy(ev);
   void* bufs[] = {ctx->status, ctx->keys, ctx->flags, ctx->sbuf, ctx->part_o, ctx->part_ml,
                   ctx->wpart_o, ctx->wpart_ml, ctx->counters, ctx->q_dev, ctx->out_dev,
-                  ctx->S_dev, ctx->bkeys};
+                  ctx->S_dev};
   for (void* b : bufs)
     if (b) cudaFree(b);
   timed_steps().erase(ctx);
@@ -1511,25 +1484,9 @@ lyc_status lyc_set_selection(lyc_ctx* ctx, const lyc_selection* sel) {
   if (s.rule == LYC_RULE_THRESHOLD) c.tau = s.tau;
   DeviceGuard guard(ctx->cfg.device);
   if (!guard.ok) return fail(ctx, LYC_ERR_CUDA, "cudaSetDevice failed");
-  // the cached plans hold the old rule's records (and score rows)
+  // the cached plans hold the old rule's records
   for (auto& kv : ctx->plans) free_plan(kv.second.get());
   ctx->plans.clear();
-  if (ctx->bkeys) {
-    LYC_CUDA(cudaFree(ctx->bkeys), "cudaFree(block scores)");
-    ctx->bkeys = nullptr;
-    ctx->bstride = 0;
-  }
-  if (c.rule == LYC_RULE_BLOCK_TOPK) {
-    const lyc_config& cf = ctx->cfg;
-    ctx->bstride = round_up((ctx->nstride + c.block - 1) / c.block, 4);
-    const size_t bytes = static_cast<size_t>(cf.num_layers) * cf.batch * ctx->Hs * ctx->bstride * sizeof(float);
-    if (cudaMalloc(&ctx->bkeys, bytes) != cudaSuccess) {
-      cudaGetLastError();
-      ctx->bkeys = nullptr;
-      ctx->bstride = 0;
-      return fail(ctx, LYC_ERR_OOM, "block-score rows");
-    }
-  }
   ctx->sel = c;
   return LYC_OK;
 }
@@ -1551,8 +1508,7 @@ lyc_status lyc_set_timing(lyc_ctx* ctx, int mode) {
   if (!ctx || (mode != LYC_TIMING_OFF && mode != LYC_TIMING_ON)) return LYC_ERR_INVALID_ARG;
   DeviceGuard guard(ctx->cfg.device);
   if (mode == LYC_TIMING_ON && ctx->events.empty()) {
-    // attention, block scores, selection per layer, and the last layer's combine launch
-    ctx->events_per_set = 6 * ctx->cfg.num_layers + 2;
+    ctx->events_per_set = 4 * ctx->cfg.num_layers + 2;  // + the last layer's combine launch
     const size_t total = static_cast<size_t>(timing_sets()) * ctx->events_per_set;
     ctx->events.resize(total, nullptr);
     for (size_t i = 0; i < total; ++i)

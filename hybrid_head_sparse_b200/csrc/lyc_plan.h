@@ -136,9 +136,10 @@ struct TopkTask {
   int32_t* S;         // the launch's k outputs
   uint32_t* done;     // NULL, or {arrival counter, ready flag}: the last CTA of the task
                       // to finish resets the counter and sets the flag to epoch + 1
-  int32_t n;          // keys of this task (a batch element's rows); 0: the launch's n
+  int32_t n;          // keys of this task (a batch element's rows; its blocks with expand > 1);
+                      // 0: the launch's n
   int32_t k;          // at most this many keys are selected; 0: the launch's k
-  int32_t rows;       // with expand > 1: the element's rows (expanded rows past it are -1)
+  int32_t rows;       // with expand > 1: the element's rows (the key row's length)
   int32_t pad_;
 };
 
@@ -163,24 +164,10 @@ struct TopkParams {
   int32_t layer;
   int32_t n, k;           // k: entries of each output set
   int32_t size_rule;      // TopkSizeRule
-  int32_t expand;         // > 1: key j stands for rows j*expand .. j*expand + expand - 1 (block
-                          // selection); the output lists those rows
+  int32_t expand;         // > 1: block selection: the task's keys are rows, key j of the selection
+                          // is the block of rows j*expand .. j*expand + expand - 1 (scored
+                          // log(sum exp(key))), and the output lists the selected blocks' rows
   double size_x;          // p (top-p) or tau (threshold)
-};
-
-// block_scores_kernel: per task, the score of every block of `block` rows of
-// a key row: log(sum over the block's rows of exp(key)), computed as
-// max + log(sum exp(key - max)) (ordering blocks by it orders them by their
-// summed probability)
-struct BlockTask {
-  const float* keys;  // the task's n key rows
-  float* scores;      // ceil(n / block) scores
-  int32_t n;
-  int32_t pad_;
-};
-struct BlockScoreParams {
-  const BlockTask* tasks;
-  int32_t ntasks, block, max_blocks;
 };
 
 // Timeline tags: kind << 32 | layer << 16 | CTA

@@ -1,13 +1,9 @@
 // misc_kernels.cu -- small helpers of the step: gathering each slot's current
 // set into the caller's contiguous [B][Hs][k] layout, and checking inherited
-// sets handed in by the caller, writing the current token's K/V rows, and
-// the block scores of block selection.
+// sets handed in by the caller, and writing the current token's K/V rows.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include <algorithm>
-
-#include "lyc_device.cuh"
 #include "lyc_plan.h"
 
 namespace lyc {
@@ -52,48 +48,6 @@ __global__ void validate_sets_kernel(const ValidateSetsParams p) {
     }
   }
   if (bad) atomicOr(p.status, kStatusBadIndex);
-}
-
-// One warp per block of rows of one task: the block's log-sum-exp of the keys
-// (max + log(sum exp(key - max)); expf and logf are CUDA's).
-__global__ void block_scores_kernel(const BlockScoreParams p) {
-  pdl_wait();  // the keys are the previous launch's output
-  pdl_launch_dependents();
-  const int warps = blockDim.x / 32;
-  const int lane = threadIdx.x & 31;
-  const int64_t gw = static_cast<int64_t>(blockIdx.x) * warps + (threadIdx.x >> 5);
-  const int64_t total = static_cast<int64_t>(p.ntasks) * p.max_blocks;
-  for (int64_t w = gw; w < total; w += static_cast<int64_t>(gridDim.x) * warps) {
-    const BlockTask t = p.tasks[w / p.max_blocks];
-    const int j = static_cast<int>(w % p.max_blocks);
-    const int64_t r0 = static_cast<int64_t>(j) * p.block;
-    if (r0 >= t.n) continue;
-    const int64_t r1 = min(static_cast<int64_t>(t.n), r0 + p.block);
-    float m = -INFINITY;
-    for (int64_t r = r0 + lane; r < r1; r += 32) m = fmaxf(m, t.keys[r]);
-#pragma unroll
-    for (int s2 = 16; s2 >= 1; s2 >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, s2));
-    float z = 0.f;
-    for (int64_t r = r0 + lane; r < r1; r += 32) z += expf(t.keys[r] - m);
-#pragma unroll
-    for (int s2 = 16; s2 >= 1; s2 >>= 1) z += __shfl_xor_sync(0xffffffffu, z, s2);
-    if (lane == 0) t.scores[j] = m + logf(z);
-  }
-}
-
-cudaError_t block_scores_launch(const BlockScoreParams* p, int sms, cudaStream_t stream) {
-  const int64_t warps = static_cast<int64_t>(p->ntasks) * p->max_blocks;
-  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>((warps + 7) / 8, 8ll * sms)));
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid, 1, 1);
-  cfg.blockDim = dim3(256, 1, 1);
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, block_scores_kernel, *p);
 }
 
 // One block per (l, b, g): 16-byte chunks of the K row, then of the V row.

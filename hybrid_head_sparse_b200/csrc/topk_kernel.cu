@@ -36,10 +36,12 @@
 //    the key value at which the running mass, larger keys first, reaches
 //    T = ceil(p * sum W): a radix descent on the same digits as the
 //    selection, with per-digit counts and masses pushed into every CTA
-//    (one more cluster barrier per digit), then how many of the keys equal
-//    to that value it takes;
-//  * block selection: the keys are block scores (block_scores_kernel) and
-//    each selected block is written out as its rows.
+//    (one more cluster barrier per digit; lanes of a warp that share a bin
+//    add once), then how many of the keys equal to that value it takes;
+//  * block selection: each CTA scores the blocks of its chunk from the key
+//    rows as it loads them (log(sum exp(key)) over the block's rows, which
+//    orders blocks by their summed probability), selects among the blocks,
+//    and writes each selected block out as its rows.
 #include <cooperative_groups.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -68,6 +70,18 @@ __device__ __forceinline__ float key_from_order(uint32_t u) {
 // round(2^40 exp(x - M)), at most 2^40.
 __device__ __forceinline__ unsigned long long key_weight(uint32_t u, float M) {
   return __float2ull_rn(expf(key_from_order(u) - M) * 1099511627776.0f);
+}
+
+__device__ __forceinline__ float warp_max_f32(float v) {
+#pragma unroll
+  for (int s = 16; s >= 1; s >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, s));
+  return v;
+}
+
+__device__ __forceinline__ float warp_sum_f32(float v) {
+#pragma unroll
+  for (int s = 16; s >= 1; s >>= 1) v += __shfl_xor_sync(0xffffffffu, v, s);
+  return v;
 }
 
 __device__ __forceinline__ unsigned long long warp_sum_u64(unsigned long long v) {
@@ -276,7 +290,9 @@ __device__ __forceinline__ void topk_signal_done(const TopkParams& p, const Topk
   }
 }
 
-template <int CL>
+// VAR: a size rule or block expansion may be in use (an instantiation of its
+// own, so that the fixed-k selection carries none of their code)
+template <int CL, bool VAR>
 __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster_kernel(const TopkParams p) {
   cg::cluster_group cluster = cg::this_cluster();
   constexpr int CAP = kTopkCandCap;   // gathered candidates (all CTAs together)
@@ -288,9 +304,9 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster_kernel(const Top
   const int n = task.n > 0 ? task.n : p.n;
   const int k = p.k;                                 // entries of the output set
   const int kcap = task.k > 0 ? task.k : k;          // keys selected at most
-  const int E = p.expand > 1 ? p.expand : 1;         // rows per selected key
+  const int E = (VAR && p.expand > 1) ? p.expand : 1;  // rows per selected key
   const int rows = task.rows > 0 ? task.rows : n * E;
-  const int rule = p.size_rule;
+  const int rule = VAR ? p.size_rule : static_cast<int>(kSizeFixed);
   int keff = kcap < n ? kcap : n;
   const int chunk = (((n + CL - 1) / CL) + 3) & ~3;
   const int lo = rank * chunk;
@@ -392,7 +408,26 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster_kernel(const Top
 
   // ---- the chunk, encoded, into shared memory, and its top-digit histogram
   uint32_t umax = 0u;  // size rules: the largest encoded key of this thread
-  {
+  if (VAR && E > 1) {
+    // block selection: the chunk's keys are block scores, log(sum exp(key))
+    // over the block's rows (max + log(sum exp(key - max))), one warp per block
+    for (int x = warp; x < cnt; x += kTopkWarps) {
+      const int64_t r0 = static_cast<int64_t>(lo + x) * E;
+      const int64_t r1 = min(static_cast<int64_t>(rows), r0 + E);
+      float m = -INFINITY;
+      for (int64_t r = r0 + lane; r < r1; r += 32) m = fmaxf(m, task.keys[r]);
+      m = warp_max_f32(m);
+      float z = 0.f;
+      for (int64_t r = r0 + lane; r < r1; r += 32) z += expf(task.keys[r] - m);
+      z = warp_sum_f32(z);
+      if (lane == 0) {
+        const uint32_t u = order_key(m + logf(z));
+        us[x] = u;
+        atomicAdd(&loc[u >> kKeyDigitShift], 1u);
+        umax = max(umax, u);
+      }
+    }
+  } else {
     const float* src = task.keys + lo;
     const bool vec = (reinterpret_cast<uintptr_t>(src) & 15u) == 0;
     for (int base = wlo; base < whi; base += 128) {
@@ -413,7 +448,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster_kernel(const Top
       for (int e = 0; e < 4; ++e)
         if (x0 + e < whi) {
           atomicAdd(&loc[u[e] >> kKeyDigitShift], 1u);
-          umax = max(umax, u[e]);
+          if (VAR) umax = max(umax, u[e]);
         }
     }
   }
@@ -424,15 +459,27 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster_kernel(const Top
   __syncthreads();
   cluster.sync();  // (1) every CTA's totals are zero and its histogram complete
 
-  // ---- size rules: the cluster's largest key, then threshold's count or
-  // top-p's digit-0 masses
-  float M = 0.f;
+  // ---- top digit: add the non-zero local bins into every CTA's totals (and,
+  // with a size rule, this CTA's largest key into every CTA)
+  if (rule != kSizeFixed && tid < CL)
+    cluster.map_shared_rank(vx, tid)[rank] = static_cast<uint32_t>(res64[5]);
+  {
+    uint2* nz = cand;  // (bin, count) of the non-zero local bins; free until the gather
+    const uint32_t nnz = compact_nonzero(loc, nz, scratch, tid, lane, warp);
+    for (uint32_t x = tid; x < nnz * CL; x += kTopkThreads) {
+      const uint2 e = nz[x / CL];
+      atomicAdd(cluster.map_shared_rank(tot, static_cast<int>(x % CL)) + e.x, e.y);
+    }
+  }
+  cluster.sync();  // (2)
+
+  // ---- size rules: how many keys to select
   if (rule != kSizeFixed) {
-    if (tid < CL) cluster.map_shared_rank(vx, tid)[rank] = static_cast<uint32_t>(res64[5]);
-    cluster.sync();
     uint32_t um = 0u;
     for (int r = 0; r < CL; ++r) um = max(um, vx[r]);
-    M = key_from_order(um);
+    const float M = key_from_order(um);  // the cluster's largest key
+    // every pass below walks the chunk in steps of the CTA's width, so that
+    // all lanes of a warp take part in each step's warp-wide operations
     if (rule == kSizeThreshold) {
       unsigned long long sw = 0ull;
       for (int x = tid; x < cnt; x += kTopkThreads) sw += key_weight(us[x], M);
@@ -457,99 +504,90 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster_kernel(const Top
       m = max(m, 1u);
       keff = min(keff, static_cast<int>(m));
     } else {
-      for (int x = tid; x < cnt; x += kTopkThreads) {
-        const uint32_t u = us[x];
-        atomicAdd(&lmass[u >> kKeyDigitShift], key_weight(u, M));
-      }
-      __syncthreads();
-      for (int x = tid; x < CL * kKeyBins; x += kTopkThreads) {
-        const int b = x % kKeyBins, r = x / kKeyBins;
-        const unsigned long long w = lmass[b];
-        if (w) atomicAdd(cluster.map_shared_rank(mt0, r) + b, w);
-      }
-      __syncthreads();  // the local masses are read before `cand` is reused below
-    }
-  }
-
-  // ---- top digit: add the non-zero local bins into every CTA's totals
-  {
-    uint2* nz = cand;  // (bin, count) of the non-zero local bins; free until the gather
-    const uint32_t nnz = compact_nonzero(loc, nz, scratch, tid, lane, warp);
-    for (uint32_t x = tid; x < nnz * CL; x += kTopkThreads) {
-      const uint2 e = nz[x / CL];
-      atomicAdd(cluster.map_shared_rank(tot, static_cast<int>(x % CL)) + e.x, e.y);
-    }
-  }
-  cluster.sync();  // (2)
-  if (rule == kSizeTopP) {
-    // the mass to reach, and a radix descent to the key value that reaches it
-    unsigned long long tm = 0ull;
-    for (int b = tid; b < kKeyBins; b += kTopkThreads) tm += mt0[b];
-    tm = warp_sum_u64(tm);
-    if (lane == 0) scr64[warp] = tm;
-    __syncthreads();
-    unsigned long long total = 0ull;
-    for (int w2 = 0; w2 < kTopkWarps; ++w2) total += scr64[w2];
-    __syncthreads();
-    const double tg = ceil(p.size_x * static_cast<double>(total));
-    unsigned long long target =
-        tg >= static_cast<double>(total) ? total : (tg < 1.0 ? 1ull : static_cast<unsigned long long>(tg));
-    uint32_t dg, ca;
-    unsigned long long ma;
-    find_digit_mass<kKeyBins>(mt0, tot, target, scr64, scratch, res64, tid, lane, warp, &dg, &ca, &ma);
-    uint32_t m_above = ca;
-    target -= ma;
-    uint32_t prefix = dg << kKeyDigitShift, pmask = 0xffe00000u;
-    unsigned long long* mt2 = mt0;  // digit-0 totals are read: digit 2 reuses them
-    for (int b = tid; b < kKeyBins; b += kTopkThreads) mt2[b] = 0ull;
-#pragma unroll
-    for (int pass = 1; pass <= 2; ++pass) {
-      const int sh = pass == 1 ? 10 : 0;
-      const uint32_t dmask = pass == 1 ? 0x7ffu : 0x3ffu;
-      unsigned long long* mt = pass == 1 ? mt1 : mt2;
-      uint32_t* ct = pass == 1 ? ct1 : ct2;
-      for (int b = tid; b < kKeyBins; b += kTopkThreads) {
-        loc[b] = 0u;
-        lmass[b] = 0ull;
-      }
-      __syncthreads();
-      for (int x = tid; x < cnt; x += kTopkThreads) {
-        const uint32_t u = us[x];
-        if ((u & pmask) == prefix) {
-          const uint32_t d = (u >> sh) & dmask;
-          atomicAdd(&loc[d], 1u);
-          atomicAdd(&lmass[d], key_weight(u, M));
+      // top-p: a radix descent on the selection's digits (11, 11, 10 bits) to
+      // the key value at which the running mass, larger keys first, reaches
+      // T = ceil(p * total mass); per digit, local (count, mass) histograms
+      // (warp-aggregated adds) pushed into every CTA's totals
+      unsigned long long* mt2 = mt0;  // digit 2 reuses the digit-0 totals once read
+      uint32_t prefix = 0u, pmask = 0u, m_above = 0u;
+      unsigned long long target = 0ull;
+#pragma unroll 1
+      for (int pass = 0; pass < 3; ++pass) {
+        const int sh = pass == 0 ? kKeyDigitShift : (pass == 1 ? 10 : 0);
+        const uint32_t dmask = pass == 2 ? 0x3ffu : 0x7ffu;
+        const int nbins = pass == 2 ? kKeyBins / 2 : kKeyBins;
+        unsigned long long* mt = pass == 0 ? mt0 : (pass == 1 ? mt1 : mt2);
+        uint32_t* ct = pass == 1 ? ct1 : ct2;  // (digit 0 counts are `tot`)
+        for (int b = tid; b < kKeyBins; b += kTopkThreads) {
+          loc[b] = 0u;
+          lmass[b] = 0ull;
         }
-      }
-      __syncthreads();
-      const int nbins = pass == 1 ? kKeyBins : kKeyBins / 2;
-      for (int x = tid; x < CL * nbins; x += kTopkThreads) {
-        const int b = x % nbins, r = x / nbins;
-        const uint32_t c = loc[b];
-        if (c) {
-          atomicAdd(cluster.map_shared_rank(ct, r) + b, c);
-          const unsigned long long w = lmass[b];
-          if (w) atomicAdd(cluster.map_shared_rank(mt, r) + b, w);
+        __syncthreads();
+        for (int x0 = 0; x0 < cnt; x0 += kTopkThreads) {
+          const int x = x0 + tid;
+          const uint32_t u = x < cnt ? us[x] : 0u;
+          const bool on = x < cnt && (u & pmask) == prefix;
+          const unsigned act = __ballot_sync(FULL, on);
+          if (on) {
+            const uint32_t d = (u >> sh) & dmask;
+            const unsigned grp = __match_any_sync(act, d);
+            const unsigned long long w = key_weight(u, M);  // <= 2^40: two 20-bit halves
+            const uint32_t hi = __reduce_add_sync(grp, static_cast<uint32_t>(w >> 20));
+            const uint32_t lw = __reduce_add_sync(grp, static_cast<uint32_t>(w & 0xfffffu));
+            if (lane == __ffs(grp) - 1) {
+              atomicAdd(&loc[d], static_cast<uint32_t>(__popc(grp)));
+              atomicAdd(&lmass[d], (static_cast<unsigned long long>(hi) << 20) + lw);
+            }
+          }
         }
+        __syncthreads();
+        for (int x = tid; x < CL * nbins; x += kTopkThreads) {
+          const int b = x % nbins, r = x / nbins;
+          const uint32_t c = loc[b];
+          if (c) {
+            if (pass > 0) atomicAdd(cluster.map_shared_rank(ct, r) + b, c);
+            const unsigned long long w = lmass[b];
+            if (w) atomicAdd(cluster.map_shared_rank(mt, r) + b, w);
+          }
+        }
+        cluster.sync();
+        if (pass == 0) {  // the mass to reach
+          unsigned long long tm = 0ull;
+          for (int b = tid; b < kKeyBins; b += kTopkThreads) tm += mt0[b];
+          tm = warp_sum_u64(tm);
+          if (lane == 0) scr64[warp] = tm;
+          __syncthreads();
+          unsigned long long total = 0ull;
+          for (int w2 = 0; w2 < kTopkWarps; ++w2) total += scr64[w2];
+          __syncthreads();
+          const double tg = ceil(p.size_x * static_cast<double>(total));
+          target = tg >= static_cast<double>(total)
+                       ? total
+                       : (tg < 1.0 ? 1ull : static_cast<unsigned long long>(tg));
+        }
+        uint32_t dg, ca;
+        unsigned long long ma;
+        if (pass == 2)
+          find_digit_mass<kKeyBins / 2>(mt, ct, target, scr64, scratch, res64, tid, lane, warp, &dg,
+                                        &ca, &ma);
+        else
+          find_digit_mass<kKeyBins>(mt, pass == 0 ? tot : ct, target, scr64, scratch, res64, tid,
+                                    lane, warp, &dg, &ca, &ma);
+        m_above += ca;
+        target -= ma;
+        prefix |= dg << sh;
+        pmask |= dmask << sh;
+        if (pass == 0)  // digit-0 totals are read: digit 2 reuses them
+          for (int b = tid; b < kKeyBins; b += kTopkThreads) mt2[b] = 0ull;
       }
-      cluster.sync();
-      if (pass == 1)
-        find_digit_mass<kKeyBins>(mt, ct, target, scr64, scratch, res64, tid, lane, warp, &dg, &ca, &ma);
-      else
-        find_digit_mass<kKeyBins / 2>(mt, ct, target, scr64, scratch, res64, tid, lane, warp, &dg, &ca,
-                                      &ma);
-      m_above += ca;
-      target -= ma;
-      prefix |= dg << sh;
-      pmask |= dmask << sh;
+      // `prefix` is now the key value that reaches the mass: its keys all
+      // have the same weight; take as many of them as the rest of the mass needs
+      const uint32_t cv = ct2[prefix & 0x3ffu];
+      const unsigned long long wv = mt2[prefix & 0x3ffu] / (cv ? cv : 1u);
+      unsigned long long r = wv ? (target + wv - 1ull) / wv : cv;
+      r = r < 1ull ? 1ull : (r > cv ? cv : r);
+      keff = min(keff, static_cast<int>(m_above + static_cast<uint32_t>(r)));
     }
-    // `prefix` is now the key value that reaches the mass: its keys all have
-    // the same weight; take as many of them as the rest of the mass needs
-    const uint32_t cv = ct2[prefix & 0x3ffu];
-    const unsigned long long wv = mt2[prefix & 0x3ffu] / (cv ? cv : 1u);
-    unsigned long long r = wv ? (target + wv - 1ull) / wv : cv;
-    r = r < 1ull ? 1ull : (r > cv ? cv : r);
-    keff = min(keff, static_cast<int>(m_above + static_cast<uint32_t>(r)));
     __syncthreads();  // every read of `sel` precedes the selection's writes to it
   }
   if (rule != kSizeFixed && keff == n) {
@@ -811,17 +849,21 @@ static size_t topk_smem_bytes(int cl, int n) {
 template <int CL>
 static cudaError_t topk_run(const TopkParams* p, int ntasks, cudaStream_t stream, bool configure_only,
                             size_t max_smem) {
-  auto kern = topk_cluster_kernel<CL>;
   if (configure_only) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(max_smem));
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
-                             cudaSharedmemCarveoutMaxShared);
-    if (e != cudaSuccess) return e;
-    if (CL > 8) e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-    return e;
+    for (auto kern : {topk_cluster_kernel<CL, false>, topk_cluster_kernel<CL, true>}) {
+      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(max_smem));
+      if (e != cudaSuccess) return e;
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                               cudaSharedmemCarveoutMaxShared);
+      if (e != cudaSuccess) return e;
+      if (CL > 8) e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+      if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
   }
+  const bool var = p->size_rule != kSizeFixed || p->expand > 1;
+  auto kern = var ? topk_cluster_kernel<CL, true> : topk_cluster_kernel<CL, false>;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(CL, ntasks, 1);
   cfg.blockDim = dim3(kTopkThreads, 1, 1);
@@ -856,7 +898,7 @@ int topk_pick_cluster(size_t smem) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int nclusters = 0;
-    if (cudaOccupancyMaxActiveClusters(&nclusters, topk_cluster_kernel<16>, &cfg) == cudaSuccess &&
+    if (cudaOccupancyMaxActiveClusters(&nclusters, topk_cluster_kernel<16, false>, &cfg) == cudaSuccess &&
         nclusters > 0)
       return 16;
   }
@@ -880,7 +922,7 @@ static int topk_max_clusters_t(size_t smem) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, topk_cluster_kernel<CL>, &cfg) != cudaSuccess) {
+  if (cudaOccupancyMaxActiveClusters(&n, topk_cluster_kernel<CL, false>, &cfg) != cudaSuccess) {
     cudaGetLastError();
     return 0;
   }

@@ -72,6 +72,17 @@ __device__ __forceinline__ unsigned long long key_weight(uint32_t u, float M) {
   return __float2ull_rn(expf(key_from_order(u) - M) * 1099511627776.0f);
 }
 
+// 64-bit add into shared or distributed shared memory as two 32-bit atomic
+// adds, the low word's carry passed on to the high word: the exact sum once
+// every add has landed, without 64-bit atomics.
+__device__ __forceinline__ void atomic_add_u64_split(unsigned long long* a, unsigned long long v) {
+  uint32_t* w = reinterpret_cast<uint32_t*>(a);
+  const uint32_t lo = static_cast<uint32_t>(v), hi = static_cast<uint32_t>(v >> 32);
+  const uint32_t old = atomicAdd(w, lo);
+  const uint32_t up = hi + (old + lo < old ? 1u : 0u);
+  if (up) atomicAdd(w + 1, up);
+}
+
 __device__ __forceinline__ float warp_max_f32(float v) {
 #pragma unroll
   for (int s = 16; s >= 1; s >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, s));
@@ -154,15 +165,16 @@ __device__ __forceinline__ void find_digit_mass(const unsigned long long* mass, 
                                                 uint32_t* scr32, unsigned long long* res, int tid,
                                                 int lane, int warp, uint32_t* digit, uint32_t* cabove,
                                                 unsigned long long* mabove) {
-  constexpr int per = NB / kTopkThreads;
+  constexpr int per = NB >= kTopkThreads ? NB / kTopkThreads : 1;  // bins per thread
   unsigned long long m[per];
   uint32_t c[per];
   unsigned long long mm = 0ull;
   uint32_t mc = 0u;
 #pragma unroll
   for (int q = 0; q < per; ++q) {
-    m[q] = mass[tid * per + q];
-    c[q] = cntb[tid * per + q];
+    const bool in = tid * per + q < NB;
+    m[q] = in ? mass[tid * per + q] : 0ull;
+    c[q] = in ? cntb[tid * per + q] : 0u;
     mm += m[q];
     mc += c[q];
   }
@@ -340,14 +352,17 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster_kernel(const Top
   unsigned long long* scr64 = vsum + 16;               // [16]
   unsigned long long* res64 = scr64 + 16;              // [8]
   uint32_t* us = reinterpret_cast<uint32_t*>(res64 + 8);  // [chunk] encoded keys (16-byte aligned)
-  // top-p, before the selection proper: cand = local masses, digit-1 mass
-  // totals; sel = digit-0 (later digit-2) mass totals, digit-2 and digit-1
-  // count totals
-  unsigned long long* lmass = reinterpret_cast<unsigned long long*>(cand);
-  unsigned long long* mt1 = lmass + kKeyBins;
+  // top-p, before the selection proper: `cand` holds the local histograms
+  // (digit 0: three 16-bit limbs of the masses, u32 [3][2048]; digits 1-3:
+  // count and limbs, u32 [4][128]); `sel` the cluster totals (digit 0: masses,
+  // u64 [2048], its counts are `tot`; digits 1-3: masses u64 [3][128], then
+  // counts u32 [3][128])
+  constexpr int kFineBins = 128;  // digits 1-3 have 7 bits
+  uint32_t* limb0 = reinterpret_cast<uint32_t*>(cand);
+  uint32_t* fine_loc = limb0 + 3 * kKeyBins;
   unsigned long long* mt0 = reinterpret_cast<unsigned long long*>(sel);
-  uint32_t* ct2 = reinterpret_cast<uint32_t*>(mt0 + kKeyBins);
-  uint32_t* ct1 = ct2 + kKeyBins;
+  unsigned long long* mtf = mt0 + kKeyBins;
+  uint32_t* ctf = reinterpret_cast<uint32_t*>(mtf + 3 * kFineBins);
 
   // the output: selected key j at position pos (its rows with block selection)
   auto put = [&](uint32_t pos, int32_t j) {
@@ -389,6 +404,10 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster_kernel(const Top
     }
   }
   __syncthreads();
+  // size rules and blocks: this CTA has started (and zeroed what other CTAs
+  // add into); the wait below, before the first access to another CTA's
+  // shared memory, lets the largest key go out before barrier (1)
+  if (VAR) asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
   // Every pass over the chunk gives warp w the contiguous range [wlo, whi)
   // and walks it 128 keys at a time, lane l holding keys 4l .. 4l+3 of the
   // step: 16-byte shared-memory accesses without bank conflicts, and index
@@ -414,11 +433,23 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster_kernel(const Top
     for (int x = warp; x < cnt; x += kTopkWarps) {
       const int64_t r0 = static_cast<int64_t>(lo + x) * E;
       const int64_t r1 = min(static_cast<int64_t>(rows), r0 + E);
-      float m = -INFINITY;
-      for (int64_t r = r0 + lane; r < r1; r += 32) m = fmaxf(m, task.keys[r]);
-      m = warp_max_f32(m);
-      float z = 0.f;
-      for (int64_t r = r0 + lane; r < r1; r += 32) z += expf(task.keys[r] - m);
+      float m = -INFINITY, z = 0.f;
+      if (E <= 128) {  // the block's keys in registers: one read of the rows
+        float v[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int64_t r = r0 + lane + 32 * j;
+          v[j] = r < r1 ? task.keys[r] : -INFINITY;
+          m = fmaxf(m, v[j]);
+        }
+        m = warp_max_f32(m);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) z += v[j] == -INFINITY ? 0.f : expf(v[j] - m);
+      } else {
+        for (int64_t r = r0 + lane; r < r1; r += 32) m = fmaxf(m, task.keys[r]);
+        m = warp_max_f32(m);
+        for (int64_t r = r0 + lane; r < r1; r += 32) z += expf(task.keys[r] - m);
+      }
       z = warp_sum_f32(z);
       if (lane == 0) {
         const uint32_t u = order_key(m + logf(z));
@@ -454,16 +485,59 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster_kernel(const Top
   }
   if (rule != kSizeFixed) {
     umax = __reduce_max_sync(FULL, umax);
-    if (lane == 0) atomicMax(&res64[5], static_cast<unsigned long long>(umax));
+    if (lane == 0) atomicMax(reinterpret_cast<uint32_t*>(&res64[5]), umax);  // low word
   }
   __syncthreads();
+  if (VAR) {
+    asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
+    if (rule != kSizeFixed && tid < CL)
+      cluster.map_shared_rank(vx, tid)[rank] = static_cast<uint32_t>(res64[5]);
+  }
   cluster.sync();  // (1) every CTA's totals are zero and its histogram complete
 
-  // ---- top digit: add the non-zero local bins into every CTA's totals (and,
-  // with a size rule, this CTA's largest key into every CTA)
-  if (rule != kSizeFixed && tid < CL)
-    cluster.map_shared_rank(vx, tid)[rank] = static_cast<uint32_t>(res64[5]);
-  {
+  // ---- size rules, first part: the cluster's largest key M; threshold's
+  // local mass, top-p's local digit-0 masses (three 16-bit limbs per bin in
+  // 32-bit words: sums of at most 2^16 keys per CTA cannot overflow, and no
+  // add needs its result)
+  float M = 0.f;
+  if (rule != kSizeFixed) {
+    uint32_t um = 0u;
+    for (int r = 0; r < CL; ++r) um = max(um, vx[r]);
+    M = key_from_order(um);
+    if (rule == kSizeThreshold) {
+      unsigned long long sw = 0ull;
+      for (int x = tid; x < cnt; x += kTopkThreads) sw += key_weight(us[x], M);
+      sw = warp_sum_u64(sw);
+      if (lane == 0) atomic_add_u64_split(&res64[4], sw);
+    } else {
+      for (int x = tid; x < cnt; x += kTopkThreads) {
+        const uint32_t u = us[x];
+        const uint32_t d = u >> kKeyDigitShift;
+        const unsigned long long w = key_weight(u, M);
+        atomicAdd(&limb0[d], static_cast<uint32_t>(w & 0xffffu));
+        atomicAdd(&limb0[kKeyBins + d], static_cast<uint32_t>((w >> 16) & 0xffffu));
+        if (w >> 32) atomicAdd(&limb0[2 * kKeyBins + d], static_cast<uint32_t>(w >> 32));
+      }
+    }
+    __syncthreads();
+  }
+
+  // ---- top digit: add the non-zero local bins into every CTA's totals (and
+  // the size rules' local masses)
+  if (rule == kSizeTopP) {
+    for (int x = tid; x < CL * kKeyBins; x += kTopkThreads) {
+      const int b = x % kKeyBins, r = x / kKeyBins;
+      const uint32_t c = loc[b];
+      if (c) {
+        atomicAdd(cluster.map_shared_rank(tot, r) + b, c);
+        const unsigned long long w = static_cast<unsigned long long>(limb0[b]) +
+                                     (static_cast<unsigned long long>(limb0[kKeyBins + b]) << 16) +
+                                     (static_cast<unsigned long long>(limb0[2 * kKeyBins + b]) << 32);
+        if (w) atomicAdd(cluster.map_shared_rank(mt0, r) + b, w);
+      }
+    }
+  } else {
+    if (rule == kSizeThreshold && tid < CL) cluster.map_shared_rank(vsum, tid)[rank] = res64[4];
     uint2* nz = cand;  // (bin, count) of the non-zero local bins; free until the gather
     const uint32_t nnz = compact_nonzero(loc, nz, scratch, tid, lane, warp);
     for (uint32_t x = tid; x < nnz * CL; x += kTopkThreads) {
@@ -473,29 +547,20 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster_kernel(const Top
   }
   cluster.sync();  // (2)
 
-  // ---- size rules: how many keys to select
+  // ---- size rules, second part: how many keys to select
   if (rule != kSizeFixed) {
-    uint32_t um = 0u;
-    for (int r = 0; r < CL; ++r) um = max(um, vx[r]);
-    const float M = key_from_order(um);  // the cluster's largest key
-    // every pass below walks the chunk in steps of the CTA's width, so that
-    // all lanes of a warp take part in each step's warp-wide operations
     if (rule == kSizeThreshold) {
-      unsigned long long sw = 0ull;
-      for (int x = tid; x < cnt; x += kTopkThreads) sw += key_weight(us[x], M);
-      sw = warp_sum_u64(sw);
-      if (lane == 0) atomicAdd(&res64[4], sw);
-      __syncthreads();
-      if (tid < CL) cluster.map_shared_rank(vsum, tid)[rank] = res64[4];
-      cluster.sync();
       unsigned long long total = 0ull;
       for (int r = 0; r < CL; ++r) total += vsum[r];
       const double tg = ceil(p.size_x * static_cast<double>(total));
       const unsigned long long thr = tg <= 0.0 ? 0ull : static_cast<unsigned long long>(tg);
       uint32_t c = 0u;
-      for (int x = tid; x < cnt; x += kTopkThreads) c += key_weight(us[x], M) >= thr ? 1u : 0u;
+      for (int x0 = 0; x0 < cnt; x0 += kTopkThreads) {  // every lane takes part in the reduce
+        const int x = x0 + tid;
+        c += (x < cnt && key_weight(us[x], M) >= thr) ? 1u : 0u;
+      }
       c = __reduce_add_sync(FULL, c);
-      if (lane == 0) atomicAdd(&res64[6], static_cast<unsigned long long>(c));
+      if (lane == 0) atomicAdd(reinterpret_cast<uint32_t*>(&res64[6]), c);  // low word
       __syncthreads();
       if (tid < CL) cluster.map_shared_rank(vcnt, tid)[rank] = static_cast<uint32_t>(res64[6]);
       cluster.sync();
@@ -504,86 +569,77 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster_kernel(const Top
       m = max(m, 1u);
       keff = min(keff, static_cast<int>(m));
     } else {
-      // top-p: a radix descent on the selection's digits (11, 11, 10 bits) to
-      // the key value at which the running mass, larger keys first, reaches
-      // T = ceil(p * total mass); per digit, local (count, mass) histograms
-      // (warp-aggregated adds) pushed into every CTA's totals
-      unsigned long long* mt2 = mt0;  // digit 2 reuses the digit-0 totals once read
+      // top-p: a radix descent (digits of 11, 7, 7 and 7 bits) to the key
+      // value at which the running mass, larger keys first, reaches
+      // T = ceil(p * total mass); digits 1-3 as digit 0, with local counts
       uint32_t prefix = 0u, pmask = 0u, m_above = 0u;
       unsigned long long target = 0ull;
+      uint32_t dg = 0u, ca = 0u;
+      unsigned long long ma = 0ull;
+      {  // the mass to reach, and digit 0
+        unsigned long long tm = 0ull;
+        for (int b = tid; b < kKeyBins; b += kTopkThreads) tm += mt0[b];
+        tm = warp_sum_u64(tm);
+        if (lane == 0) scr64[warp] = tm;
+        __syncthreads();
+        unsigned long long total = 0ull;
+        for (int w2 = 0; w2 < kTopkWarps; ++w2) total += scr64[w2];
+        __syncthreads();
+        const double tg = ceil(p.size_x * static_cast<double>(total));
+        target = tg >= static_cast<double>(total)
+                     ? total
+                     : (tg < 1.0 ? 1ull : static_cast<unsigned long long>(tg));
+        find_digit_mass<kKeyBins>(mt0, tot, target, scr64, scratch, res64, tid, lane, warp, &dg, &ca,
+                                  &ma);
+        m_above += ca;
+        target -= ma;
+        prefix = dg << kKeyDigitShift;
+        pmask = 0xffe00000u;
+      }
 #pragma unroll 1
-      for (int pass = 0; pass < 3; ++pass) {
-        const int sh = pass == 0 ? kKeyDigitShift : (pass == 1 ? 10 : 0);
-        const uint32_t dmask = pass == 2 ? 0x3ffu : 0x7ffu;
-        const int nbins = pass == 2 ? kKeyBins / 2 : kKeyBins;
-        unsigned long long* mt = pass == 0 ? mt0 : (pass == 1 ? mt1 : mt2);
-        uint32_t* ct = pass == 1 ? ct1 : ct2;  // (digit 0 counts are `tot`)
-        for (int b = tid; b < kKeyBins; b += kTopkThreads) {
-          loc[b] = 0u;
-          lmass[b] = 0ull;
+      for (int pass = 1; pass < 4; ++pass) {
+        const int sh = 21 - 7 * pass;
+        const uint32_t dmask = kFineBins - 1;
+        uint32_t* lc = fine_loc;              // local counts
+        uint32_t* lm = fine_loc + kFineBins;  // local limbs [3][kFineBins]
+        unsigned long long* mt = mtf + (pass - 1) * kFineBins;
+        uint32_t* ct = ctf + (pass - 1) * kFineBins;
+        for (int b = tid; b < 4 * kFineBins; b += kTopkThreads) fine_loc[b] = 0u;
+        __syncthreads();
+        for (int x = tid; x < cnt; x += kTopkThreads) {
+          const uint32_t u = us[x];
+          if ((u & pmask) != prefix) continue;
+          const uint32_t d = (u >> sh) & dmask;
+          const unsigned long long w = key_weight(u, M);
+          atomicAdd(&lc[d], 1u);
+          atomicAdd(&lm[d], static_cast<uint32_t>(w & 0xffffu));
+          atomicAdd(&lm[kFineBins + d], static_cast<uint32_t>((w >> 16) & 0xffffu));
+          if (w >> 32) atomicAdd(&lm[2 * kFineBins + d], static_cast<uint32_t>(w >> 32));
         }
         __syncthreads();
-        for (int x0 = 0; x0 < cnt; x0 += kTopkThreads) {
-          const int x = x0 + tid;
-          const uint32_t u = x < cnt ? us[x] : 0u;
-          const bool on = x < cnt && (u & pmask) == prefix;
-          const unsigned act = __ballot_sync(FULL, on);
-          if (on) {
-            const uint32_t d = (u >> sh) & dmask;
-            const unsigned grp = __match_any_sync(act, d);
-            const unsigned long long w = key_weight(u, M);  // <= 2^40: two 20-bit halves
-            const uint32_t hi = __reduce_add_sync(grp, static_cast<uint32_t>(w >> 20));
-            const uint32_t lw = __reduce_add_sync(grp, static_cast<uint32_t>(w & 0xfffffu));
-            if (lane == __ffs(grp) - 1) {
-              atomicAdd(&loc[d], static_cast<uint32_t>(__popc(grp)));
-              atomicAdd(&lmass[d], (static_cast<unsigned long long>(hi) << 20) + lw);
-            }
-          }
-        }
-        __syncthreads();
-        for (int x = tid; x < CL * nbins; x += kTopkThreads) {
-          const int b = x % nbins, r = x / nbins;
-          const uint32_t c = loc[b];
+        for (int x = tid; x < CL * kFineBins; x += kTopkThreads) {
+          const int b = x % kFineBins, r = x / kFineBins;
+          const uint32_t c = lc[b];
           if (c) {
-            if (pass > 0) atomicAdd(cluster.map_shared_rank(ct, r) + b, c);
-            const unsigned long long w = lmass[b];
+            atomicAdd(cluster.map_shared_rank(ct, r) + b, c);
+            const unsigned long long w = static_cast<unsigned long long>(lm[b]) +
+                                         (static_cast<unsigned long long>(lm[kFineBins + b]) << 16) +
+                                         (static_cast<unsigned long long>(lm[2 * kFineBins + b]) << 32);
             if (w) atomicAdd(cluster.map_shared_rank(mt, r) + b, w);
           }
         }
         cluster.sync();
-        if (pass == 0) {  // the mass to reach
-          unsigned long long tm = 0ull;
-          for (int b = tid; b < kKeyBins; b += kTopkThreads) tm += mt0[b];
-          tm = warp_sum_u64(tm);
-          if (lane == 0) scr64[warp] = tm;
-          __syncthreads();
-          unsigned long long total = 0ull;
-          for (int w2 = 0; w2 < kTopkWarps; ++w2) total += scr64[w2];
-          __syncthreads();
-          const double tg = ceil(p.size_x * static_cast<double>(total));
-          target = tg >= static_cast<double>(total)
-                       ? total
-                       : (tg < 1.0 ? 1ull : static_cast<unsigned long long>(tg));
-        }
-        uint32_t dg, ca;
-        unsigned long long ma;
-        if (pass == 2)
-          find_digit_mass<kKeyBins / 2>(mt, ct, target, scr64, scratch, res64, tid, lane, warp, &dg,
-                                        &ca, &ma);
-        else
-          find_digit_mass<kKeyBins>(mt, pass == 0 ? tot : ct, target, scr64, scratch, res64, tid,
-                                    lane, warp, &dg, &ca, &ma);
+        find_digit_mass<kFineBins>(mt, ct, target, scr64, scratch, res64, tid, lane, warp, &dg, &ca,
+                                   &ma);
         m_above += ca;
         target -= ma;
         prefix |= dg << sh;
         pmask |= dmask << sh;
-        if (pass == 0)  // digit-0 totals are read: digit 2 reuses them
-          for (int b = tid; b < kKeyBins; b += kTopkThreads) mt2[b] = 0ull;
       }
       // `prefix` is now the key value that reaches the mass: its keys all
       // have the same weight; take as many of them as the rest of the mass needs
-      const uint32_t cv = ct2[prefix & 0x3ffu];
-      const unsigned long long wv = mt2[prefix & 0x3ffu] / (cv ? cv : 1u);
+      const uint32_t cv = ctf[2 * kFineBins + dg];
+      const unsigned long long wv = mtf[2 * kFineBins + dg] / (cv ? cv : 1u);
       unsigned long long r = wv ? (target + wv - 1ull) / wv : cv;
       r = r < 1ull ? 1ull : (r > cv ? cv : r);
       keff = min(keff, static_cast<int>(m_above + static_cast<uint32_t>(r)));

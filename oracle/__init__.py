@@ -21,7 +21,9 @@ Inference via Hybrid-Head Sparse Decoding" (paper-graph-ui summary):
 * section 4.4.1 (Figure 6, Tables 5-6), section 4.1 / Appendix F and the
   kernel section: the selection rules other than a fixed k (ratio, the
   reasoning budget as the ratio 1/2, block top-k, top-p, threshold; see
-  ``Selection`` and the readings at the top of oracle.c).
+  ``Selection`` and the readings at the top of oracle.c);
+* section 4.2.2 (Cache Correction): the dense causal attention of the T most
+  recent positions over the cache (``correction``).
 """
 from __future__ import annotations
 
@@ -130,6 +132,8 @@ class Oracle:
                                           ctypes.POINTER(OracleSelection), p, p, p, p,
                                           ctypes.c_int, ctypes.c_int, p, p, p]
         L.ora_decode_step_sel.restype = ctypes.c_int
+        L.ora_correction.argtypes = [ctypes.POINTER(OracleShape), ctypes.c_int, p, p, p, p]
+        L.ora_correction.restype = ctypes.c_int
         self.lib = L
         self.path = path
 
@@ -138,6 +142,9 @@ class Oracle:
 
     def select(self, x, k, sel=None):
         return select(x, k, sel, self)
+
+    def correction(self, *a, **kw):
+        return correction(*a, ora=self, **kw)
 
     def layer(self, *a, **kw):
         return layer(*a, ora=self, **kw)
@@ -291,3 +298,20 @@ def decode_step(st: Stack, k: int, S_in: np.ndarray | None = None, n: int | None
     if rc != 0:
         raise ValueError(f"ora_decode_step failed ({rc})")
     return out, S, tr
+
+
+def correction(st: Stack, q: np.ndarray, ora: Oracle | None = None) -> np.ndarray:
+    """Cache Correction's dense causal attention (section 4.2.2): q is
+    [L][B][Hq][T][d] in the cache's dtype (bf16 as uint16 bit patterns); query
+    t attends rows 0 .. n - T + t of st's cache.  Returns out [L][B][Hq][T][d] f64."""
+    sh = st.shape()
+    L, B, Hq, d = sh.L, sh.B, sh.Hq, sh.d
+    q = np.ascontiguousarray(q)
+    assert q.dtype == st.k.dtype and q.shape[:3] == (L, B, Hq) and q.shape[4] == d, q.shape
+    T = q.shape[3]
+    out = np.zeros((L, B, Hq, T, d), dtype=np.float64)
+    ora = ora or default()
+    rc = ora.lib.ora_correction(ctypes.byref(sh), T, _ptr(q), _ptr(st.k), _ptr(st.v), _ptr(out))
+    if rc != 0:
+        raise ValueError(f"ora_correction failed ({rc})")
+    return out

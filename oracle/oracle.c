@@ -481,3 +481,44 @@ int ora_decode_step(const ora_shape* sh, const void* q, const void* K,
                     int32_t* S, double* out, int32_t* trace) {
   return ora_decode_step_sel(sh, NULL, q, K, V, role, k, s_in, S, out, trace);
 }
+
+/* ---------------------------------------------------------------- cache correction */
+
+/*
+ * Cache Correction (section 4.2.2; the decoding setup of section 4.1 and
+ * Appendix F): after every 32 decoded tokens the T most recent positions are
+ * prefilled again with dense attention.  The attention part of that prefill,
+ * for every layer, batch element and query head: query t sits at position
+ * p = n - T + t and attends rows 0..p of the cache (causal), whose rows
+ * n - T .. n - 1 already hold the refreshed K/V of those positions.
+ *   q   : [L][B][Hq][T][d] (dtype)
+ *   out : [L][B][Hq][T][d] fp64
+ * Returns 0, or -1 on a bad argument.
+ */
+int ora_correction(const ora_shape* sh, int T, const void* q_all, const void* K, const void* V,
+                   double* out) {
+  const int L = sh->L, B = sh->B, Hq = sh->Hq, Hkv = sh->Hkv, d = sh->d;
+  const int64_t n = sh->n;
+  if (L <= 0 || B <= 0 || Hq <= 0 || Hkv <= 0 || d <= 0 || Hq % Hkv != 0 || T <= 0 || T > n)
+    return -1;
+  const int G = Hq / Hkv;
+#pragma omp parallel for collapse(3) schedule(dynamic)
+  for (int l = 0; l < L; ++l) {
+    for (int b = 0; b < B; ++b) {
+      for (int h = 0; h < Hq; ++h) {
+        const int g = h / G;
+        const int64_t kv_base = (int64_t)l * sh->s_layer + (int64_t)b * sh->s_batch +
+                                (int64_t)g * sh->s_head;
+        double* qv = (double*)malloc((size_t)d * sizeof(double));
+        for (int t = 0; t < T; ++t) {
+          const int64_t row = (((int64_t)l * B + b) * Hq + h) * T + t;
+          for (int j = 0; j < d; ++j) qv[j] = widen(q_all, sh->dtype, row * d + j);
+          const int64_t p = n - T + t;
+          attend_rows(sh, qv, K, V, kv_base, NULL, p + 1, out + row * d, NULL);
+        }
+        free(qv);
+      }
+    }
+  }
+  return 0;
+}

@@ -573,11 +573,67 @@ def pin_select_in_step(ora):
                     assert np.array_equal(tr[l, 0, h], tr[l - 1, 0, h])
 
 
+# ----------------------------------------------------------------- cache correction
+# Section 4.2.2: every 32 decoded tokens the T most recent positions are
+# prefilled again with dense attention; query t sits at position n - T + t.
+
+
+def pin_correction_textbook_causal(ora):
+    """numpy causal attention over a random cache, fp32 and bf16: query t of
+    every head attends rows 0 .. n - T + t."""
+    rng = np.random.default_rng(50)
+    for dtype, n, T in (("fp32", 23, 5), ("bf16", 40, 8), ("fp32", 6, 6)):
+        st = rand_stack(rng, L=2, B=2, Hq=4, Hkv=2, d=8, n=n, dtype=dtype)
+        qf = rng.standard_normal((2, 2, 4, T, 8))
+        q = bf16_bits(qf) if dtype == "bf16" else qf.astype(np.float32)
+        got = ora.correction(st, q)
+        Q, K, V = widen(q), widen(st.k), widen(st.v)
+        for l in range(2):
+            for b in range(2):
+                for h in range(4):
+                    g = h // 2
+                    for t in range(T):
+                        p = n - T + t
+                        o, _ = textbook_attention(Q[l, b, h, t], K[l, b, g, :p + 1], V[l, b, g, :p + 1])
+                        close(got[l, b, h, t], o, 1e-12, f"correction {dtype} l{l} b{b} h{h} t{t}")
+
+
+def pin_correction_causality(ora):
+    """Changing cache row r moves exactly the queries at positions >= r."""
+    rng = np.random.default_rng(51)
+    n, T = 30, 6
+    st = rand_stack(rng, L=1, B=1, Hq=2, Hkv=1, d=8, n=n)
+    q = rng.standard_normal((1, 1, 2, T, 8)).astype(np.float32)
+    base = ora.correction(st, q)
+    for r in (n - T, n - 3, n - 1):
+        k2, v2 = st.k.copy(), st.v.copy()
+        k2[0, 0, 0, r] += 1.0
+        v2[0, 0, 0, r] -= 2.0
+        moved = ora.correction(stack(st.q, k2, v2, st.role), q)
+        for t in range(T):
+            same = np.array_equal(moved[0, 0, :, t], base[0, 0, :, t])
+            assert same == (n - T + t < r), f"row {r} query {t}: causality broken"
+
+
+def pin_correction_last_query_is_decode(ora):
+    """The last query (position n - 1) is the decode step's dense attention
+    of a retrieval head over all n rows (Eq. 1, layer 0 all retrieval)."""
+    rng = np.random.default_rng(52)
+    n, T = 33, 4
+    st = rand_stack(rng, L=1, B=2, Hq=4, Hkv=2, d=16, n=n)
+    q = rng.standard_normal((1, 2, 4, T, 16)).astype(np.float32)
+    got = ora.correction(st, q)
+    last = stack(np.ascontiguousarray(q[:, :, :, T - 1]), st.k, st.v, st.role)
+    out, _, _, _ = ora.layer(last, 0, 4, None, all_retrieval=True)
+    close(got[0, :, :, T - 1], out, 1e-13, "last correction query vs the dense decode pass")
+
+
 ALL_PINS = [
     pin_topk_distinct, pin_topk_ties, pin_topk_bruteforce, pin_closed_form_bf16,
     pin_dense_textbook, pin_mpmath_attention, pin_sparse_eq3, pin_k_ge_n, pin_uniform_keys,
     pin_planted_key, pin_chain, pin_layer0_forced, pin_permutation, pin_linearity,
     pin_kvgroup, pin_strided_layout, pin_batch_elements_independent,
     pin_select_topk_rule_is_topk, pin_select_ratio, pin_select_topp, pin_select_threshold,
-    pin_select_block, pin_select_in_step,
+    pin_select_block, pin_select_in_step, pin_correction_textbook_causal,
+    pin_correction_causality, pin_correction_last_query_is_decode,
 ]

@@ -48,6 +48,13 @@ MUTANTS = [
     ("short last block padded to full", "i < ((int64_t)blocks[j] + 1) * bs && i < n; ++i)",
      "i < ((int64_t)blocks[j] + 1) * bs; ++i)"),
     ("rule ignored in the step", "      ora_select(x, n, k, sel, Sout);", "      ora_topk(x, n, k, Sout);"),
+    ("correction sees one row too few", "attend_rows(sh, qv, K, V, kv_base, NULL, p + 1, out + row * d, NULL);",
+     "attend_rows(sh, qv, K, V, kv_base, NULL, p, out + row * d, NULL);"),
+    ("correction without the causal mask", "const int64_t p = n - T + t;", "const int64_t p = n - 1;"),
+    ("correction positions from the front", "const int64_t p = n - T + t;\n",
+     "const int64_t p = t < n ? t : n - 1;\n"),
+    ("correction reads the wrong KV group", "const int g = h / G;\n        const int64_t kv_base",
+     "const int g = h % Hkv;\n        const int64_t kv_base"),
     ("smallest instead of largest", "if (a->x > b->x) return -1;\n  if (a->x < b->x) return 1;",
      "if (a->x < b->x) return -1;\n  if (a->x > b->x) return 1;"),
 ]

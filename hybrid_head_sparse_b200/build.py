@@ -9,8 +9,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "liblyc.so")
-SOURCES = ["attn_kernel.cu", "attn_mma_kernel.cu", "topk_kernel.cu", "misc_kernels.cu", "lyc_api.cu", "noalloc.cu", "attn_tc_kernel.cu"]
-HEADERS = ["lyc_plan.h", "lyc_device.cuh"]
+SOURCES = ["attn_kernel.cu", "attn_mma_kernel.cu", "topk_kernel.cu", "misc_kernels.cu", "lyc_api.cu", "noalloc.cu", "attn_tc_kernel.cu", "correction_kernel.cu"]
+HEADERS = ["lyc_plan.h", "lyc_device.cuh", "tc_ptx.cuh"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",
          "-Xcompiler", "-fPIC", "-I", os.path.join(ROOT, "include")]

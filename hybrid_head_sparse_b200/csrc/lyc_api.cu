@@ -46,6 +46,10 @@ int topk_max_clusters(int cl, size_t smem);
 cudaError_t copy_sets_launch(const CopySetsParams* p, cudaStream_t stream);
 cudaError_t append_rows_launch(const AppendParams* p, cudaStream_t stream);
 cudaError_t validate_sets_launch(const ValidateSetsParams* p, cudaStream_t stream);
+int correction_smem_bytes();
+cudaError_t correction_configure();
+cudaError_t correction_launch(const CorrParams* P, int grid, const WriteRowsParams* rows,
+                              cudaStream_t stream);
 }  // namespace lyc
 
 using namespace lyc;
@@ -149,6 +153,16 @@ struct lyc_ctx {
   int timeline_cap = 0;
   // the selection rule of the steps (lyc_set_selection)
   lyc_selection sel{};
+  // Cache Correction: the work pool of the last (n, T) (pieces, CTA offsets,
+  // group offsets in one device buffer) and the piece partials
+  unsigned char* corr_dev = nullptr;
+  int64_t corr_n = -1;
+  int corr_T = -1, corr_grid = 0, corr_npieces = 0;
+  size_t corr_off_cta = 0, corr_off_group = 0;
+  float* corr_part_o = nullptr;
+  float2* corr_part_ml = nullptr;
+  size_t corr_parts_cap = 0;
+  bool corr_configured = false;
   // plans, most recent first
   std::list<std::pair<std::string, std::unique_ptr<Plan>>> plans;
   // timing pool
@@ -1290,7 +1304,7 @@ void lyc_destroy(lyc_ctx* ctx) {
   for (cudaEvent_t ev : ctx->events) cudaEventDestroy(ev);
   void* bufs[] = {ctx->status, ctx->keys, ctx->flags, ctx->sbuf, ctx->part_o, ctx->part_ml,
                   ctx->wpart_o, ctx->wpart_ml, ctx->counters, ctx->q_dev, ctx->out_dev,
-                  ctx->S_dev};
+                  ctx->S_dev, ctx->corr_dev, ctx->corr_part_o, ctx->corr_part_ml};
   for (void* b : bufs)
     if (b) cudaFree(b);
   timed_steps().erase(ctx);
@@ -1406,6 +1420,140 @@ lyc_status lyc_decode_step_batch(lyc_ctx* ctx, const void* q, const lyc_kv_batch
   if (st == LYC_OK) st = check_kv_batch(ctx, kv);
   if (st != LYC_OK) return st;
   return step_impl(ctx, q, view_of(kv, ctx->cfg.batch), role_mask, k, out, S, stream_, step_flags);
+}
+
+lyc_status lyc_cache_correction(lyc_ctx* ctx, const void* q, const lyc_kv_cache* kv, int T,
+                                const void* k_new, const void* v_new, float* out, void* stream_) {
+  if (!ctx) return LYC_ERR_INVALID_ARG;
+  const lyc_config& c = ctx->cfg;
+  if (!q || !kv || !kv->k || !kv->v || !out)
+    return fail(ctx, LYC_ERR_INVALID_ARG, "NULL pointer");
+  if ((k_new == nullptr) != (v_new == nullptr))
+    return fail(ctx, LYC_ERR_INVALID_ARG, "k_new and v_new go together");
+  if (c.dtype != LYC_BF16 || c.head_dim != 128)
+    return fail(ctx, LYC_ERR_UNSUPPORTED, "Cache Correction runs on bf16 with head_dim 128");
+  const int L = c.num_layers, B = c.batch, Hq = c.num_q_heads, Hkv = c.num_kv_heads, G = ctx->G;
+  const int64_t n = kv->n;
+  if (T < 1 || n < T || n > c.max_ctx) return fail(ctx, LYC_ERR_INVALID_ARG, "need 1 <= T <= n <= max_ctx");
+  if (static_cast<int64_t>(G) * T > 128)
+    return fail(ctx, LYC_ERR_UNSUPPORTED, "G * T query rows must fit one 128-row block");
+  auto misaligned = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; };
+  if (misaligned(q) || misaligned(out) || misaligned(kv->k) || misaligned(kv->v) ||
+      (k_new && (misaligned(k_new) || misaligned(v_new))))
+    return fail(ctx, LYC_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  if (kv->s_token < c.head_dim || kv->s_token % 8 || kv->s_head % 8 || kv->s_batch % 8 || kv->s_layer % 8)
+    return fail(ctx, LYC_ERR_INVALID_ARG, "cache strides must be multiples of 8 elements, rows >= head_dim");
+  DeviceGuard guard(c.device);
+  if (!guard.ok) return fail(ctx, LYC_ERR_CUDA, "cudaSetDevice failed");
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  if (!ctx->corr_configured) {
+    LYC_CUDA(correction_configure(), "correction kernel attributes");
+    ctx->corr_configured = true;
+  }
+  // the work pool: the (l, b, g) groups' tiles cut into equal runs, one per CTA
+  if (ctx->corr_n != n || ctx->corr_T != T) {
+    const int64_t NT = (n + 127) / 128;
+    const int64_t ngroups = static_cast<int64_t>(L) * B * Hkv;
+    const int64_t TT = ngroups * NT;
+    const int grid = static_cast<int>(std::min<int64_t>(TT, ctx->sms));
+    std::vector<CorrPiece> pieces;
+    std::vector<int32_t> cta(1, 0), group_first(ngroups + 1, 0);
+    for (int cc = 0; cc < grid; ++cc) {
+      const int64_t t0 = TT * cc / grid, t1 = TT * (cc + 1) / grid;
+      for (int64_t x = t0; x < t1;) {
+        const int64_t grp = x / NT;
+        const int64_t end = std::min(t1, (grp + 1) * NT);
+        CorrPiece pc;
+        pc.g = static_cast<int32_t>(grp % Hkv);
+        pc.b = static_cast<int32_t>((grp / Hkv) % B);
+        pc.l = static_cast<int32_t>(grp / (static_cast<int64_t>(Hkv) * B));
+        pc.t0 = static_cast<int32_t>(x - grp * NT);
+        pc.t1 = static_cast<int32_t>(end - grp * NT);
+        pc.part = static_cast<int32_t>(pieces.size());
+        pieces.push_back(pc);
+        group_first[grp + 1] = static_cast<int32_t>(pieces.size());
+        x = end;
+      }
+      cta.push_back(static_cast<int32_t>(pieces.size()));
+    }
+    for (int64_t j = 1; j <= ngroups; ++j) group_first[j] = std::max(group_first[j], group_first[j - 1]);
+    size_t bytes = pieces.size() * sizeof(CorrPiece);
+    const size_t off_cta = round_up(static_cast<int64_t>(bytes), 64);
+    bytes = off_cta + cta.size() * sizeof(int32_t);
+    const size_t off_group = round_up(static_cast<int64_t>(bytes), 64);
+    bytes = off_group + group_first.size() * sizeof(int32_t);
+    std::vector<unsigned char> host(bytes, 0);
+    memcpy(host.data(), pieces.data(), pieces.size() * sizeof(CorrPiece));
+    memcpy(host.data() + off_cta, cta.data(), cta.size() * sizeof(int32_t));
+    memcpy(host.data() + off_group, group_first.data(), group_first.size() * sizeof(int32_t));
+    if (ctx->corr_dev) {
+      LYC_CUDA(cudaFree(ctx->corr_dev), "cudaFree(correction pool)");
+      ctx->corr_dev = nullptr;
+    }
+    ctx->corr_n = -1;
+    LYC_CUDA(cudaMalloc(&ctx->corr_dev, bytes), "cudaMalloc(correction pool)");
+    LYC_CUDA(cudaMemcpy(ctx->corr_dev, host.data(), bytes, cudaMemcpyHostToDevice), "upload correction pool");
+    if (pieces.size() > ctx->corr_parts_cap) {
+      if (ctx->corr_part_o) cudaFree(ctx->corr_part_o);
+      if (ctx->corr_part_ml) cudaFree(ctx->corr_part_ml);
+      ctx->corr_part_o = nullptr;
+      ctx->corr_part_ml = nullptr;
+      ctx->corr_parts_cap = 0;
+      LYC_CUDA(cudaMalloc(&ctx->corr_part_o, pieces.size() * 128 * 128 * sizeof(float)), "cudaMalloc(correction partials)");
+      LYC_CUDA(cudaMalloc(&ctx->corr_part_ml, pieces.size() * 128 * sizeof(float2)), "cudaMalloc(correction partials)");
+      ctx->corr_parts_cap = pieces.size();
+    }
+    ctx->corr_n = n;
+    ctx->corr_T = T;
+    ctx->corr_grid = grid;
+    ctx->corr_npieces = static_cast<int>(pieces.size());
+    ctx->corr_off_cta = off_cta;
+    ctx->corr_off_group = off_group;
+  }
+  CorrParams P;
+  memset(&P, 0, sizeof P);
+  const KvView w = view_of(kv, B);
+  lyc_status st = encode_cache_map(ctx, &P.tmk, kv->k, w, 128);
+  if (st == LYC_OK) st = encode_cache_map(ctx, &P.tmv, kv->v, w, 128);
+  if (st != LYC_OK) return st;
+  P.q = q;
+  P.out = out;
+  P.pieces = reinterpret_cast<const CorrPiece*>(ctx->corr_dev);
+  P.cta_begin = reinterpret_cast<const int32_t*>(ctx->corr_dev + ctx->corr_off_cta);
+  P.group_first = reinterpret_cast<const int32_t*>(ctx->corr_dev + ctx->corr_off_group);
+  P.part_o = ctx->corr_part_o;
+  P.part_ml = ctx->corr_part_ml;
+  P.status = ctx->status;
+  P.L = L;
+  P.B = B;
+  P.Hq = Hq;
+  P.Hkv = Hkv;
+  P.G = G;
+  P.T = T;
+  P.n = static_cast<int32_t>(n);
+  P.rows = G * T;
+  P.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(128.0));
+  WriteRowsParams wr{};
+  if (k_new) {
+    wr.k_new = static_cast<const unsigned char*>(k_new);
+    wr.v_new = static_cast<const unsigned char*>(v_new);
+    wr.k = static_cast<unsigned char*>(const_cast<void*>(kv->k));
+    wr.v = static_cast<unsigned char*>(const_cast<void*>(kv->v));
+    wr.s_layer = kv->s_layer;
+    wr.s_batch = kv->s_batch;
+    wr.s_head = kv->s_head;
+    wr.s_token = kv->s_token;
+    wr.L = L;
+    wr.B = B;
+    wr.Hkv = Hkv;
+    wr.T = T;
+    wr.n = static_cast<int32_t>(n);
+    wr.row_bytes = c.head_dim * 2;
+    wr.elem_bytes = 2;
+  }
+  LYC_CUDA(correction_launch(&P, ctx->corr_grid, k_new ? &wr : nullptr, stream), "correction launch");
+  ctx->last_stream = stream;
+  return LYC_OK;
 }
 
 lyc_status lyc_decode_step_host(lyc_ctx* ctx, const void* q_host, const lyc_kv_cache* kv,

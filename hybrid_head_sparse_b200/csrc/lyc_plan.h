@@ -18,6 +18,7 @@
 // writes one partial softmax state (m, l, o[d]) per output row; the last piece
 // of a segment to finish merges them (log-sum-exp) into `out`.
 #pragma once
+#include <cuda.h>
 #include <stdint.h>
 #include <string.h>
 
@@ -168,6 +169,41 @@ struct TopkParams {
                           // is the block of rows j*expand .. j*expand + expand - 1 (scored
                           // log(sum exp(key))), and the output lists the selected blocks' rows
   double size_x;          // p (top-p) or tau (threshold)
+};
+
+// Cache Correction (correction_kernel.cu): a piece is tiles [t0, t1) (128
+// rows each) of KV group (l, b, g); its partial states go to record `part`.
+struct CorrPiece {
+  int32_t l, b, g;
+  int32_t t0, t1;
+  int32_t part;
+};
+
+struct CorrParams {
+  CUtensorMap tmk;            // 5-D maps of K and V: (d, row, g, b, l), box 64 x 128 rows
+  CUtensorMap tmv;
+  const void* q;              // [L][B][Hq][T][d] bf16
+  float* out;                 // [L][B][Hq][T][d]
+  const CorrPiece* pieces;
+  const int32_t* cta_begin;   // pieces of CTA c: [cta_begin[c], cta_begin[c+1])
+  float* part_o;              // [pieces][128 rows][d], unnormalised
+  float2* part_ml;            // [pieces][128 rows]: (running max in log2 units, sum)
+  const int32_t* group_first; // combine: pieces of group j are [group_first[j], group_first[j+1])
+  uint32_t* status;
+  int32_t L, B, Hq, Hkv, G, T, n;
+  int32_t rows;               // G * T query rows per group
+  float scale_log2;           // log2(e) / sqrt(d)
+};
+
+// write_rows_kernel (Cache Correction's refreshed rows): k_new/v_new
+// [L][B][Hkv][T][d] written at rows n - T .. n - 1 of every (l, b, g)
+struct WriteRowsParams {
+  const unsigned char* k_new;
+  const unsigned char* v_new;
+  unsigned char* k;
+  unsigned char* v;
+  int64_t s_layer, s_batch, s_head, s_token;
+  int32_t L, B, Hkv, T, n, row_bytes, elem_bytes;
 };
 
 // Timeline tags: kind << 32 | layer << 16 | CTA

@@ -53,7 +53,7 @@ EXPORTED = ["lyc_create", "lyc_decode_step", "lyc_decode_step_host", "lyc_decode
             "lyc_sync_status",
             "lyc_set_s_trace", "lyc_step_bytes", "lyc_topk_f32", "lyc_set_timing",
             "lyc_kernel_times", "lyc_set_timeline", "lyc_status_string", "lyc_last_error",
-            "lyc_destroy", "lyc_sparse_attention_noalloc", "lyc_set_selection"]
+            "lyc_destroy", "lyc_sparse_attention_noalloc", "lyc_set_selection", "lyc_cache_correction"]
 
 
 class lyc_config(ctypes.Structure):
@@ -119,6 +119,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
                                         ctypes.c_uint32]
     L.lyc_sync_status.argtypes = [P]
     L.lyc_set_selection.argtypes = [P, ctypes.POINTER(lyc_selection)]
+    L.lyc_cache_correction.argtypes = [P, P, ctypes.POINTER(lyc_kv_cache), I, P, P, P, P]
     L.lyc_set_s_trace.argtypes = [P, P]
     L.lyc_step_bytes.argtypes = [ctypes.POINTER(lyc_config), P, ctypes.c_int64, I, I,
                                  ctypes.POINTER(ctypes.c_uint64), ctypes.POINTER(ctypes.c_uint64)]
@@ -181,6 +182,10 @@ def lyc_sync_status(ctx) -> int:
 
 def lyc_set_selection(ctx, sel: lyc_selection | None) -> int:
     return load().lyc_set_selection(ctx, None if sel is None else ctypes.byref(sel))
+
+
+def lyc_cache_correction(ctx, q, kv: lyc_kv_cache, T, k_new, v_new, out, stream) -> int:
+    return load().lyc_cache_correction(ctx, q, ctypes.byref(kv), T, k_new, v_new, out, stream)
 
 
 def lyc_set_s_trace(ctx, trace) -> int:
@@ -359,6 +364,17 @@ class Lyc:
         sel = lyc_selection(int(rule), int(block), int(ratio[0]), int(ratio[1]), float(p),
                             float(tau))
         self._check(lyc_set_selection(self.ctx, sel), "lyc_set_selection")
+
+    def cache_correction(self, q, K, V, n, out, k_new=None, v_new=None, stream=None):
+        """Cache Correction's dense causal attention: q [L][B][Hq][T][d] bf16,
+        out [L][B][Hq][T][d] fp32, K/V as in decode_step (n counts the T
+        positions); k_new/v_new [L][B][Hkv][T][d] written at rows n-T..n-1 first."""
+        kv = self.kv_cache(K, V, n)
+        rc = lyc_cache_correction(self.ctx, q.data_ptr(), kv, int(q.shape[3]),
+                                  None if k_new is None else k_new.data_ptr(),
+                                  None if v_new is None else v_new.data_ptr(), out.data_ptr(),
+                                  _stream_ptr(stream))
+        self._check(rc, "lyc_cache_correction")
 
     def set_trace(self, trace):
         self._trace = trace

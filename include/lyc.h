@@ -243,6 +243,32 @@ typedef struct {
 
 lyc_status lyc_set_selection(lyc_ctx* ctx, const lyc_selection* sel);
 
+/* ---- Cache Correction (page "LycheeDecode: Accelerating Long-Context LLM
+ * Inference via Hybrid-Head Sparse Decoding", paper-graph-ui summary: section
+ * 4.2.2, and the decoding setup of section 4.1 / Appendix F).  Every 32
+ * decoded tokens, the T most recent positions are prefilled again with dense
+ * attention, and their K/V representations are updated.  This call runs the
+ * attention part of that prefill for every layer, batch element and query
+ * head: query t sits at position p = n - T + t and attends rows 0..p of the
+ * cache (causal):
+ *   out[l][b][h][t] = softmax(q[l][b][h][t] . K[0..p]^T / sqrt(d)) V[0..p].
+ *
+ *   q      device [L][B][Hq][T][d] bf16, 16-byte aligned
+ *   kv     the cache as in lyc_decode_step: kv->n counts the T positions
+ *   k_new, v_new  device [L][B][Hkv][T][d] bf16, or both NULL: the refreshed
+ *          K/V of the T positions, written at rows n-T .. n-1 before the
+ *          attention (the caller's cache is modified)
+ *   out    device [L][B][Hq][T][d] fp32
+ *   stream cudaStream_t (NULL: legacy stream)
+ * Asynchronous like lyc_decode_step; lyc_sync_status reports device errors.
+ * Needs bf16, head_dim 128, and (Hq/Hkv) * T <= 128.  The set buffers are not
+ * touched: the next decode step starts its layer 0 from all retrieval heads
+ * as always.  Errors: INVALID_ARG (NULL or misaligned pointers, T outside
+ * [1, n], n > max_ctx, bad strides), UNSUPPORTED (fp32, head_dim 64, G*T >
+ * 128), OOM, CUDA. */
+lyc_status lyc_cache_correction(lyc_ctx* ctx, const void* q, const lyc_kv_cache* kv, int T,
+                                const void* k_new, const void* v_new, float* out, void* stream);
+
 /* Synchronize the stream of the last step, read and clear the device status
  * word.  Returns LYC_OK, LYC_ERR_BAD_INDEX, LYC_ERR_TIMEOUT or LYC_ERR_CUDA. */
 lyc_status lyc_sync_status(lyc_ctx* ctx);

@@ -442,6 +442,20 @@ __device__ __forceinline__ int cta_ring(const AttnParams& p) {
   return p.wpart_by_sm ? static_cast<int>(sm_index()) : static_cast<int>(blockIdx.x);
 }
 
+// One arrival of `cnt` on the launch's selection-key counter (release: the
+// caller's warp or CTA barrier orders its threads' key stores before this
+// thread's fence); the arrival that completes `expect` resets the counter and
+// raises the flag to the step's epoch + 1.
+__device__ __forceinline__ void keys_arrive(const AttnParams& p, uint32_t cnt, uint32_t expect) {
+  __threadfence();
+  const uint32_t prev = atomicAdd(&p.keys_done[0], cnt);
+  if (prev + cnt == expect) {
+    p.keys_done[0] = 0u;
+    __threadfence();
+    st_release_u32(&p.keys_done[1], *p.epoch + 1u);
+  }
+}
+
 // ---------------------------------------------------------------- consumers
 // Fragment bookkeeping (m16n8k16, g = lane/4, c = lane%4):
 //   S^T tile mt (16 keys):  st[mt][0..1] = keys 16mt+g,   queries 2c, 2c+1
@@ -479,9 +493,17 @@ __device__ __forceinline__ void mma_consumers(const AttnMmaParams& P, unsigned c
   const int mi = lane >> 3, r8 = lane & 7;  // ldmatrix: matrix and row this lane addresses
 
   int t = 0;  // CTA-wide tile sequence number
+  const int nhome = pend - pbeg;
   for (int pi = 0;; ++pi) {
+    // the CTA's own pieces (the dense runs, the only writers of selection
+    // keys) come first: once past them, this warp's keys are written
+    if (pi == nhome && nhome > 0 && p.keys_done) {
+      __syncwarp();
+      if (lane == 0) keys_arrive(p, 1u, static_cast<uint32_t>(p.keys_ctas) * NC);
+      __syncwarp();
+    }
     Piece pc;
-    if (!cta_piece<C>(p, smem, pbeg, pend - pbeg, pi, lane, &pc)) break;
+    if (!cta_piece<C>(p, smem, pbeg, nhome, pi, lane, &pc)) break;
     const Segment& sg = p.segs[pc.seg];
     const int nq = sg.nq, nout = sg.nout, b = sg.b;
     const bool dense = sg.kind == kDense;
@@ -863,7 +885,13 @@ __global__ void __launch_bounds__(MmaCfg<D, NC, NP, STAGES, GT>::kThreads, 1)
   if (P.p.wait_prev) pdl_wait();  // the previous launch writes what this one reads or writes
   static_assert(2 * C::SMEM > 232448, "the per-SM ring needs one CTA per SM");
   if (cta_ring(P.p) >= P.p.wpart_slots) {
-    if (threadIdx.x == 0) atomicOr(P.p.status, kStatusScratch);
+    if (threadIdx.x == 0) {
+      atomicOr(P.p.status, kStatusScratch);
+      // no work, but the arrivals of its consumer warps, so that the
+      // selection does not wait out its limit
+      if (P.p.keys_done && P.p.cta_begin[blockIdx.x + 1] > P.p.cta_begin[blockIdx.x])
+        keys_arrive(P.p, NC, static_cast<uint32_t>(P.p.keys_ctas) * NC);
+    }
   } else {
     const int pbeg = P.p.cta_begin[blockIdx.x];
     const int pend = P.p.cta_begin[blockIdx.x + 1];

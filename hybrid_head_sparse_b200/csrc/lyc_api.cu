@@ -76,6 +76,7 @@ struct LayerPlan {
   int64_t pool_tiles = 0, tiles = 0;  // tiles in the pool, in the whole layer
   int topk_cl = 16;          // cluster size of the selection launch
   int topk_n = 0;            // keys of the longest selection task
+  int keys_ctas = 0;         // CTAs with pieces of their own (dense runs) in the launch
 };
 
 struct Plan {
@@ -138,6 +139,7 @@ struct lyc_ctx {
   // attention launch; then the step epoch
   uint32_t* flags = nullptr;
   uint32_t* attn_flags = nullptr;
+  uint32_t* keys_flags = nullptr;   // per layer: {arrival counter, flag} of the selection keys
   int32_t* pool_cursors = nullptr;  // [2][L + 1], by epoch parity
   uint32_t* epoch = nullptr;
   int32_t* counters = nullptr;
@@ -734,6 +736,8 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const KvVie
     lp.tiles = H.tiles;
     lp.pool_tiles = H.pool_tiles;
     lp.off_pool = take(std::max<size_t>(1, H.pool_segs.size()) * sizeof(int32_t));
+    lp.keys_ctas = 0;
+    for (size_t c = 0; c + 1 < H.cta.size(); ++c) lp.keys_ctas += H.cta[c + 1] > H.cta[c] ? 1 : 0;
   }
   plan->off_final_src = take(hl[L - 1].trace_src.size() * sizeof(void*));
   plan->off_n = take(static_cast<size_t>(B) * sizeof(int64_t));
@@ -887,6 +891,12 @@ lyc_status enqueue_step(lyc_ctx* ctx, Plan* plan, cudaStream_t stream, int set, 
       ap.pool_ups = lp.pool_ups;
       ap.pool_stride = L + 1;
       ap.pool_cursors = ctx->pool_cursors;
+      // the selection of this layer starts once the keys are written (the
+      // dense runs), not once the whole launch is done
+      if (lp.ntasks > 0 && lp.keys_ctas > 0) {
+        ap.keys_done = ctx->keys_flags + 2 * l;
+        ap.keys_ctas = lp.keys_ctas;
+      }
     }
     ap.counters = ctx->counters;
     ap.status = ctx->status;
@@ -940,6 +950,11 @@ lyc_status enqueue_step(lyc_ctx* ctx, Plan* plan, cudaStream_t stream, int set, 
       tp.timeline = plan->timeline;
       tp.timeline_cap = plan->timeline_cap;
       tp.layer = l;
+      tp.status = ctx->status;
+      if (ap.keys_done) {
+        tp.keys_ready = ap.keys_done + 1;
+        tp.prev_done = l > 0 ? ctx->attn_flags + 2 * (l - 1) + 1 : nullptr;
+      }
       if ((st = record_event(ctx, plan, set, ev++, stream, capturing)) != LYC_OK) return st;
       LYC_CUDA(topk_launch(lp.topk_cl, &tp, lp.ntasks, stream), "top-k launch");
       if ((st = record_event(ctx, plan, set, ev++, stream, capturing)) != LYC_OK) return st;
@@ -1212,9 +1227,9 @@ lyc_status lyc_create(const lyc_config* cfg, lyc_ctx** out) {
   };
   lyc_status st;
   // ready flags: two words per (layer, b, slot) and per layer, then the
-  // pool cursors, then the epoch
+  // pool cursors, the key flags (two words per layer), then the epoch
   const size_t flag_words = static_cast<size_t>(L) * B * ctx->Hs * 2 + static_cast<size_t>(L) * 2 +
-                            2 * (static_cast<size_t>(L) + 1) + 4;
+                            2 * (static_cast<size_t>(L) + 1) + static_cast<size_t>(L) * 2 + 4;
   if ((st = alloc(reinterpret_cast<void**>(&ctx->status), 16)) != LYC_OK ||
       (st = alloc(reinterpret_cast<void**>(&ctx->keys),
                   static_cast<size_t>(L) * B * ctx->Hs * ctx->nstride * sizeof(float))) != LYC_OK ||
@@ -1232,6 +1247,7 @@ lyc_status lyc_create(const lyc_config* cfg, lyc_ctx** out) {
   }
   ctx->attn_flags = ctx->flags + static_cast<size_t>(L) * B * ctx->Hs * 2;
   ctx->pool_cursors = reinterpret_cast<int32_t*>(ctx->attn_flags + static_cast<size_t>(L) * 2);
+  ctx->keys_flags = ctx->attn_flags + static_cast<size_t>(L) * 2 + 2 * (static_cast<size_t>(L) + 1);
   ctx->epoch = ctx->flags + (flag_words - 4);
   if (c.dtype == LYC_BF16) {
     // one ring per SM index (the SM a CTA runs on owns it; SM indices need
@@ -1499,8 +1515,9 @@ lyc_status lyc_cache_correction(lyc_ctx* ctx, const void* q, const lyc_kv_cache*
       ctx->corr_part_o = nullptr;
       ctx->corr_part_ml = nullptr;
       ctx->corr_parts_cap = 0;
-      LYC_CUDA(cudaMalloc(&ctx->corr_part_o, pieces.size() * 128 * 128 * sizeof(float)), "cudaMalloc(correction partials)");
-      LYC_CUDA(cudaMalloc(&ctx->corr_part_ml, pieces.size() * 128 * sizeof(float2)), "cudaMalloc(correction partials)");
+      // two partial records per piece (its two key halves)
+      LYC_CUDA(cudaMalloc(&ctx->corr_part_o, 2 * pieces.size() * 128 * 128 * sizeof(float)), "cudaMalloc(correction partials)");
+      LYC_CUDA(cudaMalloc(&ctx->corr_part_ml, 2 * pieces.size() * 128 * sizeof(float2)), "cudaMalloc(correction partials)");
       ctx->corr_parts_cap = pieces.size();
     }
     ctx->corr_n = n;

@@ -122,6 +122,11 @@ struct AttnParams {
                              // its block index
   int32_t wpart_slots;       // rings allocated
   int32_t timeline_cap;
+  uint32_t* keys_done;       // NULL, or {arrival counter, flag} of this launch's selection
+                             // keys: each consumer warp of the first keys_ctas CTAs arrives
+                             // once its own (dense) pieces are done; the last arrival raises
+                             // the flag to epoch + 1
+  int32_t keys_ctas;
   int32_t layer;
   int32_t Hq, G, n;
   int32_t paged;             // 1: the segments' rows are in pages (Segment::bt)
@@ -161,6 +166,12 @@ struct TopkParams {
   int32_t early;          // 1: let the next launch start before this one has read its keys
                           // (its readers wait on the ready flags); 0: only after
   unsigned long long* timeline;  // as in AttnParams
+  const uint32_t* keys_ready;  // NULL: start on griddepcontrol.wait (the attention launch
+                               // before has completed); else on this flag (AttnParams::keys_done)
+  const uint32_t* prev_done;   // with keys_ready: the done flag of the attention launch of the
+                               // layer before (its readers of the set buffers this launch
+                               // writes), or NULL
+  uint32_t* status;            // device status word (wait timeouts)
   int32_t timeline_cap;
   int32_t layer;
   int32_t n, k;           // k: entries of each output set
@@ -186,8 +197,9 @@ struct CorrParams {
   float* out;                 // [L][B][Hq][T][d]
   const CorrPiece* pieces;
   const int32_t* cta_begin;   // pieces of CTA c: [cta_begin[c], cta_begin[c+1])
-  float* part_o;              // [pieces][128 rows][d], unnormalised
-  float2* part_ml;            // [pieces][128 rows]: (running max in log2 units, sum)
+  float* part_o;              // [2 * pieces][128 rows][d], unnormalised: record 2p + h is
+                              // key half h (keys 64h .. 64h+63 of every tile) of piece p
+  float2* part_ml;            // [2 * pieces][128 rows]: (running max in log2 units, sum)
   const int32_t* group_first; // combine: pieces of group j are [group_first[j], group_first[j+1])
   uint32_t* status;
   int32_t L, B, Hq, Hkv, G, T, n;

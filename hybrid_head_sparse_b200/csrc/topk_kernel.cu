@@ -289,17 +289,22 @@ __device__ __forceinline__ uint32_t select_in_candidates(const uint2* cand, cons
 // per CTA: a fence in every thread stalls the whole CTA on memory barriers.)
 template <int CL>
 __device__ __forceinline__ void topk_signal_done(const TopkParams& p, const TopkTask& task, int tid) {
-  if (!task.done) return;
-  __syncthreads();
-  if (tid == 0) {
-    __threadfence();
-    const uint32_t prev = atomicAdd(&task.done[0], 1u);
-    if (prev == static_cast<uint32_t>(CL - 1)) {
-      task.done[0] = 0u;
+  if (task.done) {
+    __syncthreads();
+    if (tid == 0) {
       __threadfence();
-      st_release_u32(&task.done[1], (p.epoch ? *p.epoch : 0u) + 1u);
+      const uint32_t prev = atomicAdd(&task.done[0], 1u);
+      if (prev == static_cast<uint32_t>(CL - 1)) {
+        task.done[0] = 0u;
+        __threadfence();
+        st_release_u32(&task.done[1], (p.epoch ? *p.epoch : 0u) + 1u);
+      }
     }
   }
+  // a launch that started on the key flag rather than on griddepcontrol.wait
+  // still completes only after the attention launch before it, so that the
+  // launches of the step complete in launch order
+  if (p.keys_ready && tid == 0) pdl_wait();
 }
 
 // VAR: a size rule or block expansion may be in use (an instantiation of its
@@ -329,8 +334,26 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster_kernel(const Top
   // completed.  The next kernel (the next layer's attention) may start its
   // launch before that when its readers of this selection's sets wait on the
   // ready flags (p.early), else only after.
+  // With a key flag, the keys are complete once every consumer warp of the
+  // attention launch that writes them has finished its dense rows (the flag
+  // holds the step's epoch + 1); the rest of that launch (its gathered rows)
+  // may still run.  The sets this launch writes replace sets that the
+  // attention launch of the layer before may still read: wait for that
+  // launch's done flag as well.  Both writers were resident before this
+  // launch began (each launch of the step starts only once every CTA of the
+  // one before it has), so the waits end.
   if (p.early) pdl_launch_dependents();
-  pdl_wait();
+  if (p.keys_ready) {
+    __shared__ int wait_abort;
+    if (tid == 0) {
+      wait_abort = 0;
+      if (wait_flag(p.keys_ready, *p.epoch + 1u, &wait_abort, p.status) && p.prev_done)
+        wait_flag(p.prev_done, *p.epoch + 1u, &wait_abort, p.status);
+    }
+    __syncthreads();
+  } else {
+    pdl_wait();
+  }
   if (!p.early) pdl_launch_dependents();
   const uint64_t t_start = p.timeline ? global_timer_ns() : 0;  // work starts here
 

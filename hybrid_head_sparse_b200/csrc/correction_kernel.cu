@@ -15,20 +15,24 @@
 // K/V tiles of 128 rows arrive by TMA (128-byte swizzle) and are read by the
 // tensor core in place:
 //   S[128 q x 128 keys]  = Q[128 x 128 d] . K^T      (8 MMAs, K=16 each, into TMEM)
-//   O[128 q x 128 d]    += P[128 x 128 keys] . V     (8 MMAs, into TMEM)
-// Warps 0-3 are the softmax warps: thread i owns query row i (tensor-memory
-// lane i): it reads its 128 logits, applies the causal mask, keeps a running
-// maximum (rescaling O in tensor memory only when the maximum grows by more
-// than 2^8), and writes its row of P (bf16, 128-byte swizzle) for the PV MMA.
-// Warp 4 issues the MMAs (one thread) and owns the tensor memory; warp 5
-// issues the TMA copies (one thread).  Two S buffers and two P buffers let
-// the QK MMA of tile t+1 and the softmax of tile t overlap.
+//   O[128 q x 128 d]    += P[128 x 128 keys] . V     (8 MMAs, into TMEM: keys
+//                                                     0-63 and 64-127 into O_a, O_b)
+// Warps 0-7 are the softmax warps: warp w owns query rows 32*(w%4) .. +31
+// (their tensor-memory lanes) and key half w/4 of every tile.  Each half
+// keeps its own running maximum (O rescaled in tensor memory only when it
+// grows by more than 2^8), sum and O accumulator, and writes its half of the
+// row of P (bf16, 128-byte swizzle) for the PV MMA.  Warp 8 issues the MMAs
+// (one thread) and owns the tensor memory; warp 9 issues the TMA copies (one
+// thread).  Two S buffers and two P buffers let the QK MMA of tile t+1 and
+// the softmax of tile t overlap.  Tensor memory: S x2 (columns 0, 128), O of
+// key half 0 (256) and of key half 1 (384).
 //
 // Work pooling (Appendix C, Algorithm 2, applied to this dense pass): the
 // (l, b, g) groups times their ceil(n/128) tiles are cut into equal runs, one
 // per CTA; a run that crosses groups becomes several pieces.  Each piece
-// writes a partial (m, l, O) per query row; a second launch merges the pieces
-// of each group (log-sum-exp) into the output.
+// writes two partial states (m, l, O) per query row, one per key half; a
+// second launch merges the records of each group (log-sum-exp) into the
+// output.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <math.h>
@@ -48,10 +52,10 @@ constexpr int kCcRows = 128;  // keys per tile; query rows per block
 struct CcCfg {
   static constexpr int D = 128;
   static constexpr int STAGES = 2;
-  static constexpr int kSoftThreads = 128;  // warps 0-3
-  static constexpr int kMmaWarp = 4;
-  static constexpr int kLoadWarp = 5;
-  static constexpr int kThreads = 6 * 32;
+  static constexpr int kSoftThreads = 256;  // warps 0-7
+  static constexpr int kMmaWarp = 8;
+  static constexpr int kLoadWarp = 9;
+  static constexpr int kThreads = 10 * 32;
   static constexpr int HALF = kCcRows * 128;  // one 64-column half of a tile (bytes)
   static constexpr int TILEB = 2 * HALF;      // a K, V, Q or P tile (bytes)
   static constexpr int OFF_Q = 0;
@@ -236,7 +240,8 @@ __device__ __forceinline__ void cc_mma(const CorrParams& P, unsigned char* smem,
         const uint64_t a =
             tc::smem_desc(pbase + b * CcCfg::TILEB + (kt >> 2) * CcCfg::HALF + (kt & 3) * 32, 16, 1024, 2);
         const uint64_t bd = tc::smem_desc(vbase + stage * CcCfg::TILEB + kt * 16 * 128, CcCfg::HALF, 1024, 2);
-        tc::mma_bf16_ss(tmem + 256, a, bd, IDESC_PV, (kt > 0 || !first) ? 1u : 0u);
+        // keys 0-63 accumulate into O_a (column 256), keys 64-127 into O_b (384)
+        tc::mma_bf16_ss(tmem + 256 + (kt >> 2) * 128, a, bd, IDESC_PV, ((kt & 3) > 0 || !first) ? 1u : 0u);
       }
       tc::commit(&br.vempty[stage]);
       tc::commit(&br.pv_done[b]);
@@ -252,23 +257,40 @@ __device__ __forceinline__ void cc_mma(const CorrParams& P, unsigned char* smem,
 }
 
 // ---------------------------------------------------------------- softmax warps
-// Thread i of warps 0-3 owns query row i (tensor-memory lane i).  Per piece:
-// write its query row into Q (128-byte swizzle; rows >= G*T zero), then per
-// tile: read its 128 logits, mask keys past its position, update the running
-// maximum (rescaling O when it grows by more than 2^8: a warp-wide decision,
-// since tensor-memory reads and writes are warp-wide), and write its row of P.
-// At the piece's end: read O and write the piece's partial state.
+// Warps 0-7.  Warp w owns tensor-memory lanes 32*(w%4) .. +31, i.e. query rows
+// i = 32*(w%4) + lane, and key half hf = w/4 of every tile (keys 64*hf ..
+// 64*hf+63).  Each half keeps its own running maximum, sum and O accumulator
+// (columns 256 + 128*hf): the two halves are two split-K partial states of
+// the same rows, merged by the combine launch like any other pieces.  So the
+// two warps of a row never exchange anything, and every SM sub-partition runs
+// two softmax warps.
+// Per piece: write this half of the query row into Q (128-byte swizzle; rows
+// >= G*T zero).  Per tile: read the half's 64 logits, mask keys past the
+// row's position (only in the tiles that reach past the first query's
+// position), keep the running maximum (O rescaled in place only when it grows
+// by more than 2^8: a warp-wide decision, since tensor-memory accesses are
+// warp-wide), write P = 2^(x - max) as bf16 for the PV MMA.  At the piece's
+// end: read O and write the half's partial state.
+__device__ __forceinline__ float cc_ex2(float x) {  // 2^x (ex2.approx.ftz: 2^-inf = +0)
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ void cc_softmax(const CorrParams& P, unsigned char* smem, int pbeg, int pend,
                                            uint32_t tmem) {
   constexpr unsigned FULL = 0xffffffffu;
-  const int i = threadIdx.x;  // query row, tensor-memory lane
-  const int quarter = i >> 5;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int quarter = warp & 3, hf = warp >> 2;
+  const int i = quarter * 32 + lane;  // query row, tensor-memory lane
   CcBars br(smem);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + CcCfg::OFF_FLAGS);
   const uint32_t tl = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+  const uint32_t tl_o = tl + 256 + hf * 128;  // this half's O accumulator
   const float sl2 = P.scale_log2;
   const bool live = i < P.rows;
   const int pos = P.n - P.T + (live ? i % P.T : 0);  // keys 0 .. pos are visible to this row
+  const int pos_min = P.n - P.T;                      // the first query's position
   const bf16_t* qg = static_cast<const bf16_t*>(P.q);
   unsigned char* qbuf = smem + CcCfg::OFF_Q;
   unsigned char* pbuf = smem + CcCfg::OFF_P;
@@ -279,8 +301,9 @@ __device__ __forceinline__ void cc_softmax(const CorrParams& P, unsigned char* s
       const bf16_t* src =
           qg + (((static_cast<int64_t>(piece.l) * P.B + piece.b) * P.Hq + static_cast<int64_t>(piece.g) * P.G) *
                     P.T + i) * CcCfg::D;
-#pragma unroll 4
-      for (int ch = 0; ch < 16; ++ch) {
+#pragma unroll
+      for (int c8 = 0; c8 < 8; ++c8) {
+        const int ch = hf * 8 + c8;
         uint4 v = make_uint4(0u, 0u, 0u, 0u);
         if (live) v = *reinterpret_cast<const uint4*>(src + ch * 8);
         *reinterpret_cast<uint4*>(qbuf + cswz(i, ch)) = v;
@@ -294,74 +317,83 @@ __device__ __forceinline__ void cc_softmax(const CorrParams& P, unsigned char* s
       const int b = t & 1;
       if (!mbar_wait(&br.s_ready[b], (t >> 1) & 1, abort_flag, P.status)) return;
       tc::fence_after_sync();
-      uint32_t r[8][16];
+      uint32_t r[4][16];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) tc::ld_32x32b_x16(tl + b * 128 + c * 16, r[c]);
+      for (int c = 0; c < 4; ++c) tc::ld_32x32b_x16(tl + b * 128 + hf * 64 + c * 16, r[c]);
       tc::wait_ld();
       tc::fence_before_sync();
       mbar_arrive(&br.s_free[b]);
-      // causal mask: key kb + c is visible if kb + c <= pos
-      const int kb = (piece.t0 + u) * kCcRows;
-      float mx = -INFINITY;
+      const int kb = (piece.t0 + u) * kCcRows + hf * 64;  // this half's first key
+      float mraw = -INFINITY;
+      if (live && kb + 63 <= pos_min) {  // every key of the half is visible to every row
 #pragma unroll
-      for (int c = 0; c < 8; ++c)
+        for (int c = 0; c < 4; ++c)
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const bool vis = live && kb + c * 16 + j <= pos;
-          const float x = vis ? __uint_as_float(r[c][j]) * sl2 : -INFINITY;
-          r[c][j] = __float_as_uint(x);
-          mx = fmaxf(mx, x);
-        }
+          for (int j = 0; j < 16; ++j) mraw = fmaxf(mraw, __uint_as_float(r[c][j]));
+      } else {  // causal mask (key kb + x is visible if kb + x <= pos); rows >= G*T see nothing
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const bool vis = live && kb + c * 16 + j <= pos;
+            const float x = vis ? __uint_as_float(r[c][j]) : -INFINITY;
+            r[c][j] = __float_as_uint(x);
+            mraw = fmaxf(mraw, x);
+          }
+      }
+      const float mx = mraw * sl2;                       // sl2 > 0: the scaled maximum
       const bool grow = mx > m_used + 8.f;               // includes the first finite maximum
       const bool rescale = grow && m_used != -INFINITY;  // O already holds earlier tiles
       if (__any_sync(FULL, rescale)) {
         // O holds the tiles before this one: wait for the last PV, rescale in place
         if (!mbar_wait(&br.pv_done[(t - 1) & 1], ((t - 1) >> 1) & 1, abort_flag, P.status)) return;
         tc::fence_after_sync();
-        const float sc = rescale ? exp2f(m_used - mx) : 1.f;
+        const float sc = rescale ? cc_ex2(m_used - mx) : 1.f;
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
           uint32_t o[16];
-          tc::ld_32x32b_x16(tl + 256 + c * 16, o);
+          tc::ld_32x32b_x16(tl_o + c * 16, o);
           tc::wait_ld();
 #pragma unroll
           for (int j = 0; j < 16; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * sc);
-          cc_st_x16(tl + 256 + c * 16, o);
+          cc_st_x16(tl_o + c * 16, o);
         }
         cc_wait_st();
         lsum *= sc;
       }
       if (grow) m_used = mx;
+      // p = 2^(x sl2 - m_used); a row with no visible key yet has m_used = -inf
+      // and only masked (-inf) logits, which give 0
+      const float mneg = m_used == -INFINITY ? 0.f : -m_used;
       // P buffer b was last read by the PV of tile t-2
       if (t >= 2 && !mbar_wait(&br.pv_done[b], ((t - 2) >> 1) & 1, abort_flag, P.status)) return;
       unsigned char* prow = pbuf + b * CcCfg::TILEB;
 #pragma unroll
-      for (int ch = 0; ch < 16; ++ch) {
+      for (int c8 = 0; c8 < 8; ++c8) {
         uint32_t w[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const float x0 = __uint_as_float(r[ch >> 1][(ch & 1) * 8 + 2 * e]);
-          const float x1 = __uint_as_float(r[ch >> 1][(ch & 1) * 8 + 2 * e + 1]);
-          const float p0 = x0 == -INFINITY ? 0.f : exp2f(x0 - m_used);
-          const float p1 = x1 == -INFINITY ? 0.f : exp2f(x1 - m_used);
+          const float p0 = cc_ex2(fmaf(__uint_as_float(r[c8 >> 1][(c8 & 1) * 8 + 2 * e]), sl2, mneg));
+          const float p1 = cc_ex2(fmaf(__uint_as_float(r[c8 >> 1][(c8 & 1) * 8 + 2 * e + 1]), sl2, mneg));
           w[e] = cc_pack_bf16(p0, p1);
-          lsum += __uint_as_float(w[e] << 16) + __uint_as_float(w[e] & 0xffff0000u);
+          lsum += p0 + p1;
         }
-        *reinterpret_cast<uint4*>(prow + cswz(i, ch)) = make_uint4(w[0], w[1], w[2], w[3]);
+        *reinterpret_cast<uint4*>(prow + cswz(i, hf * 8 + c8)) = make_uint4(w[0], w[1], w[2], w[3]);
       }
       tc::fence_async_smem();
       tc::fence_before_sync();
       mbar_arrive(&br.p_ready[b]);
     }
-    // the piece's O, once the PV of its last tile is done
+    // the half's O, once the PV of the piece's last tile is done
     const int tl_last = t - 1;
     if (!mbar_wait(&br.pv_done[tl_last & 1], (tl_last >> 1) & 1, abort_flag, P.status)) return;
     tc::fence_after_sync();
-    float* dst = P.part_o + (static_cast<int64_t>(piece.part) * kCcRows + i) * CcCfg::D;
+    const int64_t rec = 2 * static_cast<int64_t>(piece.part) + hf;  // this half's partial record
+    float* dst = P.part_o + (rec * kCcRows + i) * CcCfg::D;
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
       uint32_t o[16];
-      tc::ld_32x32b_x16(tl + 256 + c * 16, o);
+      tc::ld_32x32b_x16(tl_o + c * 16, o);
       tc::wait_ld();
       if (live)
 #pragma unroll
@@ -370,7 +402,7 @@ __device__ __forceinline__ void cc_softmax(const CorrParams& P, unsigned char* s
               make_float4(__uint_as_float(o[j]), __uint_as_float(o[j + 1]), __uint_as_float(o[j + 2]),
                           __uint_as_float(o[j + 3]));
     }
-    if (live) P.part_ml[static_cast<int64_t>(piece.part) * kCcRows + i] = make_float2(m_used, lsum);
+    if (live) P.part_ml[rec * kCcRows + i] = make_float2(m_used, lsum);
     tc::fence_before_sync();
     mbar_arrive(br.o_free);
   }
@@ -419,7 +451,7 @@ __global__ void __launch_bounds__(CcCfg::kThreads, 1)
   const uint32_t tmem = flags[1];
   const int pbeg = P.cta_begin[blockIdx.x];
   const int pend = P.cta_begin[blockIdx.x + 1];
-  if (warp < 4) {
+  if (warp < 8) {
     cc_softmax(P, smem, pbeg, pend, tmem);
   } else if (warp == C::kMmaWarp) {
     cc_mma(P, smem, pbeg, pend, tmem);
@@ -433,7 +465,8 @@ __global__ void __launch_bounds__(CcCfg::kThreads, 1)
 }
 
 // One warp per (KV group, query row): the log-sum-exp merge of the group's
-// piece partials into the output.  Lane j owns columns 4j .. 4j+3.
+// partial records (two per piece) into the output.  Lane j owns columns
+// 4j .. 4j+3.
 __global__ void correction_combine_kernel(const CorrParams P) {
   const int warps = blockDim.x / 32;
   const int lane = threadIdx.x & 31;
@@ -441,7 +474,8 @@ __global__ void correction_combine_kernel(const CorrParams P) {
   const int64_t ngroups = static_cast<int64_t>(P.L) * P.B * P.Hkv;
   if (w >= ngroups * P.rows) return;
   const int grp = static_cast<int>(w / P.rows), i = static_cast<int>(w % P.rows);
-  const int f = P.group_first[grp], e = P.group_first[grp + 1];
+  // two partial records (key halves) per piece
+  const int f = 2 * P.group_first[grp], e = 2 * P.group_first[grp + 1];
   float M = -INFINITY;
   for (int pc = f; pc < e; ++pc) M = fmaxf(M, P.part_ml[static_cast<int64_t>(pc) * kCcRows + i].x);
   float L = 0.f;

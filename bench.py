@@ -45,7 +45,10 @@ def parse_args(argv=None):
     ap.add_argument("--layers", type=int, default=32, help="layers of the stack (32 = the workload)")
     ap.add_argument("--retrieval-heads", type=int, default=2,
                     help="retrieval query heads per layer after layer 0; -1 = all (dense baseline)")
-    ap.add_argument("--select-mode", choices=["per_qhead", "kvgroup_mean"], default="per_qhead")
+    ap.add_argument("--select-mode", choices=["per_qhead", "kvgroup_mean"], default="kvgroup_mean",
+                    help="kvgroup_mean: one set per KV group, keyed by the group's mean query (the "
+                         "pages' GQA handling, whose bytes are the analytic floor); per_qhead: one "
+                         "set per query head (the line also times the mode not chosen)")
     ap.add_argument("--attn-kernel", choices=["mma", "tcgen05"], default="mma",
                     help="bf16 attention kernel: mma.sync (default) or tcgen05/TMEM")
     ap.add_argument("--serving", action="store_true",
@@ -59,6 +62,10 @@ def parse_args(argv=None):
     ap.add_argument("--block", type=int, default=64, help="block rule: rows per block")
     ap.add_argument("--p", type=float, default=0.5, help="top-p rule: probability mass")
     ap.add_argument("--tau", type=float, default=1e-4, help="threshold rule: smallest probability")
+    ap.add_argument("--correction", action="store_true",
+                    help="Cache Correction instead: dense causal attention of the T most recent "
+                         "positions over the cache (lyc_cache_correction), one line")
+    ap.add_argument("--T", type=int, default=32, help="Cache Correction: positions refreshed")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-layers", type=int, default=2,
@@ -85,6 +92,16 @@ def measured_peaks():
         return float(d["hbm_gbs"]), "measured"
     except Exception:
         return FALLBACK_HBM_GBS, "fallback"
+
+
+def measured_bf16_tflops() -> float:
+    """Burst cuBLAS bf16 throughput of this GPU (the correction kernel is timed
+    alone), else the fallback figure."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"])
+    except Exception:
+        return 1590.0
 
 
 def attn_source_hash() -> str:
@@ -428,6 +445,41 @@ def run_lyc(args):
         if rc != 0:
             raise RuntimeError(f"device status after e2e: {lyc.lyc_status_string(rc)}")
 
+    # ---- the other selection mode on the same inputs (its steps/s and byte rates)
+    other = None
+    if not args.serving and args.selection == "topk":
+        omode = "per_qhead" if args.select_mode == "kvgroup_mean" else "kvgroup_mean"
+        octx = lyc.Lyc(spec.L, spec.B, spec.Hq, spec.Hkv, spec.d, spec.n, spec.k, dtype=spec.dtype,
+                       select_mode=omode, device=local,
+                       flags=lyc.LYC_CFG_TCGEN05 if args.attn_kernel == "tcgen05" else 0)
+        oS = torch.empty((spec.B, octx.Hs, spec.k), dtype=torch.int32, device=dev)
+
+        def ostep():
+            octx.decode_step(data["q"], data["k"], data["v"], spec.n, role, spec.k, out, oS,
+                             stream=stream)
+
+        for _ in range(max(args.warmup, 1)):
+            ostep()
+        torch.cuda.synchronize()
+        barrier()
+        ev0.record(stream)
+        for _ in range(args.steps):
+            ostep()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        oms = max_over_ranks(ev0.elapsed_time(ev1), dev)
+        rc = octx.sync_status()
+        if rc != 0:
+            raise RuntimeError(f"device status ({omode}): {lyc.lyc_status_string(rc)}")
+        oan, odi = octx.step_bytes(role, spec.n, spec.k)
+        octx.close()
+        oms_step = oms / args.steps
+        other = {"select_mode": omode, "value": job_steps_per_s(world, args.steps, oms),
+                 "unit": "steps/s", "ms_per_step": oms_step,
+                 "analytic_frac_of_measured_peak": round(oan / (oms_step / 1e3) / 1e9 / peak, 4),
+                 "kernel_bytes_per_step": odi,
+                 "kernel_gbs": round(odi / (oms_step / 1e3) / 1e9, 1)}
+
     # ---- the oracle on the host cores (rank 0, one GPU only)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -460,6 +512,7 @@ def run_lyc(args):
         "roofline": roofline,
         "kernels": {"attn_ms_per_step": attn_ms, "topk_ms_per_step": topk_ms,
                     "ms_per_step_with_event_nodes": ms_step_timed},
+        "other_select_mode": other,
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": launches_per_step * args.steps,
@@ -587,6 +640,118 @@ def run_serving(args):
     return 0
 
 
+def run_correction(args):
+    """Cache Correction on one GPU: the T most recent positions of the
+    Llama3-8B-shaped stack at n tokens are attended again, densely and
+    causally, over the whole cache, every layer, with their refreshed K/V rows
+    written first.  One pass = one lyc_cache_correction call (the row append,
+    the attention launch and the launch that merges split rows)."""
+    import numpy as np
+    import torch
+
+    from hybrid_head_sparse_b200 import build as Bld
+    from hybrid_head_sparse_b200 import lyc, workloads as W
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    Bld.build()
+    lyc.load()
+    spec = workload_spec(args)
+    L, B, Hq, Hkv, d, n, T = spec.L, spec.B, spec.Hq, spec.Hkv, spec.d, spec.n, args.T
+    data = W.make_stack(spec, dev)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(spec.seed + 1)
+    q = torch.randn((L, B, Hq, T, d), generator=gen, device=dev).to(torch.bfloat16)
+    k_new = torch.randn((L, B, Hkv, T, d), generator=gen, device=dev).to(torch.bfloat16)
+    v_new = torch.randn((L, B, Hkv, T, d), generator=gen, device=dev).to(torch.bfloat16)
+    out = torch.empty((L, B, Hq, T, d), device=dev)
+    ctx = lyc.Lyc(L, B, Hq, Hkv, d, n, spec.k)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        ctx.cache_correction(q, data["k"], data["v"], n, out, k_new=k_new, v_new=v_new,
+                             stream=stream)
+
+    for _ in range(max(args.warmup, 1)):
+        step()
+    torch.cuda.synchronize()
+    rc = ctx.sync_status()
+    if rc != 0:
+        raise RuntimeError(f"device status after warm-up: {lyc.lyc_status_string(rc)}")
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    torch.cuda.synchronize()
+    with ClockSampler(0) as clk:
+        evs[0].record(stream)
+        for i in range(args.steps):
+            step()
+            evs[i + 1].record(stream)
+        torch.cuda.synchronize()
+    ms_total = evs[0].elapsed_time(evs[-1])
+    per = [evs[i].elapsed_time(evs[i + 1]) for i in range(args.steps)]
+    rc = ctx.sync_status()
+    if rc != 0:
+        raise RuntimeError(f"device status after timing: {lyc.lyc_status_string(rc)}")
+    ms_pass = ms_total / args.steps
+    # algorithmic bytes: every (l, b, g) group's n K and V rows read once (the
+    # causal mask only drops rows past each query's position, all inside the
+    # last tile); q read, out written and the T refreshed rows written are
+    # counted apart
+    kv_bytes = L * B * Hkv * n * d * 2 * 2
+    io_bytes = L * B * Hq * T * d * (2 + 4) + L * B * Hkv * T * d * 2 * 2
+    flops = 0
+    for t in range(T):  # QK and PV, 2 flops per multiply-add, causal rows
+        flops += 4 * L * B * Hq * (n - T + t + 1) * d
+    peak, peak_kind = measured_peaks()
+    gbs = kv_bytes / (ms_pass / 1e3) / 1e9
+    tflops = flops / (ms_pass / 1e3) / 1e12
+    line = {
+        "metric": f"Cache Correction passes/s at {n // 1024}K ctx (T={T} positions, every layer)",
+        "value": args.steps / (ms_total / 1e3), "unit": "passes/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_pass,
+        "step_ms_distribution": {kk: round(v, 4) for kk, v in percentiles(per).items()},
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) q/K/V with sinks and planted heavy hitters; "
+                "seeded N(0,1) refreshed rows)",
+        "config": {"workload": f"llama3-8b-cache-correction-n{n}-T{T}", "L": L, "B": B,
+                   "Hq": Hq, "Hkv": Hkv, "d": d, "n": n, "T": T, "append": True,
+                   "parallelism": "replicas x1",
+                   "l2": "inputs larger than L2 (KV cache %.1f GB)" % (
+                       2 * data["k"].numel() * data["k"].element_size() / 1e9)},
+        "roofline": {
+            "bound": "hbm", "kernel": "correction_tc_kernel (tcgen05, one launch for all layers)"
+                                      " + its split-merge launch + the row append",
+            "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
+            "frac": round(gbs / peak, 4),
+            "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
+            "traffic": None, "algorithmic_bytes_per_launch": kv_bytes,
+            "avg_launch_ms": ms_pass,
+            "note": "achieved = K+V bytes of every (layer, KV group) / CUDA-event time of the "
+                    "whole call; q, out and refreshed rows (%d bytes) not counted" % io_bytes},
+        "tensor": {"tflops": round(tflops, 1), "flops_per_pass": flops,
+                   "frac_of_measured_bf16": round(tflops / measured_bf16_tflops(), 4)},
+        "clocks": clk.summary(),
+    }
+    if not args.no_cpu_baseline:
+        import oracle as O
+        idx = torch.tensor([0], device=dev)
+        Kh = W.host_view(data["k"].index_select(0, idx)[:, :, :, :n]).copy()
+        Vh = W.host_view(data["v"].index_select(0, idx)[:, :, :, :n]).copy()
+        Kh[:, :, :, n - T:n] = W.host_view(k_new.index_select(0, idx))
+        Vh[:, :, :, n - T:n] = W.host_view(v_new.index_select(0, idx))
+        st = O.Stack(W.host_view(data["q"].index_select(0, idx)), Kh, Vh,
+                     np.ones((1, Hq), dtype=np.uint8))
+        t0 = time.perf_counter()
+        O.correction(st, W.host_view(q.index_select(0, idx)))
+        sec = (time.perf_counter() - t0) * L
+        line["cpu_baseline"] = {
+            "value": 1.0 / sec, "unit": "passes/s", "cores": cpu_cores(), "kind": "oracle",
+            "sample": f"oracle (fp64 C, OpenMP) on layer 0 of one pass at full size (n={n}, "
+                      f"T={T}, all {Hq} heads); pass time = {L} x that layer"}
+    ctx.close()
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def rule_kernel_bytes(role, trace, n, L, Hq, Hkv, d, select_mode):
     """K+V bytes the attention kernels read in one step under a selection
     rule: n rows for every KV group with a retrieval head (all at layer 0),
@@ -706,6 +871,8 @@ def main(argv=None):
         return run_reference(args)
     if args.serving:
         return run_serving(args)
+    if args.correction:
+        return run_correction(args)
     if args.selection != "topk":
         return run_rule(args)
     return run_lyc(args)

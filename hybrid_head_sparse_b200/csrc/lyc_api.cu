@@ -354,20 +354,24 @@ lyc_status encode_gather_map(lyc_ctx* ctx, CUtensorMap* map, const void* base, c
 }
 
 // Cluster size of a selection launch of `ntasks` sets.  A small selection (a
-// few sets) runs beside the next layer's attention, on SMs the planner takes
-// from that attention: clusters of 16 where they fit, else 8.  The next
-// attention launch has CTAs that take those SMs back (pool units only) once
-// the selection is done, so a faster selection costs it little (measured on
-// B200 at 128K keys: 16 beats 8 by ~1% with the overlapped launches; 4 takes
-// longer than the dense rows last).  A large selection (layer 0) takes the
-// largest size whose clusters are all resident at once, so that it runs in
-// one wave and the next layer starts right away; else the smallest size.
-int pick_topk_cluster(const lyc_ctx* ctx, int ntasks) {
+// few sets) runs beside the next layer's attention, on SMs that the planner
+// leaves out of that attention's grid.  When the next layer has a large pool
+// of gathered rows (`big_pool`: at least a fifth of its tiles), its attention
+// needs the SMs more than the selection needs speed: clusters of 8.  Else
+// the selection's latency is on the critical path (the next selection waits
+// for its SMs): clusters of 16.  (Measured on B200 at 128K keys, 2 retrieval
+// heads per layer: per-head sets, pool ~1/3 of the tiles, 8 beats 16 by
+// 4.6 %; KV-group sets, pool ~1/9, 16 beats 8 by 1.2 %.)  A large selection
+// (layer 0) takes the largest size whose clusters are all resident at once,
+// so that it runs in one wave and the next layer starts right away; else the
+// smallest size.
+int pick_topk_cluster(const lyc_ctx* ctx, int ntasks, bool big_pool) {
   auto resident = [&](int cl) {
     return ctx->topk_resident[cl] > 0 ? ctx->topk_resident[cl] : ctx->sms / cl;
   };
-  if (ntasks * 16 <= ctx->sms / 4 && (ctx->topk_cls & (1u << 16)) && ntasks <= resident(16)) return 16;
-  if (ntasks * 16 <= ctx->sms / 4 && (ctx->topk_cls & (1u << 8)) && ntasks <= resident(8)) return 8;
+  if (!big_pool && ntasks * 16 <= ctx->sms / 4 && (ctx->topk_cls & (1u << 16)) && ntasks <= resident(16))
+    return 16;
+  if (ntasks * 8 <= ctx->sms / 4 && (ctx->topk_cls & (1u << 8)) && ntasks <= resident(8)) return 8;
   int best = 0, smallest = 0;
   for (int cl : {16, 8, 4}) {
     if (!(ctx->topk_cls & (1u << cl))) continue;
@@ -594,15 +598,20 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const KvVie
     // kernel then starts late behind it.
     int avail = ctx->sms;
     if (l > 0) {
+      int64_t gathered = 0;  // this layer's tiles of gathered rows (the pool)
+      for (const Segment& sg : H.segs)
+        if (sg.kind == kSparse) gathered += (sg.rows + TR - 1) / TR;
+      hl[l - 1].topk_cl = pick_topk_cluster(ctx, static_cast<int>(hl[l - 1].tasks.size()),
+                                            5 * gathered >= NT);
       const int prev = static_cast<int>(hl[l - 1].tasks.size()) * hl[l - 1].topk_cl;
       if (prev > 0 && prev <= ctx->sms / 4) avail = ctx->sms - prev;
     }
-    // With the pool the launch also has CTAs for the selection's SMs: they
-    // start once it is done and take pool units only; the dense runs go to
-    // the `home` CTAs that start at once.
+    // The grid leaves those SMs to the selection: the selection of this layer
+    // starts on its key flag and then needs SMs, which it gets at once when
+    // the previous selection ends (measured on B200: +1.9 % in KV-group mode
+    // against a grid with CTAs that take those SMs back for pool units).
     H.tiles = NT;
-    const int grid = static_cast<int>(std::min<int64_t>(NT, use_pool ? ctx->sms : avail));
-    const int home = std::min(grid, avail);
+    const int grid = static_cast<int>(std::min<int64_t>(NT, avail));
     H.grid = grid;
     std::vector<int> npieces(H.segs.size(), 0);
     std::vector<std::vector<Piece>> per_cta(grid);
@@ -620,7 +629,7 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const KvVie
         }
       }
       const int64_t nt = tstart.back();
-      const int cut = use_pool ? home : grid;
+      const int cut = grid;
       size_t si = 0;
       for (int c = 0; c < cut; ++c) {
         const int64_t t0 = nt * c / cut, t1 = nt * (c + 1) / cut;
@@ -700,7 +709,8 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const KvVie
         writer[s] = l;
       }
     prev_fresh = fresh;
-    H.topk_cl = pick_topk_cluster(ctx, static_cast<int>(H.tasks.size()));
+    // (the next layer revises this once its pool is known)
+    H.topk_cl = pick_topk_cluster(ctx, static_cast<int>(H.tasks.size()), false);
     for (int b = 0; b < B; ++b)
       for (int s = 0; s < Hs; ++s) H.trace_src.push_back(set_ptr(cur[s], b, s));
   }

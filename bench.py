@@ -112,9 +112,9 @@ def attn_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(workload: str):
+def profiled_traffic(workload: str, select_mode: str):
     """DRAM bytes per attention launch from the committed ncu summary, if it
-    was taken on the current kernel source."""
+    was taken on the current kernel source, workload and selection mode."""
     pdir = os.path.join(ROOT, "profiles")
     if not os.path.isdir(pdir):
         return None
@@ -128,7 +128,8 @@ def profiled_traffic(workload: str):
                     rec = json.loads(line.split(":", 1)[1])
                 except ValueError:
                     continue
-                if rec.get("source_sha") == want and rec.get("workload") == workload:
+                if (rec.get("source_sha") == want and rec.get("workload") == workload
+                        and rec.get("select_mode", "per_qhead") == select_mode):
                     return rec.get("bytes_per_launch")
     return None
 
@@ -398,7 +399,7 @@ def run_lyc(args):
     analytic, distinct = ctx.step_bytes(role, spec.n, spec.k)
     peak, peak_kind = measured_peaks()
     achieved = distinct / (attn_ms / 1e3) / 1e9
-    traffic = profiled_traffic(spec.name)
+    traffic = profiled_traffic(spec.name, args.select_mode)
     roofline = {
         "bound": "hbm",
         "kernel": ("attn_tc_layer_kernel" if args.attn_kernel == "tcgen05" else "attn_mma_layer_kernel")

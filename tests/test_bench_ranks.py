@@ -74,16 +74,23 @@ def test_percentiles():
 
 def test_traffic_record_lookup(tmp_path, monkeypatch):
     """The bench takes DRAM traffic from a committed ncu summary only when the
-    summary was taken on the current attention-kernel source and workload."""
+    summary was taken on the current attention-kernel source, workload and
+    selection mode."""
     import bench
     prof = tmp_path / "profiles"
     prof.mkdir()
     (prof / "attn_mma_layer_kernel_some-workload.md").write_text(
         "summary\n"
         'traffic-record: {"workload": "w1", "source_sha": "abc", "bytes_per_launch": 123}\n')
+    (prof / "attn_mma_layer_kernel_other.md").write_text(
+        'traffic-record: {"workload": "w1", "select_mode": "kvgroup_mean", "source_sha": "abc", '
+        '"bytes_per_launch": 456}\n')
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     monkeypatch.setattr(bench, "attn_source_hash", lambda: "abc")
-    assert bench.profiled_traffic("w1") == 123
-    assert bench.profiled_traffic("w2") is None
+    # a record without a selection mode was taken per head
+    assert bench.profiled_traffic("w1", "per_qhead") == 123
+    assert bench.profiled_traffic("w1", "kvgroup_mean") == 456
+    assert bench.profiled_traffic("w2", "per_qhead") is None
     monkeypatch.setattr(bench, "attn_source_hash", lambda: "def")
-    assert bench.profiled_traffic("w1") is None
+    assert bench.profiled_traffic("w1", "per_qhead") is None
+    assert bench.profiled_traffic("w1", "kvgroup_mean") is None

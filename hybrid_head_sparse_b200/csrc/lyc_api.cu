@@ -354,24 +354,20 @@ lyc_status encode_gather_map(lyc_ctx* ctx, CUtensorMap* map, const void* base, c
 }
 
 // Cluster size of a selection launch of `ntasks` sets.  A small selection (a
-// few sets) runs beside the next layer's attention, on SMs that the planner
-// leaves out of that attention's grid.  When the next layer has a large pool
-// of gathered rows (`big_pool`: at least a fifth of its tiles), its attention
-// needs the SMs more than the selection needs speed: clusters of 8.  Else
-// the selection's latency is on the critical path (the next selection waits
-// for its SMs): clusters of 16.  (Measured on B200 at 128K keys, 2 retrieval
-// heads per layer: per-head sets, pool ~1/3 of the tiles, 8 beats 16 by
-// 4.6 %; KV-group sets, pool ~1/9, 16 beats 8 by 1.2 %.)  A large selection
-// (layer 0) takes the largest size whose clusters are all resident at once,
-// so that it runs in one wave and the next layer starts right away; else the
-// smallest size.
-int pick_topk_cluster(const lyc_ctx* ctx, int ntasks, bool big_pool) {
+// few sets) takes clusters of 8 and runs beside the next layer's attention,
+// on SMs that the planner leaves out of that attention's grid: room for two
+// selections, so that the next layer's selection can start on its key flag
+// while this one still runs.  (Measured on B200 at 128K keys, 2 retrieval
+// heads per layer, against clusters of 16 with room for one: +4.2 % with
+// KV-group sets, +1.1 % per head; clusters of 4 with room for two, or of 8
+// with room for three, lose.)  A large selection (layer 0) takes the largest
+// size whose clusters are all resident at once, so that it runs in one wave
+// and the next layer starts right away; else the smallest size.
+int pick_topk_cluster(const lyc_ctx* ctx, int ntasks) {
   auto resident = [&](int cl) {
     return ctx->topk_resident[cl] > 0 ? ctx->topk_resident[cl] : ctx->sms / cl;
   };
-  if (!big_pool && ntasks * 16 <= ctx->sms / 4 && (ctx->topk_cls & (1u << 16)) && ntasks <= resident(16))
-    return 16;
-  if (ntasks * 8 <= ctx->sms / 4 && (ctx->topk_cls & (1u << 8)) && ntasks <= resident(8)) return 8;
+  if (2 * ntasks * 8 <= ctx->sms / 4 && (ctx->topk_cls & (1u << 8)) && ntasks <= resident(8)) return 8;
   int best = 0, smallest = 0;
   for (int cl : {16, 8, 4}) {
     if (!(ctx->topk_cls & (1u << cl))) continue;
@@ -598,18 +594,15 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const KvVie
     // kernel then starts late behind it.
     int avail = ctx->sms;
     if (l > 0) {
-      int64_t gathered = 0;  // this layer's tiles of gathered rows (the pool)
-      for (const Segment& sg : H.segs)
-        if (sg.kind == kSparse) gathered += (sg.rows + TR - 1) / TR;
-      hl[l - 1].topk_cl = pick_topk_cluster(ctx, static_cast<int>(hl[l - 1].tasks.size()),
-                                            5 * gathered >= NT);
       const int prev = static_cast<int>(hl[l - 1].tasks.size()) * hl[l - 1].topk_cl;
-      if (prev > 0 && prev <= ctx->sms / 4) avail = ctx->sms - prev;
+      if (prev > 0 && 2 * prev <= ctx->sms / 4) avail = ctx->sms - 2 * prev;
+      else if (prev > 0 && prev <= ctx->sms / 4) avail = ctx->sms - prev;
     }
-    // The grid leaves those SMs to the selection: the selection of this layer
-    // starts on its key flag and then needs SMs, which it gets at once when
-    // the previous selection ends (measured on B200: +1.9 % in KV-group mode
-    // against a grid with CTAs that take those SMs back for pool units).
+    // The grid leaves the SMs of the previous selection and of this layer's
+    // own to them: the selection of this layer starts on its key flag, while
+    // the previous one may still run, and takes free SMs at once (measured on
+    // B200: +1.9 % in KV-group mode for a grid that leaves one selection's SMs
+    // against one with CTAs that take them back for pool units).
     H.tiles = NT;
     const int grid = static_cast<int>(std::min<int64_t>(NT, avail));
     H.grid = grid;
@@ -709,8 +702,7 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const KvVie
         writer[s] = l;
       }
     prev_fresh = fresh;
-    // (the next layer revises this once its pool is known)
-    H.topk_cl = pick_topk_cluster(ctx, static_cast<int>(H.tasks.size()), false);
+    H.topk_cl = pick_topk_cluster(ctx, static_cast<int>(H.tasks.size()));
     for (int b = 0; b < B; ++b)
       for (int s = 0; s < Hs; ++s) H.trace_src.push_back(set_ptr(cur[s], b, s));
   }

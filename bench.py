@@ -66,6 +66,11 @@ def parse_args(argv=None):
                     help="Cache Correction instead: dense causal attention of the T most recent "
                          "positions over the cache (lyc_cache_correction), one line")
     ap.add_argument("--T", type=int, default=32, help="Cache Correction: positions refreshed")
+    ap.add_argument("--shard", choices=["heads", "batch"], default=None,
+                    help="under torchrun: split one step over the ranks (KV groups with their "
+                         "query heads, or batch elements), all-gather the outputs and sets every "
+                         "step; strong scaling.  Default: every rank runs its own replica")
+    ap.add_argument("--batch", type=int, default=1, help="batch elements of the workload")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-layers", type=int, default=2,
@@ -75,7 +80,9 @@ def parse_args(argv=None):
 
 def workload_spec(args):
     from hybrid_head_sparse_b200 import workloads as W
-    spec = W.LLAMA3_8B_128K.with_(n=args.n, k=args.k, L=args.layers)
+    spec = W.LLAMA3_8B_128K.with_(n=args.n, k=args.k, L=args.layers, B=args.batch)
+    if args.batch != 1:
+        spec = spec.with_(name=spec.name + f"-b{args.batch}")
     if args.retrieval_heads < 0:
         spec = spec.with_(roles="all", name=spec.name + "-dense")
     else:
@@ -641,6 +648,95 @@ def run_serving(args):
     return 0
 
 
+def run_sharded(args):
+    """One step split over the ranks (hybrid_head_sparse_b200/shard.py): each
+    rank runs the L-layer step on its KV groups (or batch elements) and the
+    outputs and sets are all-gathered every step (NCCL).  Total work is fixed
+    as the rank count grows (strong scaling)."""
+    import torch
+    import torch.distributed as dist
+
+    from hybrid_head_sparse_b200 import build as Bld
+    from hybrid_head_sparse_b200 import lyc, shard, workloads as W
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+    Bld.build()
+    lyc.load()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    spec = workload_spec(args)
+    data = W.make_stack(spec, dev)
+    sh = shard.shard_of(args.shard, rank, world, spec.B, spec.Hq, spec.Hkv)
+    qs, Ks, Vs, rs = shard.take(sh, data["q"], data["k"], data["v"], data["role"])
+    ss = shard.ShardedStep(sh, spec.L, spec.Hq, spec.Hkv, spec.d, spec.n, spec.k,
+                           select_mode=args.select_mode, device=local)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        return ss.step(qs, Ks, Vs, spec.n, rs, stream=stream)
+
+    for _ in range(max(args.warmup, 1)):
+        out, S = step()
+    torch.cuda.synchronize()
+    rc = ss.ctx.sync_status()
+    if rc != 0:
+        raise RuntimeError(f"device status after warm-up: {lyc.lyc_status_string(rc)}")
+    barrier()
+    torch.cuda.synchronize()
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        ev0.record(stream)
+        for _ in range(args.steps):
+            out, S = step()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    ms = max_over_ranks(ev0.elapsed_time(ev1), dev)
+    rc = ss.ctx.sync_status()
+    if rc != 0:
+        raise RuntimeError(f"device status after timing: {lyc.lyc_status_string(rc)}")
+    cfg_role = data["role"]
+    full = lyc.Lyc(spec.L, spec.B, spec.Hq, spec.Hkv, spec.d, spec.n, spec.k,
+                   select_mode=args.select_mode, device=local)
+    analytic, _ = full.step_bytes(cfg_role, spec.n, spec.k)
+    full.close()
+    ss.close()
+    ms_step = ms / args.steps
+    peak, _ = measured_peaks()
+    gbs = analytic / (ms_step / 1e3) / 1e9
+    line = {
+        "metric": METRIC + f" ({args.shard}-sharded step)", "value": args.steps / (ms / 1e3),
+        "unit": "steps/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "strong",
+        "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) q/K/V, sinks + 256 planted heavy hitters per KV head)",
+        "config": {"workload": spec.name, "L": spec.L, "B": spec.B, "Hq": spec.Hq,
+                   "Hkv": spec.Hkv, "d": spec.d, "n": spec.n, "k": spec.k,
+                   "select_mode": args.select_mode, "parallelism": f"{args.shard}-shard x{world}",
+                   "per_rank": {"kv_groups": sh.Hkv, "q_heads": sh.Hq, "batch": sh.B},
+                   "collective": "all-gather of outputs and sets per step (NCCL)"},
+        "hbm": {"analytic_bytes_per_step": analytic, "analytic_gbs_all_ranks": round(gbs, 1),
+                "frac_of_measured_peak_x_ranks": round(gbs / (peak * world), 4)},
+        "clocks": clk.summary(),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
 def run_correction(args):
     """Cache Correction on one GPU: the T most recent positions of the
     Llama3-8B-shaped stack at n tokens are attended again, densely and
@@ -874,6 +970,8 @@ def main(argv=None):
         return run_serving(args)
     if args.correction:
         return run_correction(args)
+    if args.shard:
+        return run_sharded(args)
     if args.selection != "topk":
         return run_rule(args)
     return run_lyc(args)

@@ -237,20 +237,11 @@ __device__ __forceinline__ void mma_scheduler(const AttnMmaParams& P, unsigned c
       if (!slot_free(t)) break;
       if (k >= kPoolRing && !mbar_wait(&unit_empty[r], ((k / kPoolRing) - 1) & 1, abort_flag, p.status))
         break;
-      // the next unit that holds rows (units past a shorter segment's end are skipped)
+      // the next unit, or the end (seg -1)
       pc.seg = -1;
       pc.r0 = pc.r1 = pc.ordinal = 0;
-      for (int u = atomicAdd(cursor, 1); u < p.pool_n; u = atomicAdd(cursor, 1)) {
-        const int q = u % p.pool_ups;
-        const int seg = __ldg(&p.pool_segs[u / p.pool_ups]);
-        const int rows = p.segs[seg].rows;
-        if (q * (kPoolTiles * kTileRows) >= rows) continue;
-        pc.seg = seg;
-        pc.r0 = q * (kPoolTiles * kTileRows);
-        pc.r1 = min(pc.r0 + kPoolTiles * kTileRows, rows);
-        pc.ordinal = q;
-        break;
-      }
+      const int u = atomicAdd(cursor, 1);
+      if (u < p.pool_n) pc = p.pool_units[u];
       ring[r] = pc;
       mbar_arrive(&unit_full[r]);  // release: the entry above
       if (pc.seg < 0) break;

@@ -71,8 +71,8 @@ struct LayerPlan {
   size_t off_trace_src = 0;  // copy table for the set trace after this layer
   size_t off_combine = 0;    // bf16: (segment, output) pairs combined by the next launch
   int ncombine = 0;
-  size_t off_pool = 0;       // mma kernel: the pool's segments
-  int pool_nsegs = 0, pool_ups = 0;
+  size_t off_pool = 0;       // mma kernel: the pool's units
+  int pool_n = 0;             // units in the pool
   int64_t pool_tiles = 0, tiles = 0;  // tiles in the pool, in the whole layer
   int topk_cl = 16;          // cluster size of the selection launch
   int topk_n = 0;            // keys of the longest selection task
@@ -456,8 +456,7 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const KvVie
     int nqb = 1;
     int grid = 0;
     int topk_cl = 16;           // cluster size of this layer's selection launch
-    std::vector<int32_t> pool_segs;  // mma kernel: segments of the pool, in order
-    int pool_ups = 0;                // units per pool segment
+    std::vector<Piece> pool_units;   // mma kernel: the pool's units, in order
     int64_t tiles = 0, pool_tiles = 0;
   };
   std::vector<HostLayer> hl(L);
@@ -641,18 +640,25 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const KvVie
       }
     }
     if (use_pool) {
-      // a sparse segment of r rows has ceil(r / unit) units, unit q = ordinal q;
-      // the pool counts pool_ups per segment (the most any has), and the
-      // scheduler skips the units past a shorter segment's end
-      constexpr int kUnitRows = kPoolTiles * kTileRows;
+      // a gathered segment of r rows is cut into units of kPoolTiles tiles
+      // (kPoolTilesDep for a set the previous selection writes), unit q =
+      // ordinal q; the pool lists them in order, earlier selections' sets first
       for (int dep = 0; dep < 2; ++dep)
         for (size_t s2 = 0; s2 < H.segs.size(); ++s2)
           if (H.segs[s2].kind == kSparse && H.segs[s2].dep == dep) {
-            const int units = (H.segs[s2].rows + kUnitRows - 1) / kUnitRows;
-            H.pool_segs.push_back(static_cast<int32_t>(s2));
-            H.pool_ups = std::max(H.pool_ups, units);
-            npieces[s2] = units;
-            H.pool_tiles += (H.segs[s2].rows + TR - 1) / TR;
+            const int unit_rows = (dep ? kPoolTilesDep : kPoolTiles) * kTileRows;
+            const int rows = H.segs[s2].rows;
+            int q = 0;
+            for (int r0 = 0; r0 < rows; r0 += unit_rows, ++q) {
+              Piece pc;
+              pc.seg = static_cast<int32_t>(s2);
+              pc.r0 = r0;
+              pc.r1 = std::min(r0 + unit_rows, rows);
+              pc.ordinal = q;
+              H.pool_units.push_back(pc);
+            }
+            npieces[s2] = q;
+            H.pool_tiles += (rows + TR - 1) / TR;
           }
     }
     for (int c = 0; c < grid; ++c) {
@@ -733,11 +739,10 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const KvVie
     lp.off_trace_src = take(H.trace_src.size() * sizeof(void*));
     lp.ncombine = static_cast<int>(H.combine.size());
     lp.off_combine = take(std::max<size_t>(1, H.combine.size()) * sizeof(int2));
-    lp.pool_nsegs = static_cast<int>(H.pool_segs.size());
-    lp.pool_ups = H.pool_ups;
+    lp.pool_n = static_cast<int>(H.pool_units.size());
     lp.tiles = H.tiles;
     lp.pool_tiles = H.pool_tiles;
-    lp.off_pool = take(std::max<size_t>(1, H.pool_segs.size()) * sizeof(int32_t));
+    lp.off_pool = take(std::max<size_t>(1, H.pool_units.size()) * sizeof(Piece));
     lp.keys_ctas = 0;
     for (size_t c = 0; c + 1 < H.cta.size(); ++c) lp.keys_ctas += H.cta[c + 1] > H.cta[c] ? 1 : 0;
   }
@@ -758,8 +763,8 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const KvVie
     memcpy(host.data() + lp.off_trace_src, H.trace_src.data(), H.trace_src.size() * sizeof(void*));
     if (!H.combine.empty())
       memcpy(host.data() + lp.off_combine, H.combine.data(), H.combine.size() * sizeof(int2));
-    if (!H.pool_segs.empty())
-      memcpy(host.data() + lp.off_pool, H.pool_segs.data(), H.pool_segs.size() * sizeof(int32_t));
+    if (!H.pool_units.empty())
+      memcpy(host.data() + lp.off_pool, H.pool_units.data(), H.pool_units.size() * sizeof(Piece));
   }
   memcpy(host.data() + plan->off_final_src, hl[L - 1].trace_src.data(),
          hl[L - 1].trace_src.size() * sizeof(void*));
@@ -887,9 +892,8 @@ lyc_status enqueue_step(lyc_ctx* ctx, Plan* plan, cudaStream_t stream, int set, 
       // gathered rows (mma kernel only)
       ap.done = ctx->attn_flags + 2 * l;
       ap.prev_done = l > 0 ? ctx->attn_flags + 2 * (l - 1) + 1 : nullptr;
-      ap.pool_segs = reinterpret_cast<const int32_t*>(plan->dev + lp.off_pool);
-      ap.pool_n = lp.pool_nsegs * lp.pool_ups;
-      ap.pool_ups = lp.pool_ups;
+      ap.pool_units = reinterpret_cast<const Piece*>(plan->dev + lp.off_pool);
+      ap.pool_n = lp.pool_n;
       ap.pool_stride = L + 1;
       ap.pool_cursors = ctx->pool_cursors;
       // the selection of this layer starts once the keys are written (the
@@ -1215,8 +1219,10 @@ lyc_status lyc_create(const lyc_config* cfg, lyc_ctx** out) {
   const size_t es = c.dtype == LYC_BF16 ? 2 : 4;
   const size_t nseg_max = static_cast<size_t>(B) * (Hkv + Hq);
   // pieces per layer <= 2 * sms + segments (two pooling phases), plus the
-  // pool units of the mma kernel (every sparse segment cut into units)
-  const size_t units = (static_cast<size_t>(c.max_k) + kPoolTiles * kTileRows - 1) / (kPoolTiles * kTileRows);
+  // pool units of the mma kernel (every sparse segment cut into units, at
+  // most of the smaller unit size)
+  const size_t unit_rows = static_cast<size_t>(std::min(kPoolTiles, kPoolTilesDep)) * kTileRows;
+  const size_t units = (static_cast<size_t>(c.max_k) + unit_rows - 1) / unit_rows;
   ctx->max_parts = (2 * static_cast<size_t>(ctx->sms) + nseg_max + nseg_max * units) * kMaxQ;
   ctx->max_counters = nseg_max * kMaxQ;
   auto alloc = [&](void** p, size_t bytes) -> lyc_status {

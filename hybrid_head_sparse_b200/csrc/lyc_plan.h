@@ -36,7 +36,14 @@ constexpr int kPartSlots = 4;
 // Pool of gathered rows that CTAs take at run time, kPoolTiles tiles at a
 // time; a CTA's leader publishes the pool pieces it took into a ring of
 // kPoolRing entries that every warp of the CTA reads in order.
-constexpr int kPoolTiles = 4;
+constexpr int kPoolTiles = 8;
+// Units of the sets that the previous layer's selection writes (the only
+// gathered rows that wait for a selection; taken last).  Smaller units would
+// spread them over more CTAs once that selection is done, but every unit is a
+// piece with its own partial state (measured on B200, 128K Llama3-8B stack,
+// against 8-tile units for both: KV-group sets, 4-tile units -1.2 %, 2-tile
+// -3 %, 1-tile -6 %; per head, 4-tile -1.3 %).
+constexpr int kPoolTilesDep = 8;
 constexpr int kPoolRing = 16;
 
 enum SegKind : int32_t { kDense = 0, kSparse = 1 };
@@ -109,12 +116,10 @@ struct AttnParams {
   const uint32_t* prev_done; // NULL, or the flag of the previous layer's attention launch:
                              // the epilogue waits on it (else on griddepcontrol.wait)
   // the pool (mma kernel): after its own pieces a CTA takes units u = 0, 1, ...
-  // by an atomic cursor; unit u is rows [q * kPoolTiles * 64, ...) of segment
-  // pool_segs[u / pool_ups], q = u % pool_ups, ordinal q (its partial record)
-  const int32_t* pool_segs;
+  // by an atomic cursor; unit u is the piece pool_units[u] (a row range of a
+  // gathered segment, its ordinal = its partial record)
+  const Piece* pool_units;
   int32_t pool_n;            // units in the pool (0: none)
-  int32_t pool_ups;          // units per pool segment (the most any has; a unit past a
-                             // segment's rows is skipped)
   int32_t pool_stride;       // cursors per epoch parity
   int32_t* pool_cursors;     // [2][pool_stride]: this launch's is [(epoch & 1)][layer]
   int32_t wpart_by_sm;       // 1: the piece-state ring of a CTA is the one of the SM it runs

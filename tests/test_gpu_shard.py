@@ -72,6 +72,10 @@ def test_sharded_step_world_one_is_the_step(lyc):
     S2 = torch.empty_like(S)
     whole.decode_step(data["q"], data["k"], data["v"], spec.n, data["role"], spec.k, out2, S2)
     torch.cuda.synchronize()
-    assert torch.equal(out, out2) and torch.equal(S, S2)
+    # outputs within the bf16 tolerances (which CTA takes which pool unit is
+    # decided at run time, and with it the fp32 summation order), sets exact
+    # (a tile's selection keys do not depend on who computes them)
+    P.check_out(out.cpu().numpy(), out2.cpu().numpy().astype(np.float64), "bf16", "world 1")
+    assert torch.equal(S, S2)
     st.close()
     whole.close()

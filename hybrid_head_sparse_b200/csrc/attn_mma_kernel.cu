@@ -692,9 +692,10 @@ __device__ __forceinline__ void mma_consumers(const AttnMmaParams& P, unsigned c
 //  1. first, the cross-piece combine of the previous layer: this CTA takes
 //     the (segment, output) tasks t = blockIdx.x, blockIdx.x + gridDim.x, ...
 //     and folds each output's piece partials (log-sum-exp) into that layer's
-//     output.  The previous layer's attention completed before this launch
-//     began (the selection between the two waited for it), so its partials
-//     are in place; running the combine here keeps it off the critical path;
+//     output, once the previous layer's attention launch has raised its done
+//     flag (its partials are then in place; this launch may start while that
+//     one still runs); running the combine here keeps it off the critical
+//     path;
 //  2. then, per piece of this CTA in order: wait for the NC consumer warps'
 //     states, merge them per output, and write the piece's partial (or, for a
 //     segment of one piece, the output itself).

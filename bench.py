@@ -8,7 +8,9 @@ L-layer stack (dense retrieval heads + top-k selection + sparse gathered
 heads, every layer), launched as one CUDA graph.
 
 Prints one JSON line on rank 0.  `--impl reference` times the fp64 CPU
-oracle instead (a bounded sample of the same workload, host cores).
+oracle instead: whole L-layer steps of the same workload on the host cores.
+`--workload` picks the Llama3-8B-shaped stack at 128K (default) or 32K, or the
+Qwen3-8B-shaped stack (36 layers, batch 4, 64K, k=2048).
 Multi-GPU (torchrun): every rank runs its own replica of the step (the path
 has no exchange step); value = all ranks' steps / the slowest rank's time.
 """
@@ -40,11 +42,16 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["lyc", "reference"], default="lyc")
-    ap.add_argument("--n", type=int, default=131072)
-    ap.add_argument("--k", type=int, default=4096)
-    ap.add_argument("--layers", type=int, default=32, help="layers of the stack (32 = the workload)")
-    ap.add_argument("--retrieval-heads", type=int, default=2,
-                    help="retrieval query heads per layer after layer 0; -1 = all (dense baseline)")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="llama3-8b-128k",
+                    help="llama3-8b-128k (32 layers, n=131072, k=4096, 2 retrieval heads per "
+                         "layer: the headline), llama3-8b-32k (n=32768), qwen3-8b-64k-b4 (36 "
+                         "layers, batch 4, n=65536, k=2048, 3 retrieval heads per layer)")
+    ap.add_argument("--n", type=int, default=None, help="context length (default: the workload's)")
+    ap.add_argument("--k", type=int, default=None, help="token budget (default: the workload's)")
+    ap.add_argument("--layers", type=int, default=None, help="layers (default: the workload's)")
+    ap.add_argument("--retrieval-heads", type=int, default=None,
+                    help="retrieval query heads per layer after layer 0 (default: the "
+                         "workload's); -1 = all (the all-retrieval dense baseline)")
     ap.add_argument("--select-mode", choices=["per_qhead", "kvgroup_mean"], default="kvgroup_mean",
                     help="kvgroup_mean: one set per KV group, keyed by the group's mean query (the "
                          "pages' GQA handling, whose bytes are the analytic floor); per_qhead: one "
@@ -70,25 +77,62 @@ def parse_args(argv=None):
                     help="under torchrun: split one step over the ranks (KV groups with their "
                          "query heads, or batch elements), all-gather the outputs and sets every "
                          "step; strong scaling.  Default: every rank runs its own replica")
-    ap.add_argument("--batch", type=int, default=1, help="batch elements of the workload")
+    ap.add_argument("--batch", type=int, default=None, help="batch elements (default: the workload's)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--cpu-layers", type=int, default=2,
-                    help="oracle sample: layers 0..cpu_layers-1 of the step")
+    ap.add_argument("--no-other-mode", action="store_true",
+                    help="skip timing the selection mode not chosen")
+    ap.add_argument("--sustained-ms", type=float, default=500.0,
+                    help="after the K timed steps, replay for at least this long with the clock "
+                         "sampler still running (a longer sample of the same step; reported "
+                         "apart from the timed value)")
     return ap.parse_args(argv)
 
 
+# workload choice -> (spec name in workloads.py, family prefix of the line's name)
+WORKLOADS = {"llama3-8b-128k": ("LLAMA3_8B_128K", "llama3-8b"),
+             "llama3-8b-32k": ("LLAMA3_8B_32K", "llama3-8b"),
+             "qwen3-8b-64k-b4": ("QWEN3_8B_64K_B4", "qwen3-8b")}
+
+
 def workload_spec(args):
+    """The chosen workload with the command line's overrides; its name spells
+    out the shape that differs from nothing: batch (when > 1), n, k, layers
+    (when not the workload's), retrieval heads per layer (or dense)."""
     from hybrid_head_sparse_b200 import workloads as W
-    spec = W.LLAMA3_8B_128K.with_(n=args.n, k=args.k, L=args.layers, B=args.batch)
-    if args.batch != 1:
-        spec = spec.with_(name=spec.name + f"-b{args.batch}")
-    if args.retrieval_heads < 0:
-        spec = spec.with_(roles="all", name=spec.name + "-dense")
-    else:
-        spec = spec.with_(retrieval_per_layer=args.retrieval_heads,
-                          name=spec.name + f"-r{args.retrieval_heads}")
-    return spec
+    attr, family = WORKLOADS[args.workload]
+    base = getattr(W, attr)
+    over = {}
+    for key, val in (("n", args.n), ("k", args.k), ("L", args.layers), ("B", args.batch)):
+        if val is not None:
+            over[key] = val
+    spec = base.with_(**over)
+    r = base.retrieval_per_layer if args.retrieval_heads is None else args.retrieval_heads
+    name = f"{family}-attn-stack" + (f"-b{spec.B}" if spec.B != 1 else "") + f"-n{spec.n}-k{spec.k}"
+    if spec.L != base.L:
+        name += f"-L{spec.L}"
+    if r < 0:
+        return spec.with_(roles="all", name=name + "-dense")
+    return spec.with_(retrieval_per_layer=r, name=name + f"-r{r}")
+
+
+def retrieval_heads(spec) -> int:
+    return -1 if spec.roles == "all" else spec.retrieval_per_layer
+
+
+def line_config(spec, args, world: int, kv_bytes: int) -> dict:
+    """The `config` of a line: the same for the library arm and the oracle arm."""
+    return {"workload": spec.name, "L": spec.L, "B": spec.B, "Hq": spec.Hq, "Hkv": spec.Hkv,
+            "d": spec.d, "n": spec.n, "k": spec.k,
+            "retrieval_heads_per_layer": retrieval_heads(spec),
+            "select_mode": args.select_mode, "attn_kernel": args.attn_kernel,
+            "parallelism": f"replicas x{world}",
+            "l2": "inputs larger than L2 (KV cache %.1f GB per GPU)" % (kv_bytes / 1e9)}
+
+
+def kv_cache_bytes(spec) -> int:
+    es = 2 if spec.dtype == "bf16" else 4
+    return 2 * spec.L * spec.B * spec.Hkv * spec.rows * spec.d * es
 
 
 def measured_peaks():
@@ -227,19 +271,13 @@ class ClockSampler:
 # ---------------------------------------------------------------- oracle timing
 
 
-def oracle_sample_seconds(spec, host_stack, cpu_layers: int):
-    """Time the oracle on layers 0..cpu_layers-1 (full n, every head) and
-    scale to one whole step: layer 0 + (L-1) x the mean of the later layers."""
+def oracle_step_seconds(spec, host_stack) -> float:
+    """Wall time of one whole L-layer step of the oracle (every layer, every
+    head, full n) on the host cores."""
     import oracle as O
-    times = []
-    S = None
-    for l in range(cpu_layers):
-        t0 = time.perf_counter()
-        _, S, _, _ = O.layer(host_stack, l, spec.k, S, all_retrieval=(l == 0), n=spec.n)
-        times.append(time.perf_counter() - t0)
-    later = times[1:] if len(times) > 1 else times
-    est = times[0] + (spec.L - 1) * (sum(later) / len(later))
-    return est, times
+    t0 = time.perf_counter()
+    O.decode_step(host_stack, spec.k, n=spec.n)
+    return time.perf_counter() - t0
 
 
 def cpu_cores() -> int:
@@ -252,56 +290,90 @@ def cpu_cores() -> int:
         return os.cpu_count() or 1
 
 
-def host_sample_stack(spec, data, cpu_layers: int, select_mode: str = "per_qhead"):
+def host_stack(spec, data, select_mode: str):
+    """Host copy of the whole step's inputs for the oracle."""
     import oracle as O
     from hybrid_head_sparse_b200 import workloads as W
-    layers = list(range(cpu_layers))
     mode = O.SELECT_KVGROUP_MEAN if select_mode == "kvgroup_mean" else O.SELECT_PER_QHEAD
-    return O.Stack(W.host_view(data["q"][layers]), W.host_view(data["k"][layers]),
-                   W.host_view(data["v"][layers]), data["role"][layers].copy(), mode)
+    return O.Stack(W.host_view(data["q"]), W.host_view(data["k"]), W.host_view(data["v"]),
+                   data["role"].copy(), mode)
 
 
-def sample_text(spec, cpu_layers):
-    return (f"oracle (fp64 C, OpenMP) on layers 0..{cpu_layers - 1} of one step at full size "
-            f"(n={spec.n}, k={spec.k}, all {spec.Hq} heads); step time = layer 0 + "
-            f"{spec.L - 1} x mean(later sampled layers)")
+def sample_text(spec, steps: int):
+    return (f"oracle (fp64 C, OpenMP over heads) on {steps} whole step(s) of the same workload: "
+            f"all {spec.L} layers, every head, n={spec.n}, k={spec.k}, same seeded inputs")
+
+
+def oracle_baseline(spec, hs, steps: int, single_core: bool) -> dict:
+    """cpu_baseline object: `steps` whole oracle steps on every host core, and
+    (single_core) one more whole step on one core."""
+    import oracle as O
+    cores = O.max_threads()
+    secs = [oracle_step_seconds(spec, hs) for _ in range(steps)]
+    sec = sum(secs) / len(secs)
+    res = {"value": 1.0 / sec, "unit": "steps/s", "cores": cores, "kind": "oracle",
+           "sample": sample_text(spec, steps), "step_seconds": [round(t, 3) for t in secs]}
+    if single_core:
+        O.set_threads(1)
+        try:
+            s1 = oracle_step_seconds(spec, hs)
+        finally:
+            O.set_threads(cores)
+        res["single_core"] = {"value": 1.0 / s1, "unit": "steps/s", "cores": 1,
+                              "step_seconds": round(s1, 3)}
+    return res
+
+
+def union_ms(iv) -> float:
+    """Length (ms) of the union of (start ns, end ns) intervals."""
+    tot = 0
+    cur_s = cur_e = None
+    for a, b in sorted(iv):
+        if cur_e is None or a > cur_e:
+            if cur_e is not None:
+                tot += cur_e - cur_s
+            cur_s, cur_e = a, b
+        else:
+            cur_e = max(cur_e, b)
+    if cur_e is not None:
+        tot += cur_e - cur_s
+    return tot / 1e6
 
 
 # ---------------------------------------------------------------- reference arm
 
 
 def run_reference(args):
+    """The oracle arm: whole L-layer steps of the fp64 oracle on the host
+    cores, on the library arm's workload, metric and config.  Rank 0 only."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
+    import torch
+
     import oracle as O
     from hybrid_head_sparse_b200 import workloads as W
     O.build()
     spec = workload_spec(args)
-    cl = max(1, min(args.cpu_layers, spec.L))
-    sample = W.make_stack(spec.with_(L=cl), "cpu")
-    st = host_sample_stack(spec, sample, cl, args.select_mode)
+    # the same seeded recipe as the library arm (drawn on the GPU when there
+    # is one, as the library arm does, then copied to the host)
+    data = W.make_stack(spec, "cuda" if torch.cuda.is_available() else "cpu")
+    hs = host_stack(spec, data, args.select_mode)
+    del data
     for _ in range(args.warmup):
-        oracle_sample_seconds(spec, st, cl)
-    ests = []
-    for _ in range(args.steps):
-        est, _ = oracle_sample_seconds(spec, st, cl)
-        ests.append(est)
-    sec = sum(ests) / len(ests)
+        oracle_step_seconds(spec, hs)
+    secs = [oracle_step_seconds(spec, hs) for _ in range(args.steps)]
+    sec = sum(secs) / len(secs)
     value = 1.0 / sec
-    cores = cpu_cores()
+    cores = O.max_threads()
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "steps/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": sec * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": spec.name, "L": spec.L, "B": spec.B, "Hq": spec.Hq,
-                   "Hkv": spec.Hkv, "d": spec.d, "n": spec.n, "k": spec.k,
-                   "retrieval_heads_per_layer": args.retrieval_heads,
-                   "select_mode": args.select_mode},
+        "config": line_config(spec, args, args.gpus, kv_cache_bytes(spec)),
         "cpu_baseline": {"value": value, "unit": "steps/s", "cores": cores, "kind": "oracle",
-                         "sample": sample_text(spec, cl) + "; inputs drawn on the host with the "
-                         "same recipe"},
+                         "sample": sample_text(spec, args.steps)},
         "e2e": {"value": value, "unit": "steps/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -341,9 +413,9 @@ def run_lyc(args):
     spec = workload_spec(args)
     data = W.make_stack(spec, dev)
     torch.cuda.synchronize()
+    kflags = lyc.LYC_CFG_TCGEN05 if args.attn_kernel == "tcgen05" else 0
     ctx = lyc.Lyc(spec.L, spec.B, spec.Hq, spec.Hkv, spec.d, spec.n, spec.k, dtype=spec.dtype,
-                  select_mode=args.select_mode, device=local,
-                  flags=lyc.LYC_CFG_TCGEN05 if args.attn_kernel == "tcgen05" else 0)
+                  select_mode=args.select_mode, device=local, flags=kflags)
     out = torch.empty((spec.L, spec.B, spec.Hq, spec.d), device=dev)
     S = torch.empty((spec.B, ctx.Hs, spec.k), dtype=torch.int32, device=dev)
     role = data["role"]
@@ -359,7 +431,10 @@ def run_lyc(args):
     if rc != 0:
         raise RuntimeError(f"device status after warm-up: {lyc.lyc_status_string(rc)}")
 
-    # ---- timed region: K graph replays, device-timed, max over ranks
+    # ---- timed region: K graph replays, device-timed, max over ranks.  The
+    # clock sampler keeps running through a longer window of the same replays
+    # right after it (reported apart), so that the clock record is not three
+    # samples of a 20 ms region.
     ev0 = torch.cuda.Event(enable_timing=True)
     ev1 = torch.cuda.Event(enable_timing=True)
     barrier()
@@ -371,55 +446,104 @@ def run_lyc(args):
             step()
             evs[i + 1].record(stream)
         torch.cuda.synchronize()
-    barrier()
+        barrier()
+        ms_total_local = evs[0].elapsed_time(evs[-1])
+        n_sus = max(args.steps, int(args.sustained_ms / max(ms_total_local / args.steps, 1e-3)) + 1)
+        ev0.record(stream)
+        for _ in range(n_sus):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize()
     clocks = clk.summary()
-    ms_total = max_over_ranks(evs[0].elapsed_time(evs[-1]), dev)
+    ms_total = max_over_ranks(ms_total_local, dev)
+    ms_sus = max_over_ranks(ev0.elapsed_time(ev1), dev)
     step_ms = percentiles([evs[i].elapsed_time(evs[i + 1]) for i in range(args.steps)])
     ms_step = ms_total / args.steps
     value = job_steps_per_s(world, args.steps, ms_total)
+    sustained = {"replays": n_sus, "ms_per_step": ms_sus / n_sus,
+                 "value": job_steps_per_s(world, n_sus, ms_sus), "unit": "steps/s",
+                 "note": "the same step replayed right after the timed region, clocks sampled "
+                         "through both"}
     rc = ctx.sync_status()
     if rc != 0:
         raise RuntimeError(f"device status after timing: {lyc.lyc_status_string(rc)}")
 
-    # ---- per-kernel device times: the same K steps again with event nodes in the graph
-    ctx.set_timing(True)
+    analytic, distinct = ctx.step_bytes(role, spec.n, spec.k)
+    peak, peak_kind = measured_peaks()
+    per_layer = spec.L
+
+    # ---- where the step's time goes: the same K replays with the device
+    # timeline on (every CTA of the attention and selection launches records
+    # its start and end on the GPU's global timer).  The attention kernel's
+    # share of the step is the union of its CTAs' busy intervals over the
+    # span; its time per step is that share of the timed ms_per_step, so it
+    # can never exceed the step.
+    cap = args.steps * (spec.L + 1) * (2 * 148 + 64)
+    tl = torch.zeros(1 + 3 * cap, dtype=torch.int64, device=dev)
+    ctx.set_timeline(tl, cap)
     step()
     torch.cuda.synchronize()
-    ctx.kernel_times()
+    tl.zero_()
+    torch.cuda.synchronize()
     ev0.record(stream)
     for _ in range(args.steps):
         step()
     ev1.record(stream)
     torch.cuda.synchronize()
-    ms_step_timed = ev0.elapsed_time(ev1) / args.steps
+    ms_step_tl = ev0.elapsed_time(ev1) / args.steps
+    ctx.set_timeline(None, 0)
+    rec = tl.cpu().numpy()
+    nrec = int(min(rec[0], cap))
+    r3 = rec[1:1 + 3 * nrec].reshape(-1, 3)
+    kinds = (r3[:, 2] >> 32) & 0xffff
+    att = [(int(a), int(b)) for a, b, kd in zip(r3[:, 0], r3[:, 1], kinds) if kd == 0]
+    sel = [(int(a), int(b)) for a, b, kd in zip(r3[:, 0], r3[:, 1], kinds) if kd == 1]
+    span_ms = (r3[:, 1].max() - r3[:, 0].min()) / 1e6 if nrec else float("nan")
+    attn_share = union_ms(att) / span_ms if nrec else float("nan")
+    sel_share = union_ms(sel) / span_ms if nrec else float("nan")
+    attn_ms_step = attn_share * ms_step
+    achieved = distinct / (attn_ms_step / 1e3) / 1e9
+    traffic = profiled_traffic(spec.name, args.select_mode)
+
+    # ---- the same launches one at a time: event nodes retargeted into the
+    # graph serialise them, so each one is timed alone (no overlap)
+    ctx.set_timing(True)
+    step()
+    torch.cuda.synchronize()
+    ctx.kernel_times()
+    for _ in range(args.steps):
+        step()
+    torch.cuda.synchronize()
     ktimes = ctx.kernel_times()
     ctx.set_timing(False)
-    nsteps_t = args.steps
-    attn_ms = sum(t[2] for t in ktimes if t[0] == 0) / nsteps_t
-    topk_ms = sum(t[2] for t in ktimes if t[0] == 1) / nsteps_t
-    # attention launches: one per layer plus the launch that combines the last
-    # layer's split rows; the roofline's per-launch figures are per layer
-    attn_launches = sum(1 for t in ktimes if t[0] == 0) // nsteps_t
-    topk_launches = sum(1 for t in ktimes if t[0] == 1) // nsteps_t
-    per_layer = spec.L
+    iso_attn_ms = sum(t[2] for t in ktimes if t[0] == 0) / args.steps
+    iso_topk_ms = sum(t[2] for t in ktimes if t[0] == 1) / args.steps
+    attn_launches = sum(1 for t in ktimes if t[0] == 0) // args.steps
+    topk_launches = sum(1 for t in ktimes if t[0] == 1) // args.steps
 
-    analytic, distinct = ctx.step_bytes(role, spec.n, spec.k)
-    peak, peak_kind = measured_peaks()
-    achieved = distinct / (attn_ms / 1e3) / 1e9
-    traffic = profiled_traffic(spec.name, args.select_mode)
     roofline = {
         "bound": "hbm",
         "kernel": ("attn_tc_layer_kernel" if args.attn_kernel == "tcgen05" else "attn_mma_layer_kernel")
                   + " (pooled dense + sparse attention, one launch per layer)",
         "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-        "frac": round(achieved / peak, 4), "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
+        "frac": round(achieved / peak, 4),
+        "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs), burst figure",
         "traffic": traffic,
         "algorithmic_bytes_per_launch": distinct / per_layer,
-        "avg_launch_ms": attn_ms / per_layer,
-        "note": ("achieved = K+V bytes the kernel must read (dense groups: n rows; each sparse pass: "
-                 "k rows) / CUDA-event time of the attention launches (one per layer, plus the "
-                 "small launch that combines the last layer's split rows), per layer, over K "
-                 "timed steps"),
+        "avg_launch_ms": attn_ms_step / per_layer,
+        "attn_share_of_step": round(attn_share, 4),
+        "selection_share_of_step": round(sel_share, 4),
+        "note": ("achieved = K+V bytes the attention kernel must read per step (dense groups: n "
+                 "rows; each sparse pass: k rows) / its time per step; its time per step = the "
+                 "union of its CTAs' busy intervals on the device timeline (same K replays), as "
+                 "a share of the span, times the timed ms_per_step.  Launches of consecutive "
+                 "layers overlap, so the per-launch figure is that time / L"),
+        "isolated_launches": {
+            "attn_ms_per_step": iso_attn_ms, "topk_ms_per_step": iso_topk_ms,
+            "attn_gbs": round(distinct / (iso_attn_ms / 1e3) / 1e9, 1),
+            "note": "each launch timed alone by event nodes in the graph, which serialise the "
+                    "launches (no overlap between layers): an upper bound on launch time"},
+        "timeline_ms_per_step": ms_step_tl,
     }
     step_gbs = analytic / (ms_step / 1e3) / 1e9
 
@@ -455,11 +579,10 @@ def run_lyc(args):
 
     # ---- the other selection mode on the same inputs (its steps/s and byte rates)
     other = None
-    if not args.serving and args.selection == "topk":
+    if not args.no_other_mode:
         omode = "per_qhead" if args.select_mode == "kvgroup_mean" else "kvgroup_mean"
         octx = lyc.Lyc(spec.L, spec.B, spec.Hq, spec.Hkv, spec.d, spec.n, spec.k, dtype=spec.dtype,
-                       select_mode=omode, device=local,
-                       flags=lyc.LYC_CFG_TCGEN05 if args.attn_kernel == "tcgen05" else 0)
+                       select_mode=omode, device=local, flags=kflags)
         oS = torch.empty((spec.B, octx.Hs, spec.k), dtype=torch.int32, device=dev)
 
         def ostep():
@@ -488,16 +611,14 @@ def run_lyc(args):
                  "kernel_bytes_per_step": odi,
                  "kernel_gbs": round(odi / (oms_step / 1e3) / 1e9, 1)}
 
-    # ---- the oracle on the host cores (rank 0, one GPU only)
+    # ---- the oracle on the host cores (rank 0, one GPU only): whole steps
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle as O
         O.build()
-        cl = max(1, min(args.cpu_layers, spec.L))
-        st = host_sample_stack(spec, data, cl, args.select_mode)
-        est, times = oracle_sample_seconds(spec, st, cl)
-        cpu = {"value": 1.0 / est, "unit": "steps/s", "cores": cpu_cores(), "kind": "oracle",
-               "sample": sample_text(spec, cl) + f"; sampled layer seconds {[round(t, 3) for t in times]}"}
+        hs = host_stack(spec, data, args.select_mode)
+        cpu = oracle_baseline(spec, hs, steps=1, single_core=True)
+        del hs
 
     launches_per_step = attn_launches + topk_launches + 1
     line = {
@@ -505,21 +626,16 @@ def run_lyc(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
         "step_ms_distribution": {k: round(v, 4) for k, v in step_ms.items()},
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16", "data": "synthetic (seeded N(0,1) q/K/V, sinks + 256 planted heavy hitters per KV head)",
-        "config": {"workload": spec.name, "L": spec.L, "B": spec.B, "Hq": spec.Hq,
-                   "Hkv": spec.Hkv, "d": spec.d, "n": spec.n, "k": spec.k,
-                   "retrieval_heads_per_layer": args.retrieval_heads,
-                   "select_mode": args.select_mode, "attn_kernel": args.attn_kernel,
-                   "parallelism": f"replicas x{world}",
-                   "l2": "inputs larger than L2 (KV cache %.1f GB per GPU)" % (
-                       2 * data["k"].numel() * data["k"].element_size() / 1e9)},
+        "dtype": "bf16" if spec.dtype == "bf16" else "f32",
+        "data": "synthetic (seeded N(0,1) q/K/V, sinks + 256 planted heavy hitters per KV head)",
+        "config": line_config(spec, args, world, kv_cache_bytes(spec)),
         "hbm": {"analytic_bytes_per_step": analytic, "kernel_bytes_per_step": distinct,
                 "analytic_gbs": round(step_gbs, 1),
                 "frac_of_measured_peak": round(step_gbs / peak, 4),
-                "frac_of_8tbs": round(step_gbs / NOMINAL_HBM_GBS, 4)},
+                "frac_of_8tbs": round(step_gbs / NOMINAL_HBM_GBS, 4),
+                "kernel_gbs": round(distinct / (ms_step / 1e3) / 1e9, 1)},
         "roofline": roofline,
-        "kernels": {"attn_ms_per_step": attn_ms, "topk_ms_per_step": topk_ms,
-                    "ms_per_step_with_event_nodes": ms_step_timed},
+        "sustained": sustained,
         "other_select_mode": other,
         "cpu_baseline": cpu,
         "e2e": e2e,
@@ -634,7 +750,7 @@ def run_serving(args):
         "data": "synthetic (seeded N(0,1) pages, q and appended rows; shuffled 64-row pages)",
         "config": {"workload": "llama3-8b-serving-b4-paged64", "L": L, "B": B, "Hq": Hq,
                    "Hkv": Hkv, "d": d, "n": n_list, "k": k, "page_rows": page_rows,
-                   "retrieval_heads_per_layer": args.retrieval_heads,
+                   "retrieval_heads_per_layer": retrieval_heads(base),
                    "select_mode": args.select_mode, "append": True, "parallelism": "replicas x1",
                    "l2": "inputs larger than L2 (KV pages %.1f GB)" % (
                        2 * Kp.numel() * Kp.element_size() / 1e9)},
@@ -947,7 +1063,7 @@ def run_rule(args):
         "data": "synthetic (seeded N(0,1) q/K/V, sinks + 256 planted heavy hitters per KV head)",
         "config": {"workload": spec.name, "L": spec.L, "B": spec.B, "Hq": spec.Hq, "Hkv": spec.Hkv,
                    "d": spec.d, "n": spec.n, "k_capacity": spec.k, "selection": args.selection,
-                   **params, "retrieval_heads_per_layer": args.retrieval_heads,
+                   **params, "retrieval_heads_per_layer": retrieval_heads(spec),
                    "select_mode": args.select_mode, "parallelism": "replicas x1",
                    "l2": "inputs larger than L2 (KV cache %.1f GB)" % (
                        2 * data["k"].numel() * data["k"].element_size() / 1e9)},

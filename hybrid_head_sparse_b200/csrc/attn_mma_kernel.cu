@@ -482,6 +482,7 @@ __device__ __forceinline__ void mma_consumers(const AttnMmaParams& P, unsigned c
   const bf16_t* q = static_cast<const bf16_t*>(p.q);
   const float sl2 = p.scale_log2;
   const int mi = lane >> 3, r8 = lane & 7;  // ldmatrix: matrix and row this lane addresses
+  const int wq = p.wpart_q > 0 ? p.wpart_q : kMaxQ;  // query rows per ring record
 
   int t = 0;  // CTA-wide tile sequence number
   const int nhome = pend - pbeg;
@@ -663,7 +664,7 @@ __device__ __forceinline__ void mma_consumers(const AttnMmaParams& P, unsigned c
       const int slot = pi % kPartSlots;
       if (pi >= kPartSlots)
         mbar_wait(&slot_free[slot], ((pi / kPartSlots) - 1) & 1, abort_flag, p.status);
-      const int64_t rec = ((static_cast<int64_t>(cta_ring(p)) * kPartSlots + slot) * NC + w) * kMaxQ;
+      const int64_t rec = ((static_cast<int64_t>(cta_ring(p)) * kPartSlots + slot) * NC + w) * wq;
       if (g == 0) {
         if (out0) p.wpart_ml[rec + q0] = make_float2(m0, l0);
         if (out1) p.wpart_ml[rec + q1] = make_float2(m1, l1);
@@ -752,6 +753,7 @@ __device__ __forceinline__ void mma_epilogue(const AttnMmaParams& P, unsigned ch
   uint64_t* slot_full = bars + 2 * STAGES + C::IR;
   uint64_t* slot_free = slot_full + kPartSlots;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_FLAGS);
+  const int wq = p.wpart_q > 0 ? p.wpart_q : kMaxQ;  // query rows per ring record
 
   // ---- 1. the previous layer's cross-piece combine, after that launch has
   // completed.  The wait also comes before any partial of this launch is
@@ -798,7 +800,7 @@ __device__ __forceinline__ void mma_epilogue(const AttnMmaParams& P, unsigned ch
     const int nout = sg.nout;
     const int slot = pi % kPartSlots;
     if (!mbar_wait(&slot_full[slot], (pi / kPartSlots) & 1, abort_flag, p.status)) return;
-    const int64_t rec0 = (static_cast<int64_t>(cta_ring(p)) * kPartSlots + slot) * NC * kMaxQ;
+    const int64_t rec0 = (static_cast<int64_t>(cta_ring(p)) * kPartSlots + slot) * NC * wq;
     // load every output's NC warp states first (all in flight), then merge
     for (int o0 = 0; o0 < nout; o0 += 2) {
       float2 ml[2][NC];
@@ -808,8 +810,8 @@ __device__ __forceinline__ void mma_epilogue(const AttnMmaParams& P, unsigned ch
         const int r = sg.out_row[min(o0 + h, nout - 1)];
 #pragma unroll
         for (int ww = 0; ww < NC; ++ww) {
-          ml[h][ww] = p.wpart_ml[rec0 + ww * kMaxQ + r];
-          ov[h][ww] = col ? *reinterpret_cast<const float4*>(p.wpart_o + (rec0 + ww * kMaxQ + r) * D + lane * 4)
+          ml[h][ww] = p.wpart_ml[rec0 + ww * wq + r];
+          ov[h][ww] = col ? *reinterpret_cast<const float4*>(p.wpart_o + (rec0 + ww * wq + r) * D + lane * 4)
                           : make_float4(0.f, 0.f, 0.f, 0.f);
         }
       }

@@ -41,7 +41,7 @@ int attn_tc_tile_rows();
 size_t topk_smem_for(int cl, int n);
 int topk_pick_cluster(size_t smem);
 cudaError_t topk_configure(int cl, size_t smem);
-cudaError_t topk_launch(int cl, const TopkParams* p, int ntasks, cudaStream_t stream);
+cudaError_t topk_launch(int cl, const TopkParams* p, int ntasks, cudaStream_t stream, bool force_var);
 int topk_max_clusters(int cl, size_t smem);
 cudaError_t copy_sets_launch(const CopySetsParams* p, cudaStream_t stream);
 cudaError_t append_rows_launch(const AppendParams* p, cudaStream_t stream);
@@ -68,7 +68,6 @@ struct LayerPlan {
   size_t off_segs = 0, off_pieces = 0, off_cta = 0;
   int ntasks = 0;
   size_t off_tasks = 0;
-  size_t off_trace_src = 0;  // copy table for the set trace after this layer
   size_t off_combine = 0;    // bf16: (segment, output) pairs combined by the next launch
   int ncombine = 0;
   size_t off_pool = 0;       // mma kernel: the pool's units
@@ -84,6 +83,10 @@ struct Plan {
   unsigned char* dev = nullptr;  // all records of all layers
   size_t dev_bytes = 0;
   size_t off_final_src = 0;      // copy table: current buffer of each set -> caller S
+  // set trace: the selections write their rows of it; one copy at the end of
+  // the step fills the rows of the sets a layer did not refresh
+  size_t off_fill_src = 0, off_fill_dst = 0;
+  int nfill = 0;
   int nsets = 0;
   int combine_grid = 1;       // bf16: CTAs of the launch that combines the last layer
   size_t off_empty_cta = 0;   // its CTA offsets (all zero: no pieces)
@@ -451,7 +454,7 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const KvVie
     std::vector<int32_t> cta;
     std::vector<TopkTask> tasks;
     int topk_n = 0;
-    std::vector<const int32_t*> trace_src;
+    std::vector<const int32_t*> final_src;  // the current buffer of each set after the layer
     std::vector<int2> combine;  // bf16: (segment, output) left to the next launch
     int nqb = 1;
     int grid = 0;
@@ -467,6 +470,16 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const KvVie
   const char* kbase = static_cast<const char*>(kv.k);
   const char* vbase = static_cast<const char*>(kv.v);
 
+  // the set trace [L][B][Hs][k]: row (l, b, s) holds the set slot s passes on
+  // after layer l.  A refreshed slot's row is written by its selection; the
+  // others are copies of the row of the slot's last writer (or of S^(0) in
+  // set-input mode), made by one launch at the end of the step.
+  auto trace_row = [&](int l, int b, int s) -> int32_t* {
+    if (!plan->trace) return nullptr;
+    return plan->trace + ((static_cast<int64_t>(l) * B + b) * Hs + s) * k;
+  };
+  std::vector<const int32_t*> fill_src;
+  std::vector<int32_t*> fill_dst;
   std::vector<char> prev_fresh(Hs, 1);  // slots the previous layer's selection wrote
   std::vector<int> writer(Hs, -1);      // layer whose selection wrote each slot's current set
   auto ready_flag = [&](int s, int b) -> const uint32_t* {
@@ -691,6 +704,7 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const KvVie
         tk.keys = ctx->keys + keys_base + (static_cast<int64_t>(b) * Hs + s) * ctx->nstride;
         tk.S = set_ptr(1 - cur[s], b, s);
         tk.done = ctx->flags + ((static_cast<int64_t>(l) * B + b) * Hs + s) * 2;
+        tk.trace = trace_row(l, b, s);
         tk.n = static_cast<int32_t>(kv.n[b]);
         tk.k = select_cap(kv.n[b]);
         if (sel.rule == LYC_RULE_BLOCK_TOPK) {
@@ -702,6 +716,14 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const KvVie
         H.tasks.push_back(tk);
       }
     }
+    if (plan->trace)
+      for (int b = 0; b < B; ++b)
+        for (int s = 0; s < Hs; ++s) {
+          if (fresh[s]) continue;
+          fill_dst.push_back(trace_row(l, b, s));
+          fill_src.push_back(writer[s] >= 0 ? trace_row(writer[s], b, s)
+                                            : plan->S + (static_cast<int64_t>(b) * Hs + s) * k);
+        }
     for (int s = 0; s < Hs; ++s)
       if (fresh[s]) {
         cur[s] ^= 1;
@@ -710,7 +732,7 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const KvVie
     prev_fresh = fresh;
     H.topk_cl = pick_topk_cluster(ctx, static_cast<int>(H.tasks.size()));
     for (int b = 0; b < B; ++b)
-      for (int s = 0; s < Hs; ++s) H.trace_src.push_back(set_ptr(cur[s], b, s));
+      for (int s = 0; s < Hs; ++s) H.final_src.push_back(set_ptr(cur[s], b, s));
   }
 
   // ---- one device buffer for every record
@@ -736,7 +758,6 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const KvVie
     lp.off_cta = take(H.cta.size() * sizeof(int32_t));
     lp.off_tasks = take(std::max<size_t>(1, H.tasks.size()) * sizeof(TopkTask));
     lp.topk_n = H.topk_n;
-    lp.off_trace_src = take(H.trace_src.size() * sizeof(void*));
     lp.ncombine = static_cast<int>(H.combine.size());
     lp.off_combine = take(std::max<size_t>(1, H.combine.size()) * sizeof(int2));
     lp.pool_n = static_cast<int>(H.pool_units.size());
@@ -746,7 +767,10 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const KvVie
     lp.keys_ctas = 0;
     for (size_t c = 0; c + 1 < H.cta.size(); ++c) lp.keys_ctas += H.cta[c + 1] > H.cta[c] ? 1 : 0;
   }
-  plan->off_final_src = take(hl[L - 1].trace_src.size() * sizeof(void*));
+  plan->off_final_src = take(hl[L - 1].final_src.size() * sizeof(void*));
+  plan->nfill = static_cast<int>(fill_src.size());
+  plan->off_fill_src = take(std::max<size_t>(1, fill_src.size()) * sizeof(void*));
+  plan->off_fill_dst = take(std::max<size_t>(1, fill_dst.size()) * sizeof(void*));
   plan->off_n = take(static_cast<size_t>(B) * sizeof(int64_t));
   // the last layer's combine runs in a launch of its own, whose CTAs have no pieces
   plan->combine_grid = std::max(1, std::min(ctx->sms, plan->layers[L - 1].ncombine));
@@ -760,14 +784,17 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const KvVie
     memcpy(host.data() + lp.off_cta, H.cta.data(), H.cta.size() * sizeof(int32_t));
     if (!H.tasks.empty())
       memcpy(host.data() + lp.off_tasks, H.tasks.data(), H.tasks.size() * sizeof(TopkTask));
-    memcpy(host.data() + lp.off_trace_src, H.trace_src.data(), H.trace_src.size() * sizeof(void*));
     if (!H.combine.empty())
       memcpy(host.data() + lp.off_combine, H.combine.data(), H.combine.size() * sizeof(int2));
     if (!H.pool_units.empty())
       memcpy(host.data() + lp.off_pool, H.pool_units.data(), H.pool_units.size() * sizeof(Piece));
   }
-  memcpy(host.data() + plan->off_final_src, hl[L - 1].trace_src.data(),
-         hl[L - 1].trace_src.size() * sizeof(void*));
+  memcpy(host.data() + plan->off_final_src, hl[L - 1].final_src.data(),
+         hl[L - 1].final_src.size() * sizeof(void*));
+  if (!fill_src.empty()) {
+    memcpy(host.data() + plan->off_fill_src, fill_src.data(), fill_src.size() * sizeof(void*));
+    memcpy(host.data() + plan->off_fill_dst, fill_dst.data(), fill_dst.size() * sizeof(void*));
+  }
   memcpy(host.data() + plan->off_n, kv.n.data(), static_cast<size_t>(B) * sizeof(int64_t));
   LYC_CUDA(cudaMalloc(&plan->dev, bytes), "cudaMalloc(plan)");
   plan->dev_bytes = bytes;
@@ -961,16 +988,10 @@ lyc_status enqueue_step(lyc_ctx* ctx, Plan* plan, cudaStream_t stream, int set, 
         tp.prev_done = l > 0 ? ctx->attn_flags + 2 * (l - 1) + 1 : nullptr;
       }
       if ((st = record_event(ctx, plan, set, ev++, stream, capturing)) != LYC_OK) return st;
-      LYC_CUDA(topk_launch(lp.topk_cl, &tp, lp.ntasks, stream), "top-k launch");
+      LYC_CUDA(topk_launch(lp.topk_cl, &tp, lp.ntasks, stream, false), "top-k launch");
       if ((st = record_event(ctx, plan, set, ev++, stream, capturing)) != LYC_OK) return st;
       plan->kernel_kind.push_back(1);
       plan->kernel_layer.push_back(l);
-    }
-    if (plan->trace) {
-      CopySetsParams cp{reinterpret_cast<const int32_t* const*>(plan->dev + lp.off_trace_src),
-                        plan->trace + static_cast<size_t>(l) * B * ctx->Hs * plan->k, B * ctx->Hs,
-                        plan->k};
-      LYC_CUDA(copy_sets_launch(&cp, stream), "trace copy");
     }
   }
   if (dtype == 0) {
@@ -1009,8 +1030,18 @@ lyc_status enqueue_step(lyc_ctx* ctx, Plan* plan, cudaStream_t stream, int set, 
     plan->kernel_kind.push_back(0);
     plan->kernel_layer.push_back(L - 1);
   }
+  if (plan->trace && plan->nfill > 0) {
+    // the trace rows of the sets a layer passed on unchanged (before the final
+    // copy: in set-input mode some of them come from the caller's S^(0))
+    CopySetsParams fp{};
+    fp.src = reinterpret_cast<const int32_t* const*>(plan->dev + plan->off_fill_src);
+    fp.dsts = reinterpret_cast<int32_t* const*>(plan->dev + plan->off_fill_dst);
+    fp.nsets = plan->nfill;
+    fp.k = plan->k;
+    LYC_CUDA(copy_sets_launch(&fp, stream), "trace fill");
+  }
   CopySetsParams cp{reinterpret_cast<const int32_t* const*>(plan->dev + plan->off_final_src), plan->S,
-                    B * ctx->Hs, plan->k, ctx->epoch, ctx->pool_cursors, L + 1};
+                    B * ctx->Hs, plan->k, ctx->epoch, ctx->pool_cursors, L + 1, nullptr};
   LYC_CUDA(copy_sets_launch(&cp, stream), "final set copy");
   return LYC_OK;
 }
@@ -1715,11 +1746,18 @@ lyc_status lyc_kernel_times(lyc_ctx* ctx, lyc_kernel_time* times, int cap, int* 
   return LYC_OK;
 }
 
-lyc_status lyc_topk_f32(lyc_ctx* ctx, const float* keys, int64_t n, int k, int32_t* S, void* stream) {
+lyc_status lyc_topk_f32_ex(lyc_ctx* ctx, const float* keys, int64_t n, int k, int32_t* S, int cluster,
+                           int variant, void* stream) {
   if (!ctx) return LYC_ERR_INVALID_ARG;
   if (!keys || !S) return fail(ctx, LYC_ERR_INVALID_ARG, "NULL pointer");
   if (n < 1 || n > ctx->cfg.max_ctx) return fail(ctx, LYC_ERR_INVALID_ARG, "n outside [1, max_ctx]");
   if (k < 1 || k > ctx->cfg.max_k) return fail(ctx, LYC_ERR_INVALID_ARG, "k outside [1, max_k]");
+  if (variant != LYC_TOPK_FIXED && variant != LYC_TOPK_RULES)
+    return fail(ctx, LYC_ERR_INVALID_ARG, "unknown selection instantiation");
+  const int cl = cluster == 0 ? ctx->topk_cl : cluster;
+  if (cl != 4 && cl != 8 && cl != 16) return fail(ctx, LYC_ERR_INVALID_ARG, "cluster size not in {4, 8, 16}");
+  if (!(ctx->topk_cls & (1u << cl)))
+    return fail(ctx, LYC_ERR_UNSUPPORTED, "cluster size not configured for this context's max_ctx");
   DeviceGuard guard(ctx->cfg.device);
   TopkParams tp{};
   tp.tasks = nullptr;
@@ -1727,9 +1765,14 @@ lyc_status lyc_topk_f32(lyc_ctx* ctx, const float* keys, int64_t n, int k, int32
   tp.single.S = S;
   tp.n = static_cast<int>(n);
   tp.k = k;
-  LYC_CUDA(topk_launch(ctx->topk_cl, &tp, 1, static_cast<cudaStream_t>(stream)), "top-k launch");
+  LYC_CUDA(topk_launch(cl, &tp, 1, static_cast<cudaStream_t>(stream), variant == LYC_TOPK_RULES),
+           "top-k launch");
   ctx->last_stream = static_cast<cudaStream_t>(stream);
   return LYC_OK;
+}
+
+lyc_status lyc_topk_f32(lyc_ctx* ctx, const float* keys, int64_t n, int k, int32_t* S, void* stream) {
+  return lyc_topk_f32_ex(ctx, keys, n, k, S, 0, LYC_TOPK_FIXED, stream);
 }
 
 lyc_status lyc_step_bytes(const lyc_config* cfg, const uint8_t* role_mask, int64_t n, int k, int s_in,

@@ -126,6 +126,8 @@ struct AttnParams {
                              // on (CTAs of consecutive launches may overlap in time); 0: of
                              // its block index
   int32_t wpart_slots;       // rings allocated
+  int32_t wpart_q;           // query rows per consumer-warp record of the ring (0: kMaxQ); a
+                             // caller whose segments all have one query row passes 1
   int32_t timeline_cap;
   uint32_t* keys_done;       // NULL, or {arrival counter, flag} of this launch's selection
                              // keys: each consumer warp of the first keys_ctas CTAs arrives
@@ -145,6 +147,9 @@ struct AttnParams {
 struct TopkTask {
   const float* keys;  // n selection keys
   int32_t* S;         // the launch's k outputs
+  int32_t* trace;     // NULL, or a second destination that receives the same k entries
+                      // (the set trace: written by the selection itself, so that tracing
+                      // adds no launch between the layers)
   uint32_t* done;     // NULL, or {arrival counter, ready flag}: the last CTA of the task
                       // to finish resets the counter and sets the flag to epoch + 1
   int32_t n;          // keys of this task (a batch element's rows; its blocks with expand > 1);
@@ -227,7 +232,8 @@ struct WriteRowsParams {
 constexpr unsigned long long kTagAttention = 0ull;
 constexpr unsigned long long kTagTopk = 1ull;
 
-// copy_sets_kernel: dst[(b*Hs + s)*k + j] = src[b*Hs + s][j] for j < k
+// copy_sets_kernel: dst[(b*Hs + s)*k + j] = src[b*Hs + s][j] for j < k, or
+// with a destination list, dsts[i][j] = src[i][j]
 struct CopySetsParams {
   const int32_t* const* src;
   int32_t* dst;
@@ -235,6 +241,7 @@ struct CopySetsParams {
   uint32_t* epoch;  // the step's last launch: advance the epoch once the copy is done (or NULL)
   int32_t* pool_cursors;  // with epoch: zero the next step's pool cursors, [2][pool_stride]
   int32_t pool_stride;
+  int32_t* const* dsts;  // NULL, or one destination per set (dst is then unused)
 };
 
 // append_rows_kernel: the current token's K and V ([L][B][Hkv][row_bytes]

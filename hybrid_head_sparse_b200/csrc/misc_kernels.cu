@@ -11,7 +11,7 @@ namespace lyc {
 __global__ void copy_sets_kernel(const CopySetsParams p) {
   const int set = blockIdx.x;
   const int32_t* src = p.src[set];
-  int32_t* dst = p.dst + static_cast<int64_t>(set) * p.k;
+  int32_t* dst = p.dsts ? p.dsts[set] : p.dst + static_cast<int64_t>(set) * p.k;
   for (int j = threadIdx.x; j < p.k; j += blockDim.x) dst[j] = src[j];
   // the step's last launch (every launch of the step has completed before it
   // starts, and the next step's launches start after it ends): the next

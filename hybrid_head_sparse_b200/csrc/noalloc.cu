@@ -1,6 +1,7 @@
 // noalloc.cu -- lyc_sparse_attention_noalloc: the sparse-head attention of
-// one layer (page "LycheeDecode ...", paper-graph-ui summary, section 3.4
-// Eq. 3) for callers that cannot allocate device memory.
+// one layer for callers that cannot allocate device memory.  The paper has no
+// counterpart for this entry point; the arithmetic is the library's sparse
+// head, o = softmax(q K[S]^T / sqrt(d)) V[S] over the rows of a given set.
 //
 // Who needs it: code that runs where a cudaMalloc is not allowed or not
 // acceptable -- inside a framework whose caching allocator owns all device
@@ -15,10 +16,12 @@
 // work lists, partial softmax states, the per-CTA ring of consumer-warp
 // states, arrival counters, the status word -- lives in one file-scope
 // device array of fixed size, g_noalloc_scratch.  Its address is looked up
-// once per device with cudaGetSymbolAddress.  Per call the host builds the
-// work list in a fixed host buffer and copies it in; the counters and the
-// status word are cleared on the stream first.  No cudaMalloc, cudaFree or
-// allocating library routine is called.
+// once per device with cudaGetSymbolAddress.  Per call a small kernel on the
+// caller's stream writes the work list into the array and clears the
+// counters and the status word (the call's sizes and pointers are its
+// by-value arguments), so a call enqueues kernels and one status copy only:
+// no host-to-device copy, no cudaMalloc, cudaFree or allocating library
+// routine.
 //
 // Every call shares the array, which keeps the last call's contents: calls
 // that may overlap on the GPU (two streams, two host threads without an
@@ -48,7 +51,8 @@ cudaError_t attn_mma_dispatch(int D, const AttnMmaParams* P, int grid, cudaStrea
 
 namespace {
 
-// Limits of one call (they size the array below).
+// Limits of one call (they size the array below).  Every segment has one
+// query row, so the consumer-warp ring keeps one row per warp record.
 constexpr int kNaMaxSets = LYC_NOALLOC_MAX_SETS;   // batch * query heads
 constexpr int kNaMaxCtas = LYC_NOALLOC_MAX_CTAS;   // CTAs of the attention launch
 constexpr int kNaMaxD = 128;
@@ -70,7 +74,8 @@ constexpr size_t kOffStatus = kOffCounters + sizeof(int32_t) * kNaMaxCounters;
 constexpr size_t kZeroBytes = align256(kOffStatus + 16) - kOffCounters;
 constexpr size_t kOffPartO = kOffCounters + kZeroBytes;
 constexpr size_t kOffPartMl = align256(kOffPartO + sizeof(float) * kNaMaxParts * kNaMaxD);
-constexpr size_t kRingRecs = static_cast<size_t>(kNaMaxCtas) * kPartSlots * kMaxConsumerWarps * kMaxQ;
+constexpr int kNaRingQ = 1;  // query rows per consumer-warp record (AttnParams::wpart_q)
+constexpr size_t kRingRecs = static_cast<size_t>(kNaMaxCtas) * kPartSlots * kMaxConsumerWarps * kNaRingQ;
 constexpr size_t kOffWpartO = align256(kOffPartMl + sizeof(float2) * kNaMaxParts);
 constexpr size_t kOffWpartMl = align256(kOffWpartO + sizeof(float) * kRingRecs * kNaMaxD);
 constexpr size_t kScratchUsed = align256(kOffWpartMl + sizeof(float2) * kRingRecs);
@@ -96,8 +101,129 @@ struct DeviceState {
 std::mutex g_mu;
 DeviceState g_dev[kMaxDevices];
 EncodeTiledFn g_encode = nullptr;
-// host staging of one call's work list (guarded by g_mu)
-unsigned char g_host_plan[kPlanBytes];
+
+// The CTA whose run of tiles holds tile T, when NT tiles are cut into `grid`
+// equal runs [NT*c/grid, NT*(c+1)/grid): the largest c with
+// floor(NT*c/grid) <= T.
+__host__ __device__ inline int64_t cta_of_tile(int64_t T, int64_t NT, int64_t grid) {
+  return ((T + 1) * grid + NT - 1) / NT - 1;
+}
+
+// One call's work list, computed by the plan kernel below (and its sizes by
+// the host, with the same formulas): one gathered segment per (b, h) of
+// tiles_per 64-row tiles, the NT = nsets * tiles_per tiles cut into equal
+// runs, one per CTA (the pooling of the full step); a run that crosses
+// segments becomes several pieces.
+struct NaPlanArgs {
+  unsigned char* base;        // device address of g_noalloc_scratch
+  const unsigned char* kc;    // K and V of the cache (bf16)
+  const unsigned char* vc;
+  const int32_t* S;           // [B][Hq][k]
+  int64_t s_batch, s_head, s_token;
+  int64_t NT;                 // tiles of the call
+  int32_t B, Hq, G, k, keff, n;
+  int32_t tiles_per;          // tiles of one segment
+  int32_t grid, cgrid;        // CTAs of the attention and of the combine launch
+};
+
+constexpr int kNaPlanThreads = 512;
+static_assert(kNaPlanThreads >= kNaMaxSets && kNaPlanThreads >= kNaMaxCtas, "one thread per set and CTA");
+
+// Exclusive prefix sum of one value per thread over the block; *total gets the sum.
+__device__ int na_block_scan(int v, int* tmp, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int inc = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += y;
+  }
+  if (lane == 31) tmp[warp] = inc;
+  __syncthreads();
+  int before = 0, all = 0;
+  for (int w = 0; w < kNaPlanThreads / 32; ++w) {
+    before += w < warp ? tmp[w] : 0;
+    all += tmp[w];
+  }
+  __syncthreads();
+  *total = all;
+  return before + inc - v;
+}
+
+__global__ void __launch_bounds__(kNaPlanThreads) noalloc_plan_kernel(const NaPlanArgs a) {
+  __shared__ int tmp[kNaPlanThreads / 32];
+  const int t = threadIdx.x;
+  const int nsets = a.B * a.Hq;
+  const int64_t tp = a.tiles_per;
+  // counters and status word start at zero
+  uint32_t* zero = reinterpret_cast<uint32_t*>(a.base + kOffCounters);
+  for (size_t i = t; i < kZeroBytes / 4; i += kNaPlanThreads) zero[i] = 0u;
+  // per segment: the CTAs its tiles fall in
+  int npieces = 0;
+  int64_t cfirst = 0;
+  if (t < nsets) {
+    cfirst = cta_of_tile(t * tp, a.NT, a.grid);
+    npieces = static_cast<int>(cta_of_tile((t + 1) * tp - 1, a.NT, a.grid) - cfirst + 1);
+  }
+  // per CTA: the segments its run crosses
+  int64_t t0 = 0, t1 = 0, s0 = 0;
+  int mine = 0;
+  if (t < a.grid) {
+    t0 = a.NT * t / a.grid;
+    t1 = a.NT * (t + 1) / a.grid;
+    s0 = t0 / tp;
+    mine = static_cast<int>((t1 - 1) / tp - s0 + 1);
+  }
+  int parts = 0, pieces = 0, ntasks = 0;
+  const int part_base = na_block_scan(npieces, tmp, &parts);
+  const int task_pos = na_block_scan(npieces > 1 ? 1 : 0, tmp, &ntasks);
+  const int piece0 = na_block_scan(mine, tmp, &pieces);
+  Segment* segs = reinterpret_cast<Segment*>(a.base + kOffSegs);
+  Piece* pcs = reinterpret_cast<Piece*>(a.base + kOffPieces);
+  int32_t* cta = reinterpret_cast<int32_t*>(a.base + kOffCta);
+  int2* tasks = reinterpret_cast<int2*>(a.base + kOffTasks);
+  int32_t* empty_cta = reinterpret_cast<int32_t*>(a.base + kOffEmptyCta);
+  if (t < nsets) {
+    const int b = t / a.Hq, h = t % a.Hq, g = h / a.G;
+    const int64_t off = b * a.s_batch + g * a.s_head;
+    Segment sg{};
+    sg.k = a.kc + off * 2;
+    sg.v = a.vc + off * 2;
+    sg.idx = a.S + static_cast<int64_t>(t) * a.k;
+    sg.s_token = a.s_token;
+    for (int j = 0; j < kMaxQ; ++j) sg.key_off[j] = -1;
+    sg.key_mean_off = -1;
+    sg.kind = kSparse;
+    sg.b = b;
+    sg.g = g;
+    sg.rows = a.keff;
+    sg.nvalid = a.n;
+    sg.nq = sg.nout = 1;
+    sg.dep = 1;  // the caller's sets: read after whatever ran before on the stream
+    sg.head[0] = h;
+    sg.part_base = part_base;
+    sg.npieces = npieces;
+    sg.cnt_base = t;
+    segs[t] = sg;
+    if (npieces > 1) tasks[task_pos] = make_int2(t, 0);
+  }
+  if (t < a.grid) {
+    cta[t] = piece0;
+    for (int i = 0; i < mine; ++i) {
+      const int64_t si = s0 + i;
+      const int64_t lo = (t0 > si * tp ? t0 : si * tp) - si * tp;
+      const int64_t hi = (t1 < (si + 1) * tp ? t1 : (si + 1) * tp) - si * tp;
+      Piece pc;
+      pc.seg = static_cast<int32_t>(si);
+      pc.r0 = static_cast<int32_t>(lo * kTileRows);
+      pc.r1 = static_cast<int32_t>(hi * kTileRows < a.keff ? hi * kTileRows : a.keff);
+      pc.ordinal = static_cast<int32_t>(t - cta_of_tile(si * tp, a.NT, a.grid));
+      pcs[piece0 + i] = pc;
+    }
+  }
+  if (t == 0) cta[a.grid] = pieces;
+  if (t <= a.cgrid) empty_cta[t] = 0;
+}
 
 // Once per device, with that device current: the array's address, the
 // driver's tensor-map encoder and the kernel's shared-memory attribute.
@@ -181,76 +307,44 @@ extern "C" lyc_status lyc_sparse_attention_noalloc(const void* q, const lyc_kv_c
   lyc_status st = setup_device(dev, &ds);
   if (st != LYC_OK) return st;
 
-  // ---- work list: one gathered segment per (b, h), its rows cut into equal
-  // runs of 64-row tiles, one run per CTA (the pooling of the full step)
+  // ---- the work list's sizes (the plan kernel builds the list itself)
   unsigned char* dbase = ds->scratch;
-  Segment* segs = reinterpret_cast<Segment*>(g_host_plan + kOffSegs);
-  Piece* pieces = reinterpret_cast<Piece*>(g_host_plan + kOffPieces);
-  int32_t* cta = reinterpret_cast<int32_t*>(g_host_plan + kOffCta);
   const int tiles_per = (keff + kTileRows - 1) / kTileRows;
   const int64_t NT = static_cast<int64_t>(tiles_per) * nsets;
   int sms = 0;
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return LYC_ERR_CUDA;
   const int grid = static_cast<int>(std::min<int64_t>({NT, static_cast<int64_t>(kNaMaxCtas),
                                                        static_cast<int64_t>(sms)}));
-  for (int b = 0; b < B; ++b) {
-    for (int h = 0; h < Hq; ++h) {
-      Segment& sg = segs[b * Hq + h];
-      memset(&sg, 0, sizeof sg);
-      const int g = h / G;
-      const int64_t off = b * kv->s_batch + g * kv->s_head;
-      sg.k = static_cast<const unsigned char*>(kv->k) + off * 2;
-      sg.v = static_cast<const unsigned char*>(kv->v) + off * 2;
-      sg.idx = S + static_cast<int64_t>(b * Hq + h) * k;
-      sg.s_token = kv->s_token;
-      for (int j = 0; j < kMaxQ; ++j) sg.key_off[j] = -1;
-      sg.key_mean_off = -1;
-      sg.kind = kSparse;
-      sg.l = 0;
-      sg.b = b;
-      sg.g = g;
-      sg.rows = keff;
-      sg.nvalid = static_cast<int32_t>(n);
-      sg.nq = sg.nout = 1;
-      sg.dep = 1;  // the caller's sets: read after whatever ran before on the stream
-      sg.head[0] = h;
-      sg.out_row[0] = 0;
-    }
-  }
-  int npc = 0;
-  {
-    int64_t si = 0;
-    for (int c = 0; c < grid; ++c) {
-      cta[c] = npc;
-      const int64_t t0 = NT * c / grid, t1 = NT * (c + 1) / grid;
-      for (si = t0 / tiles_per; si < nsets && si * tiles_per < t1; ++si) {
-        const int64_t a = std::max(t0, si * tiles_per) - si * tiles_per;
-        const int64_t e = std::min(t1, (si + 1) * tiles_per) - si * tiles_per;
-        if (e <= a) continue;
-        Piece& pc = pieces[npc++];
-        pc.seg = static_cast<int32_t>(si);
-        pc.r0 = static_cast<int32_t>(a * kTileRows);
-        pc.r1 = static_cast<int32_t>(std::min<int64_t>(e * kTileRows, keff));
-        pc.ordinal = segs[si].npieces++;
-      }
-    }
-    cta[grid] = npc;
-  }
-  if (npc > kNaMaxPieces) return LYC_ERR_SCRATCH_LIMIT;
-  // partials: one per piece; segments cut into several pieces are combined
-  // by a second launch of the same kernel, one (segment, output 0) task each
-  int2* tasks = reinterpret_cast<int2*>(g_host_plan + kOffTasks);
-  int32_t* empty_cta = reinterpret_cast<int32_t*>(g_host_plan + kOffEmptyCta);
-  int part = 0, ntasks = 0;
+  int64_t part = 0;
+  int ntasks = 0;
   for (int s = 0; s < nsets; ++s) {
-    segs[s].part_base = part;
-    segs[s].cnt_base = s;
-    part += segs[s].npieces;
-    if (segs[s].npieces > 1) tasks[ntasks++] = make_int2(s, 0);
+    const int64_t np = cta_of_tile(static_cast<int64_t>(s + 1) * tiles_per - 1, NT, grid) -
+                       cta_of_tile(static_cast<int64_t>(s) * tiles_per, NT, grid) + 1;
+    part += np;
+    ntasks += np > 1 ? 1 : 0;
   }
-  if (part > kNaMaxParts) return LYC_ERR_SCRATCH_LIMIT;
+  // pieces = partials (one output each); a cut of NT tiles into `grid` runs
+  // and nsets segments has at most grid + nsets - 1 of them
+  if (part > kNaMaxParts || part > kNaMaxPieces) return LYC_ERR_SCRATCH_LIMIT;
   const int cgrid = std::max(1, std::min(ntasks, grid));
-  for (int c = 0; c <= cgrid; ++c) empty_cta[c] = 0;
+  NaPlanArgs pa;
+  pa.base = dbase;
+  pa.kc = static_cast<const unsigned char*>(kv->k);
+  pa.vc = static_cast<const unsigned char*>(kv->v);
+  pa.S = S;
+  pa.s_batch = kv->s_batch;
+  pa.s_head = kv->s_head;
+  pa.s_token = kv->s_token;
+  pa.NT = NT;
+  pa.B = B;
+  pa.Hq = Hq;
+  pa.G = G;
+  pa.k = k;
+  pa.keff = keff;
+  pa.n = n;
+  pa.tiles_per = tiles_per;
+  pa.grid = grid;
+  pa.cgrid = cgrid;
 
   AttnMmaParams mp;
   memset(&mp, 0, sizeof mp);
@@ -272,6 +366,8 @@ extern "C" lyc_status lyc_sparse_attention_noalloc(const void* q, const lyc_kv_c
   ap.wpart_ml = reinterpret_cast<float2*>(dbase + kOffWpartMl);
   ap.wpart_by_sm = 0;  // one ring per CTA: the two launches of a call never overlap on an SM ring
   ap.wpart_slots = kNaMaxCtas;
+  ap.wpart_q = kNaRingQ;
+  ap.wait_prev = 1;    // the plan kernel's work list is complete before any CTA reads it
   ap.status = reinterpret_cast<uint32_t*>(dbase + kOffStatus);
   ap.timeline = nullptr;
   ap.timeline_cap = 0;
@@ -293,11 +389,10 @@ extern "C" lyc_status lyc_sparse_attention_noalloc(const void* q, const lyc_kv_c
   cmp.p.prev_part_ml = ap.part_ml;
   cmp.p.prev_out = out;
 
-  // ---- enqueue: work list in, counters and status cleared, the kernel, the
-  // combine, the status out
-  if (cudaMemcpyAsync(dbase, g_host_plan, kPlanBytes, cudaMemcpyHostToDevice, stream) != cudaSuccess ||
-      cudaMemsetAsync(dbase + kOffCounters, 0, kZeroBytes, stream) != cudaSuccess ||
-      attn_mma_dispatch(D, &mp, grid, stream, nullptr, false) != cudaSuccess)
+  // ---- enqueue: the work list (and cleared counters and status), the
+  // kernel, the combine, the status out
+  noalloc_plan_kernel<<<1, kNaPlanThreads, 0, stream>>>(pa);
+  if (cudaGetLastError() != cudaSuccess || attn_mma_dispatch(D, &mp, grid, stream, nullptr, false) != cudaSuccess)
     return LYC_ERR_CUDA;
   if (ntasks > 0 && attn_mma_dispatch(D, &cmp, cgrid, stream, nullptr, false) != cudaSuccess)
     return LYC_ERR_CUDA;

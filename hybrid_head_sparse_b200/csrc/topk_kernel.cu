@@ -388,20 +388,26 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster_kernel(const Top
   uint32_t* ctf = reinterpret_cast<uint32_t*>(mtf + 3 * kFineBins);
 
   // the output: selected key j at position pos (its rows with block selection)
+  // (and the same entry into the trace row, when there is one)
+  int32_t* const trace = task.trace;
+  auto store = [&](int64_t pos, int32_t v) {
+    task.S[pos] = v;
+    if (trace) trace[pos] = v;
+  };
   auto put = [&](uint32_t pos, int32_t j) {
     if (E == 1) {
-      task.S[pos] = j;
+      store(pos, j);
     } else {
       for (int t = 0; t < E; ++t) {
         const int64_t r = static_cast<int64_t>(j) * E + t;
-        task.S[static_cast<int64_t>(pos) * E + t] = r < rows ? static_cast<int32_t>(r) : -1;
+        store(static_cast<int64_t>(pos) * E + t, r < rows ? static_cast<int32_t>(r) : -1);
       }
     }
   };
   auto all_selected = [&]() {  // every key is selected
     for (int x = tid; x < cnt; x += kTopkThreads) put(static_cast<uint32_t>(lo + x), lo + x);
     if (rank == 0)
-      for (int x = keff * E + tid; x < k; x += kTopkThreads) task.S[x] = -1;
+      for (int x = keff * E + tid; x < k; x += kTopkThreads) store(x, -1);
     topk_signal_done<CL>(p, task, tid);
     if (tid == 0)
       timeline_record(p.timeline, p.timeline_cap, t_start,
@@ -908,7 +914,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster_kernel(const Top
   else
     emit([&](int x) { return make_uint2(us[x], static_cast<uint32_t>(lo + x)); }, cnt);
   if (rank == 0)
-    for (int x = keff * E + tid; x < k; x += kTopkThreads) task.S[x] = -1;
+    for (int x = keff * E + tid; x < k; x += kTopkThreads) store(x, -1);
   topk_signal_done<CL>(p, task, tid);
   if (tid == 0)
     timeline_record(p.timeline, p.timeline_cap, t_start,
@@ -927,7 +933,7 @@ static size_t topk_smem_bytes(int cl, int n) {
 
 template <int CL>
 static cudaError_t topk_run(const TopkParams* p, int ntasks, cudaStream_t stream, bool configure_only,
-                            size_t max_smem) {
+                            size_t max_smem, bool force_var = false) {
   if (configure_only) {
     for (auto kern : {topk_cluster_kernel<CL, false>, topk_cluster_kernel<CL, true>}) {
       cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -941,7 +947,7 @@ static cudaError_t topk_run(const TopkParams* p, int ntasks, cudaStream_t stream
     }
     return cudaSuccess;
   }
-  const bool var = p->size_rule != kSizeFixed || p->expand > 1;
+  const bool var = force_var || p->size_rule != kSizeFixed || p->expand > 1;
   auto kern = var ? topk_cluster_kernel<CL, true> : topk_cluster_kernel<CL, false>;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(CL, ntasks, 1);
@@ -1026,11 +1032,13 @@ cudaError_t topk_configure(int cl, size_t smem) {
   return cudaErrorInvalidValue;
 }
 
-cudaError_t topk_launch(int cl, const TopkParams* p, int ntasks, cudaStream_t stream) {
+// force_var: run the instantiation of the size rules even for a fixed k
+// (test hook: the same selection through both instantiations)
+cudaError_t topk_launch(int cl, const TopkParams* p, int ntasks, cudaStream_t stream, bool force_var) {
   switch (cl) {
-    case 16: return topk_run<16>(p, ntasks, stream, false, 0);
-    case 8: return topk_run<8>(p, ntasks, stream, false, 0);
-    case 4: return topk_run<4>(p, ntasks, stream, false, 0);
+    case 16: return topk_run<16>(p, ntasks, stream, false, 0, force_var);
+    case 8: return topk_run<8>(p, ntasks, stream, false, 0, force_var);
+    case 4: return topk_run<4>(p, ntasks, stream, false, 0, force_var);
   }
   return cudaErrorInvalidValue;
 }

@@ -49,9 +49,12 @@ LYC_RULE_BLOCK_TOPK = 2
 LYC_RULE_TOPP = 3
 LYC_RULE_THRESHOLD = 4
 
+LYC_TOPK_FIXED = 0
+LYC_TOPK_RULES = 1
+
 EXPORTED = ["lyc_create", "lyc_decode_step", "lyc_decode_step_host", "lyc_decode_step_batch",
             "lyc_sync_status",
-            "lyc_set_s_trace", "lyc_step_bytes", "lyc_topk_f32", "lyc_set_timing",
+            "lyc_set_s_trace", "lyc_step_bytes", "lyc_topk_f32", "lyc_topk_f32_ex", "lyc_set_timing",
             "lyc_kernel_times", "lyc_set_timeline", "lyc_status_string", "lyc_last_error",
             "lyc_destroy", "lyc_sparse_attention_noalloc", "lyc_set_selection", "lyc_cache_correction"]
 
@@ -124,6 +127,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     L.lyc_step_bytes.argtypes = [ctypes.POINTER(lyc_config), P, ctypes.c_int64, I, I,
                                  ctypes.POINTER(ctypes.c_uint64), ctypes.POINTER(ctypes.c_uint64)]
     L.lyc_topk_f32.argtypes = [P, P, ctypes.c_int64, I, P, P]
+    L.lyc_topk_f32_ex.argtypes = [P, P, ctypes.c_int64, I, P, I, I, P]
     L.lyc_set_timing.argtypes = [P, I]
     L.lyc_set_timeline.argtypes = [P, P, I]
     L.lyc_kernel_times.argtypes = [P, ctypes.POINTER(lyc_kernel_time), I, ctypes.POINTER(I)]
@@ -205,6 +209,10 @@ def lyc_step_bytes(cfg: lyc_config, role_mask: np.ndarray, n: int, k: int, s_in:
 
 def lyc_topk_f32(ctx, keys, n, k, S, stream) -> int:
     return load().lyc_topk_f32(ctx, keys, n, k, S, stream)
+
+
+def lyc_topk_f32_ex(ctx, keys, n, k, S, cluster, variant, stream) -> int:
+    return load().lyc_topk_f32_ex(ctx, keys, n, k, S, cluster, variant, stream)
 
 
 def lyc_set_timing(ctx, mode: int) -> int:
@@ -394,9 +402,16 @@ class Lyc:
         self._check(lyc_set_timeline(self.ctx, None if buf is None else buf.data_ptr(), cap),
                     "lyc_set_timeline")
 
-    def topk_f32(self, keys, n, k, S, stream=None):
-        self._check(lyc_topk_f32(self.ctx, keys.data_ptr(), n, k, S.data_ptr(),
-                                 _stream_ptr(stream)), "lyc_topk_f32")
+    def topk_f32(self, keys, n, k, S, stream=None, cluster=None, variant=LYC_TOPK_FIXED):
+        """The selection kernel alone; cluster (4, 8, 16) and variant choose its
+        launch form (lyc_topk_f32_ex), None the context's default."""
+        if cluster is None and variant == LYC_TOPK_FIXED:
+            self._check(lyc_topk_f32(self.ctx, keys.data_ptr(), n, k, S.data_ptr(),
+                                     _stream_ptr(stream)), "lyc_topk_f32")
+        else:
+            self._check(lyc_topk_f32_ex(self.ctx, keys.data_ptr(), n, k, S.data_ptr(),
+                                        cluster or 0, variant, _stream_ptr(stream)),
+                        "lyc_topk_f32_ex")
 
     def step_bytes(self, role_mask, n, k, s_in=False):
         return lyc_step_bytes(self.cfg, role_mask, n, k, s_in)

@@ -275,7 +275,11 @@ lyc_status lyc_sync_status(lyc_ctx* ctx);
 
 /* Record every layer's outgoing sets: trace is device [L][B][Hs][k] int32
  * (k of the steps that follow); trace[l] = the sets after layer l.  NULL turns
- * recording off.  Debug and test use; it adds one small copy per layer. */
+ * recording off.  Debug and test use.  The selection kernels write the rows of
+ * the sets they refresh as they write the sets themselves, and one copy launch
+ * at the end of the step fills the rows of the sets that a layer passed on
+ * unchanged, so a traced step runs the same launches between its layers as an
+ * untraced one. */
 lyc_status lyc_set_s_trace(lyc_ctx* ctx, int32_t* trace);
 
 /* Bytes one step must read from the KV cache (host-only arithmetic).
@@ -294,6 +298,21 @@ lyc_status lyc_step_bytes(const lyc_config* cfg, const uint8_t* role_mask, int64
  * pointers (keys float32 [n], S int32 [k]); n <= max_ctx, k <= max_k. */
 lyc_status lyc_topk_f32(lyc_ctx* ctx, const float* keys, int64_t n, int k, int32_t* S,
                         void* stream);
+
+/* The same test hook with the selection kernel's launch form chosen:
+ *   cluster  4, 8 or 16 CTAs per set (the sizes the step uses: 4 for a layer
+ *            with many sets, 8 beside the next layer's attention, 16 alone), or
+ *            0 for the context's default (what lyc_topk_f32 uses);
+ *   variant  LYC_TOPK_FIXED: the fixed-k instantiation (every top-k step);
+ *            LYC_TOPK_RULES: the instantiation that carries the size rules and
+ *            block selection, run here with a fixed k.
+ * Both compute the same set.  Errors: INVALID_ARG (as lyc_topk_f32, or an
+ * unknown cluster size or variant), UNSUPPORTED (that cluster size does not
+ * fit this context's max_ctx in shared memory). */
+#define LYC_TOPK_FIXED 0
+#define LYC_TOPK_RULES 1
+lyc_status lyc_topk_f32_ex(lyc_ctx* ctx, const float* keys, int64_t n, int k, int32_t* S,
+                           int cluster, int variant, void* stream);
 
 /* Per-kernel device time of the steps since the last call, from CUDA events
  * recorded around every launch when timing is on (LYC_TIMING_ON).  Writes up
@@ -328,9 +347,9 @@ lyc_status lyc_set_timeline(lyc_ctx* ctx, unsigned long long* buf, int cap);
  * cannot hold a context; this entry point needs none and calls no cudaMalloc,
  * cudaFree or allocating library routine.
  *
- * It computes the sparse-head attention of one layer, the same arithmetic as
- * a sparse head of lyc_decode_step (paper-graph-ui summary, section 3.4
- * Eq. 3), bf16 inputs: for every batch element b and query head h,
+ * It computes the attention of sparse heads over given sets, one layer, the
+ * same arithmetic as a sparse head of lyc_decode_step, bf16 inputs: for every
+ * batch element b and query head h,
  *   out[b][h] = softmax(q[b][h] K[S[b][h]]^T / sqrt(d)) V[S[b][h]]
  * over the first min(k, n) entries of the set S[b][h] (entries past n are the
  * -1 padding of k > n), with query head h reading KV head h / (Hq / Hkv).
@@ -347,10 +366,12 @@ lyc_status lyc_set_timeline(lyc_ctx* ctx, unsigned long long* buf, int cap);
  * the launch uses at most LYC_NOALLOC_MAX_CTAS CTAs.  Larger requests return
  * LYC_ERR_SCRATCH_LIMIT and enqueue nothing.
  * Scratch: one file-scope device array of LYC_NOALLOC_SCRATCH_BYTES bytes per
- * device, shared by every call; it keeps the last call's contents, and each
- * call clears the parts that must start at zero (arrival counters, status
- * word).  Calls that overlap on the GPU (different streams with no ordering
- * between them, or host threads racing) race on it.
+ * device, shared by every call; it keeps the last call's contents.  Each call
+ * enqueues a small kernel that writes its work list into the array and clears
+ * the parts that must start at zero (arrival counters, status word), then the
+ * attention kernels and the status copy.  Calls that overlap on the GPU
+ * (different streams with no ordering between them, or host threads racing)
+ * race on it.
  * Set-up: the first call on a device (with that device current) looks up the
  * array's address with cudaGetSymbolAddress and sets the kernel's attributes;
  * make that first call before any stream capture.  A host mutex serializes
@@ -358,7 +379,7 @@ lyc_status lyc_set_timeline(lyc_ctx* ctx, unsigned long long* buf, int cap);
  * Errors: INVALID_ARG (pointers, alignment, shapes, k), UNSUPPORTED (d, group
  * size), SCRATCH_LIMIT, CUDA. */
 #define LYC_NOALLOC_MAX_SETS 256
-#define LYC_NOALLOC_MAX_CTAS 32
+#define LYC_NOALLOC_MAX_CTAS 148
 #define LYC_NOALLOC_SCRATCH_BYTES (5u << 20)
 lyc_status lyc_sparse_attention_noalloc(const void* q, const lyc_kv_cache* kv, int batch,
                                         int num_q_heads, int num_kv_heads, int head_dim,

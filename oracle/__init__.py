@@ -154,6 +154,33 @@ class Oracle:
 
 
 _default: Oracle | None = None
+_gomp = None
+
+
+def _libgomp():
+    """The OpenMP runtime the oracle library is linked with (one copy per
+    process, so its thread setting applies to the oracle's parallel loops)."""
+    global _gomp
+    if _gomp is None:
+        _gomp = ctypes.CDLL("libgomp.so.1")
+        _gomp.omp_set_num_threads.argtypes = [ctypes.c_int]
+        _gomp.omp_set_num_threads.restype = None
+        _gomp.omp_get_max_threads.argtypes = []
+        _gomp.omp_get_max_threads.restype = ctypes.c_int
+    return _gomp
+
+
+def max_threads() -> int:
+    """Threads the oracle's next parallel loop uses."""
+    default()
+    return int(_libgomp().omp_get_max_threads())
+
+
+def set_threads(n: int) -> None:
+    """Threads for the oracle's parallel loops that this thread starts next
+    (timing the oracle on one core against all cores)."""
+    default()
+    _libgomp().omp_set_num_threads(int(n))
 
 
 def default() -> Oracle:

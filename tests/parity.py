@@ -144,11 +144,13 @@ def host_stack(data: dict, layers=None, select_mode=O.SELECT_PER_QHEAD) -> O.Sta
                    np.ascontiguousarray(role, dtype=np.uint8), select_mode)
 
 
-def check_layers(data: dict, out: np.ndarray, trace: np.ndarray, k: int, n: int, dtype: str,
+def check_layers(data: dict, out, trace: np.ndarray, k: int, n: int, dtype: str,
                  layers, select_mode=O.SELECT_PER_QHEAD, S0: np.ndarray | None = None, sel=None):
-    """Check the chosen layers of a GPU step (out [L][B][Hq][d], trace
-    [L][B][Hs][k]) against the oracle with teacher forcing.  S0: the sets
-    handed to layer 0 (set-input mode) or None (layer 0 all retrieval)."""
+    """Check the chosen layers of a GPU step (out [L][B][Hq][d], or a list of
+    such arrays from runs that inherited the same sets; trace [L][B][Hs][k])
+    against the oracle with teacher forcing.  S0: the sets handed to layer 0
+    (set-input mode) or None (layer 0 all retrieval)."""
+    outs = out if isinstance(out, (list, tuple)) else [out]
     worst = 0.0
     for l in layers:
         st = host_stack(data, layers=[l], select_mode=select_mode)
@@ -159,7 +161,8 @@ def check_layers(data: dict, out: np.ndarray, trace: np.ndarray, k: int, n: int,
             S_in = trace[l - 1]
             all_ret = False
         o, S_out, keys, fresh = O.layer(st, 0, k, S_in, all_retrieval=all_ret, n=n, sel=sel)
-        worst = max(worst, check_out(out[l], o, dtype, f"layer {l} outputs"))
+        for i, ou in enumerate(outs):
+            worst = max(worst, check_out(ou[l], o, dtype, f"layer {l} outputs (run {i})"))
         B, Hs = S_out.shape[:2]
         for b in range(B):
             for s in range(Hs):

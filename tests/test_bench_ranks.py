@@ -94,3 +94,40 @@ def test_traffic_record_lookup(tmp_path, monkeypatch):
     monkeypatch.setattr(bench, "attn_source_hash", lambda: "def")
     assert bench.profiled_traffic("w1", "per_qhead") is None
     assert bench.profiled_traffic("w1", "kvgroup_mean") is None
+
+
+def test_reference_arm_times_whole_steps_on_the_library_arms_config(capsys):
+    """The oracle arm runs whole L-layer steps of the chosen workload and
+    reports the same config as the library arm (a small override of the
+    Llama3-8B shape, drawn on the host)."""
+    import json
+
+    import bench
+    args = bench.parse_args(["--impl", "reference", "--n", "256", "--k", "32", "--layers", "2",
+                             "--steps", "2", "--warmup", "0"])
+    assert bench.run_reference(args) == 0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    spec = bench.workload_spec(args)
+    assert line["impl"] == "reference"
+    assert line["config"] == bench.line_config(spec, args, 1, bench.kv_cache_bytes(spec))
+    assert line["config"]["workload"] == "llama3-8b-attn-stack-n256-k32-L2-r2"
+    assert line["steps"] == 2 and line["ms_per_step"] > 0
+    assert line["cpu_baseline"]["sample"].startswith("oracle (fp64 C, OpenMP over heads) on 2 whole")
+
+
+def test_workload_names():
+    import bench
+    spec = bench.workload_spec(bench.parse_args([]))
+    assert spec.name == "llama3-8b-attn-stack-n131072-k4096-r2"
+    spec = bench.workload_spec(bench.parse_args(["--workload", "qwen3-8b-64k-b4"]))
+    assert spec.name == "qwen3-8b-attn-stack-b4-n65536-k2048-r3" and spec.L == 36 and spec.B == 4
+    spec = bench.workload_spec(bench.parse_args(["--retrieval-heads", "-1"]))
+    assert spec.name.endswith("-dense") and spec.roles == "all"
+    spec = bench.workload_spec(bench.parse_args(["--workload", "llama3-8b-32k", "--retrieval-heads", "8"]))
+    assert spec.name == "llama3-8b-attn-stack-n32768-k4096-r8" and spec.retrieval_per_layer == 8
+
+
+def test_union_ms():
+    import bench
+    assert bench.union_ms([]) == 0
+    assert bench.union_ms([(0, 1_000_000), (500_000, 2_000_000), (3_000_000, 4_000_000)]) == pytest.approx(3.0)

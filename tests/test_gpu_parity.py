@@ -55,20 +55,54 @@ def run_step(lyc, spec: W.StackSpec, select_mode="per_qhead", data=None, s_in=No
 # ---------------------------------------------------------------- selection kernel
 
 
+# Every launch form of the selection kernel that a step uses: clusters of 4
+# (a layer with many sets), 8 (beside the next attention) and 16 (alone),
+# each in the fixed-k instantiation and in the one that carries the size rules.
+TOPK_FORMS = [(cl, v) for cl in (4, 8, 16) for v in ("fixed", "rules")]
+
+
 @pytest.mark.parametrize("n,k", [(1, 1), (5, 3), (64, 64), (100, 7), (513, 64), (4096, 1000),
                                  (131072, 4096), (131071, 4097), (1000, 999), (777, 800)])
 def test_topk_bitexact_integer_keys(lyc, n, k):
-    """Integer-valued keys with many ties: the GPU selection is bit-exact."""
+    """Integer-valued keys with many ties: every launch form of the GPU
+    selection is bit-exact against the oracle's argsTopK."""
     rng = np.random.default_rng(n * 7 + k)
     x = rng.integers(-6, 7, size=n).astype(np.float32)
     x[rng.random(n) < 0.1] = -0.0
     ctx = lyc.Lyc(1, 1, 1, 1, 64, max(n, 1), k, dtype="fp32")
     keys = torch.from_numpy(x).cuda()
+    exp = O.topk(x.astype(np.float64), k)
     S = torch.full((k,), -7, dtype=torch.int32, device="cuda")
     ctx.topk_f32(keys, n, k, S)
     assert ctx.sync_status() == 0
-    exp = O.topk(x.astype(np.float64), k)
-    assert np.array_equal(S.cpu().numpy(), exp)
+    assert np.array_equal(S.cpu().numpy(), exp), "default launch form"
+    for cl, variant in TOPK_FORMS:
+        S.fill_(-7)
+        v = lyc.LYC_TOPK_FIXED if variant == "fixed" else lyc.LYC_TOPK_RULES
+        ctx.topk_f32(keys, n, k, S, cluster=cl, variant=v)
+        assert ctx.sync_status() == 0
+        assert np.array_equal(S.cpu().numpy(), exp), f"cluster {cl}, {variant} instantiation"
+    ctx.close()
+
+
+@pytest.mark.parametrize("cl,variant", TOPK_FORMS)
+def test_topk_forms_heavy_ties_and_distinct(lyc, cl, variant):
+    """Distinct fp32 keys, all-equal keys (every candidate tied: the radix
+    fallback) and -inf halves, per launch form, at the step's 128K size."""
+    n = 131072
+    ctx = lyc.Lyc(1, 1, 1, 1, 64, n, 5000, dtype="fp32")
+    rng = np.random.default_rng(cl * 10 + (variant == "rules"))
+    v = lyc.LYC_TOPK_FIXED if variant == "fixed" else lyc.LYC_TOPK_RULES
+    for x in (rng.standard_normal(n).astype(np.float32),
+              np.full(n, 0.5, dtype=np.float32),
+              np.concatenate([np.full(n // 2, -np.inf), rng.standard_normal(n // 2)]).astype(np.float32),
+              rng.integers(-2, 3, size=n).astype(np.float32)):
+        keys = torch.from_numpy(x).cuda()
+        for k in (1, 4096, 5000):
+            S = torch.full((k,), -7, dtype=torch.int32, device="cuda")
+            ctx.topk_f32(keys, n, k, S, cluster=cl, variant=v)
+            assert ctx.sync_status() == 0
+            assert np.array_equal(S.cpu().numpy(), O.topk(x.astype(np.float64), k)), (cl, variant, k)
     ctx.close()
 
 
@@ -343,8 +377,68 @@ def _full_size(lyc, spec, layers, mode="per_qhead", gather="cp_async"):
     torch.cuda.empty_cache()
 
 
+def bench_exact(lyc, spec, mode, layers, replays=4, batch_sel=None):
+    """The whole step at the workload's full size, in the launch form the
+    bench times: one context of the bench's shape, the step captured once and
+    replayed `replays` times (every replay after the first runs on the other
+    epoch parity of the flags and pool cursors), no trace.  Then the same
+    replays with the set trace on.  The selection keys and hence the sets do
+    not depend on the order in which CTAs take work, so both runs must end on
+    the same sets; the trace then gives the sets each checked layer inherited
+    (teacher forcing), and the oracle checks the sampled layers of the last
+    replay of both runs.  batch_sel: the batch elements to check (all)."""
+    om = O.SELECT_PER_QHEAD if mode == "per_qhead" else O.SELECT_KVGROUP_MEAN
+    data = W.make_stack(spec, "cuda")
+    ctx = lyc.Lyc(spec.L, spec.B, spec.Hq, spec.Hkv, spec.d, spec.n, spec.k, dtype=spec.dtype,
+                  select_mode=mode)
+    out_u = torch.full((spec.L, spec.B, spec.Hq, spec.d), float("nan"), device="cuda")
+    S_u = torch.full((spec.B, ctx.Hs, spec.k), -7, dtype=torch.int32, device="cuda")
+    for _ in range(replays):
+        ctx.decode_step(data["q"], data["k"], data["v"], spec.n, data["role"], spec.k, out_u, S_u)
+    assert ctx.sync_status() == 0, lyc.lyc_last_error(ctx.ctx)
+    out_t = torch.full_like(out_u, float("nan"))
+    S_t = torch.full_like(S_u, -7)
+    trace = torch.full((spec.L, spec.B, ctx.Hs, spec.k), -7, dtype=torch.int32, device="cuda")
+    ctx.set_trace(trace)
+    for _ in range(replays):
+        ctx.decode_step(data["q"], data["k"], data["v"], spec.n, data["role"], spec.k, out_t, S_t)
+    assert ctx.sync_status() == 0, lyc.lyc_last_error(ctx.ctx)
+    torch.cuda.synchronize()
+    ctx.close()
+    out_u, out_t = out_u.cpu().numpy(), out_t.cpu().numpy()
+    S_u, S_t, trace = S_u.cpu().numpy(), S_t.cpu().numpy(), trace.cpu().numpy()
+    assert np.isfinite(out_u).all() and np.isfinite(out_t).all()
+    assert np.array_equal(S_u, S_t), "the untraced and the traced step ended on different sets"
+    assert np.array_equal(S_t, trace[-1])
+    if batch_sel is not None:
+        bs = list(batch_sel)
+        data = {"q": data["q"][:, bs], "k": data["k"][:, bs], "v": data["v"][:, bs],
+                "role": data["role"]}
+        out_u, out_t, trace = out_u[:, bs], out_t[:, bs], trace[:, bs]
+    P.check_layers(data, [out_u, out_t], trace, spec.k, spec.n, spec.dtype, layers, select_mode=om)
+    del data
+    torch.cuda.empty_cache()
+
+
 def test_llama3_8b_32k_full_step(lyc):
     _full_size(lyc, W.LLAMA3_8B_32K, [0, 1, 2, 17, 31])
+
+
+@pytest.mark.parametrize("mode", ["kvgroup_mean", "per_qhead"])
+def test_llama3_8b_128k_bench_step(lyc, mode):
+    """The bench's own workload and launch form: 32 layers at 128K, k = 4096."""
+    bench_exact(lyc, W.LLAMA3_8B_128K, mode, [0, 1, 2, 15, 30, 31])
+
+
+@pytest.mark.parametrize("mode", ["kvgroup_mean", "per_qhead"])
+def test_llama3_8b_32k_bench_step(lyc, mode):
+    bench_exact(lyc, W.LLAMA3_8B_32K, mode, [0, 1, 16, 31], replays=3)
+
+
+@pytest.mark.parametrize("mode", ["kvgroup_mean", "per_qhead"])
+def test_qwen3_8b_64k_batch4_full_step(lyc, mode):
+    """The Qwen3-8B-shaped stack at its full 36 layers, batch 4."""
+    bench_exact(lyc, W.QWEN3_8B_64K_B4, mode, [0, 1, 17, 35], replays=3)
 
 
 @pytest.mark.parametrize("gather", ["cp_async", "tc"])
@@ -354,5 +448,23 @@ def test_llama3_8b_128k_first_layers(lyc, mode, gather):
     _full_size(lyc, W.LLAMA3_8B_128K.with_(L=6), [0, 1, 5], mode, gather)
 
 
-def test_qwen3_8b_64k_batch4(lyc):
-    _full_size(lyc, W.QWEN3_8B_64K_B4.with_(L=4), [0, 1, 3])
+@pytest.mark.parametrize("pattern", ["blocks", "scattered"])
+def test_single_layer_sweep_corner(lyc, pattern):
+    """The largest corner of the single-layer sweep: batch 8, n = 524288,
+    k = 8192, inherited sets given, two retrieval heads.  The oracle checks
+    two of the eight batch elements (elements never interact)."""
+    spec = W.StackSpec("sweep-corner", L=1, B=8, Hq=32, Hkv=8, d=128, n=524288, k=8192,
+                       planted="heavy", n_planted=256, seed=21)
+    data = W.make_stack(spec, "cuda")
+    role = np.zeros((1, 32), dtype=np.uint8)
+    role[0, [5, 30]] = 1
+    data["role"] = role
+    S0 = W.inherited_sets(spec.B, spec.Hq, spec.n, spec.k, pattern, seed=3, device="cuda")
+    _, out, S, tr = run_step(lyc, spec, data=data, s_in=S0)
+    bs = [0, 7]
+    sub = {"q": data["q"][:, bs], "k": data["k"][:, bs], "v": data["v"][:, bs], "role": role}
+    P.check_layers(sub, out[:, bs], tr[:, bs], spec.k, spec.n, "bf16", [0],
+                   S0=S0.cpu().numpy()[bs])
+    assert np.isfinite(out).all()
+    del data, sub
+    torch.cuda.empty_cache()

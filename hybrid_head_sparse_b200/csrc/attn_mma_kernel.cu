@@ -86,7 +86,10 @@ struct MmaCfg {
   // unit_full[R], unit_empty[R], idx_free[IR]
   static constexpr int BAR_UNIT = 2 * STAGES + IR + 2 * kPartSlots;
   static constexpr int BAR_IDXFREE = BAR_UNIT + 2 * kPoolRing;
-  static constexpr int OFF_FLAGS = OFF_BAR + (BAR_IDXFREE + IR) * 8;
+  // prev_ok: the epilogue warp has seen the previous launch complete (from
+  // then on this launch may write its partial states)
+  static constexpr int BAR_PREVOK = BAR_IDXFREE + IR;
+  static constexpr int OFF_FLAGS = OFF_BAR + (BAR_PREVOK + 1) * 8;
   static constexpr int OFF_RING = OFF_FLAGS + 16;  // kPoolRing pool pieces
   static constexpr int SMEM = OFF_RING + kPoolRing * 16 + 1024;  // + alignment slack
 };
@@ -226,6 +229,12 @@ __device__ __forceinline__ void mma_scheduler(const AttnMmaParams& P, unsigned c
   const uint32_t* acquired = nullptr;  // the last ready flag waited on
   bool waited = false;                 // the previous launch has completed
   int t = 0;                           // CTA-wide tile sequence number
+  // the pool unit taken last: segment, rows, ordinal (none: row == end)
+  int useg = 0, urow = 0, uend = 0, uord = 0;
+  // the current segment's fields
+  int cseg = -1, ckind = 0, cdep = 0;
+  const uint32_t* cready = nullptr;
+  const int32_t* cidx = nullptr;
   for (int i = 0;; ++i) {
     Piece pc;
     if (i < nhome) {
@@ -238,16 +247,40 @@ __device__ __forceinline__ void mma_scheduler(const AttnMmaParams& P, unsigned c
       if (k >= kPoolRing && !mbar_wait(&unit_empty[r], ((k / kPoolRing) - 1) & 1, abort_flag, p.status))
         break;
       // the next unit, or the end (seg -1)
+      if (urow >= uend) {
+        const int u = atomicAdd(cursor, 1);
+        if (u < p.pool_n) {
+          const Piece un = p.pool_units[u];
+          useg = un.seg;
+          urow = un.r0;
+          uend = un.r1;
+          uord = un.ordinal;
+        } else {
+          useg = -1;
+        }
+      }
       pc.seg = -1;
       pc.r0 = pc.r1 = pc.ordinal = 0;
-      const int u = atomicAdd(cursor, 1);
-      if (u < p.pool_n) pc = p.pool_units[u];
+      if (useg >= 0) {
+        pc.seg = useg;
+        pc.r0 = urow;
+        pc.r1 = uend;
+        pc.ordinal = uord;
+        urow = uend;
+      }
       ring[r] = pc;
       mbar_arrive(&unit_full[r]);  // release: the entry above
       if (pc.seg < 0) break;
     }
-    const Segment& sg = p.segs[pc.seg];
-    if (sg.kind != kSparse) {
+    if (pc.seg != cseg) {  // the segment's fields, kept across its consecutive pieces
+      const Segment& sg = p.segs[pc.seg];
+      cseg = pc.seg;
+      ckind = sg.kind;
+      cready = sg.ready;
+      cdep = sg.dep;
+      cidx = sg.idx;
+    }
+    if (ckind != kSparse) {
       for (int r0 = pc.r0; r0 < pc.r1; r0 += kTileRows, ++t)
         if (!slot_free(t)) return;
       continue;
@@ -257,13 +290,13 @@ __device__ __forceinline__ void mma_scheduler(const AttnMmaParams& P, unsigned c
     // running).  Otherwise a set the previous launch writes is read once
     // that launch has completed.  The bulk copies read the set through the
     // async proxy, hence the proxy fence after the acquire.
-    if (sg.ready) {
-      if (sg.ready != acquired) {
-        wait_flag(sg.ready, *p.epoch + 1u, abort_flag, p.status);
+    if (cready) {
+      if (cready != acquired) {
+        wait_flag(cready, *p.epoch + 1u, abort_flag, p.status);
         fence_proxy_async_global();
-        acquired = sg.ready;
+        acquired = cready;
       }
-    } else if (sg.dep && !waited) {
+    } else if (cdep && !waited) {
       pdl_wait();
       waited = true;
     }
@@ -274,7 +307,7 @@ __device__ __forceinline__ void mma_scheduler(const AttnMmaParams& P, unsigned c
       const uint32_t bytes = static_cast<uint32_t>(((nrows * 4) + 15) & ~15);
       fence_proxy_async_smem();
       mbar_arrive_expect_tx(&idxbar[slot], bytes);
-      bulk_g2s(idxring + slot * kTileRows, sg.idx + r0, bytes, &idxbar[slot]);
+      bulk_g2s(idxring + slot * kTileRows, cidx + r0, bytes, &idxbar[slot]);
     }
   }
 }
@@ -310,23 +343,37 @@ __device__ __forceinline__ void mma_producers(const AttnMmaParams& P, unsigned c
   constexpr int ROWS_W = kTileRows / NP;     // rows per producer warp
   uint32_t idx_phase = 0;
   int t = 0;
+  // the current segment's constants in registers (the copies below are asm
+  // with a memory clobber: fields read through the segment would be reloaded
+  // after each), kept while consecutive pieces stay in one segment
+  int cseg = -1;
+  bool dense = false;
+  int64_t s_token = 0, s_page = 0;
+  const bf16_t* kb = nullptr;
+  const bf16_t* vb = nullptr;
+  const int32_t* bt = nullptr;
+  int sl = 0, sb = 0, sgg = 0, nvalid = 0, page_rows = 0;
+  int32_t pad_ok = 0, row_base = 0;
   for (int pi = 0;; ++pi) {
     Piece pc;
     if (!cta_piece<C>(p, smem, pbeg, nhome, pi, lane, &pc)) break;
-    const Segment& sg = p.segs[pc.seg];
-    const bool dense = sg.kind == kDense;
-    const int64_t s_token = sg.s_token;
-    const bf16_t* kb = static_cast<const bf16_t*>(sg.k);
-    const bf16_t* vb = static_cast<const bf16_t*>(sg.v);
-    const int sl = sg.l, sb = sg.b, sgg = sg.g;
-    // the segment's constants in registers (the copies below are asm with a
-    // memory clobber: fields read through `sg` would be reloaded after each)
-    const int nvalid = sg.nvalid;
-    const int32_t pad_ok = sg.pad_ok;
-    const int32_t* bt = sg.bt;
-    const int page_rows = sg.page_rows;
-    const int64_t s_page = sg.s_page;
-    const int32_t row_base = sg.row_base;
+    if (pc.seg != cseg) {
+      const Segment& sg = p.segs[pc.seg];
+      cseg = pc.seg;
+      dense = sg.kind == kDense;
+      s_token = sg.s_token;
+      kb = static_cast<const bf16_t*>(sg.k);
+      vb = static_cast<const bf16_t*>(sg.v);
+      sl = sg.l;
+      sb = sg.b;
+      sgg = sg.g;
+      nvalid = sg.nvalid;
+      pad_ok = sg.pad_ok;
+      bt = sg.bt;
+      page_rows = sg.page_rows;
+      s_page = sg.s_page;
+      row_base = sg.row_base;
+    }
     for (int r0 = pc.r0; r0 < pc.r1; r0 += kTileRows, ++t) {
       const int nrows = min(kTileRows, pc.r1 - r0);
       const int stage = t % STAGES;
@@ -426,24 +473,49 @@ __device__ __forceinline__ void mma_producers(const AttnMmaParams& P, unsigned c
 
 namespace lyc {
 
-// The ring of piece states this CTA uses: the SM's own when CTAs of two
-// launches may run at once (a CTA of this kernel has the SM to itself: the
-// shared memory of two does not fit), else the block's.
-__device__ __forceinline__ int cta_ring(const AttnParams& p) {
-  return p.wpart_by_sm ? static_cast<int>(sm_index()) : static_cast<int>(blockIdx.x);
+// The ring of piece states this CTA uses (chosen at its start, kept in
+// shared memory): the SM's own when CTAs of two launches may run at once (a
+// CTA of this kernel has the SM to itself: the shared memory of two does not
+// fit), else the block's.
+template <class C>
+__device__ __forceinline__ int cta_ring(const unsigned char* smem) {
+  return *reinterpret_cast<const volatile int*>(smem + C::OFF_FLAGS + 4);
 }
 
-// One arrival of `cnt` on the launch's selection-key counter (release: the
-// caller's warp or CTA barrier orders its threads' key stores before this
-// thread's fence); the arrival that completes `expect` resets the counter and
-// raises the flag to the step's epoch + 1.
-__device__ __forceinline__ void keys_arrive(const AttnParams& p, uint32_t cnt, uint32_t expect) {
-  __threadfence();
-  const uint32_t prev = atomicAdd(&p.keys_done[0], cnt);
-  if (prev + cnt == expect) {
-    p.keys_done[0] = 0u;
-    __threadfence();
-    st_release_u32(&p.keys_done[1], *p.epoch + 1u);
+// One arrival of `cnt` on the step counter of the launch's selection keys
+// (release: the caller's warp or CTA barrier orders its threads' key stores
+// before it); the selection starts once the counter reaches keys_ctas * NC.
+__device__ __forceinline__ void keys_arrive(const AttnParams& p, uint32_t cnt) {
+  red_release_add_u32(p.keys_done + (*p.epoch & 1u) * p.pool_stride, cnt);
+}
+
+// A one-tile piece's result from the warp that computed it, for one of the
+// lane's two queries (h = 0: query 2c, columns in oa[md][0] and [2]; h = 1:
+// query 2c+1, oa[md][1] and [3]); oi = that query's output index, or -1.
+// m, l are the warp-wide running maximum (log2 units) and sum.
+template <int D>
+__device__ __forceinline__ void solo_write(const AttnParams& p, const Segment& sg, const Piece& pc, int oi,
+                                           float m, float l, const float (*oa)[4], int h, int g, int c) {
+  if (oi < 0) return;
+  constexpr int MD = D / 16;
+  if (sg.npieces == 1) {
+    float* out = (sg.out ? sg.out : p.out) + (static_cast<int64_t>(sg.b) * p.Hq + sg.head[2 * c + h]) * D;
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+    if (l <= 0.f && g == 0) atomicOr(p.status, kStatusEmptySoftmax);
+#pragma unroll
+    for (int md = 0; md < MD; ++md) {
+      out[16 * md + g] = oa[md][h] * inv;
+      out[16 * md + g + 8] = oa[md][2 + h] * inv;
+    }
+  } else {
+    const int64_t idx = sg.part_base + static_cast<int64_t>(pc.ordinal) * sg.nout + oi;
+    float* po = p.part_o + idx * D;
+#pragma unroll
+    for (int md = 0; md < MD; ++md) {
+      po[16 * md + g] = oa[md][h];
+      po[16 * md + g + 8] = oa[md][2 + h];
+    }
+    if (g == 0) p.part_ml[idx] = make_float2(m, l);
   }
 }
 
@@ -479,40 +551,60 @@ __device__ __forceinline__ void mma_consumers(const AttnMmaParams& P, unsigned c
   uint64_t* slot_free = slot_full + kPartSlots;
   uint64_t* idx_free = bars + C::BAR_IDXFREE;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_FLAGS);
-  const bf16_t* q = static_cast<const bf16_t*>(p.q);
   const float sl2 = p.scale_log2;
   const int mi = lane >> 3, r8 = lane & 7;  // ldmatrix: matrix and row this lane addresses
   const int wq = p.wpart_q > 0 ? p.wpart_q : kMaxQ;  // query rows per ring record
 
-  int t = 0;  // CTA-wide tile sequence number
+  int t = 0;   // CTA-wide tile sequence number
+  int mp = 0;  // pieces of more than one tile so far (they take ring slots in turn)
+  bool prev_ok = false;  // the previous launch has completed (partials may be written)
+  // the current segment's constants and query fragments
+  int cseg = -1, nq = 0, nout = 0, b = 0, oi0 = -1, oi1 = -1, nvalid = 0;
+  bool dense = false;
+  int64_t koff0 = -1, koff1 = -1, key_mean_off = -1;
+  float mean_scale = 0.f;
+  uint32_t qb[KSTEPS][2];
   const int nhome = pend - pbeg;
   for (int pi = 0;; ++pi) {
     // the CTA's own pieces (the dense runs, the only writers of selection
     // keys) come first: once past them, this warp's keys are written
     if (pi == nhome && nhome > 0 && p.keys_done) {
       __syncwarp();
-      if (lane == 0) keys_arrive(p, 1u, static_cast<uint32_t>(p.keys_ctas) * NC);
+      if (lane == 0) keys_arrive(p, 1u);
       __syncwarp();
     }
     Piece pc;
     if (!cta_piece<C>(p, smem, pbeg, nhome, pi, lane, &pc)) break;
-    const Segment& sg = p.segs[pc.seg];
-    const int nq = sg.nq, nout = sg.nout, b = sg.b;
-    const bool dense = sg.kind == kDense;
-    bool out0 = false, out1 = false;
-    for (int o = 0; o < nout; ++o) {
-      out0 |= sg.out_row[o] == q0;
-      out1 |= sg.out_row[o] == q1;
+    const int ntile = (pc.r1 - pc.r0 + kTileRows - 1) / kTileRows;
+    // A piece of one tile belongs to the one warp that takes its tile: that
+    // warp writes the piece's partial state (or, for a segment of one piece,
+    // its outputs) itself, with no ring slot and no epilogue merge.
+    const bool solo = ntile == 1;
+    if (solo && (t % NC) != w) {
+      ++t;
+      continue;
     }
-    const int64_t koff0 = (q0 < nq) ? sg.key_off[q0] : -1;
-    const int64_t koff1 = (q1 < nq) ? sg.key_off[q1] : -1;
-    const int64_t key_mean_off = sg.key_mean_off;
-    const float mean_scale = p.scale / static_cast<float>(nq);
-    const int nvalid = sg.nvalid;
-
-    // ---- Q^T as the B operand: this lane holds query g, d = 16kk + 2c (+8)
-    uint32_t qb[KSTEPS][2];
-    {
+    const Segment& sg = p.segs[pc.seg];
+    if (pc.seg != cseg) {
+      // a new segment: its constants and Q^T as the B operand (this lane
+      // holds query g, d = 16kk + 2c (+8)); kept while the warp's pieces stay
+      // in the segment (consecutive one-tile pieces of a pool unit)
+      cseg = pc.seg;
+      nq = sg.nq;
+      nout = sg.nout;
+      b = sg.b;
+      dense = sg.kind == kDense;
+      oi0 = oi1 = -1;
+      for (int o = 0; o < nout; ++o) {
+        if (sg.out_row[o] == q0) oi0 = o;
+        if (sg.out_row[o] == q1) oi1 = o;
+      }
+      koff0 = (q0 < nq) ? sg.key_off[q0] : -1;
+      koff1 = (q1 < nq) ? sg.key_off[q1] : -1;
+      key_mean_off = sg.key_mean_off;
+      mean_scale = p.scale / static_cast<float>(nq);
+      nvalid = sg.nvalid;
+      const bf16_t* q = static_cast<const bf16_t*>(sg.q ? sg.q : p.q);  // the segment's layer
       const bf16_t* qrow = q + (static_cast<int64_t>(b) * p.Hq + sg.head[g < nq ? g : 0]) * D;
 #pragma unroll
       for (int kk = 0; kk < KSTEPS; ++kk) {
@@ -520,13 +612,13 @@ __device__ __forceinline__ void mma_consumers(const AttnMmaParams& P, unsigned c
         qb[kk][1] = (g < nq) ? *reinterpret_cast<const uint32_t*>(qrow + kk * 16 + 8 + 2 * c) : 0u;
       }
     }
+    const bool out0 = oi0 >= 0, out1 = oi1 >= 0;
 
     float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
     float oa[MD][4];
 #pragma unroll
     for (int md = 0; md < MD; ++md) oa[md][0] = oa[md][1] = oa[md][2] = oa[md][3] = 0.f;
 
-    const int ntile = (pc.r1 - pc.r0 + kTileRows - 1) / kTileRows;
     for (int u = 0; u < ntile; ++u, ++t) {
       if ((t % NC) != w) continue;
       const int r0 = pc.r0 + u * kTileRows;
@@ -653,18 +745,34 @@ __device__ __forceinline__ void mma_consumers(const AttnMmaParams& P, unsigned c
       }
     }
 
-    // ---- hand this warp's state of the piece to the epilogue warp: slot
-    // (piece % kPartSlots) of this CTA's ring, rows that produce an output
-    {
 #pragma unroll
-      for (int s2 = 4; s2 <= 16; s2 <<= 1) {
-        l0 += __shfl_xor_sync(FULL, l0, s2);
-        l1 += __shfl_xor_sync(FULL, l1, s2);
+    for (int s2 = 4; s2 <= 16; s2 <<= 1) {
+      l0 += __shfl_xor_sync(FULL, l0, s2);
+      l1 += __shfl_xor_sync(FULL, l1, s2);
+    }
+    if (solo) {
+      // ---- this warp holds the whole piece: its partial state, or the
+      // normalised outputs when the segment is this one piece.  Partial
+      // states share their buffer with the layer two launches back, whose
+      // merge runs in the previous launch: write them once that launch has
+      // completed (seen by the epilogue warp).
+      if (sg.npieces > 1 && !prev_ok) {
+        mbar_wait(&bars[C::BAR_PREVOK], 0, abort_flag, p.status);
+        prev_ok = true;
       }
-      const int slot = pi % kPartSlots;
-      if (pi >= kPartSlots)
-        mbar_wait(&slot_free[slot], ((pi / kPartSlots) - 1) & 1, abort_flag, p.status);
-      const int64_t rec = ((static_cast<int64_t>(cta_ring(p)) * kPartSlots + slot) * NC + w) * wq;
+      solo_write<D>(p, sg, pc, oi0, m0, l0, oa, 0, g, c);
+      solo_write<D>(p, sg, pc, oi1, m1, l1, oa, 1, g, c);
+      continue;
+    }
+    // ---- hand this warp's state of the piece to the epilogue warp: slot
+    // (multi-tile piece % kPartSlots) of this CTA's ring, rows that produce
+    // an output
+    {
+      const int slot = mp % kPartSlots;
+      if (mp >= kPartSlots)
+        mbar_wait(&slot_free[slot], ((mp / kPartSlots) - 1) & 1, abort_flag, p.status);
+      ++mp;
+      const int64_t rec = ((static_cast<int64_t>(cta_ring<C>(smem)) * kPartSlots + slot) * NC + w) * wq;
       if (g == 0) {
         if (out0) p.wpart_ml[rec + q0] = make_float2(m0, l0);
         if (out1) p.wpart_ml[rec + q1] = make_float2(m1, l1);
@@ -763,11 +871,15 @@ __device__ __forceinline__ void mma_epilogue(const AttnMmaParams& P, unsigned ch
   // selection in between may still run); else on griddepcontrol.wait, which
   // returns once every earlier launch of the chain has completed.
   if (p.prev_done) {
-    if (lane == 0) wait_flag(p.prev_done, *p.epoch + 1u, abort_flag, p.status);
+    if (lane == 0)
+      wait_flag(p.prev_done + (*p.epoch & 1u) * p.pool_stride, p.prev_done_expect, abort_flag, p.status);
     __syncwarp();
   } else {
     pdl_wait();
   }
+  // the consumer warps that write one-tile pieces' partial states themselves
+  // wait for this (release: the acquire above)
+  if (lane == 0) mbar_arrive(&bars[C::BAR_PREVOK]);
   for (int t = blockIdx.x; t < p.prev_ntasks; t += gridDim.x) {
     const int2 task = p.prev_tasks[t];
     const Segment& sg = p.prev_segs[task.x];
@@ -789,18 +901,29 @@ __device__ __forceinline__ void mma_epilogue(const AttnMmaParams& P, unsigned ch
       for (int j = 0; j < 8; ++j)
         if (u0 + j < np) lse_add(acc, ml[j], ov[j]);
     }
-    lse_finish(acc, p.prev_out, p, sg, o, lane, col, D);
+    lse_finish(acc, sg.out ? sg.out : p.prev_out, p, sg, o, lane, col, D);
   }
 
-  // ---- 2. this layer's pieces
+  // ---- 2. this layer's pieces of more than one tile (a one-tile piece's
+  // warp writes its result itself).  Tile j of a piece whose first tile is
+  // the CTA's tile t0 went to consumer warp (t0 + j) % NC, which took tiles
+  // j, j + NC, ... of the piece in order; merging the warps' states in the
+  // order of j makes the piece's result independent of t0, i.e. of which
+  // CTA took the piece and what it did before (results repeat bit for bit).
+  int mp = 0;
+  int t = 0;  // CTA-wide tile sequence number, as the consumers count it
   for (int pi = 0;; ++pi) {
     Piece pc;
     if (!cta_piece<C>(p, smem, pbeg, pend - pbeg, pi, lane, &pc)) break;
+    const int t0 = t;
+    t += (pc.r1 - pc.r0 + kTileRows - 1) / kTileRows;
+    if (pc.r1 - pc.r0 <= kTileRows) continue;
     const Segment& sg = p.segs[pc.seg];
     const int nout = sg.nout;
-    const int slot = pi % kPartSlots;
-    if (!mbar_wait(&slot_full[slot], (pi / kPartSlots) & 1, abort_flag, p.status)) return;
-    const int64_t rec0 = (static_cast<int64_t>(cta_ring(p)) * kPartSlots + slot) * NC * wq;
+    const int slot = mp % kPartSlots;
+    if (!mbar_wait(&slot_full[slot], (mp / kPartSlots) & 1, abort_flag, p.status)) return;
+    ++mp;
+    const int64_t rec0 = (static_cast<int64_t>(cta_ring<C>(smem)) * kPartSlots + slot) * NC * wq;
     // load every output's NC warp states first (all in flight), then merge
     for (int o0 = 0; o0 < nout; o0 += 2) {
       float2 ml[2][NC];
@@ -809,10 +932,11 @@ __device__ __forceinline__ void mma_epilogue(const AttnMmaParams& P, unsigned ch
       for (int h = 0; h < 2; ++h) {
         const int r = sg.out_row[min(o0 + h, nout - 1)];
 #pragma unroll
-        for (int ww = 0; ww < NC; ++ww) {
-          ml[h][ww] = p.wpart_ml[rec0 + ww * wq + r];
-          ov[h][ww] = col ? *reinterpret_cast<const float4*>(p.wpart_o + (rec0 + ww * wq + r) * D + lane * 4)
-                          : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int j = 0; j < NC; ++j) {  // entry j: the warp that took tiles j, j + NC, ...
+          const int ww = (t0 + j) % NC;
+          ml[h][j] = p.wpart_ml[rec0 + ww * wq + r];
+          ov[h][j] = col ? *reinterpret_cast<const float4*>(p.wpart_o + (rec0 + ww * wq + r) * D + lane * 4)
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
         }
       }
 #pragma unroll
@@ -822,9 +946,9 @@ __device__ __forceinline__ void mma_epilogue(const AttnMmaParams& P, unsigned ch
         LseAcc acc;
         lse_init(acc);
 #pragma unroll
-        for (int ww = 0; ww < NC; ++ww) lse_add(acc, ml[h][ww], ov[h][ww]);
+        for (int j = 0; j < NC; ++j) lse_add(acc, ml[h][j], ov[h][j]);
         if (sg.npieces == 1) {
-          lse_finish(acc, p.out, p, sg, o, lane, col, D);  // the whole segment is this piece
+          lse_finish(acc, sg.out ? sg.out : p.out, p, sg, o, lane, col, D);  // the whole segment
         } else {
           const int64_t idx = sg.part_base + static_cast<int64_t>(pc.ordinal) * nout + o;
           if (col) *reinterpret_cast<float4*>(&p.part_o[idx * D + lane * 4]) = acc.o;
@@ -863,7 +987,12 @@ __global__ void __launch_bounds__(MmaCfg<D, NC, NP, STAGES, GT>::kThreads, 1)
       mbar_init(&bars[C::BAR_UNIT + kPoolRing + r], C::kRingReaders);  // unit empty: every reader
     }
     for (int r = 0; r < C::IR; ++r) mbar_init(&bars[C::BAR_IDXFREE + r], 1);  // the tile's consumer
+    mbar_init(&bars[C::BAR_PREVOK], 1);                                       // the epilogue warp
     *reinterpret_cast<int*>(smem + C::OFF_FLAGS) = 0;
+    // this CTA's ring of piece states: its SM's (CTAs of consecutive
+    // launches may overlap in time), else the block's
+    reinterpret_cast<int*>(smem + C::OFF_FLAGS)[1] =
+        P.p.wpart_by_sm ? static_cast<int>(sm_index()) : static_cast<int>(blockIdx.x);
     fence_mbar_init();
   }
   if (threadIdx.x == C::kFirstProducer) {
@@ -878,13 +1007,13 @@ __global__ void __launch_bounds__(MmaCfg<D, NC, NP, STAGES, GT>::kThreads, 1)
   pdl_launch_dependents();
   if (P.p.wait_prev) pdl_wait();  // the previous launch writes what this one reads or writes
   static_assert(2 * C::SMEM > 232448, "the per-SM ring needs one CTA per SM");
-  if (cta_ring(P.p) >= P.p.wpart_slots) {
+  if (cta_ring<C>(smem) >= P.p.wpart_slots) {
     if (threadIdx.x == 0) {
       atomicOr(P.p.status, kStatusScratch);
       // no work, but the arrivals of its consumer warps, so that the
       // selection does not wait out its limit
       if (P.p.keys_done && P.p.cta_begin[blockIdx.x + 1] > P.p.cta_begin[blockIdx.x])
-        keys_arrive(P.p, NC, static_cast<uint32_t>(P.p.keys_ctas) * NC);
+        keys_arrive(P.p, NC);
     }
   } else {
     const int pbeg = P.p.cta_begin[blockIdx.x];
@@ -899,23 +1028,21 @@ __global__ void __launch_bounds__(MmaCfg<D, NC, NP, STAGES, GT>::kThreads, 1)
       mma_consumers<D, NC, NP, STAGES, GT>(P, smem, pbeg, pend);
     }
   }
-  // every write of the CTA is done (and fenced) before its arrival on the
-  // launch's done counter; the last CTA to arrive raises the flag
-  if (P.p.done) __threadfence();
+  // every write of the CTA is done before its arrival on the launch's done
+  // counter; the last CTA to arrive raises the flag.  Release: the CTA
+  // barrier orders every thread's writes before thread 0's device-scope
+  // fence, which precedes the arrival (one fence per CTA: a fence in every
+  // thread stalls every warp on its own outstanding stores).
   __syncthreads();
-  if (threadIdx.x == 0 && P.p.done) {
-    const uint32_t prev = atomicAdd(&P.p.done[0], 1u);
-    if (prev == gridDim.x - 1) {
-      P.p.done[0] = 0u;
-      __threadfence();
-      st_release_u32(&P.p.done[1], *P.p.epoch + 1u);
-    }
-  }
-  // this grid completes only after the one it depends on (dense-only CTAs
-  // never waited above), so completion order follows launch order; the
-  // timeline's end is the end of the CTA's last warp
+  if (threadIdx.x == 0 && P.p.done) red_release_add_u32(P.p.done + (*P.p.epoch & 1u) * P.p.pool_stride, 1u);
+  // This grid completes only after the one it depends on, so that the
+  // launches of the step complete in launch order (dense-only CTAs never
+  // waited above).  With a completion counter, one CTA waits and the others
+  // leave at once: a CTA that waits here holds its SM idle, and the next
+  // launch's CTAs need the SMs.  The timeline's end is the end of the CTA's
+  // last warp.
   if (threadIdx.x == 0) {
-    pdl_wait();
+    if (!P.p.done || blockIdx.x == 0) pdl_wait();
     timeline_record(P.p.timeline, P.p.timeline_cap, t_start,
                     (kTagAttention << 32) | (static_cast<unsigned long long>(P.p.layer) << 16) | blockIdx.x);
   }
@@ -949,6 +1076,10 @@ static cudaError_t mma_run(const AttnMmaParams* P, int grid, cudaStream_t stream
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kern, *P);
 }
+
+// Consumer warps of the instantiation for head_dim D (the key counter of a
+// launch reaches keys_ctas times this).
+int attn_mma_consumer_warps(int D) { return D == 64 ? 4 : 6; }
 
 // bf16 inputs.  configure_only: set the shared-memory attribute, report the size.
 cudaError_t attn_mma_dispatch(int D, const AttnMmaParams* P, int grid, cudaStream_t stream,

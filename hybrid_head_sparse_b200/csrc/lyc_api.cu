@@ -33,6 +33,7 @@ struct AttnMmaParams {
 int attn_nq_bucket(int nq);
 cudaError_t attn_simt_dispatch(int D, int nqb, const AttnParams* p, int grid, cudaStream_t stream,
                                int* smem_out, bool configure_only);
+int attn_mma_consumer_warps(int D);
 cudaError_t attn_mma_dispatch(int D, const AttnMmaParams* P, int grid, cudaStream_t stream,
                               int* smem_out, bool configure_only);
 cudaError_t attn_tc_dispatch(const AttnMmaParams* P, int grid, cudaStream_t stream, int* smem_out,
@@ -58,6 +59,14 @@ namespace {
 
 constexpr int kMaxCtxLimit = 655360;  // 16-CTA top-k keeps every key in shared memory
 constexpr int kPlanCacheSize = 16;
+// Buffers per set slot.  A refresh writes the slot's next buffer in turn.
+// A set is read by the layers up to the slot's next refresh, and the first of
+// them may read it one attention launch late (the mma kernel runs a layer's
+// sparse passes over the sets that the selection just before that layer
+// wrote in the next layer's launch).  A selection starts writing only once
+// the attention launch of the layer before it has completed, so the buffer it
+// overwrites must hold a set written three refreshes ago: three buffers.
+constexpr int kSetBuffers = 3;
 
 
 int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
@@ -130,7 +139,7 @@ struct lyc_ctx {
   std::string err;
   uint32_t* status = nullptr;
   float* keys = nullptr;
-  int32_t* sbuf = nullptr;  // [2][B][Hs][KS]
+  int32_t* sbuf = nullptr;  // [kSetBuffers][B][Hs][KS]
   float* part_o = nullptr;
   float2* part_ml = nullptr;
   // bf16 path: per CTA ring of the consumer warps' piece states
@@ -138,12 +147,13 @@ struct lyc_ctx {
   float2* wpart_ml = nullptr;
   int wpart_slots = 0;
   // per (layer, b, slot): {arrival counter, ready flag} of the selection task
-  // that writes the slot at that layer; then per layer the same pair for the
-  // attention launch; then the step epoch
+  // that writes the slot at that layer; then the step counters; then the
+  // step epoch
   uint32_t* flags = nullptr;
-  uint32_t* attn_flags = nullptr;
-  uint32_t* keys_flags = nullptr;   // per layer: {arrival counter, flag} of the selection keys
-  int32_t* pool_cursors = nullptr;  // [2][L + 1], by epoch parity
+  // step counters [2][3][L + 1], by epoch parity: the pool cursor, the
+  // completion counter and the selection-key counter of each attention launch
+  // (zeroed for the next step by the step's last launch)
+  int32_t* pool_cursors = nullptr;
   uint32_t* epoch = nullptr;
   int32_t* counters = nullptr;
   size_t max_parts = 0, max_counters = 0;
@@ -461,6 +471,9 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const KvVie
     int topk_cl = 16;           // cluster size of this layer's selection launch
     std::vector<Piece> pool_units;   // mma kernel: the pool's units, in order
     int64_t tiles = 0, pool_tiles = 0;
+    // mma kernel: the previous layer's sparse passes over the sets that the
+    // selection before it wrote, run by this launch (see below)
+    std::vector<Segment> deferred;
   };
   std::vector<HostLayer> hl(L);
   std::vector<int> cur(Hs, 0);
@@ -469,6 +482,17 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const KvVie
   };
   const char* kbase = static_cast<const char*>(kv.k);
   const char* vbase = static_cast<const char*>(kv.v);
+  // Deferred sparse passes (mma kernel).  A sparse pass of layer l over a set
+  // that layer l-1's selection writes must wait for that selection, which
+  // starts only once layer l-1's dense rows are done.  Run in layer l's own
+  // launch, the CTAs that take it hold their SMs while they wait, and the
+  // next launch's CTAs that need those SMs start late (the chain: selection
+  // -> waiting gathers -> late dense runs -> late keys -> next selection).
+  // So such a pass runs in layer l+1's launch instead, after that launch's
+  // dense rows, by which time the selection is long done; its partial states
+  // and outputs are those of layer l (Segment::q, Segment::out).  The last
+  // layer keeps its own.
+  const bool defer_dep = use_pool;
 
   // the set trace [L][B][Hs][k]: row (l, b, s) holds the set slot s passes on
   // after layer l.  A refreshed slot's row is written by its selection; the
@@ -497,6 +521,17 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const KvVie
       is_ret[h] = (l == 0 && !s_in) || role[static_cast<int64_t>(l) * Hq + h] != 0;
       if (is_ret[h]) fresh[kvmode ? h / G : h] = 1;
     }
+    // a sparse pass of this layer: into this launch, or (a set the previous
+    // layer's selection writes) into the next one, where it needs no wait
+    // order (dep 0: its selection has long completed)
+    auto push_sparse = [&](Segment ss, int layer) {
+      if (defer_dep && layer + 1 < L && ss.dep && ss.ready) {
+        ss.dep = 0;
+        hl[layer + 1].deferred.push_back(ss);
+      } else {
+        H.segs.push_back(ss);
+      }
+    };
     int maxnq = 1;
     for (int b = 0; b < B; ++b) {
       const int nb = static_cast<int>(kv.n[b]);  // this element's rows
@@ -518,6 +553,8 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const KvVie
         base.l = l;
         base.b = b;
         base.g = g;
+        base.q = static_cast<const char*>(plan->q) + static_cast<size_t>(l) * B * Hq * cfg.head_dim * es;
+        base.out = plan->out + static_cast<size_t>(l) * B * Hq * cfg.head_dim;
         base.key_mean_off = -1;
         for (int j = 0; j < kMaxQ; ++j) {
           base.key_off[j] = -1;
@@ -564,7 +601,7 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const KvVie
             ss.dep = prev_fresh[g];
             ss.ready = ready_flag(g, b);
             maxnq = std::max(maxnq, js);
-            H.segs.push_back(ss);
+            push_sparse(ss, l);
           }
         } else {
           for (int h = g * G; h < (g + 1) * G; ++h) {
@@ -579,10 +616,15 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const KvVie
             ss.nq = ss.nout = 1;
             ss.dep = prev_fresh[h];
             ss.ready = ready_flag(h, b);
-            H.segs.push_back(ss);
+            push_sparse(ss, l);
           }
         }
       }
+    }
+    // the previous layer's deferred sparse passes, after this layer's own
+    for (const Segment& ds : H.deferred) {
+      H.segs.push_back(ds);
+      maxnq = std::max(maxnq, ds.nq);
     }
     H.nqb = attn_nq_bucket(maxnq);
 
@@ -616,7 +658,12 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const KvVie
     // B200: +1.9 % in KV-group mode for a grid that leaves one selection's SMs
     // against one with CTAs that take them back for pool units).
     H.tiles = NT;
-    const int grid = static_cast<int>(std::min<int64_t>(NT, avail));
+    // A launch with no rows of its own (a layer without retrieval heads whose
+    // sparse passes all moved to the next launch) still runs: its CTAs merge
+    // the previous launch's split rows and raise its done flag.
+    int grid = static_cast<int>(std::min<int64_t>(NT, avail));
+    if (grid == 0)
+      grid = std::max(1, std::min(avail, l > 0 ? static_cast<int>(hl[l - 1].combine.size()) : 1));
     H.grid = grid;
     std::vector<int> npieces(H.segs.size(), 0);
     std::vector<std::vector<Piece>> per_cta(grid);
@@ -655,22 +702,25 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const KvVie
     if (use_pool) {
       // a gathered segment of r rows is cut into units of kPoolTiles tiles
       // (kPoolTilesDep for a set the previous selection writes), unit q =
-      // ordinal q; the pool lists them in order, earlier selections' sets first
+      // piece q (its ordinal); CTAs take them at run time.  The pool lists
+      // the units in order, earlier selections' sets first.  (Measured on
+      // B200 against one-tile pieces whose warp writes its own partial state:
+      // per-head selection 1231 against 1348 us per step, KV-group even.)
       for (int dep = 0; dep < 2; ++dep)
         for (size_t s2 = 0; s2 < H.segs.size(); ++s2)
           if (H.segs[s2].kind == kSparse && H.segs[s2].dep == dep) {
-            const int unit_rows = (dep ? kPoolTilesDep : kPoolTiles) * kTileRows;
+            const int unit_tiles = dep ? kPoolTilesDep : kPoolTiles;
             const int rows = H.segs[s2].rows;
-            int q = 0;
-            for (int r0 = 0; r0 < rows; r0 += unit_rows, ++q) {
+            int tile = 0;
+            for (int r0 = 0; r0 < rows; r0 += unit_tiles * kTileRows, tile += unit_tiles) {
               Piece pc;
               pc.seg = static_cast<int32_t>(s2);
               pc.r0 = r0;
-              pc.r1 = std::min(r0 + unit_rows, rows);
-              pc.ordinal = q;
+              pc.r1 = std::min(r0 + unit_tiles * kTileRows, rows);
+              pc.ordinal = tile / unit_tiles;
               H.pool_units.push_back(pc);
             }
-            npieces[s2] = q;
+            npieces[s2] = (rows + unit_tiles * kTileRows - 1) / (unit_tiles * kTileRows);
             H.pool_tiles += (rows + TR - 1) / TR;
           }
     }
@@ -702,7 +752,7 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const KvVie
       for (int b = 0; b < B; ++b) {
         TopkTask tk{};
         tk.keys = ctx->keys + keys_base + (static_cast<int64_t>(b) * Hs + s) * ctx->nstride;
-        tk.S = set_ptr(1 - cur[s], b, s);
+        tk.S = set_ptr((cur[s] + 1) % kSetBuffers, b, s);
         tk.done = ctx->flags + ((static_cast<int64_t>(l) * B + b) * Hs + s) * 2;
         tk.trace = trace_row(l, b, s);
         tk.n = static_cast<int32_t>(kv.n[b]);
@@ -726,7 +776,7 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const KvVie
         }
     for (int s = 0; s < Hs; ++s)
       if (fresh[s]) {
-        cur[s] ^= 1;
+        cur[s] = (cur[s] + 1) % kSetBuffers;
         writer[s] = l;
       }
     prev_fresh = fresh;
@@ -898,6 +948,12 @@ lyc_status enqueue_step(lyc_ctx* ctx, Plan* plan, cudaStream_t stream, int set, 
     if (!early || l + 1 >= L) return false;
     return plan->layers[l + 1].tiles > 0;
   };
+  // step counters of layer l's attention launch (parity-0 addresses)
+  const int cstride = 3 * (L + 1);
+  uint32_t* cnt_base = reinterpret_cast<uint32_t*>(ctx->pool_cursors);
+  auto done_cnt = [&](int l) { return cnt_base + (L + 1) + l; };
+  auto keys_cnt = [&](int l) { return cnt_base + 2 * (L + 1) + l; };
+  const uint32_t nc = static_cast<uint32_t>(attn_mma_consumer_warps(D));
   for (int l = 0; l < L; ++l) {
     const LayerPlan& lp = plan->layers[l];
     AttnParams ap{};
@@ -917,16 +973,17 @@ lyc_status enqueue_step(lyc_ctx* ctx, Plan* plan, cudaStream_t stream, int set, 
     if (early) {
       // done flags between consecutive attention launches, and the pool of
       // gathered rows (mma kernel only)
-      ap.done = ctx->attn_flags + 2 * l;
-      ap.prev_done = l > 0 ? ctx->attn_flags + 2 * (l - 1) + 1 : nullptr;
+      ap.done = done_cnt(l);
+      ap.prev_done = l > 0 ? done_cnt(l - 1) : nullptr;
+      ap.prev_done_expect = l > 0 ? static_cast<uint32_t>(plan->layers[l - 1].grid) : 0u;
       ap.pool_units = reinterpret_cast<const Piece*>(plan->dev + lp.off_pool);
       ap.pool_n = lp.pool_n;
-      ap.pool_stride = L + 1;
+      ap.pool_stride = cstride;
       ap.pool_cursors = ctx->pool_cursors;
       // the selection of this layer starts once the keys are written (the
       // dense runs), not once the whole launch is done
       if (lp.ntasks > 0 && lp.keys_ctas > 0) {
-        ap.keys_done = ctx->keys_flags + 2 * l;
+        ap.keys_done = keys_cnt(l);
         ap.keys_ctas = lp.keys_ctas;
       }
     }
@@ -984,8 +1041,11 @@ lyc_status enqueue_step(lyc_ctx* ctx, Plan* plan, cudaStream_t stream, int set, 
       tp.layer = l;
       tp.status = ctx->status;
       if (ap.keys_done) {
-        tp.keys_ready = ap.keys_done + 1;
-        tp.prev_done = l > 0 ? ctx->attn_flags + 2 * (l - 1) + 1 : nullptr;
+        tp.keys_ready = ap.keys_done;
+        tp.keys_expect = static_cast<uint32_t>(lp.keys_ctas) * nc;
+        tp.prev_done = ap.prev_done;
+        tp.prev_done_expect = ap.prev_done_expect;
+        tp.cnt_stride = cstride;
       }
       if ((st = record_event(ctx, plan, set, ev++, stream, capturing)) != LYC_OK) return st;
       LYC_CUDA(topk_launch(lp.topk_cl, &tp, lp.ntasks, stream, false), "top-k launch");
@@ -1015,7 +1075,11 @@ lyc_status enqueue_step(lyc_ctx* ctx, Plan* plan, cudaStream_t stream, int set, 
     ap.wpart_by_sm = 1;
     ap.wpart_slots = ctx->wpart_slots;
     ap.epoch = ctx->epoch;
-    if (early) ap.prev_done = ctx->attn_flags + 2 * (L - 1) + 1;
+    if (early) {
+      ap.prev_done = done_cnt(L - 1);
+      ap.prev_done_expect = static_cast<uint32_t>(lp.grid);
+      ap.pool_stride = cstride;
+    }
     ap.layer = L;
     ap.Hq = Hq;
     ap.G = ctx->G;
@@ -1041,7 +1105,7 @@ lyc_status enqueue_step(lyc_ctx* ctx, Plan* plan, cudaStream_t stream, int set, 
     LYC_CUDA(copy_sets_launch(&fp, stream), "trace fill");
   }
   CopySetsParams cp{reinterpret_cast<const int32_t* const*>(plan->dev + plan->off_final_src), plan->S,
-                    B * ctx->Hs, plan->k, ctx->epoch, ctx->pool_cursors, L + 1, nullptr};
+                    B * ctx->Hs, plan->k, ctx->epoch, ctx->pool_cursors, cstride, nullptr};
   LYC_CUDA(copy_sets_launch(&cp, stream), "final set copy");
   return LYC_OK;
 }
@@ -1248,7 +1312,9 @@ lyc_status lyc_create(const lyc_config* cfg, lyc_ctx** out) {
   ctx->KS = static_cast<int>(round_up(c.max_k, 4));
   const int B = c.batch, Hq = c.num_q_heads, Hkv = c.num_kv_heads, D = c.head_dim, L = c.num_layers;
   const size_t es = c.dtype == LYC_BF16 ? 2 : 4;
-  const size_t nseg_max = static_cast<size_t>(B) * (Hkv + Hq);
+  // segments of one launch: dense and sparse of its layer, plus the previous
+  // layer's deferred sparse passes
+  const size_t nseg_max = static_cast<size_t>(B) * (Hkv + 2 * Hq);
   // pieces per layer <= 2 * sms + segments (two pooling phases), plus the
   // pool units of the mma kernel (every sparse segment cut into units, at
   // most of the smaller unit size)
@@ -1264,16 +1330,15 @@ lyc_status lyc_create(const lyc_config* cfg, lyc_ctx** out) {
     return LYC_OK;
   };
   lyc_status st;
-  // ready flags: two words per (layer, b, slot) and per layer, then the
-  // pool cursors, the key flags (two words per layer), then the epoch
-  const size_t flag_words = static_cast<size_t>(L) * B * ctx->Hs * 2 + static_cast<size_t>(L) * 2 +
-                            2 * (static_cast<size_t>(L) + 1) + static_cast<size_t>(L) * 2 + 4;
+  // ready flags: two words per (layer, b, slot); then the step counters;
+  // then the epoch
+  const size_t flag_words = static_cast<size_t>(L) * B * ctx->Hs * 2 + 2 * 3 * (static_cast<size_t>(L) + 1) + 4;
   if ((st = alloc(reinterpret_cast<void**>(&ctx->status), 16)) != LYC_OK ||
       (st = alloc(reinterpret_cast<void**>(&ctx->keys),
                   static_cast<size_t>(L) * B * ctx->Hs * ctx->nstride * sizeof(float))) != LYC_OK ||
       (st = alloc(reinterpret_cast<void**>(&ctx->flags), flag_words * sizeof(uint32_t))) != LYC_OK ||
       (st = alloc(reinterpret_cast<void**>(&ctx->sbuf),
-                  2ull * B * ctx->Hs * ctx->KS * sizeof(int32_t) + 64)) != LYC_OK ||
+                  static_cast<size_t>(kSetBuffers) * B * ctx->Hs * ctx->KS * sizeof(int32_t) + 64)) != LYC_OK ||
       (st = alloc(reinterpret_cast<void**>(&ctx->part_o), 2 * ctx->max_parts * D * sizeof(float))) != LYC_OK ||
       (st = alloc(reinterpret_cast<void**>(&ctx->part_ml), 2 * ctx->max_parts * sizeof(float2))) != LYC_OK ||
       (st = alloc(reinterpret_cast<void**>(&ctx->counters), ctx->max_counters * sizeof(int32_t))) != LYC_OK ||
@@ -1283,9 +1348,7 @@ lyc_status lyc_create(const lyc_config* cfg, lyc_ctx** out) {
     lyc_destroy(holder.release());
     return st;
   }
-  ctx->attn_flags = ctx->flags + static_cast<size_t>(L) * B * ctx->Hs * 2;
-  ctx->pool_cursors = reinterpret_cast<int32_t*>(ctx->attn_flags + static_cast<size_t>(L) * 2);
-  ctx->keys_flags = ctx->attn_flags + static_cast<size_t>(L) * 2 + 2 * (static_cast<size_t>(L) + 1);
+  ctx->pool_cursors = reinterpret_cast<int32_t*>(ctx->flags + static_cast<size_t>(L) * B * ctx->Hs * 2);
   ctx->epoch = ctx->flags + (flag_words - 4);
   if (c.dtype == LYC_BF16) {
     // one ring per SM index (the SM a CTA runs on owns it; SM indices need
@@ -1301,7 +1364,8 @@ lyc_status lyc_create(const lyc_config* cfg, lyc_ctx** out) {
   if (cudaMemset(ctx->status, 0, 16) != cudaSuccess ||
       cudaMemset(ctx->flags, 0, flag_words * sizeof(uint32_t)) != cudaSuccess ||
       cudaMemset(ctx->counters, 0, ctx->max_counters * sizeof(int32_t)) != cudaSuccess ||
-      cudaMemset(ctx->sbuf, 0xff, 2ull * B * ctx->Hs * ctx->KS * sizeof(int32_t) + 64) != cudaSuccess) {
+      cudaMemset(ctx->sbuf, 0xff, static_cast<size_t>(kSetBuffers) * B * ctx->Hs * ctx->KS * sizeof(int32_t) + 64) !=
+          cudaSuccess) {
     lyc_destroy(holder.release());
     return LYC_ERR_CUDA;
   }

@@ -113,6 +113,14 @@ __device__ __forceinline__ void st_release_u32(uint32_t* p, uint32_t v) {
   asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
+// Add v to a counter with release semantics at GPU scope.  No value comes
+// back, so the issuing thread does not wait for the round trip.  Called by
+// one thread after a CTA (or warp) barrier, it also releases the writes of
+// the threads that the barrier ordered before it.
+__device__ __forceinline__ void red_release_add_u32(uint32_t* p, uint32_t v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
 // Wait until *flag == want (acquire).  Same limit and abort rules as
 // mbar_wait; the flag's writer is a kernel that is already running or done.
 static __device__ __noinline__ bool wait_flag(const uint32_t* flag, uint32_t want, volatile int* abort_flag,

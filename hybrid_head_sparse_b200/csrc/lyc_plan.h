@@ -78,6 +78,12 @@ struct Segment {
   const int32_t* bt;      // paged cache: the block-table row of b (row i is in page bt[i / page_rows],
                           // at k + page * s_page + (i % page_rows) * s_token); NULL: contiguous
   int64_t s_page;         // paged cache: element stride between pages
+  // the segment's layer: its queries [B][Hq][d] and outputs [B][Hq][d] (a
+  // launch of the mma kernel may hold segments of two layers: its own, and
+  // the previous layer's sparse passes over the sets that the selection just
+  // before that layer wrote); NULL: the launch's q and out
+  const void* q;
+  float* out;
 };
 
 struct Piece {
@@ -111,17 +117,22 @@ struct AttnParams {
   uint32_t* status;          // device status word
   unsigned long long* timeline;  // NULL, or [1 + 3*cap]: count, then (start ns, end ns, tag)
   const uint32_t* epoch;     // this step's epoch (the `ready` flags hold epoch + 1), or NULL
-  uint32_t* done;            // NULL, or {arrival counter, flag} of this launch: the last CTA
-                             // to finish raises the flag to epoch + 1
-  const uint32_t* prev_done; // NULL, or the flag of the previous layer's attention launch:
-                             // the epilogue waits on it (else on griddepcontrol.wait)
+  // Step counters (zeroed for the next step by the step's last launch): the
+  // counter of this step is at ptr + (epoch & 1) * pool_stride.
+  uint32_t* done;            // NULL, or this launch's completion counter: every CTA adds 1
+                             // once its work is done (release)
+  const uint32_t* prev_done; // NULL, or the previous layer's attention launch's completion
+                             // counter: the epilogue waits until it reaches prev_done_expect
+                             // (else on griddepcontrol.wait)
+  uint32_t prev_done_expect; // CTAs of that launch
   // the pool (mma kernel): after its own pieces a CTA takes units u = 0, 1, ...
   // by an atomic cursor; unit u is the piece pool_units[u] (a row range of a
   // gathered segment, its ordinal = its partial record)
   const Piece* pool_units;
   int32_t pool_n;            // units in the pool (0: none)
-  int32_t pool_stride;       // cursors per epoch parity
-  int32_t* pool_cursors;     // [2][pool_stride]: this launch's is [(epoch & 1)][layer]
+  int32_t pool_stride;       // step counters per epoch parity (pool cursors, completion and
+                             // key counters)
+  int32_t* pool_cursors;     // [2][pool_stride]: this launch's cursor is [(epoch & 1)][layer]
   int32_t wpart_by_sm;       // 1: the piece-state ring of a CTA is the one of the SM it runs
                              // on (CTAs of consecutive launches may overlap in time); 0: of
                              // its block index
@@ -129,10 +140,9 @@ struct AttnParams {
   int32_t wpart_q;           // query rows per consumer-warp record of the ring (0: kMaxQ); a
                              // caller whose segments all have one query row passes 1
   int32_t timeline_cap;
-  uint32_t* keys_done;       // NULL, or {arrival counter, flag} of this launch's selection
-                             // keys: each consumer warp of the first keys_ctas CTAs arrives
-                             // once its own (dense) pieces are done; the last arrival raises
-                             // the flag to epoch + 1
+  uint32_t* keys_done;       // NULL, or the step counter of this launch's selection keys:
+                             // each consumer warp of the keys_ctas CTAs with pieces of their
+                             // own adds 1 once those (dense) pieces are done (release)
   int32_t keys_ctas;
   int32_t layer;
   int32_t Hq, G, n;
@@ -177,10 +187,13 @@ struct TopkParams {
                           // (its readers wait on the ready flags); 0: only after
   unsigned long long* timeline;  // as in AttnParams
   const uint32_t* keys_ready;  // NULL: start on griddepcontrol.wait (the attention launch
-                               // before has completed); else on this flag (AttnParams::keys_done)
-  const uint32_t* prev_done;   // with keys_ready: the done flag of the attention launch of the
-                               // layer before (its readers of the set buffers this launch
-                               // writes), or NULL
+                               // before has completed); else once this step counter
+                               // (AttnParams::keys_done) reaches keys_expect
+  const uint32_t* prev_done;   // with keys_ready: the completion counter of the attention
+                               // launch of the layer before (its readers of the set buffers
+                               // this launch writes) to wait for, up to prev_done_expect; or NULL
+  uint32_t keys_expect, prev_done_expect;
+  int32_t cnt_stride;          // step counters per epoch parity
   uint32_t* status;            // device status word (wait timeouts)
   int32_t timeline_cap;
   int32_t layer;

@@ -347,8 +347,9 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster_kernel(const Top
     __shared__ int wait_abort;
     if (tid == 0) {
       wait_abort = 0;
-      if (wait_flag(p.keys_ready, *p.epoch + 1u, &wait_abort, p.status) && p.prev_done)
-        wait_flag(p.prev_done, *p.epoch + 1u, &wait_abort, p.status);
+      const uint32_t par = (*p.epoch & 1u) * p.cnt_stride;
+      if (wait_flag(p.keys_ready + par, p.keys_expect, &wait_abort, p.status) && p.prev_done)
+        wait_flag(p.prev_done + par, p.prev_done_expect, &wait_abort, p.status);
     }
     __syncthreads();
   } else {

@@ -518,8 +518,9 @@ def run_lyc(args):
     ctx.set_timing(False)
     iso_attn_ms = sum(t[2] for t in ktimes if t[0] == 0) / args.steps
     iso_topk_ms = sum(t[2] for t in ktimes if t[0] == 1) / args.steps
-    attn_launches = sum(1 for t in ktimes if t[0] == 0) // args.steps
-    topk_launches = sum(1 for t in ktimes if t[0] == 1) // args.steps
+    # launches per step: attention launches (one per layer and a merge
+    # launch, or layer 0 and one persistent launch) and selection launches
+    attn_launches, topk_launches, other_launches = ctx.step_launches()
 
     roofline = {
         "bound": "hbm",
@@ -538,11 +539,13 @@ def run_lyc(args):
                  "union of its CTAs' busy intervals on the device timeline (same K replays), as "
                  "a share of the span, times the timed ms_per_step.  Launches of consecutive "
                  "layers overlap, so the per-launch figure is that time / L"),
-        "isolated_launches": {
+        "isolated_launches": ({
             "attn_ms_per_step": iso_attn_ms, "topk_ms_per_step": iso_topk_ms,
             "attn_gbs": round(distinct / (iso_attn_ms / 1e3) / 1e9, 1),
             "note": "each launch timed alone by event nodes in the graph, which serialise the "
-                    "launches (no overlap between layers): an upper bound on launch time"},
+                    "launches (no overlap between layers): an upper bound on launch time"}
+            if iso_attn_ms > 0 else
+            {"note": "not measured"}),
         "timeline_ms_per_step": ms_step_tl,
     }
     step_gbs = analytic / (ms_step / 1e3) / 1e9
@@ -620,7 +623,7 @@ def run_lyc(args):
         cpu = oracle_baseline(spec, hs, steps=1, single_core=True)
         del hs
 
-    launches_per_step = attn_launches + topk_launches + 1
+    launches_per_step = attn_launches + topk_launches + other_launches
     line = {
         "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,

@@ -163,6 +163,7 @@ struct lyc_ctx {
   int32_t* S_dev = nullptr;
   int32_t* trace = nullptr;
   cudaStream_t last_stream = nullptr;
+  int last_launches[3] = {-1, 0, 0};  // the most recent step's attention, selection, other launches
   bool timing = false;
   unsigned long long* timeline = nullptr;  // caller's buffer, or NULL
   int timeline_cap = 0;
@@ -1504,6 +1505,17 @@ lyc_status step_impl(lyc_ctx* ctx, const void* q, const KvView& kv, const uint8_
     if (static_cast<int>(v.size()) > timing_sets()) v.erase(v.begin());
   }
   ctx->last_stream = stream;
+  {
+    int a = 0, t = 0;
+    for (int kind : plan->kernel_kind) (kind == 0 ? a : t) += 1;
+    int o = 1;  // the final set copy
+    if (plan->trace && plan->nfill > 0) ++o;
+    if (plan->append) ++o;
+    if ((plan->flags & LYC_STEP_S_IN) && (plan->flags & LYC_STEP_VALIDATE_S)) o += ctx->cfg.batch;
+    ctx->last_launches[0] = a;
+    ctx->last_launches[1] = t;
+    ctx->last_launches[2] = o;
+  }
   return LYC_OK;
 }
 
@@ -1807,6 +1819,14 @@ lyc_status lyc_kernel_times(lyc_ctx* ctx, lyc_kernel_time* times, int cap, int* 
   }
   v.clear();
   *count = nout;
+  return LYC_OK;
+}
+
+lyc_status lyc_step_launches(const lyc_ctx* ctx, int* attention, int* selection, int* other) {
+  if (!ctx || !attention || !selection || !other || ctx->last_launches[0] < 0) return LYC_ERR_INVALID_ARG;
+  *attention = ctx->last_launches[0];
+  *selection = ctx->last_launches[1];
+  *other = ctx->last_launches[2];
   return LYC_OK;
 }
 

@@ -54,7 +54,8 @@ LYC_TOPK_RULES = 1
 
 EXPORTED = ["lyc_create", "lyc_decode_step", "lyc_decode_step_host", "lyc_decode_step_batch",
             "lyc_sync_status",
-            "lyc_set_s_trace", "lyc_step_bytes", "lyc_topk_f32", "lyc_topk_f32_ex", "lyc_set_timing",
+            "lyc_set_s_trace", "lyc_step_bytes", "lyc_step_launches", "lyc_topk_f32", "lyc_topk_f32_ex",
+            "lyc_set_timing",
             "lyc_kernel_times", "lyc_set_timeline", "lyc_status_string", "lyc_last_error",
             "lyc_destroy", "lyc_sparse_attention_noalloc", "lyc_set_selection", "lyc_cache_correction"]
 
@@ -126,6 +127,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     L.lyc_set_s_trace.argtypes = [P, P]
     L.lyc_step_bytes.argtypes = [ctypes.POINTER(lyc_config), P, ctypes.c_int64, I, I,
                                  ctypes.POINTER(ctypes.c_uint64), ctypes.POINTER(ctypes.c_uint64)]
+    L.lyc_step_launches.argtypes = [P, ctypes.POINTER(I), ctypes.POINTER(I), ctypes.POINTER(I)]
     L.lyc_topk_f32.argtypes = [P, P, ctypes.c_int64, I, P, P]
     L.lyc_topk_f32_ex.argtypes = [P, P, ctypes.c_int64, I, P, I, I, P]
     L.lyc_set_timing.argtypes = [P, I]
@@ -415,3 +417,10 @@ class Lyc:
 
     def step_bytes(self, role_mask, n, k, s_in=False):
         return lyc_step_bytes(self.cfg, role_mask, n, k, s_in)
+
+    def step_launches(self):
+        """(attention, selection, other) kernel launches of the most recent step."""
+        a, t, o = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
+        self._check(load().lyc_step_launches(self.ctx, ctypes.byref(a), ctypes.byref(t), ctypes.byref(o)),
+                    "lyc_step_launches")
+        return a.value, t.value, o.value

@@ -293,6 +293,13 @@ lyc_status lyc_set_s_trace(lyc_ctx* ctx, int32_t* trace);
 lyc_status lyc_step_bytes(const lyc_config* cfg, const uint8_t* role_mask, int64_t n, int k,
                           int s_in, uint64_t* analytic, uint64_t* distinct);
 
+/* Kernel launches of the most recent step enqueued on this context: its
+ * attention launches (one per layer and the launch that merges the last
+ * layer's split rows), selection launches, and the rest (the final set copy,
+ * trace fill, K/V append, S^(0) check).
+ * Errors: INVALID_ARG (NULL, or no step yet). */
+lyc_status lyc_step_launches(const lyc_ctx* ctx, int* attention, int* selection, int* other);
+
 /* Test hook for the selection kernel alone: S[0..k) = argsTopK(keys[0..n), k)
  * with ties to the lower index, ascending, -1 padded.  keys and S are device
  * pointers (keys float32 [n], S int32 [k]); n <= max_ctx, k <= max_k. */

@@ -33,7 +33,9 @@ if ROOT not in sys.path:
 METRIC = "attn-stack decode steps/s at 128K ctx, k=4096; HBM GB/s vs peak"
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
-ATTN_SOURCES = ["attn_mma_kernel.cu", "lyc_plan.h", "lyc_device.cuh"]
+# the sources that decide what an attention launch reads: the kernel and the
+# plan that cuts the rows into pieces
+ATTN_SOURCES = ["attn_mma_kernel.cu", "lyc_plan.h", "lyc_device.cuh", "lyc_api.cu"]
 
 
 def parse_args(argv=None):
@@ -78,6 +80,11 @@ def parse_args(argv=None):
                          "query heads, or batch elements), all-gather the outputs and sets every "
                          "step; strong scaling.  Default: every rank runs its own replica")
     ap.add_argument("--batch", type=int, default=None, help="batch elements (default: the workload's)")
+    ap.add_argument("--traffic-from", default=None, metavar="CSV",
+                    help="print the traffic record of an ncu capture (dram__bytes_read.sum and "
+                         "dram__bytes_write.sum, --csv) of this command line's attention "
+                         "launches: one whole step's launches, summed and divided by the layers, "
+                         "stamped with the hash of the sources here; no GPU work")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-other-mode", action="store_true",
@@ -304,15 +311,18 @@ def sample_text(spec, steps: int):
             f"all {spec.L} layers, every head, n={spec.n}, k={spec.k}, same seeded inputs")
 
 
-def oracle_baseline(spec, hs, steps: int, single_core: bool) -> dict:
-    """cpu_baseline object: `steps` whole oracle steps on every host core, and
+def oracle_baseline(spec, hs, budget_s: float, single_core: bool, max_steps: int = 5) -> dict:
+    """cpu_baseline object: whole oracle steps on every host core, as many as
+    fit in about budget_s seconds (at least one, at most max_steps), and
     (single_core) one more whole step on one core."""
     import oracle as O
     cores = O.max_threads()
-    secs = [oracle_step_seconds(spec, hs) for _ in range(steps)]
+    secs = [oracle_step_seconds(spec, hs)]
+    while len(secs) < max_steps and sum(secs) + secs[0] <= budget_s:
+        secs.append(oracle_step_seconds(spec, hs))
     sec = sum(secs) / len(secs)
     res = {"value": 1.0 / sec, "unit": "steps/s", "cores": cores, "kind": "oracle",
-           "sample": sample_text(spec, steps), "step_seconds": [round(t, 3) for t in secs]}
+           "sample": sample_text(spec, len(secs)), "step_seconds": [round(t, 3) for t in secs]}
     if single_core:
         O.set_threads(1)
         try:
@@ -620,7 +630,7 @@ def run_lyc(args):
         import oracle as O
         O.build()
         hs = host_stack(spec, data, args.select_mode)
-        cpu = oracle_baseline(spec, hs, steps=1, single_core=True)
+        cpu = oracle_baseline(spec, hs, budget_s=8.0, single_core=True)
         del hs
 
     launches_per_step = attn_launches + topk_launches + other_launches
@@ -1081,8 +1091,43 @@ def run_rule(args):
     return 0
 
 
+def traffic_record(args) -> int:
+    """The traffic record line of an ncu capture of this command's attention
+    launches (`ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum -k
+    regex:attn_mma -s S -c L+1 --csv`): one whole step of the graph, i.e. one
+    launch per layer plus the combine launch of the last layer.  Its DRAM
+    bytes are summed and divided by the layers, the same unit as the
+    roofline's algorithmic bytes per launch.  The source hash is taken from
+    the files next to this script, so run it where the capture ran."""
+    import csv
+    spec = workload_spec(args)
+    per = {}
+    with open(args.traffic_from) as f:
+        for r in csv.DictReader(line for line in f if line.startswith('"')):
+            if "attn_mma" not in r["Kernel Name"]:
+                continue
+            scale = {"byte": 1.0, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9}[r["Metric Unit"]]
+            per.setdefault(int(r["ID"]), {})[r["Metric Name"]] = float(r["Metric Value"]) * scale
+    launches = [v for _, v in sorted(per.items())
+                if "dram__bytes_read.sum" in v and "dram__bytes_write.sum" in v]
+    if len(launches) != spec.L + 1:
+        print(f"expected {spec.L + 1} attention launches (one step), found {len(launches)}",
+              file=sys.stderr)
+        return 2
+    rd = sum(v["dram__bytes_read.sum"] for v in launches)
+    wr = sum(v["dram__bytes_write.sum"] for v in launches)
+    rec = {"workload": spec.name, "select_mode": args.select_mode, "source_sha": attn_source_hash(),
+           "bytes_per_launch": round((rd + wr) / spec.L), "step_read_bytes": round(rd),
+           "step_write_bytes": round(wr), "launches": len(launches),
+           "note": "one step's attention launches of the bench command at full size, summed, / L"}
+    print("traffic-record: " + json.dumps(rec))
+    return 0
+
+
 def main(argv=None):
     args = parse_args(argv)
+    if args.traffic_from:
+        return traffic_record(args)
     if args.impl == "reference":
         return run_reference(args)
     if args.serving:

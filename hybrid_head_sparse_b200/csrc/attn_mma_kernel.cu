@@ -235,6 +235,34 @@ __device__ __forceinline__ void mma_scheduler(const AttnMmaParams& P, unsigned c
   int cseg = -1, ckind = 0, cdep = 0;
   const uint32_t* cready = nullptr;
   const int32_t* cidx = nullptr;
+  bool cpad = false;
+  auto seg_fields = [&](int seg) {  // the segment's fields, kept across its consecutive pieces
+    if (seg == cseg) return;
+    const Segment& sg = p.segs[seg];
+    cseg = seg;
+    ckind = sg.kind;
+    cready = sg.ready;
+    cdep = sg.dep;
+    cidx = sg.idx;
+    cpad = sg.pad_ok != 0;
+  };
+  // A set that a selection of this step writes is read once that selection
+  // has raised its ready flag (the selection may still be running).
+  // Otherwise a set the previous launch writes is read once that launch has
+  // completed.  The bulk copies read the set through the async proxy, hence
+  // the proxy fence after the acquire.
+  auto wait_set = [&]() {
+    if (cready) {
+      if (cready != acquired) {
+        wait_flag(cready, *p.epoch + 1u, abort_flag, p.status);
+        fence_proxy_async_global();
+        acquired = cready;
+      }
+    } else if (cdep && !waited) {
+      pdl_wait();
+      waited = true;
+    }
+  };
   for (int i = 0;; ++i) {
     Piece pc;
     if (i < nhome) {
@@ -267,39 +295,40 @@ __device__ __forceinline__ void mma_scheduler(const AttnMmaParams& P, unsigned c
         pc.r1 = uend;
         pc.ordinal = uord;
         urow = uend;
+        seg_fields(pc.seg);
+        // A set of a rule that may leave it shorter than its capacity is
+        // ascending with -1 padding at its end: the unit keeps its tiles up
+        // to the first one that starts with padding (at least one tile, so
+        // that the piece still writes its partial state: an empty softmax,
+        // which the cross-piece combine skips).  The tiles dropped here
+        // would have fetched no bytes, but they would still take their
+        // turn in the pipeline.
+        if (ckind == kSparse && cpad) {
+          wait_set();
+          constexpr int UT = kPoolTiles > kPoolTilesDep ? kPoolTiles : kPoolTilesDep;
+          int32_t first[UT];
+          const int nt = (pc.r1 - pc.r0 + kTileRows - 1) / kTileRows;
+#pragma unroll
+          for (int j = 0; j < UT; ++j) first[j] = j < nt ? __ldcg(cidx + pc.r0 + j * kTileRows) : -1;
+          int keep = 1;
+#pragma unroll
+          for (int j = 1; j < UT; ++j)
+            if (keep == j && first[j] >= 0) keep = j + 1;
+          if (first[0] < 0) pc.r1 = pc.r0 + 1;  // one padding row
+          else pc.r1 = min(pc.r1, pc.r0 + keep * kTileRows);
+        }
       }
       ring[r] = pc;
       mbar_arrive(&unit_full[r]);  // release: the entry above
       if (pc.seg < 0) break;
     }
-    if (pc.seg != cseg) {  // the segment's fields, kept across its consecutive pieces
-      const Segment& sg = p.segs[pc.seg];
-      cseg = pc.seg;
-      ckind = sg.kind;
-      cready = sg.ready;
-      cdep = sg.dep;
-      cidx = sg.idx;
-    }
+    seg_fields(pc.seg);
     if (ckind != kSparse) {
       for (int r0 = pc.r0; r0 < pc.r1; r0 += kTileRows, ++t)
         if (!slot_free(t)) return;
       continue;
     }
-    // A set that a selection of this step writes is read once that
-    // selection has raised its ready flag (the selection may still be
-    // running).  Otherwise a set the previous launch writes is read once
-    // that launch has completed.  The bulk copies read the set through the
-    // async proxy, hence the proxy fence after the acquire.
-    if (cready) {
-      if (cready != acquired) {
-        wait_flag(cready, *p.epoch + 1u, abort_flag, p.status);
-        fence_proxy_async_global();
-        acquired = cready;
-      }
-    } else if (cdep && !waited) {
-      pdl_wait();
-      waited = true;
-    }
+    wait_set();
     for (int r0 = pc.r0; r0 < pc.r1; r0 += kTileRows, ++t) {
       const int slot = t % C::IR;
       if (!slot_free(t)) return;

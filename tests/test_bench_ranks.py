@@ -96,6 +96,36 @@ def test_traffic_record_lookup(tmp_path, monkeypatch):
     assert bench.profiled_traffic("w1", "kvgroup_mean") is None
 
 
+def test_traffic_record_from_capture(tmp_path, monkeypatch, capsys):
+    """--traffic-from sums one step's attention launches of an ncu capture
+    (read + write, any byte unit), divides by the layers and stamps the
+    record with the source hash; a capture of the wrong length is refused."""
+    import json
+
+    import bench
+    head = ('"ID","Process ID","Process Name","Host Name","Kernel Name","Context","Stream",'
+            '"Block Size","Grid Size","Device","CC","Section Name","Metric Name","Metric Unit",'
+            '"Metric Value"\n')
+    rows = []
+    vals = [(100.0, "Mbyte", 1.5, "Mbyte"), (200.0, "Mbyte", 2.5, "Mbyte"), (1024.0, "byte", 0.0, "byte")]
+    for i, (r, ru, w, wu) in enumerate(vals):
+        k = '"void attn_mma_layer_kernel<128, 6, 8, 6, 0, 0>(AttnMmaParams)"'
+        base = f'"{i}","1","python","h",{k},"1","7","(512, 1, 1)","(148, 1, 1)","0","10.0","m",'
+        rows.append(base + f'"dram__bytes_read.sum","{ru}","{r}"\n')
+        rows.append(base + f'"dram__bytes_write.sum","{wu}","{w}"\n')
+    csvf = tmp_path / "t.csv"
+    csvf.write_text("==PROF== noise\n" + head + "".join(rows))
+    monkeypatch.setattr(bench, "attn_source_hash", lambda: "feed")
+    assert bench.main(["--traffic-from", str(csvf), "--layers", "2"]) == 0
+    line = capsys.readouterr().out.strip()
+    assert line.startswith("traffic-record: ")
+    rec = json.loads(line.split(":", 1)[1])
+    assert rec["source_sha"] == "feed" and rec["launches"] == 3
+    assert rec["workload"] == "llama3-8b-attn-stack-n131072-k4096-L2-r2"
+    assert rec["bytes_per_launch"] == round((300e6 + 4e6 + 1024) / 2)
+    assert bench.main(["--traffic-from", str(csvf), "--layers", "3"]) == 2
+
+
 def test_reference_arm_times_whole_steps_on_the_library_arms_config(capsys):
     """The oracle arm runs whole L-layer steps of the chosen workload and
     reports the same config as the library arm (a small override of the

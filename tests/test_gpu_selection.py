@@ -141,9 +141,41 @@ def test_rule_variable_sets_as_input(lyc):
         for h in range(spec.Hq):
             m = int(rng.integers(1, spec.k + 1))
             s0[b, h, :m] = np.sort(rng.choice(spec.n, size=m, replace=False))
-    data, rc, out, S, tr = run_rule(lyc, spec, sel, s_in=s0)
+    data = W.make_stack(spec, "cuda")
+    data["role"][0] = data["role"][1]  # layer 0 obeys its role row: its sparse heads read s0
+    assert 0 < data["role"][0].sum() < spec.Hq
+    data, rc, out, S, tr = run_rule(lyc, spec, sel, data=data, s_in=s0)
     assert rc == 0, lyc.status_string(rc)
     om = O.SELECT_PER_QHEAD
+    P.check_layers(data, out, tr, spec.k, spec.n, spec.dtype, range(spec.L), select_mode=om,
+                   S0=s0, sel=sel)
+
+
+@pytest.mark.parametrize("select_mode", ["per_qhead", "kvgroup_mean"])
+def test_rule_short_sets_many_units(lyc, select_mode):
+    """Caller sets of every length class against a capacity of four pool
+    units (k = 2048): one row, a part of a tile, whole tiles, a unit and a
+    row past it, up to the capacity.  Units and tiles past a set's valid
+    rows are dropped on the device; the outputs must still match the oracle,
+    and the sets the later layers select under the rule too."""
+    sel = RULES["topp-0.9"]
+    spec = SPEC.with_(n=5000, k=2048, L=3, name="rules-short-sets-k2048")
+    Hs = spec.Hq if select_mode == "per_qhead" else spec.Hkv
+    lengths = [1, 63, 64, 65, 511, 512, 513, 1000, 1536, 1537, 2047, 2048, 700, 129, 1025, 3]
+    rng = np.random.default_rng(11)
+    s0 = np.full((spec.B, Hs, spec.k), -1, dtype=np.int32)
+    i = 0
+    for b in range(spec.B):
+        for h in range(Hs):
+            m = lengths[i % len(lengths)]
+            i += 1
+            s0[b, h, :m] = np.sort(rng.choice(spec.n, size=m, replace=False))
+    data = W.make_stack(spec, "cuda")
+    data["role"][0] = data["role"][1]  # layer 0 obeys its role row: its sparse heads read s0
+    assert 0 < data["role"][0].sum() < spec.Hq
+    data, rc, out, S, tr = run_rule(lyc, spec, sel, select_mode=select_mode, data=data, s_in=s0)
+    assert rc == 0, lyc.status_string(rc)
+    om = O.SELECT_PER_QHEAD if select_mode == "per_qhead" else O.SELECT_KVGROUP_MEAN
     P.check_layers(data, out, tr, spec.k, spec.n, spec.dtype, range(spec.L), select_mode=om,
                    S0=s0, sel=sel)
 

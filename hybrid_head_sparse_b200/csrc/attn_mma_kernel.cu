@@ -45,14 +45,6 @@ namespace lyc {
 
 typedef uint16_t bf16_t;  // bf16 bit pattern
 
-struct AttnMmaParams {
-  CUtensorMap tmk;  // 5-D map of K: (d, row, g, b, l), box 64 x 64, 128B swizzle
-  CUtensorMap tmv;  // same for V
-  CUtensorMap tgk;  // 2-D map of K: (d, flattened row), box 64 x 1, 128B swizzle (row gathers)
-  CUtensorMap tgv;  // same for V
-  AttnParams p;
-};
-
 template <int D, int NC, int NP, int STAGES, bool GT>
 struct MmaCfg {
   // warps: NC consumers, one epilogue warp, one scheduler warp, NP producers

@@ -33,14 +33,6 @@
 
 namespace lyc {
 
-struct AttnMmaParams {  // layout shared with attn_mma_kernel.cu and lyc_api.cu
-  CUtensorMap tmk;      // 5-D map of K: (d, row, g, b, l); box 64 x kTcRows here
-  CUtensorMap tmv;
-  CUtensorMap tgk;
-  CUtensorMap tgv;
-  AttnParams p;
-};
-
 namespace {
 
 typedef uint16_t bf16_t;

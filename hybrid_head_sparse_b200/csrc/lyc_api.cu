@@ -23,13 +23,6 @@
 #include "lyc_plan.h"
 
 namespace lyc {
-struct AttnMmaParams {
-  CUtensorMap tmk;
-  CUtensorMap tmv;
-  CUtensorMap tgk;
-  CUtensorMap tgv;
-  AttnParams p;
-};
 int attn_nq_bucket(int nq);
 cudaError_t attn_simt_dispatch(int D, int nqb, const AttnParams* p, int grid, cudaStream_t stream,
                                int* smem_out, bool configure_only);

@@ -154,6 +154,16 @@ struct AttnParams {
   float scale;               // 1 / sqrt(d)
 };
 
+// The launch parameters of the bf16 attention kernels (mma.sync and
+// tcgen05): the tensor maps of the cache, then the work list.
+struct AttnMmaParams {
+  CUtensorMap tmk;  // 5-D map of K: (d, row, g, b, l), 128B swizzle; box 64 x the kernel's tile rows
+  CUtensorMap tmv;  // same for V
+  CUtensorMap tgk;  // 2-D map of K: (d, flattened row), box 64 x 1, 128B swizzle (row gathers)
+  CUtensorMap tgv;  // same for V
+  AttnParams p;
+};
+
 struct TopkTask {
   const float* keys;  // n selection keys
   int32_t* S;         // the launch's k outputs

@@ -39,13 +39,6 @@
 
 namespace lyc {
 
-struct AttnMmaParams {  // layout shared with attn_mma_kernel.cu
-  CUtensorMap tmk;
-  CUtensorMap tmv;
-  CUtensorMap tgk;
-  CUtensorMap tgv;
-  AttnParams p;
-};
 cudaError_t attn_mma_dispatch(int D, const AttnMmaParams* P, int grid, cudaStream_t stream,
                               int* smem_out, bool configure_only);
 

@@ -75,6 +75,10 @@ def parse_args(argv=None):
                     help="Cache Correction instead: dense causal attention of the T most recent "
                          "positions over the cache (lyc_cache_correction), one line")
     ap.add_argument("--T", type=int, default=32, help="Cache Correction: positions refreshed")
+    ap.add_argument("--noalloc", action="store_true",
+                    help="the allocation-free entry point instead: one layer of sparse heads "
+                         "over given sets (lyc_sparse_attention_noalloc), every head sparse, "
+                         "batch 8 unless --batch, one line")
     ap.add_argument("--shard", choices=["heads", "batch"], default=None,
                     help="under torchrun: split one step over the ranks (KV groups with their "
                          "query heads, or batch elements), all-gather the outputs and sets every "
@@ -1091,6 +1095,86 @@ def run_rule(args):
     return 0
 
 
+def run_noalloc(args):
+    """lyc_sparse_attention_noalloc on one GPU: one layer of the Llama3-8B
+    shapes with every query head sparse, each over its own set of k scattered
+    rows (ascending, seeded), B*Hq sets per call.  The timed region is K calls
+    on resident inputs; the rate counts the K/V rows the sets name."""
+    import numpy as np
+    import torch
+
+    from hybrid_head_sparse_b200 import build as Bld
+    from hybrid_head_sparse_b200 import lyc, workloads as W
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    Bld.build()
+    lyc.load()
+    base = workload_spec(args)
+    spec = base.with_(L=1, B=args.batch or 8, planted="none")
+    B, Hq, Hkv, d, n, k = spec.B, spec.Hq, spec.Hkv, spec.d, spec.n, spec.k
+    data = W.make_stack(spec, dev)
+    rng = np.random.default_rng(spec.seed + 7)
+    S = np.empty((B, Hq, k), dtype=np.int32)
+    for b in range(B):
+        for h in range(Hq):
+            S[b, h] = np.sort(rng.choice(n, size=k, replace=False))
+    S = torch.from_numpy(S).to(dev)
+    out = torch.empty((B, Hq, d), device=dev)
+    status = torch.zeros((1,), dtype=torch.int32, device=dev)
+    kv = lyc.lyc_kv_cache(data["k"].data_ptr(), data["v"].data_ptr(), n, 0, *data["k"].stride()[1:4])
+    stream = torch.cuda.current_stream(dev)
+
+    def call():
+        rc = lyc.lyc_sparse_attention_noalloc(data["q"].data_ptr(), kv, B, Hq, Hkv, d, S.data_ptr(),
+                                              k, out.data_ptr(), status.data_ptr(),
+                                              stream.cuda_stream)
+        if rc != lyc.LYC_OK:
+            raise RuntimeError(lyc.lyc_status_string(rc))
+
+    for _ in range(max(args.warmup, 3)):
+        call()
+    torch.cuda.synchronize()
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {int(status.item())}")
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    with ClockSampler(0) as clk:
+        evs[0].record(stream)
+        for i in range(args.steps):
+            call()
+            evs[i + 1].record(stream)
+        torch.cuda.synchronize()
+    ms_total = evs[0].elapsed_time(evs[-1])
+    per = [evs[i].elapsed_time(evs[i + 1]) for i in range(args.steps)]
+    ms_call = ms_total / args.steps
+    kv_bytes = B * Hq * k * d * 2 * 2
+    peak, peak_kind = measured_peaks()
+    gbs = kv_bytes / (ms_call / 1e3) / 1e9
+    line = {
+        "metric": f"allocation-free sparse attention calls/s ({B * Hq} sets of {k} rows, {n // 1024}K ctx)",
+        "value": args.steps / (ms_total / 1e3), "unit": "calls/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": ms_call,
+        "step_ms_distribution": {kk: round(v, 4) for kk, v in percentiles(per).items()},
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) q/K/V; seeded scattered ascending sets)",
+        "config": {"workload": f"llama3-8b-noalloc-b{B}-n{n}-k{k}", "B": B, "Hq": Hq, "Hkv": Hkv,
+                   "d": d, "n": n, "k": k, "parallelism": "replicas x1",
+                   "l2": "inputs larger than L2 (%.2f GB of K/V rows per call)" % (kv_bytes / 1e9)},
+        "roofline": {"bound": "hbm", "kernel": "attn_mma_layer_kernel (gathered segments only) "
+                                               "+ its work-list and combine launches",
+                     "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(gbs / peak, 4),
+                     "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
+                     "traffic": None, "algorithmic_bytes_per_launch": kv_bytes,
+                     "avg_launch_ms": ms_call,
+                     "note": "achieved = K+V bytes of the rows the sets name / CUDA-event time of "
+                             "the whole call (work-list kernel, attention, combine, status copy)"},
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def traffic_record(args) -> int:
     """The traffic record line of an ncu capture of this command's attention
     launches (`ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum -k
@@ -1134,6 +1218,8 @@ def main(argv=None):
         return run_serving(args)
     if args.correction:
         return run_correction(args)
+    if args.noalloc:
+        return run_noalloc(args)
     if args.shard:
         return run_sharded(args)
     if args.selection != "topk":

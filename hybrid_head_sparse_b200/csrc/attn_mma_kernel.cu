@@ -90,8 +90,16 @@ struct MmaCfg {
 // first, then the pool pieces the scheduler took, from the ring (false at the
 // end of both).  Each warp calls it for i = 0, 1, ... in order.
 template <class C>
-__device__ __forceinline__ bool cta_piece(const AttnParams& p, unsigned char* smem, int pbeg, int nhome,
-                                          int i, int lane, Piece* out) {
+// pbeg, pend: the CTA's range in the piece list (read only when needed, so
+// that a CTA whose first piece is in the launch parameters does not wait for
+// that read before its first piece).
+__device__ __forceinline__ bool cta_piece(const AttnParams& p, unsigned char* smem, int pbeg, int pend,
+                                          int i, int lane, Piece* out, const FirstPiece* fp = nullptr) {
+  if (i == 0 && fp && fp->pc.seg >= 0) {  // from the launch parameters
+    *out = fp->pc;
+    return true;
+  }
+  const int nhome = pend - pbeg;
   if (i < nhome) {
     *out = p.pieces[pbeg + i];
     return true;
@@ -358,8 +366,6 @@ __device__ __forceinline__ void mma_producers(const AttnMmaParams& P, unsigned c
   const uint64_t pol_keep = l2_policy_evict_normal();  // gathered rows may be read again
   const bool leader = ptid == 0;
 
-  const int nhome = pend - pbeg;
-
   constexpr int CH = D / 8;                  // 16-byte chunks per row
   constexpr int ROWS_W = kTileRows / NP;     // rows per producer warp
   uint32_t idx_phase = 0;
@@ -375,10 +381,19 @@ __device__ __forceinline__ void mma_producers(const AttnMmaParams& P, unsigned c
   const int32_t* bt = nullptr;
   int sl = 0, sb = 0, sgg = 0, nvalid = 0, page_rows = 0;
   int32_t pad_ok = 0, row_base = 0;
+  const FirstPiece* fp = static_cast<int>(blockIdx.x) < P.nfirst ? &P.first[blockIdx.x] : nullptr;
   for (int pi = 0;; ++pi) {
     Piece pc;
-    if (!cta_piece<C>(p, smem, pbeg, nhome, pi, lane, &pc)) break;
-    if (pc.seg != cseg) {
+    if (!cta_piece<C>(p, smem, pbeg, pend, pi, lane, &pc, fp)) break;
+    if (pi == 0 && fp && fp->pc.seg >= 0) {
+      // a dense piece of this launch's layer: the tile copies need no more
+      // (the next piece reads its segment's fields)
+      dense = true;
+      sgg = fp->g;
+      sb = fp->b;
+      sl = p.layer;
+      cseg = -1;
+    } else if (pc.seg != cseg) {
       const Segment& sg = p.segs[pc.seg];
       cseg = pc.seg;
       dense = sg.kind == kDense;
@@ -585,17 +600,17 @@ __device__ __forceinline__ void mma_consumers(const AttnMmaParams& P, unsigned c
   int64_t koff0 = -1, koff1 = -1, key_mean_off = -1;
   float mean_scale = 0.f;
   uint32_t qb[KSTEPS][2];
-  const int nhome = pend - pbeg;
+  const FirstPiece* fp = static_cast<int>(blockIdx.x) < P.nfirst ? &P.first[blockIdx.x] : nullptr;
   for (int pi = 0;; ++pi) {
     // the CTA's own pieces (the dense runs, the only writers of selection
     // keys) come first: once past them, this warp's keys are written
-    if (pi == nhome && nhome > 0 && p.keys_done) {
+    if (pi > 0 && pi == pend - pbeg && p.keys_done) {
       __syncwarp();
       if (lane == 0) keys_arrive(p, 1u);
       __syncwarp();
     }
     Piece pc;
-    if (!cta_piece<C>(p, smem, pbeg, nhome, pi, lane, &pc)) break;
+    if (!cta_piece<C>(p, smem, pbeg, pend, pi, lane, &pc, fp)) break;
     const int ntile = (pc.r1 - pc.r0 + kTileRows - 1) / kTileRows;
     // A piece of one tile belongs to the one warp that takes its tile: that
     // warp writes the piece's partial state (or, for a segment of one piece,
@@ -935,7 +950,7 @@ __device__ __forceinline__ void mma_epilogue(const AttnMmaParams& P, unsigned ch
   int t = 0;  // CTA-wide tile sequence number, as the consumers count it
   for (int pi = 0;; ++pi) {
     Piece pc;
-    if (!cta_piece<C>(p, smem, pbeg, pend - pbeg, pi, lane, &pc)) break;
+    if (!cta_piece<C>(p, smem, pbeg, pend, pi, lane, &pc)) break;
     const int t0 = t;
     t += (pc.r1 - pc.r0 + kTileRows - 1) / kTileRows;
     if (pc.r1 - pc.r0 <= kTileRows) continue;

@@ -78,6 +78,7 @@ struct LayerPlan {
   int topk_cl = 16;          // cluster size of the selection launch
   int topk_n = 0;            // keys of the longest selection task
   int keys_ctas = 0;         // CTAs with pieces of their own (dense runs) in the launch
+  std::vector<FirstPiece> first;  // mma kernel: each CTA's first piece, for the launch parameters
 };
 
 struct Plan {
@@ -810,6 +811,26 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const KvVie
     lp.off_pool = take(std::max<size_t>(1, H.pool_units.size()) * sizeof(Piece));
     lp.keys_ctas = 0;
     for (size_t c = 0; c + 1 < H.cta.size(); ++c) lp.keys_ctas += H.cta[c + 1] > H.cta[c] ? 1 : 0;
+    // the first piece of each CTA, when it is a dense piece of a contiguous
+    // cache (the only kind the kernel can start from the parameters)
+    lp.first.clear();
+    if (use_pool && !plan->paged) {
+      const int nf = std::min(H.grid, kFirstPieces);
+      lp.first.resize(nf);
+      for (int c = 0; c < nf; ++c) {
+        FirstPiece& f = lp.first[c];
+        f.pc.seg = -1;
+        f.pc.r0 = f.pc.r1 = f.pc.ordinal = 0;
+        f.g = f.b = 0;
+        if (H.cta[c + 1] <= H.cta[c]) continue;
+        const Piece& pc = H.pieces[H.cta[c]];
+        const Segment& sg = H.segs[pc.seg];
+        if (sg.kind != kDense || sg.l != l) continue;
+        f.pc = pc;
+        f.g = static_cast<int16_t>(sg.g);
+        f.b = static_cast<int16_t>(sg.b);
+      }
+    }
   }
   plan->off_final_src = take(hl[L - 1].final_src.size() * sizeof(void*));
   plan->nfill = static_cast<int>(fill_src.size());
@@ -1001,6 +1022,7 @@ lyc_status enqueue_step(lyc_ctx* ctx, Plan* plan, cudaStream_t stream, int set, 
     if (st != LYC_OK) return st;
     if (dtype == 0) {
       AttnMmaParams mp;
+      memset(&mp, 0, sizeof mp);
       mp.tmk = plan->tmk;
       mp.tmv = plan->tmv;
       mp.tgk = plan->tgk;
@@ -1009,6 +1031,10 @@ lyc_status enqueue_step(lyc_ctx* ctx, Plan* plan, cudaStream_t stream, int set, 
       mp.p.gather_rows = plan->gather_rows;
       mp.p.paged = plan->paged ? 1 : 0;
       if (l > 0) set_prev_combine(ctx, plan, l - 1, &mp.p);
+      if (!plan->use_tc && !lp.first.empty()) {
+        mp.nfirst = static_cast<int32_t>(lp.first.size());
+        memcpy(mp.first, lp.first.data(), lp.first.size() * sizeof(FirstPiece));
+      }
       LYC_CUDA(plan->use_tc ? attn_tc_dispatch(&mp, lp.grid, stream, nullptr, false)
                             : attn_mma_dispatch(D, &mp, lp.grid, stream, nullptr, false),
                "attention launch");
@@ -1051,6 +1077,7 @@ lyc_status enqueue_step(lyc_ctx* ctx, Plan* plan, cudaStream_t stream, int set, 
   if (dtype == 0) {
     // the last layer's cross-piece combine: the same kernel with no pieces
     AttnMmaParams mp;
+    memset(&mp, 0, sizeof mp);
     mp.tmk = plan->tmk;
     mp.tmv = plan->tmv;
     mp.tgk = plan->tgk;

@@ -154,6 +154,17 @@ struct AttnParams {
   float scale;               // 1 / sqrt(d)
 };
 
+// The first piece of a CTA (mma kernel), carried in the launch parameters:
+// the CTA issues its first tile copies, and starts reading its first
+// segment, without first reading its piece list from global memory (three
+// dependent reads, about 2 us of every CTA's start).  Only a dense piece of
+// a contiguous cache is carried.
+constexpr int kFirstPieces = 148;
+struct FirstPiece {
+  Piece pc;        // seg < 0: none (the CTA reads its pieces from the list)
+  int16_t g, b;    // the piece's KV group and batch element (of the launch's layer)
+};
+
 // The launch parameters of the bf16 attention kernels (mma.sync and
 // tcgen05): the tensor maps of the cache, then the work list.
 struct AttnMmaParams {
@@ -162,7 +173,10 @@ struct AttnMmaParams {
   CUtensorMap tgk;  // 2-D map of K: (d, flattened row), box 64 x 1, 128B swizzle (row gathers)
   CUtensorMap tgv;  // same for V
   AttnParams p;
+  int32_t nfirst;   // CTAs 0 .. nfirst-1 have an entry in `first` (0: none)
+  FirstPiece first[kFirstPieces];
 };
+static_assert(sizeof(AttnMmaParams) <= 4096, "kernel parameters are at most 4 KiB");
 
 struct TopkTask {
   const float* keys;  // n selection keys

@@ -380,9 +380,8 @@ lyc_status lyc_set_timeline(lyc_ctx* ctx, unsigned long long* buf, int cap);
  * (different streams with no ordering between them, or host threads racing)
  * race on it.
  * Set-up: the first call on a device (with that device current) looks up the
- * array's address with cudaGetSymbolAddress and sets the kernel's attributes;
- * make that first call before any stream capture.  A host mutex serializes
- * the calls' host side.
+ * array's address with cudaGetSymbolAddress and sets the kernel's attributes.
+ * A host mutex serializes the calls' host side.
  * Errors: INVALID_ARG (pointers, alignment, shapes, k), UNSUPPORTED (d, group
  * size), SCRATCH_LIMIT, CUDA. */
 #define LYC_NOALLOC_MAX_SETS 256

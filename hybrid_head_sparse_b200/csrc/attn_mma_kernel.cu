@@ -518,11 +518,13 @@ __device__ __forceinline__ int cta_ring(const unsigned char* smem) {
   return *reinterpret_cast<const volatile int*>(smem + C::OFF_FLAGS + 4);
 }
 
-// One arrival of `cnt` on the step counter of the launch's selection keys
-// (release: the caller's warp or CTA barrier orders its threads' key stores
-// before it); the selection starts once the counter reaches keys_ctas * NC.
-__device__ __forceinline__ void keys_arrive(const AttnParams& p, uint32_t cnt) {
-  red_release_add_u32(p.keys_done + (*p.epoch & 1u) * p.pool_stride, cnt);
+// One arrival of `cnt` on the step counter of layer `layer`'s selection keys
+// (the counters of a launch's layers are consecutive, from the first
+// layer's; release: the caller's warp or CTA barrier orders its threads' key
+// stores before it); that layer's selection starts once its counter reaches
+// (CTAs with dense pieces of the layer) * NC.
+__device__ __forceinline__ void keys_arrive(const AttnParams& p, int layer, uint32_t cnt) {
+  red_release_add_u32(p.keys_done + (*p.epoch & 1u) * p.pool_stride + (layer - p.layer), cnt);
 }
 
 // A one-tile piece's result from the warp that computed it, for one of the
@@ -601,16 +603,30 @@ __device__ __forceinline__ void mma_consumers(const AttnMmaParams& P, unsigned c
   float mean_scale = 0.f;
   uint32_t qb[KSTEPS][2];
   const FirstPiece* fp = static_cast<int>(blockIdx.x) < P.nfirst ? &P.first[blockIdx.x] : nullptr;
+  // The CTA's own pieces (its dense runs, the only writers of selection keys,
+  // in layer order) come first: once past a layer's, this warp's keys of
+  // that layer are written.  home_l: the layer of the own pieces so far.
+  int home_l = -1;
+  auto keys_written = [&](int layer) {
+    __syncwarp();
+    if (lane == 0) keys_arrive(p, layer, 1u);
+    __syncwarp();
+  };
   for (int pi = 0;; ++pi) {
-    // the CTA's own pieces (the dense runs, the only writers of selection
-    // keys) come first: once past them, this warp's keys are written
-    if (pi > 0 && pi == pend - pbeg && p.keys_done) {
-      __syncwarp();
-      if (lane == 0) keys_arrive(p, 1u);
-      __syncwarp();
+    if (home_l >= 0 && pi == pend - pbeg) {
+      keys_written(home_l);
+      home_l = -1;
     }
     Piece pc;
     if (!cta_piece<C>(p, smem, pbeg, pend, pi, lane, &pc, fp)) break;
+    // an own piece of another layer: the keys of the layer before are done
+    // (every warp sees every piece, those it leaves to others included)
+    if (p.keys_done && ((pi == 0 && fp && fp->pc.seg >= 0) || pi < pend - pbeg)) {
+      // (a first piece from the parameters is of the launch's first layer)
+      const int sl = (pi == 0 && fp && fp->pc.seg >= 0) ? p.layer : p.segs[pc.seg].l;
+      if (home_l >= 0 && sl != home_l) keys_written(home_l);
+      home_l = sl;
+    }
     const int ntile = (pc.r1 - pc.r0 + kTileRows - 1) / kTileRows;
     // A piece of one tile belongs to the one warp that takes its tile: that
     // warp writes the piece's partial state (or, for a segment of one piece,
@@ -1046,10 +1062,16 @@ __global__ void __launch_bounds__(MmaCfg<D, NC, NP, STAGES, GT>::kThreads, 1)
   if (cta_ring<C>(smem) >= P.p.wpart_slots) {
     if (threadIdx.x == 0) {
       atomicOr(P.p.status, kStatusScratch);
-      // no work, but the arrivals of its consumer warps, so that the
-      // selection does not wait out its limit
-      if (P.p.keys_done && P.p.cta_begin[blockIdx.x + 1] > P.p.cta_begin[blockIdx.x])
-        keys_arrive(P.p, NC);
+      // no work, but the arrivals of its consumer warps for every layer it
+      // has own pieces of, so that no selection waits out its limit
+      if (P.p.keys_done) {
+        int last = -1;
+        for (int i = P.p.cta_begin[blockIdx.x]; i < P.p.cta_begin[blockIdx.x + 1]; ++i) {
+          const int sl = P.p.segs[P.p.pieces[i].seg].l;
+          if (sl != last) keys_arrive(P.p, sl, NC);
+          last = sl;
+        }
+      }
     }
   } else {
     const int pbeg = P.p.cta_begin[blockIdx.x];

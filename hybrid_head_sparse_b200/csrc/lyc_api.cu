@@ -59,7 +59,18 @@ constexpr int kPlanCacheSize = 16;
 // wrote in the next layer's launch).  A selection starts writing only once
 // the attention launch of the layer before it has completed, so the buffer it
 // overwrites must hold a set written three refreshes ago: three buffers.
-constexpr int kSetBuffers = 3;
+// Layers per attention launch (mma kernel): each launch runs the dense rows
+// and gathered rows of this many consecutive layers, so that a CTA's fixed
+// cost (its start, the wait for its first tiles, its drain) is paid once per
+// that many layers; the selections stay one launch per layer.
+constexpr int kLayersPerLaunch = 2;
+// Buffers per set slot.  A selection overwrites the set that its slot held
+// kSetBuffers refreshes earlier.  That set's last readers run in the launch
+// of the layer that last read it, or, for a deferred pass, of the layer
+// after; a selection waits only for the attention launch before its own
+// layer's launch, so kLayersPerLaunch + 2 buffers keep every reader of the
+// overwritten set in a launch that has completed.
+constexpr int kSetBuffers = kLayersPerLaunch + 2;
 
 
 int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
@@ -77,8 +88,14 @@ struct LayerPlan {
   int64_t pool_tiles = 0, tiles = 0;  // tiles in the pool, in the whole layer
   int topk_cl = 16;          // cluster size of the selection launch
   int topk_n = 0;            // keys of the longest selection task
-  int keys_ctas = 0;         // CTAs with pieces of their own (dense runs) in the launch
+  int keys_ctas = 0;         // CTAs with dense pieces of this layer (the writers of its keys)
   std::vector<FirstPiece> first;  // mma kernel: each CTA's first piece, for the launch parameters
+  // the attention launch: this layer's record holds it when the layer is the
+  // first of the launch's layers [layer, layer + nlayers); the other layers
+  // of the launch have none (attn false) but keep their selection launch
+  bool attn = true;
+  int nlayers = 1;
+  int launch = 0;            // ordinal of the attention launch in the step
 };
 
 struct Plan {
@@ -469,6 +486,9 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const KvVie
     // mma kernel: the previous layer's sparse passes over the sets that the
     // selection before it wrote, run by this launch (see below)
     std::vector<Segment> deferred;
+    int keys_ctas = 0;        // CTAs with dense pieces of this layer
+    bool attn = true;         // this layer's record holds an attention launch
+    int nlayers = 1;          // ... of the layers [this one, this one + nlayers)
   };
   std::vector<HostLayer> hl(L);
   std::vector<int> cur(Hs, 0);
@@ -623,123 +643,6 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const KvVie
     }
     H.nqb = attn_nq_bucket(maxnq);
 
-    // Workload pooling.  The dense rows are cut into equal runs of tiles, one
-    // per CTA.  The gathered rows:
-    //  * mma kernel: go to a pool of kPoolTiles-tile units, which the CTAs
-    //    take at run time once their dense run is done (an atomic cursor per
-    //    launch), sets of earlier selections first, those the previous
-    //    layer's selection writes (the only rows that wait for it) last.  A
-    //    CTA that starts late (the launches of consecutive layers overlap) or
-    //    streams slowly then simply takes fewer units;
-    //  * other kernels: are cut into equal runs too, taken after the dense
-    //    run, the previous selection's sets last, so that few CTAs wait, and
-    //    late.
-    int64_t NT = 0;
-    for (const Segment& sg : H.segs) NT += (sg.rows + TR - 1) / TR;
-    // The previous layer's selection runs beside this layer's attention (the
-    // attention streams its dense rows meanwhile and waits for the sets only
-    // before its gathered rows).  When that selection is small, leave its SMs
-    // to it: fewer SMs still stream at full HBM bandwidth, and no CTA of this
-    // kernel then starts late behind it.
-    int avail = ctx->sms;
-    if (l > 0) {
-      const int prev = static_cast<int>(hl[l - 1].tasks.size()) * hl[l - 1].topk_cl;
-      if (prev > 0 && 2 * prev <= ctx->sms / 4) avail = ctx->sms - 2 * prev;
-      else if (prev > 0 && prev <= ctx->sms / 4) avail = ctx->sms - prev;
-    }
-    // The grid leaves the SMs of the previous selection and of this layer's
-    // own to them: the selection of this layer starts on its key flag, while
-    // the previous one may still run, and takes free SMs at once (measured on
-    // B200: +1.9 % in KV-group mode for a grid that leaves one selection's SMs
-    // against one with CTAs that take them back for pool units).
-    H.tiles = NT;
-    // A launch with no rows of its own (a layer without retrieval heads whose
-    // sparse passes all moved to the next launch) still runs: its CTAs merge
-    // the previous launch's split rows and raise its done flag.
-    int grid = static_cast<int>(std::min<int64_t>(NT, avail));
-    if (grid == 0)
-      grid = std::max(1, std::min(avail, l > 0 ? static_cast<int>(hl[l - 1].combine.size()) : 1));
-    H.grid = grid;
-    std::vector<int> npieces(H.segs.size(), 0);
-    std::vector<std::vector<Piece>> per_cta(grid);
-    for (int phase = 0; phase < (use_pool ? 1 : 2); ++phase) {
-      std::vector<size_t> ids;
-      std::vector<int64_t> tstart(1, 0);
-      for (int dep = 0; dep < 2; ++dep) {
-        for (size_t s2 = 0; s2 < H.segs.size(); ++s2) {
-          const Segment& cs = H.segs[s2];
-          if ((cs.kind == kDense ? 0 : 1) != phase || (phase == 1 && cs.dep != dep) ||
-              (phase == 0 && dep == 1))
-            continue;
-          ids.push_back(s2);
-          tstart.push_back(tstart.back() + (cs.rows + TR - 1) / TR);
-        }
-      }
-      const int64_t nt = tstart.back();
-      const int cut = grid;
-      size_t si = 0;
-      for (int c = 0; c < cut; ++c) {
-        const int64_t t0 = nt * c / cut, t1 = nt * (c + 1) / cut;
-        while (si < ids.size() && tstart[si + 1] <= t0) ++si;
-        for (size_t q = si; q < ids.size() && tstart[q] < t1; ++q) {
-          const int64_t a = std::max(t0, tstart[q]) - tstart[q];
-          const int64_t e = std::min(t1, tstart[q + 1]) - tstart[q];
-          if (e <= a) continue;
-          Piece pc;
-          pc.seg = static_cast<int32_t>(ids[q]);
-          pc.r0 = static_cast<int32_t>(a * TR);
-          pc.r1 = static_cast<int32_t>(std::min<int64_t>(e * TR, H.segs[ids[q]].rows));
-          pc.ordinal = npieces[ids[q]]++;
-          per_cta[c].push_back(pc);
-        }
-      }
-    }
-    if (use_pool) {
-      // a gathered segment of r rows is cut into units of kPoolTiles tiles
-      // (kPoolTilesDep for a set the previous selection writes), unit q =
-      // piece q (its ordinal); CTAs take them at run time.  The pool lists
-      // the units in order, earlier selections' sets first.  (Measured on
-      // B200 against one-tile pieces whose warp writes its own partial state:
-      // per-head selection 1231 against 1348 us per step, KV-group even.)
-      for (int dep = 0; dep < 2; ++dep)
-        for (size_t s2 = 0; s2 < H.segs.size(); ++s2)
-          if (H.segs[s2].kind == kSparse && H.segs[s2].dep == dep) {
-            const int unit_tiles = dep ? kPoolTilesDep : kPoolTiles;
-            const int rows = H.segs[s2].rows;
-            int tile = 0;
-            for (int r0 = 0; r0 < rows; r0 += unit_tiles * kTileRows, tile += unit_tiles) {
-              Piece pc;
-              pc.seg = static_cast<int32_t>(s2);
-              pc.r0 = r0;
-              pc.r1 = std::min(r0 + unit_tiles * kTileRows, rows);
-              pc.ordinal = tile / unit_tiles;
-              H.pool_units.push_back(pc);
-            }
-            npieces[s2] = (rows + unit_tiles * kTileRows - 1) / (unit_tiles * kTileRows);
-            H.pool_tiles += (rows + TR - 1) / TR;
-          }
-    }
-    for (int c = 0; c < grid; ++c) {
-      H.cta.push_back(static_cast<int32_t>(H.pieces.size()));
-      for (const Piece& pc : per_cta[c]) H.pieces.push_back(pc);
-    }
-    H.cta.push_back(static_cast<int32_t>(H.pieces.size()));
-    // partial records (one per piece and output) and arrival counters (one
-    // per output; the fp32 kernel's last-arrival combine); the bf16 kernel
-    // leaves the cross-piece combine of segments cut into several pieces to
-    // the next launch, as (segment, output) tasks
-    int part = 0, cnt = 0;
-    for (size_t s = 0; s < H.segs.size(); ++s) {
-      H.segs[s].npieces = npieces[s];
-      H.segs[s].part_base = part;
-      H.segs[s].cnt_base = cnt;
-      part += npieces[s] * H.segs[s].nout;
-      cnt += H.segs[s].nout;
-      if (npieces[s] > 1)
-        for (int o = 0; o < H.segs[s].nout; ++o) H.combine.push_back(make_int2(static_cast<int>(s), o));
-    }
-    if (static_cast<size_t>(part) > ctx->max_parts || static_cast<size_t>(cnt) > ctx->max_counters)
-      return fail(ctx, LYC_ERR_UNSUPPORTED, "work pool larger than the scratch sized at create");
 
     // selection tasks of this layer, then flip the refreshed slots
     for (int s = 0; s < Hs; ++s) {
@@ -780,6 +683,175 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const KvVie
       for (int s = 0; s < Hs; ++s) H.final_src.push_back(set_ptr(cur[s], b, s));
   }
 
+
+  // ---- phase B: the attention launches.  With the mma kernel a launch runs
+  // kLayersPerLaunch consecutive layers: their segments are concatenated in
+  // layer order (each layer's own passes, then the passes deferred into it).
+  // No pass of a launch may wait for a selection enqueued after that launch
+  // (the selection could find no free SM while the launch's CTAs wait): with
+  // two layers per launch, a pass of the second layer over a set of the
+  // first layer's selection is deferred to the next launch, and the last
+  // layer, which keeps such passes, gets a launch of its own.
+  static_assert(kLayersPerLaunch >= 1 && kLayersPerLaunch <= 2,
+                "more layers per launch need passes over their own selections deferred");
+  {
+    const int LG = use_pool ? kLayersPerLaunch : 1;
+    int prev_l0 = -1;
+    for (int l0 = 0, l1 = 0; l0 < L; l0 = l1) {
+      l1 = std::min(L, l0 + LG);  // the launch's layers [l0, l1)
+      if (l1 == L && l1 - l0 > 1) l1 = L - 1;  // the last layer alone
+      HostLayer& H = hl[l0];
+      std::vector<size_t> seg_begin(1, 0);
+      seg_begin.push_back(H.segs.size());
+      for (int li = l0 + 1; li < l1; ++li) {
+        for (const Segment& sg : hl[li].segs) H.segs.push_back(sg);
+        seg_begin.push_back(H.segs.size());
+        H.nqb = std::max(H.nqb, hl[li].nqb);
+        hl[li].segs.clear();
+        hl[li].attn = false;
+      }
+      H.nlayers = l1 - l0;
+      // Workload pooling.  The dense rows are cut into equal runs of tiles, one
+      // per CTA.  The gathered rows:
+      //  * mma kernel: go to a pool of kPoolTiles-tile units, which the CTAs
+      //    take at run time once their dense run is done (an atomic cursor per
+      //    launch), sets of earlier selections first, those the previous
+      //    layer's selection writes (the only rows that wait for it) last.  A
+      //    CTA that starts late (the launches of consecutive layers overlap) or
+      //    streams slowly then simply takes fewer units;
+      //  * other kernels: are cut into equal runs too, taken after the dense
+      //    run, the previous selection's sets last, so that few CTAs wait, and
+      //    late.
+      int64_t NT = 0;
+      for (const Segment& sg : H.segs) NT += (sg.rows + TR - 1) / TR;
+      // The previous layer's selection runs beside this layer's attention (the
+      // attention streams its dense rows meanwhile and waits for the sets only
+      // before its gathered rows).  When that selection is small, leave its SMs
+      // to it: fewer SMs still stream at full HBM bandwidth, and no CTA of this
+      // kernel then starts late behind it.
+      int avail = ctx->sms;
+      {
+        // the largest selection among the one before this launch and its own
+        int prev = 0;
+        for (int li = std::max(0, l0 - 1); li < l1; ++li)
+          prev = std::max(prev, static_cast<int>(hl[li].tasks.size()) * hl[li].topk_cl);
+        if (l0 > 0 && prev > 0 && 2 * prev <= ctx->sms / 4) avail = ctx->sms - 2 * prev;
+        else if (l0 > 0 && prev > 0 && prev <= ctx->sms / 4) avail = ctx->sms - prev;
+      }
+      // The grid leaves the SMs of the previous selection and of this layer's
+      // own to them: the selection of this layer starts on its key flag, while
+      // the previous one may still run, and takes free SMs at once (measured on
+      // B200: +1.9 % in KV-group mode for a grid that leaves one selection's SMs
+      // against one with CTAs that take them back for pool units).
+      H.tiles = NT;
+      // A launch with no rows of its own (a layer without retrieval heads whose
+      // sparse passes all moved to the next launch) still runs: its CTAs merge
+      // the previous launch's split rows and raise its done flag.
+      int grid = static_cast<int>(std::min<int64_t>(NT, avail));
+      if (grid == 0)
+        grid = std::max(1, std::min(avail, prev_l0 >= 0 ? static_cast<int>(hl[prev_l0].combine.size()) : 1));
+      H.grid = grid;
+      std::vector<int> npieces(H.segs.size(), 0);
+      std::vector<std::vector<Piece>> per_cta(grid);
+      // phase 0 (dense segments) is cut per layer of the launch, so that every
+      // CTA streams a run of each layer's dense rows in layer order (the keys of
+      // the first layer are then complete early, and its selection starts)
+      for (int pass = 0; pass < (use_pool ? l1 - l0 : 2); ++pass) {
+        const int phase = use_pool ? 0 : pass;
+        const size_t sg_lo = use_pool ? seg_begin[pass] : 0;
+        const size_t sg_hi = use_pool ? seg_begin[pass + 1] : H.segs.size();
+        std::vector<size_t> ids;
+        std::vector<int64_t> tstart(1, 0);
+        for (int dep = 0; dep < 2; ++dep) {
+          for (size_t s2 = sg_lo; s2 < sg_hi; ++s2) {
+            const Segment& cs = H.segs[s2];
+            if ((cs.kind == kDense ? 0 : 1) != phase || (phase == 1 && cs.dep != dep) ||
+                (phase == 0 && dep == 1))
+              continue;
+            ids.push_back(s2);
+            tstart.push_back(tstart.back() + (cs.rows + TR - 1) / TR);
+          }
+        }
+        const int64_t nt = tstart.back();
+        const int cut = grid;
+        size_t si = 0;
+        for (int c = 0; c < cut; ++c) {
+          const int64_t t0 = nt * c / cut, t1 = nt * (c + 1) / cut;
+          while (si < ids.size() && tstart[si + 1] <= t0) ++si;
+          for (size_t q = si; q < ids.size() && tstart[q] < t1; ++q) {
+            const int64_t a = std::max(t0, tstart[q]) - tstart[q];
+            const int64_t e = std::min(t1, tstart[q + 1]) - tstart[q];
+            if (e <= a) continue;
+            Piece pc;
+            pc.seg = static_cast<int32_t>(ids[q]);
+            pc.r0 = static_cast<int32_t>(a * TR);
+            pc.r1 = static_cast<int32_t>(std::min<int64_t>(e * TR, H.segs[ids[q]].rows));
+            pc.ordinal = npieces[ids[q]]++;
+            per_cta[c].push_back(pc);
+          }
+        }
+      }
+      if (use_pool) {
+        // a gathered segment of r rows is cut into units of kPoolTiles tiles
+        // (kPoolTilesDep for a set the previous selection writes), unit q =
+        // piece q (its ordinal); CTAs take them at run time.  The pool lists
+        // the units in order, earlier selections' sets first.  (Measured on
+        // B200 against one-tile pieces whose warp writes its own partial state:
+        // per-head selection 1231 against 1348 us per step, KV-group even.)
+        for (int dep = 0; dep < 2; ++dep)
+          for (size_t s2 = 0; s2 < H.segs.size(); ++s2)
+            if (H.segs[s2].kind == kSparse && H.segs[s2].dep == dep) {
+              const int unit_tiles = dep ? kPoolTilesDep : kPoolTiles;
+              const int rows = H.segs[s2].rows;
+              int tile = 0;
+              for (int r0 = 0; r0 < rows; r0 += unit_tiles * kTileRows, tile += unit_tiles) {
+                Piece pc;
+                pc.seg = static_cast<int32_t>(s2);
+                pc.r0 = r0;
+                pc.r1 = std::min(r0 + unit_tiles * kTileRows, rows);
+                pc.ordinal = tile / unit_tiles;
+                H.pool_units.push_back(pc);
+              }
+              npieces[s2] = (rows + unit_tiles * kTileRows - 1) / (unit_tiles * kTileRows);
+              H.pool_tiles += (rows + TR - 1) / TR;
+            }
+      }
+      for (int c = 0; c < grid; ++c) {
+        H.cta.push_back(static_cast<int32_t>(H.pieces.size()));
+        for (const Piece& pc : per_cta[c]) H.pieces.push_back(pc);
+      }
+      H.cta.push_back(static_cast<int32_t>(H.pieces.size()));
+      // partial records (one per piece and output) and arrival counters (one
+      // per output; the fp32 kernel's last-arrival combine); the bf16 kernel
+      // leaves the cross-piece combine of segments cut into several pieces to
+      // the next launch, as (segment, output) tasks
+      int part = 0, cnt = 0;
+      for (size_t s = 0; s < H.segs.size(); ++s) {
+        H.segs[s].npieces = npieces[s];
+        H.segs[s].part_base = part;
+        H.segs[s].cnt_base = cnt;
+        part += npieces[s] * H.segs[s].nout;
+        cnt += H.segs[s].nout;
+        if (npieces[s] > 1)
+          for (int o = 0; o < H.segs[s].nout; ++o) H.combine.push_back(make_int2(static_cast<int>(s), o));
+      }
+      if (static_cast<size_t>(part) > ctx->max_parts || static_cast<size_t>(cnt) > ctx->max_counters)
+        return fail(ctx, LYC_ERR_UNSUPPORTED, "work pool larger than the scratch sized at create");
+      // the CTAs that write each layer's selection keys (their dense pieces)
+      for (int li = l0; li < l1; ++li) {
+        int n_ctas = 0;
+        for (int c = 0; c < grid; ++c) {
+          bool has = false;
+          for (const Piece& pc : per_cta[c])
+            has = has || (H.segs[pc.seg].kind == kDense && H.segs[pc.seg].l == li);
+          n_ctas += has ? 1 : 0;
+        }
+        hl[li].keys_ctas = n_ctas;
+      }
+      prev_l0 = l0;
+    }
+  }
+
   // ---- one device buffer for every record
   size_t bytes = 0;
   auto take = [&](size_t sz) {
@@ -789,6 +861,7 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const KvVie
     return o;
   };
   plan->layers.resize(L);
+  int attn_launches = 0;
   for (int l = 0; l < L; ++l) {
     LayerPlan& lp = plan->layers[l];
     HostLayer& H = hl[l];
@@ -809,12 +882,15 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const KvVie
     lp.tiles = H.tiles;
     lp.pool_tiles = H.pool_tiles;
     lp.off_pool = take(std::max<size_t>(1, H.pool_units.size()) * sizeof(Piece));
-    lp.keys_ctas = 0;
-    for (size_t c = 0; c + 1 < H.cta.size(); ++c) lp.keys_ctas += H.cta[c + 1] > H.cta[c] ? 1 : 0;
+    lp.keys_ctas = H.keys_ctas;
+    lp.attn = H.attn;
+    lp.nlayers = H.nlayers;
+    lp.launch = attn_launches;
+    if (H.attn) ++attn_launches;
     // the first piece of each CTA, when it is a dense piece of a contiguous
     // cache (the only kind the kernel can start from the parameters)
     lp.first.clear();
-    if (use_pool && !plan->paged) {
+    if (use_pool && !plan->paged && H.attn) {
       const int nf = std::min(H.grid, kFirstPieces);
       lp.first.resize(nf);
       for (int c = 0; c < nf; ++c) {
@@ -838,7 +914,10 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const KvVie
   plan->off_fill_dst = take(std::max<size_t>(1, fill_dst.size()) * sizeof(void*));
   plan->off_n = take(static_cast<size_t>(B) * sizeof(int64_t));
   // the last layer's combine runs in a launch of its own, whose CTAs have no pieces
-  plan->combine_grid = std::max(1, std::min(ctx->sms, plan->layers[L - 1].ncombine));
+  int last_attn = 0;  // the first layer of the last attention launch
+  for (int l = 0; l < L; ++l)
+    if (plan->layers[l].attn) last_attn = l;
+  plan->combine_grid = std::max(1, std::min(ctx->sms, plan->layers[last_attn].ncombine));
   plan->off_empty_cta = take((plan->combine_grid + 1) * sizeof(int32_t));
   std::vector<unsigned char> host(bytes, 0);
   for (int l = 0; l < L; ++l) {
@@ -917,8 +996,8 @@ void set_prev_combine(lyc_ctx* ctx, Plan* plan, int pl, AttnParams* ap) {
   ap->prev_segs = reinterpret_cast<const Segment*>(plan->dev + pp.off_segs);
   ap->prev_tasks = reinterpret_cast<const int2*>(plan->dev + pp.off_combine);
   ap->prev_ntasks = pp.ncombine;
-  ap->prev_part_o = ctx->part_o + (pl & 1) * ctx->max_parts * D;
-  ap->prev_part_ml = ctx->part_ml + (pl & 1) * ctx->max_parts;
+  ap->prev_part_o = ctx->part_o + (pp.launch & 1) * ctx->max_parts * D;
+  ap->prev_part_ml = ctx->part_ml + (pp.launch & 1) * ctx->max_parts;
   ap->prev_out = plan->out + static_cast<size_t>(pl) * cfg.batch * cfg.num_q_heads * D;
 }
 
@@ -959,46 +1038,50 @@ lyc_status enqueue_step(lyc_ctx* ctx, Plan* plan, cudaStream_t stream, int set, 
   // the stagger.  (Measured on B200 with the selection started on the key
   // flag: per-head selection unchanged, KV-group selection +1.3 % against
   // letting it launch only once the selection has its keys.)
-  auto early_trigger = [&](int l) {
-    if (!early || l + 1 >= L) return false;
-    return plan->layers[l + 1].tiles > 0;
-  };
-  // step counters of layer l's attention launch (parity-0 addresses)
+  // step counters of the attention launch whose first layer is l (parity-0
+  // addresses), and of layer l's selection keys
   const int cstride = 3 * (L + 1);
   uint32_t* cnt_base = reinterpret_cast<uint32_t*>(ctx->pool_cursors);
   auto done_cnt = [&](int l) { return cnt_base + (L + 1) + l; };
   auto keys_cnt = [&](int l) { return cnt_base + 2 * (L + 1) + l; };
   const uint32_t nc = static_cast<uint32_t>(attn_mma_consumer_warps(D));
-  for (int l = 0; l < L; ++l) {
-    const LayerPlan& lp = plan->layers[l];
+  int prev_l0 = -1;  // the first layer of the previous attention launch
+  for (int l0 = 0; l0 < L; ++l0) {
+    const LayerPlan& lp = plan->layers[l0];
+    if (!lp.attn) continue;  // a later layer of a launch: enqueued with the launch
+    const int l1 = l0 + lp.nlayers;  // the launch's layers [l0, l1)
+    bool any_tasks = false;
+    for (int li = l0; li < l1; ++li) any_tasks = any_tasks || plan->layers[li].ntasks > 0;
     AttnParams ap{};
     ap.segs = reinterpret_cast<const Segment*>(plan->dev + lp.off_segs);
     ap.pieces = reinterpret_cast<const Piece*>(plan->dev + lp.off_pieces);
     ap.cta_begin = reinterpret_cast<const int32_t*>(plan->dev + lp.off_cta);
-    ap.q = static_cast<const char*>(plan->q) + static_cast<size_t>(l) * B * Hq * D * es;
-    ap.out = plan->out + static_cast<size_t>(l) * B * Hq * D;
+    ap.q = static_cast<const char*>(plan->q) + static_cast<size_t>(l0) * B * Hq * D * es;
+    ap.out = plan->out + static_cast<size_t>(l0) * B * Hq * D;
     ap.keys = ctx->keys;
-    ap.part_o = ctx->part_o + (l & 1) * ctx->max_parts * D;
-    ap.part_ml = ctx->part_ml + (l & 1) * ctx->max_parts;
+    // partial records: double-buffered by launch (the next launch merges them)
+    ap.part_o = ctx->part_o + (lp.launch & 1) * ctx->max_parts * D;
+    ap.part_ml = ctx->part_ml + (lp.launch & 1) * ctx->max_parts;
     ap.wpart_o = ctx->wpart_o;
     ap.wpart_ml = ctx->wpart_ml;
     ap.wpart_by_sm = 1;
     ap.wpart_slots = ctx->wpart_slots;
     ap.epoch = ctx->epoch;
     if (early) {
-      // done flags between consecutive attention launches, and the pool of
+      // done counters between consecutive attention launches, and the pool of
       // gathered rows (mma kernel only)
-      ap.done = done_cnt(l);
-      ap.prev_done = l > 0 ? done_cnt(l - 1) : nullptr;
-      ap.prev_done_expect = l > 0 ? static_cast<uint32_t>(plan->layers[l - 1].grid) : 0u;
+      ap.done = done_cnt(l0);
+      ap.prev_done = prev_l0 >= 0 ? done_cnt(prev_l0) : nullptr;
+      ap.prev_done_expect = prev_l0 >= 0 ? static_cast<uint32_t>(plan->layers[prev_l0].grid) : 0u;
       ap.pool_units = reinterpret_cast<const Piece*>(plan->dev + lp.off_pool);
       ap.pool_n = lp.pool_n;
       ap.pool_stride = cstride;
       ap.pool_cursors = ctx->pool_cursors;
-      // the selection of this layer starts once the keys are written (the
-      // dense runs), not once the whole launch is done
-      if (lp.ntasks > 0 && lp.keys_ctas > 0) {
-        ap.keys_done = keys_cnt(l);
+      // each layer's selection starts once that layer's keys are written (its
+      // dense runs), not once the whole launch is done: the consumer warps
+      // count their arrivals per layer, from the first layer's counter on
+      if (any_tasks) {
+        ap.keys_done = keys_cnt(l0);
         ap.keys_ctas = lp.keys_ctas;
       }
     }
@@ -1006,7 +1089,7 @@ lyc_status enqueue_step(lyc_ctx* ctx, Plan* plan, cudaStream_t stream, int set, 
     ap.status = ctx->status;
     ap.timeline = plan->timeline;
     ap.timeline_cap = plan->timeline_cap;
-    ap.layer = l;
+    ap.layer = l0;
     ap.Hq = Hq;
     ap.G = ctx->G;
     ap.n = plan->n;
@@ -1015,9 +1098,10 @@ lyc_status enqueue_step(lyc_ctx* ctx, Plan* plan, cudaStream_t stream, int set, 
     // Without a selection launch in between, the previous layer's attention
     // may still be running.  The mma kernel needs no wait for it: its
     // readers of sets wait on the sets' ready flags, its partials are written
-    // only after its epilogue's griddepcontrol.wait, and its piece-state ring
-    // is the SM's own.  The other kernels wait for it at their start.
-    ap.wait_prev = (l > 0 && plan->layers[l - 1].ntasks == 0 && !early) ? 1 : 0;
+    // only after its epilogue has seen the previous launch complete, and its
+    // piece-state ring is the SM's own.  The other kernels wait for it at
+    // their start.
+    ap.wait_prev = (l0 > 0 && plan->layers[l0 - 1].ntasks == 0 && !early) ? 1 : 0;
     lyc_status st = record_event(ctx, plan, set, ev++, stream, capturing);
     if (st != LYC_OK) return st;
     if (dtype == 0) {
@@ -1030,7 +1114,7 @@ lyc_status enqueue_step(lyc_ctx* ctx, Plan* plan, cudaStream_t stream, int set, 
       mp.p = ap;
       mp.p.gather_rows = plan->gather_rows;
       mp.p.paged = plan->paged ? 1 : 0;
-      if (l > 0) set_prev_combine(ctx, plan, l - 1, &mp.p);
+      if (prev_l0 >= 0) set_prev_combine(ctx, plan, prev_l0, &mp.p);
       if (!plan->use_tc && !lp.first.empty()) {
         mp.nfirst = static_cast<int32_t>(lp.first.size());
         memcpy(mp.first, lp.first.data(), lp.first.size() * sizeof(FirstPiece));
@@ -1043,13 +1127,23 @@ lyc_status enqueue_step(lyc_ctx* ctx, Plan* plan, cudaStream_t stream, int set, 
     }
     if ((st = record_event(ctx, plan, set, ev++, stream, capturing)) != LYC_OK) return st;
     plan->kernel_kind.push_back(0);
-    plan->kernel_layer.push_back(l);
-    if (lp.ntasks > 0) {
+    plan->kernel_layer.push_back(l0);
+    // the launch's selections, one launch per layer, in layer order.  Each
+    // lets the next kernel of the step launch at its own start (the next
+    // selection, or the next attention launch, whose CTAs then take the SMs
+    // of this launch's tail as they free up; its pool of gathered rows absorbs
+    // their staggered start).  (Measured on B200 with the selection started
+    // on its keys: per-head selection unchanged, KV-group selection +1.3 %
+    // against letting the next attention launch only once the selection has
+    // its keys.)
+    for (int li = l0; li < l1; ++li) {
+      const LayerPlan& sp = plan->layers[li];
+      if (sp.ntasks == 0) continue;
       TopkParams tp{};
-      tp.tasks = reinterpret_cast<const TopkTask*>(plan->dev + lp.off_tasks);
+      tp.tasks = reinterpret_cast<const TopkTask*>(plan->dev + sp.off_tasks);
       tp.epoch = ctx->epoch;
-      tp.early = early_trigger(l) ? 1 : 0;
-      tp.n = lp.topk_n;
+      tp.early = (early && li + 1 < L) ? 1 : 0;
+      tp.n = sp.topk_n;
       tp.k = plan->k;
       tp.size_rule = plan->sel.rule == LYC_RULE_TOPP        ? kSizeTopP
                      : plan->sel.rule == LYC_RULE_THRESHOLD ? kSizeThreshold
@@ -1058,24 +1152,27 @@ lyc_status enqueue_step(lyc_ctx* ctx, Plan* plan, cudaStream_t stream, int set, 
       tp.expand = plan->sel.rule == LYC_RULE_BLOCK_TOPK ? plan->sel.block : 1;
       tp.timeline = plan->timeline;
       tp.timeline_cap = plan->timeline_cap;
-      tp.layer = l;
+      tp.layer = li;
       tp.status = ctx->status;
-      if (ap.keys_done) {
-        tp.keys_ready = ap.keys_done;
-        tp.keys_expect = static_cast<uint32_t>(lp.keys_ctas) * nc;
+      if (ap.keys_done && sp.keys_ctas > 0) {
+        // its keys, and the previous attention launch done (it may still read
+        // the set buffers this selection overwrites)
+        tp.keys_ready = keys_cnt(li);
+        tp.keys_expect = static_cast<uint32_t>(sp.keys_ctas) * nc;
         tp.prev_done = ap.prev_done;
         tp.prev_done_expect = ap.prev_done_expect;
         tp.cnt_stride = cstride;
       }
       if ((st = record_event(ctx, plan, set, ev++, stream, capturing)) != LYC_OK) return st;
-      LYC_CUDA(topk_launch(lp.topk_cl, &tp, lp.ntasks, stream, false), "top-k launch");
+      LYC_CUDA(topk_launch(sp.topk_cl, &tp, sp.ntasks, stream, false), "top-k launch");
       if ((st = record_event(ctx, plan, set, ev++, stream, capturing)) != LYC_OK) return st;
       plan->kernel_kind.push_back(1);
-      plan->kernel_layer.push_back(l);
+      plan->kernel_layer.push_back(li);
     }
+    prev_l0 = l0;
   }
   if (dtype == 0) {
-    // the last layer's cross-piece combine: the same kernel with no pieces
+    // the last launch's cross-piece combine: the same kernel with no pieces
     AttnMmaParams mp;
     memset(&mp, 0, sizeof mp);
     mp.tmk = plan->tmk;
@@ -1084,7 +1181,7 @@ lyc_status enqueue_step(lyc_ctx* ctx, Plan* plan, cudaStream_t stream, int set, 
     mp.tgv = plan->tgv;
     AttnParams& ap = mp.p;
     ap = AttnParams{};
-    const LayerPlan& lp = plan->layers[L - 1];
+    const LayerPlan& lp = plan->layers[prev_l0];
     ap.segs = reinterpret_cast<const Segment*>(plan->dev + lp.off_segs);
     ap.pieces = reinterpret_cast<const Piece*>(plan->dev + lp.off_pieces);
     ap.cta_begin = reinterpret_cast<const int32_t*>(plan->dev + plan->off_empty_cta);
@@ -1097,7 +1194,7 @@ lyc_status enqueue_step(lyc_ctx* ctx, Plan* plan, cudaStream_t stream, int set, 
     ap.wpart_slots = ctx->wpart_slots;
     ap.epoch = ctx->epoch;
     if (early) {
-      ap.prev_done = done_cnt(L - 1);
+      ap.prev_done = done_cnt(prev_l0);
       ap.prev_done_expect = static_cast<uint32_t>(lp.grid);
       ap.pool_stride = cstride;
     }
@@ -1105,7 +1202,7 @@ lyc_status enqueue_step(lyc_ctx* ctx, Plan* plan, cudaStream_t stream, int set, 
     ap.Hq = Hq;
     ap.G = ctx->G;
     ap.n = plan->n;
-    set_prev_combine(ctx, plan, L - 1, &ap);
+    set_prev_combine(ctx, plan, prev_l0, &ap);
     lyc_status st = record_event(ctx, plan, set, ev++, stream, capturing);
     if (st != LYC_OK) return st;
     LYC_CUDA(plan->use_tc ? attn_tc_dispatch(&mp, plan->combine_grid, stream, nullptr, false)
@@ -1341,7 +1438,7 @@ lyc_status lyc_create(const lyc_config* cfg, lyc_ctx** out) {
   // most of the smaller unit size)
   const size_t unit_rows = static_cast<size_t>(std::min(kPoolTiles, kPoolTilesDep)) * kTileRows;
   const size_t units = (static_cast<size_t>(c.max_k) + unit_rows - 1) / unit_rows;
-  ctx->max_parts = (2 * static_cast<size_t>(ctx->sms) + nseg_max + nseg_max * units) * kMaxQ;
+  ctx->max_parts = (2 * static_cast<size_t>(ctx->sms) + nseg_max + nseg_max * units) * kMaxQ * kLayersPerLaunch;
   ctx->max_counters = nseg_max * kMaxQ;
   auto alloc = [&](void** p, size_t bytes) -> lyc_status {
     if (cudaMalloc(p, bytes) != cudaSuccess) {

@@ -116,14 +116,14 @@ def test_traffic_record_from_capture(tmp_path, monkeypatch, capsys):
     csvf = tmp_path / "t.csv"
     csvf.write_text("==PROF== noise\n" + head + "".join(rows))
     monkeypatch.setattr(bench, "attn_source_hash", lambda: "feed")
-    assert bench.main(["--traffic-from", str(csvf), "--layers", "2"]) == 0
+    assert bench.main(["--traffic-from", str(csvf), "--layers", "2", "--launches-per-step", "3"]) == 0
     line = capsys.readouterr().out.strip()
     assert line.startswith("traffic-record: ")
     rec = json.loads(line.split(":", 1)[1])
     assert rec["source_sha"] == "feed" and rec["launches"] == 3
     assert rec["workload"] == "llama3-8b-attn-stack-n131072-k4096-L2-r2"
     assert rec["bytes_per_launch"] == round((300e6 + 4e6 + 1024) / 2)
-    assert bench.main(["--traffic-from", str(csvf), "--layers", "3"]) == 2
+    assert bench.main(["--traffic-from", str(csvf), "--layers", "3", "--launches-per-step", "4"]) == 2
 
 
 def test_reference_arm_times_whole_steps_on_the_library_arms_config(capsys):

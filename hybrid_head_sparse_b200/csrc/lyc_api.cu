@@ -60,10 +60,16 @@ constexpr int kPlanCacheSize = 16;
 // the attention launch of the layer before it has completed, so the buffer it
 // overwrites must hold a set written three refreshes ago: three buffers.
 // Layers per attention launch (mma kernel): each launch runs the dense rows
-// and gathered rows of this many consecutive layers, so that a CTA's fixed
-// cost (its start, the wait for its first tiles, its drain) is paid once per
-// that many layers; the selections stay one launch per layer.
-constexpr int kLayersPerLaunch = 2;
+// and gathered rows of several consecutive layers, so that a CTA's fixed
+// cost (its start, the wait for its first tiles, its drain: ~7 us, about
+// what the step streams in 45 MB) is paid once per that many layers; the
+// selections stay one launch per layer.  Two layers per launch for layers
+// that read at least kSmallLayerBytes, four below (measured on B200: 128K
+// Llama3-8B shapes, ~151 MB per later layer: 1047 steps/s with two layers
+// per launch, 1026 with three, 1037 with four, ~1001 with one; 32K, ~50 MB
+// per layer: 2081, 2149, 2182 and ~1750).
+constexpr int kLayersPerLaunch = 4;  // at most
+constexpr double kSmallLayerBytes = 96e6;
 // Buffers per set slot.  A selection overwrites the set that its slot held
 // kSetBuffers refreshes earlier.  That set's last readers run in the launch
 // of the layer that last read it, or, for a deferred pass, of the layer
@@ -508,6 +514,34 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const KvVie
   // and outputs are those of layer l (Segment::q, Segment::out).  The last
   // layer keeps its own.
   const bool defer_dep = use_pool;
+  // The attention launches (mma kernel): kLayersPerLaunch consecutive layers
+  // each, the last layer alone (it keeps its passes over the sets of the
+  // selection just before it, which is enqueued before its launch).
+  // launch_first[l]: the first layer of l's launch; next_launch[l]: the first
+  // layer of the launch after it (L: none).
+  std::vector<int> launch_first(L), next_launch(L);
+  {
+    // the K/V bytes a later layer reads, on average (its dense groups' rows,
+    // and k rows per sparse-only group)
+    double layer_bytes = 0.0;
+    for (int l = 1; l < L; ++l)
+      for (int g = 0; g < Hkv; ++g) {
+        bool dense = false;
+        for (int h = g * G; h < (g + 1) * G; ++h) dense = dense || role[static_cast<int64_t>(l) * Hq + h] != 0;
+        for (int b = 0; b < B; ++b)
+          layer_bytes += static_cast<double>(dense ? kv.n[b] : std::min<int64_t>(k, kv.n[b]));
+      }
+    layer_bytes *= static_cast<double>(cfg.head_dim) * es * 2.0 / std::max(1, L - 1);
+    const int LG = !use_pool ? 1 : layer_bytes < kSmallLayerBytes ? kLayersPerLaunch : 2;
+    for (int l0 = 0, l1 = 0; l0 < L; l0 = l1) {
+      l1 = std::min(L, l0 + LG);
+      if (l1 == L && l1 - l0 > 1) l1 = L - 1;
+      for (int l = l0; l < l1; ++l) {
+        launch_first[l] = l0;
+        next_launch[l] = l1;
+      }
+    }
+  }
 
   // the set trace [L][B][Hs][k]: row (l, b, s) holds the set slot s passes on
   // after layer l.  A refreshed slot's row is written by its selection; the
@@ -539,8 +573,14 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const KvVie
     // a sparse pass of this layer: into this launch, or (a set the previous
     // layer's selection writes) into the next one, where it needs no wait
     // order (dep 0: its selection has long completed)
-    auto push_sparse = [&](Segment ss, int layer) {
-      if (defer_dep && layer + 1 < L && ss.dep && ss.ready) {
+    // w: the layer whose selection wrote the set (-1: the caller's)
+    auto push_sparse = [&](Segment ss, int layer, int w) {
+      if (defer_dep && w >= 0 && launch_first[w] == launch_first[layer] && next_launch[layer] < L) {
+        // a set of a selection of this pass's own launch: that selection is
+        // enqueued after the launch, so the pass goes to the next launch
+        ss.dep = 0;
+        hl[next_launch[layer]].deferred.push_back(ss);
+      } else if (defer_dep && layer + 1 < L && ss.dep && ss.ready) {
         ss.dep = 0;
         hl[layer + 1].deferred.push_back(ss);
       } else {
@@ -616,7 +656,7 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const KvVie
             ss.dep = prev_fresh[g];
             ss.ready = ready_flag(g, b);
             maxnq = std::max(maxnq, js);
-            push_sparse(ss, l);
+            push_sparse(ss, l, writer[g]);
           }
         } else {
           for (int h = g * G; h < (g + 1) * G; ++h) {
@@ -631,7 +671,7 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const KvVie
             ss.nq = ss.nout = 1;
             ss.dep = prev_fresh[h];
             ss.ready = ready_flag(h, b);
-            push_sparse(ss, l);
+            push_sparse(ss, l, writer[h]);
           }
         }
       }
@@ -687,19 +727,15 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const KvVie
   // ---- phase B: the attention launches.  With the mma kernel a launch runs
   // kLayersPerLaunch consecutive layers: their segments are concatenated in
   // layer order (each layer's own passes, then the passes deferred into it).
-  // No pass of a launch may wait for a selection enqueued after that launch
-  // (the selection could find no free SM while the launch's CTAs wait): with
-  // two layers per launch, a pass of the second layer over a set of the
-  // first layer's selection is deferred to the next launch, and the last
-  // layer, which keeps such passes, gets a launch of its own.
-  static_assert(kLayersPerLaunch >= 1 && kLayersPerLaunch <= 2,
-                "more layers per launch need passes over their own selections deferred");
+  // No pass of a launch waits for a selection enqueued after that launch
+  // (the selection could find no free SM while the launch's CTAs wait): a
+  // pass over a set of a selection of its own launch goes to the next launch
+  // (see push_sparse), and the last layer, which keeps its passes over the
+  // sets of the selection just before it, has a launch of its own.
   {
-    const int LG = use_pool ? kLayersPerLaunch : 1;
     int prev_l0 = -1;
     for (int l0 = 0, l1 = 0; l0 < L; l0 = l1) {
-      l1 = std::min(L, l0 + LG);  // the launch's layers [l0, l1)
-      if (l1 == L && l1 - l0 > 1) l1 = L - 1;  // the last layer alone
+      l1 = next_launch[l0];  // the launch's layers [l0, l1)
       HostLayer& H = hl[l0];
       std::vector<size_t> seg_begin(1, 0);
       seg_begin.push_back(H.segs.size());

@@ -535,14 +535,15 @@ def run_lyc(args):
     ctx.set_timing(False)
     iso_attn_ms = sum(t[2] for t in ktimes if t[0] == 0) / args.steps
     iso_topk_ms = sum(t[2] for t in ktimes if t[0] == 1) / args.steps
-    # launches per step: attention launches (one per layer and a merge
-    # launch, or layer 0 and one persistent launch) and selection launches
+    # launches per step: attention launches (each of two or four layers, the
+    # last layer's own, and a merge launch) and selection launches (one per
+    # layer)
     attn_launches, topk_launches, other_launches = ctx.step_launches()
 
     roofline = {
         "bound": "hbm",
         "kernel": ("attn_tc_layer_kernel" if args.attn_kernel == "tcgen05" else "attn_mma_layer_kernel")
-                  + " (pooled dense + sparse attention, one launch per layer)",
+                  + " (pooled dense + sparse attention of two or four layers per launch)",
         "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
         "frac": round(achieved / peak, 4),
         "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs), burst figure",
@@ -554,8 +555,9 @@ def run_lyc(args):
         "note": ("achieved = K+V bytes the attention kernel must read per step (dense groups: n "
                  "rows; each sparse pass: k rows) / its time per step; its time per step = the "
                  "union of its CTAs' busy intervals on the device timeline (same K replays), as "
-                 "a share of the span, times the timed ms_per_step.  Launches of consecutive "
-                 "layers overlap, so the per-launch figure is that time / L"),
+                 "a share of the span, times the timed ms_per_step.  Launches overlap and each "
+                 "runs several layers, so bytes and time 'per launch' are both per layer "
+                 "(divided by L), like the traffic record"),
         "isolated_launches": ({
             "attn_ms_per_step": iso_attn_ms, "topk_ms_per_step": iso_topk_ms,
             "attn_gbs": round(distinct / (iso_attn_ms / 1e3) / 1e9, 1),

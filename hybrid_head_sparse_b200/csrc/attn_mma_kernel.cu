@@ -805,7 +805,7 @@ __device__ __forceinline__ void mma_consumers(const AttnMmaParams& P, unsigned c
     if (solo) {
       // ---- this warp holds the whole piece: its partial state, or the
       // normalised outputs when the segment is this one piece.  Partial
-      // states share their buffer with the layer two launches back, whose
+      // states share their buffer with the launch two launches back, whose
       // merge runs in the previous launch: write them once that launch has
       // completed (seen by the epilogue warp).
       if (sg.npieces > 1 && !prev_ok) {
@@ -850,13 +850,13 @@ __device__ __forceinline__ void mma_consumers(const AttnMmaParams& P, unsigned c
 
 // ---------------------------------------------------------------- epilogue warp
 // Two jobs (Appendix C, Algorithm 2, steps 5-6):
-//  1. first, the cross-piece combine of the previous layer: this CTA takes
-//     the (segment, output) tasks t = blockIdx.x, blockIdx.x + gridDim.x, ...
-//     and folds each output's piece partials (log-sum-exp) into that layer's
-//     output, once the previous layer's attention launch has raised its done
-//     flag (its partials are then in place; this launch may start while that
-//     one still runs); running the combine here keeps it off the critical
-//     path;
+//  1. first, the cross-piece combine of the previous attention launch: this
+//     CTA takes the (segment, output) tasks t = blockIdx.x, blockIdx.x +
+//     gridDim.x, ... and folds each output's piece partials (log-sum-exp)
+//     into the output of the segment's layer, once that launch's done counter
+//     is complete (its partials are then in place; this launch may start
+//     while that one still runs); running the combine here keeps it off the
+//     critical path;
 //  2. then, per piece of this CTA in order: wait for the NC consumer warps'
 //     states, merge them per output, and write the piece's partial (or, for a
 //     segment of one piece, the output itself).
@@ -915,10 +915,10 @@ __device__ __forceinline__ void mma_epilogue(const AttnMmaParams& P, unsigned ch
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_FLAGS);
   const int wq = p.wpart_q > 0 ? p.wpart_q : kMaxQ;  // query rows per ring record
 
-  // ---- 1. the previous layer's cross-piece combine, after that launch has
+  // ---- 1. the previous launch's cross-piece combine, after that launch has
   // completed.  The wait also comes before any partial of this launch is
   // written: this launch may start while the previous attention launch still
-  // runs, and that launch reads the partials of the layer before it, which
+  // runs, and that launch reads the partials of the launch before it, which
   // share this launch's buffer.  With a flag for it, wait on the flag (the
   // selection in between may still run); else on griddepcontrol.wait, which
   // returns once every earlier launch of the chain has completed.
@@ -956,7 +956,7 @@ __device__ __forceinline__ void mma_epilogue(const AttnMmaParams& P, unsigned ch
     lse_finish(acc, sg.out ? sg.out : p.prev_out, p, sg, o, lane, col, D);
   }
 
-  // ---- 2. this layer's pieces of more than one tile (a one-tile piece's
+  // ---- 2. this launch's pieces of more than one tile (a one-tile piece's
   // warp writes its result itself).  Tile j of a piece whose first tile is
   // the CTA's tile t0 went to consumer warp (t0 + j) % NC, which took tiles
   // j, j + NC, ... of the piece in order; merging the warps' states in the

@@ -52,13 +52,6 @@ namespace {
 
 constexpr int kMaxCtxLimit = 655360;  // 16-CTA top-k keeps every key in shared memory
 constexpr int kPlanCacheSize = 16;
-// Buffers per set slot.  A refresh writes the slot's next buffer in turn.
-// A set is read by the layers up to the slot's next refresh, and the first of
-// them may read it one attention launch late (the mma kernel runs a layer's
-// sparse passes over the sets that the selection just before that layer
-// wrote in the next layer's launch).  A selection starts writing only once
-// the attention launch of the layer before it has completed, so the buffer it
-// overwrites must hold a set written three refreshes ago: three buffers.
 // Layers per attention launch (mma kernel): each launch runs the dense rows
 // and gathered rows of several consecutive layers, so that a CTA's fixed
 // cost (its start, the wait for its first tiles, its drain: ~7 us, about
@@ -489,8 +482,8 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const KvVie
     int topk_cl = 16;           // cluster size of this layer's selection launch
     std::vector<Piece> pool_units;   // mma kernel: the pool's units, in order
     int64_t tiles = 0, pool_tiles = 0;
-    // mma kernel: the previous layer's sparse passes over the sets that the
-    // selection before it wrote, run by this launch (see below)
+    // mma kernel: sparse passes of earlier layers deferred to this layer's
+    // rows (see push_sparse below)
     std::vector<Segment> deferred;
     int keys_ctas = 0;        // CTAs with dense pieces of this layer
     bool attn = true;         // this layer's record holds an attention launch
@@ -676,7 +669,7 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const KvVie
         }
       }
     }
-    // the previous layer's deferred sparse passes, after this layer's own
+    // the sparse passes deferred to this layer, after its own
     for (const Segment& ds : H.deferred) {
       H.segs.push_back(ds);
       maxnq = std::max(maxnq, ds.nq);

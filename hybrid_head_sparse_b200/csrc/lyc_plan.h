@@ -37,8 +37,9 @@ constexpr int kPartSlots = 4;
 // time; a CTA's leader publishes the pool pieces it took into a ring of
 // kPoolRing entries that every warp of the CTA reads in order.
 constexpr int kPoolTiles = 8;
-// Units of the sets that the previous layer's selection writes (the only
-// gathered rows that wait for a selection; taken last).  Smaller units would
+// Units of the sets that the selection just before a pass's layer writes
+// (passes deferred to the end of a later pool, or the last layer's own:
+// the only gathered rows that may wait for a selection; taken last).  Smaller units would
 // spread them over more CTAs once that selection is done, but every unit is a
 // piece with its own partial state (measured on B200, 128K Llama3-8B stack,
 // against 8-tile units for both: KV-group sets, 4-tile units -1.2 %, 2-tile
@@ -79,15 +80,15 @@ struct Segment {
                           // at k + page * s_page + (i % page_rows) * s_token); NULL: contiguous
   int64_t s_page;         // paged cache: element stride between pages
   // the segment's layer: its queries [B][Hq][d] and outputs [B][Hq][d] (a
-  // launch of the mma kernel may hold segments of two layers: its own, and
-  // the previous layer's sparse passes over the sets that the selection just
-  // before that layer wrote); NULL: the launch's q and out
+  // launch of the mma kernel holds segments of several layers: its own
+  // layers', and sparse passes deferred to it from earlier layers); NULL:
+  // the launch's q and out
   const void* q;
   float* out;
 };
 
 struct Piece {
-  int32_t seg;      // segment index within the layer
+  int32_t seg;      // segment index within the launch
   int32_t r0, r1;   // row range within the segment (token or list positions)
   int32_t ordinal;  // which piece of its segment (partials at part_base + ordinal*nout + o)
 };
@@ -96,22 +97,22 @@ struct AttnParams {
   const Segment* segs;
   const Piece* pieces;
   const int32_t* cta_begin;  // pieces of CTA c: [cta_begin[c], cta_begin[c+1])
-  const void* q;             // this layer's queries, [B][Hq][d]
-  float* out;                // this layer's outputs, [B][Hq][d]
+  const void* q;             // the launch's first layer's queries, [B][Hq][d] (segments carry their own)
+  float* out;                // the launch's first layer's outputs, [B][Hq][d] (likewise)
   float* keys;               // selection-key buffer
   float* part_o;             // [parts][d]
   float2* part_ml;           // [parts] (running max in log2 units, sum)
   int32_t* counters;         // arrival counters, left at zero after use
   float* wpart_o;            // per CTA: [kPartSlots][consumer warp][kMaxQ][d] piece states
   float2* wpart_ml;          // per CTA: [kPartSlots][consumer warp][kMaxQ] (max, sum)
-  // bf16 path: the cross-piece combine of a layer runs in the next launch
-  // (the previous layer's outputs, taken by this launch's epilogue warps)
-  const Segment* prev_segs;  // previous layer's segments
+  // bf16 path: the cross-piece combine of a launch runs in the next launch
+  // (taken by that launch's epilogue warps)
+  const Segment* prev_segs;  // the previous attention launch's segments
   const int2* prev_tasks;    // (segment, output) pairs of segments cut into > 1 piece
   int32_t prev_ntasks;
-  const float* prev_part_o;  // previous layer's piece partials
+  const float* prev_part_o;  // the previous launch's piece partials
   const float2* prev_part_ml;
-  float* prev_out;           // previous layer's outputs, [B][Hq][d]
+  float* prev_out;           // outputs of the previous launch's first layer (segments carry their own)
   int32_t wait_prev;         // 1: wait for the previous launch to complete before any
                              // work (it is not a selection launch, which would have)
   uint32_t* status;          // device status word
@@ -121,7 +122,7 @@ struct AttnParams {
   // counter of this step is at ptr + (epoch & 1) * pool_stride.
   uint32_t* done;            // NULL, or this launch's completion counter: every CTA adds 1
                              // once its work is done (release)
-  const uint32_t* prev_done; // NULL, or the previous layer's attention launch's completion
+  const uint32_t* prev_done; // NULL, or the previous attention launch's completion
                              // counter: the epilogue waits until it reaches prev_done_expect
                              // (else on griddepcontrol.wait)
   uint32_t prev_done_expect; // CTAs of that launch
@@ -140,11 +141,12 @@ struct AttnParams {
   int32_t wpart_q;           // query rows per consumer-warp record of the ring (0: kMaxQ); a
                              // caller whose segments all have one query row passes 1
   int32_t timeline_cap;
-  uint32_t* keys_done;       // NULL, or the step counter of this launch's selection keys:
-                             // each consumer warp of the keys_ctas CTAs with pieces of their
-                             // own adds 1 once those (dense) pieces are done (release)
-  int32_t keys_ctas;
-  int32_t layer;
+  uint32_t* keys_done;       // NULL, or the step counter of the selection keys of the launch's
+                             // first layer; the counters of its later layers follow it.  Each
+                             // consumer warp of a CTA with own (dense) pieces of a layer adds 1
+                             // to that layer's counter once it is past them (release)
+  int32_t keys_ctas;         // CTAs with own pieces of the first layer
+  int32_t layer;             // the launch's first layer
   int32_t Hq, G, n;
   int32_t paged;             // 1: the segments' rows are in pages (Segment::bt)
   int32_t gather_rows;       // rows of the flattened row-gather maps (an index past
@@ -211,11 +213,13 @@ struct TopkParams {
                           // (its readers wait on the ready flags); 0: only after
   unsigned long long* timeline;  // as in AttnParams
   const uint32_t* keys_ready;  // NULL: start on griddepcontrol.wait (the attention launch
-                               // before has completed); else once this step counter
-                               // (AttnParams::keys_done) reaches keys_expect
+                               // before has completed); else once this step counter (the
+                               // layer's key counter, see AttnParams::keys_done) reaches
+                               // keys_expect
   const uint32_t* prev_done;   // with keys_ready: the completion counter of the attention
-                               // launch of the layer before (its readers of the set buffers
-                               // this launch writes) to wait for, up to prev_done_expect; or NULL
+                               // launch before the one of this layer (the last readers of the
+                               // set buffers this launch writes) to wait for, up to
+                               // prev_done_expect; or NULL
   uint32_t keys_expect, prev_done_expect;
   int32_t cnt_stride;          // step counters per epoch parity
   uint32_t* status;            // device status word (wait timeouts)

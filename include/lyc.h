@@ -294,9 +294,11 @@ lyc_status lyc_step_bytes(const lyc_config* cfg, const uint8_t* role_mask, int64
                           int s_in, uint64_t* analytic, uint64_t* distinct);
 
 /* Kernel launches of the most recent step enqueued on this context: its
- * attention launches (one per layer and the launch that merges the last
- * layer's split rows), selection launches, and the rest (the final set copy,
- * trace fill, K/V append, S^(0) check).
+ * attention launches (bf16: each of two or four consecutive layers, the last
+ * layer alone, and the launch that merges the last layer's split rows; fp32
+ * and the tcgen05 kernel: one per layer and the merge launch), selection
+ * launches (one per layer with retrieval heads), and the rest (the final set
+ * copy, trace fill, K/V append, S^(0) check).
  * Errors: INVALID_ARG (NULL, or no step yet). */
 lyc_status lyc_step_launches(const lyc_ctx* ctx, int* attention, int* selection, int* other);
 
@@ -340,7 +342,7 @@ lyc_status lyc_kernel_times(lyc_ctx* ctx, lyc_kernel_time* times, int cap, int* 
  * 1 + 3*cap unsigned 64-bit words; the caller zeroes word 0.  Every CTA of the
  * attention and selection kernels appends (start ns, end ns, tag) read from
  * the GPU's global timer, tag = kind << 32 | layer << 16 | CTA (kind 0 =
- * attention, 1 = selection); word 0 counts the records (records past cap are
+ * attention, with the first layer of its launch; 1 = selection); word 0 counts the records (records past cap are
  * dropped).  NULL turns it off.  Profiling use. */
 lyc_status lyc_set_timeline(lyc_ctx* ctx, unsigned long long* buf, int cap);
 

@@ -1,12 +1,12 @@
-// attn_mma_kernel.cu -- pooled hybrid-head decode attention for one layer,
-// bf16 inputs, tensor cores.
+// attn_mma_kernel.cu -- pooled hybrid-head decode attention of one launch
+// (two or four consecutive layers), bf16 inputs, tensor cores.
 //
-// Computes, for every segment of the layer's work pool (lyc_plan.h):
+// Computes, for every segment of the launch's work pool (lyc_plan.h):
 //   retrieval rows, page "LycheeDecode ..." (paper-graph-ui summary),
 //   section 3.4 Eq. (1): o = softmax(q K^T / sqrt(d)) V over all n cached rows,
 //   sparse rows, section 3.4 Eq. (3): the same over the rows of the set they
 //   inherit,
-// plus the selection key of every cached row for the sets refreshed at this
+// plus the selection key of every cached row for the sets refreshed at its
 // layer (Eq. 2 then runs in topk_kernel.cu).  The pieces of a segment cut
 // over several CTAs are merged with log-sum-exp (Appendix C, Algorithm 2
 // steps 5-6) by the epilogue warps of the next launch, so no CTA waits for
@@ -386,7 +386,7 @@ __device__ __forceinline__ void mma_producers(const AttnMmaParams& P, unsigned c
     Piece pc;
     if (!cta_piece<C>(p, smem, pbeg, pend, pi, lane, &pc, fp)) break;
     if (pi == 0 && fp && fp->pc.seg >= 0) {
-      // a dense piece of this launch's layer: the tile copies need no more
+      // a dense piece of the launch's first layer: the tile copies need no more
       // (the next piece reads its segment's fields)
       dense = true;
       sgg = fp->g;

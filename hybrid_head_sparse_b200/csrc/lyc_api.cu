@@ -403,11 +403,11 @@ int pick_topk_cluster(const lyc_ctx* ctx, int ntasks) {
 
 // ---------------------------------------------------------------- planner
 //
-// Builds every layer's work pool for one (role mask, n, k, flags, pointers)
+// Builds every launch's work pool for one (role mask, n, k, flags, pointers)
 // combination and uploads it in one buffer.  Set buffers: each set slot has
-// two buffers; a refreshed slot is written into the buffer it is not
-// currently read from, so a layer's readers and its own selection never touch
-// the same memory (double buffering), and unrefreshed slots cost no copy.
+// kSetBuffers buffers; a refreshed slot is written into the next one in turn,
+// never one that a pass still in flight may read (see kSetBuffers), and
+// unrefreshed slots cost no copy.
 lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const KvView& kv,
                       int k, uint32_t flags) {
   const lyc_config& cfg = ctx->cfg;
@@ -1459,12 +1459,13 @@ lyc_status lyc_create(const lyc_config* cfg, lyc_ctx** out) {
   ctx->KS = static_cast<int>(round_up(c.max_k, 4));
   const int B = c.batch, Hq = c.num_q_heads, Hkv = c.num_kv_heads, D = c.head_dim, L = c.num_layers;
   const size_t es = c.dtype == LYC_BF16 ? 2 : 4;
-  // segments of one launch: dense and sparse of its layer, plus the previous
-  // layer's deferred sparse passes
+  // segments of one layer: dense and sparse of its own, plus the sparse
+  // passes deferred to it
   const size_t nseg_max = static_cast<size_t>(B) * (Hkv + 2 * Hq);
   // pieces per layer <= 2 * sms + segments (two pooling phases), plus the
   // pool units of the mma kernel (every sparse segment cut into units, at
-  // most of the smaller unit size)
+  // most of the smaller unit size); a launch holds up to kLayersPerLaunch
+  // layers
   const size_t unit_rows = static_cast<size_t>(std::min(kPoolTiles, kPoolTilesDep)) * kTileRows;
   const size_t units = (static_cast<size_t>(c.max_k) + unit_rows - 1) / unit_rows;
   ctx->max_parts = (2 * static_cast<size_t>(ctx->sms) + nseg_max + nseg_max * units) * kMaxQ * kLayersPerLaunch;

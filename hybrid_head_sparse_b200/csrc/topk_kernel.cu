@@ -331,17 +331,17 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster_kernel(const Top
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const unsigned lt = (1u << lane) - 1u;
   // The keys are the attention kernel's output: read only once it has
-  // completed.  The next kernel (the next layer's attention) may start its
-  // launch before that when its readers of this selection's sets wait on the
-  // ready flags (p.early), else only after.
-  // With a key flag, the keys are complete once every consumer warp of the
-  // attention launch that writes them has finished its dense rows (the flag
-  // holds the step's epoch + 1); the rest of that launch (its gathered rows)
-  // may still run.  The sets this launch writes replace sets that the
-  // attention launch of the layer before may still read: wait for that
-  // launch's done flag as well.  Both writers were resident before this
-  // launch began (each launch of the step starts only once every CTA of the
-  // one before it has), so the waits end.
+  // written them.  The next kernel (the next selection, or the next
+  // attention launch) may start its launch before that when its readers of
+  // this selection's sets wait on the ready flags (p.early), else only after.
+  // With a key counter, the keys are complete once every consumer warp of the
+  // attention launch that writes them has finished its dense rows of this
+  // layer (the counter reaches keys_expect); the rest of that launch may
+  // still run.  The sets this launch writes replace sets that the attention
+  // launch before that one may still read: wait for its done counter as
+  // well.  Both writers were resident before this launch began (each launch
+  // of the step starts only once every CTA of the one before it has), so the
+  // waits end.
   if (p.early) pdl_launch_dependents();
   if (p.keys_ready) {
     __shared__ int wait_abort;

@@ -378,20 +378,23 @@ lyc_status encode_gather_map(lyc_ctx* ctx, CUtensorMap* map, const void* base, c
 }
 
 // Cluster size of a selection launch of `ntasks` sets.  A small selection (a
-// few sets) takes clusters of 8 and runs beside the next layer's attention,
-// on SMs that the planner leaves out of that attention's grid: room for two
-// selections, so that the next layer's selection can start on its key flag
-// while this one still runs.  (Measured on B200 at 128K keys, 2 retrieval
-// heads per layer, against clusters of 16 with room for one: +4.2 % with
-// KV-group sets, +1.1 % per head; clusters of 4 with room for two, or of 8
-// with room for three, lose.)  A large selection (layer 0) takes the largest
-// size whose clusters are all resident at once, so that it runs in one wave
-// and the next layer starts right away; else the smallest size.
+// few sets) takes clusters of 4 and runs beside the attention launches, on
+// SMs that the planner leaves out of their grid: room for two selections, so
+// that a layer's selection can start on its keys while the one before still
+// runs.  Its time is off the step's critical path (passes over its sets run
+// in later launches), so the SMs it does not take are worth more to the
+// attention grid.  (Measured on B200 at 128K keys, 2 retrieval heads per
+// layer, two layers per attention launch: clusters of 4, grid 132, 1082
+// steps/s against 1047 with clusters of 8, grid 116; per head 840 against
+// 801; 32K 2230 against 2172.  With one layer per launch clusters of 8
+// won, 999 against 983.)  A large selection (layer 0) takes the largest size
+// whose clusters are all resident at once, so that it runs in one wave and
+// the next layer starts right away; else the smallest size.
 int pick_topk_cluster(const lyc_ctx* ctx, int ntasks) {
   auto resident = [&](int cl) {
     return ctx->topk_resident[cl] > 0 ? ctx->topk_resident[cl] : ctx->sms / cl;
   };
-  if (2 * ntasks * 8 <= ctx->sms / 4 && (ctx->topk_cls & (1u << 8)) && ntasks <= resident(8)) return 8;
+  if (2 * ntasks * 4 <= ctx->sms / 4 && (ctx->topk_cls & (1u << 4)) && ntasks <= resident(4)) return 4;
   int best = 0, smallest = 0;
   for (int cl : {16, 8, 4}) {
     if (!(ctx->topk_cls & (1u << cl))) continue;

@@ -387,14 +387,20 @@ lyc_status encode_gather_map(lyc_ctx* ctx, CUtensorMap* map, const void* base, c
 // layer, two layers per attention launch: clusters of 4, grid 132, 1082
 // steps/s against 1047 with clusters of 8, grid 116; per head 840 against
 // 801; 32K 2230 against 2172.  With one layer per launch clusters of 8
-// won, 999 against 983.)  A large selection (layer 0) takes the largest size
-// whose clusters are all resident at once, so that it runs in one wave and
-// the next layer starts right away; else the smallest size.
-int pick_topk_cluster(const lyc_ctx* ctx, int ntasks) {
+// won, 999 against 983.)  The size rules and block selection (variable) do
+// more work per key, and on clusters of 4 their selections last long enough
+// to hold up the passes over their sets: clusters of 8 (measured: top-p 0.5
+// 998 against 894 steps/s, threshold 1120 against 1082, block 1040 against
+// 1030).  A large selection (layer 0) takes the largest size whose clusters
+// are all resident at once, so that it runs in one wave and the next layer
+// starts right away; else the smallest size.
+int pick_topk_cluster(const lyc_ctx* ctx, int ntasks, bool variable) {
   auto resident = [&](int cl) {
     return ctx->topk_resident[cl] > 0 ? ctx->topk_resident[cl] : ctx->sms / cl;
   };
-  if (2 * ntasks * 4 <= ctx->sms / 4 && (ctx->topk_cls & (1u << 4)) && ntasks <= resident(4)) return 4;
+  const int small = variable ? 8 : 4;
+  if (2 * ntasks * small <= ctx->sms / 4 && (ctx->topk_cls & (1u << small)) && ntasks <= resident(small))
+    return small;
   int best = 0, smallest = 0;
   for (int cl : {16, 8, 4}) {
     if (!(ctx->topk_cls & (1u << cl))) continue;
@@ -714,7 +720,7 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const KvVie
         writer[s] = l;
       }
     prev_fresh = fresh;
-    H.topk_cl = pick_topk_cluster(ctx, static_cast<int>(H.tasks.size()));
+    H.topk_cl = pick_topk_cluster(ctx, static_cast<int>(H.tasks.size()), plan->variable);
     for (int b = 0; b < B; ++b)
       for (int s = 0; s < Hs; ++s) H.final_src.push_back(set_ptr(cur[s], b, s));
   }

@@ -60,16 +60,25 @@ constexpr int kPlanCacheSize = 16;
 // that read at least kSmallLayerBytes, four below (measured on B200: 128K
 // Llama3-8B shapes, ~151 MB per later layer: 1047 steps/s with two layers
 // per launch, 1026 with three, 1037 with four, ~1001 with one; 32K, ~50 MB
-// per layer: 2081, 2149, 2182 and ~1750).
-constexpr int kLayersPerLaunch = 4;  // at most
+// per layer: 2081, 2149, 2182 and ~1750; with selections on clusters of 4,
+// 128K 1078 with two against 1065 with four, 32K KV-group 2287 with eight
+// against 2230 with four but per head 1451 against 1476).  When no layer
+// after the first selects (every later head a sparse head, so layer 0's sets
+// serve the whole step), only layer 0's readers are deferred and a launch
+// holds eight layers (128K with no later retrieval heads: 3889 against 3478
+// steps/s with four).
+constexpr int kLayersPerLaunch = 8;     // at most
+constexpr int kLayersPerLaunchSel = 4;  // at most, when a later layer selects
 constexpr double kSmallLayerBytes = 96e6;
 // Buffers per set slot.  A selection overwrites the set that its slot held
 // kSetBuffers refreshes earlier.  That set's last readers run in the launch
 // of the layer that last read it, or, for a deferred pass, of the layer
 // after; a selection waits only for the attention launch before its own
-// layer's launch, so kLayersPerLaunch + 2 buffers keep every reader of the
-// overwritten set in a launch that has completed.
-constexpr int kSetBuffers = kLayersPerLaunch + 2;
+// layer's launch, so kLayersPerLaunchSel + 2 buffers keep every reader of
+// the overwritten set in a launch that has completed.  (A plan whose
+// launches hold more layers selects in layer 0 only: each slot is refreshed
+// once per step.)
+constexpr int kSetBuffers = kLayersPerLaunchSel + 2;
 
 
 int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
@@ -391,16 +400,22 @@ lyc_status encode_gather_map(lyc_ctx* ctx, CUtensorMap* map, const void* base, c
 // more work per key, and on clusters of 4 their selections last long enough
 // to hold up the passes over their sets: clusters of 8 (measured: top-p 0.5
 // 998 against 894 steps/s, threshold 1120 against 1082, block 1040 against
-// 1030).  A large selection (layer 0) takes the largest size whose clusters
-// are all resident at once, so that it runs in one wave and the next layer
-// starts right away; else the smallest size.
-int pick_topk_cluster(const lyc_ctx* ctx, int ntasks, bool variable) {
+// 1030).  Layer 0's selection (first), when its sets fit on clusters of 4
+// in a quarter of the SMs, takes clusters of 4: it starts as its launch ends
+// and holds SMs that the next launch's CTAs are waiting for (measured: 1084
+// against 1077-1079 steps/s with clusters of 8, 8 sets at 128K).  Another
+// large selection takes the largest size whose clusters are all resident at
+// once, so that it runs in one wave and the next layer starts right away;
+// else the smallest size.
+int pick_topk_cluster(const lyc_ctx* ctx, int ntasks, bool variable, bool first) {
   auto resident = [&](int cl) {
     return ctx->topk_resident[cl] > 0 ? ctx->topk_resident[cl] : ctx->sms / cl;
   };
   const int small = variable ? 8 : 4;
   if (2 * ntasks * small <= ctx->sms / 4 && (ctx->topk_cls & (1u << small)) && ntasks <= resident(small))
     return small;
+  if (first && !variable && ntasks * 4 <= ctx->sms / 4 && (ctx->topk_cls & (1u << 4)) && ntasks <= resident(4))
+    return 4;
   int best = 0, smallest = 0;
   for (int cl : {16, 8, 4}) {
     if (!(ctx->topk_cls & (1u << cl))) continue;
@@ -534,7 +549,12 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const KvVie
           layer_bytes += static_cast<double>(dense ? kv.n[b] : std::min<int64_t>(k, kv.n[b]));
       }
     layer_bytes *= static_cast<double>(cfg.head_dim) * es * 2.0 / std::max(1, L - 1);
-    const int LG = !use_pool ? 1 : layer_bytes < kSmallLayerBytes ? kLayersPerLaunch : 2;
+    bool later_sel = false;  // a layer after the first has a retrieval head
+    for (int64_t i = Hq; i < static_cast<int64_t>(L) * Hq && !later_sel; ++i) later_sel = role[i] != 0;
+    const int LG = !use_pool                       ? 1
+                   : !later_sel                    ? kLayersPerLaunch
+                   : layer_bytes < kSmallLayerBytes ? kLayersPerLaunchSel
+                                                   : 2;
     for (int l0 = 0, l1 = 0; l0 < L; l0 = l1) {
       l1 = std::min(L, l0 + LG);
       if (l1 == L && l1 - l0 > 1) l1 = L - 1;
@@ -720,7 +740,7 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const KvVie
         writer[s] = l;
       }
     prev_fresh = fresh;
-    H.topk_cl = pick_topk_cluster(ctx, static_cast<int>(H.tasks.size()), plan->variable);
+    H.topk_cl = pick_topk_cluster(ctx, static_cast<int>(H.tasks.size()), plan->variable, l == 0);
     for (int b = 0; b < B; ++b)
       for (int s = 0; s < Hs; ++s) H.final_src.push_back(set_ptr(cur[s], b, s));
   }

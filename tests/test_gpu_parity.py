@@ -218,6 +218,19 @@ def test_no_retrieval_after_layer0_bf16(lyc, mode):
     assert np.array_equal(S, tr[0])  # nothing refreshed after layer 0
 
 
+@pytest.mark.parametrize("mode", ["per_qhead", "kvgroup_mean"])
+def test_no_retrieval_after_layer0_launches_of_eight(lyc, mode):
+    """With no selection after layer 0 an attention launch holds eight
+    layers: layers 1-7 read layer 0's sets in the launch of layers 8-15
+    (with its own), then layer 16 alone before the last layer's launch."""
+    om = O.SELECT_PER_QHEAD if mode == "per_qhead" else O.SELECT_KVGROUP_MEAN
+    spec = W.StackSpec("r0-long", L=18, B=1, Hq=32, Hkv=8, d=128, n=8192, k=1024,
+                       retrieval_per_layer=0, planted="heavy", n_planted=32, seed=15)
+    data, out, S, tr = run_step(lyc, spec, select_mode=mode)
+    P.check_layers(data, out, tr, spec.k, spec.n, "bf16", range(spec.L), select_mode=om)
+    assert np.array_equal(S, tr[0])
+
+
 @pytest.mark.parametrize("gather", GATHERS)
 def test_ragged_sets_bf16(lyc, gather):
     """k not a multiple of the 64-row tile nor of the four-row gather: the

@@ -535,7 +535,7 @@ def run_lyc(args):
     ctx.set_timing(False)
     iso_attn_ms = sum(t[2] for t in ktimes if t[0] == 0) / args.steps
     iso_topk_ms = sum(t[2] for t in ktimes if t[0] == 1) / args.steps
-    # launches per step: attention launches (each of two or four layers, the
+    # launches per step: attention launches (each of two, four or eight layers, the
     # last layer's own, and a merge launch) and selection launches (one per
     # layer)
     attn_launches, topk_launches, other_launches = ctx.step_launches()
@@ -543,7 +543,7 @@ def run_lyc(args):
     roofline = {
         "bound": "hbm",
         "kernel": ("attn_tc_layer_kernel" if args.attn_kernel == "tcgen05" else "attn_mma_layer_kernel")
-                  + " (pooled dense + sparse attention of two or four layers per launch)",
+                  + " (pooled dense + sparse attention of two, four or eight layers per launch)",
         "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
         "frac": round(achieved / peak, 4),
         "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs), burst figure",

@@ -1,5 +1,5 @@
 // attn_mma_kernel.cu -- pooled hybrid-head decode attention of one launch
-// (two or four consecutive layers), bf16 inputs, tensor cores.
+// (two, four or eight consecutive layers), bf16 inputs, tensor cores.
 //
 // Computes, for every segment of the launch's work pool (lyc_plan.h):
 //   retrieval rows, page "LycheeDecode ..." (paper-graph-ui summary),

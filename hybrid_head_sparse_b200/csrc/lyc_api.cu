@@ -531,8 +531,8 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const KvVie
   // and outputs are those of layer l (Segment::q, Segment::out).  The last
   // layer keeps its own.
   const bool defer_dep = use_pool;
-  // The attention launches (mma kernel): kLayersPerLaunch consecutive layers
-  // each, the last layer alone (it keeps its passes over the sets of the
+  // The attention launches (mma kernel): LG consecutive layers each (two,
+  // four or eight, see kLayersPerLaunch), the last layer alone (it keeps its passes over the sets of the
   // selection just before it, which is enqueued before its launch).
   // launch_first[l]: the first layer of l's launch; next_launch[l]: the first
   // layer of the launch after it (L: none).
@@ -747,7 +747,7 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const KvVie
 
 
   // ---- phase B: the attention launches.  With the mma kernel a launch runs
-  // kLayersPerLaunch consecutive layers: their segments are concatenated in
+  // several consecutive layers: their segments are concatenated in
   // layer order (each layer's own passes, then the passes deferred into it).
   // No pass of a launch waits for a selection enqueued after that launch
   // (the selection could find no free SM while the launch's CTAs wait): a

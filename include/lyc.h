@@ -294,7 +294,7 @@ lyc_status lyc_step_bytes(const lyc_config* cfg, const uint8_t* role_mask, int64
                           int s_in, uint64_t* analytic, uint64_t* distinct);
 
 /* Kernel launches of the most recent step enqueued on this context: its
- * attention launches (bf16: each of two or four consecutive layers, the last
+ * attention launches (bf16: each of two, four or eight consecutive layers, the last
  * layer alone, and the launch that merges the last layer's split rows; fp32
  * and the tcgen05 kernel: one per layer and the merge launch), selection
  * launches (one per layer with retrieval heads), and the rest (the final set

@@ -57,28 +57,27 @@ constexpr int kPlanCacheSize = 16;
 // cost (its start, the wait for its first tiles, its drain: ~7 us, about
 // what the step streams in 45 MB) is paid once per that many layers; the
 // selections stay one launch per layer.  Two layers per launch for layers
-// that read at least kSmallLayerBytes, four below (measured on B200: 128K
-// Llama3-8B shapes, ~151 MB per later layer: 1047 steps/s with two layers
-// per launch, 1026 with three, 1037 with four, ~1001 with one; 32K, ~50 MB
-// per layer: 2081, 2149, 2182 and ~1750; with selections on clusters of 4,
-// 128K 1078 with two against 1065 with four, 32K KV-group 2287 with eight
-// against 2230 with four but per head 1451 against 1476).  When no layer
-// after the first selects (every later head a sparse head, so layer 0's sets
-// serve the whole step), only layer 0's readers are deferred and a launch
-// holds eight layers (128K with no later retrieval heads: 3889 against 3478
-// steps/s with four).
-constexpr int kLayersPerLaunch = 8;     // at most
-constexpr int kLayersPerLaunchSel = 4;  // at most, when a later layer selects
+// that read at least kSmallLayerBytes; below, four with per-head selection
+// and eight with KV-group selection, whose gathered rows (one set per
+// sparse group, not per sparse head) are a small share of a layer's bytes.
+// Measured on B200: 128K Llama3-8B shapes, ~151 MB per later layer: 1047
+// steps/s with two layers per launch, 1026 with three, 1037 with four,
+// ~1001 with one; 32K, ~50 MB per layer: 2081, 2149, 2182 and ~1750.  With
+// selections on clusters of 4: 128K 1078 with two against 1065 with four;
+// 32K KV-group 2287 with eight against 2230 with four, per head 1451
+// against 1476.  When no layer after the first selects (every later head a
+// sparse head, so layer 0's sets serve the whole step), only layer 0's
+// readers are deferred and a launch holds eight layers (128K with no later
+// retrieval heads: 3889 against 3478 steps/s with four).
+constexpr int kLayersPerLaunch = 8;  // at most
 constexpr double kSmallLayerBytes = 96e6;
 // Buffers per set slot.  A selection overwrites the set that its slot held
 // kSetBuffers refreshes earlier.  That set's last readers run in the launch
 // of the layer that last read it, or, for a deferred pass, of the layer
 // after; a selection waits only for the attention launch before its own
-// layer's launch, so kLayersPerLaunchSel + 2 buffers keep every reader of
-// the overwritten set in a launch that has completed.  (A plan whose
-// launches hold more layers selects in layer 0 only: each slot is refreshed
-// once per step.)
-constexpr int kSetBuffers = kLayersPerLaunchSel + 2;
+// layer's launch, so kLayersPerLaunch + 2 buffers keep every reader of the
+// overwritten set in a launch that has completed.
+constexpr int kSetBuffers = kLayersPerLaunch + 2;
 
 
 int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
@@ -551,10 +550,11 @@ lyc_status build_plan(lyc_ctx* ctx, Plan* plan, const uint8_t* role, const KvVie
     layer_bytes *= static_cast<double>(cfg.head_dim) * es * 2.0 / std::max(1, L - 1);
     bool later_sel = false;  // a layer after the first has a retrieval head
     for (int64_t i = Hq; i < static_cast<int64_t>(L) * Hq && !later_sel; ++i) later_sel = role[i] != 0;
-    const int LG = !use_pool                       ? 1
-                   : !later_sel                    ? kLayersPerLaunch
-                   : layer_bytes < kSmallLayerBytes ? kLayersPerLaunchSel
-                                                   : 2;
+    const int LG = !use_pool                        ? 1
+                   : !later_sel                     ? kLayersPerLaunch
+                   : layer_bytes >= kSmallLayerBytes ? 2
+                   : kvmode                          ? kLayersPerLaunch
+                                                    : 4;
     for (int l0 = 0, l1 = 0; l0 < L; l0 = l1) {
       l1 = std::min(L, l0 + LG);
       if (l1 == L && l1 - l0 > 1) l1 = L - 1;

@@ -489,28 +489,47 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster_kernel(const Top
       }
     }
   } else {
+    // The keys were just written by the attention launch, which may still
+    // stream beside this one, so each read waits on a loaded memory system.
+    // A warp issues kLoadBatch steps' reads before it uses any of them: the
+    // histogram's shared-memory atomics would otherwise hold each step's
+    // read back until the step before it is done.
+    constexpr int kLoadBatch = 8;
     const float* src = task.keys + lo;
     const bool vec = (reinterpret_cast<uintptr_t>(src) & 15u) == 0;
-    for (int base = wlo; base < whi; base += 128) {
-      const int x0 = base + 4 * lane;
-      uint32_t u[4];
-      if (vec && x0 + 3 < whi) {
-        const float4 v = *reinterpret_cast<const float4*>(src + x0);
-        u[0] = order_key(v.x); u[1] = order_key(v.y); u[2] = order_key(v.z); u[3] = order_key(v.w);
-        *reinterpret_cast<uint4*>(us + x0) = make_uint4(u[0], u[1], u[2], u[3]);
-      } else {
+    for (int base = wlo; base < whi; base += 128 * kLoadBatch) {
+      float4 v[kLoadBatch];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          u[e] = (x0 + e < whi) ? order_key(src[x0 + e]) : 0u;
-          if (x0 + e < whi) us[x0 + e] = u[e];
+      for (int j = 0; j < kLoadBatch; ++j) {
+        const int x0 = base + 128 * j + 4 * lane;
+        if (vec && x0 + 3 < whi) {
+          v[j] = *reinterpret_cast<const float4*>(src + x0);
+        } else {
+          v[j].x = x0 < whi ? src[x0] : 0.f;
+          v[j].y = x0 + 1 < whi ? src[x0 + 1] : 0.f;
+          v[j].z = x0 + 2 < whi ? src[x0 + 2] : 0.f;
+          v[j].w = x0 + 3 < whi ? src[x0 + 3] : 0.f;
         }
       }
 #pragma unroll
-      for (int e = 0; e < 4; ++e)
-        if (x0 + e < whi) {
-          atomicAdd(&loc[u[e] >> kKeyDigitShift], 1u);
-          if (VAR) umax = max(umax, u[e]);
+      for (int j = 0; j < kLoadBatch; ++j) {
+        const int x0 = base + 128 * j + 4 * lane;
+        const uint32_t u[4] = {order_key(v[j].x), order_key(v[j].y), order_key(v[j].z),
+                               order_key(v[j].w)};
+        if (x0 + 3 < whi) {
+          *reinterpret_cast<uint4*>(us + x0) = make_uint4(u[0], u[1], u[2], u[3]);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            if (x0 + e < whi) us[x0 + e] = u[e];
         }
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          if (x0 + e < whi) {
+            atomicAdd(&loc[u[e] >> kKeyDigitShift], 1u);
+            if (VAR) umax = max(umax, u[e]);
+          }
+      }
     }
   }
   if (rule != kSizeFixed) {
